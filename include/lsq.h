@@ -1,0 +1,256 @@
+/*
+ * lsq.h - C ABI of the layer-streamed QLoRA (NF4) library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes the hot path of layer-streamed QLoRA fine-tuning as the
+ * pages on "Exact Layer Streaming" describe it:
+ *   - the frozen decoder weights are stored as blockwise-absmax NF4 (Soup
+ *     layer-streaming tutorial, "Soup layer streaming 的四段資料路徑", part 1 "NF4");
+ *   - each frozen linear carries a trainable LoRA branch, y = x W^T + s (x A^T) B^T,
+ *     and its backward still reads W: dX = dY W + s (dY B) A (same page, part 3
+ *     "Forward＋backward" and FAQ 4);
+ *   - the decoder stack sits in page-locked host memory and is fed to the GPU one
+ *     layer at a time through two fixed VRAM buffers, the copy running on its own
+ *     stream so that it overlaps compute (same page, part 2 "Pinned memory";
+ *     Layer Streaming blog, "層流技術：技術實作與記憶體效率");
+ *   - every layer is recomputed in backward (tutorial, part 3 and the
+ *     "gradient_checkpointing: true" bullet), so each layer is read twice per
+ *     micro-batch.
+ *
+ * Conventions (all entry points):
+ *   - Return value: LSQ_OK (0) or one of the LSQ_ERR_* codes below; nothing
+ *     aborts or throws.  lsq_last_error() gives a message for the calling thread.
+ *   - Memory: the caller owns every buffer (device tensors, pinned host blobs,
+ *     workspaces, streams).  The library never allocates or frees caller memory
+ *     and allocates no device memory per call.  Opaque handles (lsq_stack) own
+ *     only their CUDA events and copy stream.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Unless stated otherwise a call only enqueues work on it; pointers must stay
+ *     valid until that work completes.
+ *   - Layouts are row-major and contiguous.  bf16 tensors are passed as uint16_t
+ *     bit patterns.  Device pointers must be 16-byte aligned.
+ *   - Kernel-side errors (a bounded wait that gave up) are latched in a device
+ *     status word; lsq_device_status() reads it, the synchronous calls check it.
+ */
+#ifndef LSQ_H
+#define LSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  LSQ_OK = 0,
+  LSQ_ERR_INVALID = 1,   /* null pointer, bad enum, non-finite input */
+  LSQ_ERR_SHAPE = 2,     /* a size that violates the documented constraints */
+  LSQ_ERR_CUDA = 3,      /* a CUDA runtime error (launch or asynchronous) */
+  LSQ_ERR_TIMEOUT = 4,   /* a host wait passed its deadline */
+  LSQ_ERR_WORKSPACE = 5, /* workspace smaller than the *_workspace_bytes query */
+  LSQ_ERR_ALIGN = 6,     /* a pointer that is not 16-byte aligned */
+  LSQ_ERR_DEVICE = 7     /* a kernel latched an error in the device status word */
+};
+
+/* Message for the last error raised on the calling thread ("" if none). */
+const char* lsq_last_error(void);
+/* ABI version (major * 100 + minor). */
+int lsq_version(void);
+/* Reads (and, if clear != 0, resets) the device status word of the current
+ * device into *flags.  Synchronises the device.  Returns LSQ_OK or LSQ_ERR_CUDA. */
+int lsq_device_status(int* flags, int clear);
+
+/* ------------------------------------------------------------------- NF4 */
+
+/* The 16 NF4 levels as fp32, ascending, derived inside the library from the
+ * definition of 4-bit NormalFloat (normal quantiles with an exact zero, scaled
+ * to [-1, 1]); host only, needs no GPU. */
+int lsq_nf4_codebook(float out_levels[16]);
+
+/* nf4_quantize - blockwise-absmax NF4 quantisation of a frozen weight.
+ * Tutorial, "四段資料路徑" part 1 (weights are quantised offline to NF4 shards).
+ *   W       device fp32 [N, K] row-major.
+ *   block   elements per absmax block; must be 64.  K % 64 == 0, N*K even.
+ *   codes   device uint8 [N*K/2]: element 2j in the high nibble of byte j,
+ *           element 2j+1 in the low nibble.  Code = index of the nearest level
+ *           of w/absmax (fp32 division, exact midpoint -> lower code).
+ *   absmax  device fp32 [N*K/64]: max |w| of each block (0 -> all codes 7).
+ * Synchronous: waits for the stream, then returns LSQ_ERR_INVALID if W held a
+ * NaN or Inf (codes/absmax are then unspecified).  Deterministic. */
+int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block, uint8_t* codes,
+                 float* absmax, void* stream);
+
+/* nf4_dequantize - w~ = fl32(level[code] * absmax) into fp32 W_out [N, K].
+ * Same layouts and constraints as nf4_quantize; asynchronous. */
+int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+                   int32_t block, float* W_out, void* stream);
+
+/* ------------------------------------------------------- NF4 + LoRA linear */
+
+/* Workspace bytes needed by nf4_lora_linear_fwd/bwd for these sizes. */
+size_t nf4_lora_linear_workspace_bytes(int64_t T, int64_t K, int64_t N, int32_t r);
+
+/* nf4_lora_linear_fwd - y = x W~^T + scale * (x A^T) B^T (+ residual).
+ * Tutorial part 1 (LoRA A/B trained on top of the frozen NF4 base).
+ *   x        device bf16 [T, K];  T >= 1, K % 64 == 0.
+ *   codes, absmax  the NF4 weight W [N, K] (layout of nf4_quantize); N % 8 == 0.
+ *   A        device fp32 [r, K];  B  device fp32 [N, r];  r % 16 == 0, 16 <= r <= 256.
+ *   residual device bf16 [T, N] or NULL.
+ *   y        device bf16 [T, N] (output).
+ *   u_out    device fp32 [T, r] = x A^T, or NULL.
+ *   ws       device workspace of nf4_lora_linear_workspace_bytes(T, K, N, r).
+ * The dequantised weight is rounded to bf16 for the tensor cores; accumulation
+ * is fp32.  Asynchronous, deterministic. */
+int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int64_t N,
+                        const uint8_t* codes, const float* absmax, int32_t block,
+                        const float* A, const float* B, int32_t r, float scale,
+                        const uint16_t* residual, uint16_t* y, float* u_out, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* nf4_lora_linear_bwd - backward of the linear above (W frozen).
+ * Tutorial part 3 and FAQ 4: dX still needs W.
+ *   dy [T, N] bf16, x [T, K] bf16 (the forward input).
+ *   dx  device bf16 [T, K] = dy W~ + scale (dy B) A.
+ *   dA  device fp32 [r, K] (+)= scale (dy B)^T x;  dB device fp32 [N, r] (+)= scale dy^T (x A^T).
+ *   accumulate  0: overwrite dA/dB, 1: add to them.
+ * Asynchronous, deterministic (fixed-order reductions, no atomics). */
+int nf4_lora_linear_bwd(const uint16_t* dy, const uint16_t* x, int64_t T, int64_t K, int64_t N,
+                        const uint8_t* codes, const float* absmax, int32_t block,
+                        const float* A, const float* B, int32_t r, float scale, uint16_t* dx,
+                        float* dA, float* dB, int32_t accumulate, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* --------------------------------------------------------- decoder layer */
+
+/* Llama-style decoder configuration.  The pages name the model (Llama-3.1-8B,
+ * tutorial "維護者的 4GB／8B 成績"); the hyper-parameters are the caller's. */
+typedef struct lsq_cfg {
+  int64_t hidden;      /* D */
+  int64_t ffn;         /* F, SwiGLU inner size */
+  int64_t vocab;       /* V */
+  int32_t n_heads;     /* H */
+  int32_t n_kv_heads;  /* Hkv, H % Hkv == 0 */
+  int32_t head_dim;    /* d, must be 128 or 64 */
+  int32_t n_layers;    /* L */
+  int32_t lora_r;      /* r, multiple of 16 */
+  int32_t block;       /* NF4 block, must be 64 */
+  float lora_alpha;    /* s = alpha / r */
+  float rope_theta;    /* rotate-half RoPE base */
+  float rms_eps;       /* RMSNorm epsilon */
+  int32_t reserved;    /* must be 0 */
+} lsq_cfg;
+
+/* Byte layout of one layer's blob (the unit that is streamed).  Projection
+ * order q, k, v, o, gate, up, down.  All codes come first, contiguous, so q|k|v
+ * and gate|up each form one stacked NF4 matrix; then all absmax arrays; then
+ * the two RMSNorm gains (bf16 [D]).  Every section starts 256-byte aligned. */
+typedef struct lsq_layer_layout {
+  uint64_t codes_off[7];
+  uint64_t absmax_off[7];
+  uint64_t g1_off, g2_off;
+  int64_t rows[7], cols[7]; /* N, K of each projection */
+  uint64_t bytes;           /* total blob size (multiple of 256) */
+} lsq_layer_layout;
+
+/* Fills *out for cfg.  Host only.  LSQ_ERR_SHAPE unless D, F, H*d, Hkv*d are
+ * multiples of 128 and head_dim is 64 or 128. */
+int lsq_layer_layout_get(const lsq_cfg* cfg, lsq_layer_layout* out);
+
+/* Layout of one layer's LoRA masters (fp32), offsets in floats:
+ *   A_qkv [3r, D] (A_q; A_k; A_v), B_qkv [H*d + 2*Hkv*d, r] (B_q; B_k; B_v),
+ *   A_o [r, H*d], B_o [D, r], A_gu [2r, D] (A_gate; A_up), B_gu [2F, r],
+ *   A_down [r, F], B_down [D, r].
+ * A stack's LoRA buffer is n_layers such blocks back to back (floats_per_layer
+ * each); gradients and AdamW moments use the same layout. */
+typedef struct lsq_lora_layout {
+  int64_t a_off[7], b_off[7]; /* per projection, q..down */
+  int64_t floats_per_layer;
+} lsq_lora_layout;
+int lsq_lora_layout_get(const lsq_cfg* cfg, lsq_lora_layout* out);
+
+/* Workspace for decoder_layer_fwd/bwd with T = batch * seq tokens. */
+size_t decoder_layer_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t seq);
+
+/* decoder_layer_fwd - one decoder layer: RMSNorm -> q/k/v (NF4 + LoRA) -> RoPE
+ * -> causal GQA attention -> o (+residual) -> RMSNorm -> gate/up -> SwiGLU ->
+ * down (+residual).
+ *   blob    device pointer to the layer blob (lsq_layer_layout).
+ *   lora    device fp32, one layer's LoRA block (lsq_lora_layout).
+ *   x_in    device bf16 [batch*seq, D]; x_out device bf16 [batch*seq, D].
+ * Asynchronous, deterministic. */
+int decoder_layer_fwd(const lsq_cfg* cfg, const void* blob, const float* lora,
+                      const uint16_t* x_in, int32_t batch, int32_t seq, uint16_t* x_out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* decoder_layer_bwd - recomputes the layer's forward from x_in, then
+ * backpropagates dx_out (fp32 [T, D], gradient w.r.t. x_out) into dx_in (fp32
+ * [T, D]) and the LoRA gradients (fp32, lsq_lora_layout; accumulate 0/1).
+ * The frozen weights and gains get no gradient.  Asynchronous, deterministic. */
+int decoder_layer_bwd(const lsq_cfg* cfg, const void* blob, const float* lora,
+                      const uint16_t* x_in, const float* dx_out, int32_t batch, int32_t seq,
+                      float* dx_in, float* lora_grad, int32_t accumulate, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------- streamed stack */
+
+typedef struct lsq_stack lsq_stack;
+
+/* stream_stack_create - binds a decoder stack to two VRAM layer buffers.
+ *   layer_blobs  n_layers pointers to layer blobs (lsq_layer_layout).  With
+ *                resident == 0 they are page-locked host memory (pinned with
+ *                cudaHostAlloc/cudaHostRegister by the caller) and are copied
+ *                into vram_buf0/vram_buf1 on the stack's own copy stream; with
+ *                resident == 1 they are device memory and are used in place
+ *                (the two buffers are then ignored and may be NULL).
+ *   vram_buf0/1  device buffers of lsq_layer_layout.bytes each.
+ * Creates the handle's copy stream and events on the current device. */
+int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_blobs, int32_t n_layers,
+                        void* vram_buf0, void* vram_buf1, int32_t resident, lsq_stack** out);
+int stream_stack_destroy(lsq_stack* stack);
+
+/* AdamW on the LoRA masters (decoupled weight decay, bias correction with
+ * step >= 1).  m and v are device fp32 in the LoRA layout. */
+typedef struct lsq_adamw {
+  float lr, beta1, beta2, eps, weight_decay;
+  int32_t step;
+  float* m;
+  float* v;
+} lsq_adamw;
+
+/* Workspace for stream_stack_step with micro-batches of batch x seq tokens. */
+size_t stream_stack_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t seq);
+
+/* stream_stack_step - one SFT optimiser step through the streamed stack.
+ *   tokens      device int32 [micro_batches, batch, seq], ids in [0, vocab).
+ *   emb, lm_head  device bf16 [V, D] (untied, resident); final_norm bf16 [D].
+ *   lora        device fp32 stack LoRA buffer (updated in place if opt != NULL).
+ *   lora_grad   device fp32, same layout; overwritten with the gradient of the
+ *               mean loss over all micro-batches.
+ *   opt         AdamW state, or NULL for no update.
+ *   loss_out    host float: mean cross-entropy over every predicted position
+ *               (positions 0..seq-2 of each sequence, target = next token).
+ *   logits_out  device fp32 [batch*seq, V] of the last micro-batch, or NULL.
+ * Each micro-batch streams layers 0..L-1 forward, then the lm_head and loss,
+ * then L-1..0 backward with per-layer recomputation.  A layer already in a
+ * buffer when it is needed again is not copied again.  Synchronous: returns once
+ * the loss is on the host, LSQ_ERR_TIMEOUT if that takes longer than
+ * timeout_ms (the work is then still in flight on the streams). */
+int stream_stack_step(lsq_stack* stack, const int32_t* tokens, int32_t micro_batches,
+                      int32_t batch, int32_t seq, const uint16_t* emb, const uint16_t* lm_head,
+                      const uint16_t* final_norm, float* lora, float* lora_grad,
+                      const lsq_adamw* opt, float* loss_out, float* logits_out, void* ws,
+                      size_t ws_bytes, void* stream, int64_t timeout_ms);
+
+/* Per-step counters of the last stream_stack_step. */
+typedef struct lsq_step_stats {
+  int32_t layer_copies;     /* host->device layer copies issued */
+  int64_t h2d_bytes;        /* bytes those copies moved */
+  float step_ms;            /* device time of the step (events on the compute stream) */
+  float copy_wait_ms;       /* summed stall of the compute stream on copy-ready events */
+} lsq_step_stats;
+int stream_stack_last_stats(const lsq_stack* stack, lsq_step_stats* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSQ_H */

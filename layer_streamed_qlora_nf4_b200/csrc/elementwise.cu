@@ -1,0 +1,481 @@
+// Memory-bound kernels of the decoder layer and the stack ends: split-K reduce,
+// RMSNorm fwd/bwd, rotate-half RoPE fwd/bwd, SwiGLU fwd/bwd, embedding gather,
+// cross-entropy, AdamW.  Vectorised 16-byte accesses, warp-shuffle reductions
+// in a fixed order (deterministic), fp32 arithmetic on bf16 storage.
+//
+// Definitions (Llama-style decoder named by the Soup layer-streaming tutorial,
+// "維護者的 4GB／8B 成績"; norms kept at higher precision, "四段資料路徑" part 1):
+//   RMSNorm  y = x (mean(x^2) + eps)^-1/2 g
+//   RoPE     rotate-half pairs (i, i + d/2), angle = pos theta^(-2i/d)
+//   SwiGLU   m = silu(gate) * up
+//   SFT loss mean cross-entropy of next-token targets
+//   AdamW    decoupled weight decay, bias-corrected moments
+#include <math.h>
+
+#include "common.cuh"
+
+namespace lsq {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+unsigned grid_for(int64_t n, int threads, int per_thread = 1) {
+  int64_t g = (n + (int64_t)threads * per_thread - 1) / ((int64_t)threads * per_thread);
+  const int64_t cap = (int64_t)gemm_num_sms() * 32;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (unsigned)g;
+}
+
+// ------------------------------------------------------------------ split-K reduce
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t T,
+                                     int64_t M, void* __restrict__ out, int out_f32, int64_t ldo,
+                                     const uint16_t* __restrict__ res, int64_t ldr) {
+  const int64_t n4 = T * M / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i * 4;
+    const int64_t t = e / M, m = e % M;
+    float4 acc = reinterpret_cast<const float4*>(part)[i];
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = reinterpret_cast<const float4*>(part + (size_t)s * T * M)[i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (res) {
+      const uint2 r = *reinterpret_cast<const uint2*>(res + t * ldr + m);
+      const float2 r0 = unpack_bf16x2(r.x), r1 = unpack_bf16x2(r.y);
+      acc.x += r0.x;
+      acc.y += r0.y;
+      acc.z += r1.x;
+      acc.w += r1.y;
+    }
+    if (out_f32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(out) + t * ldo + m) = acc;
+    } else {
+      uint2 o;
+      o.x = pack_bf16x2(acc.x, acc.y);
+      o.y = pack_bf16x2(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + t * ldo + m) = o;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// One warp per row; D % 8 == 0.
+__global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
+                                   int64_t T, int64_t D, float eps, uint16_t* __restrict__ y,
+                                   float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row >= T) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + row * D);
+  const int64_t nv = D / 8;
+  float ss = 0.f;
+  for (int64_t i = lane; i < nv; i += 32) {
+    const uint4 v = xr[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = unpack_bf16x2(w[q]);
+      ss = fmaf(f.x, f.x, ss);
+      ss = fmaf(f.y, f.y, ss);
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)D + eps);
+  if (lane == 0 && rstd) rstd[row] = r;
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  uint4* yr = reinterpret_cast<uint4*>(y + row * D);
+  for (int64_t i = lane; i < nv; i += 32) {
+    const uint4 v = xr[i], gv = gr[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = unpack_bf16x2(w[q]), gg = unpack_bf16x2(gw[q]);
+      o[q] = pack_bf16x2(f.x * r * gg.x, f.y * r * gg.y);
+    }
+    yr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// dx = dres + r (g dy) - x r^3 sum(g dy x) / D
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t* __restrict__ x,
+                                   const uint16_t* __restrict__ g, const float* __restrict__ rstd,
+                                   const float* __restrict__ dres, int64_t T, int64_t D,
+                                   float* __restrict__ dx, uint16_t* __restrict__ dxb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row >= T) return;
+  const int64_t nv = D / 4;
+  const float4* dyr = reinterpret_cast<const float4*>(dy + row * D);
+  const uint2* xr = reinterpret_cast<const uint2*>(x + row * D);
+  const uint2* gr = reinterpret_cast<const uint2*>(g);
+  float dot = 0.f;
+  for (int64_t i = lane; i < nv; i += 32) {
+    const float4 d = dyr[i];
+    const uint2 xv = xr[i], gv = gr[i];
+    const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
+    const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
+    dot += d.x * g0.x * x0.x + d.y * g0.y * x0.y + d.z * g1.x * x1.x + d.w * g1.y * x1.y;
+  }
+  dot = warp_sum(dot);
+  const float r = rstd[row];
+  const float c = r * r * r * dot / (float)D;
+  const float4* rr = dres ? reinterpret_cast<const float4*>(dres + row * D) : nullptr;
+  float4* o = reinterpret_cast<float4*>(dx + row * D);
+  for (int64_t i = lane; i < nv; i += 32) {
+    const float4 d = dyr[i];
+    const uint2 xv = xr[i], gv = gr[i];
+    const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
+    const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
+    float4 v;
+    v.x = r * g0.x * d.x - x0.x * c;
+    v.y = r * g0.y * d.y - x0.y * c;
+    v.z = r * g1.x * d.z - x1.x * c;
+    v.w = r * g1.y * d.w - x1.y * c;
+    if (rr) {
+      const float4 a = rr[i];
+      v.x += a.x;
+      v.y += a.y;
+      v.z += a.z;
+      v.w += a.w;
+    }
+    o[i] = v;
+    if (dxb) {
+      uint2 b;
+      b.x = pack_bf16x2(v.x, v.y);
+      b.y = pack_bf16x2(v.z, v.w);
+      reinterpret_cast<uint2*>(dxb + row * D)[i] = b;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ RoPE
+// angle(pos, i) = pos * theta^(-2i/d), evaluated in double and rounded to fp32
+__device__ __forceinline__ void rope_cs(int pos, int i, int d, double log_theta, float* c,
+                                        float* s) {
+  const double ang = (double)pos * exp(-2.0 * (double)i / (double)d * log_theta);
+  double sd, cd;
+  sincos(ang, &sd, &cd);
+  *c = (float)cd;
+  *s = (float)sd;
+}
+
+// In-place rotation of the q and k heads of the fused qkv buffer (bf16).
+__global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int H, int Hkv, int d,
+                            double log_theta, int inverse) {
+  const int half = d / 2;
+  const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
+  const int64_t n = T * (H + Hkv) * half;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(i % half);
+    const int64_t th = i / half;
+    const int head = (int)(th % (H + Hkv));
+    const int64_t t = th / (H + Hkv);
+    const int pos = (int)(t % seq);
+    float c, s;
+    rope_cs(pos, j, d, log_theta, &c, &s);
+    if (inverse) s = -s;
+    uint16_t* base = qkv + t * ld + (int64_t)head * d;
+    const float x1 = bf16_bits_to_float(base[j]), x2 = bf16_bits_to_float(base[j + half]);
+    base[j] = float_to_bf16_bits(x1 * c - x2 * s);
+    base[j + half] = float_to_bf16_bits(x2 * c + x1 * s);
+  }
+}
+
+// dqkv (bf16) <- [rope^-1(dq), rope^-1(dk), dv]  from fp32 gradients [T, H d], [T, Hkv d] x2
+__global__ void rope_grad_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
+                                 const float* __restrict__ dv, int64_t T, int seq, int H, int Hkv,
+                                 int d, double log_theta, uint16_t* __restrict__ dqkv) {
+  const int half = d / 2;
+  const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
+  const int64_t n = T * (H + 2 * Hkv) * half;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(i % half);
+    const int64_t th = i / half;
+    const int head = (int)(th % (H + 2 * Hkv));
+    const int64_t t = th / (H + 2 * Hkv);
+    uint16_t* out = dqkv + t * ld + (int64_t)head * d;
+    if (head >= H + Hkv) {
+      const float* src = dv + t * (int64_t)Hkv * d + (int64_t)(head - H - Hkv) * d;
+      out[j] = float_to_bf16_bits(src[j]);
+      out[j + half] = float_to_bf16_bits(src[j + half]);
+      continue;
+    }
+    const float* src = (head < H) ? dq + t * (int64_t)H * d + (int64_t)head * d
+                                  : dk + t * (int64_t)Hkv * d + (int64_t)(head - H) * d;
+    const int pos = (int)(t % seq);
+    float c, s;
+    rope_cs(pos, j, d, log_theta, &c, &s);
+    const float g1 = src[j], g2 = src[j + half];
+    out[j] = float_to_bf16_bits(g1 * c + g2 * s);
+    out[j + half] = float_to_bf16_bits(g2 * c - g1 * s);
+  }
+}
+
+// ------------------------------------------------------------------ SwiGLU
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+
+__global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, int64_t F,
+                                  uint16_t* __restrict__ m) {
+  const int64_t nv = T * F / 2;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i * 2;
+    const int64_t t = e / F, f = e % F;
+    const float2 g = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + f));
+    const float2 u = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + F + f));
+    *reinterpret_cast<uint32_t*>(m + e) =
+        pack_bf16x2(g.x * sigmoidf_(g.x) * u.x, g.y * sigmoidf_(g.y) * u.y);
+  }
+}
+
+__global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* __restrict__ gu,
+                                  int64_t T, int64_t F, uint16_t* __restrict__ dgu) {
+  const int64_t nv = T * F / 2;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i * 2;
+    const int64_t t = e / F, f = e % F;
+    const float2 g = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + f));
+    const float2 u = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + F + f));
+    const float2 d = *reinterpret_cast<const float2*>(dm + e);
+    const float s0 = sigmoidf_(g.x), s1 = sigmoidf_(g.y);
+    const float dg0 = d.x * u.x * s0 * (1.f + g.x * (1.f - s0));
+    const float dg1 = d.y * u.y * s1 * (1.f + g.y * (1.f - s1));
+    const float du0 = d.x * g.x * s0, du1 = d.y * g.y * s1;
+    *reinterpret_cast<uint32_t*>(dgu + t * 2 * F + f) = pack_bf16x2(dg0, dg1);
+    *reinterpret_cast<uint32_t*>(dgu + t * 2 * F + F + f) = pack_bf16x2(du0, du1);
+  }
+}
+
+// ------------------------------------------------------------------ embedding, CE, AdamW
+__global__ void embedding_kernel(const int32_t* __restrict__ tok, int64_t T,
+                                 const uint16_t* __restrict__ emb, int64_t D, int64_t V,
+                                 uint16_t* __restrict__ out) {
+  const int64_t nv = D / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T * nv;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nv, c = i % nv;
+    int64_t id = tok[t];
+    if (id < 0 || id >= V) id = 0;  // ids are validated on the host side where possible
+    reinterpret_cast<uint4*>(out + t * D)[c] = reinterpret_cast<const uint4*>(emb + id * D)[c];
+  }
+}
+
+// One CTA (512 threads) per row.  Rows whose position is the last of its
+// sequence have no target: zero gradient, zero loss.
+__global__ void cross_entropy_kernel(const float* __restrict__ logits,
+                                     const int32_t* __restrict__ tok, int64_t T, int seq,
+                                     int64_t V, float inv_count, uint16_t* __restrict__ dlogits,
+                                     float* __restrict__ row_loss) {
+  __shared__ float red[32];
+  __shared__ float bcast;
+  const int64_t row = blockIdx.x;
+  const float* lr = logits + row * V;
+  uint16_t* dr = dlogits + row * V;
+  const bool has_target = (row % seq) != (seq - 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (!has_target) {
+    for (int64_t i = threadIdx.x; i < V; i += blockDim.x) dr[i] = 0;
+    if (threadIdx.x == 0) row_loss[row] = 0.f;
+    return;
+  }
+  float mx = -INFINITY;
+  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) mx = fmaxf(mx, lr[i]);
+  mx = warp_max(mx);
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (warp == 0) {
+    float v = lane < nw ? red[lane] : -INFINITY;
+    v = warp_max(v);
+    if (lane == 0) bcast = v;
+  }
+  __syncthreads();
+  mx = bcast;
+  float sum = 0.f;
+  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) sum += expf(lr[i] - mx);
+  sum = warp_sum(sum);
+  __syncthreads();
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  if (warp == 0) {
+    float v = lane < nw ? red[lane] : 0.f;
+    v = warp_sum(v);
+    if (lane == 0) bcast = v;
+  }
+  __syncthreads();
+  sum = bcast;
+  const float lse = mx + logf(sum);
+  const int64_t tgt = tok[row + 1];
+  const float inv = 1.f / sum;
+  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) {
+    float p = expf(lr[i] - mx) * inv;
+    if (i == tgt) p -= 1.f;
+    dr[i] = float_to_bf16_bits(p * inv_count);
+  }
+  if (threadIdx.x == 0) row_loss[row] = lse - lr[tgt];
+}
+
+__global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float scale,
+                                int accumulate, float* __restrict__ out) {
+  __shared__ float red[32];
+  float s = 0.f;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += v[i];
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) *out = (accumulate ? *out : 0.f) + scale * t;
+  }
+}
+
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                             float* __restrict__ m, float* __restrict__ v, int64_t n, float lr,
+                             float b1, float b2, float eps, float wd, float bc1, float bc2) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float gi = g[i];
+    const float mi = b1 * m[i] + (1.f - b1) * gi;
+    const float vi = b2 * v[i] + (1.f - b2) * gi * gi;
+    m[i] = mi;
+    v[i] = vi;
+    const float mh = mi / bc1, vh = vi / bc2;
+    p[i] = p[i] * (1.f - lr * wd) - lr * mh / (sqrtf(vh) + eps);
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t n,
+                                   uint16_t* __restrict__ y) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = float_to_bf16_bits(x[i]);
+}
+
+__global__ void scale_kernel(float* __restrict__ x, int64_t n, float s) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    x[i] *= s;
+}
+
+}  // namespace
+
+int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
+                         int out_f32, int64_t ldo, const uint16_t* residual, int64_t ldr,
+                         cudaStream_t st) {
+  if (M % 4 != 0) return set_error(LSQ_ERR_SHAPE, "splitk_reduce: M %% 4 != 0");
+  splitk_reduce_kernel<<<grid_for(T * M / 4, 256), 256, 0, st>>>(partial, splits, T, M, out,
+                                                                 out_f32, ldo, residual, ldr);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
+                       uint16_t* y, float* rstd, cudaStream_t st) {
+  rmsnorm_fwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(x, g, T, D, eps, y, rstd);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
+                       const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
+                       cudaStream_t st) {
+  rmsnorm_bwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(dy, x, g, rstd, dres, T, D,
+                                                                      dx, dx_bf16);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, float theta, int inverse,
+                cudaStream_t st) {
+  const int64_t n = T * (H + Hkv) * (d / 2);
+  rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(qkv, T, seq, H, Hkv, d, log((double)theta),
+                                                inverse);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
+                     int Hkv, int d, float theta, uint16_t* dqkv, cudaStream_t st) {
+  const int64_t n = T * (H + 2 * Hkv) * (d / 2);
+  rope_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dq, dk, dv, T, seq, H, Hkv, d,
+                                                     log((double)theta), dqkv);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st) {
+  swiglu_fwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(gu, T, F, m);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
+                      cudaStream_t st) {
+  swiglu_bwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(dm, gu, T, F, dgu);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D, int64_t V,
+                     uint16_t* out, cudaStream_t st) {
+  embedding_kernel<<<grid_for(T * D / 8, 256), 256, 0, st>>>(tokens, T, emb, D, V, out);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq, int64_t V,
+                         float inv_count, uint16_t* dlogits, float* row_loss, cudaStream_t st) {
+  cross_entropy_kernel<<<(unsigned)T, 512, 0, st>>>(logits, tokens, T, seq, V, inv_count, dlogits,
+                                                    row_loss);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_sum_rows(const float* row_loss, int64_t T, float scale, int accumulate, float* out,
+                    cudaStream_t st) {
+  sum_rows_kernel<<<1, 1024, 0, st>>>(row_loss, T, scale, accumulate, out);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr, float b1,
+                 float b2, float eps, float wd, int step, cudaStream_t st) {
+  const float bc1 = (float)(1.0 - pow((double)b1, (double)step));
+  const float bc2 = (float)(1.0 - pow((double)b2, (double)step));
+  adamw_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st) {
+  f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, y);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st) {
+  scale_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, s);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+}  // namespace lsq

@@ -1,0 +1,658 @@
+// Tensor-core GEMM with the NF4 dequantisation fused into the operand load and
+// the LoRA up-projection fused as an extra K range ("slab"), for sm_100a.
+//
+// What it computes (per call): out[t, m] = sum_c Wop[m, c] act[t, c]
+//                                         + sum_j la[m, j] lb[t, j] (+ residual)
+// Forward of a frozen NF4 linear with LoRA (Soup layer-streaming tutorial,
+// "四段資料路徑" part 1): Wop = deq(W), act = x, la = s*B, lb = u = x A^T.
+// Its input gradient (part 3 and FAQ 4, W is re-read in backward):
+// Wop = deq(W)^T, act = dY, la = s*A^T, lb = v = dY B.
+//
+// Design for B200 (one CTA per SM, 256 threads, warp-specialised):
+//   warp 0   : TMA producer for the activation tile (128-byte swizzle) [and
+//              the bf16 weight tile in W_BF16_N mode]
+//   warp 1   : allocates TMEM, one elected thread issues tcgen05.mma
+//              (M = 128 output features x N = up to 256 tokens x K = 16),
+//              accumulators in TMEM (up to 2 x 256 fp32 columns)
+//   warp 2   : TMA producer for the packed NF4 codes (or the bf16 tile to be
+//              transposed) into a deep staging ring
+//   warps 4-7: operand stage - expand the staged codes to bf16 (level[code] *
+//              absmax in fp32, then round-to-nearest bf16) straight into the
+//              UMMA canonical K-major 128-byte-swizzle layout, fence the async
+//              proxy, arrive; they also write the LoRA slab; then the epilogue
+//              (tcgen05.ld of their TMEM lane quarter).
+// The output tile is 128 features x all tokens of the CTA (up to 512), so each
+// weight element is dequantised once per token tile.  Small problems use a
+// fixed-order split over K with an fp32 partial buffer and a separate reduce:
+// results are deterministic and independent of scheduling.
+// Every mbarrier wait is bounded (1 s) and aborts the CTA with a device status
+// bit instead of hanging.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace lsq {
+
+__device__ int g_lsq_dev_status;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBM = 128;        // output features per CTA (UMMA M)
+constexpr int kBK = 64;         // contraction per stage = one SW128 atom = one NF4 block
+constexpr int kWStageBytes = kBM * kBK * 2;  // 16 KB bf16 operand tile
+constexpr int kMaxStages = 4;
+constexpr int kMaxRing = 8;
+constexpr uint32_t kSmemBudget = 227 * 1024;
+
+struct KParams {
+  int M, T, Kc;
+  int bn, nacc, stages, ring_stages;
+  int kt_total, kt_per_split, splits;
+  uint32_t ring_bytes, alloc_cols;
+  const float* absmax;
+  int w_rows, w_cols;
+  int slab_w, jofs_by_part, n_parts;
+  const float* la;
+  long long la_rs, la_cs;
+  float la_scale;
+  const float* lb;
+  long long lb_ld;
+  long long part_end[4];
+  void* out;
+  int out_f32;
+  long long ldo;
+  const uint16_t* residual;
+  long long ldr;
+  float* partial;
+  int* dev_err;
+  float levels[16];
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int WMODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
+                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ KParams p) {
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ __align__(8) uint64_t bar_full[kMaxStages];
+  __shared__ __align__(8) uint64_t bar_empty[kMaxStages];
+  __shared__ __align__(8) uint64_t bar_cfull[kMaxRing];
+  __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
+  __shared__ __align__(8) uint64_t bar_acc;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float lv_sh[16];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &abort_sh;
+
+  const int BT = p.nacc * p.bn;
+  const uint32_t acc_stride = (p.nacc > 1) ? 256u : 0u;  // TMEM column of accumulator 1
+  const uint32_t xs_bytes = (uint32_t)BT * 128u;
+  uint8_t* dsm = align1024(dsm_raw);
+  uint8_t* xs0 = dsm;
+  uint8_t* ws0 = xs0 + (size_t)p.stages * xs_bytes;
+  uint8_t* rg0 = ws0 + (size_t)p.stages * kWStageBytes;
+
+  const int m0 = blockIdx.x * kBM;
+  const int t0 = blockIdx.y * BT;
+  const int split = blockIdx.z;
+  const int kt_begin = split * p.kt_per_split;
+  const int kt_end = min(p.kt_total, kt_begin + p.kt_per_split);
+  const int n_main = max(0, kt_end - kt_begin);
+  const int n_slab = (split == 0 && p.slab_w > 0) ? (p.slab_w + 63) / 64 : 0;
+  const int n_iter = n_main + n_slab;
+  const int S = p.stages, CS = p.ring_stages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 5);  // 1 producer + 4 operand warps
+      mbar_init(smem_u32(&bar_empty[s]), 1); // tcgen05.commit
+    }
+    for (int c = 0; c < CS; ++c) {
+      mbar_init(smem_u32(&bar_cfull[c]), 1);
+      mbar_init(smem_u32(&bar_cempty[c]), 4);
+    }
+    mbar_init(smem_u32(&bar_acc), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (threadIdx.x < 16) lv_sh[threadIdx.x] = p.levels[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_sh), p.alloc_cols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- activation TMA producer
+    // The whole warp walks the loop (so it reaches the final barrier converged);
+    // lane 0 issues.
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      bool ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                  DEV_ERR_WAIT_GEMM);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      const uint32_t fb = smem_u32(&bar_full[s]);
+      if (lane == 0) {
+        if (it < n_main) {
+          const int kt = kt_begin + it;
+          uint32_t bytes = xs_bytes + (WMODE == W_BF16_N ? (uint32_t)kWStageBytes : 0u);
+          mbar_arrive_expect_tx(fb, bytes);
+          for (int a = 0; a < p.nacc; ++a)
+            tma_load_2d(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * p.bn * 128), &tm_act, fb,
+                        kt * kBK, t0 + a * p.bn);
+          if (WMODE == W_BF16_N)
+            tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fb, kt * kBK, m0);
+        } else {
+          mbar_arrive(fb);
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer (lane 0)
+    const uint32_t idesc = umma_idesc_bf16(kBM, p.bn);
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      bool ok = mbar_wait_bounded(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
+                                  DEV_ERR_WAIT_GEMM);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        int nk = 4;
+        if (it >= n_main) nk = min(4, (p.slab_w - (it - n_main) * 64) / 16);
+        const uint32_t wa = smem_u32(ws0 + (size_t)s * kWStageBytes);
+        const uint32_t xa = smem_u32(xs0 + (size_t)s * xs_bytes);
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint64_t ad = umma_desc_k_sw128(wa + kk * 32);
+          for (int a = 0; a < p.nacc; ++a) {
+            const uint64_t bd = umma_desc_k_sw128(xa + (uint32_t)(a * p.bn * 128) + kk * 32);
+            tc_mma_bf16(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
+                        (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(smem_u32(&bar_empty[s]));
+      }
+      __syncwarp();
+    }
+    if (lane == 0) tc_commit(smem_u32(&bar_acc));
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------------------------------------------------- staging-ring TMA producer
+    if (WMODE != W_BF16_N) {
+      for (int it = 0; it < n_main; ++it) {
+        const int c = it % CS;
+        const uint32_t ph = (uint32_t)(it / CS) & 1u;
+        bool ok = mbar_wait_bounded(smem_u32(&bar_cempty[c]), ph ^ 1u, abort_flag, p.dev_err,
+                                    DEV_ERR_WAIT_GEMM);
+        if (!__all_sync(0xFFFFFFFFu, ok)) break;
+        if (lane == 0) {
+          const int kt = kt_begin + it;
+          const uint32_t cb = smem_u32(&bar_cfull[c]);
+          const uint32_t dst = smem_u32(rg0 + (size_t)c * p.ring_bytes);
+          mbar_arrive_expect_tx(cb, p.ring_bytes);
+          if (WMODE == W_NF4_N) tma_load_2d(dst, &tm_w, cb, kt * 32, m0);       // [128 rows][32 B]
+          if (WMODE == W_NF4_T) tma_load_2d(dst, &tm_w, cb, m0 / 2, kt * kBK);  // [64 rows][64 B]
+          if (WMODE == W_BF16_T) tma_load_2d(dst, &tm_w, cb, m0, kt * kBK);     // [64][128 bf16]
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- operand stage
+    const int tid = threadIdx.x - 128;  // 0..127
+    const int nblk = p.w_cols / 64;
+    bool ok = true;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      uint8_t* wst = ws0 + (size_t)s * kWStageBytes;
+      if (it < n_main) {
+        const int kt = kt_begin + it;
+        if (WMODE == W_BF16_N) {
+          ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                 DEV_ERR_WAIT_GEMM);
+          ok = __all_sync(0xFFFFFFFFu, ok);
+        } else {
+          const int c = it % CS;
+          const uint32_t cph = (uint32_t)(it / CS) & 1u;
+          const uint8_t* ring = rg0 + (size_t)c * p.ring_bytes;
+          if (WMODE == W_NF4_N) {
+            const int m = m0 + tid;
+            const float am = (m < p.w_rows) ? __ldg(p.absmax + (size_t)m * nblk + kt) : 0.f;
+            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM) &&
+                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) {
+              const uint4 c0 = *reinterpret_cast<const uint4*>(ring + tid * 32);
+              const uint4 c1 = *reinterpret_cast<const uint4*>(ring + tid * 32 + 16);
+              const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint32_t w = words[q];
+                uint32_t o[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const uint32_t byte = (w >> (8 * b)) & 0xFFu;
+                  o[b] = pack_bf16x2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
+                }
+                *reinterpret_cast<uint4*>(wst + sw128_offset(tid, q)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          } else if (WMODE == W_NF4_T) {
+            const int bi = tid & 7;   // rows 8bi..8bi+7 of the staged [64 x 128] tile
+            const int bj = tid >> 3;  // columns 8bj..8bj+7 (output features)
+            const int mcol = m0 + 8 * bj;
+            float am[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+              const int n = kt * kBK + 8 * bi + rr;
+              am[rr] = (n < p.w_rows && mcol < p.w_cols)
+                           ? __ldg(p.absmax + (size_t)n * nblk + (mcol >> 6))
+                           : 0.f;
+            }
+            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM) &&
+                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) {
+              uint32_t w[8];
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr)
+                w[rr] = *reinterpret_cast<const uint32_t*>(ring + (8 * bi + rr) * 64 + 4 * bj);
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                float v[8];
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                  const uint32_t byte = (w[rr] >> (8 * (cc >> 1))) & 0xFFu;
+                  const uint32_t code = (cc & 1) ? (byte & 15u) : (byte >> 4);
+                  v[rr] = lv_sh[code] * am[rr];
+                }
+                *reinterpret_cast<uint4*>(wst + sw128_offset(8 * bj + cc, bi)) =
+                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+              }
+            }
+          } else {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
+            const int bi = tid & 7, bj = tid >> 3;
+            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM) &&
+                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                   DEV_ERR_WAIT_GEMM);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) {
+              uint4 rowv[8];
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr)
+                rowv[rr] = *reinterpret_cast<const uint4*>(ring + (8 * bi + rr) * 256 + 16 * bj);
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                uint32_t o[4];
+#pragma unroll
+                for (int pr = 0; pr < 4; ++pr) {
+                  const uint4 a = rowv[2 * pr], b = rowv[2 * pr + 1];
+                  const uint32_t wa = (cc >> 1) == 0 ? a.x : (cc >> 1) == 1 ? a.y : (cc >> 1) == 2 ? a.z : a.w;
+                  const uint32_t wb = (cc >> 1) == 0 ? b.x : (cc >> 1) == 1 ? b.y : (cc >> 1) == 2 ? b.z : b.w;
+                  o[pr] = (cc & 1) ? __byte_perm(wa, wb, 0x7632) : __byte_perm(wa, wb, 0x5410);
+                }
+                *reinterpret_cast<uint4*>(wst + sw128_offset(8 * bj + cc, bi)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          }
+          if (ok) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar_cempty[c]));
+          }
+        }
+      } else {
+        // LoRA slab: la -> weight stage, lb -> activation stage
+        ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (ok) {
+          const int j0 = (it - n_main) * 64;
+          const int wq = min(64, p.slab_w - j0) / 8;  // chunks of 8 slab columns
+          int jofs = 0;
+          if (p.jofs_by_part) {
+            int part = 0;
+            while (part + 1 < p.n_parts && m0 >= p.part_end[part]) ++part;
+            jofs = part * p.slab_w;
+          }
+          {
+            const int m = m0 + tid;
+            for (int q = 0; q < wq; ++q) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const long long j = j0 + 8 * q + e;
+                v[e] = (m < p.M) ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + j * p.la_cs)
+                                 : 0.f;
+              }
+              *reinterpret_cast<uint4*>(wst + sw128_offset(tid, q)) =
+                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                             pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            }
+          }
+          uint8_t* xst = xs0 + (size_t)s * xs_bytes;
+          for (int t = tid; t < BT; t += 128) {
+            const int tg = t0 + t;
+            for (int q = 0; q < wq; ++q) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + jofs + j0 + 8 * q + e)
+                                  : 0.f;
+              *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
+                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                             pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+      }
+      if (ok && lane == 0) mbar_arrive(smem_u32(&bar_full[s]));
+    }
+
+    // ---------------------------------------------------------- epilogue
+    bool acc_ok = ok && mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
+                                          DEV_ERR_WAIT_GEMM);
+    acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
+    if (acc_ok) {
+      tc_fence_after();
+      const int qtr = warp & 3;
+      const int m = m0 + qtr * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(qtr * 32) << 16);
+      for (int a = 0; a < p.nacc; ++a) {
+        for (int c0 = 0; c0 < p.bn; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, r);
+          tmem_ld_wait();
+          const int tb = t0 + a * p.bn + c0;
+          if (m < p.M) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int t = tb + j;
+              if (t < p.T) {
+                float val = __uint_as_float(r[j]);
+                if (p.splits > 1) {
+                  p.partial[((size_t)split * p.T + t) * p.M + m] = val;
+                } else {
+                  if (p.residual) val += bf16_bits_to_float(p.residual[(size_t)t * p.ldr + m]);
+                  if (p.out_f32)
+                    static_cast<float*>(p.out)[(size_t)t * p.ldo + m] = val;
+                  else
+                    static_cast<uint16_t*>(p.out)[(size_t)t * p.ldo + m] = float_to_bf16_bits(val);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (abort_sh) settle_ns(2000000);  // let issued copies and MMAs land before freeing TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.alloc_cols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled get_encode() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(f);
+  });
+  return fn;
+}
+
+int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
+              uint64_t inner, uint64_t rows, uint64_t row_stride_elems, uint32_t box_inner,
+              uint32_t box_rows, CUtensorMapSwizzle sw) {
+  PFN_encodeTiled enc = get_encode();
+  if (!enc) return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_elems * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu rows=%llu",
+                     (int)r, (unsigned long long)inner, (unsigned long long)rows);
+  return LSQ_OK;
+}
+
+struct Plan {
+  int bn, nacc, t_tiles, m_tiles, kt_total, kt_per_split, splits, stages, ring_stages;
+  uint32_t ring_bytes, smem_bytes, alloc_cols;
+  size_t partial_bytes;
+};
+
+int g_num_sms = 0;
+
+Plan make_plan(const GemmDesc& d) {
+  Plan pl{};
+  const int64_t T = d.T;
+  if (T <= 256) {
+    pl.nacc = 1;
+    pl.bn = (int)((T + 15) / 16 * 16);
+  } else {
+    pl.nacc = 2;
+    const int64_t half = (std::min<int64_t>(T, 512) + 1) / 2;
+    pl.bn = (int)std::min<int64_t>(256, (half + 15) / 16 * 16);
+  }
+  const int BT = pl.nacc * pl.bn;
+  pl.t_tiles = (int)((T + BT - 1) / BT);
+  pl.m_tiles = (int)((d.M + kBM - 1) / kBM);
+  pl.kt_total = (int)((d.Kc + kBK - 1) / kBK);
+  const int sms = gemm_num_sms();
+  const int base = pl.m_tiles * pl.t_tiles;
+  int splits = 1;
+  if (d.force_splits > 0) {
+    splits = d.force_splits;
+  } else if (base < sms) {
+    splits = std::max(1, std::min(sms / base, pl.kt_total / 4));
+    splits = std::min(splits, 16);
+  }
+  splits = std::max(1, std::min(splits, pl.kt_total));
+  pl.kt_per_split = (pl.kt_total + splits - 1) / splits;
+  pl.splits = (pl.kt_total + pl.kt_per_split - 1) / pl.kt_per_split;
+  pl.partial_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)T * (size_t)d.M * 4 : 0;
+  pl.ring_bytes = (d.wmode == W_BF16_T) ? 64 * 128 * 2 : (d.wmode == W_BF16_N ? 0 : 4096);
+  const uint32_t xs = (uint32_t)BT * 128;
+  int ring = (d.wmode == W_BF16_N) ? 0 : (d.wmode == W_BF16_T ? 2 : kMaxRing);
+  int stages = kMaxStages;
+  auto total = [&](int st, int rs) {
+    return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes;
+  };
+  while (stages > 2 && total(stages, ring) > kSmemBudget - 4096) --stages;
+  while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;
+  pl.stages = stages;
+  pl.ring_stages = std::max(ring, 1);
+  pl.smem_bytes = total(stages, ring);
+  uint32_t cols = 32;
+  while (cols < (uint32_t)pl.bn) cols <<= 1;
+  pl.alloc_cols = (pl.nacc > 1) ? 512u : cols;
+  return pl;
+}
+
+template <int WMODE>
+int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t st) {
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    LSQ_CUDA(cudaFuncSetAttribute(tc_gemm_kernel<WMODE>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(kSmemBudget - 2048)));
+    attr_done[dev] = true;
+  }
+  CUtensorMap tm_act, tm_w;
+  LSQ_TRY(make_tmap(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.act, (uint64_t)d.Kc,
+                    (uint64_t)d.T, (uint64_t)d.act_ld, kBK, (uint32_t)pl.bn,
+                    CU_TENSOR_MAP_SWIZZLE_128B));
+  if (WMODE == W_NF4_N)
+    LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.w, (uint64_t)d.w_cols / 2,
+                      (uint64_t)d.w_rows, (uint64_t)d.w_cols / 2, 32, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (WMODE == W_NF4_T)
+    LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.w, (uint64_t)d.w_cols / 2,
+                      (uint64_t)d.w_rows, (uint64_t)d.w_cols / 2, 64, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (WMODE == W_BF16_N)
+    LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
+                      (uint64_t)d.w_rows, (uint64_t)d.w_cols, kBK, kBM,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+  if (WMODE == W_BF16_T)
+    LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
+                      (uint64_t)d.w_rows, (uint64_t)d.w_cols, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
+  KParams p{};
+  p.M = (int)d.M;
+  p.T = (int)d.T;
+  p.Kc = (int)d.Kc;
+  p.bn = pl.bn;
+  p.nacc = pl.nacc;
+  p.stages = pl.stages;
+  p.ring_stages = pl.ring_stages;
+  p.kt_total = pl.kt_total;
+  p.kt_per_split = pl.kt_per_split;
+  p.splits = pl.splits;
+  p.ring_bytes = pl.ring_bytes;
+  p.alloc_cols = pl.alloc_cols;
+  p.absmax = d.absmax;
+  p.w_rows = (int)d.w_rows;
+  p.w_cols = (int)d.w_cols;
+  p.slab_w = d.slab_w;
+  p.jofs_by_part = d.jofs_by_part;
+  p.n_parts = d.n_parts;
+  p.la = d.la;
+  p.la_rs = d.la_rs;
+  p.la_cs = d.la_cs;
+  p.la_scale = d.la_scale;
+  p.lb = d.lb;
+  p.lb_ld = d.lb_ld;
+  for (int i = 0; i < 4; ++i) p.part_end[i] = d.part_end[i];
+  p.out = d.out;
+  p.out_f32 = d.out_f32;
+  p.ldo = d.ldo;
+  p.residual = d.residual;
+  p.ldr = d.ldr;
+  p.partial = partial;
+  p.dev_err = device_status_ptr();
+  const float* lv = nf4_levels();
+  for (int i = 0; i < 16; ++i) p.levels[i] = lv[i];
+  if (!p.dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  dim3 grid(pl.m_tiles, pl.t_tiles, pl.splits);
+  tc_gemm_kernel<WMODE><<<grid, kThreads, pl.smem_bytes, st>>>(tm_act, tm_w, p);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
+
+}  // namespace
+
+int gemm_num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_num_sms = n > 0 ? n : 148;
+  }
+  return g_num_sms;
+}
+
+int* device_status_ptr() {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_lsq_dev_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(a);
+  }
+  return ptrs[dev];
+}
+
+size_t gemm_workspace_bytes(const GemmDesc& d) {
+  if (d.M <= 0 || d.T <= 0 || d.Kc <= 0) return 0;
+  return make_plan(d).partial_bytes;
+}
+
+int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (d.M <= 0 || d.T <= 0 || d.Kc <= 0) return set_error(LSQ_ERR_SHAPE, "gemm: empty problem");
+  if (!d.w || !d.act || !d.out) return set_error(LSQ_ERR_INVALID, "gemm: null operand");
+  if ((d.wmode == W_NF4_N || d.wmode == W_NF4_T) && !d.absmax)
+    return set_error(LSQ_ERR_INVALID, "gemm: null absmax");
+  if (d.w_cols % 64 != 0 && (d.wmode == W_NF4_N || d.wmode == W_NF4_T))
+    return set_error(LSQ_ERR_SHAPE, "gemm: NF4 weight columns must be a multiple of 64");
+  if (d.act_ld % 8 != 0 || d.w_cols % 8 != 0)
+    return set_error(LSQ_ERR_SHAPE, "gemm: row strides must be multiples of 16 bytes");
+  if (d.slab_w % 16 != 0 || d.slab_w < 0)
+    return set_error(LSQ_ERR_SHAPE, "gemm: LoRA slab width must be a multiple of 16");
+  if (d.slab_w > 0 && (!d.la || !d.lb)) return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
+  if (d.M > INT32_MAX || d.T > INT32_MAX || d.Kc > INT32_MAX)
+    return set_error(LSQ_ERR_SHAPE, "gemm: dimension too large");
+  Plan pl = make_plan(d);
+  float* partial = nullptr;
+  if (pl.splits > 1) {
+    if (!ws || ws_bytes < pl.partial_bytes)
+      return set_error(LSQ_ERR_WORKSPACE, "gemm: split-K workspace %zu < %zu", ws_bytes,
+                       pl.partial_bytes);
+    partial = static_cast<float*>(ws);
+  }
+  switch (d.wmode) {
+    case W_NF4_N: LSQ_TRY(launch_mode<W_NF4_N>(d, pl, partial, st)); break;
+    case W_NF4_T: LSQ_TRY(launch_mode<W_NF4_T>(d, pl, partial, st)); break;
+    case W_BF16_N: LSQ_TRY(launch_mode<W_BF16_N>(d, pl, partial, st)); break;
+    case W_BF16_T: LSQ_TRY(launch_mode<W_BF16_T>(d, pl, partial, st)); break;
+    default: return set_error(LSQ_ERR_INVALID, "gemm: bad operand mode");
+  }
+  if (pl.splits > 1)
+    LSQ_TRY(launch_splitk_reduce(partial, pl.splits, d.T, d.M, d.out, d.out_f32, d.ldo,
+                                 d.residual, d.ldr, st));
+  return LSQ_OK;
+}
+
+}  // namespace lsq

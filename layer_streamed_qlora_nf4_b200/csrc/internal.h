@@ -1,0 +1,166 @@
+// Internal (non-ABI) declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lsq.h"
+
+namespace lsq {
+
+// ---------------------------------------------------------------- errors
+int set_error(int code, const char* fmt, ...);   // records a message, returns code
+int cuda_status(cudaError_t e, const char* what); // LSQ_OK or LSQ_ERR_CUDA with message
+#define LSQ_TRY(expr)            \
+  do {                           \
+    int _rc = (expr);            \
+    if (_rc != LSQ_OK) return _rc; \
+  } while (0)
+#define LSQ_CUDA(expr) LSQ_TRY(::lsq::cuda_status((expr), #expr))
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device status word bits (latched by kernels, read by lsq_device_status).
+enum { DEV_ERR_WAIT_GEMM = 1, DEV_ERR_NONFINITE = 2 };
+int* device_status_ptr();  // device address of the status word (current device)
+
+// NF4 levels and fp32 decision midpoints, derived on the host from the
+// definition of the data type (see nf4_quant.cu).
+const float* nf4_levels();     // 16
+const float* nf4_midpoints();  // 15
+
+// ---------------------------------------------------------------- workspace
+// Bump allocator over a caller-provided device workspace (256-B granules).
+struct Arena {
+  uint8_t* base = nullptr;
+  size_t cap = 0, used = 0;
+  bool overflow = false;
+  template <class T>
+  T* take(size_t n) {
+    size_t bytes = (n * sizeof(T) + 255) & ~size_t(255);
+    if (used + bytes > cap) {
+      overflow = true;
+      used += bytes;
+      return nullptr;
+    }
+    T* p = reinterpret_cast<T*>(base + used);
+    used += bytes;
+    return p;
+  }
+};
+
+// ---------------------------------------------------------------- tensor-core GEMM
+// out[t, m] = sum_c Wop[m, c] * act[t, c] + sum_j la[m, j] * lb[t, j]  (+ residual[t, m])
+// Wop is produced per tile by the operand stage:
+//   W_NF4_N : Wop[m, c] = deq(W)[m, c]   (W [w_rows = M, w_cols = Kc] NF4; forward)
+//   W_NF4_T : Wop[m, c] = deq(W)[c, m]   (W [w_rows = Kc, w_cols = M] NF4; dX)
+//   W_BF16_N: Wop[m, c] = W[m, c]        (W bf16 [M, Kc])
+//   W_BF16_T: Wop[m, c] = W[c, m]        (W bf16 [Kc, M])
+enum WMode { W_NF4_N = 0, W_NF4_T = 1, W_BF16_N = 2, W_BF16_T = 3 };
+
+struct GemmDesc {
+  int wmode = W_NF4_N;
+  int64_t M = 0, T = 0, Kc = 0;
+  const void* w = nullptr;          // NF4 codes or bf16 weight
+  const float* absmax = nullptr;    // NF4 only
+  int64_t w_rows = 0, w_cols = 0;   // storage shape of W
+  const uint16_t* act = nullptr;    // bf16 [T, act_ld], contraction over the first Kc columns
+  int64_t act_ld = 0;
+  // LoRA slab (an extra K range appended to split 0): la[m, j] = la_scale *
+  // la_ptr[m * la_rs + j * la_cs]; lb[t, j] = lb_ptr[t * lb_ld + jofs + j];
+  // jofs = 0, or part(m) * slab_w when jofs_by_part (part boundaries part_end[]).
+  int slab_w = 0;
+  const float* la = nullptr;
+  int64_t la_rs = 0, la_cs = 0;
+  float la_scale = 0.f;
+  const float* lb = nullptr;
+  int64_t lb_ld = 0;
+  int jofs_by_part = 0;
+  int n_parts = 0;
+  int64_t part_end[4] = {0, 0, 0, 0};
+  // epilogue
+  void* out = nullptr;
+  int out_f32 = 0;
+  int64_t ldo = 0;
+  const uint16_t* residual = nullptr;
+  int64_t ldr = 0;
+  int force_splits = 0;             // 0 = heuristic
+};
+size_t gemm_workspace_bytes(const GemmDesc& d);
+int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st);
+int gemm_num_sms();
+
+// ---------------------------------------------------------------- small kernels
+int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
+                         int out_f32, int64_t ldo, const uint16_t* residual, int64_t ldr,
+                         cudaStream_t st);
+int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
+                       uint16_t* y, float* rstd, cudaStream_t st);
+// dx = dres + rmsnorm_bwd(dy);  writes fp32 dx and (optionally) its bf16 copy
+int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
+                       const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
+                       cudaStream_t st);
+int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, float theta,
+                int inverse, cudaStream_t st);
+int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
+                     int Hkv, int d, float theta, uint16_t* dqkv, cudaStream_t st);
+int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st);
+int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
+                      cudaStream_t st);
+int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D,
+                     int64_t V, uint16_t* out, cudaStream_t st);
+int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq,
+                         int64_t V, float inv_count, uint16_t* dlogits, float* row_loss,
+                         cudaStream_t st);
+int launch_sum_rows(const float* row_loss, int64_t T, float scale, int accumulate, float* out,
+                    cudaStream_t st);
+int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr, float b1,
+                 float b2, float eps, float wd, int step, cudaStream_t st);
+int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st);
+int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
+
+// LoRA skinny products (CUDA cores, fixed-order fp32 reductions)
+// u[t, j] = sum_k x[t, k] * A[j, k]                     x bf16 [T, K], A fp32 [R, K] -> u [T, R]
+// scratch: lora_scratch_bytes(T, K, R) bytes for the fixed-order K-split partials
+size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
+int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K,
+                     int R, float* u, float* scratch, size_t scratch_bytes, cudaStream_t st);
+// v[t, p*r + j] = sum_{n in part p} dy[t, n] * B[n, j] dy bf16 [T, N], B fp32 [N, r]
+// scratch: lora_scratch_bytes(T, max part size, n_parts * r) bytes
+int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r,
+                      int n_parts, const int64_t* part_end, float* v, float* scratch,
+                      size_t scratch_bytes, cudaStream_t st);
+// dA[j, k] (+)= s * sum_t v[t, j] * x[t, k]              v fp32 [T, R], x bf16 [T, K]
+int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
+                       int accumulate, float* dA, cudaStream_t st);
+// dB[n, j] (+)= s * sum_t dy[t, n] * u[t, part(n)*r + j]  dy bf16 [T, N], u fp32 [T, R]
+int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
+                       int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
+                       cudaStream_t st);
+
+// attention (causal GQA), q/k/v read from the fused qkv buffer [T, (H + 2 Hkv) d]
+int launch_attention_fwd(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d,
+                         uint16_t* o, float* lse, cudaStream_t st);
+int launch_attention_bwd(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
+                         const float* lse, int64_t T, int seq, int H, int Hkv, int d, float* delta,
+                         float* dq, float* dk, float* dv, cudaStream_t st);
+
+// ---------------------------------------------------------------- layer internals
+struct LayerShapes {
+  int64_t D, F, qd, kvd, qkv_n, gu_n;
+  int H, Hkv, hd, r;
+  float s;
+};
+int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
+size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);
+// dx_out_bf16 may be null (then converted internally).
+int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+                   int batch, int seq, uint16_t* x_out, void* ws, size_t ws_bytes,
+                   cudaStream_t st);
+int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+                   const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
+                   float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate,
+                   void* ws, size_t ws_bytes, cudaStream_t st);
+
+}  // namespace lsq

@@ -1,0 +1,194 @@
+// NF4 codebook (derived on the host from its definition), blockwise-absmax
+// quantisation and dequantisation kernels.
+//
+// Definition followed (Soup layer-streaming tutorial, "四段資料路徑" part 1: the
+// frozen Linear weights are stored as 4-bit NormalFloat, NF4, computed offline):
+//   levels: standard-normal quantiles with an exact zero - 8 positive levels at
+//   p = delta + i (1/2 - delta) / 8 (i = 0..7), 7 negative levels at
+//   -Phi^-1(delta + i (1/2 - delta) / 7) (i = 0..6), plus 0, divided by
+//   Phi^-1(delta), with delta = ((1 - 1/30) + (1 - 1/32)) / 2; each level is
+//   rounded once to fp32.  Phi^-1 here is found by bisection on
+//   Phi(x) = erfc(-x / sqrt 2) / 2 in long double.
+//   block of 64 consecutive elements, absmax = max |w| (fp32);
+//   code = #{ fp32 midpoints strictly below fl32(w / absmax) }; absmax 0 -> 7;
+//   two codes per byte, even element in the high nibble.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace lsq {
+
+namespace {
+
+float g_levels[16];
+float g_mids[15];
+
+long double phi_inv(long double p) {
+  long double lo = -12.0L, hi = 12.0L;
+  const long double rs2 = 0.70710678118654752440084436210484903928L;
+  for (int i = 0; i < 200; ++i) {
+    long double mid = 0.5L * (lo + hi);
+    long double cdf = 0.5L * erfcl(-mid * rs2);
+    if (cdf < p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return 0.5L * (lo + hi);
+}
+
+void build_codebook() {
+  const long double delta = ((1.0L - 1.0L / 30.0L) + (1.0L - 1.0L / 32.0L)) / 2.0L;
+  long double v[16];
+  int n = 0;
+  for (int i = 0; i < 7; ++i) v[n++] = -phi_inv(delta + i * (0.5L - delta) / 7.0L);
+  v[n++] = 0.0L;
+  for (int i = 7; i >= 0; --i) v[n++] = phi_inv(delta + i * (0.5L - delta) / 8.0L);
+  const long double top = phi_inv(delta);
+  for (int i = 0; i < 16; ++i) g_levels[i] = (float)(v[i] / top);
+  g_levels[0] = -1.0f;   // -Phi^-1(delta)/Phi^-1(delta), exact
+  g_levels[7] = 0.0f;
+  g_levels[15] = 1.0f;
+  for (int i = 0; i < 15; ++i) {
+    volatile float s = g_levels[i] + g_levels[i + 1];  // fp32 sum, then exact halving
+    g_mids[i] = s * 0.5f;
+  }
+}
+
+std::once_flag g_once;
+
+struct QuantParams {
+  float mids[15];
+};
+
+// One warp per 64-element block; lane l owns elements 2l and 2l+1 (one byte).
+__global__ void nf4_quantize_kernel(const float* __restrict__ W, int64_t n_blocks,
+                                    uint8_t* __restrict__ codes, float* __restrict__ absmax,
+                                    QuantParams qp, int* dev_err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t b = warp_global; b < n_blocks; b += n_warps) {
+    const float2 w = reinterpret_cast<const float2*>(W + b * 64)[lane];
+    const bool finite = isfinite(w.x) && isfinite(w.y);
+    if (!__all_sync(0xFFFFFFFFu, finite) && lane == 0) atomicOr(dev_err, DEV_ERR_NONFINITE);
+    float am = fmaxf(fabsf(w.x), fabsf(w.y));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+    uint32_t c0 = 7, c1 = 7;
+    if (am > 0.f) {
+      const float v0 = __fdiv_rn(w.x, am), v1 = __fdiv_rn(w.y, am);
+      c0 = 0;
+      c1 = 0;
+#pragma unroll
+      for (int i = 0; i < 15; ++i) {
+        c0 += (v0 > qp.mids[i]) ? 1u : 0u;
+        c1 += (v1 > qp.mids[i]) ? 1u : 0u;
+      }
+    }
+    codes[b * 32 + lane] = (uint8_t)((c0 << 4) | c1);
+    if (lane == 0) absmax[b] = am;
+  }
+}
+
+struct LevelParams {
+  float lv[16];
+};
+
+__global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                      const float* __restrict__ absmax, int64_t n_bytes,
+                                      float* __restrict__ W, LevelParams lp) {
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_bytes;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    const uint8_t c = codes[j];
+    const float am = absmax[j >> 5];  // 32 bytes per 64-element block
+    W[2 * j] = lp.lv[c >> 4] * am;
+    W[2 * j + 1] = lp.lv[c & 15] * am;
+  }
+}
+
+}  // namespace
+
+const float* nf4_levels() {
+  std::call_once(g_once, build_codebook);
+  return g_levels;
+}
+const float* nf4_midpoints() {
+  std::call_once(g_once, build_codebook);
+  return g_mids;
+}
+
+}  // namespace lsq
+
+using namespace lsq;
+
+extern "C" int lsq_nf4_codebook(float out_levels[16]) {
+  if (!out_levels) return set_error(LSQ_ERR_INVALID, "lsq_nf4_codebook: null output");
+  const float* lv = nf4_levels();
+  for (int i = 0; i < 16; ++i) out_levels[i] = lv[i];
+  return LSQ_OK;
+}
+
+static int check_nf4_shape(int64_t N, int64_t K, int32_t block, const char* who) {
+  if (block != 64) return set_error(LSQ_ERR_SHAPE, "%s: block must be 64 (got %d)", who, block);
+  if (N <= 0 || K <= 0) return set_error(LSQ_ERR_SHAPE, "%s: N and K must be positive", who);
+  if (K % 64 != 0) return set_error(LSQ_ERR_SHAPE, "%s: K %% 64 != 0 (K=%lld)", who, (long long)K);
+  if ((N * K) % 2 != 0) return set_error(LSQ_ERR_SHAPE, "%s: N*K must be even", who);
+  return LSQ_OK;
+}
+
+extern "C" int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block, uint8_t* codes,
+                            float* absmax, void* stream) {
+  LSQ_TRY(check_nf4_shape(N, K, block, "nf4_quantize"));
+  if (!W || !codes || !absmax) return set_error(LSQ_ERR_INVALID, "nf4_quantize: null pointer");
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(absmax))
+    return set_error(LSQ_ERR_ALIGN, "nf4_quantize: pointers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* err = device_status_ptr();
+  if (!err) return set_error(LSQ_ERR_CUDA, "nf4_quantize: no device status word");
+  int h_before = 0;
+  LSQ_CUDA(cudaMemcpyAsync(&h_before, err, sizeof(int), cudaMemcpyDeviceToHost, st));
+  LSQ_CUDA(cudaStreamSynchronize(st));
+  if (h_before & DEV_ERR_NONFINITE) {
+    int v = h_before & ~DEV_ERR_NONFINITE;
+    LSQ_CUDA(cudaMemcpyAsync(err, &v, sizeof(int), cudaMemcpyHostToDevice, st));
+  }
+  QuantParams qp;
+  const float* m = nf4_midpoints();
+  for (int i = 0; i < 15; ++i) qp.mids[i] = m[i];
+  const int64_t n_blocks = N * K / 64;
+  const int threads = 256;
+  int64_t grid = (n_blocks * 32 + threads - 1) / threads;
+  const int64_t cap = (int64_t)gemm_num_sms() * 32;
+  if (grid > cap) grid = cap;
+  nf4_quantize_kernel<<<(unsigned)grid, threads, 0, st>>>(W, n_blocks, codes, absmax, qp, err);
+  LSQ_CUDA(cudaGetLastError());
+  int h_after = 0;
+  LSQ_CUDA(cudaMemcpyAsync(&h_after, err, sizeof(int), cudaMemcpyDeviceToHost, st));
+  LSQ_CUDA(cudaStreamSynchronize(st));
+  if (h_after & DEV_ERR_NONFINITE) {
+    int v = h_after & ~DEV_ERR_NONFINITE;
+    LSQ_CUDA(cudaMemcpy(err, &v, sizeof(int), cudaMemcpyHostToDevice));
+    return set_error(LSQ_ERR_INVALID, "nf4_quantize: W holds a NaN or Inf");
+  }
+  return LSQ_OK;
+}
+
+extern "C" int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+                              int32_t block, float* W_out, void* stream) {
+  LSQ_TRY(check_nf4_shape(N, K, block, "nf4_dequantize"));
+  if (!W_out || !codes || !absmax) return set_error(LSQ_ERR_INVALID, "nf4_dequantize: null pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LevelParams lp;
+  const float* lv = nf4_levels();
+  for (int i = 0; i < 16; ++i) lp.lv[i] = lv[i];
+  const int64_t n_bytes = N * K / 2;
+  int64_t grid = (n_bytes + 255) / 256;
+  const int64_t cap = (int64_t)gemm_num_sms() * 16;
+  if (grid > cap) grid = cap;
+  nf4_dequantize_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, absmax, n_bytes, W_out, lp);
+  LSQ_CUDA(cudaGetLastError());
+  return LSQ_OK;
+}
