@@ -1,0 +1,445 @@
+// One Llama-style decoder layer whose seven frozen projections are NF4 with a
+// LoRA branch each: forward, and backward with the layer recomputed from its
+// saved input (Soup layer-streaming tutorial, "四段資料路徑" part 3, and the
+// "gradient_checkpointing: true" bullet: the streaming wrapper checkpoints
+// every layer, so backward re-reads the layer and rebuilds its activations).
+//
+// Fusions: q|k|v and gate|up are stored back to back in the layer blob, so each
+// group is one NF4 GEMM; the LoRA up-projections ride in those GEMMs as an
+// extra K slab; the o and down GEMMs add the residual in their epilogue.
+#include "common.cuh"
+
+namespace lsq {
+
+int layer_shapes(const lsq_cfg* cfg, LayerShapes* o) {
+  if (!cfg) return set_error(LSQ_ERR_INVALID, "null config");
+  if (cfg->reserved != 0) return set_error(LSQ_ERR_INVALID, "cfg.reserved must be 0");
+  if (cfg->block != 64) return set_error(LSQ_ERR_SHAPE, "cfg.block must be 64");
+  if (cfg->head_dim != 64 && cfg->head_dim != 128)
+    return set_error(LSQ_ERR_SHAPE, "cfg.head_dim must be 64 or 128");
+  if (cfg->n_heads <= 0 || cfg->n_kv_heads <= 0 || cfg->n_heads % cfg->n_kv_heads != 0)
+    return set_error(LSQ_ERR_SHAPE, "cfg: n_heads must be a positive multiple of n_kv_heads");
+  if (cfg->n_heads + cfg->n_kv_heads > 4 * cfg->n_heads)
+    return set_error(LSQ_ERR_SHAPE, "cfg: bad head counts");
+  if (cfg->lora_r <= 0 || cfg->lora_r % 16 != 0 || cfg->lora_r > 64)
+    return set_error(LSQ_ERR_SHAPE, "cfg.lora_r must be 16, 32, 48 or 64");
+  const int64_t qd = (int64_t)cfg->n_heads * cfg->head_dim;
+  const int64_t kvd = (int64_t)cfg->n_kv_heads * cfg->head_dim;
+  if (cfg->hidden <= 0 || cfg->hidden % 128 || cfg->ffn <= 0 || cfg->ffn % 128 || qd % 128 ||
+      kvd % 128)
+    return set_error(LSQ_ERR_SHAPE, "cfg: hidden, ffn, n_heads*head_dim and n_kv_heads*head_dim "
+                                    "must be multiples of 128");
+  o->D = cfg->hidden;
+  o->F = cfg->ffn;
+  o->qd = qd;
+  o->kvd = kvd;
+  o->qkv_n = qd + 2 * kvd;
+  o->gu_n = 2 * cfg->ffn;
+  o->H = cfg->n_heads;
+  o->Hkv = cfg->n_kv_heads;
+  o->hd = cfg->head_dim;
+  o->r = cfg->lora_r;
+  o->s = cfg->lora_alpha / (float)cfg->lora_r;
+  return LSQ_OK;
+}
+
+namespace {
+
+struct Views {  // pointers into one layer blob / one LoRA block
+  const uint8_t* codes[7];
+  const float* absmax[7];
+  const uint16_t* g1;
+  const uint16_t* g2;
+  const float *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_d, *B_d;
+};
+
+void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) {
+  const int64_t rows[7] = {s.qd, s.kvd, s.kvd, s.D, s.F, s.F, s.D};
+  const int64_t cols[7] = {s.D, s.D, s.D, s.qd, s.D, s.D, s.F};
+  uint64_t off = 0;
+  for (int p = 0; p < 7; ++p) {
+    L->rows[p] = rows[p];
+    L->cols[p] = cols[p];
+    L->codes_off[p] = off;
+    off += (uint64_t)rows[p] * cols[p] / 2;
+  }
+  off = (off + 255) & ~uint64_t(255);
+  for (int p = 0; p < 7; ++p) {
+    L->absmax_off[p] = off;
+    off += (uint64_t)rows[p] * cols[p] / 64 * 4;
+  }
+  off = (off + 255) & ~uint64_t(255);
+  L->g1_off = off;
+  off += (uint64_t)s.D * 2;
+  off = (off + 255) & ~uint64_t(255);
+  L->g2_off = off;
+  off += (uint64_t)s.D * 2;
+  L->bytes = (off + 255) & ~uint64_t(255);
+  // LoRA block, each piece 64-float aligned
+  auto al = [](int64_t x) { return (x + 63) & ~int64_t(63); };
+  const int64_t r = s.r;
+  int64_t f = 0;
+  const int64_t a_qkv = f;  f = al(f + 3 * r * s.D);
+  const int64_t b_qkv = f;  f = al(f + s.qkv_n * r);
+  const int64_t a_o = f;    f = al(f + r * s.qd);
+  const int64_t b_o = f;    f = al(f + s.D * r);
+  const int64_t a_gu = f;   f = al(f + 2 * r * s.D);
+  const int64_t b_gu = f;   f = al(f + s.gu_n * r);
+  const int64_t a_d = f;    f = al(f + r * s.F);
+  const int64_t b_d = f;    f = al(f + s.D * r);
+  R->a_off[0] = a_qkv;             R->b_off[0] = b_qkv;
+  R->a_off[1] = a_qkv + r * s.D;   R->b_off[1] = b_qkv + s.qd * r;
+  R->a_off[2] = a_qkv + 2 * r * s.D; R->b_off[2] = b_qkv + (s.qd + s.kvd) * r;
+  R->a_off[3] = a_o;               R->b_off[3] = b_o;
+  R->a_off[4] = a_gu;              R->b_off[4] = b_gu;
+  R->a_off[5] = a_gu + r * s.D;    R->b_off[5] = b_gu + s.F * r;
+  R->a_off[6] = a_d;               R->b_off[6] = b_d;
+  R->floats_per_layer = f;
+}
+
+Views views(const LayerShapes& s, const void* blob, const float* lora) {
+  lsq_layer_layout L;
+  lsq_lora_layout R;
+  fill_layout(s, &L, &R);
+  Views v;
+  const uint8_t* b = static_cast<const uint8_t*>(blob);
+  for (int p = 0; p < 7; ++p) {
+    v.codes[p] = b + L.codes_off[p];
+    v.absmax[p] = reinterpret_cast<const float*>(b + L.absmax_off[p]);
+  }
+  v.g1 = reinterpret_cast<const uint16_t*>(b + L.g1_off);
+  v.g2 = reinterpret_cast<const uint16_t*>(b + L.g2_off);
+  v.A_qkv = lora + R.a_off[0];
+  v.B_qkv = lora + R.b_off[0];
+  v.A_o = lora + R.a_off[3];
+  v.B_o = lora + R.b_off[3];
+  v.A_gu = lora + R.a_off[4];
+  v.B_gu = lora + R.b_off[4];
+  v.A_d = lora + R.a_off[6];
+  v.B_d = lora + R.b_off[6];
+  return v;
+}
+
+// Workspace carve-up (identical for the forward and the backward).
+struct Buffers {
+  uint16_t *n1, *qkv, *ao, *h, *n2, *gu, *m, *dgu, *dqkv, *da, *dout_b, *dh_b;
+  float *rstd1, *rstd2, *u_qkv, *u_o, *u_gu, *u_d, *lse, *v_qkv, *v_o, *v_gu, *v_d;
+  float *dm, *dn2, *dh, *dn1, *dq, *dk, *dv, *delta;
+  float* lscratch;
+  size_t lscratch_bytes;
+  void* gemm;
+  size_t gemm_bytes;
+};
+
+GemmDesc nf4_fwd(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+                 const uint16_t* act, int64_t T, const float* B, int r, float s, const float* u,
+                 int64_t u_ld, int n_parts, const int64_t* pe, const uint16_t* res, void* out,
+                 int64_t ldo) {
+  GemmDesc d;
+  d.wmode = W_NF4_N;
+  d.M = N;
+  d.T = T;
+  d.Kc = K;
+  d.w = codes;
+  d.absmax = absmax;
+  d.w_rows = N;
+  d.w_cols = K;
+  d.act = act;
+  d.act_ld = K;
+  d.slab_w = r;
+  d.la = B;
+  d.la_rs = r;
+  d.la_cs = 1;
+  d.la_scale = s;
+  d.lb = u;
+  d.lb_ld = u_ld;
+  d.jofs_by_part = n_parts > 1;
+  d.n_parts = n_parts;
+  for (int i = 0; i < n_parts && i < 4; ++i) d.part_end[i] = pe[i];
+  d.out = out;
+  d.ldo = ldo;
+  d.residual = res;
+  d.ldr = ldo;
+  return d;
+}
+
+// dX of a stacked NF4 weight W [N, K]: out [T, K] = dy W + s v A_stack, v [T, R], A [R, K]
+GemmDesc nf4_dx(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+                const uint16_t* dy, int64_t T, const float* A, int R, float s, const float* v,
+                void* out, int out_f32) {
+  GemmDesc d;
+  d.wmode = W_NF4_T;
+  d.M = K;
+  d.T = T;
+  d.Kc = N;
+  d.w = codes;
+  d.absmax = absmax;
+  d.w_rows = N;
+  d.w_cols = K;
+  d.act = dy;
+  d.act_ld = N;
+  d.slab_w = R;
+  d.la = A;
+  d.la_rs = 1;
+  d.la_cs = K;
+  d.la_scale = s;
+  d.lb = v;
+  d.lb_ld = R;
+  d.out = out;
+  d.out_f32 = out_f32;
+  d.ldo = K;
+  return d;
+}
+
+size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
+  Arena a;
+  a.base = static_cast<uint8_t*>(base);
+  a.cap = SIZE_MAX;
+  const int r = s.r;
+  Buffers x{};
+  x.n1 = a.take<uint16_t>(T * s.D);
+  x.qkv = a.take<uint16_t>(T * s.qkv_n);
+  x.ao = a.take<uint16_t>(T * s.qd);
+  x.h = a.take<uint16_t>(T * s.D);
+  x.n2 = a.take<uint16_t>(T * s.D);
+  x.gu = a.take<uint16_t>(T * s.gu_n);
+  x.m = a.take<uint16_t>(T * s.F);
+  x.dgu = a.take<uint16_t>(T * s.gu_n);
+  x.dqkv = a.take<uint16_t>(T * s.qkv_n);
+  x.da = a.take<uint16_t>(T * s.qd);
+  x.dout_b = a.take<uint16_t>(T * s.D);
+  x.dh_b = a.take<uint16_t>(T * s.D);
+  x.rstd1 = a.take<float>(T);
+  x.rstd2 = a.take<float>(T);
+  x.u_qkv = a.take<float>(T * 3 * r);
+  x.u_o = a.take<float>(T * r);
+  x.u_gu = a.take<float>(T * 2 * r);
+  x.u_d = a.take<float>(T * r);
+  x.lse = a.take<float>(T * s.H);
+  x.v_qkv = a.take<float>(T * 3 * r);
+  x.v_o = a.take<float>(T * r);
+  x.v_gu = a.take<float>(T * 2 * r);
+  x.v_d = a.take<float>(T * r);
+  x.dm = a.take<float>(T * s.F);
+  x.dn2 = a.take<float>(T * s.D);
+  x.dh = a.take<float>(T * s.D);
+  x.dn1 = a.take<float>(T * s.D);
+  x.dq = a.take<float>(T * s.qd);
+  x.dk = a.take<float>(T * s.kvd);
+  x.dv = a.take<float>(T * s.kvd);
+  x.delta = a.take<float>(T * s.H);
+  // LoRA K-split scratch: the largest of every skinny product in the layer
+  size_t ls = 0;
+  const int64_t Ks[4] = {s.D, s.qd, s.F, std::max(s.qkv_n, s.gu_n)};
+  for (int i = 0; i < 4; ++i) ls = std::max(ls, lora_scratch_bytes(T, Ks[i], 3 * r));
+  x.lscratch = a.take<float>(ls / sizeof(float) + 1);
+  x.lscratch_bytes = ls;
+  // GEMM split-K partials: the largest of the layer's GEMMs
+  const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
+  const int64_t pe2[2] = {s.F, s.gu_n};
+  size_t gb = 0;
+  GemmDesc ds[8] = {
+      nf4_fwd(nullptr, nullptr, s.qkv_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 3 * r, 3, pe3,
+              nullptr, nullptr, s.qkv_n),
+      nf4_fwd(nullptr, nullptr, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
+              nullptr, s.D),
+      nf4_fwd(nullptr, nullptr, s.gu_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 2 * r, 2, pe2,
+              nullptr, nullptr, s.gu_n),
+      nf4_fwd(nullptr, nullptr, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
+              nullptr, s.D),
+      nf4_dx(nullptr, nullptr, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, nullptr, 1),
+      nf4_dx(nullptr, nullptr, s.gu_n, s.D, nullptr, T, nullptr, 2 * r, 0, nullptr, nullptr, 1),
+      nf4_dx(nullptr, nullptr, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, nullptr, 0),
+      nf4_dx(nullptr, nullptr, s.qkv_n, s.D, nullptr, T, nullptr, 3 * r, 0, nullptr, nullptr, 1)};
+  for (auto& d : ds) gb = std::max(gb, gemm_workspace_bytes(d));
+  x.gemm = a.take<uint8_t>(gb + 256);
+  x.gemm_bytes = gb + 256;
+  if (b) *b = x;
+  return a.used;
+}
+
+int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, const void* x,
+                     int batch, int seq, const void* out, LayerShapes* s, const char* who) {
+  LSQ_TRY(layer_shapes(cfg, s));
+  if (!blob || !lora || !x || !out) return set_error(LSQ_ERR_INVALID, "%s: null pointer", who);
+  if (batch <= 0 || seq <= 0) return set_error(LSQ_ERR_SHAPE, "%s: batch and seq must be >= 1", who);
+  if (!aligned16(blob) || !aligned16(lora) || !aligned16(x) || !aligned16(out))
+    return set_error(LSQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", who);
+  return LSQ_OK;
+}
+
+// Forward through the SwiGLU product (everything the backward needs) and,
+// when x_out is given, the down projection with its residual.
+int forward_core(const LayerShapes& s, const Views& v, const uint16_t* x, int batch, int seq,
+                 float theta, float eps, const Buffers& b, uint16_t* x_out, cudaStream_t st) {
+  const int64_t T = (int64_t)batch * seq;
+  const int r = s.r;
+  const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
+  const int64_t pe2[2] = {s.F, s.gu_n};
+  LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, b.rstd1, st));
+  LSQ_TRY(launch_lora_down(b.n1, s.D, v.A_qkv, T, s.D, 3 * r, b.u_qkv, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
+                           3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, theta, 0, st));
+  LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
+  LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
+                           pe3, x, b.h, s.D),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, b.rstd2, st));
+  LSQ_TRY(launch_lora_down(b.n2, s.D, v.A_gu, T, s.D, 2 * r, b.u_gu, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
+                           2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_swiglu_fwd(b.gu, T, s.F, b.m, st));
+  LSQ_TRY(launch_lora_down(b.m, s.F, v.A_d, T, s.F, r, b.u_d, b.lscratch, b.lscratch_bytes, st));
+  if (x_out)
+    LSQ_TRY(gemm_run(nf4_fwd(v.codes[6], v.absmax[6], s.D, s.F, b.m, T, v.B_d, r, s.s, b.u_d, r, 1,
+                             pe3, b.h, x_out, s.D),
+                     b.gemm, b.gemm_bytes, st));
+  return LSQ_OK;
+}
+
+}  // namespace
+
+size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
+  LayerShapes s;
+  if (layer_shapes(cfg, &s) != LSQ_OK || T <= 0) return 0;
+  return plan_buffers(s, T, nullptr, nullptr);
+}
+
+int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+                   int batch, int seq, uint16_t* x_out, void* ws, size_t ws_bytes,
+                   cudaStream_t st) {
+  LayerShapes s;
+  LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd"));
+  const int64_t T = (int64_t)batch * seq;
+  const size_t need = plan_buffers(s, T, nullptr, nullptr);
+  if (!ws || ws_bytes < need)
+    return set_error(LSQ_ERR_WORKSPACE, "decoder_layer_fwd: workspace %zu < %zu", ws_bytes, need);
+  Buffers b;
+  plan_buffers(s, T, ws, &b);
+  const Views v = views(s, blob, lora);
+  return forward_core(s, v, x_in, batch, seq, cfg->rope_theta, cfg->rms_eps, b, x_out, st);
+}
+
+int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+                   const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
+                   float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate, void* ws,
+                   size_t ws_bytes, cudaStream_t st) {
+  LayerShapes s;
+  LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, dx_in, &s, "decoder_layer_bwd"));
+  if (!dx_out || !lora_grad) return set_error(LSQ_ERR_INVALID, "decoder_layer_bwd: null pointer");
+  const int64_t T = (int64_t)batch * seq;
+  const size_t need = plan_buffers(s, T, nullptr, nullptr);
+  if (!ws || ws_bytes < need)
+    return set_error(LSQ_ERR_WORKSPACE, "decoder_layer_bwd: workspace %zu < %zu", ws_bytes, need);
+  Buffers b;
+  plan_buffers(s, T, ws, &b);
+  const Views v = views(s, blob, lora);
+  lsq_layer_layout LL;
+  lsq_lora_layout RL;
+  fill_layout(s, &LL, &RL);
+  float* gA_qkv = lora_grad + RL.a_off[0];
+  float* gB_qkv = lora_grad + RL.b_off[0];
+  float* gA_o = lora_grad + RL.a_off[3];
+  float* gB_o = lora_grad + RL.b_off[3];
+  float* gA_gu = lora_grad + RL.a_off[4];
+  float* gB_gu = lora_grad + RL.b_off[4];
+  float* gA_d = lora_grad + RL.a_off[6];
+  float* gB_d = lora_grad + RL.b_off[6];
+  const int r = s.r;
+  const float sc = s.s;
+  const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
+  const int64_t pe2[2] = {s.F, s.gu_n};
+  const int64_t pe1[1] = {s.D};
+
+  // recompute the forward from the saved input
+  LSQ_TRY(forward_core(s, v, x_in, batch, seq, cfg->rope_theta, cfg->rms_eps, b, nullptr, st));
+
+  const uint16_t* dout_b = dx_out_bf16;
+  if (!dout_b) {
+    LSQ_TRY(launch_f32_to_bf16(dx_out, T * s.D, b.dout_b, st));
+    dout_b = b.dout_b;
+  }
+  // down projection
+  LSQ_TRY(launch_lora_vproj(dout_b, T, s.D, v.B_d, r, 1, pe1, b.v_d, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.A_d, r, sc, b.v_d, b.dm, 1),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_d, b.m, T, s.F, r, sc, accumulate, gA_d, st));
+  LSQ_TRY(launch_lora_grad_b(dout_b, b.u_d, T, s.D, r, r, 1, pe1, sc, accumulate, gB_d, st));
+  // SwiGLU and gate|up
+  LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
+  LSQ_TRY(launch_lora_vproj(b.dgu, T, s.gu_n, v.B_gu, r, 2, pe2, b.v_gu, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc, b.v_gu,
+                          b.dn2, 1),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, st));
+  LSQ_TRY(launch_lora_grad_b(b.dgu, b.u_gu, T, s.gu_n, r, 2 * r, 2, pe2, sc, accumulate, gB_gu, st));
+  // second RMSNorm + residual
+  LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
+  // o projection
+  LSQ_TRY(launch_lora_vproj(b.dh_b, T, s.D, v.B_o, r, 1, pe1, b.v_o, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.A_o, r, sc, b.v_o, b.da, 0),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, st));
+  LSQ_TRY(launch_lora_grad_b(b.dh_b, b.u_o, T, s.D, r, r, 1, pe1, sc, accumulate, gB_o, st));
+  // attention, RoPE
+  LSQ_TRY(launch_attention_bwd(b.qkv, b.ao, b.da, b.lse, T, seq, s.H, s.Hkv, s.hd, b.delta, b.dq,
+                               b.dk, b.dv, st));
+  LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, cfg->rope_theta, b.dqkv, st));
+  // q|k|v projections
+  LSQ_TRY(launch_lora_vproj(b.dqkv, T, s.qkv_n, v.B_qkv, r, 3, pe3, b.v_qkv, b.lscratch,
+                            b.lscratch_bytes, st));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
+                          b.v_qkv, b.dn1, 1),
+                   b.gemm, b.gemm_bytes, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, st));
+  LSQ_TRY(launch_lora_grad_b(b.dqkv, b.u_qkv, T, s.qkv_n, r, 3 * r, 3, pe3, sc, accumulate, gB_qkv, st));
+  // first RMSNorm + residual
+  LSQ_TRY(launch_rmsnorm_bwd(b.dn1, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16, st));
+  return LSQ_OK;
+}
+
+}  // namespace lsq
+
+using namespace lsq;
+
+extern "C" int lsq_layer_layout_get(const lsq_cfg* cfg, lsq_layer_layout* out) {
+  if (!out) return set_error(LSQ_ERR_INVALID, "lsq_layer_layout_get: null output");
+  LayerShapes s;
+  LSQ_TRY(layer_shapes(cfg, &s));
+  lsq_lora_layout R;
+  fill_layout(s, out, &R);
+  return LSQ_OK;
+}
+
+extern "C" int lsq_lora_layout_get(const lsq_cfg* cfg, lsq_lora_layout* out) {
+  if (!out) return set_error(LSQ_ERR_INVALID, "lsq_lora_layout_get: null output");
+  LayerShapes s;
+  LSQ_TRY(layer_shapes(cfg, &s));
+  lsq_layer_layout L;
+  fill_layout(s, &L, out);
+  return LSQ_OK;
+}
+
+extern "C" size_t decoder_layer_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t seq) {
+  if (batch <= 0 || seq <= 0) return 0;
+  return layer_ws_bytes(cfg, (int64_t)batch * seq);
+}
+
+extern "C" int decoder_layer_fwd(const lsq_cfg* cfg, const void* blob, const float* lora,
+                                 const uint16_t* x_in, int32_t batch, int32_t seq, uint16_t* x_out,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return layer_fwd_impl(cfg, blob, lora, x_in, batch, seq, x_out, ws, ws_bytes,
+                        static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int decoder_layer_bwd(const lsq_cfg* cfg, const void* blob, const float* lora,
+                                 const uint16_t* x_in, const float* dx_out, int32_t batch,
+                                 int32_t seq, float* dx_in, float* lora_grad, int32_t accumulate,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return layer_bwd_impl(cfg, blob, lora, x_in, dx_out, nullptr, batch, seq, dx_in, nullptr,
+                        lora_grad, accumulate, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,415 @@
+// The streamed decoder stack and one SFT optimiser step.
+//
+// Method (Soup layer-streaming tutorial, "四段資料路徑" parts 2-3; Layer Streaming
+// blog, "層流技術：技術實作與記憶體效率"; RepoDaily review, "架构解读"): the frozen
+// decoder stack lives in page-locked host memory; two fixed VRAM buffers take
+// one layer each; while the GPU computes layer i from one buffer, a dedicated
+// copy stream loads the next layer into the other; forward walks 0..L-1,
+// backward walks L-1..0 recomputing each layer, so each layer is needed twice
+// per micro-batch.  Embedding, lm_head, LoRA, gradients and optimiser state
+// stay resident.
+//
+// Schedule: the sequence of layer visits of the whole step is planned on the
+// host.  A visit whose layer is already in a buffer uses it in place (the turn
+// from forward to backward, and the first layers of the next step or
+// micro-batch, find their layers still resident); otherwise the layer is copied
+// into the buffer the previous visit did not use.  Fences: the copy stream
+// waits on the event recorded after the last compute that read the target
+// buffer ("free"); the compute stream waits on the event recorded after the
+// copy ("ready").  Copies run one visit ahead.  Kernels are deterministic, so
+// a streamed step is bit-identical to the same step with the stack resident.
+#include <chrono>
+#include <thread>
+#include <vector>
+
+#include "common.cuh"
+
+struct lsq_stack {
+  lsq_cfg cfg;
+  lsq::LayerShapes shapes;
+  lsq_layer_layout layout;
+  lsq_lora_layout lora_layout;
+  std::vector<const void*> blobs;
+  void* buf[2];
+  int resident;
+  int device;
+  cudaStream_t copy_stream;
+  cudaEvent_t ready[2], freed[2];
+  int buf_layer[2];            // layer held by each buffer (after the enqueued copies)
+  std::vector<cudaEvent_t> wait_ev;  // pairs around each compute-side wait (timing)
+  cudaEvent_t t_start, t_end, done;
+  float* loss_host;            // pinned
+  lsq_step_stats stats;
+  int n_waits_last;
+};
+
+namespace lsq {
+namespace {
+
+struct StackWs {
+  uint16_t* xs;      // [L+1][T][D] bf16: layer inputs (saved for backward) and final hidden
+  uint16_t* hf;      // [T][D] final-norm output
+  float* rstd_f;     // [T]
+  float* logits;     // [T][V]
+  uint16_t* dlogits; // [T][V]
+  float* row_loss;   // [T]
+  float* loss_dev;   // [1]
+  float* dhf;        // [T][D]
+  float* dh[2];      // [T][D] fp32 residual-stream gradient (ping-pong)
+  uint16_t* dhb[2];  // bf16 copies
+  void* gemm;
+  size_t gemm_bytes;
+  void* layer_ws;
+  size_t layer_ws_bytes;
+};
+
+GemmDesc head_fwd(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* hf, int64_t T,
+                  float* logits) {
+  GemmDesc d;
+  d.wmode = W_BF16_N;
+  d.M = V;
+  d.T = T;
+  d.Kc = D;
+  d.w = lm_head;
+  d.w_rows = V;
+  d.w_cols = D;
+  d.act = hf;
+  d.act_ld = D;
+  d.out = logits;
+  d.out_f32 = 1;
+  d.ldo = V;
+  return d;
+}
+
+GemmDesc head_dx(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* dlogits,
+                 int64_t T, float* dhf) {
+  GemmDesc d;
+  d.wmode = W_BF16_T;
+  d.M = D;
+  d.T = T;
+  d.Kc = V;
+  d.w = lm_head;
+  d.w_rows = V;
+  d.w_cols = D;
+  d.act = dlogits;
+  d.act_ld = V;
+  d.out = dhf;
+  d.out_f32 = 1;
+  d.ldo = D;
+  return d;
+}
+
+size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* base, StackWs* w) {
+  Arena a;
+  a.base = static_cast<uint8_t*>(base);
+  a.cap = SIZE_MAX;
+  StackWs x{};
+  const int64_t V = cfg->vocab, D = s.D;
+  x.xs = a.take<uint16_t>((size_t)(cfg->n_layers + 1) * T * D);
+  x.hf = a.take<uint16_t>(T * D);
+  x.rstd_f = a.take<float>(T);
+  x.logits = a.take<float>((size_t)T * V);
+  x.dlogits = a.take<uint16_t>((size_t)T * V);
+  x.row_loss = a.take<float>(T);
+  x.loss_dev = a.take<float>(64);
+  x.dhf = a.take<float>(T * D);
+  for (int i = 0; i < 2; ++i) {
+    x.dh[i] = a.take<float>(T * D);
+    x.dhb[i] = a.take<uint16_t>(T * D);
+  }
+  const size_t gb = std::max(gemm_workspace_bytes(head_fwd(nullptr, V, D, nullptr, T, nullptr)),
+                             gemm_workspace_bytes(head_dx(nullptr, V, D, nullptr, T, nullptr)));
+  x.gemm = a.take<uint8_t>(gb + 256);
+  x.gemm_bytes = gb + 256;
+  x.layer_ws_bytes = layer_ws_bytes(cfg, T);
+  x.layer_ws = a.take<uint8_t>(x.layer_ws_bytes);
+  if (w) *w = x;
+  return a.used;
+}
+
+struct Visit {
+  int layer;
+  int fwd;
+  int buf;
+  int copy;
+};
+
+// Plans buffer use for the visit sequence, starting from the buffers' contents.
+std::vector<Visit> plan_visits(int L, int micro_batches, int bl0, int bl1) {
+  std::vector<Visit> v;
+  int held[2] = {bl0, bl1};
+  int prev_buf = 1;  // so that the first copy goes to buffer 0
+  for (int mb = 0; mb < micro_batches; ++mb) {
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int k = 0; k < L; ++k) {
+        const int layer = pass == 0 ? k : L - 1 - k;
+        Visit x{layer, pass == 0, 0, 0};
+        if (held[0] == layer)
+          x.buf = 0;
+        else if (held[1] == layer)
+          x.buf = 1;
+        else {
+          x.buf = 1 - prev_buf;
+          x.copy = 1;
+          held[x.buf] = layer;
+        }
+        prev_buf = x.buf;
+        v.push_back(x);
+      }
+    }
+  }
+  return v;
+}
+
+int wait_event_timeout(cudaEvent_t ev, int64_t timeout_ms) {
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    cudaError_t e = cudaEventQuery(ev);
+    if (e == cudaSuccess) return LSQ_OK;
+    if (e != cudaErrorNotReady) return cuda_status(e, "cudaEventQuery");
+    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                        std::chrono::steady_clock::now() - t0)
+                        .count();
+    if (timeout_ms >= 0 && ms > timeout_ms)
+      return set_error(LSQ_ERR_TIMEOUT, "stream_stack_step: no completion after %lld ms",
+                       (long long)timeout_ms);
+    std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+}
+
+}  // namespace
+}  // namespace lsq
+
+using namespace lsq;
+
+extern "C" size_t stream_stack_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t seq) {
+  LayerShapes s;
+  if (batch <= 0 || seq <= 0 || layer_shapes(cfg, &s) != LSQ_OK || cfg->n_layers <= 0 ||
+      cfg->vocab <= 0)
+    return 0;
+  return plan_stack_ws(cfg, s, (int64_t)batch * seq, nullptr, nullptr);
+}
+
+extern "C" int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_blobs,
+                                   int32_t n_layers, void* vram_buf0, void* vram_buf1,
+                                   int32_t resident, lsq_stack** out) {
+  if (!out) return set_error(LSQ_ERR_INVALID, "stream_stack_create: null output");
+  *out = nullptr;
+  LayerShapes s;
+  LSQ_TRY(layer_shapes(cfg, &s));
+  if (n_layers != cfg->n_layers || n_layers <= 0)
+    return set_error(LSQ_ERR_SHAPE, "stream_stack_create: n_layers %d != cfg.n_layers %d", n_layers,
+                     cfg->n_layers);
+  if (cfg->vocab <= 0 || cfg->vocab % 8 != 0)
+    return set_error(LSQ_ERR_SHAPE, "stream_stack_create: vocab must be a positive multiple of 8");
+  if (!layer_blobs) return set_error(LSQ_ERR_INVALID, "stream_stack_create: null layer list");
+  for (int i = 0; i < n_layers; ++i)
+    if (!layer_blobs[i] || !aligned16(layer_blobs[i]))
+      return set_error(LSQ_ERR_INVALID, "stream_stack_create: layer %d blob null or unaligned", i);
+  if (resident != 0 && resident != 1) return set_error(LSQ_ERR_INVALID, "resident must be 0 or 1");
+  if (!resident && (!vram_buf0 || !vram_buf1 || !aligned16(vram_buf0) || !aligned16(vram_buf1)))
+    return set_error(LSQ_ERR_INVALID, "stream_stack_create: two aligned VRAM buffers are needed");
+  if (!resident) {
+    for (int i = 0; i < n_layers; ++i) {
+      cudaPointerAttributes at;
+      if (cudaPointerGetAttributes(&at, layer_blobs[i]) != cudaSuccess ||
+          at.type != cudaMemoryTypeHost) {
+        cudaGetLastError();
+        return set_error(LSQ_ERR_INVALID,
+                         "stream_stack_create: layer %d blob is not page-locked host memory", i);
+      }
+    }
+  }
+  lsq_stack* h = new lsq_stack();
+  h->cfg = *cfg;
+  h->shapes = s;
+  lsq_layer_layout_get(cfg, &h->layout);
+  lsq_lora_layout_get(cfg, &h->lora_layout);
+  h->blobs.assign(layer_blobs, layer_blobs + n_layers);
+  h->buf[0] = vram_buf0;
+  h->buf[1] = vram_buf1;
+  h->resident = resident;
+  h->buf_layer[0] = h->buf_layer[1] = -1;
+  h->n_waits_last = 0;
+  h->stats = lsq_step_stats{};
+  cudaGetDevice(&h->device);
+  int rc = LSQ_OK;
+  if (cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+    rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create copy stream");
+  for (int i = 0; rc == LSQ_OK && i < 2; ++i)
+    if (cudaEventCreateWithFlags(&h->ready[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->freed[i], cudaEventDisableTiming) != cudaSuccess)
+      rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create events");
+  if (rc == LSQ_OK &&
+      (cudaEventCreate(&h->t_start) != cudaSuccess || cudaEventCreate(&h->t_end) != cudaSuccess ||
+       cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) != cudaSuccess))
+    rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create events");
+  if (rc == LSQ_OK && cudaMallocHost(&h->loss_host, sizeof(float)) != cudaSuccess)
+    rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot allocate the pinned loss slot");
+  if (rc != LSQ_OK) {
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return LSQ_OK;
+}
+
+extern "C" int stream_stack_destroy(lsq_stack* h) {
+  if (!h) return LSQ_OK;
+  cudaStreamSynchronize(h->copy_stream);
+  cudaStreamDestroy(h->copy_stream);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventDestroy(h->ready[i]);
+    cudaEventDestroy(h->freed[i]);
+  }
+  for (auto e : h->wait_ev) cudaEventDestroy(e);
+  cudaEventDestroy(h->t_start);
+  cudaEventDestroy(h->t_end);
+  cudaEventDestroy(h->done);
+  cudaFreeHost(h->loss_host);
+  delete h;
+  return LSQ_OK;
+}
+
+extern "C" int stream_stack_last_stats(const lsq_stack* h, lsq_step_stats* out) {
+  if (!h || !out) return set_error(LSQ_ERR_INVALID, "stream_stack_last_stats: null pointer");
+  *out = h->stats;
+  return LSQ_OK;
+}
+
+extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t micro_batches,
+                                 int32_t batch, int32_t seq, const uint16_t* emb,
+                                 const uint16_t* lm_head, const uint16_t* final_norm, float* lora,
+                                 float* lora_grad, const lsq_adamw* opt, float* loss_out,
+                                 float* logits_out, void* ws, size_t ws_bytes, void* stream,
+                                 int64_t timeout_ms) {
+  if (!h) return set_error(LSQ_ERR_INVALID, "stream_stack_step: null handle");
+  if (!tokens || !emb || !lm_head || !final_norm || !lora || !lora_grad || !loss_out)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_step: null pointer");
+  if (micro_batches <= 0 || batch <= 0 || seq < 2)
+    return set_error(LSQ_ERR_SHAPE, "stream_stack_step: need micro_batches, batch >= 1, seq >= 2");
+  if (opt && (!opt->m || !opt->v || opt->step < 1))
+    return set_error(LSQ_ERR_INVALID, "stream_stack_step: AdamW needs m, v and step >= 1");
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != h->device) return set_error(LSQ_ERR_INVALID, "stream_stack_step: wrong current device");
+  const lsq_cfg* cfg = &h->cfg;
+  const LayerShapes& s = h->shapes;
+  const int L = cfg->n_layers;
+  const int64_t T = (int64_t)batch * seq, D = s.D, V = cfg->vocab;
+  const size_t need = plan_stack_ws(cfg, s, T, nullptr, nullptr);
+  if (!ws || ws_bytes < need)
+    return set_error(LSQ_ERR_WORKSPACE, "stream_stack_step: workspace %zu < %zu", ws_bytes, need);
+  StackWs w;
+  plan_stack_ws(cfg, s, T, ws, &w);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int64_t layer_floats = h->lora_layout.floats_per_layer;
+  const float inv_count = 1.f / (float)((double)micro_batches * batch * (seq - 1));
+
+  // The buffers' contents are only trusted after a step that completed; a
+  // failed step leaves them unknown.
+  const int held0 = h->buf_layer[0], held1 = h->buf_layer[1];
+  h->buf_layer[0] = h->buf_layer[1] = -1;
+  std::vector<Visit> visits;
+  if (!h->resident) visits = plan_visits(L, micro_batches, held0, held1);
+  const size_t n_vis = (size_t)2 * L * micro_batches;
+  while (h->wait_ev.size() < 2 * n_vis) {
+    cudaEvent_t e;
+    LSQ_CUDA(cudaEventCreate(&e));
+    h->wait_ev.push_back(e);
+  }
+  const size_t bytes = h->layout.bytes;
+  int copies = 0;
+  auto enqueue_copy = [&](size_t j) -> int {
+    const Visit& x = visits[j];
+    if (!x.copy) return LSQ_OK;
+    LSQ_CUDA(cudaStreamWaitEvent(h->copy_stream, h->freed[x.buf], 0));
+    LSQ_CUDA(cudaMemcpyAsync(h->buf[x.buf], h->blobs[x.layer], bytes, cudaMemcpyHostToDevice,
+                             h->copy_stream));
+    LSQ_CUDA(cudaEventRecord(h->ready[x.buf], h->copy_stream));
+    ++copies;
+    return LSQ_OK;
+  };
+  // Returns the device pointer of visit j's layer, after fencing the compute stream.
+  auto acquire = [&](size_t j, const void** blob) -> int {
+    if (h->resident) return LSQ_OK;
+    const Visit& x = visits[j];
+    if (j + 1 < visits.size()) LSQ_TRY(enqueue_copy(j + 1));
+    LSQ_CUDA(cudaEventRecord(h->wait_ev[2 * j], cs));
+    LSQ_CUDA(cudaStreamWaitEvent(cs, h->ready[x.buf], 0));
+    LSQ_CUDA(cudaEventRecord(h->wait_ev[2 * j + 1], cs));
+    *blob = h->buf[x.buf];
+    return LSQ_OK;
+  };
+
+  LSQ_CUDA(cudaEventRecord(h->t_start, cs));
+  if (!h->resident && !visits.empty()) LSQ_TRY(enqueue_copy(0));
+  size_t j = 0;
+  for (int mb = 0; mb < micro_batches; ++mb) {
+    const int32_t* tok = tokens + (int64_t)mb * T;
+    LSQ_TRY(launch_embedding(tok, T, emb, D, V, w.xs, cs));
+    for (int i = 0; i < L; ++i, ++j) {
+      const void* blob = h->blobs[i];
+      if (!h->resident) LSQ_TRY(acquire(j, &blob));
+      LSQ_TRY(layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats, w.xs + (size_t)i * T * D,
+                             batch, seq, w.xs + (size_t)(i + 1) * T * D, w.layer_ws,
+                             w.layer_ws_bytes, cs));
+      if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
+    }
+    const uint16_t* xL = w.xs + (size_t)L * T * D;
+    LSQ_TRY(launch_rmsnorm_fwd(xL, final_norm, T, D, cfg->rms_eps, w.hf, w.rstd_f, cs));
+    LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
+    LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, inv_count, w.dlogits, w.row_loss, cs));
+    LSQ_TRY(launch_sum_rows(w.row_loss, T, inv_count, mb > 0 ? 1 : 0, w.loss_dev, cs));
+    LSQ_TRY(gemm_run(head_dx(lm_head, V, D, w.dlogits, T, w.dhf), w.gemm, w.gemm_bytes, cs));
+    LSQ_TRY(launch_rmsnorm_bwd(w.dhf, xL, final_norm, w.rstd_f, nullptr, T, D, w.dh[0], w.dhb[0], cs));
+    int cur = 0;
+    for (int i = L - 1; i >= 0; --i, ++j) {
+      const void* blob = h->blobs[i];
+      if (!h->resident) LSQ_TRY(acquire(j, &blob));
+      LSQ_TRY(layer_bwd_impl(cfg, blob, lora + (int64_t)i * layer_floats, w.xs + (size_t)i * T * D,
+                             w.dh[cur], w.dhb[cur], batch, seq, w.dh[1 - cur], w.dhb[1 - cur],
+                             lora_grad + (int64_t)i * layer_floats, mb > 0 ? 1 : 0, w.layer_ws,
+                             w.layer_ws_bytes, cs));
+      if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
+      cur = 1 - cur;
+    }
+  }
+  if (logits_out)
+    LSQ_CUDA(cudaMemcpyAsync(logits_out, w.logits, (size_t)T * V * sizeof(float),
+                             cudaMemcpyDeviceToDevice, cs));
+  if (opt)
+    LSQ_TRY(launch_adamw(lora, lora_grad, opt->m, opt->v, layer_floats * L, opt->lr, opt->beta1,
+                         opt->beta2, opt->eps, opt->weight_decay, opt->step, cs));
+  LSQ_CUDA(cudaMemcpyAsync(h->loss_host, w.loss_dev, sizeof(float), cudaMemcpyDeviceToHost, cs));
+  LSQ_CUDA(cudaEventRecord(h->t_end, cs));
+  LSQ_CUDA(cudaEventRecord(h->done, cs));
+  LSQ_TRY(wait_event_timeout(h->done, timeout_ms));
+  int flags = 0;
+  int* st = device_status_ptr();
+  if (st) {
+    LSQ_CUDA(cudaMemcpy(&flags, st, sizeof(int), cudaMemcpyDeviceToHost));
+    if (flags) return set_error(LSQ_ERR_DEVICE, "stream_stack_step: device status 0x%x", flags);
+  }
+  if (!h->resident) {
+    int held[2] = {held0, held1};
+    for (const Visit& x : visits)
+      if (x.copy) held[x.buf] = x.layer;
+    h->buf_layer[0] = held[0];
+    h->buf_layer[1] = held[1];
+  }
+  *loss_out = *h->loss_host;
+  h->stats.layer_copies = copies;
+  h->stats.h2d_bytes = (int64_t)copies * (int64_t)bytes;
+  cudaEventElapsedTime(&h->stats.step_ms, h->t_start, h->t_end);
+  float wait_ms = 0.f;
+  if (!h->resident) {
+    for (size_t k = 0; k < visits.size(); ++k) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, h->wait_ev[2 * k], h->wait_ev[2 * k + 1]) == cudaSuccess)
+        wait_ms += ms;
+    }
+  }
+  h->stats.copy_wait_ms = wait_ms;
+  return LSQ_OK;
+}

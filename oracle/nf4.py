@@ -74,9 +74,16 @@ def quantize(W, block=BLOCK):
     mids = midpoints()
     codes = np.full(blocks.shape, 7, dtype=np.uint8)
     nz = absmax > 0
-    with np.errstate(divide="ignore", invalid="ignore"):
-        v = (blocks[nz] / absmax[nz, None]).astype(np.float32)
-    codes[nz] = np.sum(v[..., None] > mids, axis=-1).astype(np.uint8)
+    # code = number of midpoints strictly below v: searchsorted(side="left")
+    # returns exactly that count.  Processed in chunks to bound memory.
+    step = 1 << 20
+    for b0 in range(0, blocks.shape[0], step):
+        sl = slice(b0, b0 + step)
+        z = nz[sl]
+        v = (blocks[sl][z] / absmax[sl][z, None]).astype(np.float32)
+        c = codes[sl]
+        c[z] = np.searchsorted(mids, v, side="left").astype(np.uint8)
+        codes[sl] = c
     flat = codes.reshape(-1)
     packed = ((flat[0::2] << 4) | flat[1::2]).astype(np.uint8)
     return packed, absmax

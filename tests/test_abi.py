@@ -1,0 +1,95 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/lsq.h declares, and its host-only entry points behave: the library's
+own NF4 codebook derivation equals the oracle's bit for bit, the layout queries
+give the documented sizes, and invalid arguments are rejected before any CUDA
+call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import nf4 as onf4
+from layer_streamed_qlora_nf4_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from layer_streamed_qlora_nf4_b200 import build, lib
+    if not os.path.exists(lib.LIB_PATH):
+        build.build()
+    lib.load()
+    return lib
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "lsq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s+([a-z_][a-z_0-9]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert len(names) >= 19
+    lib = L.load()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.EXPORTS)
+
+
+def test_library_codebook_equals_oracle_bitwise(L):
+    got = np.array(L.lsq_nf4_codebook(), np.float32)
+    assert np.array_equal(got.view(np.uint32), onf4.codebook().view(np.uint32))
+
+
+def test_layer_layout_matches_the_documented_sizes(L):
+    cfg = synth.LLAMA8B
+    lay = L.lsq_layer_layout_get(cfg)
+    P = 218103808                    # NF4 weights per 8B layer
+    expect = P // 2 + 4 * P // 64 + 2 * 4096 * 2
+    assert lay.bytes == expect == 122699776
+    shapes = synth.proj_shapes(cfg)
+    for p, name in enumerate(synth.PROJ):
+        assert (lay.rows[p], lay.cols[p]) == shapes[name]
+    # q|k|v and gate|up codes are contiguous (stacked GEMM operands)
+    assert lay.codes_off[1] == lay.codes_off[0] + 4096 * 4096 // 2
+    assert lay.codes_off[2] == lay.codes_off[1] + 1024 * 4096 // 2
+    assert lay.codes_off[5] == lay.codes_off[4] + 14336 * 4096 // 2
+    for o in list(lay.codes_off) + list(lay.absmax_off) + [lay.g1_off, lay.g2_off]:
+        assert o % 256 == 0
+    ll = L.lsq_lora_layout_get(cfg)
+    r = 16
+    n_lora = sum(r * (shapes[p][0] + shapes[p][1]) for p in synth.PROJ)
+    assert ll.floats_per_layer >= n_lora and ll.floats_per_layer - n_lora < 64 * 8
+    assert n_lora * 32 == 41943040   # 41.9 M LoRA parameters for the 32-layer stack
+
+
+def test_workspace_queries_are_host_only(L):
+    assert L.nf4_lora_linear_workspace_bytes(128, 1024, 1024, 16) > 0
+    assert L.decoder_layer_workspace_bytes(synth.LLAMA8B, 1, 512) > 0
+    assert L.stream_stack_workspace_bytes(synth.LLAMA8B, 1, 512) > 0
+    assert L.nf4_lora_linear_workspace_bytes(0, 1024, 1024, 16) == 0
+
+
+def test_invalid_arguments_are_rejected_without_a_gpu(L):
+    lib = L.load()
+    p = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    assert lib.nf4_quantize(p, 4, 96, 64, p, p, None) == L.LSQ_ERR_SHAPE
+    assert lib.nf4_quantize(p, 4, 128, 32, p, p, None) == L.LSQ_ERR_SHAPE
+    assert lib.nf4_quantize(None, 4, 128, 64, p, p, None) == L.LSQ_ERR_INVALID
+    assert lib.nf4_lora_linear_fwd(p, 8, 128, 64, p, p, 64, p, p, 8, 2.0, None, p, None, p, 1 << 20,
+                                   None) == L.LSQ_ERR_SHAPE       # r % 16 != 0
+    assert b"r must be" in lib.lsq_last_error()
+    bad = dict(synth.SMALL, head_dim=96)
+    with pytest.raises(L.LsqError) as e:
+        L.lsq_layer_layout_get(bad)
+    assert e.value.code == L.LSQ_ERR_SHAPE
+    h = ctypes.c_void_p()
+    c = L.cfg_struct(synth.SMALL)
+    arr = (ctypes.c_void_p * 2)(16, 32)
+    assert lib.stream_stack_create(ctypes.byref(c), arr, 2, p, p, 0, ctypes.byref(h)) == L.LSQ_ERR_SHAPE
+    assert lib.stream_stack_destroy(None) == L.LSQ_OK
