@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark: one streamed QLoRA SFT step through a 32-layer Llama-3.1-8B-shaped
+NF4 stack (batch 1, seq 512, LoRA r16 on all seven projections, cross-entropy,
+AdamW on the LoRA masters), the stack in page-locked host memory and fed to the
+GPU through two VRAM layer buffers.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  N > 1 runs data-parallel replicas (one rank per
+GPU, torch.distributed over NCCL): every rank streams its own stack copy on its
+own micro-batch, the LoRA gradients are averaged with an NCCL all-reduce, then
+every rank applies the same AdamW update ("scaling": "weak").
+
+--impl reference times the CPU oracle (the slow fp64 restatement of the method)
+on the host cores instead, on a bounded sample of the same workload.
+"""
+import argparse
+import csv
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "streamed QLoRA train tokens/sec (8B shapes, seq 512) and % of step roofline"
+WORKLOAD = ("Llama-3.1-8B-shaped 32-layer NF4 stack (block 64, fp32 absmax) streamed from "
+            "pinned host memory through two VRAM layer buffers; bf16 untied embedding and "
+            "lm_head (vocab 128256) resident; batch 1 x seq 512 per GPU; one SFT step "
+            "(cross-entropy + AdamW on LoRA r16 alpha32, all 7 projections)")
+BATCH, SEQ = 1, 512
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (for quick runs)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d["bf16_tflops_sustained"], source="measured")
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(seed=1):
+    """Bounded sample of one step, run by the CPU oracle: one 8B-shaped layer's
+    forward and its recomputing backward (T = 512), and the lm_head forward and
+    input-gradient products on a 8192-row slice of the vocabulary.  Returns
+    (seconds for a whole step, description, threads)."""
+    import numpy as np
+    from layer_streamed_qlora_nf4_b200 import synth
+    from oracle import model as om
+    from oracle import nf4 as onf4
+    cfg = synth.LLAMA8B
+    lw = synth.layer_weights(seed, cfg)
+    W = {}
+    for p in synth.PROJ:
+        N, K = lw["W"][p].shape
+        W[p] = onf4.dequantize(*onf4.quantize(lw["W"][p]), N, K)
+    params = dict(W=W, A=lw["A"], B=lw["B"], g1=synth.bf16_bits_to_f32(lw["g1"]),
+                  g2=synth.bf16_bits_to_f32(lw["g2"]))
+    T = BATCH * SEQ
+    x = synth.bf16_bits_to_f32(synth.activations(seed + 1, T, cfg["hidden"]))
+    dout = synth.normal_f32(synth.rng(seed + 2), (T, cfg["hidden"]), 1.0)
+    t0 = time.perf_counter()
+    om.decoder_layer_fwd(params, x, cfg, SEQ)
+    t1 = time.perf_counter()
+    om.decoder_layer_bwd(params, x, dout, cfg, SEQ)
+    t2 = time.perf_counter()
+    vs = 8192
+    g = synth.rng(seed + 3)
+    head = synth.bf16_bits_to_f32(synth.normal_bf16(g, (vs, cfg["hidden"]), 0.02)).astype(np.float64)
+    hf = x.astype(np.float64)
+    t3 = time.perf_counter()
+    logits = hf @ head.T
+    _ = logits @ head
+    t4 = time.perf_counter()
+    L = cfg["n_layers"]
+    step_s = L * ((t1 - t0) + (t2 - t1)) + (t4 - t3) * cfg["vocab"] / vs
+    desc = ("fp64 oracle: one 8B-shaped layer forward (%.2fs) + recomputing backward (%.2fs) at "
+            "T=512, x%d layers; lm_head fwd+dX on %d of %d vocab rows (%.2fs), scaled"
+            % (t1 - t0, t2 - t1, L, vs, cfg["vocab"], t4 - t3))
+    return step_s, desc
+
+
+def cpu_threads():
+    return os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        s, desc = oracle_sample(seed=1)
+        if i >= args.warmup:
+            times.append(s)
+    step_s = statistics.median(times)
+    tok = BATCH * SEQ / step_s
+    line = dict(impl="reference", metric=METRIC, value=tok, unit="tokens/s", n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic",
+                config=dict(workload=WORKLOAD, global_batch=BATCH, seq_len=SEQ,
+                            parallelism="cpu oracle, rank 0 only"),
+                cpu_baseline=dict(value=tok, unit="tokens/s", cores=cpu_threads(), kind="oracle",
+                                  sample=desc),
+                e2e=dict(value=tok, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r for r in csv.reader(self.f) if len(r) >= 8]
+        os.unlink(self.f.name)
+        mine = [r for r in rows if self.uuid and r[0].strip() in self.uuid] or rows
+        if not mine:
+            return None
+        sm = [float(r[1]) for r in mine if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in mine if r[2].strip().replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in mine for i in range(4) if "Active" == r[4 + i].strip()})
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(mx) if mx else None, reasons=reasons, samples=len(mine))
+
+
+# ---------------------------------------------------------------- our arm
+def build_stack(L, cfg, rank):
+    import torch
+    from layer_streamed_qlora_nf4_b200 import pack, synth
+    lay = L.lsq_layer_layout_get(cfg)
+    g = torch.Generator(device="cuda").manual_seed(2)      # same frozen stack on every rank
+    shapes = synth.proj_shapes(cfg)
+    ones = torch.ones(cfg["hidden"], dtype=torch.bfloat16, device="cuda")
+    host_blobs = []
+    tmp = torch.empty(lay.bytes, dtype=torch.uint8, device="cuda")
+    for _ in range(cfg["n_layers"]):
+        W = {p: torch.randn(shapes[p], generator=g, device="cuda") * 0.02 for p in synth.PROJ}
+        pack.pack_layer(cfg, W, ones, ones, tmp)
+        hb = torch.empty(lay.bytes, dtype=torch.uint8).pin_memory()
+        hb.copy_(tmp)
+        host_blobs.append(hb)
+        del W
+    r = cfg["lora_r"]
+    A = {p: torch.randn(r, shapes[p][1], generator=g, device="cuda") / r for p in synth.PROJ}
+    B = {p: torch.randn(shapes[p][0], r, generator=g, device="cuda") * 0.01 for p in synth.PROJ}
+    lora = torch.cat([pack.lora_block(cfg, A, B) for _ in range(cfg["n_layers"])])
+    emb = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
+    head = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
+    gt = torch.Generator(device="cuda").manual_seed(1000 + rank)
+    tokens = torch.randint(0, cfg["vocab"], (BATCH, SEQ), generator=gt, device="cuda",
+                           dtype=torch.int32)
+    bufs = [torch.empty(lay.bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    return dict(lay=lay, host_blobs=host_blobs, lora=lora, emb=emb, head=head, gf=ones,
+                tokens=tokens, bufs=bufs)
+
+
+def h2d_bandwidth(nbytes, reps=10):
+    """Best of `reps` pinned host->device copies of one layer on a non-default stream (GB/s)."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    best = 0.0
+    with torch.cuda.stream(s):
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            dst.copy_(src, non_blocking=True)
+            e1.record(s)
+            e1.synchronize()
+            best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    return best
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    from layer_streamed_qlora_nf4_b200 import lib as L
+    from layer_streamed_qlora_nf4_b200 import synth
+    L.load()
+    cfg = synth.LLAMA8B
+    st = build_stack(L, cfg, rank)
+    lay = st["lay"]
+    handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
+    ws = torch.empty(L.stream_stack_workspace_bytes(cfg, BATCH, SEQ), dtype=torch.uint8,
+                     device="cuda")
+    lora, grad = st["lora"], torch.zeros_like(st["lora"])
+    m, v = torch.zeros_like(lora), torch.zeros_like(lora)
+    opt = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, m=m, v=v)
+    stream = torch.cuda.current_stream()
+
+    def step(tokens):
+        if world == 1:
+            loss = L.stream_stack_step(handle, tokens, 1, BATCH, SEQ, st["emb"], st["head"],
+                                       st["gf"], lora, grad, opt, ws)
+        else:
+            loss = L.stream_stack_step(handle, tokens, 1, BATCH, SEQ, st["emb"], st["head"],
+                                       st["gf"], lora, grad, None, ws)
+            dist.all_reduce(grad, op=dist.ReduceOp.AVG)
+            L.lora_adamw_step(lora, grad, opt)
+        opt["step"] += 1
+        return loss
+
+    for _ in range(args.warmup):
+        loss = step(st["tokens"])
+    torch.cuda.synchronize()
+    h2d_gbs = h2d_bandwidth(lay.bytes)
+
+    uuid = str(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "uuid", ""))
+    sampler = ClockSampler(uuid)
+    # ------------------------------------------------------------ timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    L.lsq_profile_enable(True)
+    n0 = L.lsq_launch_counter()
+    copies, wait_ms = 0, 0.0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        loss = step(st["tokens"])
+        s = L.stream_stack_last_stats(handle)
+        copies += s["layer_copies"]
+        wait_ms += s["copy_wait_ms"]
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = L.lsq_launch_counter() - n0
+    L.lsq_profile_enable(False)
+    clocks = sampler.stop()
+    prof = L.lsq_profile_read()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * BATCH * SEQ / (ms * 1e-3)
+
+    # ------------------------------------------------------------ end to end (host buffers)
+    tok_host = st["tokens"].cpu().pin_memory()
+    tok_dev = torch.empty_like(st["tokens"])
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        tok_dev.copy_(tok_host, non_blocking=True)
+        loss = step(tok_dev)           # returns the loss on the host
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = dict(value=world * BATCH * SEQ / (e2e_ms * 1e-3), unit="tokens/s",
+               h2d_bytes_per_step=tok_host.numel() * 4, d2h_bytes_per_step=4,
+               layer_stream_h2d_bytes_per_step=copies // args.steps * lay.bytes)
+
+    pk = peaks()
+    # dominant kernel: the class with the most device time in the timed region
+    dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+    per_launch_ms = dom["total_ms"] / dom["launches"]
+    tc = dom_name.startswith("gemm") or dom_name.startswith("attention")
+    achieved = (dom["flops"] / dom["launches"]) / (per_launch_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    roofline = dict(bound="tensor" if tc else "hbm", kernel=dom_name, achieved=achieved,
+                    peak=peak, unit="TFLOP/s", frac=achieved / peak, traffic=None,
+                    peak_source="%s (bf16 sustained, kernel timed inside a long step)" % pk["source"],
+                    launches_per_step=dom["launches"] / args.steps,
+                    per_launch_ms=per_launch_ms,
+                    step_share=dom["total_ms"] / args.steps / ms)
+    # step roofline: slowest of tensor FLOPs at peak, algorithmic DRAM bytes at the
+    # measured copy bandwidth, and the streamed layer bytes at the measured H2D bandwidth
+    flops_step = sum(e["flops"] for e in prof.values()) / args.steps
+    bytes_step = sum(e["bytes"] for e in prof.values()) / args.steps
+    cps = copies / args.steps
+    t_tc = flops_step / (pk["bf16_tflops_sustained"] * 1e12) * 1e3
+    t_hbm = (bytes_step + cps * lay.bytes) / (pk["hbm_gbs"] * 1e9) * 1e3
+    t_h2d = cps * lay.bytes / (h2d_gbs * 1e9) * 1e3
+    t_roof = max(t_tc, t_hbm, t_h2d)
+    step_roof = dict(t_tensor_ms=t_tc, t_hbm_ms=t_hbm, t_h2d_ms=t_h2d,
+                     bound=["tensor", "hbm", "h2d"][[t_tc, t_hbm, t_h2d].index(t_roof)],
+                     frac=t_roof / ms, h2d_gbs_measured=h2d_gbs, layer_copies_per_step=cps,
+                     layer_bytes=lay.bytes, copy_wait_ms_per_step=wait_ms / args.steps,
+                     tflop_per_step=flops_step / 1e12,
+                     kernels={k: dict(launches_per_step=e["launches"] / args.steps,
+                                      ms_per_step=e["total_ms"] / args.steps,
+                                      tflops=(e["flops"] / e["total_ms"] * 1e-9)
+                                      if e["total_ms"] > 0 else None)
+                              for k, e in prof.items()})
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s, desc = oracle_sample(seed=1)
+        cpu = dict(value=BATCH * SEQ / s, unit="tokens/s", cores=cpu_threads(), kind="oracle",
+                   sample=desc)
+    handle.close()
+    if rank == 0:
+        line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak",
+                    vs_baseline=None, dtype="bf16", data="synthetic (seeded random weights and "
+                    "uniform token ids at the 8B shapes)",
+                    config=dict(workload=WORKLOAD, global_batch=world * BATCH, seq_len=SEQ,
+                                parallelism="dp%d" % world,
+                                l2="inputs larger than L2: %.2f GB of layer bytes stream per step"
+                                % (cps * lay.bytes / 1e9)),
+                    loss=loss, roofline=roofline, step_roofline=step_roof, cpu_baseline=cpu,
+                    e2e=e2e, gpu_launches=int(launches), clocks=clocks)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

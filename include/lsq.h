@@ -250,6 +250,38 @@ typedef struct lsq_step_stats {
 } lsq_step_stats;
 int stream_stack_last_stats(const lsq_stack* stack, lsq_step_stats* out);
 
+/* ------------------------------------------------------------ optimiser */
+
+/* lora_adamw_step - one AdamW update of n LoRA parameters (fp32, any layout
+ * shared by lora, grad, opt->m, opt->v): m = b1 m + (1-b1) g, v = b2 v + (1-b2) g^2,
+ * p = p (1 - lr wd) - lr (m / (1-b1^step)) / (sqrt(v / (1-b2^step)) + eps).
+ * The same update stream_stack_step applies; exported so that data-parallel
+ * callers can reduce gradients across ranks between the step and the update.
+ * Asynchronous. */
+int lora_adamw_step(float* lora, const float* grad, const lsq_adamw* opt, int64_t n, void* stream);
+
+/* ------------------------------------------------------------ measurement */
+
+/* Number of kernel launches the library has issued in this process. */
+int64_t lsq_launch_counter(void);
+
+/* Per-launch device timing of the library's heavy kernels.  While enabled,
+ * every tensor-core GEMM and attention launch is bracketed by CUDA events
+ * recorded on the stream it is launched on, together with its algorithmic
+ * work (FLOPs, and the minimum DRAM bytes it must move).  Enabling costs two
+ * event records per such launch. */
+typedef struct lsq_prof_entry {
+  char name[32];       /* kernel class, e.g. "gemm_nf4_fwd" */
+  int64_t launches;
+  double total_ms;     /* summed event time of those launches */
+  double flops;        /* summed algorithmic FLOPs */
+  double bytes;        /* summed algorithmic DRAM bytes */
+} lsq_prof_entry;
+/* enable != 0 starts recording (and clears earlier records); 0 stops. */
+int lsq_profile_enable(int enable);
+/* Synchronises the recorded events and fills up to max entries (one per class). */
+int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -475,7 +475,7 @@ int attn_fwd_t(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv, uint16_t
   dim3 grid((seq + kTile - 1) / kTile, H, batch);
   const float sl2 = 1.4426950408889634f / sqrtf((float)D);
   attn_fwd_kernel<D><<<grid, 128, smem, st>>>(qkv, T, seq, H, Hkv, o, lse, sl2);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -498,14 +498,14 @@ int attn_bwd_t(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout, con
   const float sl2 = 1.4426950408889634f * scale;
   const int64_t nw = T * H;
   attn_delta_kernel<D><<<(unsigned)((nw * 32 + 255) / 256), 256, 0, st>>>(o, dout, T, H, delta);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   dim3 gkv((seq + kTile - 1) / kTile, Hkv, batch);
   attn_bwd_dkdv_kernel<D><<<gkv, 128, s_kv, st>>>(qkv, dout, lse, delta, T, seq, H, Hkv, sl2, scale,
                                                   dk, dv);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   dim3 gq((seq + kTile - 1) / kTile, H, batch);
   attn_bwd_dq_kernel<D><<<gq, 128, s_q, st>>>(qkv, dout, lse, delta, T, seq, H, Hkv, sl2, scale, dq);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -515,9 +515,15 @@ int launch_attention_fwd(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv
                          uint16_t* o, float* lse, cudaStream_t st) {
   if (seq <= 0 || T % seq != 0 || H % Hkv != 0)
     return set_error(LSQ_ERR_SHAPE, "attention: bad batch/seq/head shape");
-  if (d == 128) return attn_fwd_t<128>(qkv, T, seq, H, Hkv, o, lse, st);
-  if (d == 64) return attn_fwd_t<64>(qkv, T, seq, H, Hkv, o, lse, st);
-  return set_error(LSQ_ERR_SHAPE, "attention: head_dim must be 64 or 128");
+  if (d != 128 && d != 64) return set_error(LSQ_ERR_SHAPE, "attention: head_dim must be 64 or 128");
+  const int prof = prof_begin(st);
+  LSQ_TRY(d == 128 ? attn_fwd_t<128>(qkv, T, seq, H, Hkv, o, lse, st)
+                   : attn_fwd_t<64>(qkv, T, seq, H, Hkv, o, lse, st));
+  // causal: 2 GEMMs of d per (query, key<=query) pair and head
+  const double pairs = (double)(T / seq) * (double)seq * (seq + 1) / 2.0;
+  prof_end(prof, st, "attention_fwd", 4.0 * H * d * pairs,
+           2.0 * T * (double)(H + 2 * Hkv) * d + 2.0 * T * H * d);
+  return LSQ_OK;
 }
 
 int launch_attention_bwd(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
@@ -525,9 +531,15 @@ int launch_attention_bwd(const uint16_t* qkv, const uint16_t* o, const uint16_t*
                          float* dq, float* dk, float* dv, cudaStream_t st) {
   if (seq <= 0 || T % seq != 0 || H % Hkv != 0)
     return set_error(LSQ_ERR_SHAPE, "attention: bad batch/seq/head shape");
-  if (d == 128) return attn_bwd_t<128>(qkv, o, dout, lse, T, seq, H, Hkv, delta, dq, dk, dv, st);
-  if (d == 64) return attn_bwd_t<64>(qkv, o, dout, lse, T, seq, H, Hkv, delta, dq, dk, dv, st);
-  return set_error(LSQ_ERR_SHAPE, "attention: head_dim must be 64 or 128");
+  if (d != 128 && d != 64) return set_error(LSQ_ERR_SHAPE, "attention: head_dim must be 64 or 128");
+  const int prof = prof_begin(st);
+  LSQ_TRY(d == 128 ? attn_bwd_t<128>(qkv, o, dout, lse, T, seq, H, Hkv, delta, dq, dk, dv, st)
+                   : attn_bwd_t<64>(qkv, o, dout, lse, T, seq, H, Hkv, delta, dq, dk, dv, st));
+  // five causal GEMMs (S, dP, dV, dK, dQ) = 2.5x the forward's two
+  const double pairs = (double)(T / seq) * (double)seq * (seq + 1) / 2.0;
+  prof_end(prof, st, "attention_bwd", 10.0 * H * d * pairs,
+           2.0 * T * (double)(H + 2 * Hkv) * d + 6.0 * T * H * d + 4.0 * T * (H + 2 * Hkv) * d);
+  return LSQ_OK;
 }
 
 }  // namespace lsq

@@ -384,14 +384,14 @@ int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M,
   if (M % 4 != 0) return set_error(LSQ_ERR_SHAPE, "splitk_reduce: M %% 4 != 0");
   splitk_reduce_kernel<<<grid_for(T * M / 4, 256), 256, 0, st>>>(partial, splits, T, M, out,
                                                                  out_f32, ldo, residual, ldr);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
                        uint16_t* y, float* rstd, cudaStream_t st) {
   rmsnorm_fwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(x, g, T, D, eps, y, rstd);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -400,7 +400,7 @@ int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, co
                        cudaStream_t st) {
   rmsnorm_bwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(dy, x, g, rstd, dres, T, D,
                                                                       dx, dx_bf16);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -409,7 +409,7 @@ int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, float 
   const int64_t n = T * (H + Hkv) * (d / 2);
   rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(qkv, T, seq, H, Hkv, d, log((double)theta),
                                                 inverse);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -418,27 +418,27 @@ int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t 
   const int64_t n = T * (H + 2 * Hkv) * (d / 2);
   rope_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dq, dk, dv, T, seq, H, Hkv, d,
                                                      log((double)theta), dqkv);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st) {
   swiglu_fwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(gu, T, F, m);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
                       cudaStream_t st) {
   swiglu_bwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(dm, gu, T, F, dgu);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D, int64_t V,
                      uint16_t* out, cudaStream_t st) {
   embedding_kernel<<<grid_for(T * D / 8, 256), 256, 0, st>>>(tokens, T, emb, D, V, out);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -446,14 +446,14 @@ int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, 
                          float inv_count, uint16_t* dlogits, float* row_loss, cudaStream_t st) {
   cross_entropy_kernel<<<(unsigned)T, 512, 0, st>>>(logits, tokens, T, seq, V, inv_count, dlogits,
                                                     row_loss);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_sum_rows(const float* row_loss, int64_t T, float scale, int accumulate, float* out,
                     cudaStream_t st) {
   sum_rows_kernel<<<1, 1024, 0, st>>>(row_loss, T, scale, accumulate, out);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -462,19 +462,19 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
   const float bc1 = (float)(1.0 - pow((double)b1, (double)step));
   const float bc2 = (float)(1.0 - pow((double)b2, (double)step));
   adamw_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st) {
   f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, y);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st) {
   scale_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, s);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 

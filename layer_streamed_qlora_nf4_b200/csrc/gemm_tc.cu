@@ -587,7 +587,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   if (!p.dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
   dim3 grid(pl.m_tiles, pl.t_tiles, pl.splits);
   tc_gemm_kernel<WMODE><<<grid, kThreads, pl.smem_bytes, st>>>(tm_act, tm_w, p);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -642,6 +642,7 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
                        pl.partial_bytes);
     partial = static_cast<float*>(ws);
   }
+  const int prof = prof_begin(st);
   switch (d.wmode) {
     case W_NF4_N: LSQ_TRY(launch_mode<W_NF4_N>(d, pl, partial, st)); break;
     case W_NF4_T: LSQ_TRY(launch_mode<W_NF4_T>(d, pl, partial, st)); break;
@@ -652,6 +653,19 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (pl.splits > 1)
     LSQ_TRY(launch_splitk_reduce(partial, pl.splits, d.T, d.M, d.out, d.out_f32, d.ldo,
                                  d.residual, d.ldr, st));
+  if (prof >= 0) {
+    // algorithmic work: the contraction plus the LoRA slab; minimum DRAM traffic:
+    // the weight once, the activation once, the output (and residual) once
+    const double M = (double)d.M, T = (double)d.T, K = (double)d.Kc;
+    const double flops = 2.0 * M * T * (K + d.slab_w);
+    const bool nf4 = d.wmode == W_NF4_N || d.wmode == W_NF4_T;
+    const double wbytes = nf4 ? M * K * (0.5 + 4.0 / 64.0) : 2.0 * M * K;
+    const double bytes = wbytes + 2.0 * T * K + T * M * (d.out_f32 ? 4.0 : 2.0) +
+                         (d.residual ? 2.0 * T * M : 0.0);
+    static const char* names[4] = {"gemm_nf4_fwd", "gemm_nf4_dx", "gemm_bf16_head",
+                                   "gemm_bf16_head_dx"};
+    prof_end(prof, st, names[d.wmode], flops, bytes);
+  }
   return LSQ_OK;
 }
 

@@ -19,6 +19,12 @@ int cuda_status(cudaError_t e, const char* what); // LSQ_OK or LSQ_ERR_CUDA with
   } while (0)
 #define LSQ_CUDA(expr) LSQ_TRY(::lsq::cuda_status((expr), #expr))
 
+// Counts a kernel launch (wraps the cudaGetLastError check after every launch).
+cudaError_t launched(cudaError_t e);
+// Per-launch event timing of heavy kernels (no-ops unless lsq_profile_enable).
+int prof_begin(cudaStream_t st);
+void prof_end(int token, cudaStream_t st, const char* name, double flops, double bytes);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Device status word bits (latched by kernels, read by lsq_device_status).

@@ -158,11 +158,11 @@ int run_skinny(const uint16_t* X, int64_t ldx, const float* Y, int64_t ysj, int6
     attr = true;
   }
   skinny_partial_kernel<<<grid, 256, smem, st>>>(X, ldx, Y, ysj, ysk, T, K, R, part, ldo, col0);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   const int64_t n = T * R;
   partial_sum_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
       part, nkc, T, ldo, col0, R, out, ldo);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -202,7 +202,7 @@ int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, 
                        int accumulate, float* dA, cudaStream_t st) {
   dim3 grid((unsigned)((K + 127) / 128), (unsigned)((R + 7) / 8));
   lora_grad_a_kernel<<<grid, 128, 0, st>>>(v, x, T, K, R, s, accumulate, dA);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
@@ -224,7 +224,7 @@ int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N,
                                                  pe[3], s, accumulate, dB);
   else
     return set_error(LSQ_ERR_SHAPE, "lora_grad_b: r > 64 unsupported");
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 

@@ -164,7 +164,7 @@ extern "C" int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block,
   const int64_t cap = (int64_t)gemm_num_sms() * 32;
   if (grid > cap) grid = cap;
   nf4_quantize_kernel<<<(unsigned)grid, threads, 0, st>>>(W, n_blocks, codes, absmax, qp, err);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   int h_after = 0;
   LSQ_CUDA(cudaMemcpyAsync(&h_after, err, sizeof(int), cudaMemcpyDeviceToHost, st));
   LSQ_CUDA(cudaStreamSynchronize(st));
@@ -189,6 +189,6 @@ extern "C" int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t
   const int64_t cap = (int64_t)gemm_num_sms() * 16;
   if (grid > cap) grid = cap;
   nf4_dequantize_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, absmax, n_bytes, W_out, lp);
-  LSQ_CUDA(cudaGetLastError());
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }

@@ -23,6 +23,7 @@ EXPORTS = (
     "lsq_lora_layout_get", "decoder_layer_workspace_bytes", "decoder_layer_fwd",
     "decoder_layer_bwd", "stream_stack_create", "stream_stack_destroy",
     "stream_stack_workspace_bytes", "stream_stack_step", "stream_stack_last_stats",
+    "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
 )
 
 
@@ -57,6 +58,12 @@ class lsq_adamw(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("step", ctypes.c_int32), ("m", ctypes.c_void_p), ("v", ctypes.c_void_p)]
+
+
+class lsq_prof_entry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
 
 
 class lsq_step_stats(ctypes.Structure):
@@ -95,6 +102,11 @@ _PROTOS = {
                                          ctypes.POINTER(lsq_adamw), ctypes.POINTER(ctypes.c_float),
                                          _P, _P, _SZ, _P, _I64]),
     "stream_stack_last_stats": (ctypes.c_int, [_P, ctypes.POINTER(lsq_step_stats)]),
+    "lora_adamw_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(lsq_adamw), _I64, _P]),
+    "lsq_launch_counter": (ctypes.c_int64, []),
+    "lsq_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "lsq_profile_read": (ctypes.c_int, [ctypes.POINTER(lsq_prof_entry), _I32,
+                                        ctypes.POINTER(ctypes.c_int32)]),
 }
 
 _lib = None
@@ -264,11 +276,7 @@ def stream_stack_step(stack, tokens, micro_batches, batch, seq, emb, lm_head, fi
     """Returns the mean loss (host float).  opt: dict(lr, beta1, beta2, eps, weight_decay,
     step, m, v) or None."""
     loss = ctypes.c_float(0.0)
-    o = None
-    if opt is not None:
-        o = lsq_adamw(lr=opt["lr"], beta1=opt["beta1"], beta2=opt["beta2"], eps=opt["eps"],
-                      weight_decay=opt["weight_decay"], step=opt["step"],
-                      m=opt["m"].data_ptr(), v=opt["v"].data_ptr())
+    o = _adamw_struct(opt) if opt is not None else None
     _check(load().stream_stack_step(stack.handle, _ptr(tokens), micro_batches, batch, seq,
                                     _ptr(emb), _ptr(lm_head), _ptr(final_norm), _ptr(lora),
                                     _ptr(lora_grad), ctypes.byref(o) if o is not None else None,
@@ -282,3 +290,33 @@ def stream_stack_last_stats(stack):
     _check(load().stream_stack_last_stats(stack.handle, ctypes.byref(s)))
     return dict(layer_copies=s.layer_copies, h2d_bytes=s.h2d_bytes, step_ms=s.step_ms,
                 copy_wait_ms=s.copy_wait_ms)
+
+
+def _adamw_struct(opt):
+    return lsq_adamw(lr=opt["lr"], beta1=opt["beta1"], beta2=opt["beta2"], eps=opt["eps"],
+                     weight_decay=opt["weight_decay"], step=opt["step"],
+                     m=opt["m"].data_ptr(), v=opt["v"].data_ptr())
+
+
+def lora_adamw_step(lora, grad, opt, stream=None):
+    o = _adamw_struct(opt)
+    _check(load().lora_adamw_step(_ptr(lora), _ptr(grad), ctypes.byref(o), lora.numel(),
+                                  _stream(stream)))
+
+
+def lsq_launch_counter():
+    return load().lsq_launch_counter()
+
+
+def lsq_profile_enable(enable=True):
+    _check(load().lsq_profile_enable(1 if enable else 0))
+
+
+def lsq_profile_read():
+    """-> dict kernel class -> dict(launches, total_ms, flops, bytes)."""
+    arr = (lsq_prof_entry * 64)()
+    n = ctypes.c_int32(0)
+    _check(load().lsq_profile_read(arr, 64, ctypes.byref(n)))
+    return {arr[i].name.decode(): dict(launches=arr[i].launches, total_ms=arr[i].total_ms,
+                                       flops=arr[i].flops, bytes=arr[i].bytes)
+            for i in range(n.value)}
