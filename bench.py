@@ -45,6 +45,10 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (for quick runs)")
+    ap.add_argument("--case", choices=("step", "layer", "gemm"), default="step",
+                    help="step: the streamed 32-layer SFT step (default); layer: one resident "
+                         "8B-shaped layer forward + recomputing backward; gemm: one fused NF4 "
+                         "GEMM at the q|k|v shape (a small case for profiling)")
     return ap.parse_args()
 
 
@@ -195,7 +199,7 @@ def build_stack(L, cfg, rank):
     emb = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
     head = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
     gt = torch.Generator(device="cuda").manual_seed(1000 + rank)
-    tokens = torch.randint(0, cfg["vocab"], (BATCH, SEQ), generator=gt, device="cuda",
+    tokens = torch.randint(0, cfg["vocab"], (8, BATCH, SEQ), generator=gt, device="cuda",
                            dtype=torch.int32)
     bufs = [torch.empty(lay.bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
     return dict(lay=lay, host_blobs=host_blobs, lora=lora, emb=emb, head=head, gf=ones,
@@ -257,8 +261,9 @@ def run_ours(args):
         opt["step"] += 1
         return loss
 
-    for _ in range(args.warmup):
-        loss = step(st["tokens"])
+    pool = st["tokens"]           # a few distinct batches, cycled
+    for i in range(args.warmup):
+        loss = step(pool[i % len(pool)])
     torch.cuda.synchronize()
     h2d_gbs = h2d_bandwidth(lay.bytes)
 
@@ -274,8 +279,8 @@ def run_ours(args):
     copies, wait_ms = 0, 0.0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        loss = step(st["tokens"])
+    for i in range(args.steps):
+        loss = step(pool[i % len(pool)])
         s = L.stream_stack_last_stats(handle)
         copies += s["layer_copies"]
         wait_ms += s["copy_wait_ms"]
@@ -295,15 +300,15 @@ def run_ours(args):
     value = world * BATCH * SEQ / (ms * 1e-3)
 
     # ------------------------------------------------------------ end to end (host buffers)
-    tok_host = st["tokens"].cpu().pin_memory()
-    tok_dev = torch.empty_like(st["tokens"])
+    tok_host = pool.cpu().pin_memory()
+    tok_dev = torch.empty_like(pool[0])
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    for _ in range(args.steps):
-        tok_dev.copy_(tok_host, non_blocking=True)
+    for i in range(args.steps):
+        tok_dev.copy_(tok_host[i % len(tok_host)], non_blocking=True)
         loss = step(tok_dev)           # returns the loss on the host
     f1.record(stream)
     torch.cuda.synchronize()
@@ -313,7 +318,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e = dict(value=world * BATCH * SEQ / (e2e_ms * 1e-3), unit="tokens/s",
-               h2d_bytes_per_step=tok_host.numel() * 4, d2h_bytes_per_step=4,
+               h2d_bytes_per_step=tok_dev.numel() * 4, d2h_bytes_per_step=4,
                layer_stream_h2d_bytes_per_step=copies // args.steps * lay.bytes)
 
     pk = peaks()
@@ -372,10 +377,132 @@ def run_ours(args):
     return 0
 
 
+def run_layer(args):
+    """One resident 8B-shaped decoder layer: forward + recomputing backward (batch 1, seq 512)."""
+    import torch
+    from layer_streamed_qlora_nf4_b200 import lib as L
+    from layer_streamed_qlora_nf4_b200 import pack, synth
+    L.load()
+    cfg = synth.LLAMA8B
+    lay = L.lsq_layer_layout_get(cfg)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    shapes = synth.proj_shapes(cfg)
+    ones = torch.ones(cfg["hidden"], dtype=torch.bfloat16, device="cuda")
+    blob = torch.empty(lay.bytes, dtype=torch.uint8, device="cuda")
+    W = {p: torch.randn(shapes[p], generator=g, device="cuda") * 0.02 for p in synth.PROJ}
+    pack.pack_layer(cfg, W, ones, ones, blob)
+    del W
+    r = cfg["lora_r"]
+    A = {p: torch.randn(r, shapes[p][1], generator=g, device="cuda") / r for p in synth.PROJ}
+    B = {p: torch.randn(shapes[p][0], r, generator=g, device="cuda") * 0.01 for p in synth.PROJ}
+    lora = pack.lora_block(cfg, A, B)
+    grad = torch.zeros_like(lora)
+    T = BATCH * SEQ
+    x = (torch.randn(T, cfg["hidden"], generator=g, device="cuda")).bfloat16()
+    y = torch.empty_like(x)
+    dy = torch.randn(T, cfg["hidden"], generator=g, device="cuda")
+    dx = torch.empty_like(dy)
+    ws = torch.empty(L.decoder_layer_workspace_bytes(cfg, BATCH, SEQ), dtype=torch.uint8,
+                     device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")   # > L2, between iterations
+
+    def it():
+        L.decoder_layer_fwd(cfg, blob, lora, x, BATCH, SEQ, y, ws)
+        L.decoder_layer_bwd(cfg, blob, lora, x, dy, BATCH, SEQ, dx, grad, ws)
+
+    for _ in range(args.warmup):
+        it()
+    torch.cuda.synchronize()
+    L.lsq_profile_enable(True)
+    n0 = L.lsq_launch_counter()
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        it()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    launches = L.lsq_launch_counter() - n0
+    L.lsq_profile_enable(False)
+    prof = L.lsq_profile_read()
+    ms = tot / args.steps
+    pk = peaks()
+    flops = sum(e["flops"] for e in prof.values()) / args.steps
+    gemm = {k: e for k, e in prof.items() if k.startswith("gemm")}
+    gms = sum(e["total_ms"] for e in gemm.values()) / args.steps
+    gfl = sum(e["flops"] for e in gemm.values()) / args.steps
+    line = dict(metric="decoder layer fwd + recomputing bwd tokens/s (one 8B-shaped NF4 layer, "
+                "resident, seq 512)", value=T / (ms * 1e-3), unit="tokens/s", n_gpus=1,
+                steps=args.steps, warmup=args.warmup, ms_per_step=ms, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+                config=dict(workload="one Llama-3.1-8B-shaped NF4 decoder layer, batch 1, seq "
+                            "512, forward + backward with recompute, resident", global_batch=1,
+                            seq_len=SEQ, parallelism="dp1", l2="L2 flushed (256 MB write) "
+                            "between iterations"),
+                roofline=dict(bound="tensor", kernel="all tensor-core GEMMs of the layer",
+                              achieved=gfl / (gms * 1e-3) / 1e12, peak=pk["bf16_tflops"],
+                              unit="TFLOP/s", frac=gfl / (gms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                              traffic=None, peak_source="%s (bf16 burst)" % pk["source"]),
+                layer_roofline=dict(t_tensor_ms=flops / (pk["bf16_tflops"] * 1e12) * 1e3,
+                                    frac=flops / (pk["bf16_tflops"] * 1e12) * 1e3 / ms),
+                kernels={k: dict(launches=e["launches"] / args.steps,
+                                 ms=e["total_ms"] / args.steps,
+                                 tflops=e["flops"] / e["total_ms"] * 1e-9)
+                         for k, e in prof.items()},
+                gpu_launches=int(launches))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gemm(args):
+    """One fused NF4 + LoRA GEMM at the stacked q|k|v shape (M 6144, K 4096, T 512)."""
+    import torch
+    from layer_streamed_qlora_nf4_b200 import lib as L
+    L.load()
+    N, K, T, r = 6144, 4096, BATCH * SEQ, 16
+    g = torch.Generator(device="cuda").manual_seed(4)
+    W = torch.randn(N, K, generator=g, device="cuda") * 0.02
+    codes = torch.empty(N * K // 2, dtype=torch.uint8, device="cuda")
+    absmax = torch.empty(N * K // 64, dtype=torch.float32, device="cuda")
+    L.nf4_quantize(W, codes, absmax)
+    del W
+    # rotate over copies of the weight totalling > 2x L2, so each launch reads it from DRAM
+    n_copies = 24
+    wts = [(codes.clone(), absmax.clone()) for _ in range(n_copies)]
+    A = torch.randn(r, K, generator=g, device="cuda") / r
+    B = torch.randn(N, r, generator=g, device="cuda") * 0.01
+    x = torch.randn(T, K, generator=g, device="cuda").bfloat16()
+    y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(L.nf4_lora_linear_workspace_bytes(T, K, N, r), dtype=torch.uint8,
+                     device="cuda")
+    for i in range(args.warmup):
+        c, a = wts[i % n_copies]
+        L.nf4_lora_linear_fwd(x, c, a, A, B, 2.0, y, ws=ws)
+    torch.cuda.synchronize()
+    L.lsq_profile_enable(True)
+    for i in range(args.steps):
+        c, a = wts[(args.warmup + i) % n_copies]
+        L.nf4_lora_linear_fwd(x, c, a, A, B, 2.0, y, ws=ws)
+    torch.cuda.synchronize()
+    L.lsq_profile_enable(False)
+    prof = L.lsq_profile_read()["gemm_nf4_fwd"]
+    ms = prof["total_ms"] / prof["launches"]
+    tf = prof["flops"] / prof["launches"] / (ms * 1e-3) / 1e12
+    print(json.dumps(dict(case="gemm_qkv", M=N, K=K, T=T, ms=ms, tflops=tf,
+                          frac_of_burst=tf / peaks()["bf16_tflops"])), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.case == "layer":
+        return run_layer(args)
+    if args.case == "gemm":
+        return run_gemm(args)
     return run_ours(args)
 
 
