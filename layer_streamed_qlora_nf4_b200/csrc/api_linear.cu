@@ -190,7 +190,8 @@ extern "C" int nf4_lora_linear_bwd(const uint16_t* dy, const uint16_t* x, int64_
   LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, 1, pe, w.v, w.scratch, w.scratch_bytes, st));
   GemmDesc d = bwd_desc(dy, T, K, N, codes, absmax, A, r, scale, w.v, dx);
   LSQ_TRY(gemm_run(d, w.gemm, w.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(w.v, x, T, K, r, scale, accumulate, dA, st));
-  LSQ_TRY(launch_lora_grad_b(dy, w.u, T, N, r, r, 1, pe, scale, accumulate, dB, st));
+  LSQ_TRY(launch_lora_grad_a(w.v, x, T, K, r, scale, accumulate, dA, w.scratch, w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b(dy, w.u, T, N, r, r, 1, pe, scale, accumulate, dB, w.scratch,
+                             w.scratch_bytes, st));
   return LSQ_OK;
 }

@@ -222,7 +222,8 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
   if (lane == 0) delta[(int64_t)h * T + t] = acc;
 }
 
-// dK, dV for one key block of one kv head (sums over its query heads in order).
+// dK, dV contributions of one query head for one key block (written per query
+// head; the sum over a kv head's query heads happens later, in a fixed order).
 template <int D>
 __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ dout,
@@ -235,8 +236,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
   uint16_t* dOs = Qs + kTile * (D + 8);
   float* lse_s = reinterpret_cast<float*>(dOs + kTile * (D + 8));
   float* del_s = lse_s + kTile;
-  const int kb = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int rep = H / Hkv;
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (H / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int64_t ld = (int64_t)(H + 2 * Hkv) * D;
@@ -252,8 +253,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     for (int e = 0; e < 4; ++e) dkacc[j][e] = dvacc[j][e] = 0.f;
   const int krow[2] = {k0 + warp * 16 + gid, k0 + warp * 16 + gid + 8};
   const int nqb = (seq + kTile - 1) / kTile;
-  for (int hh = 0; hh < rep; ++hh) {
-    const int h = g * rep + hh;
+  {
     for (int qb = kb; qb < nqb; ++qb) {
       const int q0 = qb * kTile;
       __syncthreads();
@@ -350,8 +350,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
   for (int rI = 0; rI < 2; ++rI) {
     const int kr = krow[rI];
     if (kr >= seq) continue;
-    float* dkr = dk + (tok0 + kr) * (int64_t)Hkv * D + (int64_t)g * D;
-    float* dvr = dv + (tok0 + kr) * (int64_t)Hkv * D + (int64_t)g * D;
+    float* dkr = dk + (tok0 + kr) * (int64_t)H * D + (int64_t)h * D;
+    float* dvr = dv + (tok0 + kr) * (int64_t)H * D + (int64_t)h * D;
 #pragma unroll
     for (int j = 0; j < D / 8; ++j) {
       const int col = 8 * j + 2 * tig;
@@ -499,7 +499,7 @@ int attn_bwd_t(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout, con
   const int64_t nw = T * H;
   attn_delta_kernel<D><<<(unsigned)((nw * 32 + 255) / 256), 256, 0, st>>>(o, dout, T, H, delta);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  dim3 gkv((seq + kTile - 1) / kTile, Hkv, batch);
+  dim3 gkv((seq + kTile - 1) / kTile, H, batch);
   attn_bwd_dkdv_kernel<D><<<gkv, 128, s_kv, st>>>(qkv, dout, lse, delta, T, seq, H, Hkv, sl2, scale,
                                                   dk, dv);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));

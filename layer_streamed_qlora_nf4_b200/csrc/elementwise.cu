@@ -74,17 +74,29 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
 }
 
 // ------------------------------------------------------------------ RMSNorm
-// One warp per row; D % 8 == 0.
+// One CTA per row, 8 elements (16 bytes of bf16) per thread per pass; D % 8 == 0.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int i = 0; i < nw; ++i) t += red[i];  // fixed order
+  return t;
+}
+
 __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
-                                   int64_t T, int64_t D, float eps, uint16_t* __restrict__ y,
+                                   int64_t D, float eps, uint16_t* __restrict__ y,
                                    float* __restrict__ rstd) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (row >= T) return;
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + row * D);
-  const int64_t nv = D / 8;
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  uint4* yr = reinterpret_cast<uint4*>(y + row * D);
+  const int nv = (int)(D / 8);
   float ss = 0.f;
-  for (int64_t i = lane; i < nv; i += 32) {
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     const uint4 v = xr[i];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -94,12 +106,10 @@ __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_
       ss = fmaf(f.y, f.y, ss);
     }
   }
-  ss = warp_sum(ss);
+  ss = block_sum(ss, red);
   const float r = rsqrtf(ss / (float)D + eps);
-  if (lane == 0 && rstd) rstd[row] = r;
-  const uint4* gr = reinterpret_cast<const uint4*>(g);
-  uint4* yr = reinterpret_cast<uint4*>(y + row * D);
-  for (int64_t i = lane; i < nv; i += 32) {
+  if (threadIdx.x == 0 && rstd) rstd[row] = r;
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     const uint4 v = xr[i], gv = gr[i];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
     uint32_t o[4];
@@ -112,32 +122,31 @@ __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_
   }
 }
 
-// dx = dres + r (g dy) - x r^3 sum(g dy x) / D
+// dx = dres + r (g dy) - x r^3 sum(g dy x) / D;  one CTA per row, 4 elements per thread per pass
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t* __restrict__ x,
                                    const uint16_t* __restrict__ g, const float* __restrict__ rstd,
-                                   const float* __restrict__ dres, int64_t T, int64_t D,
+                                   const float* __restrict__ dres, int64_t D,
                                    float* __restrict__ dx, uint16_t* __restrict__ dxb) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (row >= T) return;
-  const int64_t nv = D / 4;
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const int nv = (int)(D / 4);
   const float4* dyr = reinterpret_cast<const float4*>(dy + row * D);
   const uint2* xr = reinterpret_cast<const uint2*>(x + row * D);
   const uint2* gr = reinterpret_cast<const uint2*>(g);
   float dot = 0.f;
-  for (int64_t i = lane; i < nv; i += 32) {
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     const float4 d = dyr[i];
     const uint2 xv = xr[i], gv = gr[i];
     const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
     const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
     dot += d.x * g0.x * x0.x + d.y * g0.y * x0.y + d.z * g1.x * x1.x + d.w * g1.y * x1.y;
   }
-  dot = warp_sum(dot);
+  dot = block_sum(dot, red);
   const float r = rstd[row];
   const float c = r * r * r * dot / (float)D;
   const float4* rr = dres ? reinterpret_cast<const float4*>(dres + row * D) : nullptr;
   float4* o = reinterpret_cast<float4*>(dx + row * D);
-  for (int64_t i = lane; i < nv; i += 32) {
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
     const float4 d = dyr[i];
     const uint2 xv = xr[i], gv = gr[i];
     const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
@@ -165,103 +174,154 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t*
 }
 
 // ------------------------------------------------------------------ RoPE
-// angle(pos, i) = pos * theta^(-2i/d), evaluated in double and rounded to fp32
-__device__ __forceinline__ void rope_cs(int pos, int i, int d, double log_theta, float* c,
-                                        float* s) {
-  const double ang = (double)pos * exp(-2.0 * (double)i / (double)d * log_theta);
-  double sd, cd;
-  sincos(ang, &sd, &cd);
-  *c = (float)cd;
-  *s = (float)sd;
-}
-
-// In-place rotation of the q and k heads of the fused qkv buffer (bf16).
-__global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int H, int Hkv, int d,
-                            double log_theta, int inverse) {
-  const int half = d / 2;
-  const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
-  const int64_t n = T * (H + Hkv) * half;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int j = (int)(i % half);
-    const int64_t th = i / half;
-    const int head = (int)(th % (H + Hkv));
-    const int64_t t = th / (H + Hkv);
-    const int pos = (int)(t % seq);
-    float c, s;
-    rope_cs(pos, j, d, log_theta, &c, &s);
-    if (inverse) s = -s;
-    uint16_t* base = qkv + t * ld + (int64_t)head * d;
-    const float x1 = bf16_bits_to_float(base[j]), x2 = bf16_bits_to_float(base[j + half]);
-    base[j] = float_to_bf16_bits(x1 * c - x2 * s);
-    base[j + half] = float_to_bf16_bits(x2 * c + x1 * s);
+// cs[pos][i] = (cos, sin)(pos * theta^(-2i/d)), evaluated in double, rounded to fp32.
+__global__ void rope_table_kernel(int seq, int half, int d, double log_theta, float2* __restrict__ cs) {
+  const int n = seq * half;
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
+    const int pos = k / half, i = k % half;
+    const double ang = (double)pos * exp(-2.0 * (double)i / (double)d * log_theta);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    cs[k] = make_float2((float)cd, (float)sd);
   }
 }
 
-// dqkv (bf16) <- [rope^-1(dq), rope^-1(dk), dv]  from fp32 gradients [T, H d], [T, Hkv d] x2
-__global__ void rope_grad_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
-                                 const float* __restrict__ dv, int64_t T, int seq, int H, int Hkv,
-                                 int d, double log_theta, uint16_t* __restrict__ dqkv) {
-  const int half = d / 2;
+// In-place rotation of the q and k heads of the fused qkv buffer (bf16); a
+// thread rotates 8 pairs (i, i + d/2).
+__global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int H, int Hkv, int d,
+                            const float2* __restrict__ cs) {
+  const int half = d / 2, chunks = half / 8;
   const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
-  const int64_t n = T * (H + 2 * Hkv) * half;
+  const int64_t n = T * (H + Hkv) * chunks;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int j = (int)(i % half);
-    const int64_t th = i / half;
+    const int ch = (int)(i % chunks);
+    const int64_t th = i / chunks;
+    const int head = (int)(th % (H + Hkv));
+    const int64_t t = th / (H + Hkv);
+    const int pos = (int)(t % seq);
+    uint16_t* base = qkv + t * ld + (int64_t)head * d + ch * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(base);
+    const uint4 b = *reinterpret_cast<const uint4*>(base + half);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+    const float2* c = cs + (int64_t)pos * half + ch * 8;
+    uint32_t oa[4], ob[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 x1 = unpack_bf16x2(aw[q]), x2 = unpack_bf16x2(bw[q]);
+      const float2 c0 = c[2 * q], c1 = c[2 * q + 1];
+      oa[q] = pack_bf16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
+      ob[q] = pack_bf16x2(x2.x * c0.x + x1.x * c0.y, x2.y * c1.x + x1.y * c1.y);
+    }
+    *reinterpret_cast<uint4*>(base) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+    *reinterpret_cast<uint4*>(base + half) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+  }
+}
+
+// dqkv (bf16) <- [rope^-1(dq), rope^-1(dk), dv].  dq is fp32 [T, H d]; dk and dv
+// arrive per query head (fp32 [T, H d]) and are summed over each kv head's
+// H/Hkv query heads in a fixed order here.  A thread handles 4 pairs.
+__global__ void rope_grad_kernel(const float* __restrict__ dq, const float* __restrict__ dk,
+                                 const float* __restrict__ dv, int64_t T, int seq, int H, int Hkv,
+                                 int d, const float2* __restrict__ cs,
+                                 uint16_t* __restrict__ dqkv) {
+  const int half = d / 2, chunks = half / 4, rep = H / Hkv;
+  const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
+  const int64_t hd = (int64_t)H * d;
+  const int64_t n = T * (H + 2 * Hkv) * chunks;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int ch = (int)(i % chunks);
+    const int64_t th = i / chunks;
     const int head = (int)(th % (H + 2 * Hkv));
     const int64_t t = th / (H + 2 * Hkv);
-    uint16_t* out = dqkv + t * ld + (int64_t)head * d;
+    uint16_t* out = dqkv + t * ld + (int64_t)head * d + ch * 4;
+    float4 g1 = make_float4(0, 0, 0, 0), g2 = make_float4(0, 0, 0, 0);
+    const float* src;
+    int nsum;
+    if (head < H) {
+      src = dq + t * hd + (int64_t)head * d;
+      nsum = 1;
+    } else if (head < H + Hkv) {
+      src = dk + t * hd + (int64_t)(head - H) * rep * d;
+      nsum = rep;
+    } else {
+      src = dv + t * hd + (int64_t)(head - H - Hkv) * rep * d;
+      nsum = rep;
+    }
+    for (int k = 0; k < nsum; ++k) {
+      const float4 a = *reinterpret_cast<const float4*>(src + (int64_t)k * d + ch * 4);
+      const float4 b = *reinterpret_cast<const float4*>(src + (int64_t)k * d + half + ch * 4);
+      g1.x += a.x; g1.y += a.y; g1.z += a.z; g1.w += a.w;
+      g2.x += b.x; g2.y += b.y; g2.z += b.z; g2.w += b.w;
+    }
     if (head >= H + Hkv) {
-      const float* src = dv + t * (int64_t)Hkv * d + (int64_t)(head - H - Hkv) * d;
-      out[j] = float_to_bf16_bits(src[j]);
-      out[j + half] = float_to_bf16_bits(src[j + half]);
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(g1.x, g1.y), pack_bf16x2(g1.z, g1.w));
+      *reinterpret_cast<uint2*>(out + half) =
+          make_uint2(pack_bf16x2(g2.x, g2.y), pack_bf16x2(g2.z, g2.w));
       continue;
     }
-    const float* src = (head < H) ? dq + t * (int64_t)H * d + (int64_t)head * d
-                                  : dk + t * (int64_t)Hkv * d + (int64_t)(head - H) * d;
     const int pos = (int)(t % seq);
-    float c, s;
-    rope_cs(pos, j, d, log_theta, &c, &s);
-    const float g1 = src[j], g2 = src[j + half];
-    out[j] = float_to_bf16_bits(g1 * c + g2 * s);
-    out[j + half] = float_to_bf16_bits(g2 * c - g1 * s);
+    const float2* c = cs + (int64_t)pos * half + ch * 4;
+    const float2 c0 = c[0], c1 = c[1], c2 = c[2], c3 = c[3];
+    *reinterpret_cast<uint2*>(out) =
+        make_uint2(pack_bf16x2(g1.x * c0.x + g2.x * c0.y, g1.y * c1.x + g2.y * c1.y),
+                   pack_bf16x2(g1.z * c2.x + g2.z * c2.y, g1.w * c3.x + g2.w * c3.y));
+    *reinterpret_cast<uint2*>(out + half) =
+        make_uint2(pack_bf16x2(g2.x * c0.x - g1.x * c0.y, g2.y * c1.x - g1.y * c1.y),
+                   pack_bf16x2(g2.z * c2.x - g1.z * c2.y, g2.w * c3.x - g1.w * c3.y));
   }
 }
 
 // ------------------------------------------------------------------ SwiGLU
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
 
+// 8 elements per thread (F % 8 == 0)
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, int64_t F,
                                   uint16_t* __restrict__ m) {
-  const int64_t nv = T * F / 2;
+  const int64_t nv = T * F / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t e = i * 2;
+    const int64_t e = i * 8;
     const int64_t t = e / F, f = e % F;
-    const float2 g = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + f));
-    const float2 u = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + F + f));
-    *reinterpret_cast<uint32_t*>(m + e) =
-        pack_bf16x2(g.x * sigmoidf_(g.x) * u.x, g.y * sigmoidf_(g.y) * u.y);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + f);
+    const uint4 uv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + F + f);
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 g = unpack_bf16x2(gw[q]), u = unpack_bf16x2(uw[q]);
+      o[q] = pack_bf16x2(g.x * sigmoidf_(g.x) * u.x, g.y * sigmoidf_(g.y) * u.y);
+    }
+    *reinterpret_cast<uint4*>(m + e) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
 __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* __restrict__ gu,
                                   int64_t T, int64_t F, uint16_t* __restrict__ dgu) {
-  const int64_t nv = T * F / 2;
+  const int64_t nv = T * F / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t e = i * 2;
+    const int64_t e = i * 8;
     const int64_t t = e / F, f = e % F;
-    const float2 g = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + f));
-    const float2 u = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(gu + t * 2 * F + F + f));
-    const float2 d = *reinterpret_cast<const float2*>(dm + e);
-    const float s0 = sigmoidf_(g.x), s1 = sigmoidf_(g.y);
-    const float dg0 = d.x * u.x * s0 * (1.f + g.x * (1.f - s0));
-    const float dg1 = d.y * u.y * s1 * (1.f + g.y * (1.f - s1));
-    const float du0 = d.x * g.x * s0, du1 = d.y * g.y * s1;
-    *reinterpret_cast<uint32_t*>(dgu + t * 2 * F + f) = pack_bf16x2(dg0, dg1);
-    *reinterpret_cast<uint32_t*>(dgu + t * 2 * F + F + f) = pack_bf16x2(du0, du1);
+    const uint4 gv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + f);
+    const uint4 uv = *reinterpret_cast<const uint4*>(gu + t * 2 * F + F + f);
+    const float4 d0 = *reinterpret_cast<const float4*>(dm + e);
+    const float4 d1 = *reinterpret_cast<const float4*>(dm + e + 4);
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    uint32_t og[4], ou[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 g = unpack_bf16x2(gw[q]), u = unpack_bf16x2(uw[q]);
+      const float s0 = sigmoidf_(g.x), s1 = sigmoidf_(g.y);
+      const float a = dd[2 * q], b = dd[2 * q + 1];
+      og[q] = pack_bf16x2(a * u.x * s0 * (1.f + g.x * (1.f - s0)),
+                          b * u.y * s1 * (1.f + g.y * (1.f - s1)));
+      ou[q] = pack_bf16x2(a * g.x * s0, b * g.y * s1);
+    }
+    *reinterpret_cast<uint4*>(dgu + t * 2 * F + f) = make_uint4(og[0], og[1], og[2], og[3]);
+    *reinterpret_cast<uint4*>(dgu + t * 2 * F + F + f) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
   }
 }
 
@@ -388,9 +448,14 @@ int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M,
   return LSQ_OK;
 }
 
+int threads_for_row(int64_t D, int per) {
+  int t = (int)std::min<int64_t>(256, (D / per + 31) / 32 * 32);
+  return t < 32 ? 32 : t;
+}
+
 int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
                        uint16_t* y, float* rstd, cudaStream_t st) {
-  rmsnorm_fwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(x, g, T, D, eps, y, rstd);
+  rmsnorm_fwd_kernel<<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -398,39 +463,45 @@ int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t 
 int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
                        const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
                        cudaStream_t st) {
-  rmsnorm_bwd_kernel<<<(unsigned)((T * 32 + 255) / 256), 256, 0, st>>>(dy, x, g, rstd, dres, T, D,
-                                                                      dx, dx_bf16);
+  rmsnorm_bwd_kernel<<<(unsigned)T, threads_for_row(D, 4), 0, st>>>(dy, x, g, rstd, dres, D, dx,
+                                                                   dx_bf16);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
-int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, float theta, int inverse,
+int launch_rope_table(int seq, int d, float theta, float2* cs, cudaStream_t st) {
+  const int n = seq * (d / 2);
+  rope_table_kernel<<<(unsigned)std::max(1, std::min(1024, (n + 255) / 256)), 256, 0, st>>>(
+      seq, d / 2, d, log((double)theta), cs);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
+int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, const float2* cs,
                 cudaStream_t st) {
-  const int64_t n = T * (H + Hkv) * (d / 2);
-  rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(qkv, T, seq, H, Hkv, d, log((double)theta),
-                                                inverse);
+  const int64_t n = T * (H + Hkv) * (d / 16);
+  rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(qkv, T, seq, H, Hkv, d, cs);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
-                     int Hkv, int d, float theta, uint16_t* dqkv, cudaStream_t st) {
-  const int64_t n = T * (H + 2 * Hkv) * (d / 2);
-  rope_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dq, dk, dv, T, seq, H, Hkv, d,
-                                                     log((double)theta), dqkv);
+                     int Hkv, int d, const float2* cs, uint16_t* dqkv, cudaStream_t st) {
+  const int64_t n = T * (H + 2 * Hkv) * (d / 8);
+  rope_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dq, dk, dv, T, seq, H, Hkv, d, cs, dqkv);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st) {
-  swiglu_fwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(gu, T, F, m);
+  swiglu_fwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(gu, T, F, m);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
                       cudaStream_t st) {
-  swiglu_bwd_kernel<<<grid_for(T * F / 2, 256), 256, 0, st>>>(dm, gu, T, F, dgu);
+  swiglu_bwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(dm, gu, T, F, dgu);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }

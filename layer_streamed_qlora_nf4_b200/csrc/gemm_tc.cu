@@ -46,6 +46,7 @@ constexpr int kWStageBytes = kBM * kBK * 2;  // 16 KB bf16 operand tile
 constexpr int kMaxStages = 4;
 constexpr int kMaxRing = 8;
 constexpr uint32_t kSmemBudget = 227 * 1024;
+constexpr uint32_t kAmRingBytes = 3 * 128 * 8 * 4;  // absmax slots: 3 k-tiles x 128 threads x 8
 
 struct KParams {
   int M, T, Kc;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* xs0 = dsm;
   uint8_t* ws0 = xs0 + (size_t)p.stages * xs_bytes;
   uint8_t* rg0 = ws0 + (size_t)p.stages * kWStageBytes;
+  float* am_ring = reinterpret_cast<float*>(rg0 + (size_t)p.ring_stages * p.ring_bytes);  // [3][128][8]
 
   const int m0 = blockIdx.x * kBM;
   const int t0 = blockIdx.y * BT;
@@ -219,13 +221,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- operand stage
     const int tid = threadIdx.x - 128;  // 0..127
     const int nblk = p.w_cols / 64;
+    // absmax of this thread's rows for k-tile `it`, copied into a per-thread
+    // shared-memory slot ring two k-tiles ahead with cp.async (the global
+    // latency stays off the critical path): NF4_N needs one value per k-tile
+    // (row m0 + tid, block kt), NF4_T eight (rows kt*64 + 8bi .. +7, block
+    // (m0 + 8bj) / 64).
+    const int bi = tid & 7, bj = tid >> 3;
+    auto am_slot = [&](int it, int rr) -> float* { return am_ring + ((it % 3) * 128 + tid) * 8 + rr; };
+    auto issue_am = [&](int it) {
+      if (it < n_main && (WMODE == W_NF4_N || WMODE == W_NF4_T)) {
+        const int kt = kt_begin + it;
+        if (WMODE == W_NF4_N) {
+          const int m = m0 + tid;
+          const bool in = m < p.w_rows;
+          cp_async4(smem_u32(am_slot(it, 0)), p.absmax + (in ? (size_t)m * nblk + kt : 0),
+                    in ? 4u : 0u);
+        } else {
+          const int mcol = m0 + 8 * bj;
+#pragma unroll
+          for (int rr = 0; rr < 8; ++rr) {
+            const int n = kt * kBK + 8 * bi + rr;
+            const bool in = n < p.w_rows && mcol < p.w_cols;
+            cp_async4(smem_u32(am_slot(it, rr)),
+                      p.absmax + (in ? (size_t)n * nblk + (mcol >> 6) : 0), in ? 4u : 0u);
+          }
+        }
+      }
+      cp_async_commit();  // one group per k-tile (possibly empty) keeps the counting uniform
+    };
+    issue_am(0);
+    issue_am(1);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
       uint8_t* wst = ws0 + (size_t)s * kWStageBytes;
+      issue_am(it + 2);
+      cp_async_wait<2>();  // the group of k-tile `it` has landed
       if (it < n_main) {
-        const int kt = kt_begin + it;
         if (WMODE == W_BF16_N) {
           ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                  DEV_ERR_WAIT_GEMM);
@@ -234,9 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = it % CS;
           const uint32_t cph = (uint32_t)(it / CS) & 1u;
           const uint8_t* ring = rg0 + (size_t)c * p.ring_bytes;
+          const float* amc = am_slot(it, 0);
           if (WMODE == W_NF4_N) {
-            const int m = m0 + tid;
-            const float am = (m < p.w_rows) ? __ldg(p.absmax + (size_t)m * nblk + kt) : 0.f;
+            const float am = amc[0];
             ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                    DEV_ERR_WAIT_GEMM) &&
                  mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -260,17 +293,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           } else if (WMODE == W_NF4_T) {
-            const int bi = tid & 7;   // rows 8bi..8bi+7 of the staged [64 x 128] tile
-            const int bj = tid >> 3;  // columns 8bj..8bj+7 (output features)
-            const int mcol = m0 + 8 * bj;
-            float am[8];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-              const int n = kt * kBK + 8 * bi + rr;
-              am[rr] = (n < p.w_rows && mcol < p.w_cols)
-                           ? __ldg(p.absmax + (size_t)n * nblk + (mcol >> 6))
-                           : 0.f;
-            }
             ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                    DEV_ERR_WAIT_GEMM) &&
                  mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -288,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int rr = 0; rr < 8; ++rr) {
                   const uint32_t byte = (w[rr] >> (8 * (cc >> 1))) & 0xFFu;
                   const uint32_t code = (cc & 1) ? (byte & 15u) : (byte >> 4);
-                  v[rr] = lv_sh[code] * am[rr];
+                  v[rr] = lv_sh[code] * amc[rr];
                 }
                 *reinterpret_cast<uint4*>(wst + sw128_offset(8 * bj + cc, bi)) =
                     make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
@@ -296,7 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           } else {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
-            const int bi = tid & 7, bj = tid >> 3;
             ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                    DEV_ERR_WAIT_GEMM) &&
                  mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -505,7 +526,8 @@ Plan make_plan(const GemmDesc& d) {
   int ring = (d.wmode == W_BF16_N) ? 0 : (d.wmode == W_BF16_T ? 2 : kMaxRing);
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
-    return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes;
+    return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes +
+           kAmRingBytes;
   };
   while (stages > 2 && total(stages, ring) > kSmemBudget - 4096) --stages;
   while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;

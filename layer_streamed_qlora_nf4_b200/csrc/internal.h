@@ -107,10 +107,13 @@ int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t 
 int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
                        const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
                        cudaStream_t st);
-int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, float theta,
-                int inverse, cudaStream_t st);
+// cos/sin table [seq][d/2] for rotate-half RoPE
+int launch_rope_table(int seq, int d, float theta, float2* cs, cudaStream_t st);
+int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, const float2* cs,
+                cudaStream_t st);
+// dk, dv are per query head [T, H d] (summed over each kv group here)
 int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
-                     int Hkv, int d, float theta, uint16_t* dqkv, cudaStream_t st);
+                     int Hkv, int d, const float2* cs, uint16_t* dqkv, cudaStream_t st);
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st);
 int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
                       cudaStream_t st);
@@ -139,15 +142,17 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
                       size_t scratch_bytes, cudaStream_t st);
 // dA[j, k] (+)= s * sum_t v[t, j] * x[t, k]              v fp32 [T, R], x bf16 [T, K]
 int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
-                       int accumulate, float* dA, cudaStream_t st);
+                       int accumulate, float* dA, float* scratch, size_t scratch_bytes,
+                       cudaStream_t st);
 // dB[n, j] (+)= s * sum_t dy[t, n] * u[t, part(n)*r + j]  dy bf16 [T, N], u fp32 [T, R]
 int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
                        int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
-                       cudaStream_t st);
+                       float* scratch, size_t scratch_bytes, cudaStream_t st);
 
 // attention (causal GQA), q/k/v read from the fused qkv buffer [T, (H + 2 Hkv) d]
 int launch_attention_fwd(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d,
                          uint16_t* o, float* lse, cudaStream_t st);
+// dk, dv are written per query head: [T, H d] fp32 (the kv-group sum happens in rope_grad)
 int launch_attention_bwd(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout,
                          const float* lse, int64_t T, int seq, int H, int Hkv, int d, float* delta,
                          float* dq, float* dk, float* dv, cudaStream_t st);

@@ -125,6 +125,7 @@ struct Buffers {
   uint16_t *n1, *qkv, *ao, *h, *n2, *gu, *m, *dgu, *dqkv, *da, *dout_b, *dh_b;
   float *rstd1, *rstd2, *u_qkv, *u_o, *u_gu, *u_d, *lse, *v_qkv, *v_o, *v_gu, *v_d;
   float *dm, *dn2, *dh, *dn1, *dq, *dk, *dv, *delta;
+  float2* rope_cs;
   float* lscratch;
   size_t lscratch_bytes;
   void* gemm;
@@ -225,9 +226,10 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   x.dh = a.take<float>(T * s.D);
   x.dn1 = a.take<float>(T * s.D);
   x.dq = a.take<float>(T * s.qd);
-  x.dk = a.take<float>(T * s.kvd);
-  x.dv = a.take<float>(T * s.kvd);
+  x.dk = a.take<float>(T * s.qd);   // per query head, summed per kv head in rope_grad
+  x.dv = a.take<float>(T * s.qd);
   x.delta = a.take<float>(T * s.H);
+  x.rope_cs = a.take<float2>(T * s.hd / 2);  // >= seq * d/2 entries
   // LoRA K-split scratch: the largest of every skinny product in the layer
   size_t ls = 0;
   const int64_t Ks[4] = {s.D, s.qd, s.F, std::max(s.qkv_n, s.gu_n)};
@@ -281,7 +283,8 @@ int forward_core(const LayerShapes& s, const Views& v, const uint16_t* x, int ba
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
                            3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, theta, 0, st));
+  LSQ_TRY(launch_rope_table(seq, s.hd, theta, b.rope_cs, st));
+  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
   LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
@@ -367,36 +370,36 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   LSQ_TRY(launch_lora_vproj(dout_b, T, s.D, v.B_d, r, 1, pe1, b.v_d, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.A_d, r, sc, b.v_d, b.dm, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_d, b.m, T, s.F, r, sc, accumulate, gA_d, st));
-  LSQ_TRY(launch_lora_grad_b(dout_b, b.u_d, T, s.D, r, r, 1, pe1, sc, accumulate, gB_d, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_d, b.m, T, s.F, r, sc, accumulate, gA_d, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b(dout_b, b.u_d, T, s.D, r, r, 1, pe1, sc, accumulate, gB_d, b.lscratch, b.lscratch_bytes, st));
   // SwiGLU and gate|up
   LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
   LSQ_TRY(launch_lora_vproj(b.dgu, T, s.gu_n, v.B_gu, r, 2, pe2, b.v_gu, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc, b.v_gu,
                           b.dn2, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, st));
-  LSQ_TRY(launch_lora_grad_b(b.dgu, b.u_gu, T, s.gu_n, r, 2 * r, 2, pe2, sc, accumulate, gB_gu, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b(b.dgu, b.u_gu, T, s.gu_n, r, 2 * r, 2, pe2, sc, accumulate, gB_gu, b.lscratch, b.lscratch_bytes, st));
   // second RMSNorm + residual
   LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
   // o projection
   LSQ_TRY(launch_lora_vproj(b.dh_b, T, s.D, v.B_o, r, 1, pe1, b.v_o, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.A_o, r, sc, b.v_o, b.da, 0),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, st));
-  LSQ_TRY(launch_lora_grad_b(b.dh_b, b.u_o, T, s.D, r, r, 1, pe1, sc, accumulate, gB_o, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b(b.dh_b, b.u_o, T, s.D, r, r, 1, pe1, sc, accumulate, gB_o, b.lscratch, b.lscratch_bytes, st));
   // attention, RoPE
   LSQ_TRY(launch_attention_bwd(b.qkv, b.ao, b.da, b.lse, T, seq, s.H, s.Hkv, s.hd, b.delta, b.dq,
                                b.dk, b.dv, st));
-  LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, cfg->rope_theta, b.dqkv, st));
+  LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, b.rope_cs, b.dqkv, st));
   // q|k|v projections
   LSQ_TRY(launch_lora_vproj(b.dqkv, T, s.qkv_n, v.B_qkv, r, 3, pe3, b.v_qkv, b.lscratch,
                             b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
                           b.v_qkv, b.dn1, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, st));
-  LSQ_TRY(launch_lora_grad_b(b.dqkv, b.u_qkv, T, s.qkv_n, r, 3 * r, 3, pe3, sc, accumulate, gB_qkv, st));
+  LSQ_TRY(launch_lora_grad_a(b.v_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b(b.dqkv, b.u_qkv, T, s.qkv_n, r, 3 * r, 3, pe3, sc, accumulate, gB_qkv, b.lscratch, b.lscratch_bytes, st));
   // first RMSNorm + residual
   LSQ_TRY(launch_rmsnorm_bwd(b.dn1, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16, st));
   return LSQ_OK;
