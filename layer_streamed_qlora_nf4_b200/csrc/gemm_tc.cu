@@ -79,13 +79,16 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 template <int WMODE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
-                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ KParams p) {
+                   const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_out,
+                   const __grid_constant__ CUtensorMap tm_res, const __grid_constant__ KParams p) {
   extern __shared__ uint8_t dsm_raw[];
   __shared__ __align__(8) uint64_t bar_full[kMaxStages];
   __shared__ __align__(8) uint64_t bar_empty[kMaxStages];
   __shared__ __align__(8) uint64_t bar_cfull[kMaxRing];
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
+  __shared__ __align__(8) uint64_t bar_epi;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float lv_sh[16];
@@ -122,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bar_cempty[c]), 4);
     }
     mbar_init(smem_u32(&bar_acc), 1);
+    mbar_init(smem_u32(&bar_epi), 1);
     abort_sh = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -404,36 +408,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           DEV_ERR_WAIT_GEMM);
     acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
     if (acc_ok) {
+      // Stage 32-token chunks of the [tokens x 128 features] tile in shared
+      // memory (the drained pipeline buffers: 4 chunk slots of 2 x 16 rows x 128
+      // features, i.e. 16 KB for fp32 and 8 KB for bf16 outputs) and write
+      // them with TMA stores of 16-row boxes, so each CTA writes only its own
+      // token range.  Residual tiles arrive by TMA into the slot and are added
+      // in place.
       tc_fence_after();
       const int qtr = warp & 3;
-      const int m = m0 + qtr * 32 + lane;
+      const int row = qtr * 32 + lane;   // feature within the tile
       const uint32_t tbase = tmem + ((uint32_t)(qtr * 32) << 16);
+      const bool leader = (warp == 4 && lane == 0);
+      const bool partial = p.splits > 1;
+      const bool f32 = partial || p.out_f32;
+      const int es = f32 ? 4 : 2;
+      const bool res = !partial && p.residual != nullptr;
+      const uint32_t sub_bytes = 16u * 128u * (uint32_t)es;
+      int q = 0, nres = 0;
       for (int a = 0; a < p.nacc; ++a) {
-        for (int c0 = 0; c0 < p.bn; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, r);
-          tmem_ld_wait();
+        for (int c0 = 0; c0 < p.bn; c0 += 32, ++q) {
           const int tb = t0 + a * p.bn + c0;
-          if (m < p.M) {
+          if (tb >= p.T) break;                         // uniform across the 128 threads
+          const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
+          uint8_t* slot = dsm + (size_t)(q & 3) * (2 * sub_bytes);  // a 32-token chunk
+          if (q >= 4 && leader) bulk_wait_read<3>();    // the store that used this slot has read it
+          named_barrier(1, 128);
+          if (res) {
+            if (leader) {
+              mbar_arrive_expect_tx(smem_u32(&bar_epi), (uint32_t)nsub * sub_bytes);
+              for (int sb = 0; sb < nsub; ++sb)
+                tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, smem_u32(&bar_epi), m0,
+                            tb + 16 * sb);
+            }
+            acc_ok = mbar_wait_bounded(smem_u32(&bar_epi), (uint32_t)(nres & 1), abort_flag,
+                                       p.dev_err, DEV_ERR_WAIT_GEMM);
+            ++nres;
+          }
+          uint32_t r[2][16];
+          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, r[0]);
+          if (nsub == 2) tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0 + 16, r[1]);
+          tmem_ld_wait();
+          for (int sb = 0; sb < nsub; ++sb) {
+            uint8_t* base = slot + sb * sub_bytes;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const int t = tb + j;
-              if (t < p.T) {
-                float val = __uint_as_float(r[j]);
-                if (p.splits > 1) {
-                  p.partial[((size_t)split * p.T + t) * p.M + m] = val;
-                } else {
-                  if (p.residual) val += bf16_bits_to_float(p.residual[(size_t)t * p.ldr + m]);
-                  if (p.out_f32)
-                    static_cast<float*>(p.out)[(size_t)t * p.ldo + m] = val;
-                  else
-                    static_cast<uint16_t*>(p.out)[(size_t)t * p.ldo + m] = float_to_bf16_bits(val);
-                }
+              float v = __uint_as_float(r[sb][j]);
+              if (f32) {
+                *reinterpret_cast<float*>(base + (j * 128 + row) * 4) = v;
+              } else {
+                uint16_t* d = reinterpret_cast<uint16_t*>(base + (j * 128 + row) * 2);
+                if (res) v += bf16_bits_to_float(*d);
+                *d = float_to_bf16_bits(v);
               }
             }
           }
+          fence_proxy_async_smem();
+          named_barrier(1, 128);
+          if (leader) {
+            for (int sb = 0; sb < nsub; ++sb) {
+              if (tb + 16 * sb >= p.T) break;
+              if (partial)
+                tma_store_3d(&tm_out, smem_u32(slot + sb * sub_bytes), m0, tb + 16 * sb, split);
+              else
+                tma_store_2d(&tm_out, smem_u32(slot + sb * sub_bytes), m0, tb + 16 * sb);
+            }
+            bulk_commit();
+          }
         }
       }
+      if (leader) bulk_wait_all();
     }
   }
 
@@ -533,7 +576,7 @@ Plan make_plan(const GemmDesc& d) {
   while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;
   pl.stages = stages;
   pl.ring_stages = std::max(ring, 1);
-  pl.smem_bytes = total(stages, ring);
+  pl.smem_bytes = std::max(total(stages, ring), 1024u + 4u * 16384u);  // epilogue chunk slots
   uint32_t cols = 32;
   while (cols < (uint32_t)pl.bn) cols <<= 1;
   pl.alloc_cols = (pl.nacc > 1) ? 512u : cols;
@@ -571,6 +614,31 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
                       (uint64_t)d.w_rows, (uint64_t)d.w_cols, 128, 64,
                       CU_TENSOR_MAP_SWIZZLE_NONE));
+  CUtensorMap tm_out, tm_res;
+  if (partial) {
+    PFN_encodeTiled enc = get_encode();
+    if (!enc) return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)d.M, (cuuint64_t)d.T, (cuuint64_t)pl.splits};
+    cuuint64_t strides[2] = {(cuuint64_t)d.M * 4, (cuuint64_t)d.M * (cuuint64_t)d.T * 4};
+    cuuint32_t box[3] = {128, 16, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, partial, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled (partials) failed (%d)", (int)r);
+  } else if (d.out_f32) {
+    LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d.out, (uint64_t)d.M,
+                      (uint64_t)d.T, (uint64_t)d.ldo, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+  } else {
+    LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.out, (uint64_t)d.M,
+                      (uint64_t)d.T, (uint64_t)d.ldo, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+  }
+  if (d.residual && !partial)
+    LSQ_TRY(make_tmap(&tm_res, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.residual, (uint64_t)d.M,
+                      (uint64_t)d.T, (uint64_t)d.ldr, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+  else
+    tm_res = tm_out;  // unused
   KParams p{};
   p.M = (int)d.M;
   p.T = (int)d.T;
@@ -608,7 +676,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   for (int i = 0; i < 16; ++i) p.levels[i] = lv[i];
   if (!p.dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
   dim3 grid(pl.m_tiles, pl.t_tiles, pl.splits);
-  tc_gemm_kernel<WMODE><<<grid, kThreads, pl.smem_bytes, st>>>(tm_act, tm_w, p);
+  tc_gemm_kernel<WMODE><<<grid, kThreads, pl.smem_bytes, st>>>(tm_act, tm_w, tm_out, tm_res, p);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -654,6 +722,9 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (d.slab_w % 16 != 0 || d.slab_w < 0)
     return set_error(LSQ_ERR_SHAPE, "gemm: LoRA slab width must be a multiple of 16");
   if (d.slab_w > 0 && (!d.la || !d.lb)) return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
+  if (d.residual && d.out_f32) return set_error(LSQ_ERR_INVALID, "gemm: residual needs a bf16 output");
+  if (d.ldo % 8 != 0 || (d.residual && d.ldr % 8 != 0))
+    return set_error(LSQ_ERR_SHAPE, "gemm: output strides must be multiples of 16 bytes");
   if (d.M > INT32_MAX || d.T > INT32_MAX || d.Kc > INT32_MAX)
     return set_error(LSQ_ERR_SHAPE, "gemm: dimension too large");
   Plan pl = make_plan(d);
