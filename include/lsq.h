@@ -282,6 +282,29 @@ int lsq_profile_enable(int enable);
 /* Synchronises the recorded events and fills up to max entries (one per class). */
 int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out);
 
+/* --------------------------------------------------- allocation-free variant */
+
+/* nf4_lora_linear_fwd_noalloc - the same computation and kernels as
+ * nf4_lora_linear_fwd, for callers that cannot provide a device workspace (a
+ * host framework that keeps all device memory in its own pool and gives plugins
+ * no allocator, or a latency-critical caller that cannot afford the device-wide
+ * synchronisation cudaMalloc/cudaFree may cause).  This entry point is an
+ * engineering addition with no counterpart on the pages the method comes from.
+ *   Arguments as nf4_lora_linear_fwd, without ws/ws_bytes.
+ *   Scratch: a fixed 32 MiB device array built into the library; every GPU that
+ *   loads the library holds it until the process exits.  Sizes whose
+ *   nf4_lora_linear_workspace_bytes exceeds 32 MiB are rejected with
+ *   LSQ_ERR_WORKSPACE.  No allocation happens in the call.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array: calls that can overlap on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  Nothing in the array needs to start at zero. */
+int nf4_lora_linear_fwd_noalloc(const uint16_t* x, int64_t T, int64_t K, int64_t N,
+                                const uint8_t* codes, const float* absmax, int32_t block,
+                                const float* A, const float* B, int32_t r, float scale,
+                                const uint16_t* residual, uint16_t* y, float* u_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

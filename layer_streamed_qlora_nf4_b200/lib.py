@@ -24,6 +24,7 @@ EXPORTS = (
     "decoder_layer_bwd", "stream_stack_create", "stream_stack_destroy",
     "stream_stack_workspace_bytes", "stream_stack_step", "stream_stack_last_stats",
     "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
+    "nf4_lora_linear_fwd_noalloc",
 )
 
 
@@ -104,6 +105,8 @@ _PROTOS = {
     "stream_stack_last_stats": (ctypes.c_int, [_P, ctypes.POINTER(lsq_step_stats)]),
     "lora_adamw_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(lsq_adamw), _I64, _P]),
     "lsq_launch_counter": (ctypes.c_int64, []),
+    "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
+                                                   _F, _P, _P, _P, _P]),
     "lsq_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "lsq_profile_read": (ctypes.c_int, [ctypes.POINTER(lsq_prof_entry), _I32,
                                         ctypes.POINTER(ctypes.c_int32)]),
@@ -320,3 +323,14 @@ def lsq_profile_read():
     return {arr[i].name.decode(): dict(launches=arr[i].launches, total_ms=arr[i].total_ms,
                                        flops=arr[i].flops, bytes=arr[i].bytes)
             for i in range(n.value)}
+
+
+def nf4_lora_linear_fwd_noalloc(x, codes, absmax, A, B, scale, y, residual=None, u_out=None,
+                                block=64, stream=None):
+    """nf4_lora_linear_fwd with the library's built-in scratch instead of a workspace."""
+    T, K = x.shape
+    N = y.shape[1]
+    r = A.shape[0]
+    _check(load().nf4_lora_linear_fwd_noalloc(_ptr(x), T, K, N, _ptr(codes), _ptr(absmax), block,
+                                              _ptr(A), _ptr(B), r, scale, _ptr(residual), _ptr(y),
+                                              _ptr(u_out), _stream(stream)))
