@@ -226,15 +226,11 @@ def h2d_bandwidth(nbytes, reps=10):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    from layer_streamed_qlora_nf4_b200 import dp
+    _, _, local = dp.env()
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
         torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+    rank, world = dp.init("nccl", device=torch.device("cuda", local))
     from layer_streamed_qlora_nf4_b200 import lib as L
     from layer_streamed_qlora_nf4_b200 import synth
     L.load()
@@ -248,6 +244,7 @@ def run_ours(args):
     m, v = torch.zeros_like(lora), torch.zeros_like(lora)
     opt = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, m=m, v=v)
     stream = torch.cuda.current_stream()
+    pool = st["tokens"]           # a few distinct batches, cycled
 
     def step(tokens):
         if world == 1:
@@ -256,86 +253,85 @@ def run_ours(args):
         else:
             loss = L.stream_stack_step(handle, tokens, 1, BATCH, SEQ, st["emb"], st["head"],
                                        st["gf"], lora, grad, None, ws)
-            dist.all_reduce(grad, op=dist.ReduceOp.AVG)
+            dp.average_(grad)                       # NCCL all-reduce of the LoRA gradients
             L.lora_adamw_step(lora, grad, opt)
         opt["step"] += 1
         return loss
 
-    pool = st["tokens"]           # a few distinct batches, cycled
+    def timed(steps, tokens_of, profile=False, label="timed"):
+        """Device time per step over `steps` steps (barrier + sync on both sides,
+        CUDA events on the compute stream, max over ranks)."""
+        dp.barrier()
+        torch.cuda.synchronize()
+        copies, wait_ms = 0, 0.0
+        if profile:
+            L.lsq_profile_enable(True)
+        n0 = L.lsq_launch_counter()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        torch.cuda.nvtx.range_push(label)     # lets a profiler select exactly these steps
+        loss = None
+        for i in range(steps):
+            loss = step(tokens_of(i))
+            s = L.stream_stack_last_stats(handle)
+            copies += s["layer_copies"]
+            wait_ms += s["copy_wait_ms"]
+        torch.cuda.nvtx.range_pop()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dp.barrier()
+        launches = L.lsq_launch_counter() - n0
+        prof = None
+        if profile:
+            L.lsq_profile_enable(False)
+            prof = L.lsq_profile_read()
+        ms = dp.max_over_ranks(e0.elapsed_time(e1) / steps, "cuda")
+        return ms, loss, copies, wait_ms, launches, prof
+
     for i in range(args.warmup):
         loss = step(pool[i % len(pool)])
     torch.cuda.synchronize()
     h2d_gbs = h2d_bandwidth(lay.bytes)
 
+    # ------------------------------------------------------------ timed region (headline)
     uuid = str(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "uuid", ""))
     sampler = ClockSampler(uuid)
-    # ------------------------------------------------------------ timed region
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     sampler.start()
-    L.lsq_profile_enable(True)
-    n0 = L.lsq_launch_counter()
-    copies, wait_ms = 0, 0.0
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    torch.cuda.nvtx.range_push("timed")   # lets a profiler select exactly the timed steps
-    for i in range(args.steps):
-        loss = step(pool[i % len(pool)])
-        s = L.stream_stack_last_stats(handle)
-        copies += s["layer_copies"]
-        wait_ms += s["copy_wait_ms"]
-    torch.cuda.nvtx.range_pop()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    launches = L.lsq_launch_counter() - n0
-    L.lsq_profile_enable(False)
+    ms, loss, copies, wait_ms, launches, _ = timed(args.steps, lambda i: pool[i % len(pool)])
     clocks = sampler.stop()
-    prof = L.lsq_profile_read()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     value = world * BATCH * SEQ / (ms * 1e-3)
+
+    # ------------------------------------------------------------ same steps, kernels timed
+    # every tensor-core GEMM and attention launch bracketed by CUDA events on its stream
+    ms_prof, _, _, _, _, prof = timed(args.steps, lambda i: pool[i % len(pool)], profile=True,
+                                      label="timed_kernels")
 
     # ------------------------------------------------------------ end to end (host buffers)
     tok_host = pool.cpu().pin_memory()
     tok_dev = torch.empty_like(pool[0])
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for i in range(args.steps):
+
+    def from_host(i):
         tok_dev.copy_(tok_host[i % len(tok_host)], non_blocking=True)
-        loss = step(tok_dev)           # returns the loss on the host
-    f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+        return tok_dev                  # the step itself returns the loss on the host
+    e2e_ms = timed(args.steps, from_host, label="timed_e2e")[0]
     e2e = dict(value=world * BATCH * SEQ / (e2e_ms * 1e-3), unit="tokens/s",
                h2d_bytes_per_step=tok_dev.numel() * 4, d2h_bytes_per_step=4,
                layer_stream_h2d_bytes_per_step=copies // args.steps * lay.bytes)
 
     pk = peaks()
-    # dominant kernel: the class with the most device time in the timed region
+    # dominant kernel: the class with the most device time in the profiled steps
     dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
     per_launch_ms = dom["total_ms"] / dom["launches"]
-    tc = dom_name.startswith("gemm") or dom_name.startswith("attention")
     achieved = (dom["flops"] / dom["launches"]) / (per_launch_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops_sustained"]
-    roofline = dict(bound="tensor" if tc else "hbm", kernel=dom_name, achieved=achieved,
-                    peak=peak, unit="TFLOP/s", frac=achieved / peak, traffic=None,
-                    peak_source="%s (bf16 sustained, kernel timed inside a long step)" % pk["source"],
-                    launches_per_step=dom["launches"] / args.steps,
-                    per_launch_ms=per_launch_ms,
-                    step_share=dom["total_ms"] / args.steps / ms)
+    roofline = dict(bound="tensor", kernel=dom_name, achieved=achieved, peak=peak, unit="TFLOP/s",
+                    frac=achieved / peak, traffic=None,
+                    peak_source="%s bf16 sustained (kernel timed inside a long step)" % pk["source"],
+                    launches_per_step=dom["launches"] / args.steps, per_launch_ms=per_launch_ms,
+                    step_share=dom["total_ms"] / args.steps / ms_prof,
+                    timing="CUDA events around every launch of the class on its stream, over a "
+                           "second timed region of the same %d steps (%.1f ms/step with the "
+                           "events)" % (args.steps, ms_prof))
     # step roofline: slowest of tensor FLOPs at peak, algorithmic DRAM bytes at the
     # measured copy bandwidth, and the streamed layer bytes at the measured H2D bandwidth
     flops_step = sum(e["flops"] for e in prof.values()) / args.steps
@@ -347,8 +343,9 @@ def run_ours(args):
     t_roof = max(t_tc, t_hbm, t_h2d)
     step_roof = dict(t_tensor_ms=t_tc, t_hbm_ms=t_hbm, t_h2d_ms=t_h2d,
                      bound=["tensor", "hbm", "h2d"][[t_tc, t_hbm, t_h2d].index(t_roof)],
-                     frac=t_roof / ms, h2d_gbs_measured=h2d_gbs, layer_copies_per_step=cps,
-                     layer_bytes=lay.bytes, copy_wait_ms_per_step=wait_ms / args.steps,
+                     frac=t_roof / ms, frac_e2e=t_roof / e2e_ms, h2d_gbs_measured=h2d_gbs,
+                     layer_copies_per_step=cps, layer_bytes=lay.bytes,
+                     copy_wait_ms_per_step=wait_ms / args.steps,
                      tflop_per_step=flops_step / 1e12,
                      kernels={k: dict(launches_per_step=e["launches"] / args.steps,
                                       ms_per_step=e["total_ms"] / args.steps,
@@ -375,6 +372,7 @@ def run_ours(args):
                     e2e=e2e, gpu_launches=int(launches), clocks=clocks)
         print(json.dumps(line), flush=True)
     if world > 1:
+        import torch.distributed as dist
         dist.destroy_process_group()
     return 0
 
@@ -477,23 +475,31 @@ def run_gemm(args):
     B = torch.randn(N, r, generator=g, device="cuda") * 0.01
     x = torch.randn(T, K, generator=g, device="cuda").bfloat16()
     y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    dy = torch.randn(T, N, generator=g, device="cuda").bfloat16()
+    dx = torch.empty(T, K, dtype=torch.bfloat16, device="cuda")
+    dA, dB = torch.empty(r, K, device="cuda"), torch.empty(N, r, device="cuda")
     ws = torch.empty(L.nf4_lora_linear_workspace_bytes(T, K, N, r), dtype=torch.uint8,
                      device="cuda")
-    for i in range(args.warmup):
+
+    def it(i):
         c, a = wts[i % n_copies]
         L.nf4_lora_linear_fwd(x, c, a, A, B, 2.0, y, ws=ws)
+        L.nf4_lora_linear_bwd(dy, x, c, a, A, B, 2.0, dx, dA, dB, ws=ws)
+
+    for i in range(args.warmup):
+        it(i)
     torch.cuda.synchronize()
     L.lsq_profile_enable(True)
     for i in range(args.steps):
-        c, a = wts[(args.warmup + i) % n_copies]
-        L.nf4_lora_linear_fwd(x, c, a, A, B, 2.0, y, ws=ws)
+        it(args.warmup + i)
     torch.cuda.synchronize()
     L.lsq_profile_enable(False)
-    prof = L.lsq_profile_read()["gemm_nf4_fwd"]
-    ms = prof["total_ms"] / prof["launches"]
-    tf = prof["flops"] / prof["launches"] / (ms * 1e-3) / 1e12
-    print(json.dumps(dict(case="gemm_qkv", M=N, K=K, T=T, ms=ms, tflops=tf,
-                          frac_of_burst=tf / peaks()["bf16_tflops"])), flush=True)
+    out = dict(case="gemm_qkv", M=N, K=K, T=T)
+    for k, e in L.lsq_profile_read().items():
+        ms = e["total_ms"] / e["launches"]
+        tf = e["flops"] / e["launches"] / (ms * 1e-3) / 1e12
+        out[k] = dict(us=ms * 1e3, tflops=tf, frac_of_burst=tf / peaks()["bf16_tflops"])
+    print(json.dumps(out), flush=True)
     return 0
 
 

@@ -1,0 +1,55 @@
+"""Data-parallel plumbing for running N replicas of the streamed step (one
+process per GPU, torch.distributed).  Each rank streams its own copy of the
+frozen stack on its own micro-batch; the only exchange is the average of the
+LoRA gradients before the (identical) AdamW update on every rank.  Timing is
+the maximum over ranks.  NCCL on GPUs; the same code runs on gloo for tests.
+"""
+import datetime
+import os
+
+import torch
+import torch.distributed as dist
+
+
+def env():
+    """(rank, world_size, local_rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init(backend, timeout_s=300, device=None):
+    """Initialise the default process group if the job has more than one rank."""
+    rank, world, _ = env()
+    if world > 1 and not dist.is_initialized():
+        kw = dict(timeout=datetime.timedelta(seconds=timeout_s))
+        if device is not None:
+            kw["device_id"] = device
+        dist.init_process_group(backend, **kw)
+    return rank, world
+
+
+def average_(t):
+    """In-place mean over ranks (sum then divide, valid for every backend)."""
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        t.div_(dist.get_world_size())
+    return t
+
+
+def max_over_ranks(x, device):
+    """Maximum of a host float over ranks."""
+    if not (dist.is_initialized() and dist.get_world_size() > 1):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def token_seed(base, rank):
+    """Each rank draws its own micro-batches."""
+    return base + 1000 * rank

@@ -1,0 +1,59 @@
+"""Data-parallel host logic with two gloo ranks on the CPU: every rank ends a
+step with the same averaged LoRA gradient, hence the same AdamW update, and the
+step time reported is the maximum over ranks."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    from layer_streamed_qlora_nf4_b200 import dp
+    from oracle import model as om
+    r, w = dp.init("gloo", timeout_s=60)
+    assert (r, w) == (rank, world)
+    g = np.random.default_rng(dp.token_seed(5, rank))
+    grad = torch.from_numpy(g.standard_normal(1000))          # this rank's gradient
+    mine = grad.clone()
+    dp.average_(grad)
+    gathered = [torch.zeros_like(mine) for _ in range(world)]
+    torch.distributed.all_gather(gathered, mine)
+    p0 = np.linspace(-1, 1, 1000)
+    p1, _, _ = om.adamw_step(p0, grad.numpy(), np.zeros(1000), np.zeros(1000), 1)
+    t = dp.max_over_ranks(10.0 + rank, "cpu")
+    out[rank] = (grad.numpy().copy(), torch.stack(gathered).mean(0).numpy(), p1, t)
+    dp.barrier()
+    torch.distributed.destroy_process_group()
+
+
+def test_two_rank_gradient_average_and_timing():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    g0, mean0, p0, t0 = out[0]
+    g1, mean1, p1, t1 = out[1]
+    assert np.array_equal(g0, g1)                  # identical averaged gradient on both ranks
+    assert np.allclose(g0, mean0, atol=1e-15)      # equal to the mean of the ranks' gradients
+    assert np.array_equal(p0, p1)                  # hence identical parameters after AdamW
+    assert t0 == t1 == 11.0                        # max over ranks
