@@ -157,9 +157,13 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Barrier among a subset of warps (id != 0, count = threads taking part).
-__device__ __forceinline__ void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+// Transposing store of four 8x8 bf16 tiles: lane t holds, in r[j], elements
+// (row t/4, cols 2(t%4), 2(t%4)+1) of tile j; memory row i of tile j (16 bytes at
+// the address lane 8j+i supplies) receives column i of that tile.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, const uint32_t (&r)[4]) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05

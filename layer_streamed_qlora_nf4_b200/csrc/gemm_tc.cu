@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
   __shared__ __align__(8) uint64_t bar_epi;
+  __shared__ __align__(8) uint64_t bar_grp;   // the four operand/epilogue warps
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float lv_sh[16];
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&bar_acc), 1);
     mbar_init(smem_u32(&bar_epi), 1);
+    mbar_init(smem_u32(&bar_grp), 4);
     abort_sh = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -225,30 +227,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- operand stage
     const int tid = threadIdx.x - 128;  // 0..127
     const int nblk = p.w_cols / 64;
-    // absmax of this thread's rows for k-tile `it`, copied into a per-thread
-    // shared-memory slot ring two k-tiles ahead with cp.async (the global
-    // latency stays off the critical path): NF4_N needs one value per k-tile
-    // (row m0 + tid, block kt), NF4_T eight (rows kt*64 + 8bi .. +7, block
-    // (m0 + 8bj) / 64).
-    const int bi = tid & 7, bj = tid >> 3;
-    auto am_slot = [&](int it, int rr) -> float* { return am_ring + ((it % 3) * 128 + tid) * 8 + rr; };
+    // Bounded barrier among the four operand warps (an mbarrier of count 4, one
+    // arrival per warp), so that an abort in one warp cannot strand the others.
+    int grp_phase = 0;
+    auto grp_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_grp));
+      const bool r = mbar_wait_bounded(smem_u32(&bar_grp), (uint32_t)(grp_phase & 1), abort_flag,
+                                       p.dev_err, DEV_ERR_WAIT_GEMM);
+      ++grp_phase;
+      return __all_sync(0xFFFFFFFFu, r);
+    };
+    // absmax for k-tile `it` lands in slot it % 3 of a shared ring, copied with
+    // cp.async two k-tiles ahead (the global latency stays off the critical
+    // path).  NF4_N: thread tid fetches row m0 + tid, block kt.  NF4_T: the 128
+    // threads fetch the tile's 64 rows x 2 blocks together, thread tid taking
+    // row kt*64 + tid/2, block m0/64 + tid%2.
     auto issue_am = [&](int it) {
       if (it < n_main && (WMODE == W_NF4_N || WMODE == W_NF4_T)) {
         const int kt = kt_begin + it;
+        float* dst = am_ring + (it % 3) * 128 + tid;
         if (WMODE == W_NF4_N) {
           const int m = m0 + tid;
           const bool in = m < p.w_rows;
-          cp_async4(smem_u32(am_slot(it, 0)), p.absmax + (in ? (size_t)m * nblk + kt : 0),
-                    in ? 4u : 0u);
+          cp_async4(smem_u32(dst), p.absmax + (in ? (size_t)m * nblk + kt : 0), in ? 4u : 0u);
         } else {
-          const int mcol = m0 + 8 * bj;
-#pragma unroll
-          for (int rr = 0; rr < 8; ++rr) {
-            const int n = kt * kBK + 8 * bi + rr;
-            const bool in = n < p.w_rows && mcol < p.w_cols;
-            cp_async4(smem_u32(am_slot(it, rr)),
-                      p.absmax + (in ? (size_t)n * nblk + (mcol >> 6) : 0), in ? 4u : 0u);
-          }
+          const int n = kt * kBK + (tid >> 1);
+          const int bcol = (m0 >> 6) + (tid & 1);
+          const bool in = n < p.w_rows && bcol < nblk;
+          cp_async4(smem_u32(dst), p.absmax + (in ? (size_t)n * nblk + bcol : 0), in ? 4u : 0u);
         }
       }
       cp_async_commit();  // one group per k-tile (possibly empty) keeps the counting uniform
@@ -260,8 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
       uint8_t* wst = ws0 + (size_t)s * kWStageBytes;
+      cp_async_wait<1>();  // this thread's copies for k-tile `it` have landed
+      if (WMODE == W_NF4_T) {
+        // every thread's copies visible to all, and slot (it + 2) % 3 (read in
+        // iteration it - 1) free for reuse
+        if (!grp_sync()) { ok = false; break; }
+      }
       issue_am(it + 2);
-      cp_async_wait<2>();  // the group of k-tile `it` has landed
       if (it < n_main) {
         if (WMODE == W_BF16_N) {
           ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -271,9 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = it % CS;
           const uint32_t cph = (uint32_t)(it / CS) & 1u;
           const uint8_t* ring = rg0 + (size_t)c * p.ring_bytes;
-          const float* amc = am_slot(it, 0);
+          const float* amc = am_ring + (it % 3) * 128;
           if (WMODE == W_NF4_N) {
-            const float am = amc[0];
+            const float am = amc[tid];
             ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                    DEV_ERR_WAIT_GEMM) &&
                  mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -303,25 +315,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    DEV_ERR_WAIT_GEMM);
             ok = __all_sync(0xFFFFFFFFu, ok);
             if (ok) {
-              uint32_t w[8];
+              // The [64 n x 128 m] tile is 8 x 16 blocks of 8 x 8.  Warp w4 stores the
+              // blocks of n-blocks 2w4, 2w4+1, four consecutive m-blocks per
+              // stmatrix: lane t dequantises (n = 8nb + t/4, m = 32mq + 8j + 2(t%4) +
+              // {0,1}) for j = 0..3 - the fragment layout - from one 16-byte code
+              // read, and the transposing store puts 8 consecutive n of one m into
+              // each 16-byte chunk of the K-major tile.
+              const int w4 = warp - 4;
 #pragma unroll
-              for (int rr = 0; rr < 8; ++rr)
-                w[rr] = *reinterpret_cast<const uint32_t*>(ring + (8 * bi + rr) * 64 + 4 * bj);
+              for (int ii = 0; ii < 8; ++ii) {
+                const int nb = 2 * w4 + (ii >> 2);
+                const int mq = ii & 3;
+                const int n = nb * 8 + (lane >> 2);
+                const uint4 seg = *reinterpret_cast<const uint4*>(ring + n * 64 + mq * 16);
+                const float am = amc[n * 2 + (mq >> 1)];
+                const uint32_t words[4] = {seg.x, seg.y, seg.z, seg.w};
+                uint32_t regs[4];
 #pragma unroll
-              for (int cc = 0; cc < 8; ++cc) {
-                float v[8];
-#pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                  const uint32_t byte = (w[rr] >> (8 * (cc >> 1))) & 0xFFu;
-                  const uint32_t code = (cc & 1) ? (byte & 15u) : (byte >> 4);
-                  v[rr] = lv_sh[code] * amc[rr];
+                for (int j = 0; j < 4; ++j) {
+                  const uint32_t byte = (words[j] >> (8 * (lane & 3))) & 0xFFu;
+                  regs[j] = pack_bf16x2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
                 }
-                *reinterpret_cast<uint4*>(wst + sw128_offset(8 * bj + cc, bi)) =
-                    make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                               pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                const int m = mq * 32 + (lane >> 3) * 8 + (lane & 7);
+                stmatrix_x4_trans(smem_u32(wst + sw128_offset(m, nb)), regs);
               }
             }
           } else {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
+            const int bi = tid & 7, bj = tid >> 3;
             ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                    DEV_ERR_WAIT_GEMM) &&
                  mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -406,6 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue
     bool acc_ok = ok && mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
                                           DEV_ERR_WAIT_GEMM);
+    acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
+    // all four warps take the same branch: a failed warp has raised the abort flag
+    // before its arrival, and every warp reads the flag after the barrier
+    acc_ok = grp_sync() && acc_ok;
     acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
     if (acc_ok) {
       // Stage 32-token chunks of the [tokens x 128 features] tile in shared
@@ -432,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
           uint8_t* slot = dsm + (size_t)(q & 3) * (2 * sub_bytes);  // a 32-token chunk
           if (q >= 4 && leader) bulk_wait_read<3>();    // the store that used this slot has read it
-          named_barrier(1, 128);
+          if (!grp_sync()) break;
           if (res) {
             if (leader) {
               mbar_arrive_expect_tx(smem_u32(&bar_epi), (uint32_t)nsub * sub_bytes);
@@ -463,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          named_barrier(1, 128);
+          if (!grp_sync()) break;
           if (leader) {
             for (int sb = 0; sb < nsub; ++sb) {
               if (tb + 16 * sb >= p.T) break;
