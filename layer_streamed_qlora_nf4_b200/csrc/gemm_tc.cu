@@ -8,19 +8,23 @@
 // Its input gradient (part 3 and FAQ 4, W is re-read in backward):
 // Wop = deq(W)^T, act = dY, la = s*A^T, lb = v = dY B.
 //
-// Design for B200 (one CTA per SM, 256 threads, warp-specialised):
-//   warp 0   : TMA producer for the activation tile (128-byte swizzle) [and
-//              the bf16 weight tile in W_BF16_N mode]
-//   warp 1   : allocates TMEM, one elected thread issues tcgen05.mma
-//              (M = 128 output features x N = up to 256 tokens x K = 16),
-//              accumulators in TMEM (up to 2 x 256 fp32 columns)
-//   warp 2   : TMA producer for the packed NF4 codes (or the bf16 tile to be
-//              transposed) into a deep staging ring
-//   warps 4-7: operand stage - expand the staged codes to bf16 (level[code] *
-//              absmax in fp32, then round-to-nearest bf16) straight into the
-//              UMMA canonical K-major 128-byte-swizzle layout, fence the async
-//              proxy, arrive; they also write the LoRA slab; then the epilogue
-//              (tcgen05.ld of their TMEM lane quarter).
+// Design for B200 (one CTA per SM, 384 threads, warp-specialised):
+//   warp 0    : TMA producer for the activation tile (128-byte swizzle) [and
+//               the bf16 weight tile in W_BF16_N mode]
+//   warp 1    : allocates TMEM, one elected thread issues tcgen05.mma
+//               (M = 128 output features x N = up to 256 tokens x K = 16),
+//               accumulators in TMEM (up to 2 x 256 fp32 columns)
+//   warp 2    : TMA producer for the packed NF4 codes (or the bf16 tile to be
+//               transposed) into a deep staging ring
+//   warps 4-11: operand stage - expand the staged codes to bf16 (level[code] *
+//               absmax in fp32, then round-to-nearest bf16) straight into the
+//               UMMA canonical K-major 128-byte-swizzle layout, fence the async
+//               proxy, arrive; they also write the LoRA slab.  Two warps per
+//               SM sub-partition, because expanding the codes, not the tensor
+//               core, sets the pace of a k-tile.  Then the epilogue: each warp
+//               reads its TMEM lane quarter (32 features) for every other
+//               32-token chunk and writes it with its own TMA stores, with no
+//               barrier between warps.
 // The output tile is 128 features x all tokens of the CTA (up to 512), so each
 // weight element is dequantised once per token tile.  Small problems use a
 // fixed-order split over K with an fp32 partial buffer and a separate reduce:
@@ -39,14 +43,17 @@ __device__ int g_lsq_dev_status;
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // 4 control warps + 8 operand/epilogue warps
+constexpr int kOpWarps = 8;
+constexpr int kOpThreads = kOpWarps * 32;
 constexpr int kBM = 128;        // output features per CTA (UMMA M)
 constexpr int kBK = 64;         // contraction per stage = one SW128 atom = one NF4 block
 constexpr int kWStageBytes = kBM * kBK * 2;  // 16 KB bf16 operand tile
 constexpr int kMaxStages = 4;
 constexpr int kMaxRing = 8;
 constexpr uint32_t kSmemBudget = 227 * 1024;
-constexpr uint32_t kAmRingBytes = 3 * 128 * 8 * 4;  // absmax slots: 3 k-tiles x 128 threads x 8
+constexpr int kAmDepth = 8;  // absmax prefetch ring: 8 k-tiles x 256 floats
+constexpr uint32_t kAmRingBytes = kAmDepth * 256 * 4;
 
 struct KParams {
   int M, T, Kc;
@@ -88,8 +95,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_cfull[kMaxRing];
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
-  __shared__ __align__(8) uint64_t bar_epi;
-  __shared__ __align__(8) uint64_t bar_grp;   // the four operand/epilogue warps
+  __shared__ __align__(8) uint64_t bar_res[kOpWarps];  // per epilogue warp: residual tile landed
+  __shared__ __align__(8) uint64_t bar_grp;            // the operand warps
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ float lv_sh[16];
@@ -104,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* xs0 = dsm;
   uint8_t* ws0 = xs0 + (size_t)p.stages * xs_bytes;
   uint8_t* rg0 = ws0 + (size_t)p.stages * kWStageBytes;
-  float* am_ring = reinterpret_cast<float*>(rg0 + (size_t)p.ring_stages * p.ring_bytes);  // [3][128][8]
+  float* am_ring = reinterpret_cast<float*>(rg0 + (size_t)p.ring_stages * p.ring_bytes);  // [kAmDepth][256]
 
   const int m0 = blockIdx.x * kBM;
   const int t0 = blockIdx.y * BT;
@@ -118,16 +125,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 5);  // 1 producer + 4 operand warps
-      mbar_init(smem_u32(&bar_empty[s]), 1); // tcgen05.commit
+      mbar_init(smem_u32(&bar_full[s]), 1 + kOpWarps);  // producer + operand warps
+      mbar_init(smem_u32(&bar_empty[s]), 1);            // tcgen05.commit
     }
     for (int c = 0; c < CS; ++c) {
       mbar_init(smem_u32(&bar_cfull[c]), 1);
-      mbar_init(smem_u32(&bar_cempty[c]), 4);
+      mbar_init(smem_u32(&bar_cempty[c]), kOpWarps);
     }
     mbar_init(smem_u32(&bar_acc), 1);
-    mbar_init(smem_u32(&bar_epi), 1);
-    mbar_init(smem_u32(&bar_grp), 4);
+    for (int w = 0; w < kOpWarps; ++w) mbar_init(smem_u32(&bar_res[w]), 1);
+    mbar_init(smem_u32(&bar_grp), kOpWarps);
     abort_sh = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -140,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_act);
     tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_out);
   }
   tc_fence_before();
   __syncthreads();
@@ -224,11 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    // ---------------------------------------------------------- operand stage
-    const int tid = threadIdx.x - 128;  // 0..127
+    // ---------------------------------------------------------- operand stage (8 warps)
+    const int tid = threadIdx.x - 128;  // 0..255
+    const int ow = warp - 4;            // 0..7
     const int nblk = p.w_cols / 64;
-    // Bounded barrier among the four operand warps (an mbarrier of count 4, one
-    // arrival per warp), so that an abort in one warp cannot strand the others.
+    // Bounded barrier among the operand warps (an mbarrier with one arrival per
+    // warp), so that an abort in one warp cannot strand the others.
     int grp_phase = 0;
     auto grp_sync = [&]() -> bool {
       __syncwarp();
@@ -238,17 +247,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++grp_phase;
       return __all_sync(0xFFFFFFFFu, r);
     };
-    // absmax for k-tile `it` lands in slot it % 3 of a shared ring, copied with
-    // cp.async two k-tiles ahead (the global latency stays off the critical
-    // path).  NF4_N: thread tid fetches row m0 + tid, block kt.  NF4_T: the 128
-    // threads fetch the tile's 64 rows x 2 blocks together, thread tid taking
-    // row kt*64 + tid/2, block m0/64 + tid%2.
+    // absmax for k-tile `it` lands in slot it % kAmDepth of a shared ring, copied
+    // with cp.async kAmDepth - 1 k-tiles ahead.  NF4_N: thread tid fetches the
+    // absmax of its own row m0 + (tid & 127), block kt.  NF4_T: threads 0..127
+    // fetch the tile's 64 rows x 2 blocks together (row kt*64 + tid/2, block
+    // m0/64 + tid%2).
     auto issue_am = [&](int it) {
-      if (it < n_main && (WMODE == W_NF4_N || WMODE == W_NF4_T)) {
+      if (it < n_main && (WMODE == W_NF4_N || (WMODE == W_NF4_T && tid < 128))) {
         const int kt = kt_begin + it;
-        float* dst = am_ring + (it % 3) * 128 + tid;
+        float* dst = am_ring + (it % kAmDepth) * 256 + tid;
         if (WMODE == W_NF4_N) {
-          const int m = m0 + tid;
+          const int m = m0 + (tid & 127);
           const bool in = m < p.w_rows;
           cp_async4(smem_u32(dst), p.absmax + (in ? (size_t)m * nblk + kt : 0), in ? 4u : 0u);
         } else {
@@ -260,20 +269,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cp_async_commit();  // one group per k-tile (possibly empty) keeps the counting uniform
     };
-    issue_am(0);
-    issue_am(1);
+#pragma unroll 1
+    for (int i = 0; i < kAmDepth - 1; ++i) issue_am(i);
     bool ok = true;
     for (int it = 0; it < n_iter && ok; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
       uint8_t* wst = ws0 + (size_t)s * kWStageBytes;
-      cp_async_wait<1>();  // this thread's copies for k-tile `it` have landed
+      cp_async_wait<kAmDepth - 2>();  // this thread's copies for k-tile `it` have landed
       if (WMODE == W_NF4_T) {
-        // every thread's copies visible to all, and slot (it + 2) % 3 (read in
-        // iteration it - 1) free for reuse
+        // every thread's copies visible to all, and the slot of k-tile it - 1 free
         if (!grp_sync()) { ok = false; break; }
       }
-      issue_am(it + 2);
+      issue_am(it + kAmDepth - 1);
       if (it < n_main) {
         if (WMODE == W_BF16_N) {
           ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -283,20 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = it % CS;
           const uint32_t cph = (uint32_t)(it / CS) & 1u;
           const uint8_t* ring = rg0 + (size_t)c * p.ring_bytes;
-          const float* amc = am_ring + (it % 3) * 128;
-          if (WMODE == W_NF4_N) {
-            const float am = amc[tid];
-            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM) &&
-                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (ok) {
-              const uint4 c0 = *reinterpret_cast<const uint4*>(ring + tid * 32);
-              const uint4 c1 = *reinterpret_cast<const uint4*>(ring + tid * 32 + 16);
-              const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const float* amc = am_ring + (it % kAmDepth) * 256;
+          ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
+                                 DEV_ERR_WAIT_GEMM) &&
+               mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                                 DEV_ERR_WAIT_GEMM);
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          if (ok) {
+            if (WMODE == W_NF4_N) {
+              // thread: row r, half h of its 64 codes (chunks 4h .. 4h+3)
+              const int r = tid & 127, h = tid >> 7;
+              const float am = amc[tid];
+              const uint4 cw = *reinterpret_cast<const uint4*>(ring + r * 32 + h * 16);
+              const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
+              for (int q = 0; q < 4; ++q) {
                 const uint32_t w = words[q];
                 uint32_t o[4];
 #pragma unroll
@@ -304,29 +313,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const uint32_t byte = (w >> (8 * b)) & 0xFFu;
                   o[b] = pack_bf16x2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
                 }
-                *reinterpret_cast<uint4*>(wst + sw128_offset(tid, q)) =
+                *reinterpret_cast<uint4*>(wst + sw128_offset(r, 4 * h + q)) =
                     make_uint4(o[0], o[1], o[2], o[3]);
               }
-            }
-          } else if (WMODE == W_NF4_T) {
-            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM) &&
-                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (ok) {
-              // The [64 n x 128 m] tile is 8 x 16 blocks of 8 x 8.  Warp w4 stores the
-              // blocks of n-blocks 2w4, 2w4+1, four consecutive m-blocks per
-              // stmatrix: lane t dequantises (n = 8nb + t/4, m = 32mq + 8j + 2(t%4) +
-              // {0,1}) for j = 0..3 - the fragment layout - from one 16-byte code
-              // read, and the transposing store puts 8 consecutive n of one m into
-              // each 16-byte chunk of the K-major tile.
-              const int w4 = warp - 4;
+            } else if (WMODE == W_NF4_T) {
+              // The [64 n x 128 m] tile is 8 x 16 blocks of 8 x 8.  Warp ow stores the
+              // blocks of n-block ow, four consecutive m-blocks per stmatrix: lane t
+              // dequantises (n = 8 ow + t/4, m = 32 mq + 8j + 2(t%4) + {0,1}) for
+              // j = 0..3 - the fragment layout - from one 16-byte code read, and the
+              // transposing store puts 8 consecutive n of one m into each 16-byte
+              // chunk of the K-major tile.
+              const int nb = ow;
+              const int n = nb * 8 + (lane >> 2);
 #pragma unroll
-              for (int ii = 0; ii < 8; ++ii) {
-                const int nb = 2 * w4 + (ii >> 2);
-                const int mq = ii & 3;
-                const int n = nb * 8 + (lane >> 2);
+              for (int mq = 0; mq < 4; ++mq) {
                 const uint4 seg = *reinterpret_cast<const uint4*>(ring + n * 64 + mq * 16);
                 const float am = amc[n * 2 + (mq >> 1)];
                 const uint32_t words[4] = {seg.x, seg.y, seg.z, seg.w};
@@ -339,15 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m = mq * 32 + (lane >> 3) * 8 + (lane & 7);
                 stmatrix_x4_trans(smem_u32(wst + sw128_offset(m, nb)), regs);
               }
-            }
-          } else {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
-            const int bi = tid & 7, bj = tid >> 3;
-            ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM) &&
-                 mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
-                                   DEV_ERR_WAIT_GEMM);
-            ok = __all_sync(0xFFFFFFFFu, ok);
-            if (ok) {
+            } else if (tid < 128) {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
+              const int bi = tid & 7, bj = tid >> 3;
               uint4 rowv[8];
 #pragma unroll
               for (int rr = 0; rr < 8; ++rr)
@@ -366,8 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(o[0], o[1], o[2], o[3]);
               }
             }
-          }
-          if (ok) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bar_cempty[c]));
@@ -387,34 +378,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (part + 1 < p.n_parts && m0 >= p.part_end[part]) ++part;
             jofs = part * p.slab_w;
           }
-          {
-            const int m = m0 + tid;
-            for (int q = 0; q < wq; ++q) {
-              float v[8];
+          for (int i = tid; i < 128 * wq; i += kOpThreads) {
+            const int row = i & 127, q = i >> 7;
+            const int m = m0 + row;
+            float v[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const long long j = j0 + 8 * q + e;
-                v[e] = (m < p.M) ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + j * p.la_cs)
-                                 : 0.f;
-              }
-              *reinterpret_cast<uint4*>(wst + sw128_offset(tid, q)) =
-                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                             pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+            for (int e = 0; e < 8; ++e) {
+              const long long j = j0 + 8 * q + e;
+              v[e] = (m < p.M) ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + j * p.la_cs)
+                               : 0.f;
             }
+            *reinterpret_cast<uint4*>(wst + sw128_offset(row, q)) =
+                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
           }
           uint8_t* xst = xs0 + (size_t)s * xs_bytes;
-          for (int t = tid; t < BT; t += 128) {
+          for (int i = tid; i < BT * wq; i += kOpThreads) {
+            const int t = i % BT, q = i / BT;
             const int tg = t0 + t;
-            for (int q = 0; q < wq; ++q) {
-              float v[8];
+            float v[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + jofs + j0 + 8 * q + e)
-                                  : 0.f;
-              *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
-                  make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                             pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-            }
+            for (int e = 0; e < 8; ++e)
+              v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + jofs + j0 + 8 * q + e)
+                                : 0.f;
+            *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
+                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -423,84 +412,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && lane == 0) mbar_arrive(smem_u32(&bar_full[s]));
     }
 
-    // ---------------------------------------------------------- epilogue
+    // ---------------------------------------------------------- epilogue (per warp)
+    // Each warp owns a 32-feature quarter of the tile (its TMEM lanes) and every
+    // other 32-token chunk; it stages a chunk in two private shared-memory slots
+    // and writes it with TMA stores of [16 tokens x 32 features] boxes, so no
+    // warp waits for another.  Residual tiles arrive by TMA into the slot and are
+    // added in place.
     bool acc_ok = ok && mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
                                           DEV_ERR_WAIT_GEMM);
-    acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
-    // all four warps take the same branch: a failed warp has raised the abort flag
-    // before its arrival, and every warp reads the flag after the barrier
-    acc_ok = grp_sync() && acc_ok;
     acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
     if (acc_ok) {
-      // Stage 32-token chunks of the [tokens x 128 features] tile in shared
-      // memory (the drained pipeline buffers: 4 chunk slots of 2 x 16 rows x 128
-      // features, i.e. 16 KB for fp32 and 8 KB for bf16 outputs) and write
-      // them with TMA stores of 16-row boxes, so each CTA writes only its own
-      // token range.  Residual tiles arrive by TMA into the slot and are added
-      // in place.
       tc_fence_after();
-      const int qtr = warp & 3;
-      const int row = qtr * 32 + lane;   // feature within the tile
+      const int qtr = warp & 3;          // TMEM lane quarter = features 32 qtr .. +31
+      const int cgrp = ow >> 2;          // chunks q with q % 2 == cgrp
       const uint32_t tbase = tmem + ((uint32_t)(qtr * 32) << 16);
-      const bool leader = (warp == 4 && lane == 0);
       const bool partial = p.splits > 1;
       const bool f32 = partial || p.out_f32;
       const int es = f32 ? 4 : 2;
       const bool res = !partial && p.residual != nullptr;
-      const uint32_t sub_bytes = 16u * 128u * (uint32_t)es;
-      int q = 0, nres = 0;
-      for (int a = 0; a < p.nacc; ++a) {
+      const uint32_t sub_bytes = 16u * 32u * (uint32_t)es;   // one [16 x 32] box
+      uint8_t* myslots = dsm + (size_t)ow * 8192;            // 2 slots of <= 4 KB
+      const int mcol = m0 + qtr * 32;
+      int q = 0, nq = 0, nres = 0;
+      for (int a = 0; a < p.nacc && acc_ok; ++a) {
         for (int c0 = 0; c0 < p.bn; c0 += 32, ++q) {
           const int tb = t0 + a * p.bn + c0;
-          if (tb >= p.T) break;                         // uniform across the 128 threads
+          if (tb >= p.T) break;
+          if ((q & 1) != cgrp) continue;
           const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
-          uint8_t* slot = dsm + (size_t)(q & 3) * (2 * sub_bytes);  // a 32-token chunk
-          if (q >= 4 && leader) bulk_wait_read<3>();    // the store that used this slot has read it
-          if (!grp_sync()) break;
+          uint8_t* slot = myslots + (nq & 1) * (2 * sub_bytes);
+          if (nq >= 2 && lane == 0) bulk_wait_read<1>();  // the store that used this slot has read it
+          __syncwarp();
           if (res) {
-            if (leader) {
-              mbar_arrive_expect_tx(smem_u32(&bar_epi), (uint32_t)nsub * sub_bytes);
+            if (lane == 0) {
+              mbar_arrive_expect_tx(smem_u32(&bar_res[ow]), (uint32_t)nsub * sub_bytes);
               for (int sb = 0; sb < nsub; ++sb)
-                tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, smem_u32(&bar_epi), m0,
+                tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, smem_u32(&bar_res[ow]), mcol,
                             tb + 16 * sb);
             }
-            acc_ok = mbar_wait_bounded(smem_u32(&bar_epi), (uint32_t)(nres & 1), abort_flag,
+            acc_ok = mbar_wait_bounded(smem_u32(&bar_res[ow]), (uint32_t)(nres & 1), abort_flag,
                                        p.dev_err, DEV_ERR_WAIT_GEMM);
+            acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
             ++nres;
+            if (!acc_ok) break;
           }
-          uint32_t r[2][16];
-          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, r[0]);
-          if (nsub == 2) tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0 + 16, r[1]);
+          uint32_t rg[2][16];
+          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, rg[0]);
+          if (nsub == 2) tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0 + 16, rg[1]);
           tmem_ld_wait();
           for (int sb = 0; sb < nsub; ++sb) {
             uint8_t* base = slot + sb * sub_bytes;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              float v = __uint_as_float(r[sb][j]);
+              float v = __uint_as_float(rg[sb][j]);
               if (f32) {
-                *reinterpret_cast<float*>(base + (j * 128 + row) * 4) = v;
+                *reinterpret_cast<float*>(base + (j * 32 + lane) * 4) = v;
               } else {
-                uint16_t* d = reinterpret_cast<uint16_t*>(base + (j * 128 + row) * 2);
+                uint16_t* d = reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2);
                 if (res) v += bf16_bits_to_float(*d);
                 *d = float_to_bf16_bits(v);
               }
             }
           }
           fence_proxy_async_smem();
-          if (!grp_sync()) break;
-          if (leader) {
+          __syncwarp();
+          if (lane == 0) {
             for (int sb = 0; sb < nsub; ++sb) {
               if (tb + 16 * sb >= p.T) break;
               if (partial)
-                tma_store_3d(&tm_out, smem_u32(slot + sb * sub_bytes), m0, tb + 16 * sb, split);
+                tma_store_3d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb, split);
               else
-                tma_store_2d(&tm_out, smem_u32(slot + sb * sub_bytes), m0, tb + 16 * sb);
+                tma_store_2d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb);
             }
             bulk_commit();
           }
+          __syncwarp();
+          ++nq;
         }
       }
-      if (leader) bulk_wait_all();
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   }
 
@@ -644,7 +635,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
     if (!enc) return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     cuuint64_t dims[3] = {(cuuint64_t)d.M, (cuuint64_t)d.T, (cuuint64_t)pl.splits};
     cuuint64_t strides[2] = {(cuuint64_t)d.M * 4, (cuuint64_t)d.M * (cuuint64_t)d.T * 4};
-    cuuint32_t box[3] = {128, 16, 1};
+    cuuint32_t box[3] = {32, 16, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(&tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, partial, dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -653,14 +644,14 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
       return set_error(LSQ_ERR_CUDA, "cuTensorMapEncodeTiled (partials) failed (%d)", (int)r);
   } else if (d.out_f32) {
     LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d.out, (uint64_t)d.M,
-                      (uint64_t)d.T, (uint64_t)d.ldo, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+                      (uint64_t)d.T, (uint64_t)d.ldo, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
     LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.out, (uint64_t)d.M,
-                      (uint64_t)d.T, (uint64_t)d.ldo, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+                      (uint64_t)d.T, (uint64_t)d.ldo, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   }
   if (d.residual && !partial)
     LSQ_TRY(make_tmap(&tm_res, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.residual, (uint64_t)d.M,
-                      (uint64_t)d.T, (uint64_t)d.ldr, 128, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+                      (uint64_t)d.T, (uint64_t)d.ldr, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   else
     tm_res = tm_out;  // unused
   KParams p{};
