@@ -26,6 +26,20 @@ so every constant below is a stated reading:
   * Packing: byte j holds element 2j in its high nibble and element 2j+1 in its
     low nibble.
   * Dequantisation: w~ = fl32(c[code] * absmax), a single fp32 multiply.
+
+Optional second stage (double quantisation of the absmax).  The pages give only
+sizes for it: a 3.60 GB store for 32 layers and 113 MB layer buffers (article
+"架构解读：layer streaming 如何塞进 4 GB" and the "工作原理" list), which is what an
+8-bit absmax with one fp32 scale per 256 blocks gives for Llama-3.1-8B shapes
+(fp32 absmax would give 3.93 GB).  The scheme itself is not printed, so it is a
+reading, the plainest linear one:
+
+  * Groups: runs of ABSMAX_GROUP = 256 consecutive absmax values of one weight
+    matrix (block order, row-major); the last run may be shorter.
+  * Scale: s = fl32(max(run) / 255) (IEEE fp32 division); q = rint(fl32(a / s))
+    rounded half to even, at most 255; a run whose max is 0 gets s = 0, q = 0.
+  * The NF4 codes are still chosen with the fp32 absmax; dequantisation uses
+    a~ = fl32(q * s) and then w~ = fl32(c[code] * a~).
 """
 
 from statistics import NormalDist
@@ -33,6 +47,7 @@ from statistics import NormalDist
 import numpy as np
 
 BLOCK = 64
+ABSMAX_GROUP = 256
 DELTA = ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0)) / 2.0
 
 
@@ -104,3 +119,34 @@ def dequantize(codes, absmax, N, K, block=BLOCK):
     idx = unpack(codes, N * K).reshape(-1, block)
     am = np.asarray(absmax, dtype=np.float32)[:, None]
     return (c[idx] * am).astype(np.float32).reshape(N, K)
+
+
+def quantize_absmax8(absmax, group=ABSMAX_GROUP):
+    """fp32 absmax [nb] -> (q uint8 [nb], scale fp32 [ceil(nb / group)])."""
+    a = np.asarray(absmax, dtype=np.float32).reshape(-1)
+    assert np.all(np.isfinite(a)) and np.all(a >= 0), "absmax values are finite and >= 0"
+    ng = (a.size + group - 1) // group
+    q = np.zeros(a.size, dtype=np.uint8)
+    scale = np.zeros(ng, dtype=np.float32)
+    for g in range(ng):
+        run = a[g * group:(g + 1) * group]
+        mx = np.float32(run.max())
+        if mx == 0:
+            continue
+        s = np.float32(mx / np.float32(255.0))
+        scale[g] = s
+        v = (run / s).astype(np.float32)
+        q[g * group:(g + 1) * group] = np.minimum(np.rint(v), 255).astype(np.uint8)
+    return q, scale
+
+
+def dequantize_absmax8(q, scale, group=ABSMAX_GROUP):
+    """(q, scale) -> fp32 a~ [nb], a~ = fl32(q * scale[run])."""
+    q = np.asarray(q, dtype=np.uint8).reshape(-1)
+    s = np.asarray(scale, dtype=np.float32)[np.arange(q.size) // group]
+    return (q.astype(np.float32) * s).astype(np.float32)
+
+
+def dequantize_dq(codes, q, scale, N, K, block=BLOCK, group=ABSMAX_GROUP):
+    """NF4 with a double-quantised absmax -> fp32 W~ [N, K]."""
+    return dequantize(codes, dequantize_absmax8(q, scale, group), N, K, block)

@@ -159,3 +159,69 @@ def test_dequantize_is_level_times_absmax_and_error_bound():
     gap = float(np.max(np.diff(C.astype(np.float64)))) / 2
     err = np.abs(W.reshape(-1, 64).astype(np.float64) - Wt.reshape(-1, 64))
     assert np.all(err <= absmax[:, None] * (gap + 1e-6))
+
+
+# ----------------------------------------------------------------- absmax, 8 bit
+
+
+def test_absmax8_exact_on_its_own_grid():
+    # a run whose values are j * 2^-10 (max 255 * 2^-10): s = 2^-10 exactly, q = j
+    j = np.array(list(range(256)), dtype=np.float32)
+    a = (j * np.float32(2.0 ** -10)).astype(np.float32)
+    q, s = nf4.quantize_absmax8(a)
+    assert s.tolist() == [2.0 ** -10]
+    assert np.array_equal(q, j.astype(np.uint8))
+    assert np.array_equal(nf4.dequantize_absmax8(q, s), a)
+
+
+def test_absmax8_nearest_step_and_bound():
+    rng = np.random.default_rng(5)
+    a = np.abs(rng.normal(0.0, 0.06, 256 * 7 + 100)).astype(np.float32)   # ragged last run
+    q, s = nf4.quantize_absmax8(a)
+    assert s.size == 8 and q.dtype == np.uint8
+    idx = np.arange(a.size) // 256
+    for g in range(8):
+        run = a[idx == g]
+        assert q[idx == g][np.argmax(run)] == 255, "each run's max takes the top code"
+        # s is max/255 to within half an fp32 ulp
+        assert abs(float(s[g]) - float(run.max()) / 255.0) <= 2.0 ** -24 * float(s[g])
+    # q is the nearest integer to a / s (checked in fp64), so |a~ - a| <= s/2 (+ rounding)
+    sd = s[idx].astype(np.float64)
+    ratio = a.astype(np.float64) / sd
+    assert np.all(np.abs(q - ratio) <= 0.5 + 1e-5)
+    back = nf4.dequantize_absmax8(q, s).astype(np.float64)
+    assert np.all(np.abs(back - a) <= 0.5 * sd * (1 + 1e-5) + 2.0 ** -23 * a)
+    # order is kept inside a run
+    for g in range(8):
+        m = idx == g
+        o = np.argsort(a[m], kind="stable")
+        assert np.all(np.diff(q[m][o].astype(int)) >= 0)
+
+
+def test_absmax8_zero_run_and_tie_to_even():
+    a = np.zeros(300, dtype=np.float32)
+    a[256:] = np.float32(2.0 ** -10) * np.float32(255.0)
+    a[257] = np.float32(2.5 * 2.0 ** -10)    # exactly q = 2.5 -> even 2
+    a[258] = np.float32(3.5 * 2.0 ** -10)    # exactly q = 3.5 -> even 4
+    q, s = nf4.quantize_absmax8(a)
+    assert s[0] == 0 and np.all(q[:256] == 0)
+    assert np.all(nf4.dequantize_absmax8(q, s)[:256] == 0)
+    assert s[1] == np.float32(2.0 ** -10) and q[257] == 2 and q[258] == 4
+
+
+def test_dequantize_dq_is_codes_times_rounded_absmax():
+    rng = np.random.default_rng(6)
+    N, K = 8, 256 * 4
+    W = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    codes, am = nf4.quantize(W)
+    q, s = nf4.quantize_absmax8(am)
+    got = nf4.dequantize_dq(codes, q, s, N, K)
+    a2 = nf4.dequantize_absmax8(q, s)
+    # brute force per element: level[code] * a~ of its block
+    idx = nf4.unpack(codes, N * K)
+    want = np.array([np.float32(C[idx[i]] * a2[i // 64]) for i in range(N * K)], np.float32)
+    assert np.array_equal(got.reshape(-1), want)
+    # and the double-quantised weight stays within half an absmax step of the fp32 one
+    ref = nf4.dequantize(codes, am, N, K)
+    step = np.repeat(s[np.arange(am.size) // 256], 64).reshape(N, K)
+    assert np.all(np.abs(got - ref) <= 0.5 * step * (1 + 1e-5) + 2.0 ** -22 * np.abs(ref))
