@@ -37,6 +37,13 @@ BATCH, SEQ = 1, 512
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 
 
+def workload_name(absmax_bits):
+    if absmax_bits == 8:
+        return WORKLOAD.replace("fp32 absmax", "8-bit double-quantised absmax, one fp32 scale "
+                                "per 256 blocks")
+    return WORKLOAD
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -45,6 +52,10 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (for quick runs)")
+    ap.add_argument("--absmax-bits", type=int, choices=(32, 8), default=32,
+                    help="32: fp32 absmax per NF4 block (the default workload); 8: the absmax "
+                         "double-quantised to 8 bits with one fp32 scale per 256 blocks, the "
+                         "pages' 113 MB layers / 3.60 GB store")
     ap.add_argument("--case", choices=("step", "layer", "gemm"), default="step",
                     help="step: the streamed 32-layer SFT step (default); layer: one resident "
                          "8B-shaped layer forward + recomputing backward; gemm: one fused NF4 "
@@ -235,7 +246,7 @@ def run_ours(args):
     from layer_streamed_qlora_nf4_b200 import lib as L
     from layer_streamed_qlora_nf4_b200 import synth
     L.load()
-    cfg = synth.LLAMA8B
+    cfg = dict(synth.LLAMA8B, absmax_bits=args.absmax_bits)
     st = build_stack(L, cfg, rank)
     lay = st["lay"]
     handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
@@ -365,7 +376,8 @@ def run_ours(args):
                     warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak",
                     vs_baseline=None, dtype="bf16", data="synthetic (seeded random weights and "
                     "uniform token ids at the 8B shapes)",
-                    config=dict(workload=WORKLOAD, global_batch=world * BATCH, seq_len=SEQ,
+                    config=dict(workload=workload_name(args.absmax_bits),
+                                global_batch=world * BATCH, seq_len=SEQ,
                                 parallelism="dp%d" % world,
                                 l2="inputs larger than L2: %.2f GB of layer bytes stream per step"
                                 % (cps * lay.bytes / 1e9)),
@@ -384,7 +396,7 @@ def run_layer(args):
     from layer_streamed_qlora_nf4_b200 import lib as L
     from layer_streamed_qlora_nf4_b200 import pack, synth
     L.load()
-    cfg = synth.LLAMA8B
+    cfg = dict(synth.LLAMA8B, absmax_bits=args.absmax_bits)
     lay = L.lsq_layer_layout_get(cfg)
     g = torch.Generator(device="cuda").manual_seed(3)
     shapes = synth.proj_shapes(cfg)

@@ -85,6 +85,26 @@ int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block, uint8_t* c
 int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
                    int32_t block, float* W_out, void* stream);
 
+/* nf4_absmax_quantize8 - second-stage (double) quantisation of an NF4 absmax
+ * array to 8 bits.  The pages give the stored sizes only (a 3.60 GB store for
+ * 32 Llama-3.1-8B layers, 113 MB layer buffers: article "架构解读：layer streaming
+ * 如何塞进 4 GB"), which an 8-bit absmax with one fp32 scale per 256 blocks
+ * reproduces; the linear scheme below is this library's reading.
+ *   absmax    device fp32 [n_blocks], values finite and >= 0 (nf4_quantize's output).
+ *   q         device uint8 [n_blocks], 16-byte aligned.
+ *   scale     device fp32 [ceil(n_blocks / 256)].
+ * For each run of 256 consecutive values (the last may be shorter):
+ * scale = fl32(max / 255), q = rint(fl32(a / scale)) half to even, at most 255;
+ * a run of zeros gets scale 0, q 0.  Asynchronous, deterministic.  The NF4 codes
+ * stay those chosen with the fp32 absmax. */
+int nf4_absmax_quantize8(const float* absmax, int64_t n_blocks, uint8_t* q, float* scale,
+                         void* stream);
+
+/* nf4_dequantize_dq - w~ = fl32(level[code] * fl32(q[b] * scale[b / 256])) into
+ * fp32 W_out [N, K], b = element / 64.  Constraints of nf4_quantize; asynchronous. */
+int nf4_dequantize_dq(const uint8_t* codes, const uint8_t* q, const float* scale, int64_t N,
+                      int64_t K, int32_t block, float* W_out, void* stream);
+
 /* ------------------------------------------------------- NF4 + LoRA linear */
 
 /* Workspace bytes needed by nf4_lora_linear_fwd/bwd for these sizes. */
@@ -137,19 +157,26 @@ typedef struct lsq_cfg {
   float lora_alpha;    /* s = alpha / r */
   float rope_theta;    /* rotate-half RoPE base */
   float rms_eps;       /* RMSNorm epsilon */
-  int32_t reserved;    /* must be 0 */
+  int32_t absmax_bits; /* 0 or 32: fp32 absmax per block; 8: 8-bit absmax with one
+                          fp32 scale per 256 blocks (nf4_absmax_quantize8) */
 } lsq_cfg;
 
 /* Byte layout of one layer's blob (the unit that is streamed).  Projection
  * order q, k, v, o, gate, up, down.  All codes come first, contiguous, so q|k|v
- * and gate|up each form one stacked NF4 matrix; then all absmax arrays; then
- * the two RMSNorm gains (bf16 [D]).  Every section starts 256-byte aligned. */
+ * and gate|up each form one stacked NF4 matrix; then all absmax arrays (fp32,
+ * or uint8 with absmax_bits = 8, then all their fp32 scale arrays); then the
+ * two RMSNorm gains (bf16 [D]).  Every section starts 256-byte aligned.  For
+ * Llama-3.1-8B shapes a layer is 122,699,776 bytes with fp32 absmax and
+ * 112,529,408 bytes (the pages' 113 MB; 3.60 GB for 32 layers) with 8-bit. */
 typedef struct lsq_layer_layout {
   uint64_t codes_off[7];
-  uint64_t absmax_off[7];
+  uint64_t absmax_off[7];   /* fp32 [N*K/64], or uint8 [N*K/64] with absmax_bits 8 */
   uint64_t g1_off, g2_off;
   int64_t rows[7], cols[7]; /* N, K of each projection */
   uint64_t bytes;           /* total blob size (multiple of 256) */
+  uint64_t scale_off[7];    /* absmax_bits 8: fp32 [N*K/64/256]; else 0 */
+  int32_t absmax_bits;      /* 32 or 8 */
+  int32_t pad;
 } lsq_layer_layout;
 
 /* Fills *out for cfg.  Host only.  LSQ_ERR_SHAPE unless D, F, H*d, Hkv*d are

@@ -53,7 +53,7 @@ constexpr int kMaxStages = 4;
 constexpr int kMaxRing = 8;
 constexpr uint32_t kSmemBudget = 227 * 1024;
 constexpr int kAmDepth = 8;  // absmax prefetch ring: 8 k-tiles x 256 floats
-constexpr uint32_t kAmRingBytes = kAmDepth * 256 * 4;
+constexpr uint32_t kAmRingBytes = kAmDepth * 256 * 4 * 2;  // absmax (or 8-bit words) + scales
 
 struct KParams {
   int M, T, Kc;
@@ -61,6 +61,8 @@ struct KParams {
   int kt_total, kt_per_split, splits;
   uint32_t ring_bytes, alloc_cols;
   const float* absmax;
+  const uint8_t* am_q;  // 8-bit absmax mode when non-null
+  const float* am_s;
   int w_rows, w_cols;
   int slab_w, jofs_by_part, n_parts;
   const float* la;
@@ -112,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ws0 = xs0 + (size_t)p.stages * xs_bytes;
   uint8_t* rg0 = ws0 + (size_t)p.stages * kWStageBytes;
   float* am_ring = reinterpret_cast<float*>(rg0 + (size_t)p.ring_stages * p.ring_bytes);  // [kAmDepth][256]
+  float* sc_ring = am_ring + kAmDepth * 256;  // 8-bit mode: the scale of each fetched absmax
 
   const int m0 = blockIdx.x * kBM;
   const int t0 = blockIdx.y * BT;
@@ -251,20 +254,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     // with cp.async kAmDepth - 1 k-tiles ahead.  NF4_N: thread tid fetches the
     // absmax of its own row m0 + (tid & 127), block kt.  NF4_T: threads 0..127
     // fetch the tile's 64 rows x 2 blocks together (row kt*64 + tid/2, block
-    // m0/64 + tid%2).
+    // m0/64 + tid%2).  With an 8-bit absmax the slot receives the aligned 32-bit
+    // word holding the code, and the scale ring the run's fp32 scale; the user
+    // of the value extracts the byte and multiplies (absmax_value below).
+    const bool q8 = p.am_q != nullptr;
     auto issue_am = [&](int it) {
       if (it < n_main && (WMODE == W_NF4_N || (WMODE == W_NF4_T && tid < 128))) {
         const int kt = kt_begin + it;
         float* dst = am_ring + (it % kAmDepth) * 256 + tid;
+        size_t b = 0;
+        bool in;
         if (WMODE == W_NF4_N) {
           const int m = m0 + (tid & 127);
-          const bool in = m < p.w_rows;
-          cp_async4(smem_u32(dst), p.absmax + (in ? (size_t)m * nblk + kt : 0), in ? 4u : 0u);
+          in = m < p.w_rows;
+          b = in ? (size_t)m * nblk + kt : 0;
         } else {
           const int n = kt * kBK + (tid >> 1);
           const int bcol = (m0 >> 6) + (tid & 1);
-          const bool in = n < p.w_rows && bcol < nblk;
-          cp_async4(smem_u32(dst), p.absmax + (in ? (size_t)n * nblk + bcol : 0), in ? 4u : 0u);
+          in = n < p.w_rows && bcol < nblk;
+          b = in ? (size_t)n * nblk + bcol : 0;
+        }
+        if (q8) {
+          cp_async4(smem_u32(dst), p.am_q + (b & ~size_t(3)), in ? 4u : 0u);
+          cp_async4(smem_u32(sc_ring + (it % kAmDepth) * 256 + tid), p.am_s + (b >> 8),
+                    in ? 4u : 0u);
+        } else {
+          cp_async4(smem_u32(dst), p.absmax + b, in ? 4u : 0u);
         }
       }
       cp_async_commit();  // one group per k-tile (possibly empty) keeps the counting uniform
@@ -292,6 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t cph = (uint32_t)(it / CS) & 1u;
           const uint8_t* ring = rg0 + (size_t)c * p.ring_bytes;
           const float* amc = am_ring + (it % kAmDepth) * 256;
+          const float* scc = sc_ring + (it % kAmDepth) * 256;
+          // absmax of ring entry e, fetched for block b of W
+          auto absmax_value = [&](int e, size_t b) -> float {
+            if (!q8) return amc[e];
+            const uint32_t w = __float_as_uint(amc[e]);
+            return (float)((w >> (8u * (uint32_t)(b & 3))) & 0xFFu) * scc[e];
+          };
           ok = mbar_wait_bounded(smem_u32(&bar_cfull[c]), cph, abort_flag, p.dev_err,
                                  DEV_ERR_WAIT_GEMM) &&
                mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
@@ -301,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (WMODE == W_NF4_N) {
               // thread: row r, half h of its 64 codes (chunks 4h .. 4h+3)
               const int r = tid & 127, h = tid >> 7;
-              const float am = amc[tid];
+              const int kt = kt_begin + it;
+              const float am = absmax_value(tid, (size_t)(m0 + r) * nblk + kt);
               const uint4 cw = *reinterpret_cast<const uint4*>(ring + r * 32 + h * 16);
               const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
@@ -328,7 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int mq = 0; mq < 4; ++mq) {
                 const uint4 seg = *reinterpret_cast<const uint4*>(ring + n * 64 + mq * 16);
-                const float am = amc[n * 2 + (mq >> 1)];
+                const float am = absmax_value(
+                    n * 2 + (mq >> 1),
+                    (size_t)((kt_begin + it) * kBK + n) * nblk + (m0 >> 6) + (mq >> 1));
                 const uint32_t words[4] = {seg.x, seg.y, seg.z, seg.w};
                 uint32_t regs[4];
 #pragma unroll
@@ -668,6 +693,8 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   p.ring_bytes = pl.ring_bytes;
   p.alloc_cols = pl.alloc_cols;
   p.absmax = d.absmax;
+  p.am_q = d.absmax_q;
+  p.am_s = d.absmax_s;
   p.w_rows = (int)d.w_rows;
   p.w_cols = (int)d.w_cols;
   p.slab_w = d.slab_w;
@@ -728,7 +755,7 @@ size_t gemm_workspace_bytes(const GemmDesc& d) {
 int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (d.M <= 0 || d.T <= 0 || d.Kc <= 0) return set_error(LSQ_ERR_SHAPE, "gemm: empty problem");
   if (!d.w || !d.act || !d.out) return set_error(LSQ_ERR_INVALID, "gemm: null operand");
-  if ((d.wmode == W_NF4_N || d.wmode == W_NF4_T) && !d.absmax)
+  if ((d.wmode == W_NF4_N || d.wmode == W_NF4_T) && !d.absmax && !(d.absmax_q && d.absmax_s))
     return set_error(LSQ_ERR_INVALID, "gemm: null absmax");
   if (d.w_cols % 64 != 0 && (d.wmode == W_NF4_N || d.wmode == W_NF4_T))
     return set_error(LSQ_ERR_SHAPE, "gemm: NF4 weight columns must be a multiple of 64");

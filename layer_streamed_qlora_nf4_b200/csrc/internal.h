@@ -69,7 +69,9 @@ struct GemmDesc {
   int wmode = W_NF4_N;
   int64_t M = 0, T = 0, Kc = 0;
   const void* w = nullptr;          // NF4 codes or bf16 weight
-  const float* absmax = nullptr;    // NF4 only
+  const float* absmax = nullptr;    // NF4 only: fp32 absmax per 64-block, or
+  const uint8_t* absmax_q = nullptr;  // 8-bit absmax (double quantised) with
+  const float* absmax_s = nullptr;    // one fp32 scale per 256 blocks
   int64_t w_rows = 0, w_cols = 0;   // storage shape of W
   const uint16_t* act = nullptr;    // bf16 [T, act_ld], contraction over the first Kc columns
   int64_t act_ld = 0;
@@ -162,6 +164,7 @@ struct LayerShapes {
   int64_t D, F, qd, kvd, qkv_n, gu_n;
   int H, Hkv, hd, r;
   float s;
+  int absmax_bits;  // 32 or 8
 };
 int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);

@@ -13,7 +13,8 @@ namespace lsq {
 
 int layer_shapes(const lsq_cfg* cfg, LayerShapes* o) {
   if (!cfg) return set_error(LSQ_ERR_INVALID, "null config");
-  if (cfg->reserved != 0) return set_error(LSQ_ERR_INVALID, "cfg.reserved must be 0");
+  if (cfg->absmax_bits != 0 && cfg->absmax_bits != 32 && cfg->absmax_bits != 8)
+    return set_error(LSQ_ERR_INVALID, "cfg.absmax_bits must be 0, 32 or 8");
   if (cfg->block != 64) return set_error(LSQ_ERR_SHAPE, "cfg.block must be 64");
   if (cfg->head_dim != 64 && cfg->head_dim != 128)
     return set_error(LSQ_ERR_SHAPE, "cfg.head_dim must be 64 or 128");
@@ -40,14 +41,24 @@ int layer_shapes(const lsq_cfg* cfg, LayerShapes* o) {
   o->hd = cfg->head_dim;
   o->r = cfg->lora_r;
   o->s = cfg->lora_alpha / (float)cfg->lora_r;
+  // With 8-bit absmax every projection has a multiple of 256 blocks (its rows
+  // and columns are multiples of 128), so a scale run never straddles two
+  // projections and the stacked q|k|v and gate|up matrices index one array.
+  o->absmax_bits = cfg->absmax_bits == 8 ? 8 : 32;
   return LSQ_OK;
 }
 
 namespace {
 
+struct AbsmaxRef {  // fp32 absmax, or 8-bit absmax with its run scales
+  const float* f32 = nullptr;
+  const uint8_t* q = nullptr;
+  const float* s = nullptr;
+};
+
 struct Views {  // pointers into one layer blob / one LoRA block
   const uint8_t* codes[7];
-  const float* absmax[7];
+  AbsmaxRef absmax[7];
   const uint16_t* g1;
   const uint16_t* g2;
   const float *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_d, *B_d;
@@ -64,9 +75,19 @@ void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) 
     off += (uint64_t)rows[p] * cols[p] / 2;
   }
   off = (off + 255) & ~uint64_t(255);
+  L->absmax_bits = s.absmax_bits;
+  L->pad = 0;
   for (int p = 0; p < 7; ++p) {
     L->absmax_off[p] = off;
-    off += (uint64_t)rows[p] * cols[p] / 64 * 4;
+    off += (uint64_t)rows[p] * cols[p] / 64 * (s.absmax_bits == 8 ? 1 : 4);
+  }
+  off = (off + 255) & ~uint64_t(255);
+  for (int p = 0; p < 7; ++p) {
+    L->scale_off[p] = 0;
+    if (s.absmax_bits == 8) {
+      L->scale_off[p] = off;
+      off += ((uint64_t)rows[p] * cols[p] / 64 + 255) / 256 * 4;
+    }
   }
   off = (off + 255) & ~uint64_t(255);
   L->g1_off = off;
@@ -105,7 +126,12 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
   const uint8_t* b = static_cast<const uint8_t*>(blob);
   for (int p = 0; p < 7; ++p) {
     v.codes[p] = b + L.codes_off[p];
-    v.absmax[p] = reinterpret_cast<const float*>(b + L.absmax_off[p]);
+    if (s.absmax_bits == 8) {
+      v.absmax[p].q = b + L.absmax_off[p];
+      v.absmax[p].s = reinterpret_cast<const float*>(b + L.scale_off[p]);
+    } else {
+      v.absmax[p].f32 = reinterpret_cast<const float*>(b + L.absmax_off[p]);
+    }
   }
   v.g1 = reinterpret_cast<const uint16_t*>(b + L.g1_off);
   v.g2 = reinterpret_cast<const uint16_t*>(b + L.g2_off);
@@ -132,7 +158,7 @@ struct Buffers {
   size_t gemm_bytes;
 };
 
-GemmDesc nf4_fwd(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
                  const uint16_t* act, int64_t T, const float* B, int r, float s, const float* u,
                  int64_t u_ld, int n_parts, const int64_t* pe, const uint16_t* res, void* out,
                  int64_t ldo) {
@@ -142,7 +168,9 @@ GemmDesc nf4_fwd(const uint8_t* codes, const float* absmax, int64_t N, int64_t K
   d.T = T;
   d.Kc = K;
   d.w = codes;
-  d.absmax = absmax;
+  d.absmax = absmax.f32;
+  d.absmax_q = absmax.q;
+  d.absmax_s = absmax.s;
   d.w_rows = N;
   d.w_cols = K;
   d.act = act;
@@ -165,7 +193,7 @@ GemmDesc nf4_fwd(const uint8_t* codes, const float* absmax, int64_t N, int64_t K
 }
 
 // dX of a stacked NF4 weight W [N, K]: out [T, K] = dy W + s v A_stack, v [T, R], A [R, K]
-GemmDesc nf4_dx(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
+GemmDesc nf4_dx(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
                 const uint16_t* dy, int64_t T, const float* A, int R, float s, const float* v,
                 void* out, int out_f32) {
   GemmDesc d;
@@ -174,7 +202,9 @@ GemmDesc nf4_dx(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
   d.T = T;
   d.Kc = N;
   d.w = codes;
-  d.absmax = absmax;
+  d.absmax = absmax.f32;
+  d.absmax_q = absmax.q;
+  d.absmax_s = absmax.s;
   d.w_rows = N;
   d.w_cols = K;
   d.act = dy;
@@ -241,18 +271,18 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   const int64_t pe2[2] = {s.F, s.gu_n};
   size_t gb = 0;
   GemmDesc ds[8] = {
-      nf4_fwd(nullptr, nullptr, s.qkv_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 3 * r, 3, pe3,
+      nf4_fwd(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 3 * r, 3, pe3,
               nullptr, nullptr, s.qkv_n),
-      nf4_fwd(nullptr, nullptr, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
+      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
               nullptr, s.D),
-      nf4_fwd(nullptr, nullptr, s.gu_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 2 * r, 2, pe2,
+      nf4_fwd(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 2 * r, 2, pe2,
               nullptr, nullptr, s.gu_n),
-      nf4_fwd(nullptr, nullptr, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
+      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
               nullptr, s.D),
-      nf4_dx(nullptr, nullptr, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, nullptr, 1),
-      nf4_dx(nullptr, nullptr, s.gu_n, s.D, nullptr, T, nullptr, 2 * r, 0, nullptr, nullptr, 1),
-      nf4_dx(nullptr, nullptr, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, nullptr, 0),
-      nf4_dx(nullptr, nullptr, s.qkv_n, s.D, nullptr, T, nullptr, 3 * r, 0, nullptr, nullptr, 1)};
+      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, nullptr, 1),
+      nf4_dx(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, 2 * r, 0, nullptr, nullptr, 1),
+      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, nullptr, 0),
+      nf4_dx(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, 3 * r, 0, nullptr, nullptr, 1)};
   for (auto& d : ds) gb = std::max(gb, gemm_workspace_bytes(d));
   x.gemm = a.take<uint8_t>(gb + 256);
   x.gemm_bytes = gb + 256;

@@ -109,6 +109,45 @@ __global__ void nf4_dequantize_kernel(const uint8_t* __restrict__ codes,
   }
 }
 
+// Double quantisation of the absmax: one CTA of 256 threads per run of 256
+// absmax values (the last run may be short).  s = fl32(max / 255), q =
+// rint(fl32(a / s)) (half to even), at most 255; a run of zeros gets s = 0, q = 0.
+__global__ void absmax_q8_kernel(const float* __restrict__ absmax, int64_t n,
+                                 uint8_t* __restrict__ q, float* __restrict__ scale) {
+  __shared__ float wmax[8];
+  const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const float a = (i < n) ? absmax[i] : 0.f;
+  float m = a;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float mx = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, wmax[w]);
+  const float s = (mx > 0.f) ? __fdiv_rn(mx, 255.f) : 0.f;
+  if (i < n) {
+    int v = 0;
+    if (mx > 0.f) v = min(255, __float2int_rn(__fdiv_rn(a, s)));
+    q[i] = (uint8_t)v;
+  }
+  if (threadIdx.x == 0) scale[blockIdx.x] = s;
+}
+
+__global__ void nf4_dequantize_dq_kernel(const uint8_t* __restrict__ codes,
+                                         const uint8_t* __restrict__ q,
+                                         const float* __restrict__ scale, int64_t n_bytes,
+                                         float* __restrict__ W, LevelParams lp) {
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_bytes;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    const uint8_t c = codes[j];
+    const int64_t b = j >> 5;  // 32 bytes per 64-element block
+    const float am = (float)q[b] * scale[b >> 8];
+    W[2 * j] = lp.lv[c >> 4] * am;
+    W[2 * j + 1] = lp.lv[c & 15] * am;
+  }
+}
+
 }  // namespace
 
 const float* nf4_levels() {
@@ -189,6 +228,37 @@ extern "C" int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t
   const int64_t cap = (int64_t)gemm_num_sms() * 16;
   if (grid > cap) grid = cap;
   nf4_dequantize_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, absmax, n_bytes, W_out, lp);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
+extern "C" int nf4_absmax_quantize8(const float* absmax, int64_t n_blocks, uint8_t* q,
+                                    float* scale, void* stream) {
+  if (n_blocks <= 0) return set_error(LSQ_ERR_SHAPE, "nf4_absmax_quantize8: n_blocks must be positive");
+  if (!absmax || !q || !scale) return set_error(LSQ_ERR_INVALID, "nf4_absmax_quantize8: null pointer");
+  if (!aligned16(q)) return set_error(LSQ_ERR_ALIGN, "nf4_absmax_quantize8: q must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t groups = (n_blocks + 255) / 256;
+  if (groups > INT32_MAX) return set_error(LSQ_ERR_SHAPE, "nf4_absmax_quantize8: too many blocks");
+  absmax_q8_kernel<<<(unsigned)groups, 256, 0, st>>>(absmax, n_blocks, q, scale);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
+extern "C" int nf4_dequantize_dq(const uint8_t* codes, const uint8_t* q, const float* scale,
+                                 int64_t N, int64_t K, int32_t block, float* W_out, void* stream) {
+  LSQ_TRY(check_nf4_shape(N, K, block, "nf4_dequantize_dq"));
+  if (!W_out || !codes || !q || !scale)
+    return set_error(LSQ_ERR_INVALID, "nf4_dequantize_dq: null pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LevelParams lp;
+  const float* lv = nf4_levels();
+  for (int i = 0; i < 16; ++i) lp.lv[i] = lv[i];
+  const int64_t n_bytes = N * K / 2;
+  int64_t grid = (n_bytes + 255) / 256;
+  const int64_t cap = (int64_t)gemm_num_sms() * 16;
+  if (grid > cap) grid = cap;
+  nf4_dequantize_dq_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, q, scale, n_bytes, W_out, lp);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }

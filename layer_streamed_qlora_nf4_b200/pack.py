@@ -3,7 +3,8 @@
 ``pack_layer`` quantises a layer's seven frozen weights into one blob with the
 library's ``nf4_quantize`` (the offline NF4 shard step of the Soup layer-streaming
 tutorial, "四段資料路徑" part 1), writing at the offsets ``lsq_layer_layout_get``
-returns, and copies the two RMSNorm gains.  ``lora_block`` places the fp32 LoRA
+returns (with an 8-bit absmax, ``nf4_absmax_quantize8`` then stores the absmax
+in 8 bits), and copies the two RMSNorm gains.  ``lora_block`` places the fp32 LoRA
 masters at the offsets of ``lsq_lora_layout_get``.  No arithmetic happens here.
 """
 import torch
@@ -23,8 +24,17 @@ def pack_layer(cfg, W, g1, g2, blob, stream=None):
         w = W[name]
         assert tuple(w.shape) == (N, K) and w.dtype == torch.float32 and w.is_contiguous()
         codes = blob[lay.codes_off[p]: lay.codes_off[p] + N * K // 2]
-        absmax = blob[lay.absmax_off[p]: lay.absmax_off[p] + N * K // 64 * 4].view(torch.float32)
-        lib.nf4_quantize(w, codes, absmax, stream=stream)
+        nb = N * K // 64
+        if lay.absmax_bits == 8:
+            # codes from the fp32 absmax, then the absmax itself to 8 bits
+            absmax = torch.empty(nb, dtype=torch.float32, device=blob.device)
+            lib.nf4_quantize(w, codes, absmax, stream=stream)
+            q = blob[lay.absmax_off[p]: lay.absmax_off[p] + nb]
+            sc = blob[lay.scale_off[p]: lay.scale_off[p] + (nb + 255) // 256 * 4].view(torch.float32)
+            lib.nf4_absmax_quantize8(absmax, q, sc, stream=stream)
+        else:
+            absmax = blob[lay.absmax_off[p]: lay.absmax_off[p] + nb * 4].view(torch.float32)
+            lib.nf4_quantize(w, codes, absmax, stream=stream)
     D = cfg["hidden"]
     blob[lay.g1_off: lay.g1_off + 2 * D].copy_(g1.contiguous().view(torch.uint8))
     blob[lay.g2_off: lay.g2_off + 2 * D].copy_(g2.contiguous().view(torch.uint8))

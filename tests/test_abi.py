@@ -68,6 +68,29 @@ def test_layer_layout_matches_the_documented_sizes(L):
     assert n_lora * 32 == 41943040   # 41.9 M LoRA parameters for the 32-layer stack
 
 
+def test_layer_layout_with_8bit_absmax_gives_the_pages_store_size(L):
+    # The pages: a 3.60 GB store for the 32 layers, 113 MB layer buffers (article
+    # "架构解读：layer streaming 如何塞进 4 GB").  An fp32 absmax gives 122.7 MB and
+    # 3.93 GB; an 8-bit absmax with one fp32 scale per 256 blocks gives the pages'.
+    cfg = dict(synth.LLAMA8B, absmax_bits=8)
+    lay = L.lsq_layer_layout_get(cfg)
+    P = 218103808
+    expect = P // 2 + P // 64 + 4 * (P // 64 // 256) + 2 * 4096 * 2
+    assert lay.bytes == expect == 112529408 and lay.absmax_bits == 8
+    assert round(lay.bytes / 1e6) == 113 and round(32 * lay.bytes / 1e9, 2) == 3.60
+    assert round(32 * L.lsq_layer_layout_get(synth.LLAMA8B).bytes / 1e9, 2) == 3.93
+    for p in range(7):
+        nb = lay.rows[p] * lay.cols[p] // 64
+        assert nb % 256 == 0           # a scale run never straddles two projections
+        if p + 1 < 7:
+            assert lay.absmax_off[p + 1] == lay.absmax_off[p] + nb          # uint8, stacked
+            assert lay.scale_off[p + 1] == lay.scale_off[p] + nb // 256 * 4
+    for o in list(lay.absmax_off) + list(lay.scale_off) + [lay.g1_off, lay.g2_off]:
+        assert o % 256 == 0
+    with pytest.raises(L.LsqError):
+        L.lsq_layer_layout_get(dict(synth.LLAMA8B, absmax_bits=16))
+
+
 def test_workspace_queries_are_host_only(L):
     assert L.nf4_lora_linear_workspace_bytes(128, 1024, 1024, 16) > 0
     assert L.decoder_layer_workspace_bytes(synth.LLAMA8B, 1, 512) > 0

@@ -18,11 +18,17 @@ def L():
     return lib
 
 
+def _oracle_weight(W, absmax_bits):
+    """The weight the layer sees: NF4 with fp32 absmax, or with the 8-bit absmax."""
+    N, K = W.shape
+    codes, am = onf4.quantize(W)
+    if absmax_bits == 8:
+        return onf4.dequantize_dq(codes, *onf4.quantize_absmax8(am), N, K)
+    return onf4.dequantize(codes, am, N, K)
+
+
 def _oracle_params(lw, cfg):
-    W = {}
-    for p in synth.PROJ:
-        N, K = lw["W"][p].shape
-        W[p] = onf4.dequantize(*onf4.quantize(lw["W"][p]), N, K)
+    W = {p: _oracle_weight(lw["W"][p], cfg.get("absmax_bits", 32)) for p in synth.PROJ}
     return dict(W=W, A=lw["A"], B=lw["B"], g1=synth.bf16_bits_to_f32(lw["g1"]),
                 g2=synth.bf16_bits_to_f32(lw["g2"]))
 
@@ -120,3 +126,8 @@ def test_layer_rejects_bad_config(L):
     with pytest.raises(L.LsqError) as e:
         L.lsq_layer_layout_get(cfg)
     assert e.value.code == L.LSQ_ERR_SHAPE
+
+
+def test_layer_small_absmax8(L):
+    # the 8-bit double-quantised absmax, dequantised inside the GEMM operand stage
+    _run_layer(L, dict(synth.SMALL, absmax_bits=8), batch=2, seq=100, seed=17)

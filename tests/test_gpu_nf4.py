@@ -86,3 +86,41 @@ def test_quantize_rejects_nonfinite_and_bad_shapes(L):
     # a later valid call still works and the status word is clean
     codes, absmax = _quant_gpu(L, np.ones((2, 64), np.float32))
     assert L.lsq_device_status() == 0
+
+
+def _absmax8_case(n, seed):
+    a = np.abs(synth.normal_f32(synth.rng(seed), (n,), 0.05))
+    a[:256] = 0.0                                       # a zero run
+    a[256:512] = np.float32(2.0 ** -10) * np.arange(256, dtype=np.float32)   # exact grid
+    a[300] = np.float32(2.5 * 2.0 ** -10)              # tie -> even
+    return a
+
+
+@pytest.mark.parametrize("n", [1024, 256 * 37 + 77, 4096 * 4096 // 64])
+def test_absmax_quantize8_bit_exact(L, n):
+    import torch
+    from gpu_util import dev
+    a = _absmax8_case(n, 200 + n % 97)
+    q = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = torch.full(((n + 255) // 256,), float("nan"), dtype=torch.float32, device="cuda")
+    L.nf4_absmax_quantize8(dev(a), q, s)
+    rq, rs = onf4.quantize_absmax8(a)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K", [(512, 1024), (1024, 14336)])
+def test_dequantize_dq_bit_exact(L, N, K):
+    import torch
+    W = synth.normal_f32(synth.rng(300 + N), (N, K), 0.02)
+    codes, absmax = _quant_gpu(L, W)
+    nb = N * K // 64
+    q = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    s = torch.empty((nb + 255) // 256, dtype=torch.float32, device="cuda")
+    L.nf4_absmax_quantize8(absmax, q, s)
+    out = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    L.nf4_dequantize_dq(codes, q, s, N, K, out)
+    rc, ra = onf4.quantize(W)
+    rq, rs = onf4.quantize_absmax8(ra)
+    ref = onf4.dequantize_dq(rc, rq, rs, N, K)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))

@@ -55,11 +55,16 @@ class Stack:
 
     def oracle_layers(self):
         out = []
+        bits = self.cfg.get("absmax_bits", 32)
         for lw in self.lw:
             W = {}
             for p in synth.PROJ:
                 N, K = lw["W"][p].shape
-                W[p] = onf4.dequantize(*onf4.quantize(lw["W"][p]), N, K)
+                codes, am = onf4.quantize(lw["W"][p])
+                if bits == 8:
+                    W[p] = onf4.dequantize_dq(codes, *onf4.quantize_absmax8(am), N, K)
+                else:
+                    W[p] = onf4.dequantize(codes, am, N, K)
             out.append(dict(W=W, A=lw["A"], B=lw["B"], g1=synth.bf16_bits_to_f32(lw["g1"]),
                             g2=synth.bf16_bits_to_f32(lw["g2"])))
         return out
@@ -85,7 +90,36 @@ def small(L):
     return Stack(L, synth.SMALL, 5)
 
 
+@pytest.fixture(scope="module")
+def small8(L):
+    # the same weights as `small`, stored with the 8-bit absmax
+    return Stack(L, dict(synth.SMALL, absmax_bits=8), 5)
+
+
 def test_stack_matches_oracle(L, small):
+    _check_against_oracle(L, small)
+
+
+def test_stack_absmax8_matches_oracle(L, small8):
+    _check_against_oracle(L, small8)
+
+
+def test_stack_absmax8_streamed_equals_resident_bitwise(L, small8):
+    import torch
+    tokens = synth.tokens(34, 1, 96, small8.cfg["vocab"])
+    hs = small8.handle(L, resident=False)
+    hr = small8.handle(L, resident=True)
+    ls, lgs, gs, _ = _step(L, small8, hs, tokens, 1, 1, 96)
+    st = L.stream_stack_last_stats(hs)
+    lr_, lgr, gr, _ = _step(L, small8, hr, tokens, 1, 1, 96)
+    hs.close()
+    hr.close()
+    assert ls == lr_ and torch.equal(lgs, lgr) and torch.equal(gs, gr)
+    assert st["h2d_bytes"] == st["layer_copies"] * small8.blob_bytes
+    assert small8.blob_bytes < L.lsq_layer_layout_get(synth.SMALL).bytes
+
+
+def _check_against_oracle(L, small):
     from gpu_util import normwise_err
     from layer_streamed_qlora_nf4_b200 import pack
     cfg = small.cfg
