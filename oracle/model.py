@@ -28,6 +28,16 @@ What the pages fix, and the readings taken where they are silent:
     YAML, betas (0.9, 0.999), eps 1e-8, decoupled weight decay 0, bias-corrected,
     step counter starting at 1).
 
+  * DPO step (Soup release notes "Layer streaming ... 扩展到偏好损失" and the Layer
+    Streaming blog, "無記憶體消耗的參考模型"): the reference model is the same
+    streamed base with its adapter turned off, i.e. every LoRA branch removed
+    (y = x W~^T).  The pages name DPO but print no formula; the reading is the
+    published Direct Preference Optimization loss: for a pair (chosen c,
+    rejected r), z = beta * ((log pi(c) - log ref(c)) - (log pi(r) - log ref(r))),
+    loss = mean over pairs of -log sigmoid(z).  A sequence's log-probability is
+    the sum over positions 0..S-2 of log softmax(logits)[tokens[t+1]] (synthetic
+    pairs: no prompt mask).
+
 Projection order everywhere: q, k, v, o, gate, up, down.
 """
 
@@ -281,6 +291,73 @@ def stack_loss_and_grads(layers, emb, lm_head, g_final, tokens, cfg):
     for i in range(len(layers) - 1, -1, -1):
         dh, grads[i] = decoder_layer_bwd(layers[i], c["xs"][i], dh, cfg, S)
     return loss, logits, grads
+
+
+def adapter_off(layers):
+    """The reference model of the DPO step: the same layers with the LoRA branch removed."""
+    out = []
+    for p in layers:
+        q = dict(p)
+        q["B"] = {n: np.zeros_like(np.asarray(b, np.float64)) for n, b in p["B"].items()}
+        out.append(q)
+    return out
+
+
+def sequence_logprobs(logits, tokens):
+    """Sum over positions 0..S-2 of log softmax(logits[t])[tokens[t+1]] -> [B]."""
+    tokens = np.asarray(tokens)
+    Bsz, S = tokens.shape
+    lg = np.asarray(logits, np.float64).reshape(Bsz, S, -1)
+    m = np.max(lg, axis=-1, keepdims=True)
+    lse = (m + np.log(np.sum(np.exp(lg - m), axis=-1, keepdims=True)))[..., 0]
+    picked = np.take_along_axis(lg[:, :-1, :], tokens[:, 1:, None], axis=-1)[..., 0]
+    return np.sum(picked - lse[:, :-1], axis=1)
+
+
+def dpo_loss(lp_pol, lp_ref, beta):
+    """lp_* [P, 2] (chosen, rejected) -> (loss, dloss/dlp_pol [P, 2], z [P])."""
+    lp_pol = np.asarray(lp_pol, np.float64)
+    lp_ref = np.asarray(lp_ref, np.float64)
+    P = lp_pol.shape[0]
+    z = beta * ((lp_pol[:, 0] - lp_ref[:, 0]) - (lp_pol[:, 1] - lp_ref[:, 1]))
+    # -log sigmoid(z) = softplus(-z), written to stay finite for large |z|
+    loss = float(np.mean(np.maximum(-z, 0.0) + np.log1p(np.exp(-np.abs(z)))))
+    sig_neg = 1.0 / (1.0 + np.exp(z))            # sigmoid(-z) = -d softplus(-z) / dz
+    g = np.empty((P, 2))
+    g[:, 0] = -beta * sig_neg / P
+    g[:, 1] = beta * sig_neg / P
+    return loss, g, z
+
+
+def dpo_loss_and_grads(layers, emb, lm_head, g_final, tokens, cfg, beta):
+    """One DPO forward + backward; tokens [P, 2, S] (pair, chosen/rejected, position).
+
+    Returns (loss, policy logits [2P*S, V], LoRA grads per layer, dict(lp_pol, lp_ref, z)).
+    """
+    tokens = np.asarray(tokens)
+    P, two, S = tokens.shape
+    assert two == 2
+    flat = tokens.reshape(2 * P, S)
+    ref_logits, _ = stack_forward(adapter_off(layers), emb, lm_head, g_final, flat, cfg)
+    logits, c = stack_forward(layers, emb, lm_head, g_final, flat, cfg)
+    lp_ref = sequence_logprobs(ref_logits, flat).reshape(P, 2)
+    lp_pol = sequence_logprobs(logits, flat).reshape(P, 2)
+    loss, g, z = dpo_loss(lp_pol, lp_ref, beta)
+    # d lp_b / d logits[b, t] = onehot(tokens[b, t+1]) - softmax(logits[b, t]), t < S-1
+    lg = logits.reshape(2 * P, S, -1)
+    sm = np.exp(lg - np.max(lg, axis=-1, keepdims=True))
+    sm /= np.sum(sm, axis=-1, keepdims=True)
+    dlp = -sm
+    dlp[:, -1, :] = 0.0
+    bi, ti = np.meshgrid(np.arange(2 * P), np.arange(S - 1), indexing="ij")
+    dlp[bi, ti, flat[:, 1:]] += 1.0
+    dlogits = (dlp * g.reshape(2 * P)[:, None, None]).reshape(2 * P * S, -1)
+    dhf = dlogits @ np.asarray(lm_head, np.float64)
+    dh = rmsnorm_bwd(dhf, c["h"], g_final, cfg["rms_eps"])
+    grads = [None] * len(layers)
+    for i in range(len(layers) - 1, -1, -1):
+        dh, grads[i] = decoder_layer_bwd(layers[i], c["xs"][i], dh, cfg, S)
+    return loss, logits, grads, dict(lp_pol=lp_pol, lp_ref=lp_ref, z=z)
 
 
 def adamw_step(param, grad, m, v, step, lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, wd=0.0):

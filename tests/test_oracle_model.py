@@ -318,3 +318,91 @@ def test_adamw_matches_torch():
         opt.step()
         p, m, v = om.adamw_step(p, grad, m, v, step, wd=0.01)
     assert np.max(np.abs(p - tp.detach().numpy())) < 1e-14
+
+
+# ------------------------------------------------------------------ DPO step
+def _dpo_case(seed, P=2, S=7, V=97, nl=2):
+    cfg = TINY
+    layers = [_layer_params(seed + i, cfg) for i in range(nl)]
+    g = np.random.default_rng(seed + 50)
+    emb, head = g.standard_normal((V, cfg["hidden"])) * 0.5, g.standard_normal((V, cfg["hidden"])) * 0.5
+    gf = 1.0 + 0.1 * g.standard_normal(cfg["hidden"])
+    tokens = g.integers(0, V, size=(P, 2, S))
+    return cfg, layers, emb, head, gf, tokens
+
+
+def test_sequence_logprobs_brute_force_loops():
+    g = np.random.default_rng(60)
+    lg = g.standard_normal((2 * 5, 11))
+    tok = g.integers(0, 11, size=(2, 5))
+    got = om.sequence_logprobs(lg, tok)
+    for b in range(2):
+        want = 0.0
+        for t in range(4):
+            row = lg[b * 5 + t]
+            want += math.log(math.exp(row[tok[b, t + 1]]) / sum(math.exp(v) for v in row))
+        assert abs(got[b] - want) < 1e-12
+
+
+def test_dpo_matches_hf_llama_autograd():
+    # Policy: the HF Llama with LoRA on all seven projections; reference: the same
+    # model with every LoRA branch removed; the DPO loss written with torch ops.
+    cfg, layers, emb, head, gf, tokens = _dpo_case(70)
+    V, nl, beta = 97, 2, 0.1
+    pol = _hf_model(cfg, layers, nl, V, emb, head, gf)
+    ref = _hf_model(cfg, om.adapter_off(layers), nl, V, emb, head, gf)
+    ids = torch.tensor(tokens.reshape(-1, tokens.shape[-1]), dtype=torch.long)
+
+    def seq_lp(model):
+        lp = torch.log_softmax(model(input_ids=ids).logits, dim=-1)
+        return torch.gather(lp[:, :-1], 2, ids[:, 1:, None])[..., 0].sum(1).reshape(-1, 2)
+    with torch.no_grad():
+        lr = seq_lp(ref)
+    lpp = seq_lp(pol)
+    z = beta * ((lpp[:, 0] - lr[:, 0]) - (lpp[:, 1] - lr[:, 1]))
+    tloss = -torch.nn.functional.logsigmoid(z).mean()
+    tloss.backward()
+    loss, logits, grads, aux = om.dpo_loss_and_grads(layers, emb, head, gf, tokens, cfg, beta)
+    assert abs(loss - tloss.item()) < 1e-5 * abs(loss)
+    assert _close(aux["lp_ref"], lr.numpy()) and _close(aux["lp_pol"], lpp.detach().numpy())
+    for i, L in enumerate(pol.model.layers):
+        mods = dict(q=L.self_attn.q_proj, k=L.self_attn.k_proj, v=L.self_attn.v_proj, o=L.self_attn.o_proj,
+                    gate=L.mlp.gate_proj, up=L.mlp.up_proj, down=L.mlp.down_proj)
+        for n, mod in mods.items():
+            assert _close(grads[i][n][0], mod.A.grad.numpy(), 1e-4), (i, n)
+            assert _close(grads[i][n][1], mod.B.grad.numpy(), 1e-4), (i, n)
+
+
+def test_dpo_with_the_adapter_at_zero_is_log2_and_swaps_sign():
+    cfg, layers, emb, head, gf, tokens = _dpo_case(80)
+    zero = om.adapter_off(layers)           # policy == reference
+    loss, _, grads, aux = om.dpo_loss_and_grads(zero, emb, head, gf, tokens, cfg, 0.1)
+    assert abs(loss - math.log(2.0)) < 1e-12 and np.allclose(aux["z"], 0.0, atol=1e-12)
+    for gl in grads:                        # B = 0: no gradient can reach A
+        for n in om.PROJ:
+            assert np.max(np.abs(gl[n][0])) == 0.0
+    # swapping chosen and rejected flips z: softplus(z) - softplus(-z) = z
+    l1, _, _, a1 = om.dpo_loss_and_grads(layers, emb, head, gf, tokens, cfg, 0.1)
+    l2, _, _, a2 = om.dpo_loss_and_grads(layers, emb, head, gf, tokens[:, ::-1, :], cfg, 0.1)
+    assert np.allclose(a2["z"], -a1["z"], atol=1e-12)
+    assert abs((l2 - l1) - np.mean(a1["z"])) < 1e-12
+
+
+def test_dpo_finite_differences():
+    cfg, layers, emb, head, gf, tokens = _dpo_case(90, P=1, S=5)
+    beta = 0.5
+    _, _, grads, _ = om.dpo_loss_and_grads(layers, emb, head, gf, tokens, cfg, beta)
+    g = np.random.default_rng(91)
+    h = 1e-6
+    for (li, n, k) in ((0, "q", "A"), (1, "down", "B"), (0, "gate", "B"), (1, "v", "A")):
+        arr = layers[li][k][n]
+        idx = tuple(int(g.integers(0, d)) for d in arr.shape)
+        old = arr[idx]
+        arr[idx] = old + h
+        lp = om.dpo_loss_and_grads(layers, emb, head, gf, tokens, cfg, beta)[0]
+        arr[idx] = old - h
+        lm = om.dpo_loss_and_grads(layers, emb, head, gf, tokens, cfg, beta)[0]
+        arr[idx] = old
+        fd = (lp - lm) / (2 * h)
+        an = grads[li][n][0 if k == "A" else 1][idx]
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)) + 1e-8, (li, n, k, fd, an)
