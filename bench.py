@@ -37,11 +37,21 @@ BATCH, SEQ = 1, 512
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 
 
-def workload_name(absmax_bits):
+def workload_name(absmax_bits, dpo=False, pairs=2, batch=1, micro_batches=1):
+    w = WORKLOAD
     if absmax_bits == 8:
-        return WORKLOAD.replace("fp32 absmax", "8-bit double-quantised absmax, one fp32 scale "
-                                "per 256 blocks")
-    return WORKLOAD
+        w = w.replace("fp32 absmax", "8-bit double-quantised absmax, one fp32 scale per 256 "
+                      "blocks")
+    if dpo:
+        w = w.replace("batch 1 x seq 512 per GPU; one SFT step (cross-entropy + AdamW",
+                      "%d chosen/rejected pairs x seq 512 per GPU; one DPO step (beta 0.1, the "
+                      "same streamed base with its adapter off as reference, run from the same "
+                      "layer buffer; AdamW" % pairs)
+    elif batch != 1 or micro_batches != 1:
+        w = w.replace("batch 1 x seq 512 per GPU; one SFT step",
+                      "batch %d x seq 512 x %d gradient-accumulation micro-batches per GPU; one "
+                      "SFT step" % (batch, micro_batches))
+    return w
 
 
 def parse():
@@ -56,8 +66,13 @@ def parse():
                     help="32: fp32 absmax per NF4 block (the default workload); 8: the absmax "
                          "double-quantised to 8 bits with one fp32 scale per 256 blocks, the "
                          "pages' 113 MB layers / 3.60 GB store")
-    ap.add_argument("--case", choices=("step", "layer", "gemm"), default="step",
-                    help="step: the streamed 32-layer SFT step (default); layer: one resident "
+    ap.add_argument("--batch", type=int, default=1, help="sequences per micro-batch (SFT step)")
+    ap.add_argument("--micro-batches", type=int, default=1,
+                    help="gradient-accumulation micro-batches per optimiser step (SFT step)")
+    ap.add_argument("--pairs", type=int, default=2, help="chosen/rejected pairs (DPO step)")
+    ap.add_argument("--case", choices=("step", "dpo", "layer", "gemm"), default="step",
+                    help="step: the streamed 32-layer SFT step (default); dpo: the streamed DPO "
+                         "step (beta 0.1, adapter-off reference); layer: one resident "
                          "8B-shaped layer forward + recomputing backward; gemm: one fused NF4 "
                          "GEMM at the q|k|v shape (a small case for profiling)")
     return ap.parse_args()
@@ -187,7 +202,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
-def build_stack(L, cfg, rank):
+def build_stack(L, cfg, rank, tok_shape=(1, SEQ)):
     import torch
     from layer_streamed_qlora_nf4_b200 import pack, synth
     lay = L.lsq_layer_layout_get(cfg)
@@ -210,7 +225,7 @@ def build_stack(L, cfg, rank):
     emb = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
     head = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
     gt = torch.Generator(device="cuda").manual_seed(1000 + rank)
-    tokens = torch.randint(0, cfg["vocab"], (8, BATCH, SEQ), generator=gt, device="cuda",
+    tokens = torch.randint(0, cfg["vocab"], (8,) + tuple(tok_shape), generator=gt, device="cuda",
                            dtype=torch.int32)
     bufs = [torch.empty(lay.bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
     return dict(lay=lay, host_blobs=host_blobs, lora=lora, emb=emb, head=head, gf=ones,
@@ -247,11 +262,16 @@ def run_ours(args):
     from layer_streamed_qlora_nf4_b200 import synth
     L.load()
     cfg = dict(synth.LLAMA8B, absmax_bits=args.absmax_bits)
-    st = build_stack(L, cfg, rank)
+    dpo = args.case == "dpo"
+    batch, mbs = (2 * args.pairs, 1) if dpo else (args.batch, args.micro_batches)
+    tok_shape = (args.pairs, 2, SEQ) if dpo else (mbs, batch, SEQ)
+    tokens_per_step = mbs * batch * SEQ
+    st = build_stack(L, cfg, rank, tok_shape)
     lay = st["lay"]
     handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
-    ws = torch.empty(L.stream_stack_workspace_bytes(cfg, BATCH, SEQ), dtype=torch.uint8,
-                     device="cuda")
+    ws_bytes = (L.stream_stack_dpo_workspace_bytes(cfg, args.pairs, SEQ) if dpo
+                else L.stream_stack_workspace_bytes(cfg, batch, SEQ))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     lora, grad = st["lora"], torch.zeros_like(st["lora"])
     m, v = torch.zeros_like(lora), torch.zeros_like(lora)
     opt = dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1, m=m, v=v)
@@ -259,12 +279,14 @@ def run_ours(args):
     pool = st["tokens"]           # a few distinct batches, cycled
 
     def step(tokens):
-        if world == 1:
-            loss = L.stream_stack_step(handle, tokens, 1, BATCH, SEQ, st["emb"], st["head"],
-                                       st["gf"], lora, grad, opt, ws)
+        o = opt if world == 1 else None
+        if dpo:
+            loss, _ = L.stream_stack_dpo_step(handle, tokens, args.pairs, SEQ, 0.1, st["emb"],
+                                              st["head"], st["gf"], lora, grad, o, ws)
         else:
-            loss = L.stream_stack_step(handle, tokens, 1, BATCH, SEQ, st["emb"], st["head"],
-                                       st["gf"], lora, grad, None, ws)
+            loss = L.stream_stack_step(handle, tokens, mbs, batch, SEQ, st["emb"], st["head"],
+                                       st["gf"], lora, grad, o, ws)
+        if world > 1:
             dp.average_(grad)                       # NCCL all-reduce of the LoRA gradients
             L.lora_adamw_step(lora, grad, opt)
         opt["step"] += 1
@@ -311,7 +333,7 @@ def run_ours(args):
     sampler.start()
     ms, loss, copies, wait_ms, launches, _ = timed(args.steps, lambda i: pool[i % len(pool)])
     clocks = sampler.stop()
-    value = world * BATCH * SEQ / (ms * 1e-3)
+    value = world * tokens_per_step / (ms * 1e-3)
 
     # ------------------------------------------------------------ same steps, kernels timed
     # every tensor-core GEMM and attention launch bracketed by CUDA events on its stream
@@ -326,7 +348,7 @@ def run_ours(args):
         tok_dev.copy_(tok_host[i % len(tok_host)], non_blocking=True)
         return tok_dev                  # the step itself returns the loss on the host
     e2e_ms = timed(args.steps, from_host, label="timed_e2e")[0]
-    e2e = dict(value=world * BATCH * SEQ / (e2e_ms * 1e-3), unit="tokens/s",
+    e2e = dict(value=world * tokens_per_step / (e2e_ms * 1e-3), unit="tokens/s",
                h2d_bytes_per_step=tok_dev.numel() * 4, d2h_bytes_per_step=4,
                layer_stream_h2d_bytes_per_step=copies // args.steps * lay.bytes)
 
@@ -366,7 +388,7 @@ def run_ours(args):
                               for k, e in prof.items()})
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not dpo and tokens_per_step == SEQ:
         s, desc = oracle_sample(seed=1)
         cpu = dict(value=BATCH * SEQ / s, unit="tokens/s", cores=cpu_threads(), kind="oracle",
                    sample=desc)
@@ -376,8 +398,9 @@ def run_ours(args):
                     warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak",
                     vs_baseline=None, dtype="bf16", data="synthetic (seeded random weights and "
                     "uniform token ids at the 8B shapes)",
-                    config=dict(workload=workload_name(args.absmax_bits),
-                                global_batch=world * BATCH, seq_len=SEQ,
+                    config=dict(workload=workload_name(args.absmax_bits, dpo, args.pairs, batch,
+                                                       mbs),
+                                global_batch=world * tokens_per_step // SEQ, seq_len=SEQ,
                                 parallelism="dp%d" % world,
                                 l2="inputs larger than L2: %.2f GB of layer bytes stream per step"
                                 % (cps * lay.bytes / 1e9)),

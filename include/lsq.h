@@ -202,7 +202,9 @@ size_t decoder_layer_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t 
  * -> causal GQA attention -> o (+residual) -> RMSNorm -> gate/up -> SwiGLU ->
  * down (+residual).
  *   blob    device pointer to the layer blob (lsq_layer_layout).
- *   lora    device fp32, one layer's LoRA block (lsq_lora_layout).
+ *   lora    device fp32, one layer's LoRA block (lsq_lora_layout), or NULL to
+ *           run the layer with its adapter off (every LoRA branch removed: the
+ *           reference model of the DPO step).
  *   x_in    device bf16 [batch*seq, D]; x_out device bf16 [batch*seq, D].
  * Asynchronous, deterministic. */
 int decoder_layer_fwd(const lsq_cfg* cfg, const void* blob, const float* lora,
@@ -268,7 +270,34 @@ int stream_stack_step(lsq_stack* stack, const int32_t* tokens, int32_t micro_bat
                       const lsq_adamw* opt, float* loss_out, float* logits_out, void* ws,
                       size_t ws_bytes, void* stream, int64_t timeout_ms);
 
-/* Per-step counters of the last stream_stack_step. */
+/* Workspace for stream_stack_dpo_step with `pairs` chosen/rejected pairs of seq tokens. */
+size_t stream_stack_dpo_workspace_bytes(const lsq_cfg* cfg, int32_t pairs, int32_t seq);
+
+/* stream_stack_dpo_step - one DPO optimiser step through the streamed stack,
+ * with the same streamed base and its adapter off as the reference model
+ * (Soup release notes, preference losses under layer streaming; Layer
+ * Streaming blog, "無記憶體消耗的參考模型").  The pages name DPO and that
+ * reference; the loss is the published Direct Preference Optimization one:
+ * z = beta ((lp(c) - lr(c)) - (lp(r) - lr(r))), loss = mean over pairs of
+ * -log sigmoid(z), where a sequence's log-probability is the sum over positions
+ * 0..seq-2 of log softmax(logits)[next token] (no prompt mask).
+ *   tokens      device int32 [pairs, 2, seq]: chosen then rejected of each pair.
+ *   pairs       1..32; beta > 0.
+ *   logps_out   host float [4 * pairs] or NULL: per pair (policy chosen, policy
+ *               rejected, reference chosen, reference rejected).
+ *   logits_out  device fp32 [2*pairs*seq, V] policy logits, or NULL.
+ *   other arguments as stream_stack_step (one micro-batch of 2*pairs sequences).
+ * Each layer's reference forward runs right after its policy forward from the
+ * same VRAM buffer, so the step copies each layer as often as an SFT step.
+ * Synchronous like stream_stack_step. */
+int stream_stack_dpo_step(lsq_stack* stack, const int32_t* tokens, int32_t pairs, int32_t seq,
+                          float beta, const uint16_t* emb, const uint16_t* lm_head,
+                          const uint16_t* final_norm, float* lora, float* lora_grad,
+                          const lsq_adamw* opt, float* loss_out, float* logps_out,
+                          float* logits_out, void* ws, size_t ws_bytes, void* stream,
+                          int64_t timeout_ms);
+
+/* Per-step counters of the last stream_stack_step or stream_stack_dpo_step. */
 typedef struct lsq_step_stats {
   int32_t layer_copies;     /* host->device layer copies issued */
   int64_t h2d_bytes;        /* bytes those copies moved */

@@ -341,19 +341,27 @@ __global__ void embedding_kernel(const int32_t* __restrict__ tok, int64_t T,
 
 // One CTA (512 threads) per row.  Rows whose position is the last of its
 // sequence have no target: zero gradient, zero loss.
+// One CTA per row: row_loss = lse - logit[target] (= -log p(target)); and, when
+// dlogits is given, dlogits = scale * (softmax - onehot(target)) in bf16, with
+// scale = inv_count, or seq_scale[row / seq] when seq_scale is given (the DPO
+// step's per-sequence coefficient).  The last position of each sequence has no
+// target: zero loss and zero gradient.
 __global__ void cross_entropy_kernel(const float* __restrict__ logits,
                                      const int32_t* __restrict__ tok, int64_t T, int seq,
-                                     int64_t V, float inv_count, uint16_t* __restrict__ dlogits,
+                                     int64_t V, float inv_count,
+                                     const float* __restrict__ seq_scale,
+                                     uint16_t* __restrict__ dlogits,
                                      float* __restrict__ row_loss) {
   __shared__ float red[32];
   __shared__ float bcast;
   const int64_t row = blockIdx.x;
   const float* lr = logits + row * V;
-  uint16_t* dr = dlogits + row * V;
+  uint16_t* dr = dlogits ? dlogits + row * V : nullptr;
   const bool has_target = (row % seq) != (seq - 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   if (!has_target) {
-    for (int64_t i = threadIdx.x; i < V; i += blockDim.x) dr[i] = 0;
+    if (dr)
+      for (int64_t i = threadIdx.x; i < V; i += blockDim.x) dr[i] = 0;
     if (threadIdx.x == 0) row_loss[row] = 0.f;
     return;
   }
@@ -385,10 +393,13 @@ __global__ void cross_entropy_kernel(const float* __restrict__ logits,
   const float lse = mx + logf(sum);
   const int64_t tgt = tok[row + 1];
   const float inv = 1.f / sum;
-  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) {
-    float p = expf(lr[i] - mx) * inv;
-    if (i == tgt) p -= 1.f;
-    dr[i] = float_to_bf16_bits(p * inv_count);
+  if (dr) {
+    const float scale = seq_scale ? seq_scale[row / seq] : inv_count;
+    for (int64_t i = threadIdx.x; i < V; i += blockDim.x) {
+      float p = expf(lr[i] - mx) * inv;
+      if (i == tgt) p -= 1.f;
+      dr[i] = float_to_bf16_bits(p * scale);
+    }
   }
   if (threadIdx.x == 0) row_loss[row] = lse - lr[tgt];
 }
@@ -514,9 +525,75 @@ int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int6
 }
 
 int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq, int64_t V,
-                         float inv_count, uint16_t* dlogits, float* row_loss, cudaStream_t st) {
-  cross_entropy_kernel<<<(unsigned)T, 512, 0, st>>>(logits, tokens, T, seq, V, inv_count, dlogits,
-                                                    row_loss);
+                         float inv_count, uint16_t* dlogits, float* row_loss, cudaStream_t st,
+                         const float* seq_scale) {
+  cross_entropy_kernel<<<(unsigned)T, 512, 0, st>>>(logits, tokens, T, seq, V, inv_count, seq_scale,
+                                                    dlogits, row_loss);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
+// DPO loss of P pairs from the per-row losses (-log p) of the policy and the
+// reference (rows: sequence q = 2 p + {0 chosen, 1 rejected}, seq positions
+// each).  One CTA: each sequence's log-probability is summed in a fixed order
+// (fp64), then z_p = beta ((lp_c - lr_c) - (lp_r - lr_r)), loss = mean
+// softplus(-z_p); seq_scale gets -dloss/dlp per sequence (the scale of
+// softmax - onehot in dlogits); logps gets (lp_c, lp_r, lr_c, lr_r) per pair.
+__global__ void dpo_loss_kernel(const float* __restrict__ row_pol,
+                                const float* __restrict__ row_ref, int pairs, int seq, float beta,
+                                float* __restrict__ seq_scale, float* __restrict__ logps,
+                                float* __restrict__ loss_out) {
+  __shared__ double red[2][32];
+  __shared__ double lp[2][64];  // [pol/ref][sequence], pairs <= 32
+  const int nseq = 2 * pairs;
+  for (int q = 0; q < nseq; ++q) {
+    double a = 0.0, b = 0.0;
+    for (int t = threadIdx.x; t < seq - 1; t += blockDim.x) {
+      a += (double)row_pol[(int64_t)q * seq + t];
+      b += (double)row_ref[(int64_t)q * seq + t];
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+      b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+      red[0][threadIdx.x >> 5] = a;
+      red[1][threadIdx.x >> 5] = b;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double sa = 0.0, sb = 0.0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        sa += red[0][w];
+        sb += red[1][w];
+      }
+      lp[0][q] = -sa;
+      lp[1][q] = -sb;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    double loss = 0.0;
+    for (int p = 0; p < pairs; ++p) {
+      const double z = (double)beta * ((lp[0][2 * p] - lp[1][2 * p]) - (lp[0][2 * p + 1] - lp[1][2 * p + 1]));
+      loss += fmax(-z, 0.0) + log1p(exp(-fabs(z)));
+      const double sig_neg = 1.0 / (1.0 + exp(z));
+      seq_scale[2 * p] = (float)((double)beta * sig_neg / pairs);
+      seq_scale[2 * p + 1] = (float)(-(double)beta * sig_neg / pairs);
+      logps[4 * p + 0] = (float)lp[0][2 * p];
+      logps[4 * p + 1] = (float)lp[0][2 * p + 1];
+      logps[4 * p + 2] = (float)lp[1][2 * p];
+      logps[4 * p + 3] = (float)lp[1][2 * p + 1];
+    }
+    loss_out[0] = (float)(loss / pairs);
+  }
+}
+
+int launch_dpo_loss(const float* row_pol, const float* row_ref, int pairs, int seq, float beta,
+                    float* seq_scale, float* logps, float* loss_out, cudaStream_t st) {
+  if (pairs <= 0 || pairs > 32) return set_error(LSQ_ERR_SHAPE, "dpo: 1..32 pairs per step");
+  dpo_loss_kernel<<<1, 256, 0, st>>>(row_pol, row_ref, pairs, seq, beta, seq_scale, logps,
+                                     loss_out);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }

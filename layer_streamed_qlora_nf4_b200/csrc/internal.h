@@ -121,9 +121,12 @@ int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F,
                       cudaStream_t st);
 int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D,
                      int64_t V, uint16_t* out, cudaStream_t st);
+// dlogits may be null (row losses only); seq_scale (per sequence) replaces inv_count.
 int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq,
                          int64_t V, float inv_count, uint16_t* dlogits, float* row_loss,
-                         cudaStream_t st);
+                         cudaStream_t st, const float* seq_scale = nullptr);
+int launch_dpo_loss(const float* row_pol, const float* row_ref, int pairs, int seq, float beta,
+                    float* seq_scale, float* logps, float* loss_out, cudaStream_t st);
 int launch_sum_rows(const float* row_loss, int64_t T, float scale, int accumulate, float* out,
                     cudaStream_t st);
 int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr, float b1,

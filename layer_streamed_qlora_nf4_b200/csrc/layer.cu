@@ -62,6 +62,7 @@ struct Views {  // pointers into one layer blob / one LoRA block
   const uint16_t* g1;
   const uint16_t* g2;
   const float *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_d, *B_d;
+  bool lora_on;  // false: adapter disabled, every LoRA branch removed
 };
 
 void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) {
@@ -135,14 +136,18 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
   }
   v.g1 = reinterpret_cast<const uint16_t*>(b + L.g1_off);
   v.g2 = reinterpret_cast<const uint16_t*>(b + L.g2_off);
-  v.A_qkv = lora + R.a_off[0];
-  v.B_qkv = lora + R.b_off[0];
-  v.A_o = lora + R.a_off[3];
-  v.B_o = lora + R.b_off[3];
-  v.A_gu = lora + R.a_off[4];
-  v.B_gu = lora + R.b_off[4];
-  v.A_d = lora + R.a_off[6];
-  v.B_d = lora + R.b_off[6];
+  v.lora_on = lora != nullptr;
+  v.A_qkv = v.B_qkv = v.A_o = v.B_o = v.A_gu = v.B_gu = v.A_d = v.B_d = nullptr;
+  if (v.lora_on) {
+    v.A_qkv = lora + R.a_off[0];
+    v.B_qkv = lora + R.b_off[0];
+    v.A_o = lora + R.a_off[3];
+    v.B_o = lora + R.b_off[3];
+    v.A_gu = lora + R.a_off[4];
+    v.B_gu = lora + R.b_off[4];
+    v.A_d = lora + R.a_off[6];
+    v.B_d = lora + R.b_off[6];
+  }
   return v;
 }
 
@@ -291,11 +296,13 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
 }
 
 int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, const void* x,
-                     int batch, int seq, const void* out, LayerShapes* s, const char* who) {
+                     int batch, int seq, const void* out, LayerShapes* s, const char* who,
+                     bool lora_optional = false) {
   LSQ_TRY(layer_shapes(cfg, s));
-  if (!blob || !lora || !x || !out) return set_error(LSQ_ERR_INVALID, "%s: null pointer", who);
+  if (!blob || (!lora && !lora_optional) || !x || !out)
+    return set_error(LSQ_ERR_INVALID, "%s: null pointer", who);
   if (batch <= 0 || seq <= 0) return set_error(LSQ_ERR_SHAPE, "%s: batch and seq must be >= 1", who);
-  if (!aligned16(blob) || !aligned16(lora) || !aligned16(x) || !aligned16(out))
+  if (!aligned16(blob) || (lora && !aligned16(lora)) || !aligned16(x) || !aligned16(out))
     return set_error(LSQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", who);
   return LSQ_OK;
 }
@@ -305,28 +312,28 @@ int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, co
 int forward_core(const LayerShapes& s, const Views& v, const uint16_t* x, int batch, int seq,
                  float theta, float eps, const Buffers& b, uint16_t* x_out, cudaStream_t st) {
   const int64_t T = (int64_t)batch * seq;
-  const int r = s.r;
+  const int r = v.lora_on ? s.r : 0;  // r = 0: no LoRA slab in the GEMMs
   const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
   const int64_t pe2[2] = {s.F, s.gu_n};
   LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, b.rstd1, st));
-  LSQ_TRY(launch_lora_down(b.n1, s.D, v.A_qkv, T, s.D, 3 * r, b.u_qkv, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on) LSQ_TRY(launch_lora_down(b.n1, s.D, v.A_qkv, T, s.D, 3 * r, b.u_qkv, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
                            3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_rope_table(seq, s.hd, theta, b.rope_cs, st));
   LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
-  LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on) LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
                            pe3, x, b.h, s.D),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, b.rstd2, st));
-  LSQ_TRY(launch_lora_down(b.n2, s.D, v.A_gu, T, s.D, 2 * r, b.u_gu, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on) LSQ_TRY(launch_lora_down(b.n2, s.D, v.A_gu, T, s.D, 2 * r, b.u_gu, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
                            2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_swiglu_fwd(b.gu, T, s.F, b.m, st));
-  LSQ_TRY(launch_lora_down(b.m, s.F, v.A_d, T, s.F, r, b.u_d, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on) LSQ_TRY(launch_lora_down(b.m, s.F, v.A_d, T, s.F, r, b.u_d, b.lscratch, b.lscratch_bytes, st));
   if (x_out)
     LSQ_TRY(gemm_run(nf4_fwd(v.codes[6], v.absmax[6], s.D, s.F, b.m, T, v.B_d, r, s.s, b.u_d, r, 1,
                              pe3, b.h, x_out, s.D),
@@ -346,7 +353,8 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
                    int batch, int seq, uint16_t* x_out, void* ws, size_t ws_bytes,
                    cudaStream_t st) {
   LayerShapes s;
-  LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd"));
+  LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd",
+                           true));
   const int64_t T = (int64_t)batch * seq;
   const size_t need = plan_buffers(s, T, nullptr, nullptr);
   if (!ws || ws_bytes < need)

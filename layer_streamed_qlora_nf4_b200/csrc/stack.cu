@@ -19,6 +19,7 @@
 // copy ("ready").  Copies run one visit ahead.  Kernels are deterministic, so
 // a streamed step is bit-identical to the same step with the stack resident.
 #include <chrono>
+#include <cmath>
 #include <thread>
 #include <vector>
 
@@ -38,7 +39,7 @@ struct lsq_stack {
   int buf_layer[2];            // layer held by each buffer (after the enqueued copies)
   std::vector<cudaEvent_t> wait_ev;  // pairs around each compute-side wait (timing)
   cudaEvent_t t_start, t_end, done;
-  float* loss_host;            // pinned
+  float* loss_host;            // pinned: [0] loss, [1 ..] DPO log-probabilities
   lsq_step_stats stats;
   int n_waits_last;
 };
@@ -61,7 +62,14 @@ struct StackWs {
   size_t gemm_bytes;
   void* layer_ws;
   size_t layer_ws_bytes;
+  // DPO step only
+  uint16_t* xr[2];   // [T][D] bf16: the reference (adapter-off) hidden state, ping-pong
+  float* row_ref;    // [T] reference per-row -log p
+  float* seq_scale;  // [2 * pairs] dlogits coefficient per sequence
+  float* logps;      // [4 * pairs]
 };
+
+constexpr int kMaxPairs = 32;
 
 GemmDesc head_fwd(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* hf, int64_t T,
                   float* logits) {
@@ -99,7 +107,8 @@ GemmDesc head_dx(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* 
   return d;
 }
 
-size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* base, StackWs* w) {
+size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* base, StackWs* w,
+                     bool dpo = false) {
   Arena a;
   a.base = static_cast<uint8_t*>(base);
   a.cap = SIZE_MAX;
@@ -123,6 +132,13 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.gemm_bytes = gb + 256;
   x.layer_ws_bytes = layer_ws_bytes(cfg, T);
   x.layer_ws = a.take<uint8_t>(x.layer_ws_bytes);
+  if (dpo) {
+    x.xr[0] = a.take<uint16_t>(T * D);
+    x.xr[1] = a.take<uint16_t>(T * D);
+    x.row_ref = a.take<float>(T);
+    x.seq_scale = a.take<float>(2 * kMaxPairs);
+    x.logps = a.take<float>(4 * kMaxPairs);
+  }
   if (w) *w = x;
   return a.used;
 }
@@ -244,7 +260,7 @@ extern "C" int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_
       (cudaEventCreate(&h->t_start) != cudaSuccess || cudaEventCreate(&h->t_end) != cudaSuccess ||
        cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) != cudaSuccess))
     rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create events");
-  if (rc == LSQ_OK && cudaMallocHost(&h->loss_host, sizeof(float)) != cudaSuccess)
+  if (rc == LSQ_OK && cudaMallocHost(&h->loss_host, (1 + 4 * kMaxPairs) * sizeof(float)) != cudaSuccess)
     rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot allocate the pinned loss slot");
   if (rc != LSQ_OK) {
     delete h;
@@ -277,12 +293,24 @@ extern "C" int stream_stack_last_stats(const lsq_stack* h, lsq_step_stats* out) 
   return LSQ_OK;
 }
 
-extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t micro_batches,
-                                 int32_t batch, int32_t seq, const uint16_t* emb,
-                                 const uint16_t* lm_head, const uint16_t* final_norm, float* lora,
-                                 float* lora_grad, const lsq_adamw* opt, float* loss_out,
-                                 float* logits_out, void* ws, size_t ws_bytes, void* stream,
-                                 int64_t timeout_ms) {
+namespace lsq {
+namespace {
+
+struct DpoArgs {
+  int pairs;
+  float beta;
+  float* logps_out;  // host [4 * pairs] or null
+};
+
+// One optimiser step over the streamed stack: SFT (dpo == null) or DPO.  The
+// DPO step runs the reference (adapter off) forward of each layer right after
+// the policy forward, from the same resident layer buffer, so it reads the
+// stack as often as an SFT step does.
+int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_t batch,
+              int32_t seq, const uint16_t* emb, const uint16_t* lm_head,
+              const uint16_t* final_norm, float* lora, float* lora_grad, const lsq_adamw* opt,
+              float* loss_out, float* logits_out, void* ws, size_t ws_bytes, void* stream,
+              int64_t timeout_ms, const DpoArgs* dpo) {
   if (!h) return set_error(LSQ_ERR_INVALID, "stream_stack_step: null handle");
   if (!tokens || !emb || !lm_head || !final_norm || !lora || !lora_grad || !loss_out)
     return set_error(LSQ_ERR_INVALID, "stream_stack_step: null pointer");
@@ -297,11 +325,11 @@ extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t mi
   const LayerShapes& s = h->shapes;
   const int L = cfg->n_layers;
   const int64_t T = (int64_t)batch * seq, D = s.D, V = cfg->vocab;
-  const size_t need = plan_stack_ws(cfg, s, T, nullptr, nullptr);
+  const size_t need = plan_stack_ws(cfg, s, T, nullptr, nullptr, dpo != nullptr);
   if (!ws || ws_bytes < need)
     return set_error(LSQ_ERR_WORKSPACE, "stream_stack_step: workspace %zu < %zu", ws_bytes, need);
   StackWs w;
-  plan_stack_ws(cfg, s, T, ws, &w);
+  plan_stack_ws(cfg, s, T, ws, &w, dpo != nullptr);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int64_t layer_floats = h->lora_layout.floats_per_layer;
   const float inv_count = 1.f / (float)((double)micro_batches * batch * (seq - 1));
@@ -354,13 +382,29 @@ extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t mi
       LSQ_TRY(layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats, w.xs + (size_t)i * T * D,
                              batch, seq, w.xs + (size_t)(i + 1) * T * D, w.layer_ws,
                              w.layer_ws_bytes, cs));
+      if (dpo)  // reference model: the same layer with its adapter off
+        LSQ_TRY(layer_fwd_impl(cfg, blob, nullptr, i == 0 ? w.xs : w.xr[(i - 1) & 1], batch, seq,
+                               w.xr[i & 1], w.layer_ws, w.layer_ws_bytes, cs));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
     }
     const uint16_t* xL = w.xs + (size_t)L * T * D;
+    if (dpo) {
+      LSQ_TRY(launch_rmsnorm_fwd(w.xr[(L - 1) & 1], final_norm, T, D, cfg->rms_eps, w.hf, w.rstd_f, cs));
+      LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
+      LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_ref, cs));
+    }
     LSQ_TRY(launch_rmsnorm_fwd(xL, final_norm, T, D, cfg->rms_eps, w.hf, w.rstd_f, cs));
     LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
-    LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, inv_count, w.dlogits, w.row_loss, cs));
-    LSQ_TRY(launch_sum_rows(w.row_loss, T, inv_count, mb > 0 ? 1 : 0, w.loss_dev, cs));
+    if (dpo) {
+      LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_loss, cs));
+      LSQ_TRY(launch_dpo_loss(w.row_loss, w.row_ref, dpo->pairs, seq, dpo->beta, w.seq_scale,
+                              w.logps, w.loss_dev, cs));
+      LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, w.dlogits, w.row_loss, cs,
+                                   w.seq_scale));
+    } else {
+      LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, inv_count, w.dlogits, w.row_loss, cs));
+      LSQ_TRY(launch_sum_rows(w.row_loss, T, inv_count, mb > 0 ? 1 : 0, w.loss_dev, cs));
+    }
     LSQ_TRY(gemm_run(head_dx(lm_head, V, D, w.dlogits, T, w.dhf), w.gemm, w.gemm_bytes, cs));
     LSQ_TRY(launch_rmsnorm_bwd(w.dhf, xL, final_norm, w.rstd_f, nullptr, T, D, w.dh[0], w.dhb[0], cs));
     int cur = 0;
@@ -382,6 +426,9 @@ extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t mi
     LSQ_TRY(launch_adamw(lora, lora_grad, opt->m, opt->v, layer_floats * L, opt->lr, opt->beta1,
                          opt->beta2, opt->eps, opt->weight_decay, opt->step, cs));
   LSQ_CUDA(cudaMemcpyAsync(h->loss_host, w.loss_dev, sizeof(float), cudaMemcpyDeviceToHost, cs));
+  if (dpo)
+    LSQ_CUDA(cudaMemcpyAsync(h->loss_host + 1, w.logps, 4 * dpo->pairs * sizeof(float),
+                             cudaMemcpyDeviceToHost, cs));
   LSQ_CUDA(cudaEventRecord(h->t_end, cs));
   LSQ_CUDA(cudaEventRecord(h->done, cs));
   LSQ_TRY(wait_event_timeout(h->done, timeout_ms));
@@ -399,6 +446,8 @@ extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t mi
     h->buf_layer[1] = held[1];
   }
   *loss_out = *h->loss_host;
+  if (dpo && dpo->logps_out)
+    for (int k = 0; k < 4 * dpo->pairs; ++k) dpo->logps_out[k] = h->loss_host[1 + k];
   h->stats.layer_copies = copies;
   h->stats.h2d_bytes = (int64_t)copies * (int64_t)bytes;
   cudaEventElapsedTime(&h->stats.step_ms, h->t_start, h->t_end);
@@ -412,4 +461,40 @@ extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t mi
   }
   h->stats.copy_wait_ms = wait_ms;
   return LSQ_OK;
+}
+
+}  // namespace
+}  // namespace lsq
+
+extern "C" int stream_stack_step(lsq_stack* h, const int32_t* tokens, int32_t micro_batches,
+                                 int32_t batch, int32_t seq, const uint16_t* emb,
+                                 const uint16_t* lm_head, const uint16_t* final_norm, float* lora,
+                                 float* lora_grad, const lsq_adamw* opt, float* loss_out,
+                                 float* logits_out, void* ws, size_t ws_bytes, void* stream,
+                                 int64_t timeout_ms) {
+  return step_impl(h, tokens, micro_batches, batch, seq, emb, lm_head, final_norm, lora, lora_grad,
+                   opt, loss_out, logits_out, ws, ws_bytes, stream, timeout_ms, nullptr);
+}
+
+extern "C" size_t stream_stack_dpo_workspace_bytes(const lsq_cfg* cfg, int32_t pairs, int32_t seq) {
+  LayerShapes s;
+  if (pairs <= 0 || pairs > kMaxPairs || seq <= 0 || layer_shapes(cfg, &s) != LSQ_OK ||
+      cfg->n_layers <= 0 || cfg->vocab <= 0)
+    return 0;
+  return plan_stack_ws(cfg, s, (int64_t)2 * pairs * seq, nullptr, nullptr, true);
+}
+
+extern "C" int stream_stack_dpo_step(lsq_stack* h, const int32_t* tokens, int32_t pairs,
+                                     int32_t seq, float beta, const uint16_t* emb,
+                                     const uint16_t* lm_head, const uint16_t* final_norm,
+                                     float* lora, float* lora_grad, const lsq_adamw* opt,
+                                     float* loss_out, float* logps_out, float* logits_out,
+                                     void* ws, size_t ws_bytes, void* stream, int64_t timeout_ms) {
+  if (pairs <= 0 || pairs > kMaxPairs)
+    return set_error(LSQ_ERR_SHAPE, "stream_stack_dpo_step: pairs must be 1..%d", kMaxPairs);
+  if (!(beta > 0.f) || !std::isfinite(beta))
+    return set_error(LSQ_ERR_INVALID, "stream_stack_dpo_step: beta must be positive and finite");
+  DpoArgs d{pairs, beta, logps_out};
+  return step_impl(h, tokens, 1, 2 * pairs, seq, emb, lm_head, final_norm, lora, lora_grad, opt,
+                   loss_out, logits_out, ws, ws_bytes, stream, timeout_ms, &d);
 }

@@ -25,6 +25,7 @@ EXPORTS = (
     "stream_stack_workspace_bytes", "stream_stack_step", "stream_stack_last_stats",
     "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
+    "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step",
 )
 
 
@@ -106,6 +107,12 @@ _PROTOS = {
                                          ctypes.POINTER(lsq_adamw), ctypes.POINTER(ctypes.c_float),
                                          _P, _P, _SZ, _P, _I64]),
     "stream_stack_last_stats": (ctypes.c_int, [_P, ctypes.POINTER(lsq_step_stats)]),
+    "stream_stack_dpo_workspace_bytes": (_SZ, [ctypes.POINTER(lsq_cfg), _I32, _I32]),
+    "stream_stack_dpo_step": (ctypes.c_int, [_P, _P, _I32, _I32, _F, _P, _P, _P, _P, _P,
+                                             ctypes.POINTER(lsq_adamw),
+                                             ctypes.POINTER(ctypes.c_float),
+                                             ctypes.POINTER(ctypes.c_float), _P, _P, _SZ, _P,
+                                             _I64]),
     "lora_adamw_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(lsq_adamw), _I64, _P]),
     "lsq_launch_counter": (ctypes.c_int64, []),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
@@ -300,6 +307,28 @@ def stream_stack_step(stack, tokens, micro_batches, batch, seq, emb, lm_head, fi
                                     ctypes.byref(loss), _ptr(logits_out), _ptr(ws), ws.numel(),
                                     _stream(stream), timeout_ms))
     return loss.value
+
+
+def stream_stack_dpo_workspace_bytes(cfg, pairs, seq):
+    c = cfg_struct(cfg)
+    return load().stream_stack_dpo_workspace_bytes(ctypes.byref(c), pairs, seq)
+
+
+def stream_stack_dpo_step(stack, tokens, pairs, seq, beta, emb, lm_head, final_norm, lora,
+                          lora_grad, opt, ws, logits_out=None, timeout_ms=600000, stream=None):
+    """tokens: int32 device [pairs, 2, seq] (chosen, rejected).  Returns (loss, logps) with
+    logps a list of (policy chosen, policy rejected, reference chosen, reference rejected)
+    per pair."""
+    loss = ctypes.c_float(0.0)
+    lp = (ctypes.c_float * (4 * pairs))()
+    o = _adamw_struct(opt) if opt is not None else None
+    _check(load().stream_stack_dpo_step(stack.handle, _ptr(tokens), pairs, seq, beta, _ptr(emb),
+                                        _ptr(lm_head), _ptr(final_norm), _ptr(lora),
+                                        _ptr(lora_grad),
+                                        ctypes.byref(o) if o is not None else None,
+                                        ctypes.byref(loss), lp, _ptr(logits_out), _ptr(ws),
+                                        ws.numel(), _stream(stream), timeout_ms))
+    return loss.value, [tuple(lp[4 * p: 4 * p + 4]) for p in range(pairs)]
 
 
 def stream_stack_last_stats(stack):

@@ -96,6 +96,10 @@ def test_workspace_queries_are_host_only(L):
     assert L.decoder_layer_workspace_bytes(synth.LLAMA8B, 1, 512) > 0
     assert L.stream_stack_workspace_bytes(synth.LLAMA8B, 1, 512) > 0
     assert L.nf4_lora_linear_workspace_bytes(0, 1024, 1024, 16) == 0
+    assert L.stream_stack_dpo_workspace_bytes(synth.LLAMA8B, 2, 512) > \
+        L.stream_stack_workspace_bytes(synth.LLAMA8B, 4, 512)
+    assert L.stream_stack_dpo_workspace_bytes(synth.LLAMA8B, 0, 512) == 0
+    assert L.stream_stack_dpo_workspace_bytes(synth.LLAMA8B, 33, 512) == 0
 
 
 def test_invalid_arguments_are_rejected_without_a_gpu(L):
