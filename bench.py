@@ -34,6 +34,12 @@ WORKLOAD = ("Llama-3.1-8B-shaped 32-layer NF4 stack (block 64, fp32 absmax) stre
             "lm_head (vocab 128256) resident; batch 1 x seq 512 per GPU; one SFT step "
             "(cross-entropy + AdamW on LoRA r16 alpha32, all 7 projections)")
 BATCH, SEQ = 1, 512
+METRIC_QWEN = ("streamed LoRA train tokens/sec (Qwen2.5-3B shapes, bf16 base, seq 2048) and % of "
+               "step roofline")
+WORKLOAD_QWEN = ("Qwen2.5-3B-shaped 36-layer stack, unquantised bf16 weights (154.1 MB per "
+                 "layer), streamed from pinned host memory through two VRAM layer buffers; bf16 "
+                 "tied embedding / lm_head (vocab 151936) resident; batch 8 x seq 2048 per GPU; "
+                 "one SFT step (cross-entropy + AdamW on LoRA r64 alpha128, all 7 projections)")
 FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
 
 
@@ -66,7 +72,12 @@ def parse():
                     help="32: fp32 absmax per NF4 block (the default workload); 8: the absmax "
                          "double-quantised to 8 bits with one fp32 scale per 256 blocks, the "
                          "pages' 113 MB layers / 3.60 GB store")
-    ap.add_argument("--batch", type=int, default=1, help="sequences per micro-batch (SFT step)")
+    ap.add_argument("--model", choices=("llama8b", "qwen3b"), default="llama8b",
+                    help="llama8b: the 32-layer Llama-3.1-8B-shaped NF4 stack, seq 512 (default); "
+                         "qwen3b: the 36-layer Qwen2.5-3B-shaped stack streamed unquantised "
+                         "(bf16), tied embedding, LoRA r64, batch 8 x seq 2048")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per micro-batch (SFT step; default 1, or 8 for qwen3b)")
     ap.add_argument("--micro-batches", type=int, default=1,
                     help="gradient-accumulation micro-batches per optimiser step (SFT step)")
     ap.add_argument("--pairs", type=int, default=2, help="chosen/rejected pairs (DPO step)")
@@ -202,7 +213,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
-def build_stack(L, cfg, rank, tok_shape=(1, SEQ)):
+def build_stack(L, cfg, rank, tok_shape=(1, SEQ), tied=False):
     import torch
     from layer_streamed_qlora_nf4_b200 import pack, synth
     lay = L.lsq_layer_layout_get(cfg)
@@ -223,7 +234,8 @@ def build_stack(L, cfg, rank, tok_shape=(1, SEQ)):
     B = {p: torch.randn(shapes[p][0], r, generator=g, device="cuda") * 0.01 for p in synth.PROJ}
     lora = torch.cat([pack.lora_block(cfg, A, B) for _ in range(cfg["n_layers"])])
     emb = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
-    head = (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
+    head = emb if tied else \
+        (torch.randn(cfg["vocab"], cfg["hidden"], generator=g, device="cuda") * 0.02).bfloat16()
     gt = torch.Generator(device="cuda").manual_seed(1000 + rank)
     tokens = torch.randint(0, cfg["vocab"], (8,) + tuple(tok_shape), generator=gt, device="cuda",
                            dtype=torch.int32)
@@ -261,12 +273,15 @@ def run_ours(args):
     from layer_streamed_qlora_nf4_b200 import lib as L
     from layer_streamed_qlora_nf4_b200 import synth
     L.load()
-    cfg = dict(synth.LLAMA8B, absmax_bits=args.absmax_bits)
+    qwen = args.model == "qwen3b"
+    cfg = synth.QWEN3B if qwen else dict(synth.LLAMA8B, absmax_bits=args.absmax_bits)
+    SEQ = 2048 if qwen else globals()["SEQ"]
     dpo = args.case == "dpo"
-    batch, mbs = (2 * args.pairs, 1) if dpo else (args.batch, args.micro_batches)
+    batch = args.batch if args.batch is not None else (8 if qwen else 1)
+    batch, mbs = (2 * args.pairs, 1) if dpo else (batch, args.micro_batches)
     tok_shape = (args.pairs, 2, SEQ) if dpo else (mbs, batch, SEQ)
     tokens_per_step = mbs * batch * SEQ
-    st = build_stack(L, cfg, rank, tok_shape)
+    st = build_stack(L, cfg, rank, tok_shape, tied=qwen)
     lay = st["lay"]
     handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
     ws_bytes = (L.stream_stack_dpo_workspace_bytes(cfg, args.pairs, SEQ) if dpo
@@ -388,18 +403,19 @@ def run_ours(args):
                               for k, e in prof.items()})
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not dpo and tokens_per_step == SEQ:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not dpo and not qwen
+            and tokens_per_step == SEQ):
         s, desc = oracle_sample(seed=1)
         cpu = dict(value=BATCH * SEQ / s, unit="tokens/s", cores=cpu_threads(), kind="oracle",
                    sample=desc)
     handle.close()
     if rank == 0:
-        line = dict(metric=METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
+        line = dict(metric=METRIC_QWEN if qwen else METRIC, value=value, unit="tokens/s", n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak",
                     vs_baseline=None, dtype="bf16", data="synthetic (seeded random weights and "
                     "uniform token ids at the 8B shapes)",
-                    config=dict(workload=workload_name(args.absmax_bits, dpo, args.pairs, batch,
-                                                       mbs),
+                    config=dict(workload=WORKLOAD_QWEN if qwen else
+                                workload_name(args.absmax_bits, dpo, args.pairs, batch, mbs),
                                 global_batch=world * tokens_per_step // SEQ, seq_len=SEQ,
                                 parallelism="dp%d" % world,
                                 l2="inputs larger than L2: %.2f GB of layer bytes stream per step"

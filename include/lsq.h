@@ -80,6 +80,11 @@ int lsq_nf4_codebook(float out_levels[16]);
 int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block, uint8_t* codes,
                  float* absmax, void* stream);
 
+/* lsq_bf16_from_f32 - round fp32 to bf16 (nearest, ties to even): the storage
+ * of an unquantised frozen weight.  x device fp32 [n], y device uint16 [n].
+ * Asynchronous. */
+int lsq_bf16_from_f32(const float* x, int64_t n, uint16_t* y, void* stream);
+
 /* nf4_dequantize - w~ = fl32(level[code] * absmax) into fp32 W_out [N, K].
  * Same layouts and constraints as nf4_quantize; asynchronous. */
 int nf4_dequantize(const uint8_t* codes, const float* absmax, int64_t N, int64_t K,
@@ -159,6 +164,9 @@ typedef struct lsq_cfg {
   float rms_eps;       /* RMSNorm epsilon */
   int32_t absmax_bits; /* 0 or 32: fp32 absmax per block; 8: 8-bit absmax with one
                           fp32 scale per 256 blocks (nf4_absmax_quantize8) */
+  int32_t weight_bits; /* 0 or 4: NF4 frozen weights; 16: unquantised bf16 weights
+                          (the streamed bf16 stacks of the Layer Streaming blog, e.g.
+                          Qwen2.5-3B); absmax_bits is then ignored */
 } lsq_cfg;
 
 /* Byte layout of one layer's blob (the unit that is streamed).  Projection
@@ -167,7 +175,9 @@ typedef struct lsq_cfg {
  * or uint8 with absmax_bits = 8, then all their fp32 scale arrays); then the
  * two RMSNorm gains (bf16 [D]).  Every section starts 256-byte aligned.  For
  * Llama-3.1-8B shapes a layer is 122,699,776 bytes with fp32 absmax and
- * 112,529,408 bytes (the pages' 113 MB; 3.60 GB for 32 layers) with 8-bit. */
+ * 112,529,408 bytes (the pages' 113 MB; 3.60 GB for 32 layers) with 8-bit.
+ * With weight_bits = 16, codes_off[p] is the offset of the bf16 weight [N, K]
+ * (row-major, back to back) and there are no absmax arrays. */
 typedef struct lsq_layer_layout {
   uint64_t codes_off[7];
   uint64_t absmax_off[7];   /* fp32 [N*K/64], or uint8 [N*K/64] with absmax_bits 8 */
@@ -175,8 +185,8 @@ typedef struct lsq_layer_layout {
   int64_t rows[7], cols[7]; /* N, K of each projection */
   uint64_t bytes;           /* total blob size (multiple of 256) */
   uint64_t scale_off[7];    /* absmax_bits 8: fp32 [N*K/64/256]; else 0 */
-  int32_t absmax_bits;      /* 32 or 8 */
-  int32_t pad;
+  int32_t absmax_bits;      /* 32 or 8 (NF4 only) */
+  int32_t weight_bits;      /* 4 or 16 */
 } lsq_layer_layout;
 
 /* Fills *out for cfg.  Host only.  LSQ_ERR_SHAPE unless D, F, H*d, Hkv*d are

@@ -627,3 +627,10 @@ int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st) {
 }
 
 }  // namespace lsq
+
+extern "C" int lsq_bf16_from_f32(const float* x, int64_t n, uint16_t* y, void* stream) {
+  using namespace lsq;
+  if (n <= 0) return set_error(LSQ_ERR_SHAPE, "lsq_bf16_from_f32: n must be positive");
+  if (!x || !y) return set_error(LSQ_ERR_INVALID, "lsq_bf16_from_f32: null pointer");
+  return launch_f32_to_bf16(x, n, y, static_cast<cudaStream_t>(stream));
+}

@@ -794,12 +794,13 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
     const double M = (double)d.M, T = (double)d.T, K = (double)d.Kc;
     const double flops = 2.0 * M * T * (K + d.slab_w);
     const bool nf4 = d.wmode == W_NF4_N || d.wmode == W_NF4_T;
-    const double wbytes = nf4 ? M * K * (0.5 + 4.0 / 64.0) : 2.0 * M * K;
+    const double am_bytes = d.absmax_q ? 1.0 / 64.0 + 4.0 / (64.0 * 256.0) : 4.0 / 64.0;
+    const double wbytes = nf4 ? M * K * (0.5 + am_bytes) : 2.0 * M * K;
     const double bytes = wbytes + 2.0 * T * K + T * M * (d.out_f32 ? 4.0 : 2.0) +
                          (d.residual ? 2.0 * T * M : 0.0);
-    static const char* names[4] = {"gemm_nf4_fwd", "gemm_nf4_dx", "gemm_bf16_head",
-                                   "gemm_bf16_head_dx"};
-    prof_end(prof, st, names[d.wmode], flops, bytes);
+    static const char* names[4] = {"gemm_nf4_fwd", "gemm_nf4_dx", "gemm_bf16_fwd",
+                                   "gemm_bf16_dx"};
+    prof_end(prof, st, d.prof_name ? d.prof_name : names[d.wmode], flops, bytes);
   }
   return LSQ_OK;
 }

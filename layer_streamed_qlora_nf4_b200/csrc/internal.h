@@ -94,6 +94,7 @@ struct GemmDesc {
   const uint16_t* residual = nullptr;
   int64_t ldr = 0;
   int force_splits = 0;             // 0 = heuristic
+  const char* prof_name = nullptr;  // profiler class (default: by operand mode)
 };
 size_t gemm_workspace_bytes(const GemmDesc& d);
 int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st);
@@ -168,6 +169,7 @@ struct LayerShapes {
   int H, Hkv, hd, r;
   float s;
   int absmax_bits;  // 32 or 8
+  int weight_bits;  // 4 (NF4) or 16 (bf16)
 };
 int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);

@@ -15,6 +15,8 @@ int layer_shapes(const lsq_cfg* cfg, LayerShapes* o) {
   if (!cfg) return set_error(LSQ_ERR_INVALID, "null config");
   if (cfg->absmax_bits != 0 && cfg->absmax_bits != 32 && cfg->absmax_bits != 8)
     return set_error(LSQ_ERR_INVALID, "cfg.absmax_bits must be 0, 32 or 8");
+  if (cfg->weight_bits != 0 && cfg->weight_bits != 4 && cfg->weight_bits != 16)
+    return set_error(LSQ_ERR_INVALID, "cfg.weight_bits must be 0, 4 or 16");
   if (cfg->block != 64) return set_error(LSQ_ERR_SHAPE, "cfg.block must be 64");
   if (cfg->head_dim != 64 && cfg->head_dim != 128)
     return set_error(LSQ_ERR_SHAPE, "cfg.head_dim must be 64 or 128");
@@ -45,15 +47,17 @@ int layer_shapes(const lsq_cfg* cfg, LayerShapes* o) {
   // and columns are multiples of 128), so a scale run never straddles two
   // projections and the stacked q|k|v and gate|up matrices index one array.
   o->absmax_bits = cfg->absmax_bits == 8 ? 8 : 32;
+  o->weight_bits = cfg->weight_bits == 16 ? 16 : 4;
   return LSQ_OK;
 }
 
 namespace {
 
-struct AbsmaxRef {  // fp32 absmax, or 8-bit absmax with its run scales
+struct AbsmaxRef {  // fp32 absmax, or 8-bit absmax with its run scales; or a bf16 weight
   const float* f32 = nullptr;
   const uint8_t* q = nullptr;
   const float* s = nullptr;
+  bool bf16 = false;  // the weight is unquantised bf16 (no absmax)
 };
 
 struct Views {  // pointers into one layer blob / one LoRA block
@@ -69,23 +73,26 @@ void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) 
   const int64_t rows[7] = {s.qd, s.kvd, s.kvd, s.D, s.F, s.F, s.D};
   const int64_t cols[7] = {s.D, s.D, s.D, s.qd, s.D, s.D, s.F};
   uint64_t off = 0;
+  const bool bf16 = s.weight_bits == 16;
   for (int p = 0; p < 7; ++p) {
     L->rows[p] = rows[p];
     L->cols[p] = cols[p];
     L->codes_off[p] = off;
-    off += (uint64_t)rows[p] * cols[p] / 2;
+    off += (uint64_t)rows[p] * cols[p] * (bf16 ? 2 : 1) / (bf16 ? 1 : 2);
   }
   off = (off + 255) & ~uint64_t(255);
   L->absmax_bits = s.absmax_bits;
-  L->pad = 0;
+  L->weight_bits = s.weight_bits;
   for (int p = 0; p < 7; ++p) {
+    L->absmax_off[p] = 0;
+    if (bf16) continue;
     L->absmax_off[p] = off;
     off += (uint64_t)rows[p] * cols[p] / 64 * (s.absmax_bits == 8 ? 1 : 4);
   }
   off = (off + 255) & ~uint64_t(255);
   for (int p = 0; p < 7; ++p) {
     L->scale_off[p] = 0;
-    if (s.absmax_bits == 8) {
+    if (!bf16 && s.absmax_bits == 8) {
       L->scale_off[p] = off;
       off += ((uint64_t)rows[p] * cols[p] / 64 + 255) / 256 * 4;
     }
@@ -127,7 +134,9 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
   const uint8_t* b = static_cast<const uint8_t*>(blob);
   for (int p = 0; p < 7; ++p) {
     v.codes[p] = b + L.codes_off[p];
-    if (s.absmax_bits == 8) {
+    if (s.weight_bits == 16) {
+      v.absmax[p].bf16 = true;
+    } else if (s.absmax_bits == 8) {
       v.absmax[p].q = b + L.absmax_off[p];
       v.absmax[p].s = reinterpret_cast<const float*>(b + L.scale_off[p]);
     } else {
@@ -163,12 +172,15 @@ struct Buffers {
   size_t gemm_bytes;
 };
 
+// Forward of a stacked frozen weight W [N, K] (NF4, or bf16 when absmax is
+// empty): out [T, N] = act W^T + s u B^T (+ residual).
 GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
                  const uint16_t* act, int64_t T, const float* B, int r, float s, const float* u,
                  int64_t u_ld, int n_parts, const int64_t* pe, const uint16_t* res, void* out,
                  int64_t ldo) {
   GemmDesc d;
-  d.wmode = W_NF4_N;
+  const bool bf16 = absmax.bf16;
+  d.wmode = bf16 ? W_BF16_N : W_NF4_N;
   d.M = N;
   d.T = T;
   d.Kc = K;
@@ -202,7 +214,8 @@ GemmDesc nf4_dx(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_
                 const uint16_t* dy, int64_t T, const float* A, int R, float s, const float* v,
                 void* out, int out_f32) {
   GemmDesc d;
-  d.wmode = W_NF4_T;
+  const bool bf16 = absmax.bf16;
+  d.wmode = bf16 ? W_BF16_T : W_NF4_T;
   d.M = K;
   d.T = T;
   d.Kc = N;

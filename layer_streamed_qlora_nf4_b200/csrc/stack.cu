@@ -86,6 +86,7 @@ GemmDesc head_fwd(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t*
   d.out = logits;
   d.out_f32 = 1;
   d.ldo = V;
+  d.prof_name = "gemm_bf16_head";
   return d;
 }
 
@@ -104,6 +105,7 @@ GemmDesc head_dx(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* 
   d.out = dhf;
   d.out_f32 = 1;
   d.ldo = D;
+  d.prof_name = "gemm_bf16_head_dx";
   return d;
 }
 

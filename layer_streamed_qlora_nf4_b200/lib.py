@@ -25,7 +25,7 @@ EXPORTS = (
     "stream_stack_workspace_bytes", "stream_stack_step", "stream_stack_last_stats",
     "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
-    "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step",
+    "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
 )
 
 
@@ -41,7 +41,8 @@ class lsq_cfg(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("lora_r", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("lora_alpha", ctypes.c_float), ("rope_theta", ctypes.c_float),
-                ("rms_eps", ctypes.c_float), ("absmax_bits", ctypes.c_int32)]
+                ("rms_eps", ctypes.c_float), ("absmax_bits", ctypes.c_int32),
+                ("weight_bits", ctypes.c_int32)]
 
 
 class lsq_layer_layout(ctypes.Structure):
@@ -49,7 +50,7 @@ class lsq_layer_layout(ctypes.Structure):
                 ("g1_off", ctypes.c_uint64), ("g2_off", ctypes.c_uint64),
                 ("rows", ctypes.c_int64 * 7), ("cols", ctypes.c_int64 * 7),
                 ("bytes", ctypes.c_uint64), ("scale_off", ctypes.c_uint64 * 7),
-                ("absmax_bits", ctypes.c_int32), ("pad", ctypes.c_int32)]
+                ("absmax_bits", ctypes.c_int32), ("weight_bits", ctypes.c_int32)]
 
 
 class lsq_lora_layout(ctypes.Structure):
@@ -84,6 +85,7 @@ _PROTOS = {
     "nf4_quantize": (ctypes.c_int, [_P, _I64, _I64, _I32, _P, _P, _P]),
     "nf4_dequantize": (ctypes.c_int, [_P, _P, _I64, _I64, _I32, _P, _P]),
     "nf4_absmax_quantize8": (ctypes.c_int, [_P, _I64, _P, _P, _P]),
+    "lsq_bf16_from_f32": (ctypes.c_int, [_P, _I64, _P, _P]),
     "nf4_dequantize_dq": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I32, _P, _P]),
     "nf4_lora_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I32]),
     "nf4_lora_linear_fwd": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _F,
@@ -166,7 +168,8 @@ def cfg_struct(cfg):
                    head_dim=cfg["head_dim"], n_layers=cfg["n_layers"], lora_r=cfg["lora_r"],
                    block=cfg["block"], lora_alpha=cfg["lora_alpha"],
                    rope_theta=cfg["rope_theta"], rms_eps=cfg["rms_eps"],
-                   absmax_bits=cfg.get("absmax_bits", 32))
+                   absmax_bits=cfg.get("absmax_bits", 32),
+                   weight_bits=cfg.get("weight_bits", 4))
 
 
 # ------------------------------------------------------------------ entry points
@@ -194,6 +197,10 @@ def nf4_quantize(W, codes, absmax, block=64, stream=None):
 def nf4_dequantize(codes, absmax, N, K, W_out, block=64, stream=None):
     _check(load().nf4_dequantize(_ptr(codes), _ptr(absmax), N, K, block, _ptr(W_out),
                                  _stream(stream)))
+
+
+def lsq_bf16_from_f32(x, y, stream=None):
+    _check(load().lsq_bf16_from_f32(_ptr(x), x.numel(), _ptr(y), _stream(stream)))
 
 
 def nf4_absmax_quantize8(absmax, q, scale, stream=None):

@@ -4,7 +4,8 @@
 library's ``nf4_quantize`` (the offline NF4 shard step of the Soup layer-streaming
 tutorial, "四段資料路徑" part 1), writing at the offsets ``lsq_layer_layout_get``
 returns (with an 8-bit absmax, ``nf4_absmax_quantize8`` then stores the absmax
-in 8 bits), and copies the two RMSNorm gains.  ``lora_block`` places the fp32 LoRA
+in 8 bits; an unquantised bf16 stack stores each weight with ``lsq_bf16_from_f32``),
+and copies the two RMSNorm gains.  ``lora_block`` places the fp32 LoRA
 masters at the offsets of ``lsq_lora_layout_get``.  No arithmetic happens here.
 """
 import torch
@@ -23,6 +24,10 @@ def pack_layer(cfg, W, g1, g2, blob, stream=None):
         N, K = lay.rows[p], lay.cols[p]
         w = W[name]
         assert tuple(w.shape) == (N, K) and w.dtype == torch.float32 and w.is_contiguous()
+        if lay.weight_bits == 16:     # unquantised: the weight stored as bf16
+            wb = blob[lay.codes_off[p]: lay.codes_off[p] + N * K * 2].view(torch.int16)
+            lib.lsq_bf16_from_f32(w, wb, stream=stream)
+            continue
         codes = blob[lay.codes_off[p]: lay.codes_off[p] + N * K // 2]
         nb = N * K // 64
         if lay.absmax_bits == 8:

@@ -22,6 +22,13 @@ LLAMA8B = dict(hidden=4096, ffn=14336, n_heads=32, n_kv_heads=8, head_dim=128,
                n_layers=32, vocab=128256, rope_theta=500000.0, rms_eps=1e-5,
                lora_r=16, lora_alpha=32.0, block=64)
 
+# Qwen2.5-3B shapes, streamed unquantised (bf16 weights), tied embedding, LoRA
+# r 64 on all seven projections.  RoPE base and RMSNorm epsilon are the Qwen2.5
+# family's published values; QKV biases are left out (the layer has none).
+QWEN3B = dict(hidden=2048, ffn=11008, n_heads=16, n_kv_heads=2, head_dim=128,
+              n_layers=36, vocab=151936, rope_theta=1000000.0, rms_eps=1e-6,
+              lora_r=64, lora_alpha=128.0, block=64, weight_bits=16)
+
 # Small Llama-shaped configs for oracle-sized parity cases (same structure,
 # several GEMM tiles plus ragged tails).
 SMALL = dict(hidden=512, ffn=1408, n_heads=8, n_kv_heads=2, head_dim=64,

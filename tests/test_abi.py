@@ -91,6 +91,20 @@ def test_layer_layout_with_8bit_absmax_gives_the_pages_store_size(L):
         L.lsq_layer_layout_get(dict(synth.LLAMA8B, absmax_bits=16))
 
 
+def test_layer_layout_of_the_bf16_stack(L):
+    # Qwen2.5-3B shapes streamed unquantised: 77,070,336 bf16 weights + two gains per layer
+    lay = L.lsq_layer_layout_get(synth.QWEN3B)
+    assert lay.weight_bits == 16
+    assert lay.bytes == 2 * 77070336 + 2 * 2048 * 2 == 154148864
+    shapes = synth.proj_shapes(synth.QWEN3B)
+    for p, name in enumerate(synth.PROJ):
+        assert (lay.rows[p], lay.cols[p]) == shapes[name] and lay.absmax_off[p] == 0
+        if p + 1 < 7:
+            assert lay.codes_off[p + 1] == lay.codes_off[p] + 2 * shapes[name][0] * shapes[name][1]
+    with pytest.raises(L.LsqError):
+        L.lsq_layer_layout_get(dict(synth.QWEN3B, weight_bits=8))
+
+
 def test_workspace_queries_are_host_only(L):
     assert L.nf4_lora_linear_workspace_bytes(128, 1024, 1024, 16) > 0
     assert L.decoder_layer_workspace_bytes(synth.LLAMA8B, 1, 512) > 0

@@ -18,8 +18,11 @@ def L():
     return lib
 
 
-def _oracle_weight(W, absmax_bits):
-    """The weight the layer sees: NF4 with fp32 absmax, or with the 8-bit absmax."""
+def _oracle_weight(W, absmax_bits, weight_bits=4):
+    """The weight the layer sees: NF4 with fp32 absmax, or with the 8-bit absmax, or
+    the weight rounded to bf16 (an unquantised stack)."""
+    if weight_bits == 16:
+        return synth.bf16_bits_to_f32(synth.to_bf16_bits(W))
     N, K = W.shape
     codes, am = onf4.quantize(W)
     if absmax_bits == 8:
@@ -28,7 +31,8 @@ def _oracle_weight(W, absmax_bits):
 
 
 def _oracle_params(lw, cfg):
-    W = {p: _oracle_weight(lw["W"][p], cfg.get("absmax_bits", 32)) for p in synth.PROJ}
+    W = {p: _oracle_weight(lw["W"][p], cfg.get("absmax_bits", 32), cfg.get("weight_bits", 4))
+         for p in synth.PROJ}
     return dict(W=W, A=lw["A"], B=lw["B"], g1=synth.bf16_bits_to_f32(lw["g1"]),
                 g2=synth.bf16_bits_to_f32(lw["g2"]))
 
@@ -131,3 +135,9 @@ def test_layer_rejects_bad_config(L):
 def test_layer_small_absmax8(L):
     # the 8-bit double-quantised absmax, dequantised inside the GEMM operand stage
     _run_layer(L, dict(synth.SMALL, absmax_bits=8), batch=2, seq=100, seed=17)
+
+
+def test_layer_small_bf16_weights_rank64(L):
+    # an unquantised (bf16) stack's layer, LoRA rank 64 (the Qwen2.5-3B configuration)
+    cfg = dict(synth.SMALL, weight_bits=16, lora_r=64, lora_alpha=128.0)
+    _run_layer(L, cfg, batch=2, seq=100, seed=19)

@@ -26,7 +26,7 @@ def L():
 class Stack:
     """Host-generated small stack, packed on the device, pinned copies for streaming."""
 
-    def __init__(self, L, cfg, seed):
+    def __init__(self, L, cfg, seed, tied=False):
         import torch
         from gpu_util import dev, dev_bf16
         from layer_streamed_qlora_nf4_b200 import pack
@@ -34,6 +34,8 @@ class Stack:
         nl = cfg["n_layers"]
         self.lw = [synth.layer_weights(seed + 100 + i, cfg) for i in range(nl)]
         emb, head = synth.embeddings(seed + 1, cfg["vocab"], cfg["hidden"])
+        if tied:                       # one matrix is both the embedding and the lm_head
+            head = emb
         self.emb_bits, self.head_bits = emb, head
         self.gf_bits = synth.to_bf16_bits(np.ones(cfg["hidden"], np.float32))
         lay = L.lsq_layer_layout_get(cfg)
@@ -60,6 +62,9 @@ class Stack:
             W = {}
             for p in synth.PROJ:
                 N, K = lw["W"][p].shape
+                if self.cfg.get("weight_bits", 4) == 16:
+                    W[p] = synth.bf16_bits_to_f32(synth.to_bf16_bits(lw["W"][p]))
+                    continue
                 codes, am = onf4.quantize(lw["W"][p])
                 if bits == 8:
                     W[p] = onf4.dequantize_dq(codes, *onf4.quantize_absmax8(am), N, K)
@@ -102,6 +107,28 @@ def test_stack_matches_oracle(L, small):
 
 def test_stack_absmax8_matches_oracle(L, small8):
     _check_against_oracle(L, small8)
+
+
+@pytest.fixture(scope="module")
+def small_bf16(L):
+    # unquantised bf16 stack, tied embedding, LoRA rank 64 (Qwen2.5-3B-style)
+    return Stack(L, dict(synth.SMALL, weight_bits=16, lora_r=64, lora_alpha=128.0), 7, tied=True)
+
+
+def test_stack_bf16_tied_matches_oracle(L, small_bf16):
+    _check_against_oracle(L, small_bf16)
+
+
+def test_stack_bf16_streamed_equals_resident_bitwise(L, small_bf16):
+    import torch
+    tokens = synth.tokens(35, 2, 64, small_bf16.cfg["vocab"])
+    hs = small_bf16.handle(L, resident=False)
+    hr = small_bf16.handle(L, resident=True)
+    ls, lgs, gs, _ = _step(L, small_bf16, hs, tokens, 1, 2, 64)
+    lr_, lgr, gr, _ = _step(L, small_bf16, hr, tokens, 1, 2, 64)
+    hs.close()
+    hr.close()
+    assert ls == lr_ and torch.equal(lgs, lgr) and torch.equal(gs, gr)
 
 
 def test_stack_absmax8_streamed_equals_resident_bitwise(L, small8):
