@@ -1,25 +1,28 @@
-// LoRA rank-r products around the fused NF4 GEMM (CUDA cores, fp32).
+// LoRA rank-r products around the fused NF4 GEMM (tensor cores, mma.sync).
 //
 // For y = x W^T + s (x A^T) B^T (Soup layer-streaming tutorial, "四段資料路徑"
 // part 1) and its backward (part 3): u = x A^T (forward), v = dY B, and the
 // trainable gradients dA = s v^T x, dB = s dY^T u.  All four are "tall x
-// skinny" products: C[m, n] = sum_k P(m, k) Q(k, n) with n spanning at most a
-// few r = 16 columns, P a bf16 activation and Q an fp32 LoRA tensor.
+// skinny" products: C[m, n] = sum_k P(m, k) Q(k, n) with n spanning at most
+// 3 r <= 192 columns, P a bf16 activation and Q an fp32 LoRA tensor.
 //
-// One tiled kernel serves all four: a CTA owns 64 rows x BN columns of C over
-// one slice of the reduction; bf16 P and fp32 Q tiles are staged through shared
-// memory with coalesced loads along whichever index is contiguous in memory,
-// each thread keeps a 4 x (BN/16) register tile, and the slices are summed by
-// a second kernel in a fixed order - so results are deterministic (no atomics)
-// and keep fp32 precision end to end.
+// One kernel serves all four.  A CTA owns 128 rows x BN columns of C over one
+// slice of the reduction; P tiles arrive by cp.async (16-byte chunks along
+// whichever index is contiguous in memory; ldmatrix, transposing where P's rows
+// are the contiguous index, gives the A fragments), and each fp32 Q tile is
+// split into two bf16 tiles, hi = bf16(q) and lo = bf16(q - hi), so that the
+// two m16n8k16 products P hi + P lo carry about 16 bits of q: with P exact in
+// bf16 and fp32 accumulation the products keep close to fp32 accuracy.  The
+// slices are summed by a second kernel in a fixed order, so results are
+// deterministic (no atomics).
 #include "common.cuh"
 
 namespace lsq {
 
 namespace {
 
-constexpr int kBM = 64;   // rows of C per CTA
-constexpr int kBK = 32;   // reduction elements per smem tile
+constexpr int kBM = 128;  // rows of C per CTA
+constexpr int kBK = 32;   // reduction elements per stage
 constexpr int kThreads = 256;
 
 struct SkinnyArgs {
@@ -32,87 +35,217 @@ struct SkinnyArgs {
   float* part;         // [splits][M][N]
 };
 
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Shared-memory tiles per stage (bf16, rows padded by 8 elements so that the
+// eight 16-byte rows an ldmatrix reads fall in distinct banks):
+//   P_RED: P as [kBM m][kBK + 8]   else P as [kBK k][kBM + 8]
+//   Q hi and lo as [BN n][kBK + 8]
+template <bool P_RED>
+__host__ __device__ constexpr int p_stage_elems() {
+  return P_RED ? kBM * (kBK + 8) : kBK * (kBM + 8);
+}
+template <int BN>
+__host__ __device__ constexpr int q_stage_elems() {
+  return BN * (kBK + 8);
+}
+template <bool P_RED, int BN>
+constexpr size_t skinny_smem_bytes() {
+  return 2 * (size_t)(p_stage_elems<P_RED>() + 2 * q_stage_elems<BN>()) * 2;
+}
+
 // P_RED: the reduction index is the contiguous one in P (else the row index m is).
 // Q_RED: the reduction index is the contiguous one in Q (else the column n is).
 template <bool P_RED, bool Q_RED, int BN>
 __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
-  __shared__ float Ps[kBK][kBM + 4];
-  __shared__ float Qs[kBK][BN + 4];
-  constexpr int TN = BN / 16;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
+  extern __shared__ __align__(16) uint16_t sk_smem[];
+  constexpr int PE = p_stage_elems<P_RED>(), QE = q_stage_elems<BN>();
+  uint16_t* Ps = sk_smem;        // [2][PE]
+  uint16_t* Qh = Ps + 2 * PE;    // [2][QE]
+  uint16_t* Ql = Qh + 2 * QE;    // [2][QE]
+  constexpr int WN = BN / 2;     // columns per warp (warps: 4 along m x 2 along n)
+  constexpr int NF = WN / 8;     // n8 fragments per warp
+  constexpr int QV = BN * kBK / 4 / kThreads;  // float4 of Q per thread per stage
+  static_assert(QV >= 1 && (BN * kBK / 4) % kThreads == 0, "Q tile split");
+  static_assert(NF % 2 == 0, "B fragments are loaded in pairs");
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp & 3, wn = warp >> 2;
   const int64_t m0 = (int64_t)blockIdx.x * kBM;
   const int64_t n0 = (int64_t)blockIdx.y * BN;
-  const int z = blockIdx.z;
-  const int64_t k_begin = (int64_t)z * a.k_per_split;
+  const int64_t k_begin = (int64_t)blockIdx.z * a.k_per_split;
   const int64_t k_end = min(a.K, k_begin + a.k_per_split);
-  float acc[4][TN];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
 
-  for (int64_t kb = k_begin; kb < k_end; kb += kBK) {
-    // stage P tile (64 x 32) -> Ps[k][m]
+  float acc[2][NF][4];
 #pragma unroll
-    for (int it = 0; it < (kBM * kBK) / kThreads; ++it) {
-      const int idx = tid + it * kThreads;
-      int mm, kk;
-      if (P_RED) {
-        mm = idx / kBK;
-        kk = idx % kBK;
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < NF; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+
+  // ---- P tile of the stage starting at kb: 512 chunks of 8 bf16 (two per thread)
+  auto load_p = [&](int st, int64_t kb) {
+    uint16_t* dst = Ps + st * PE;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + i * kThreads;
+      if (P_RED) {  // row m, 4 chunks of k per row
+        const int mm = c >> 2, kc = (c & 3) * 8;
+        const int64_t m = m0 + mm, k = kb + kc;
+        const bool in = m < a.M && k < k_end;
+        cp_async16(smem_u32(dst + mm * (kBK + 8) + kc), a.P + (in ? m * a.p_m + k : 0),
+                   in ? 16u : 0u);
+      } else {      // row k, 16 chunks of m per row
+        const int kk = c >> 4, mc = (c & 15) * 8;
+        const int64_t m = m0 + mc, k = kb + kk;
+        const bool in = m < a.M && k < k_end;
+        cp_async16(smem_u32(dst + kk * (kBM + 8) + mc), a.P + (in ? k * a.p_k + m : 0),
+                   in ? 16u : 0u);
+      }
+    }
+  };
+  // ---- Q tile: QV float4 per thread into registers, then split into hi/lo bf16
+  float4 qr[QV];
+  auto load_q = [&](int64_t kb) {
+#pragma unroll
+    for (int i = 0; i < QV; ++i) {
+      const int c = tid + i * kThreads;
+      int nn, kk;
+      if (Q_RED) {
+        nn = c / (kBK / 4);
+        kk = (c % (kBK / 4)) * 4;
       } else {
-        kk = idx / kBM;
-        mm = idx % kBM;
+        kk = c / (BN / 4);
+        nn = (c % (BN / 4)) * 4;
       }
-      const int64_t m = m0 + mm, k = kb + kk;
-      float v = 0.f;
-      if (m < a.M && k < k_end) v = bf16_bits_to_float(__ldg(a.P + m * a.p_m + k * a.p_k));
-      Ps[kk][mm] = v;
+      const int64_t n = n0 + nn, k = kb + kk;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (n < a.N && k < k_end)
+        v = __ldg(reinterpret_cast<const float4*>(a.Q + k * a.q_k + n * a.q_n));
+      qr[i] = v;
     }
-    // stage Q tile (32 x BN) -> Qs[k][n]
+  };
+  auto store_q = [&](int st) {
+    uint16_t* hi = Qh + st * QE;
+    uint16_t* lo = Ql + st * QE;
 #pragma unroll
-    for (int it = 0; it < (kBK * BN + kThreads - 1) / kThreads; ++it) {
-      const int idx = tid + it * kThreads;
-      if (idx < kBK * BN) {
-        int nn, kk;
-        if (Q_RED) {
-          nn = idx / kBK;
-          kk = idx % kBK;
-        } else {
-          kk = idx / BN;
-          nn = idx % BN;
+    for (int i = 0; i < QV; ++i) {
+      const int c = tid + i * kThreads;
+      const float v[4] = {qr[i].x, qr[i].y, qr[i].z, qr[i].w};
+      uint16_t h[4], l[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[e] = float_to_bf16_bits(v[e]);
+        l[e] = float_to_bf16_bits(v[e] - bf16_bits_to_float(h[e]));
+      }
+      if (Q_RED) {  // four consecutive k of one n: one 8-byte store each
+        const int nn = c / (kBK / 4), kk = (c % (kBK / 4)) * 4;
+        *reinterpret_cast<uint2*>(hi + nn * (kBK + 8) + kk) =
+            make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
+        *reinterpret_cast<uint2*>(lo + nn * (kBK + 8) + kk) =
+            make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
+      } else {      // one k of four consecutive n
+        const int kk = c / (BN / 4), nn = (c % (BN / 4)) * 4;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[(nn + e) * (kBK + 8) + kk] = h[e];
+          lo[(nn + e) * (kBK + 8) + kk] = l[e];
         }
-        const int64_t n = n0 + nn, k = kb + kk;
-        float v = 0.f;
-        if (n < a.N && k < k_end) v = __ldg(a.Q + k * a.q_k + n * a.q_n);
-        Qs[kk][nn] = v;
       }
     }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kBK; ++kk) {
-      float pv[4], qv[TN];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = Ps[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < TN; ++j) qv[j] = Qs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(pv[i], qv[j], acc[i][j]);
-    }
-    __syncthreads();
+  };
+
+  int st = 0;
+  if (k_begin < k_end) {
+    load_p(0, k_begin);
+    cp_async_commit();
+    load_q(k_begin);
+    store_q(0);
   }
-  float* out = a.part + (size_t)z * a.M * a.N;
+  for (int64_t kb = k_begin; kb < k_end; kb += kBK) {
+    const bool has_next = kb + kBK < k_end;
+    if (has_next) {
+      load_p(st ^ 1, kb + kBK);
+      cp_async_commit();
+      load_q(kb + kBK);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // P and Q of stage st visible to every warp
+    const uint16_t* ps = Ps + st * PE;
+    const uint16_t* qh = Qh + st * QE;
+    const uint16_t* ql = Ql + st * QE;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t m = m0 + ty + 16 * i;
-    if (m >= a.M) continue;
+    for (int k16 = 0; k16 < kBK; k16 += 16) {
+      uint32_t af[2][4];
 #pragma unroll
-    for (int j = 0; j < TN; ++j) {
-      const int64_t n = n0 + tx + 16 * j;
-      if (n < a.N) out[m * a.N + n] = acc[i][j];
+      for (int mi = 0; mi < 2; ++mi) {
+        const int r0 = wm * 32 + mi * 16;
+        if (P_RED) {
+          ldsm4(af[mi], smem_u32(ps + (r0 + (lane & 15)) * (kBK + 8) + k16 + 8 * (lane >> 4)));
+        } else {
+          const int i = lane >> 3, j = lane & 7;
+          ldsm4_t(af[mi], smem_u32(ps + (k16 + j + 8 * (i >> 1)) * (kBM + 8) + r0 + 8 * (i & 1)));
+        }
+      }
+#pragma unroll
+      for (int nj = 0; nj < NF; nj += 2) {
+        const int nr = wn * WN + nj * 8 + (lane & 7) + 8 * (lane >> 4);
+        const int kc = k16 + 8 * ((lane >> 3) & 1);
+        uint32_t bh[4], bl[4];
+        ldsm4(bh, smem_u32(qh + nr * (kBK + 8) + kc));
+        ldsm4(bl, smem_u32(ql + nr * (kBK + 8) + kc));
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+          mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
+          mma_bf16(acc[mi][nj], af[mi], bl[0], bl[1]);
+          mma_bf16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
+          mma_bf16(acc[mi][nj + 1], af[mi], bl[2], bl[3]);
+        }
+      }
+    }
+    if (has_next) store_q(st ^ 1);  // stage st ^ 1 was last read before the previous sync
+    __syncthreads();                // every warp is done with stage st
+    st ^= 1;
+  }
+
+  float* out = a.part + (size_t)blockIdx.z * a.M * a.N;
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi) {
+#pragma unroll
+    for (int nj = 0; nj < NF; ++nj) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t m = m0 + wm * 32 + mi * 16 + (lane >> 2) + 8 * h;
+        const int64_t n = n0 + wn * WN + nj * 8 + 2 * (lane & 3);
+        if (m >= a.M) continue;
+        if (n < a.N) out[m * a.N + n] = acc[mi][nj][2 * h];
+        if (n + 1 < a.N) out[m * a.N + n + 1] = acc[mi][nj][2 * h + 1];
+      }
     }
   }
 }
@@ -132,10 +265,10 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
   }
 }
 
-int bn_for(int64_t N) { return N <= 16 ? 16 : N <= 32 ? 32 : N <= 48 ? 48 : 64; }
+int bn_for(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : 192; }
 
 // Splits of the reduction for a product: about two waves of CTAs on 148 SMs,
-// each slice at least two smem tiles long.
+// each slice at least two stages long.
 int splits_for(int64_t M, int64_t N, int64_t K) {
   const int bn = bn_for(N);
   const int64_t xy = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
@@ -146,6 +279,22 @@ int splits_for(int64_t M, int64_t N, int64_t K) {
   return (int)((K + kps - 1) / kps);
 }
 
+template <bool P_RED, bool Q_RED, int BN>
+int launch_bn(const SkinnyArgs& a, dim3 grid, cudaStream_t st) {
+  constexpr size_t smem = skinny_smem_bytes<P_RED, BN>();
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    LSQ_CUDA(cudaFuncSetAttribute(skinny_kernel<P_RED, Q_RED, BN>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    attr_done[dev] = true;
+  }
+  skinny_kernel<P_RED, Q_RED, BN><<<grid, kThreads, smem, st>>>(a);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
 template <bool P_RED, bool Q_RED>
 int run(const SkinnyArgs& a0, int splits, cudaStream_t st) {
   SkinnyArgs a = a0;
@@ -153,13 +302,10 @@ int run(const SkinnyArgs& a0, int splits, cudaStream_t st) {
   const int bn = bn_for(a.N);
   dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)splits);
   switch (bn) {
-    case 16: skinny_kernel<P_RED, Q_RED, 16><<<grid, kThreads, 0, st>>>(a); break;
-    case 32: skinny_kernel<P_RED, Q_RED, 32><<<grid, kThreads, 0, st>>>(a); break;
-    case 48: skinny_kernel<P_RED, Q_RED, 48><<<grid, kThreads, 0, st>>>(a); break;
-    default: skinny_kernel<P_RED, Q_RED, 64><<<grid, kThreads, 0, st>>>(a); break;
+    case 64: return launch_bn<P_RED, Q_RED, 64>(a, grid, st);
+    case 128: return launch_bn<P_RED, Q_RED, 128>(a, grid, st);
+    default: return launch_bn<P_RED, Q_RED, 192>(a, grid, st);
   }
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return LSQ_OK;
 }
 
 int finish(const float* part, int splits, int64_t M, int64_t N, float alpha, int accumulate,

@@ -28,6 +28,29 @@ def normwise_err(got, ref):
     return float(np.max(np.abs(got - ref)) / den) if den > 0 else float(np.max(np.abs(got)))
 
 
+def frobenius_err(got, ref):
+    """||got - ref||_F / ||ref||_F (relative error of the tensor as a whole)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
+
+
+# Stack-level LoRA gradients: every tensor within 2e-2 relative (Frobenius); by the
+# max-element reading every tensor within 2e-2 too, except the q and k projections,
+# whose gradients carry the forward error of all the layers above through the
+# attention backward (measured 0.015-0.022 on the small random-init stacks), bounded
+# at 3e-2.
+STACK_GRAD_TOL, STACK_QK_MAX_TOL = 2e-2, 3e-2
+
+
+def check_stack_grad(got, ref, name, where):
+    f = frobenius_err(got, ref)
+    m = normwise_err(got, ref)
+    lim = STACK_QK_MAX_TOL if name in ("q", "k") else STACK_GRAD_TOL
+    assert f <= STACK_GRAD_TOL and m <= lim, (where, name, f, m)
+
+
 def elementwise_err(got, ref, floor=1e-3):
     """max |got - ref| / max(|ref|, floor * max|ref|)."""
     got = np.asarray(got, np.float64)

@@ -60,7 +60,7 @@ def test_layer_forward_with_the_adapter_off(L):
 
 
 def test_dpo_step_matches_oracle(L, small):
-    from gpu_util import normwise_err
+    from gpu_util import check_stack_grad, normwise_err
     from layer_streamed_qlora_nf4_b200 import pack
     cfg = small.cfg
     pairs, seq = 2, 64
@@ -83,9 +83,8 @@ def test_dpo_step_matches_oracle(L, small):
     for i in range(cfg["n_layers"]):
         gv = pack.lora_views(cfg, grad[i * nf:(i + 1) * nf])
         for name in synth.PROJ:
-            eA = normwise_err(gv[name][0].cpu().numpy(), rgrads[i][name][0])
-            eB = normwise_err(gv[name][1].cpu().numpy(), rgrads[i][name][1])
-            assert eA <= TOL and eB <= TOL, (i, name, eA, eB)
+            check_stack_grad(gv[name][0].cpu().numpy(), rgrads[i][name][0], name, (i, "A"))
+            check_stack_grad(gv[name][1].cpu().numpy(), rgrads[i][name][1], name, (i, "B"))
     assert L.lsq_device_status() == 0
 
 

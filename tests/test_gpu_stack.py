@@ -1,5 +1,6 @@
 """GPU parity for the streamed stack step: against the fp64 oracle (loss within
-1e-3 relative, logits and LoRA gradients within normwise 2e-2, post-AdamW
+1e-3 relative, logits within normwise 2e-2, LoRA gradients within 2e-2 relative
+Frobenius and normwise, 3e-2 normwise for q and k (gpu_util.check_stack_grad), post-AdamW
 parameters within 2*lr), and streamed vs resident bit-equality (max |dlogit| =
 0.0, identical gradients), at a small Llama-shaped stack and at the full
 32-layer Llama-3.1-8B-shaped stack."""
@@ -147,7 +148,7 @@ def test_stack_absmax8_streamed_equals_resident_bitwise(L, small8):
 
 
 def _check_against_oracle(L, small):
-    from gpu_util import normwise_err
+    from gpu_util import check_stack_grad, normwise_err
     from layer_streamed_qlora_nf4_b200 import pack
     cfg = small.cfg
     batch, seq = 2, 80
@@ -165,9 +166,8 @@ def _check_against_oracle(L, small):
     for i in range(cfg["n_layers"]):
         gv = pack.lora_views(cfg, grad[i * nf:(i + 1) * nf])
         for name in synth.PROJ:
-            eA = normwise_err(gv[name][0].cpu().numpy(), rgrads[i][name][0])
-            eB = normwise_err(gv[name][1].cpu().numpy(), rgrads[i][name][1])
-            assert eA <= TOL and eB <= TOL, (i, name, eA, eB)
+            check_stack_grad(gv[name][0].cpu().numpy(), rgrads[i][name][0], name, (i, "A"))
+            check_stack_grad(gv[name][1].cpu().numpy(), rgrads[i][name][1], name, (i, "B"))
 
 
 def test_stack_streamed_equals_resident_bitwise(L, small):
@@ -195,7 +195,7 @@ def test_stack_streamed_equals_resident_bitwise(L, small):
 
 def test_stack_grad_accumulation_and_adamw(L, small):
     import torch
-    from gpu_util import normwise_err
+    from gpu_util import check_stack_grad
     cfg = small.cfg
     batch, seq, mb = 1, 64, 2
     tokens = synth.tokens(33, mb * batch, seq, cfg["vocab"]).reshape(mb, batch, seq)
@@ -222,7 +222,7 @@ def test_stack_grad_accumulation_and_adamw(L, small):
         for j, name in enumerate(synth.PROJ):
             for k, key in ((0, "A"), (1, "B")):
                 rg = 0.5 * (r0[2][i][name][k] + r1[2][i][name][k])
-                assert normwise_err(gv[name][k].cpu().numpy(), rg) <= TOL, (i, name, key)
+                check_stack_grad(gv[name][k].cpu().numpy(), rg, name, (i, key))
                 p0 = layers[i][key][name]
                 rp, _, _ = om.adamw_step(p0, rg, np.zeros_like(rg), np.zeros_like(rg), 1, lr=lr)
                 got = pv[name][k].cpu().numpy()
