@@ -34,6 +34,11 @@ WORKLOAD = ("Llama-3.1-8B-shaped 32-layer NF4 stack (block 64, fp32 absmax) stre
             "lm_head (vocab 128256) resident; batch 1 x seq 512 per GPU; one SFT step "
             "(cross-entropy + AdamW on LoRA r16 alpha32, all 7 projections)")
 BATCH, SEQ = 1, 512
+# DRAM bytes per launch of the fused NF4 GEMM classes at the 8B shapes with T = 512
+# (one ncu capture of every GEMM launch of one layer's forward + recomputing
+# backward; each launch reads its algorithmic bytes once).  The per-step mix of
+# launches is the same as in that layer, so the averages hold for the step.
+DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 37.14e6, "gemm_nf4_dx": 42.46e6}
 METRIC_QWEN = ("streamed LoRA train tokens/sec (Qwen2.5-3B shapes, bf16 base, seq 2048) and % of "
                "step roofline")
 WORKLOAD_QWEN = ("Qwen2.5-3B-shaped 36-layer stack, unquantised bf16 weights (154.1 MB per "
@@ -373,8 +378,14 @@ def run_ours(args):
     per_launch_ms = dom["total_ms"] / dom["launches"]
     achieved = (dom["flops"] / dom["launches"]) / (per_launch_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops_sustained"]
+    traffic = None
+    if not qwen and args.absmax_bits == 32 and tokens_per_step // mbs == SEQ:
+        traffic = DRAM_BYTES_PER_LAUNCH_8B_T512.get(dom_name)
     roofline = dict(bound="tensor", kernel=dom_name, achieved=achieved, peak=peak, unit="TFLOP/s",
-                    frac=achieved / peak, traffic=None,
+                    frac=achieved / peak, traffic=traffic,
+                    traffic_source=("dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+                                    "averaged over the class's launches of one 8B layer (ncu)")
+                    if traffic else None,
                     peak_source="%s bf16 sustained (kernel timed inside a long step)" % pk["source"],
                     launches_per_step=dom["launches"] / args.steps, per_launch_ms=per_launch_ms,
                     step_share=dom["total_ms"] / args.steps / ms_prof,
