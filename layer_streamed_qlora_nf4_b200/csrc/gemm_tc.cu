@@ -33,6 +33,7 @@
 // bit instead of hanging.
 #include <cuda.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -64,7 +65,7 @@ struct KParams {
   const uint8_t* am_q;  // 8-bit absmax mode when non-null
   const float* am_s;
   int w_rows, w_cols;
-  int slab_w, jofs_by_part, n_parts;
+  int slab_w, part_r, n_parts;
   const float* la;
   long long la_rs, la_cs;
   float la_scale;
@@ -85,7 +86,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int WMODE>
+template <int WMODE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_w,
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_cfull[kMaxRing];
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
+  __shared__ __align__(8) uint64_t bar_opd[kMaxStages];  // PAIR, odd CTA: its operand warps done
   __shared__ __align__(8) uint64_t bar_res[kOpWarps];  // per epilogue warp: residual tile landed
   __shared__ __align__(8) uint64_t bar_grp;            // the operand warps
   __shared__ uint32_t tmem_base_sh;
@@ -108,7 +110,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int BT = p.nacc * p.bn;
   const uint32_t acc_stride = (p.nacc > 1) ? 256u : 0u;  // TMEM column of accumulator 1
-  const uint32_t xs_bytes = (uint32_t)BT * 128u;
+  // With PAIR, the CTA pair (cluster of 2) computes a 256-feature tile: this CTA
+  // dequantises its own 128 features (half of A) and loads half of each
+  // accumulator's tokens (half of B); the even CTA issues cta_group::2 MMAs.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int hb = PAIR ? p.bn / 2 : p.bn;  // tokens of each accumulator held here
+  const uint32_t xs_bytes = (uint32_t)(p.nacc * hb) * 128u;
   uint8_t* dsm = align1024(dsm_raw);
   uint8_t* xs0 = dsm;
   uint8_t* ws0 = xs0 + (size_t)p.stages * xs_bytes;
@@ -128,7 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 1 + kOpWarps);  // producer + operand warps
+      // producer + this CTA's operand warps (+ one forwarded arrival from the odd CTA)
+      mbar_init(smem_u32(&bar_full[s]), 1 + kOpWarps + (PAIR ? 1 : 0));
+      mbar_init(smem_u32(&bar_opd[s]), kOpWarps);
       mbar_init(smem_u32(&bar_empty[s]), 1);            // tcgen05.commit
     }
     for (int c = 0; c < CS; ++c) {
@@ -144,8 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x < 16) lv_sh[threadIdx.x] = p.levels[threadIdx.x];
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_base_sh), p.alloc_cols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(smem_u32(&tmem_base_sh), p.alloc_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&tmem_base_sh), p.alloc_cols);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_act);
@@ -154,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
@@ -171,27 +187,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         if (it < n_main) {
           const int kt = kt_begin + it;
-          uint32_t bytes = xs_bytes + (WMODE == W_BF16_N ? (uint32_t)kWStageBytes : 0u);
-          mbar_arrive_expect_tx(fb, bytes);
-          for (int a = 0; a < p.nacc; ++a)
-            tma_load_2d(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * p.bn * 128), &tm_act, fb,
-                        kt * kBK, t0 + a * p.bn);
-          if (WMODE == W_BF16_N)
-            tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fb, kt * kBK, m0);
-        } else {
+          const uint32_t bytes = xs_bytes + (WMODE == W_BF16_N ? (uint32_t)kWStageBytes : 0u);
+          if (PAIR) {
+            // both CTAs' bytes complete on the even CTA's barrier
+            const uint32_t fl = mapa_shared(fb, 0);
+            if (leader) mbar_arrive_expect_tx(fb, 2 * bytes);
+            for (int a = 0; a < p.nacc; ++a)
+              tma_load_2d_pair(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * hb * 128), &tm_act,
+                               fl, kt * kBK, t0 + a * p.bn + (int)rank * hb);
+            if (WMODE == W_BF16_N)
+              tma_load_2d_pair(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fl, kt * kBK, m0);
+          } else {
+            mbar_arrive_expect_tx(fb, bytes);
+            for (int a = 0; a < p.nacc; ++a)
+              tma_load_2d(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * p.bn * 128), &tm_act,
+                          fb, kt * kBK, t0 + a * p.bn);
+            if (WMODE == W_BF16_N)
+              tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fb, kt * kBK, m0);
+          }
+        } else if (!PAIR || leader) {
           mbar_arrive(fb);
         }
       }
       __syncwarp();
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 && (!PAIR || leader)) {
     // ---------------------------------------------------------- MMA issuer (lane 0)
-    const uint32_t idesc = umma_idesc_bf16(kBM, p.bn);
+    const uint32_t idesc = umma_idesc_bf16(PAIR ? 2 * kBM : kBM, p.bn);
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
-      bool ok = mbar_wait_bounded(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
-                                  DEV_ERR_WAIT_GEMM);
+      bool ok = PAIR ? mbar_wait_bounded_cluster(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
+                                                 DEV_ERR_WAIT_GEMM)
+                     : mbar_wait_bounded(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
+                                         DEV_ERR_WAIT_GEMM);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
       if (lane == 0) {
@@ -202,17 +231,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < nk; ++kk) {
           const uint64_t ad = umma_desc_k_sw128(wa + kk * 32);
           for (int a = 0; a < p.nacc; ++a) {
-            const uint64_t bd = umma_desc_k_sw128(xa + (uint32_t)(a * p.bn * 128) + kk * 32);
-            tc_mma_bf16(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
-                        (it > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bd = umma_desc_k_sw128(xa + (uint32_t)(a * hb * 128) + kk * 32);
+            if (PAIR)
+              tc_mma_bf16_pair(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+            else
+              tc_mma_bf16(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
+                          (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc_commit(smem_u32(&bar_empty[s]));
+        if (PAIR)
+          tc_commit_pair(smem_u32(&bar_empty[s]));
+        else
+          tc_commit(smem_u32(&bar_empty[s]));
       }
       __syncwarp();
     }
-    if (lane == 0) tc_commit(smem_u32(&bar_acc));
+    if (lane == 0) {
+      if (PAIR)
+        tc_commit_pair(smem_u32(&bar_acc));
+      else
+        tc_commit(smem_u32(&bar_acc));
+    }
     __syncwarp();
+  } else if (PAIR && warp == 1) {
+    // ---------------------------------------------------------- odd CTA: operand forwarder
+    // Once this CTA's eight operand warps have filled stage s, one arrival
+    // (release, cluster scope) on the even CTA's operand-ready barrier.
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      bool ok = mbar_wait_bounded(smem_u32(&bar_opd[s]), ph, abort_flag, p.dev_err,
+                                  DEV_ERR_WAIT_GEMM);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bar_full[s]), 0));
+      __syncwarp();
+    }
   } else if (warp == 2) {
     // ---------------------------------------------------------- staging-ring TMA producer
     if (WMODE != W_BF16_N) {
@@ -397,35 +451,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
           const int j0 = (it - n_main) * 64;
           const int wq = min(64, p.slab_w - j0) / 8;  // chunks of 8 slab columns
-          int jofs = 0;
-          if (p.jofs_by_part) {
-            int part = 0;
-            while (part + 1 < p.n_parts && m0 >= p.part_end[part]) ++part;
-            jofs = part * p.slab_w;
-          }
           for (int i = tid; i < 128 * wq; i += kOpThreads) {
             const int row = i & 127, q = i >> 7;
             const int m = m0 + row;
+            int jlo = 0;  // this row's slab columns: [jlo, jlo + part_r) of a stacked weight
+            if (p.part_r > 0) {
+              int part = 0;
+              while (part + 1 < p.n_parts && m >= p.part_end[part]) ++part;
+              jlo = part * p.part_r;
+            }
             float v[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const long long j = j0 + 8 * q + e;
-              v[e] = (m < p.M) ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + j * p.la_cs)
-                               : 0.f;
+              const int j = j0 + 8 * q + e;
+              const int jl = j - jlo;
+              const bool in = m < p.M && (p.part_r == 0 || (jl >= 0 && jl < p.part_r));
+              v[e] = in ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + (long long)jl * p.la_cs)
+                        : 0.f;
             }
             *reinterpret_cast<uint4*>(wst + sw128_offset(row, q)) =
                 make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
           }
           uint8_t* xst = xs0 + (size_t)s * xs_bytes;
-          for (int i = tid; i < BT * wq; i += kOpThreads) {
-            const int t = i % BT, q = i / BT;
-            const int tg = t0 + t;
+          const int HT = p.nacc * hb;  // token rows of this CTA's activation stage
+          for (int i = tid; i < HT * wq; i += kOpThreads) {
+            const int t = i % HT, q = i / HT;
+            const int tg = t0 + (t / hb) * p.bn + (int)rank * hb + t % hb;
             float v[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + jofs + j0 + 8 * q + e)
-                                : 0.f;
+              v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + j0 + 8 * q + e) : 0.f;
             *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
                 make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
@@ -434,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       }
-      if (ok && lane == 0) mbar_arrive(smem_u32(&bar_full[s]));
+      if (ok && lane == 0)
+        mbar_arrive(smem_u32(PAIR && !leader ? &bar_opd[s] : &bar_full[s]));
     }
 
     // ---------------------------------------------------------- epilogue (per warp)
@@ -524,9 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (abort_sh) settle_ns(2000000);  // let issued copies and MMAs land before freeing TMEM
+  // The even CTA's MMAs read the odd CTA's shared memory and write its TMEM:
+  // neither leaves (or frees TMEM) before both are here.
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, p.alloc_cols);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, p.alloc_cols);
+    else
+      tmem_dealloc(tmem, p.alloc_cols);
   }
 }
 
@@ -570,26 +633,41 @@ int make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void
 
 struct Plan {
   int bn, nacc, t_tiles, m_tiles, kt_total, kt_per_split, splits, stages, ring_stages;
+  bool pair;  // CTA pairs with cta_group::2 MMAs (M = 256 per pair)
   uint32_t ring_bytes, smem_bytes, alloc_cols;
   size_t partial_bytes;
 };
 
 int g_num_sms = 0;
 
+// CTA pairs are used unless LSQ_GEMM_PAIR=0 is set in the environment (which
+// selects the one-CTA kernel, e.g. to compare the two).
+bool pair_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("LSQ_GEMM_PAIR");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 Plan make_plan(const GemmDesc& d) {
   Plan pl{};
   const int64_t T = d.T;
+  pl.m_tiles = (int)((d.M + kBM - 1) / kBM);
+  pl.pair = pair_enabled() && pl.m_tiles >= 2;
+  const int64_t gran = pl.pair ? 32 : 16;  // a pair splits each accumulator's tokens in two
   if (T <= 256) {
     pl.nacc = 1;
-    pl.bn = (int)((T + 15) / 16 * 16);
+    pl.bn = (int)((T + gran - 1) / gran * gran);
   } else {
     pl.nacc = 2;
     const int64_t half = (std::min<int64_t>(T, 512) + 1) / 2;
-    pl.bn = (int)std::min<int64_t>(256, (half + 15) / 16 * 16);
+    pl.bn = (int)std::min<int64_t>(256, (half + gran - 1) / gran * gran);
   }
+  if (pl.pair) pl.m_tiles = (pl.m_tiles + 1) / 2 * 2;
   const int BT = pl.nacc * pl.bn;
   pl.t_tiles = (int)((T + BT - 1) / BT);
-  pl.m_tiles = (int)((d.M + kBM - 1) / kBM);
   pl.kt_total = (int)((d.Kc + kBK - 1) / kBK);
   const int sms = gemm_num_sms();
   const int base = pl.m_tiles * pl.t_tiles;
@@ -605,7 +683,7 @@ Plan make_plan(const GemmDesc& d) {
   pl.splits = (pl.kt_total + pl.kt_per_split - 1) / pl.kt_per_split;
   pl.partial_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)T * (size_t)d.M * 4 : 0;
   pl.ring_bytes = (d.wmode == W_BF16_T) ? 64 * 128 * 2 : (d.wmode == W_BF16_N ? 0 : 4096);
-  const uint32_t xs = (uint32_t)BT * 128;
+  const uint32_t xs = (uint32_t)(pl.pair ? BT / 2 : BT) * 128;
   int ring = (d.wmode == W_BF16_N) ? 0 : (d.wmode == W_BF16_T ? 2 : kMaxRing);
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
@@ -623,20 +701,20 @@ Plan make_plan(const GemmDesc& d) {
   return pl;
 }
 
-template <int WMODE>
+template <int WMODE, bool PAIR>
 int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t st) {
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    LSQ_CUDA(cudaFuncSetAttribute(tc_gemm_kernel<WMODE>,
+    LSQ_CUDA(cudaFuncSetAttribute(tc_gemm_kernel<WMODE, PAIR>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)(kSmemBudget - 2048)));
     attr_done[dev] = true;
   }
   CUtensorMap tm_act, tm_w;
   LSQ_TRY(make_tmap(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.act, (uint64_t)d.Kc,
-                    (uint64_t)d.T, (uint64_t)d.act_ld, kBK, (uint32_t)pl.bn,
+                    (uint64_t)d.T, (uint64_t)d.act_ld, kBK, (uint32_t)(PAIR ? pl.bn / 2 : pl.bn),
                     CU_TENSOR_MAP_SWIZZLE_128B));
   if (WMODE == W_NF4_N)
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.w, (uint64_t)d.w_cols / 2,
@@ -698,7 +776,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   p.w_rows = (int)d.w_rows;
   p.w_cols = (int)d.w_cols;
   p.slab_w = d.slab_w;
-  p.jofs_by_part = d.jofs_by_part;
+  p.part_r = d.part_r;
   p.n_parts = d.n_parts;
   p.la = d.la;
   p.la_rs = d.la_rs;
@@ -717,9 +795,20 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   const float* lv = nf4_levels();
   for (int i = 0; i < 16; ++i) p.levels[i] = lv[i];
   if (!p.dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
-  dim3 grid(pl.m_tiles, pl.t_tiles, pl.splits);
-  tc_gemm_kernel<WMODE><<<grid, kThreads, pl.smem_bytes, st>>>(tm_act, tm_w, tm_out, tm_res, p);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.m_tiles, pl.t_tiles, pl.splits);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pl.smem_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  LSQ_CUDA(::lsq::launched(
+      cudaLaunchKernelEx(&cfg, tc_gemm_kernel<WMODE, PAIR>, tm_act, tm_w, tm_out, tm_res, p)));
   return LSQ_OK;
 }
 
@@ -779,10 +868,22 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
   }
   const int prof = prof_begin(st);
   switch (d.wmode) {
-    case W_NF4_N: LSQ_TRY(launch_mode<W_NF4_N>(d, pl, partial, st)); break;
-    case W_NF4_T: LSQ_TRY(launch_mode<W_NF4_T>(d, pl, partial, st)); break;
-    case W_BF16_N: LSQ_TRY(launch_mode<W_BF16_N>(d, pl, partial, st)); break;
-    case W_BF16_T: LSQ_TRY(launch_mode<W_BF16_T>(d, pl, partial, st)); break;
+    case W_NF4_N:
+      LSQ_TRY((pl.pair ? launch_mode<W_NF4_N, true>(d, pl, partial, st)
+                       : launch_mode<W_NF4_N, false>(d, pl, partial, st)));
+      break;
+    case W_NF4_T:
+      LSQ_TRY((pl.pair ? launch_mode<W_NF4_T, true>(d, pl, partial, st)
+                       : launch_mode<W_NF4_T, false>(d, pl, partial, st)));
+      break;
+    case W_BF16_N:
+      LSQ_TRY((pl.pair ? launch_mode<W_BF16_N, true>(d, pl, partial, st)
+                       : launch_mode<W_BF16_N, false>(d, pl, partial, st)));
+      break;
+    case W_BF16_T:
+      LSQ_TRY((pl.pair ? launch_mode<W_BF16_T, true>(d, pl, partial, st)
+                       : launch_mode<W_BF16_T, false>(d, pl, partial, st)));
+      break;
     default: return set_error(LSQ_ERR_INVALID, "gemm: bad operand mode");
   }
   if (pl.splits > 1)

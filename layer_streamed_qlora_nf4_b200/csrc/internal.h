@@ -75,16 +75,19 @@ struct GemmDesc {
   int64_t w_rows = 0, w_cols = 0;   // storage shape of W
   const uint16_t* act = nullptr;    // bf16 [T, act_ld], contraction over the first Kc columns
   int64_t act_ld = 0;
-  // LoRA slab (an extra K range appended to split 0): la[m, j] = la_scale *
-  // la_ptr[m * la_rs + j * la_cs]; lb[t, j] = lb_ptr[t * lb_ld + jofs + j];
-  // jofs = 0, or part(m) * slab_w when jofs_by_part (part boundaries part_end[]).
+  // LoRA slab (an extra K range appended to split 0): lb[t, j] = lb_ptr[t * lb_ld + j]
+  // and la[m, j] = la_scale * la_ptr[m * la_rs + j * la_cs]; or, for a stacked
+  // weight with part_r > 0 (parts ending at rows part_end[]), slab_w = n_parts *
+  // part_r and la[m, j] = la_scale * la_ptr[m * la_rs + (j - p part_r) * la_cs]
+  // when row m is in part p and j in [p part_r, (p + 1) part_r), else 0: every
+  // row then uses the same lb, as a CTA pair's shared B operand requires.
   int slab_w = 0;
   const float* la = nullptr;
   int64_t la_rs = 0, la_cs = 0;
   float la_scale = 0.f;
   const float* lb = nullptr;
   int64_t lb_ld = 0;
-  int jofs_by_part = 0;
+  int part_r = 0;
   int n_parts = 0;
   int64_t part_end[4] = {0, 0, 0, 0};
   // epilogue

@@ -192,14 +192,14 @@ GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64
   d.w_cols = K;
   d.act = act;
   d.act_ld = K;
-  d.slab_w = r;
+  d.slab_w = n_parts > 1 ? n_parts * r : r;
   d.la = B;
   d.la_rs = r;
   d.la_cs = 1;
   d.la_scale = s;
   d.lb = u;
   d.lb_ld = u_ld;
-  d.jofs_by_part = n_parts > 1;
+  d.part_r = n_parts > 1 ? r : 0;
   d.n_parts = n_parts;
   for (int i = 0; i < n_parts && i < 4; ++i) d.part_end[i] = pe[i];
   d.out = out;
