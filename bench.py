@@ -38,7 +38,7 @@ BATCH, SEQ = 1, 512
 # (one ncu capture of every GEMM launch of one layer's forward + recomputing
 # backward; each launch reads its algorithmic bytes once).  The per-step mix of
 # launches is the same as in that layer, so the averages hold for the step.
-DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 37.14e6, "gemm_nf4_dx": 42.46e6}
+DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 37.26e6, "gemm_nf4_dx": 42.45e6}
 METRIC_QWEN = ("streamed LoRA train tokens/sec (Qwen2.5-3B shapes, bf16 base, seq 2048) and % of "
                "step roofline")
 WORKLOAD_QWEN = ("Qwen2.5-3B-shaped 36-layer stack, unquantised bf16 weights (154.1 MB per "
