@@ -10,11 +10,11 @@
 // slice of the reduction; P tiles arrive by cp.async (16-byte chunks along
 // whichever index is contiguous in memory; ldmatrix, transposing where P's rows
 // are the contiguous index, gives the A fragments), and each fp32 Q tile is
-// split into two bf16 tiles, hi = bf16(q) and lo = bf16(q - hi), so that the
-// two m16n8k16 products P hi + P lo carry about 16 bits of q: with P exact in
-// bf16 and fp32 accumulation the products keep close to fp32 accuracy.  The
-// slices are summed by a second kernel in a fixed order, so results are
-// deterministic (no atomics).
+// rounded once to bf16 (nearest even) on its way to shared memory: bf16
+// operands with fp32 accumulation, the compute precision of QLoRA's LoRA branch
+// (the tutorial's part 1: the LoRA A/B matrices are computed at a higher
+// precision than the NF4 storage).  The slices are summed by a second kernel in
+// a fixed order, so results are deterministic (no atomics).
 #include "common.cuh"
 
 namespace lsq {
@@ -62,7 +62,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 // Shared-memory tiles per stage (bf16, rows padded by 8 elements so that the
 // eight 16-byte rows an ldmatrix reads fall in distinct banks):
 //   P_RED: P as [kBM m][kBK + 8]   else P as [kBK k][kBM + 8]
-//   Q hi and lo as [BN n][kBK + 8]
+//   Q as [BN n][kBK + 8]
 template <bool P_RED>
 __host__ __device__ constexpr int p_stage_elems() {
   return P_RED ? kBM * (kBK + 8) : kBK * (kBM + 8);
@@ -73,7 +73,7 @@ __host__ __device__ constexpr int q_stage_elems() {
 }
 template <bool P_RED, int BN>
 constexpr size_t skinny_smem_bytes() {
-  return 2 * (size_t)(p_stage_elems<P_RED>() + 2 * q_stage_elems<BN>()) * 2;
+  return 2 * (size_t)(p_stage_elems<P_RED>() + q_stage_elems<BN>()) * 2;
 }
 
 // P_RED: the reduction index is the contiguous one in P (else the row index m is).
@@ -84,7 +84,6 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
   constexpr int PE = p_stage_elems<P_RED>(), QE = q_stage_elems<BN>();
   uint16_t* Ps = sk_smem;        // [2][PE]
   uint16_t* Qh = Ps + 2 * PE;    // [2][QE]
-  uint16_t* Ql = Qh + 2 * QE;    // [2][QE]
   constexpr int WN = BN / 2;     // columns per warp (warps: 4 along m x 2 along n)
   constexpr int NF = WN / 8;     // n8 fragments per warp
   constexpr int QV = BN * kBK / 4 / kThreads;  // float4 of Q per thread per stage
@@ -127,7 +126,7 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
       }
     }
   };
-  // ---- Q tile: QV float4 per thread into registers, then split into hi/lo bf16
+  // ---- Q tile: QV float4 per thread into registers, then rounded to bf16
   float4 qr[QV];
   auto load_q = [&](int64_t kb) {
 #pragma unroll
@@ -149,31 +148,22 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
     }
   };
   auto store_q = [&](int st) {
-    uint16_t* hi = Qh + st * QE;
-    uint16_t* lo = Ql + st * QE;
+    uint16_t* qs = Qh + st * QE;
 #pragma unroll
     for (int i = 0; i < QV; ++i) {
       const int c = tid + i * kThreads;
       const float v[4] = {qr[i].x, qr[i].y, qr[i].z, qr[i].w};
-      uint16_t h[4], l[4];
+      uint16_t h[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        h[e] = float_to_bf16_bits(v[e]);
-        l[e] = float_to_bf16_bits(v[e] - bf16_bits_to_float(h[e]));
-      }
-      if (Q_RED) {  // four consecutive k of one n: one 8-byte store each
+      for (int e = 0; e < 4; ++e) h[e] = float_to_bf16_bits(v[e]);
+      if (Q_RED) {  // four consecutive k of one n: one 8-byte store
         const int nn = c / (kBK / 4), kk = (c % (kBK / 4)) * 4;
-        *reinterpret_cast<uint2*>(hi + nn * (kBK + 8) + kk) =
+        *reinterpret_cast<uint2*>(qs + nn * (kBK + 8) + kk) =
             make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
-        *reinterpret_cast<uint2*>(lo + nn * (kBK + 8) + kk) =
-            make_uint2(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16));
       } else {      // one k of four consecutive n
         const int kk = c / (BN / 4), nn = (c % (BN / 4)) * 4;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hi[(nn + e) * (kBK + 8) + kk] = h[e];
-          lo[(nn + e) * (kBK + 8) + kk] = l[e];
-        }
+        for (int e = 0; e < 4; ++e) qs[(nn + e) * (kBK + 8) + kk] = h[e];
       }
     }
   };
@@ -198,7 +188,6 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
     __syncthreads();  // P and Q of stage st visible to every warp
     const uint16_t* ps = Ps + st * PE;
     const uint16_t* qh = Qh + st * QE;
-    const uint16_t* ql = Ql + st * QE;
 #pragma unroll
     for (int k16 = 0; k16 < kBK; k16 += 16) {
       uint32_t af[2][4];
@@ -216,15 +205,12 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
       for (int nj = 0; nj < NF; nj += 2) {
         const int nr = wn * WN + nj * 8 + (lane & 7) + 8 * (lane >> 4);
         const int kc = k16 + 8 * ((lane >> 3) & 1);
-        uint32_t bh[4], bl[4];
+        uint32_t bh[4];
         ldsm4(bh, smem_u32(qh + nr * (kBK + 8) + kc));
-        ldsm4(bl, smem_u32(ql + nr * (kBK + 8) + kc));
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
           mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
-          mma_bf16(acc[mi][nj], af[mi], bl[0], bl[1]);
           mma_bf16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
-          mma_bf16(acc[mi][nj + 1], af[mi], bl[2], bl[3]);
         }
       }
     }
@@ -336,8 +322,11 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
     return set_error(LSQ_ERR_WORKSPACE, "lora_down: scratch %zu < %zu", scratch_bytes, need);
   // C[t, j] = sum_k x[t, k] A[j, k]
   SkinnyArgs a{x, ldx, 1, A, 1, K, T, R, K, 0, scratch};
+  const int prof = prof_begin(st);
   LSQ_TRY((run<true, true>(a, s, st)));
-  return finish(scratch, s, T, R, 1.f, 0, u, R, 1, st);
+  LSQ_TRY(finish(scratch, s, T, R, 1.f, 0, u, R, 1, st));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
+  return LSQ_OK;
 }
 
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, int n_parts,
@@ -353,8 +342,11 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
       return set_error(LSQ_ERR_WORKSPACE, "lora_vproj: scratch %zu < %zu", scratch_bytes, need);
     // C[t, j] = sum_n dy[t, start + n] B[start + n, j]
     SkinnyArgs a{dy + start, N, 1, B + start * r, r, 1, T, r, Np, 0, scratch};
+    const int prof = prof_begin(st);
     LSQ_TRY((run<true, false>(a, s, st)));
     LSQ_TRY(finish(scratch, s, T, r, 1.f, 0, v + p * r, R, 1, st));
+    if (prof >= 0)
+      prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
     start = part_end[p];
   }
   return LSQ_OK;
@@ -369,8 +361,11 @@ int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, 
   if (!scratch || scratch_bytes < need)
     return set_error(LSQ_ERR_WORKSPACE, "lora_grad_a: scratch %zu < %zu", scratch_bytes, need);
   SkinnyArgs a{x, 1, K, v, R, 1, K, R, T, 0, scratch};
+  const int prof = prof_begin(st);
   LSQ_TRY((run<false, false>(a, z, st)));
-  return finish(scratch, z, K, R, s, accumulate, dA, 1, K, st);
+  LSQ_TRY(finish(scratch, z, K, R, s, accumulate, dA, 1, K, st));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
+  return LSQ_OK;
 }
 
 int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
@@ -385,8 +380,11 @@ int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N,
     if (!scratch || scratch_bytes < need)
       return set_error(LSQ_ERR_WORKSPACE, "lora_grad_b: scratch %zu < %zu", scratch_bytes, need);
     SkinnyArgs a{dy + start, 1, N, u + p * r, R, 1, Np, r, T, 0, scratch};
+    const int prof = prof_begin(st);
     LSQ_TRY((run<false, false>(a, z, st)));
     LSQ_TRY(finish(scratch, z, Np, r, s, accumulate, dB + start * r, r, 1, st));
+    if (prof >= 0)
+      prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
     start = part_end[p];
   }
   return LSQ_OK;

@@ -45,7 +45,11 @@ def _run(L, N, K, T, r=16, alpha=32.0, seed=0, residual=False, accumulate=False,
     e_y = normwise_err(host_bf16_to_f32(y), ref_y)
     e_u = normwise_err(u.cpu().numpy(), x @ case["A"].astype(np.float64).T)
     assert e_y <= TOL, e_y
-    assert e_u <= 1e-5, e_u
+    # u = x A^T on tensor cores: x is exact in bf16, A is rounded once to bf16
+    # (an independent error of at most 2^-9 relative per element, standard
+    # deviation 2^-9/sqrt(3)), accumulation in fp32; so du/u is about 1e-3
+    # (measured 1.5e-3) and the check allows 2^-8
+    assert e_u <= 2.0 ** -8, e_u
     if not check_bwd:
         return
     ref_dx, ref_dA, ref_dB = om.lora_linear_bwd(dy, x, Wt, case["A"], case["B"], s)
