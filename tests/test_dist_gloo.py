@@ -57,3 +57,59 @@ def test_two_rank_gradient_average_and_timing():
     assert np.allclose(g0, mean0, atol=1e-15)      # equal to the mean of the ranks' gradients
     assert np.array_equal(p0, p1)                  # hence identical parameters after AdamW
     assert t0 == t1 == 11.0                        # max over ranks
+
+
+def _dp_sft_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    from layer_streamed_qlora_nf4_b200 import dp
+    from oracle import model as om
+    from test_oracle_model import TINY, _layer_params
+    dp.init("gloo", timeout_s=60)
+    layers = [_layer_params(40 + i, TINY) for i in range(2)]
+    g = np.random.default_rng(41)
+    V = 97
+    emb, head = g.standard_normal((V, 64)) * 0.5, g.standard_normal((V, 64)) * 0.5
+    gf = np.ones(64)
+    tokens = g.integers(0, V, size=(world, 6))          # one sequence per rank
+    loss, _, grads = om.stack_loss_and_grads(layers, emb, head, gf, tokens[rank:rank + 1], TINY)
+    flat = torch.from_numpy(np.concatenate([np.concatenate([grads[i][n][0].ravel(),
+                                                            grads[i][n][1].ravel()])
+                                            for i in range(2) for n in om.PROJ]))
+    dp.average_(flat)
+    lt = torch.tensor([loss], dtype=torch.float64)
+    dp.average_(lt)
+    out[rank] = (flat.numpy().copy(), float(lt[0]), tokens)
+    dp.barrier()
+    torch.distributed.destroy_process_group()
+
+
+def test_two_rank_sft_step_equals_the_union_batch():
+    # Data-parallel replicas (one sequence per rank), gradients averaged across the
+    # ranks: the same loss and LoRA gradient as one step on both sequences together.
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    from oracle import model as om
+    from test_oracle_model import TINY, _layer_params
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_dp_sft_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    f0, l0, tokens = out[0]
+    f1, l1, _ = out[1]
+    assert np.array_equal(f0, f1) and l0 == l1
+    layers = [_layer_params(40 + i, TINY) for i in range(2)]
+    g = np.random.default_rng(41)
+    emb, head = g.standard_normal((97, 64)) * 0.5, g.standard_normal((97, 64)) * 0.5
+    loss, _, grads = om.stack_loss_and_grads(layers, emb, head, np.ones(64), tokens, TINY)
+    ref = np.concatenate([np.concatenate([grads[i][n][0].ravel(), grads[i][n][1].ravel()])
+                          for i in range(2) for n in om.PROJ])
+    assert abs(l0 - loss) <= 1e-12 * abs(loss)
+    assert np.max(np.abs(f0 - ref)) <= 1e-12 * np.max(np.abs(ref))
