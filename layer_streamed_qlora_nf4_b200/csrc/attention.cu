@@ -52,6 +52,22 @@ __device__ __forceinline__ void load_tile(uint16_t* sm, const uint16_t* g, int64
   }
 }
 
+// The same with cp.async (16-byte chunks, zero-filled rows >= valid): the copy
+// completes at the caller's cp.async wait, so it can overlap the previous tile's math.
+template <int D>
+__device__ __forceinline__ void load_tile_async(uint16_t* sm, const uint16_t* g, int64_t ld,
+                                                int valid) {
+  constexpr int CH = D / 8;
+  for (int i = threadIdx.x; i < kTile * CH; i += blockDim.x) {
+    const int r = i / CH, c = i % CH;
+    const bool in = r < valid;
+    const uint16_t* src = g + (in ? (int64_t)r * ld + c * 8 : 0);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sm + r * (D + 8) + c * 8)),
+                 "l"(src), "r"(in ? 16u : 0u)
+                 : "memory");
+  }
+}
+
 // A-operand fragment (16 rows x 16 cols) of a row-major smem tile: rows r0..r0+15, cols c0..
 template <int D>
 __device__ __forceinline__ void frag_a(uint32_t (&a)[4], const uint16_t* sm, int r0, int c0) {
@@ -82,8 +98,8 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
                                                        float* __restrict__ lse_out, float sl2) {
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Qs = smem_attn;
-  uint16_t* Ks = Qs + kTile * (D + 8);
-  uint16_t* Vs = Ks + kTile * (D + 8);
+  uint16_t* Kb = Qs + kTile * (D + 8);      // [2] K tiles
+  uint16_t* Vb = Kb + 2 * kTile * (D + 8);  // [2] V tiles
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (H / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -91,7 +107,17 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
   const int64_t ld = (int64_t)(H + 2 * Hkv) * D;
   const int64_t tok0 = (int64_t)b * seq;
   const int q0 = qb * kTile;
-  load_tile<D>(Qs, qkv + (tok0 + q0) * ld + (int64_t)h * D, ld, min(kTile, seq - q0));
+  load_tile_async<D>(Qs, qkv + (tok0 + q0) * ld + (int64_t)h * D, ld, min(kTile, seq - q0));
+  // K/V tile kb goes to buffer kb & 1, one tile ahead of the math
+  auto load_kv = [&](int kb) {
+    const int k0 = kb * kTile;
+    load_tile_async<D>(Kb + (kb & 1) * kTile * (D + 8), qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D,
+                       ld, min(kTile, seq - k0));
+    load_tile_async<D>(Vb + (kb & 1) * kTile * (D + 8),
+                       qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  load_kv(0);
 
   float o[D / 8][4];
 #pragma unroll
@@ -101,10 +127,15 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
 
   for (int kb = 0; kb <= qb; ++kb) {
     const int k0 = kb * kTile;
-    __syncthreads();
-    load_tile<D>(Ks, qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D, ld, min(kTile, seq - k0));
-    load_tile<D>(Vs, qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
-    __syncthreads();
+    if (kb < qb) {
+      load_kv(kb + 1);  // its buffer was last read before the previous iteration's end barrier
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();  // tile kb (and Q) visible to every warp
+    const uint16_t* Ks = Kb + (kb & 1) * kTile * (D + 8);
+    const uint16_t* Vs = Vb + (kb & 1) * kTile * (D + 8);
     float s[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
@@ -181,6 +212,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
         mma16816(o[2 * j + 1], a, bb[2], bb[3]);
       }
     }
+    __syncthreads();  // every warp is done with buffer kb & 1 before it is refilled
   }
   // finalize
 #pragma unroll
@@ -232,10 +264,10 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Ks = smem_attn;
   uint16_t* Vs = Ks + kTile * (D + 8);
-  uint16_t* Qs = Vs + kTile * (D + 8);
-  uint16_t* dOs = Qs + kTile * (D + 8);
-  float* lse_s = reinterpret_cast<float*>(dOs + kTile * (D + 8));
-  float* del_s = lse_s + kTile;
+  uint16_t* Qb = Vs + kTile * (D + 8);       // [2] Q tiles
+  uint16_t* dOb = Qb + 2 * kTile * (D + 8);  // [2] dO tiles
+  float* lse_b = reinterpret_cast<float*>(dOb + 2 * kTile * (D + 8));  // [2][kTile]
+  float* del_b = lse_b + 2 * kTile;                                      // [2][kTile]
   const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (H / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -253,18 +285,37 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     for (int e = 0; e < 4; ++e) dkacc[j][e] = dvacc[j][e] = 0.f;
   const int krow[2] = {k0 + warp * 16 + gid, k0 + warp * 16 + gid + 8};
   const int nqb = (seq + kTile - 1) / kTile;
+  // the Q / dO tiles (and their lse, delta rows) of query block qb go to buffer
+  // (qb - kb) & 1, one block ahead of the math
+  auto load_q = [&](int qb) {
+    const int q0 = qb * kTile, sl = (qb - kb) & 1;
+    load_tile_async<D>(Qb + sl * kTile * (D + 8), qkv + (tok0 + q0) * ld + (int64_t)h * D, ld,
+                       min(kTile, seq - q0));
+    load_tile_async<D>(dOb + sl * kTile * (D + 8), dout + (tok0 + q0) * ldo + (int64_t)h * D, ldo,
+                       min(kTile, seq - q0));
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int i = threadIdx.x; i < kTile; i += blockDim.x) {
+      const bool ok = q0 + i < seq;
+      lse_b[sl * kTile + i] = ok ? lse[(int64_t)h * T + tok0 + q0 + i] * 1.4426950408889634f : 0.f;
+      del_b[sl * kTile + i] = ok ? delta[(int64_t)h * T + tok0 + q0 + i] : 0.f;
+    }
+  };
+  load_q(kb);
   {
     for (int qb = kb; qb < nqb; ++qb) {
       const int q0 = qb * kTile;
-      __syncthreads();
-      load_tile<D>(Qs, qkv + (tok0 + q0) * ld + (int64_t)h * D, ld, min(kTile, seq - q0));
-      load_tile<D>(dOs, dout + (tok0 + q0) * ldo + (int64_t)h * D, ldo, min(kTile, seq - q0));
-      for (int i = threadIdx.x; i < kTile; i += blockDim.x) {
-        const bool ok = q0 + i < seq;
-        lse_s[i] = ok ? lse[(int64_t)h * T + tok0 + q0 + i] * 1.4426950408889634f : 0.f;
-        del_s[i] = ok ? delta[(int64_t)h * T + tok0 + q0 + i] : 0.f;
+      if (qb + 1 < nqb) {
+        load_q(qb + 1);  // its buffers were last read before the previous iteration's end barrier
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
       }
-      __syncthreads();
+      __syncthreads();  // block qb (and K, V) visible to every warp
+      const int sl = (qb - kb) & 1;
+      const uint16_t* Qs = Qb + sl * kTile * (D + 8);
+      const uint16_t* dOs = dOb + sl * kTile * (D + 8);
+      const float* lse_s = lse_b + sl * kTile;
+      const float* del_s = del_b + sl * kTile;
       // S^T = K Q^T  (16 keys of this warp x 64 queries)
       float st[8][4];
 #pragma unroll
@@ -344,6 +395,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
           mma16816(dkacc[2 * j + 1], a, bb[2], bb[3]);
         }
       }
+      __syncthreads();  // every warp is done with buffer (qb - kb) & 1 before it is refilled
     }
   }
 #pragma unroll
@@ -371,8 +423,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Qs = smem_attn;
   uint16_t* dOs = Qs + kTile * (D + 8);
-  uint16_t* Ks = dOs + kTile * (D + 8);
-  uint16_t* Vs = Ks + kTile * (D + 8);
+  uint16_t* Kb = dOs + kTile * (D + 8);     // [2] K tiles
+  uint16_t* Vb = Kb + 2 * kTile * (D + 8);  // [2] V tiles
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (H / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -394,12 +446,27 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
   float dqacc[D / 8][4];
 #pragma unroll
   for (int j = 0; j < D / 8; ++j) dqacc[j][0] = dqacc[j][1] = dqacc[j][2] = dqacc[j][3] = 0.f;
+  // K/V tile kb goes to buffer kb & 1, one tile ahead of the math
+  auto load_kv = [&](int kb) {
+    const int k0 = kb * kTile;
+    load_tile_async<D>(Kb + (kb & 1) * kTile * (D + 8), qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D,
+                       ld, min(kTile, seq - k0));
+    load_tile_async<D>(Vb + (kb & 1) * kTile * (D + 8),
+                       qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  load_kv(0);
   for (int kb = 0; kb <= qb; ++kb) {
     const int k0 = kb * kTile;
-    __syncthreads();
-    load_tile<D>(Ks, qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D, ld, min(kTile, seq - k0));
-    load_tile<D>(Vs, qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
-    __syncthreads();
+    if (kb < qb) {
+      load_kv(kb + 1);  // its buffer was last read before the previous iteration's end barrier
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();  // tile kb (and Q, dO) visible to every warp
+    const uint16_t* Ks = Kb + (kb & 1) * kTile * (D + 8);
+    const uint16_t* Vs = Vb + (kb & 1) * kTile * (D + 8);
     float s[8][4], dp[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -446,6 +513,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
         mma16816(dqacc[2 * j + 1], a, bb[2], bb[3]);
       }
     }
+    __syncthreads();  // every warp is done with buffer kb & 1 before it is refilled
   }
 #pragma unroll
   for (int rI = 0; rI < 2; ++rI) {
@@ -464,7 +532,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
 template <int D>
 int attn_fwd_t(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv, uint16_t* o, float* lse,
                cudaStream_t st) {
-  const size_t smem = 3 * kTile * (D + 8) * sizeof(uint16_t);
+  const size_t smem = 5 * kTile * (D + 8) * sizeof(uint16_t);  // Q + two K + two V tiles
   static bool attr = false;
   if (!attr) {
     LSQ_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -483,8 +551,8 @@ template <int D>
 int attn_bwd_t(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout, const float* lse,
                int64_t T, int seq, int H, int Hkv, float* delta, float* dq, float* dk, float* dv,
                cudaStream_t st) {
-  const size_t s_kv = 4 * kTile * (D + 8) * sizeof(uint16_t) + 2 * kTile * sizeof(float);
-  const size_t s_q = 4 * kTile * (D + 8) * sizeof(uint16_t);
+  const size_t s_kv = 6 * kTile * (D + 8) * sizeof(uint16_t) + 4 * kTile * sizeof(float);
+  const size_t s_q = 6 * kTile * (D + 8) * sizeof(uint16_t);
   static bool attr = false;
   if (!attr) {
     LSQ_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>,
