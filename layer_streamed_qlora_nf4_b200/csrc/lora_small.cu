@@ -7,14 +7,17 @@
 // 3 r <= 192 columns, P a bf16 activation and Q an fp32 LoRA tensor.
 //
 // One kernel serves all four.  A CTA owns 128 rows x BN columns of C over one
-// slice of the reduction; P tiles arrive by cp.async (16-byte chunks along
-// whichever index is contiguous in memory; ldmatrix, transposing where P's rows
-// are the contiguous index, gives the A fragments), and each fp32 Q tile is
-// rounded once to bf16 (nearest even) on its way to shared memory: bf16
-// operands with fp32 accumulation, the compute precision of QLoRA's LoRA branch
-// (the tutorial's part 1: the LoRA A/B matrices are computed at a higher
-// precision than the NF4 storage).  The slices are summed by a second kernel in
-// a fixed order, so results are deterministic (no atomics).
+// slice of the reduction.  Q is first rounded once to bf16 (nearest even) into
+// scratch, rows padded to a multiple of 8 elements with zeros: bf16 operands
+// with fp32 accumulation, the compute precision of QLoRA's LoRA branch (the
+// tutorial's part 1: the LoRA A/B matrices are computed at a higher precision
+// than the NF4 storage).  Both operands then stream through a ring of 4 to 6
+// cp.async stages (16-byte chunks along whichever index is contiguous in
+// memory; ldmatrix, transposing where needed, gives the MMA fragments), so
+// that each SM keeps enough bytes in flight to run these HBM-bound products
+// near the memory roofline.  When a product is split along its reduction, the
+// slices are summed by a second kernel in a fixed order, so results are
+// deterministic (no atomics); an unsplit product writes its result directly.
 #include "common.cuh"
 
 namespace lsq {
@@ -24,15 +27,22 @@ namespace {
 constexpr int kBM = 128;  // rows of C per CTA
 constexpr int kBK = 32;   // reduction elements per stage
 constexpr int kThreads = 256;
+constexpr int kSMs = 148;
 
 struct SkinnyArgs {
   const uint16_t* P;   // bf16: P(m, k) = P[m * p_m + k * p_k]
   int64_t p_m, p_k;
-  const float* Q;      // fp32: Q(k, n) = Q[k * q_k + n * q_n]
+  const uint16_t* Q;   // bf16: Q(k, n) = Q[k * q_k + n * q_n]; rows padded to 8 elements
   int64_t q_k, q_n;
   int64_t M, N, K;     // C is M x N, reduction over K
   int64_t k_per_split;
-  float* part;         // [splits][M][N]
+  float* part;         // [splits][M][N] when split
+  // unsplit: dst[m * c_m + n * c_n] = alpha * C[m, n] (+ dst if accumulate)
+  float* dst;
+  int64_t c_m, c_n;
+  float alpha;
+  int accumulate;
+  int direct;
 };
 
 __device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
@@ -62,32 +72,32 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 // Shared-memory tiles per stage (bf16, rows padded by 8 elements so that the
 // eight 16-byte rows an ldmatrix reads fall in distinct banks):
 //   P_RED: P as [kBM m][kBK + 8]   else P as [kBK k][kBM + 8]
-//   Q as [BN n][kBK + 8]
-template <bool P_RED>
-__host__ __device__ constexpr int p_stage_elems() {
-  return P_RED ? kBM * (kBK + 8) : kBK * (kBM + 8);
-}
-template <int BN>
-__host__ __device__ constexpr int q_stage_elems() {
-  return BN * (kBK + 8);
-}
-template <bool P_RED, int BN>
-constexpr size_t skinny_smem_bytes() {
-  return 2 * (size_t)(p_stage_elems<P_RED>() + q_stage_elems<BN>()) * 2;
-}
+//   Q_RED: Q as [BN n][kBK + 8]    else Q as [kBK k][BN + 8]
+// Stages and CTAs per SM: BN 64 -> 4 stages, 3 CTAs (61 KB each); BN 128 -> 4
+// stages, 2 CTAs (82 KB); BN 192 -> 6 stages, 1 CTA (154 KB).
+template <bool P_RED, bool Q_RED, int BN>
+struct Tile {
+  static constexpr int kStages = BN > 128 ? 6 : 4;
+  static constexpr int kMinBlocks = BN <= 64 ? 3 : BN <= 128 ? 2 : 1;
+  static constexpr int kPE = P_RED ? kBM * (kBK + 8) : kBK * (kBM + 8);
+  static constexpr int kQE = Q_RED ? BN * (kBK + 8) : kBK * (BN + 8);
+  static constexpr size_t kSmem = (size_t)kStages * (kPE + kQE) * 2;
+};
 
 // P_RED: the reduction index is the contiguous one in P (else the row index m is).
 // Q_RED: the reduction index is the contiguous one in Q (else the column n is).
 template <bool P_RED, bool Q_RED, int BN>
-__global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
+__global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks))
+    skinny_kernel(const SkinnyArgs a) {
+  using TL = Tile<P_RED, Q_RED, BN>;
+  constexpr int S = TL::kStages, PE = TL::kPE, QE = TL::kQE;
   extern __shared__ __align__(16) uint16_t sk_smem[];
-  constexpr int PE = p_stage_elems<P_RED>(), QE = q_stage_elems<BN>();
-  uint16_t* Ps = sk_smem;        // [2][PE]
-  uint16_t* Qh = Ps + 2 * PE;    // [2][QE]
+  uint16_t* Ps = sk_smem;        // [S][PE]
+  uint16_t* Qs = Ps + S * PE;    // [S][QE]
   constexpr int WN = BN / 2;     // columns per warp (warps: 4 along m x 2 along n)
   constexpr int NF = WN / 8;     // n8 fragments per warp
-  constexpr int QV = BN * kBK / 4 / kThreads;  // float4 of Q per thread per stage
-  static_assert(QV >= 1 && (BN * kBK / 4) % kThreads == 0, "Q tile split");
+  constexpr int QC = BN * kBK / 8 / kThreads;  // 16-byte chunks of Q per thread per stage
+  static_assert(QC >= 1 && (BN * kBK / 8) % kThreads == 0, "Q tile split");
   static_assert(NF % 2 == 0, "B fragments are loaded in pairs");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,6 +106,7 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
   const int64_t n0 = (int64_t)blockIdx.y * BN;
   const int64_t k_begin = (int64_t)blockIdx.z * a.k_per_split;
   const int64_t k_end = min(a.K, k_begin + a.k_per_split);
+  const int64_t n_it = k_end > k_begin ? (k_end - k_begin + kBK - 1) / kBK : 0;
 
   float acc[2][NF][4];
 #pragma unroll
@@ -105,9 +116,10 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 
-  // ---- P tile of the stage starting at kb: 512 chunks of 8 bf16 (two per thread)
-  auto load_p = [&](int st, int64_t kb) {
-    uint16_t* dst = Ps + st * PE;
+  // One stage: 512 chunks of P (two per thread) and BN * 4 chunks of Q.  Chunks
+  // outside the product (or this CTA's slice of the reduction) are zero-filled.
+  auto load_stage = [&](int slot, int64_t kb) {
+    uint16_t* pd = Ps + slot * PE;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int c = tid + i * kThreads;
@@ -115,79 +127,53 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
         const int mm = c >> 2, kc = (c & 3) * 8;
         const int64_t m = m0 + mm, k = kb + kc;
         const bool in = m < a.M && k < k_end;
-        cp_async16(smem_u32(dst + mm * (kBK + 8) + kc), a.P + (in ? m * a.p_m + k : 0),
+        cp_async16(smem_u32(pd + mm * (kBK + 8) + kc), a.P + (in ? m * a.p_m + k : 0),
                    in ? 16u : 0u);
       } else {      // row k, 16 chunks of m per row
         const int kk = c >> 4, mc = (c & 15) * 8;
         const int64_t m = m0 + mc, k = kb + kk;
         const bool in = m < a.M && k < k_end;
-        cp_async16(smem_u32(dst + kk * (kBM + 8) + mc), a.P + (in ? k * a.p_k + m : 0),
+        cp_async16(smem_u32(pd + kk * (kBM + 8) + mc), a.P + (in ? k * a.p_k + m : 0),
+                   in ? 16u : 0u);
+      }
+    }
+    uint16_t* qd = Qs + slot * QE;
+#pragma unroll
+    for (int i = 0; i < QC; ++i) {
+      const int c = tid + i * kThreads;
+      if (Q_RED) {  // row n, 4 chunks of k per row
+        const int nn = c >> 2, kc = (c & 3) * 8;
+        const int64_t n = n0 + nn, k = kb + kc;
+        const bool in = n < a.N && k < k_end;
+        cp_async16(smem_u32(qd + nn * (kBK + 8) + kc), a.Q + (in ? n * a.q_n + k : 0),
+                   in ? 16u : 0u);
+      } else {      // row k, BN / 8 chunks of n per row (the padded row ends on a chunk)
+        const int kk = c / (BN / 8), nc = (c % (BN / 8)) * 8;
+        const int64_t n = n0 + nc, k = kb + kk;
+        const bool in = n < a.N && k < k_end;
+        cp_async16(smem_u32(qd + kk * (BN + 8) + nc), a.Q + (in ? k * a.q_k + n : 0),
                    in ? 16u : 0u);
       }
     }
   };
-  // ---- Q tile: QV float4 per thread into registers, then rounded to bf16
-  float4 qr[QV];
-  auto load_q = [&](int64_t kb) {
-#pragma unroll
-    for (int i = 0; i < QV; ++i) {
-      const int c = tid + i * kThreads;
-      int nn, kk;
-      if (Q_RED) {
-        nn = c / (kBK / 4);
-        kk = (c % (kBK / 4)) * 4;
-      } else {
-        kk = c / (BN / 4);
-        nn = (c % (BN / 4)) * 4;
-      }
-      const int64_t n = n0 + nn, k = kb + kk;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (n < a.N && k < k_end)
-        v = __ldg(reinterpret_cast<const float4*>(a.Q + k * a.q_k + n * a.q_n));
-      qr[i] = v;
-    }
-  };
-  auto store_q = [&](int st) {
-    uint16_t* qs = Qh + st * QE;
-#pragma unroll
-    for (int i = 0; i < QV; ++i) {
-      const int c = tid + i * kThreads;
-      const float v[4] = {qr[i].x, qr[i].y, qr[i].z, qr[i].w};
-      uint16_t h[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) h[e] = float_to_bf16_bits(v[e]);
-      if (Q_RED) {  // four consecutive k of one n: one 8-byte store
-        const int nn = c / (kBK / 4), kk = (c % (kBK / 4)) * 4;
-        *reinterpret_cast<uint2*>(qs + nn * (kBK + 8) + kk) =
-            make_uint2(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16));
-      } else {      // one k of four consecutive n
-        const int kk = c / (BN / 4), nn = (c % (BN / 4)) * 4;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) qs[(nn + e) * (kBK + 8) + kk] = h[e];
-      }
-    }
-  };
 
-  int st = 0;
-  if (k_begin < k_end) {
-    load_p(0, k_begin);
+  // Ring: stage j lives in slot j % S; S - 1 stages are in flight ahead of the math.
+#pragma unroll
+  for (int j = 0; j < S - 1; ++j) {
+    if (j < n_it) load_stage(j, k_begin + (int64_t)j * kBK);
     cp_async_commit();
-    load_q(k_begin);
-    store_q(0);
   }
-  for (int64_t kb = k_begin; kb < k_end; kb += kBK) {
-    const bool has_next = kb + kBK < k_end;
-    if (has_next) {
-      load_p(st ^ 1, kb + kBK);
+  for (int64_t it = 0; it < n_it; ++it) {
+    cp_async_wait<S - 2>();  // stage it has landed (this thread's chunks)
+    __syncthreads();         // ... every thread's, and slot (it - 1) % S is free again
+    {
+      const int64_t nx = it + S - 1;
+      if (nx < n_it) load_stage((int)(nx % S), k_begin + nx * kBK);
       cp_async_commit();
-      load_q(kb + kBK);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
     }
-    __syncthreads();  // P and Q of stage st visible to every warp
-    const uint16_t* ps = Ps + st * PE;
-    const uint16_t* qh = Qh + st * QE;
+    const int slot = (int)(it % S);
+    const uint16_t* ps = Ps + slot * PE;
+    const uint16_t* qs = Qs + slot * QE;
 #pragma unroll
     for (int k16 = 0; k16 < kBK; k16 += 16) {
       uint32_t af[2][4];
@@ -203,10 +189,16 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
       }
 #pragma unroll
       for (int nj = 0; nj < NF; nj += 2) {
-        const int nr = wn * WN + nj * 8 + (lane & 7) + 8 * (lane >> 4);
-        const int kc = k16 + 8 * ((lane >> 3) & 1);
+        // matrices: (n block nj, k 0-7), (nj, k 8-15), (nj + 1, k 0-7), (nj + 1, k 8-15)
+        const int i = lane >> 3, j = lane & 7;
         uint32_t bh[4];
-        ldsm4(bh, smem_u32(qh + nr * (kBK + 8) + kc));
+        if (Q_RED) {
+          const int nr = wn * WN + (nj + (i >> 1)) * 8 + j;
+          ldsm4(bh, smem_u32(qs + nr * (kBK + 8) + k16 + 8 * (i & 1)));
+        } else {
+          const int kr = k16 + 8 * (i & 1) + j;
+          ldsm4_t(bh, smem_u32(qs + kr * (BN + 8) + wn * WN + (nj + (i >> 1)) * 8));
+        }
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
           mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
@@ -214,12 +206,9 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
         }
       }
     }
-    if (has_next) store_q(st ^ 1);  // stage st ^ 1 was last read before the previous sync
-    __syncthreads();                // every warp is done with stage st
-    st ^= 1;
   }
+  cp_async_wait<0>();  // only empty groups can remain; leave none behind
 
-  float* out = a.part + (size_t)blockIdx.z * a.M * a.N;
 #pragma unroll
   for (int mi = 0; mi < 2; ++mi) {
 #pragma unroll
@@ -229,8 +218,17 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(const SkinnyArgs a) {
         const int64_t m = m0 + wm * 32 + mi * 16 + (lane >> 2) + 8 * h;
         const int64_t n = n0 + wn * WN + nj * 8 + 2 * (lane & 3);
         if (m >= a.M) continue;
-        if (n < a.N) out[m * a.N + n] = acc[mi][nj][2 * h];
-        if (n + 1 < a.N) out[m * a.N + n + 1] = acc[mi][nj][2 * h + 1];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if (n + e >= a.N) continue;
+          const float v = acc[mi][nj][2 * h + e];
+          if (a.direct) {
+            float* d = a.dst + m * a.c_m + (n + e) * a.c_n;
+            *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
+          } else {
+            a.part[((size_t)blockIdx.z * a.M + m) * a.N + n + e] = v;
+          }
+        }
       }
     }
   }
@@ -244,6 +242,8 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
        i += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
+    // unrolled so that several slices' loads are in flight; the adds stay in z order
+#pragma unroll 8
     for (int z = 0; z < splits; ++z) s += part[(size_t)z * n_el + i];
     const int64_t m = i / N, n = i % N;
     float* d = dst + m * c_m + n * c_n;
@@ -251,15 +251,33 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
   }
 }
 
-int bn_for(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : 192; }
+// out[i * ld_out + j] = bf16(in[i * ld_in + j]) for j < cols, 0 for cols <= j < ld_out
+__global__ void to_bf16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
+                                    int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
+  const int64_t n_el = rows * ld_out;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / ld_out, j = i % ld_out;
+    out[i] = j < cols ? float_to_bf16_bits(in[r * ld_in + j]) : (uint16_t)0;
+  }
+}
 
-// Splits of the reduction for a product: about two waves of CTAs on 148 SMs,
-// each slice at least two stages long.
+int64_t pad8(int64_t n) { return (n + 7) / 8 * 8; }
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+int bn_for(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : 192; }
+int ctas_per_sm(int bn) { return bn <= 64 ? 3 : bn <= 128 ? 2 : 1; }
+
+// Splits of the reduction: only where the product's own tiles leave at least
+// half of the resident CTA slots (148 SMs x CTAs per SM) empty, up to filling
+// them, each slice at least four stages long (the partials cost a round trip
+// through HBM, so a grid that already fills the GPU is not split).
 int splits_for(int64_t M, int64_t N, int64_t K) {
+  if (K <= 0 || M <= 0 || N <= 0) return 1;
   const int bn = bn_for(N);
   const int64_t xy = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
-  int64_t z = (2 * 148 + xy - 1) / xy;
-  const int64_t zmax = std::max<int64_t>(1, K / (2 * kBK));
+  int64_t z = (int64_t)kSMs * ctas_per_sm(bn) / xy;
+  const int64_t zmax = std::max<int64_t>(1, K / (4 * kBK));
   z = std::max<int64_t>(1, std::min<int64_t>(z, std::min<int64_t>(zmax, 64)));
   const int64_t kps = ((K + z - 1) / z + kBK - 1) / kBK * kBK;
   return (int)((K + kps - 1) / kps);
@@ -267,7 +285,7 @@ int splits_for(int64_t M, int64_t N, int64_t K) {
 
 template <bool P_RED, bool Q_RED, int BN>
 int launch_bn(const SkinnyArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr size_t smem = skinny_smem_bytes<P_RED, BN>();
+  constexpr size_t smem = Tile<P_RED, Q_RED, BN>::kSmem;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -281,50 +299,100 @@ int launch_bn(const SkinnyArgs& a, dim3 grid, cudaStream_t st) {
   return LSQ_OK;
 }
 
-template <bool P_RED, bool Q_RED>
-int run(const SkinnyArgs& a0, int splits, cudaStream_t st) {
-  SkinnyArgs a = a0;
-  a.k_per_split = ((a.K + splits - 1) / splits + kBK - 1) / kBK * kBK;
-  const int bn = bn_for(a.N);
-  dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)splits);
-  switch (bn) {
-    case 64: return launch_bn<P_RED, Q_RED, 64>(a, grid, st);
-    case 128: return launch_bn<P_RED, Q_RED, 128>(a, grid, st);
-    default: return launch_bn<P_RED, Q_RED, 192>(a, grid, st);
-  }
+int convert_rows(const float* in, int64_t rows, int64_t cols, int64_t ld_in, uint16_t* out,
+                 int64_t ld_out, cudaStream_t st) {
+  int64_t g = (rows * ld_out + 255) / 256;
+  if (g > kSMs * 8) g = kSMs * 8;
+  if (g < 1) return LSQ_OK;
+  to_bf16_rows_kernel<<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
 }
 
-int finish(const float* part, int splits, int64_t M, int64_t N, float alpha, int accumulate,
-           float* dst, int64_t c_m, int64_t c_n, cudaStream_t st) {
-  int64_t g = (M * N + 255) / 256;
-  if (g > 148 * 8) g = 148 * 8;
-  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(part, splits, M, N, alpha, accumulate, dst, c_m,
+// C = P Q over K, then dst[m * c_m + n * c_n] = alpha * C (+ dst if accumulate).
+// scratch holds the bf16 Q (already written at its start) and, after q_bytes,
+// room for the partials when the product is split.
+template <bool P_RED, bool Q_RED>
+int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float* dst,
+        int64_t c_m, int64_t c_n, float alpha, int accumulate, cudaStream_t st) {
+  if (a.M <= 0 || a.N <= 0) return LSQ_OK;
+  const int z = splits_for(a.M, a.N, a.K);
+  const size_t need = align256(q_bytes) + (z > 1 ? (size_t)z * a.M * a.N * sizeof(float) : 0);
+  if (scratch_bytes < need)
+    return set_error(LSQ_ERR_WORKSPACE, "lora product: scratch %zu < %zu", scratch_bytes, need);
+  a.k_per_split = a.K > 0 ? ((a.K + z - 1) / z + kBK - 1) / kBK * kBK : kBK;
+  a.direct = z == 1;
+  a.part = z > 1 ? reinterpret_cast<float*>(scratch + align256(q_bytes)) : nullptr;
+  a.dst = dst;
+  a.c_m = c_m;
+  a.c_n = c_n;
+  a.alpha = alpha;
+  a.accumulate = accumulate;
+  const int bn = bn_for(a.N);
+  dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)z);
+  switch (bn) {
+    case 64: LSQ_TRY((launch_bn<P_RED, Q_RED, 64>(a, grid, st))); break;
+    case 128: LSQ_TRY((launch_bn<P_RED, Q_RED, 128>(a, grid, st))); break;
+    default: LSQ_TRY((launch_bn<P_RED, Q_RED, 192>(a, grid, st))); break;
+  }
+  if (z == 1) return LSQ_OK;
+  int64_t g = (a.M * a.N + 255) / 256;
+  if (g > kSMs * 8) g = kSMs * 8;
+  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, z, a.M, a.N, alpha, accumulate, dst, c_m,
                                                 c_n);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  return LSQ_OK;
+}
+
+int check_ranks(int64_t R) {
+  if (R < 1 || R > 192)
+    return set_error(LSQ_ERR_SHAPE, "lora: rank-r products need 1 <= columns <= 192 (got %lld)",
+                     (long long)R);
   return LSQ_OK;
 }
 
 }  // namespace
 
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
-  // the largest partial buffer a product of these sizes needs:
-  // u or v: M = T, N = R, reduction K;  dA or dB: M = K, N = R, reduction T
-  const size_t a = (size_t)splits_for(T, R, K) * T * R;
-  const size_t b = (size_t)splits_for(K, R, T) * K * R;
-  return std::max(a, b) * sizeof(float);
+  // An upper bound over every product a caller sizing by (T, K, R) can make:
+  // any rank r' <= R per part, a reduction or a part of up to K elements:
+  //   u = x A^T, v part   M = T, N = r', reduction <= K, Q = A [r'][K] or B [<= K][pad8(r')]
+  //   dA, dB part         M <= K, N = r', reduction T,   Q = v or u [T][pad8(r')]
+  // The first needs z(T, r', K) slices at most (splits grow with the reduction);
+  // the second z * M <= min(64, T / (4 kBK)) K, and z * M <= slots * kBM as well,
+  // since z <= slots / (M / kBM tiles).
+  size_t best = 0;
+  for (int rr = 1; rr <= R; ++rr) {
+    const int64_t q1 = K * pad8(rr);
+    const int z1 = splits_for(T, rr, K);
+    best = std::max(best, align256((size_t)q1 * 2) +
+                              (z1 > 1 ? (size_t)z1 * T * rr * sizeof(float) : 0));
+    const int64_t q2 = T * pad8(rr);
+    const int64_t zcap = std::max<int64_t>(1, std::min<int64_t>(64, T / (4 * kBK)));
+    const int64_t zm = std::min<int64_t>(zcap * K, (int64_t)kSMs * ctas_per_sm(bn_for(rr)) * kBM);
+    best = std::max(best, align256((size_t)q2 * 2) +
+                              (zcap > 1 ? (size_t)zm * rr * sizeof(float) : 0));
+  }
+  return best;
 }
 
 int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
                      float* u, float* scratch, size_t scratch_bytes, cudaStream_t st) {
-  const int s = splits_for(T, R, K);
-  const size_t need = (size_t)s * T * R * sizeof(float);
-  if (!scratch || scratch_bytes < need)
-    return set_error(LSQ_ERR_WORKSPACE, "lora_down: scratch %zu < %zu", scratch_bytes, need);
+  LSQ_TRY(check_ranks(R));
+  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
   // C[t, j] = sum_k x[t, k] A[j, k]
-  SkinnyArgs a{x, ldx, 1, A, 1, K, T, R, K, 0, scratch};
+  char* sc = reinterpret_cast<char*>(scratch);
+  uint16_t* Ab = reinterpret_cast<uint16_t*>(sc);
+  const size_t qb = (size_t)R * K * 2;
+  if (!scratch || scratch_bytes < qb)
+    return set_error(LSQ_ERR_WORKSPACE, "lora_down: scratch %zu < %zu", scratch_bytes, qb);
   const int prof = prof_begin(st);
-  LSQ_TRY((run<true, true>(a, s, st)));
-  LSQ_TRY(finish(scratch, s, T, R, 1.f, 0, u, R, 1, st));
+  LSQ_TRY(convert_rows(A, R, K, K, Ab, K, st));
+  SkinnyArgs a{};
+  a.P = x; a.p_m = ldx; a.p_k = 1;
+  a.Q = Ab; a.q_k = 1; a.q_n = K;
+  a.M = T; a.N = R; a.K = K;
+  LSQ_TRY((run<true, true>(a, sc, qb, scratch_bytes, u, R, 1, 1.f, 0, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
   return LSQ_OK;
 }
@@ -332,19 +400,25 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, int n_parts,
                       const int64_t* part_end, float* v, float* scratch, size_t scratch_bytes,
                       cudaStream_t st) {
+  LSQ_TRY(check_ranks(r));
   const int R = n_parts * r;
+  const int64_t r8 = pad8(r);
+  char* sc = reinterpret_cast<char*>(scratch);
+  uint16_t* Bb = reinterpret_cast<uint16_t*>(sc);
   int64_t start = 0;
   for (int p = 0; p < n_parts; ++p) {
     const int64_t Np = part_end[p] - start;
-    const int s = splits_for(T, r, Np);
-    const size_t need = (size_t)s * T * r * sizeof(float);
-    if (!scratch || scratch_bytes < need)
-      return set_error(LSQ_ERR_WORKSPACE, "lora_vproj: scratch %zu < %zu", scratch_bytes, need);
+    const size_t qb = (size_t)Np * r8 * 2;
+    if (!scratch || scratch_bytes < qb)
+      return set_error(LSQ_ERR_WORKSPACE, "lora_vproj: scratch %zu < %zu", scratch_bytes, qb);
     // C[t, j] = sum_n dy[t, start + n] B[start + n, j]
-    SkinnyArgs a{dy + start, N, 1, B + start * r, r, 1, T, r, Np, 0, scratch};
     const int prof = prof_begin(st);
-    LSQ_TRY((run<true, false>(a, s, st)));
-    LSQ_TRY(finish(scratch, s, T, r, 1.f, 0, v + p * r, R, 1, st));
+    LSQ_TRY(convert_rows(B + start * r, Np, r, r, Bb, r8, st));
+    SkinnyArgs a{};
+    a.P = dy + start; a.p_m = N; a.p_k = 1;
+    a.Q = Bb; a.q_k = r8; a.q_n = 1;
+    a.M = T; a.N = r; a.K = Np;
+    LSQ_TRY((run<true, false>(a, sc, qb, scratch_bytes, v + p * r, R, 1, 1.f, 0, st)));
     if (prof >= 0)
       prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
     start = part_end[p];
@@ -355,15 +429,21 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
 int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
                        int accumulate, float* dA, float* scratch, size_t scratch_bytes,
                        cudaStream_t st) {
+  LSQ_TRY(check_ranks(R));
   // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]
-  const int z = splits_for(K, R, T);
-  const size_t need = (size_t)z * K * R * sizeof(float);
-  if (!scratch || scratch_bytes < need)
-    return set_error(LSQ_ERR_WORKSPACE, "lora_grad_a: scratch %zu < %zu", scratch_bytes, need);
-  SkinnyArgs a{x, 1, K, v, R, 1, K, R, T, 0, scratch};
+  const int64_t R8 = pad8(R);
+  const size_t qb = (size_t)T * R8 * 2;
+  if (!scratch || scratch_bytes < qb)
+    return set_error(LSQ_ERR_WORKSPACE, "lora_grad_a: scratch %zu < %zu", scratch_bytes, qb);
+  char* sc = reinterpret_cast<char*>(scratch);
+  uint16_t* vb = reinterpret_cast<uint16_t*>(sc);
   const int prof = prof_begin(st);
-  LSQ_TRY((run<false, false>(a, z, st)));
-  LSQ_TRY(finish(scratch, z, K, R, s, accumulate, dA, 1, K, st));
+  LSQ_TRY(convert_rows(v, T, R, R, vb, R8, st));
+  SkinnyArgs a{};
+  a.P = x; a.p_m = 1; a.p_k = K;
+  a.Q = vb; a.q_k = R8; a.q_n = 1;
+  a.M = K; a.N = R; a.K = T;
+  LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dA, 1, K, s, accumulate, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
   return LSQ_OK;
 }
@@ -371,18 +451,25 @@ int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, 
 int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
                        int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
                        float* scratch, size_t scratch_bytes, cudaStream_t st) {
+  LSQ_TRY(check_ranks(r));
+  const int64_t r8 = pad8(r);
+  const size_t qb = (size_t)T * r8 * 2;
+  if (!scratch || scratch_bytes < qb)
+    return set_error(LSQ_ERR_WORKSPACE, "lora_grad_b: scratch %zu < %zu", scratch_bytes, qb);
+  char* sc = reinterpret_cast<char*>(scratch);
+  uint16_t* ub = reinterpret_cast<uint16_t*>(sc);
   int64_t start = 0;
   for (int p = 0; p < n_parts; ++p) {
     const int64_t Np = part_end[p] - start;
     // C[n, j] = sum_t dy[t, start + n] u[t, p r + j];  dB[start + n, j] (+)= s C[n, j]
-    const int z = splits_for(Np, r, T);
-    const size_t need = (size_t)z * Np * r * sizeof(float);
-    if (!scratch || scratch_bytes < need)
-      return set_error(LSQ_ERR_WORKSPACE, "lora_grad_b: scratch %zu < %zu", scratch_bytes, need);
-    SkinnyArgs a{dy + start, 1, N, u + p * r, R, 1, Np, r, T, 0, scratch};
     const int prof = prof_begin(st);
-    LSQ_TRY((run<false, false>(a, z, st)));
-    LSQ_TRY(finish(scratch, z, Np, r, s, accumulate, dB + start * r, r, 1, st));
+    LSQ_TRY(convert_rows(u + p * r, T, r, R, ub, r8, st));
+    SkinnyArgs a{};
+    a.P = dy + start; a.p_m = 1; a.p_k = N;
+    a.Q = ub; a.q_k = r8; a.q_n = 1;
+    a.M = Np; a.N = r; a.K = T;
+    LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dB + start * r, r, 1, s, accumulate,
+                               st)));
     if (prof >= 0)
       prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
     start = part_end[p];

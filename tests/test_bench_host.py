@@ -1,0 +1,26 @@
+"""Host-side logic of bench.py (no GPU): which kernel class the roofline object describes."""
+import importlib.util
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(HERE, "..", "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    return b
+
+
+def test_roofline_subject_is_a_single_kernel():
+    b = _bench()
+    # the rank-r region (three kernels per timed region) has the most event time here,
+    # but the roofline object must name one kernel: the NF4 forward GEMM
+    prof = {"lora_rank_r": dict(total_ms=168.0, launches=4160),
+            "gemm_nf4_fwd": dict(total_ms=137.5, launches=1120),
+            "gemm_nf4_dx": dict(total_ms=76.0, launches=640)}
+    assert b.dominant_kernel(prof)[0] == "gemm_nf4_fwd"
+    prof["attention_fwd"] = dict(total_ms=140.0, launches=320)
+    assert b.dominant_kernel(prof)[0] == "attention_fwd"
+    # a profile holding only multi-kernel classes still yields a subject
+    assert b.dominant_kernel({"lora_rank_r": dict(total_ms=1.0, launches=1)})[0] == "lora_rank_r"
