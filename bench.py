@@ -102,6 +102,10 @@ def parse():
                          "step (beta 0.1, adapter-off reference); layer: one resident "
                          "8B-shaped layer forward + recomputing backward; gemm: one fused NF4 "
                          "GEMM at the q|k|v shape (a small case for profiling)")
+    ap.add_argument("--shard-layers", action="store_true",
+                    help="data-parallel layer sharding: each of the N ranks copies 1/N of every "
+                         "layer from host memory and an NCCL all-gather on the GPUs assembles it "
+                         "(stream_stack_shard); off by default")
     return ap.parse_args()
 
 
@@ -229,7 +233,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
-def build_stack(L, cfg, rank, tok_shape=(1, SEQ), tied=False):
+def build_stack(L, cfg, rank, tok_shape=(1, SEQ), tied=False, buf_bytes=None):
     import torch
     from layer_streamed_qlora_nf4_b200 import pack, synth
     lay = L.lsq_layer_layout_get(cfg)
@@ -255,7 +259,7 @@ def build_stack(L, cfg, rank, tok_shape=(1, SEQ), tied=False):
     gt = torch.Generator(device="cuda").manual_seed(1000 + rank)
     tokens = torch.randint(0, cfg["vocab"], (8,) + tuple(tok_shape), generator=gt, device="cuda",
                            dtype=torch.int32)
-    bufs = [torch.empty(lay.bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    bufs = [torch.empty(buf_bytes or lay.bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
     return dict(lay=lay, host_blobs=host_blobs, lora=lora, emb=emb, head=head, gf=ones,
                 tokens=tokens, bufs=bufs)
 
@@ -297,9 +301,14 @@ def run_ours(args):
     batch, mbs = (2 * args.pairs, 1) if dpo else (batch, args.micro_batches)
     tok_shape = (args.pairs, 2, SEQ) if dpo else (mbs, batch, SEQ)
     tokens_per_step = mbs * batch * SEQ
-    st = build_stack(L, cfg, rank, tok_shape, tied=qwen)
+    buf_bytes = None
+    if args.shard_layers:
+        buf_bytes = world * L.lsq_shard_bytes(L.lsq_layer_layout_get(cfg).bytes, world)
+    st = build_stack(L, cfg, rank, tok_shape, tied=qwen, buf_bytes=buf_bytes)
     lay = st["lay"]
     handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
+    if args.shard_layers:
+        dp.shard_stack(L, handle, buf_bytes)
     ws_bytes = (L.stream_stack_dpo_workspace_bytes(cfg, args.pairs, SEQ) if dpo
                 else L.stream_stack_workspace_bytes(cfg, batch, SEQ))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -328,7 +337,7 @@ def run_ours(args):
         CUDA events on the compute stream, max over ranks)."""
         dp.barrier()
         torch.cuda.synchronize()
-        copies, wait_ms = 0, 0.0
+        copies, wait_ms, h2d = 0, 0.0, 0
         if profile:
             L.lsq_profile_enable(True)
         n0 = L.lsq_launch_counter()
@@ -340,6 +349,7 @@ def run_ours(args):
             loss = step(tokens_of(i))
             s = L.stream_stack_last_stats(handle)
             copies += s["layer_copies"]
+            h2d += s["h2d_bytes"]
             wait_ms += s["copy_wait_ms"]
         torch.cuda.nvtx.range_pop()
         e1.record(stream)
@@ -351,7 +361,7 @@ def run_ours(args):
             L.lsq_profile_enable(False)
             prof = L.lsq_profile_read()
         ms = dp.max_over_ranks(e0.elapsed_time(e1) / steps, "cuda")
-        return ms, loss, copies, wait_ms, launches, prof
+        return ms, loss, (copies, h2d), wait_ms, launches, prof
 
     for i in range(args.warmup):
         loss = step(pool[i % len(pool)])
@@ -362,7 +372,8 @@ def run_ours(args):
     uuid = str(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "uuid", ""))
     sampler = ClockSampler(uuid)
     sampler.start()
-    ms, loss, copies, wait_ms, launches, _ = timed(args.steps, lambda i: pool[i % len(pool)])
+    ms, loss, (copies, h2d), wait_ms, launches, _ = timed(args.steps,
+                                                          lambda i: pool[i % len(pool)])
     clocks = sampler.stop()
     value = world * tokens_per_step / (ms * 1e-3)
 
@@ -381,7 +392,7 @@ def run_ours(args):
     e2e_ms = timed(args.steps, from_host, label="timed_e2e")[0]
     e2e = dict(value=world * tokens_per_step / (e2e_ms * 1e-3), unit="tokens/s",
                h2d_bytes_per_step=tok_dev.numel() * 4, d2h_bytes_per_step=4,
-               layer_stream_h2d_bytes_per_step=copies // args.steps * lay.bytes)
+               layer_stream_h2d_bytes_per_step=h2d // args.steps)
 
     pk = peaks()
     dom_name, dom = dominant_kernel(prof)
@@ -409,12 +420,18 @@ def run_ours(args):
     cps = copies / args.steps
     t_tc = flops_step / (pk["bf16_tflops_sustained"] * 1e12) * 1e3
     t_hbm = (bytes_step + cps * lay.bytes) / (pk["hbm_gbs"] * 1e9) * 1e3
-    t_h2d = cps * lay.bytes / (h2d_gbs * 1e9) * 1e3
-    t_roof = max(t_tc, t_hbm, t_h2d)
-    step_roof = dict(t_tensor_ms=t_tc, t_hbm_ms=t_hbm, t_h2d_ms=t_h2d,
-                     bound=["tensor", "hbm", "h2d"][[t_tc, t_hbm, t_h2d].index(t_roof)],
+    # this rank's host->device bytes (a 1/N slice of each layer when sharded)
+    t_h2d = h2d / args.steps / (h2d_gbs * 1e9) * 1e3
+    # sharded: each GPU receives the other ranks' slices over NVLink (measured peer
+    # copy bandwidth, 770 GB/s per direction)
+    t_nvl = (cps * lay.bytes * (world - 1) / world / 770e9 * 1e3) if args.shard_layers else 0.0
+    t_roof = max(t_tc, t_hbm, t_h2d, t_nvl)
+    step_roof = dict(t_tensor_ms=t_tc, t_hbm_ms=t_hbm, t_h2d_ms=t_h2d, t_nvlink_ms=t_nvl,
+                     bound=["tensor", "hbm", "h2d", "nvlink"][
+                         [t_tc, t_hbm, t_h2d, t_nvl].index(t_roof)],
                      frac=t_roof / ms, frac_e2e=t_roof / e2e_ms, h2d_gbs_measured=h2d_gbs,
                      layer_copies_per_step=cps, layer_bytes=lay.bytes,
+                     h2d_bytes_per_step=h2d / args.steps,
                      copy_wait_ms_per_step=wait_ms / args.steps,
                      tflop_per_step=flops_step / 1e12,
                      kernels={k: dict(launches_per_step=e["launches"] / args.steps,
@@ -440,7 +457,8 @@ def run_ours(args):
                     config=dict(workload=WORKLOAD_QWEN if qwen else
                                 workload_name(args.absmax_bits, dpo, args.pairs, batch, mbs),
                                 global_batch=world * tokens_per_step // SEQ, seq_len=SEQ,
-                                parallelism="dp%d" % world,
+                                parallelism="dp%d" % world + (
+                                    " + layer all-gather" if args.shard_layers else ""),
                                 l2="inputs larger than L2: %.2f GB of layer bytes stream per step"
                                 % (cps * lay.bytes / 1e9)),
                     loss=loss, roofline=roofline, step_roofline=step_roof, cpu_baseline=cpu,

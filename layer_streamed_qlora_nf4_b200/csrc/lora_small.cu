@@ -3,8 +3,9 @@
 // For y = x W^T + s (x A^T) B^T (Soup layer-streaming tutorial, "四段資料路徑"
 // part 1) and its backward (part 3): u = x A^T (forward), v = dY B, and the
 // trainable gradients dA = s v^T x, dB = s dY^T u.  All four are "tall x
-// skinny" products: C[m, n] = sum_k P(m, k) Q(k, n) with n spanning at most
-// 3 r <= 192 columns, P a bf16 activation and Q an fp32 LoRA tensor.
+// skinny" products: C[m, n] = sum_k P(m, k) Q(k, n) with n spanning r to 3 r
+// columns (one tile of up to 192 columns, more tiles beyond), P a bf16
+// activation and Q an fp32 LoRA tensor.
 //
 // One kernel serves all four.  A CTA owns 128 rows x BN columns of C over one
 // slice of the reduction.  Q is first rounded once to bf16 (nearest even) into
@@ -345,8 +346,8 @@ int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float
 }
 
 int check_ranks(int64_t R) {
-  if (R < 1 || R > 192)
-    return set_error(LSQ_ERR_SHAPE, "lora: rank-r products need 1 <= columns <= 192 (got %lld)",
+  if (R < 1)
+    return set_error(LSQ_ERR_SHAPE, "lora: rank-r products need at least one column (got %lld)",
                      (long long)R);
   return LSQ_OK;
 }

@@ -18,8 +18,22 @@
 // buffer ("free"); the compute stream waits on the event recorded after the
 // copy ("ready").  Copies run one visit ahead.  Kernels are deterministic, so
 // a streamed step is bit-identical to the same step with the stack resident.
+//
+// Data-parallel layer sharding (stream_stack_shard): with G ranks, one process
+// per GPU, each rank copies only its 1/G slice of a layer from host memory, and
+// an in-place NCCL all-gather on the copy stream (NVLink / NVSwitch, far faster
+// than each GPU's own host link) assembles the whole layer in every rank's
+// buffer before the "ready" event.  Per-GPU host->device bytes fall by G.  The
+// NCCL library is loaded at run time (the one torch already loaded, else the
+// system's), so the library has no link-time dependency on it.
+#include <dlfcn.h>
+#include <nccl.h>
+#include <string.h>
+
+#include <algorithm>
 #include <chrono>
 #include <cmath>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -42,6 +56,12 @@ struct lsq_stack {
   float* loss_host;            // pinned: [0] loss, [1 ..] DPO log-probabilities
   lsq_step_stats stats;
   int n_waits_last;
+  // data-parallel layer sharding (stream_stack_shard); shard == 0: every layer
+  // is copied whole from this rank's host blob
+  int world = 1, rank = 0;
+  size_t shard = 0;            // bytes of a layer each rank fetches from host
+  void* comm = nullptr;        // ncclComm_t
+  int aborted = 0;             // the communicator was aborted after a timeout
 };
 
 namespace lsq {
@@ -179,6 +199,76 @@ std::vector<Visit> plan_visits(int L, int micro_batches, int bl0, int bl1) {
   return v;
 }
 
+// NCCL entry points, resolved once from libnccl.so.2 at run time.
+struct NcclFns {
+  decltype(&ncclGetUniqueId) get_unique_id = nullptr;
+  decltype(&ncclCommInitRank) init_rank = nullptr;
+  decltype(&ncclAllGather) all_gather = nullptr;
+  decltype(&ncclCommDestroy) destroy = nullptr;
+  decltype(&ncclCommAbort) abort = nullptr;
+  decltype(&ncclGetErrorString) error_string = nullptr;
+};
+
+int nccl_fns(const NcclFns** out) {
+  static std::mutex mu;
+  static NcclFns f;
+  static int state = 0;  // 0 not tried, 1 loaded, -1 missing
+  std::lock_guard<std::mutex> g(mu);
+  if (state == 0) {
+    state = -1;
+    void* lib = dlopen("libnccl.so.2", RTLD_NOW | RTLD_LOCAL);
+    if (lib) {
+      f.get_unique_id = reinterpret_cast<decltype(f.get_unique_id)>(dlsym(lib, "ncclGetUniqueId"));
+      f.init_rank = reinterpret_cast<decltype(f.init_rank)>(dlsym(lib, "ncclCommInitRank"));
+      f.all_gather = reinterpret_cast<decltype(f.all_gather)>(dlsym(lib, "ncclAllGather"));
+      f.destroy = reinterpret_cast<decltype(f.destroy)>(dlsym(lib, "ncclCommDestroy"));
+      f.abort = reinterpret_cast<decltype(f.abort)>(dlsym(lib, "ncclCommAbort"));
+      f.error_string =
+          reinterpret_cast<decltype(f.error_string)>(dlsym(lib, "ncclGetErrorString"));
+      if (f.get_unique_id && f.init_rank && f.all_gather && f.destroy && f.abort &&
+          f.error_string)
+        state = 1;
+    }
+  }
+  if (state != 1)
+    return set_error(LSQ_ERR_CUDA, "NCCL (libnccl.so.2) is not loadable or lacks an entry point");
+  *out = &f;
+  return LSQ_OK;
+}
+
+// This rank's slice of a layer of `bytes`: [off, off + len) of the blob.
+void shard_slice(const lsq_stack* h, size_t bytes, size_t* off, size_t* len) {
+  *off = (size_t)h->rank * h->shard;
+  *len = *off < bytes ? std::min(h->shard, bytes - *off) : 0;
+}
+
+// Sharded fetch of `layer` into buffer b, on the copy stream: this rank's slice
+// from host, then the in-place all-gather of every rank's slice.
+int shard_fetch(lsq_stack* h, int b, int layer, size_t bytes) {
+  const NcclFns* f = nullptr;
+  LSQ_TRY(nccl_fns(&f));
+  size_t off = 0, len = 0;
+  shard_slice(h, bytes, &off, &len);
+  uint8_t* dst = static_cast<uint8_t*>(h->buf[b]);
+  if (len)
+    LSQ_CUDA(cudaMemcpyAsync(dst + off, static_cast<const uint8_t*>(h->blobs[layer]) + off, len,
+                             cudaMemcpyHostToDevice, h->copy_stream));
+  const ncclResult_t r = f->all_gather(dst + off, dst, h->shard, ncclUint8,
+                                       static_cast<ncclComm_t>(h->comm), h->copy_stream);
+  if (r != ncclSuccess)
+    return set_error(LSQ_ERR_CUDA, "ncclAllGather: %s", f->error_string(r));
+  return LSQ_OK;
+}
+
+// After a step timed out: abort the communicator, which ends any all-gather
+// still waiting for a peer, and refuse further steps on this stack.
+void shard_abort(lsq_stack* h) {
+  const NcclFns* f = nullptr;
+  if (h->comm && nccl_fns(&f) == LSQ_OK) f->abort(static_cast<ncclComm_t>(h->comm));
+  h->comm = nullptr;
+  h->aborted = 1;
+}
+
 int wait_event_timeout(cudaEvent_t ev, int64_t timeout_ms) {
   const auto t0 = std::chrono::steady_clock::now();
   while (true) {
@@ -285,6 +375,8 @@ extern "C" int stream_stack_destroy(lsq_stack* h) {
   cudaEventDestroy(h->t_end);
   cudaEventDestroy(h->done);
   cudaFreeHost(h->loss_host);
+  const NcclFns* f = nullptr;
+  if (h->comm && nccl_fns(&f) == LSQ_OK) f->destroy(static_cast<ncclComm_t>(h->comm));
   delete h;
   return LSQ_OK;
 }
@@ -292,6 +384,62 @@ extern "C" int stream_stack_destroy(lsq_stack* h) {
 extern "C" int stream_stack_last_stats(const lsq_stack* h, lsq_step_stats* out) {
   if (!h || !out) return set_error(LSQ_ERR_INVALID, "stream_stack_last_stats: null pointer");
   *out = h->stats;
+  return LSQ_OK;
+}
+
+extern "C" int64_t lsq_shard_bytes(int64_t layer_bytes, int32_t world) {
+  if (layer_bytes <= 0 || world < 1) return 0;
+  const int64_t s = (layer_bytes + world - 1) / world;
+  return (s + 255) / 256 * 256;
+}
+
+extern "C" int lsq_nccl_unique_id(void* id_out, int64_t id_bytes) {
+  if (!id_out || id_bytes != (int64_t)sizeof(ncclUniqueId))
+    return set_error(LSQ_ERR_INVALID, "lsq_nccl_unique_id: need a %d-byte output",
+                     (int)sizeof(ncclUniqueId));
+  const NcclFns* f = nullptr;
+  LSQ_TRY(nccl_fns(&f));
+  ncclUniqueId id;
+  const ncclResult_t r = f->get_unique_id(&id);
+  if (r != ncclSuccess) return set_error(LSQ_ERR_CUDA, "ncclGetUniqueId: %s", f->error_string(r));
+  memcpy(id_out, &id, sizeof(id));
+  return LSQ_OK;
+}
+
+extern "C" int stream_stack_shard(lsq_stack* h, const void* nccl_id, int64_t id_bytes,
+                                  int32_t world, int32_t rank, int64_t buf_bytes) {
+  if (!h || !nccl_id) return set_error(LSQ_ERR_INVALID, "stream_stack_shard: null pointer");
+  if (id_bytes != (int64_t)sizeof(ncclUniqueId))
+    return set_error(LSQ_ERR_INVALID, "stream_stack_shard: the id has %d bytes",
+                     (int)sizeof(ncclUniqueId));
+  if (h->resident)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_shard: a resident stack copies no layers");
+  if (h->shard || h->comm || h->aborted)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_shard: the stack is already sharded");
+  if (world < 1 || rank < 0 || rank >= world)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_shard: rank %d of world %d", rank, world);
+  const int64_t S = lsq_shard_bytes((int64_t)h->layout.bytes, world);
+  if (buf_bytes < S * world)
+    return set_error(LSQ_ERR_WORKSPACE,
+                     "stream_stack_shard: layer buffers of %lld bytes, %lld needed (world x %lld)",
+                     (long long)buf_bytes, (long long)(S * world), (long long)S);
+  int dev = -1;
+  LSQ_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_shard: call on the stack's device (%d, not %d)",
+                     h->device, dev);
+  const NcclFns* f = nullptr;
+  LSQ_TRY(nccl_fns(&f));
+  ncclUniqueId id;
+  memcpy(&id, nccl_id, sizeof(id));
+  ncclComm_t comm = nullptr;
+  const ncclResult_t r = f->init_rank(&comm, world, id, rank);
+  if (r != ncclSuccess)
+    return set_error(LSQ_ERR_CUDA, "ncclCommInitRank: %s", f->error_string(r));
+  h->comm = comm;
+  h->world = world;
+  h->rank = rank;
+  h->shard = (size_t)S;
   return LSQ_OK;
 }
 
@@ -314,6 +462,9 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
               float* loss_out, float* logits_out, void* ws, size_t ws_bytes, void* stream,
               int64_t timeout_ms, const DpoArgs* dpo) {
   if (!h) return set_error(LSQ_ERR_INVALID, "stream_stack_step: null handle");
+  if (h->aborted)
+    return set_error(LSQ_ERR_INVALID,
+                     "stream_stack_step: the stack's communicator was aborted after a timeout");
   if (!tokens || !emb || !lm_head || !final_norm || !lora || !lora_grad || !loss_out)
     return set_error(LSQ_ERR_INVALID, "stream_stack_step: null pointer");
   if (micro_batches <= 0 || batch <= 0 || seq < 2)
@@ -354,8 +505,11 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
     const Visit& x = visits[j];
     if (!x.copy) return LSQ_OK;
     LSQ_CUDA(cudaStreamWaitEvent(h->copy_stream, h->freed[x.buf], 0));
-    LSQ_CUDA(cudaMemcpyAsync(h->buf[x.buf], h->blobs[x.layer], bytes, cudaMemcpyHostToDevice,
-                             h->copy_stream));
+    if (h->shard)
+      LSQ_TRY(shard_fetch(h, x.buf, x.layer, bytes));
+    else
+      LSQ_CUDA(cudaMemcpyAsync(h->buf[x.buf], h->blobs[x.layer], bytes, cudaMemcpyHostToDevice,
+                               h->copy_stream));
     LSQ_CUDA(cudaEventRecord(h->ready[x.buf], h->copy_stream));
     ++copies;
     return LSQ_OK;
@@ -373,6 +527,10 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   };
 
   LSQ_CUDA(cudaEventRecord(h->t_start, cs));
+  // Sharded: the step's first all-gather waits for everything the caller put on
+  // the compute stream before the step (e.g. a gradient all-reduce on another
+  // communicator), so that collectives of the two never run interleaved.
+  if (h->shard) LSQ_CUDA(cudaStreamWaitEvent(h->copy_stream, h->t_start, 0));
   if (!h->resident && !visits.empty()) LSQ_TRY(enqueue_copy(0));
   size_t j = 0;
   for (int mb = 0; mb < micro_batches; ++mb) {
@@ -433,7 +591,13 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
                              cudaMemcpyDeviceToHost, cs));
   LSQ_CUDA(cudaEventRecord(h->t_end, cs));
   LSQ_CUDA(cudaEventRecord(h->done, cs));
-  LSQ_TRY(wait_event_timeout(h->done, timeout_ms));
+  {
+    const int rc = wait_event_timeout(h->done, timeout_ms);
+    if (rc != LSQ_OK) {
+      if (rc == LSQ_ERR_TIMEOUT && h->comm) shard_abort(h);
+      return rc;
+    }
+  }
   int flags = 0;
   int* st = device_status_ptr();
   if (st) {
@@ -451,7 +615,12 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   if (dpo && dpo->logps_out)
     for (int k = 0; k < 4 * dpo->pairs; ++k) dpo->logps_out[k] = h->loss_host[1 + k];
   h->stats.layer_copies = copies;
-  h->stats.h2d_bytes = (int64_t)copies * (int64_t)bytes;
+  size_t fetched = bytes;
+  if (h->shard) {
+    size_t off = 0;
+    shard_slice(h, bytes, &off, &fetched);
+  }
+  h->stats.h2d_bytes = (int64_t)copies * (int64_t)fetched;
   cudaEventElapsedTime(&h->stats.step_ms, h->t_start, h->t_end);
   float wait_ms = 0.f;
   if (!h->resident) {

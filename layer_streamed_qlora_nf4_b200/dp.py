@@ -53,3 +53,21 @@ def barrier():
 def token_seed(base, rank):
     """Each rank draws its own micro-batches."""
     return base + 1000 * rank
+
+
+def broadcast_bytes(make, src=0):
+    """The bytes `make()` returns on rank `src`, delivered to every rank (host channel)."""
+    multi = dist.is_initialized() and dist.get_world_size() > 1
+    obj = [make() if (not multi or dist.get_rank() == src) else None]
+    if multi:
+        dist.broadcast_object_list(obj, src=src)
+    return obj[0]
+
+
+def shard_stack(L, stack, buf_bytes):
+    """stream_stack_shard over this job's ranks: rank 0 makes the NCCL id, every
+    rank joins with its own rank.  Each layer copy is then split over the ranks
+    and reassembled by an all-gather on the GPUs."""
+    rank, world = ((dist.get_rank(), dist.get_world_size()) if dist.is_initialized() else (0, 1))
+    stack.shard(broadcast_bytes(L.lsq_nccl_unique_id), world, rank, buf_bytes)
+

@@ -26,7 +26,9 @@ EXPORTS = (
     "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
     "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
+    "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard",
 )
+LSQ_NCCL_ID_BYTES = 128
 
 
 class LsqError(RuntimeError):
@@ -116,6 +118,9 @@ _PROTOS = {
                                              ctypes.POINTER(ctypes.c_float), _P, _P, _SZ, _P,
                                              _I64]),
     "lora_adamw_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(lsq_adamw), _I64, _P]),
+    "lsq_shard_bytes": (_I64, [_I64, _I32]),
+    "lsq_nccl_unique_id": (ctypes.c_int, [_P, _I64]),
+    "stream_stack_shard": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64]),
     "lsq_launch_counter": (ctypes.c_int64, []),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
                                                    _F, _P, _P, _P, _P]),
@@ -285,6 +290,10 @@ class StreamStack:
                                           _ptr(buf0), _ptr(buf1), 1 if resident else 0,
                                           ctypes.byref(self.handle)))
 
+    def shard(self, nccl_id, world, rank, buf_bytes):
+        """stream_stack_shard: spread every layer copy over `world` ranks."""
+        stream_stack_shard(self, nccl_id, world, rank, buf_bytes)
+
     def close(self):
         if self.handle:
             _check(load().stream_stack_destroy(self.handle))
@@ -295,6 +304,26 @@ class StreamStack:
             self.close()
         except Exception:
             pass
+
+
+def lsq_shard_bytes(layer_bytes, world):
+    return int(load().lsq_shard_bytes(int(layer_bytes), int(world)))
+
+
+def lsq_nccl_unique_id():
+    """-> bytes (LSQ_NCCL_ID_BYTES) of a new NCCL communicator id."""
+    buf = ctypes.create_string_buffer(LSQ_NCCL_ID_BYTES)
+    _check(load().lsq_nccl_unique_id(buf, LSQ_NCCL_ID_BYTES))
+    return buf.raw
+
+
+def stream_stack_shard(stack, nccl_id, world, rank, buf_bytes):
+    nccl_id = bytes(nccl_id)
+    if len(nccl_id) != LSQ_NCCL_ID_BYTES:
+        raise ValueError("the NCCL id has %d bytes" % LSQ_NCCL_ID_BYTES)
+    buf = ctypes.create_string_buffer(nccl_id, LSQ_NCCL_ID_BYTES)
+    _check(load().stream_stack_shard(stack.handle, buf, LSQ_NCCL_ID_BYTES, int(world), int(rank),
+                                     int(buf_bytes)))
 
 
 def stream_stack_workspace_bytes(cfg, batch, seq):

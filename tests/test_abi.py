@@ -134,3 +134,15 @@ def test_invalid_arguments_are_rejected_without_a_gpu(L):
     arr = (ctypes.c_void_p * 2)(16, 32)
     assert lib.stream_stack_create(ctypes.byref(c), arr, 2, p, p, 0, ctypes.byref(h)) == L.LSQ_ERR_SHAPE
     assert lib.stream_stack_destroy(None) == L.LSQ_OK
+
+
+def test_shard_bytes(L):
+    assert L.lsq_shard_bytes(122_699_776, 8) == 15_337_472          # 1/8 of an 8B layer
+    assert L.lsq_shard_bytes(122_699_776, 1) == 122_699_776
+    assert L.lsq_shard_bytes(1000, 3) == 512                        # ceil(1000/3) -> 256 B units
+    assert L.lsq_shard_bytes(0, 4) == 0 and L.lsq_shard_bytes(100, 0) == 0
+    for b in (1, 255, 257, 4096, 112_529_408):
+        for w in (1, 2, 3, 7, 8):
+            S = L.lsq_shard_bytes(b, w)
+            assert S % 256 == 0 and S * w >= b and (S - 256) * w < b
+

@@ -113,3 +113,56 @@ def test_two_rank_sft_step_equals_the_union_batch():
                           for i in range(2) for n in om.PROJ])
     assert abs(l0 - loss) <= 1e-12 * abs(loss)
     assert np.max(np.abs(f0 - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def _shard_worker(rank, world, port, sizes, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    from layer_streamed_qlora_nf4_b200 import dp
+    from layer_streamed_qlora_nf4_b200 import lib as L
+    L.load()                     # lsq_shard_bytes is host-only
+    dp.init("gloo", timeout_s=60)
+    nid = dp.broadcast_bytes(lambda: os.urandom(L.LSQ_NCCL_ID_BYTES))
+    res = []
+    for nbytes in sizes:
+        S = L.lsq_shard_bytes(nbytes, world)
+        # every rank holds the same frozen layer in host memory
+        blob = torch.from_numpy(np.random.default_rng(nbytes).integers(0, 256, nbytes, np.uint8))
+        buf = torch.zeros(world * S, dtype=torch.uint8)             # this rank's layer buffer
+        off = rank * S
+        ln = max(0, min(S, nbytes - off))
+        buf[off:off + ln] = blob[off:off + ln]                       # its host->device slice
+        parts = [torch.empty(S, dtype=torch.uint8) for _ in range(world)]
+        torch.distributed.all_gather(parts, buf[off:off + S].clone())  # the in-place all-gather
+        buf = torch.cat(parts)
+        res.append((S, ln, bool(torch.equal(buf[:nbytes], blob))))
+    out[rank] = (nid, res)
+    dp.barrier()
+    torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_layer_shard_plan_reassembles_the_layer(world):
+    """Each rank copies only bytes [r S, min((r+1) S, bytes)) of a layer (the
+    slice stream_stack_shard documents, S from lsq_shard_bytes) and the
+    all-gather of the ranks' S-byte slots rebuilds the layer on every rank; the
+    NCCL id made on rank 0 reaches every rank unchanged."""
+    sizes = [300, 1000, 3 * 4096 + 17, 122_699_776]   # the last: one 8B NF4 layer
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, sizes, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        assert p.exitcode == 0
+    ids = {out[r][0] for r in range(world)}
+    assert len(ids) == 1 and len(ids.pop()) == 128
+    for k, nbytes in enumerate(sizes):
+        S = out[0][1][k][0]
+        assert S % 256 == 0 and S * world >= nbytes and (S - 256) * world < nbytes
+        assert sum(out[r][1][k][1] for r in range(world)) == nbytes   # every byte read once
+        assert all(out[r][1][k][2] for r in range(world))

@@ -93,6 +93,15 @@ def test_linear_rank_32(L):
     _run(L, N=512, K=1024, T=130, r=32, alpha=64.0, seed=5)
 
 
+@pytest.mark.parametrize("N,K,T,r", [
+    (96, 128, 200, 96),     # every rank-r product unsplit (written directly), 128-column tile
+    (384, 512, 130, 192),   # one 192-column tile; u and v split, dA and dB direct
+    (256, 256, 64, 256),    # two column tiles (192 + 64)
+])
+def test_linear_wide_ranks(L, N, K, T, r):
+    _run(L, N=N, K=K, T=T, r=r, alpha=2.0 * r, seed=N + r)
+
+
 @pytest.mark.parametrize("N,K", [(4096, 4096), (1024, 4096), (4096, 14336)])
 def test_linear_8b_shapes(L, N, K):
     _run(L, N=N, K=K, T=512, seed=N + K)
