@@ -363,10 +363,12 @@ def run_ours(args):
         ms = dp.max_over_ranks(e0.elapsed_time(e1) / steps, "cuda")
         return ms, loss, (copies, h2d), wait_ms, launches, prof
 
+    # measured before the first step: the handle then holds no layer in its buffers,
+    # so overwriting buffer 0 here cannot leave it a stale layer to reuse
+    h2d_gbs = h2d_bandwidth(st["host_blobs"], st["bufs"][0])
     for i in range(args.warmup):
         loss = step(pool[i % len(pool)])
     torch.cuda.synchronize()
-    h2d_gbs = h2d_bandwidth(st["host_blobs"], st["bufs"][0])
 
     # ------------------------------------------------------------ timed region (headline)
     uuid = str(getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "uuid", ""))
