@@ -138,9 +138,11 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st);
 int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 
-// LoRA skinny products (CUDA cores, fixed-order fp32 reductions)
+// LoRA rank-r products (tensor cores, bf16 operands, fp32 accumulation, fixed-order
+// reductions)
 // u[t, j] = sum_k x[t, k] * A[j, k]                     x bf16 [T, K], A fp32 [R, K] -> u [T, R]
-// scratch: lora_scratch_bytes(T, K, R) bytes for the fixed-order K-split partials
+// scratch: lora_scratch_bytes(T, K, R) bytes for the bf16 copy of the LoRA operand and the
+// fixed-order partials of a product split along its reduction
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
 int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K,
                      int R, float* u, float* scratch, size_t scratch_bytes, cudaStream_t st);
