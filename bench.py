@@ -39,11 +39,12 @@ BATCH, SEQ = 1, 512
 # backward; each launch reads its algorithmic bytes once).  The per-step mix of
 # launches is the same as in that layer, so the averages hold for the step.
 DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 37.26e6, "gemm_nf4_dx": 42.45e6}
-# Profiler classes whose one timed region spans several kernels (the rank-r
-# products: bf16 copy of the LoRA operand, the product, the fixed-order sum of
-# its reduction slices).  The roofline object describes one kernel, so these
-# are reported in step_roofline.kernels but never chosen as its subject.
-MULTI_KERNEL_CLASSES = ("lora_rank_r",)
+# Profiler classes whose one timed region spans several kernels: the rank-r
+# products lora_rank_r_{u,v,dA,dB} (bf16 copy of the LoRA operand, the product,
+# the fixed-order sum of its reduction slices).  The roofline object describes
+# one kernel, so these are reported in step_roofline.kernels (each, and summed
+# as "lora_rank_r") but never chosen as its subject.
+MULTI_KERNEL_PREFIXES = ("lora_rank_r",)
 METRIC_QWEN = ("streamed LoRA train tokens/sec (Qwen2.5-3B shapes, bf16 base, seq 2048) and % of "
                "step roofline")
 WORKLOAD_QWEN = ("Qwen2.5-3B-shaped 36-layer stack, unquantised bf16 weights (154.1 MB per "
@@ -55,8 +56,22 @@ FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=
 
 def dominant_kernel(prof):
     """The single-kernel class with the most device time in the profiled steps."""
-    single = {k: v for k, v in prof.items() if k not in MULTI_KERNEL_CLASSES}
+    single = {k: v for k, v in prof.items() if not k.startswith(MULTI_KERNEL_PREFIXES)}
     return max((single or prof).items(), key=lambda kv: kv[1]["total_ms"])
+
+
+def kernel_table(prof, steps):
+    """Per-step launches, time, TF/s and algorithmic GB/s of every profiled class,
+    plus the rank-r products summed over their kinds as "lora_rank_r"."""
+    rows = dict(prof)
+    kinds = [v for k, v in prof.items() if k.startswith("lora_rank_r_")]
+    if kinds:
+        rows["lora_rank_r"] = {f: sum(v[f] for v in kinds)
+                               for f in ("launches", "total_ms", "flops", "bytes")}
+    return {k: dict(launches_per_step=e["launches"] / steps, ms_per_step=e["total_ms"] / steps,
+                    tflops=(e["flops"] / e["total_ms"] * 1e-9) if e["total_ms"] > 0 else None,
+                    gbs=(e["bytes"] / e["total_ms"] * 1e-6) if e["total_ms"] > 0 else None)
+            for k, e in rows.items()}
 
 
 def workload_name(absmax_bits, dpo=False, pairs=2, batch=1, micro_batches=1):
@@ -436,13 +451,7 @@ def run_ours(args):
                      h2d_bytes_per_step=h2d / args.steps,
                      copy_wait_ms_per_step=wait_ms / args.steps,
                      tflop_per_step=flops_step / 1e12,
-                     kernels={k: dict(launches_per_step=e["launches"] / args.steps,
-                                      ms_per_step=e["total_ms"] / args.steps,
-                                      tflops=(e["flops"] / e["total_ms"] * 1e-9)
-                                      if e["total_ms"] > 0 else None,
-                                      gbs=(e["bytes"] / e["total_ms"] * 1e-6)
-                                      if e["total_ms"] > 0 else None)
-                              for k, e in prof.items()})
+                     kernels=kernel_table(prof, args.steps))
 
     cpu = None
     if (rank == 0 and world == 1 and not args.no_cpu_baseline and not dpo and not qwen

@@ -394,7 +394,7 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
   a.Q = Ab; a.q_k = 1; a.q_n = K;
   a.M = T; a.N = R; a.K = K;
   LSQ_TRY((run<true, true>(a, sc, qb, scratch_bytes, u, R, 1, 1.f, 0, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
   return LSQ_OK;
 }
 
@@ -421,7 +421,7 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
     a.M = T; a.N = r; a.K = Np;
     LSQ_TRY((run<true, false>(a, sc, qb, scratch_bytes, v + p * r, R, 1, 1.f, 0, st)));
     if (prof >= 0)
-      prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
+      prof_end(prof, st, "lora_rank_r_v", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
     start = part_end[p];
   }
   return LSQ_OK;
@@ -445,7 +445,7 @@ int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, 
   a.Q = vb; a.q_k = R8; a.q_n = 1;
   a.M = K; a.N = R; a.K = T;
   LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dA, 1, K, s, accumulate, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
   return LSQ_OK;
 }
 
@@ -472,7 +472,7 @@ int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N,
     LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dB + start * r, r, 1, s, accumulate,
                                st)));
     if (prof >= 0)
-      prof_end(prof, st, "lora_rank_r", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
+      prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
     start = part_end[p];
   }
   return LSQ_OK;
