@@ -19,6 +19,8 @@
 // near the memory roofline.  When a product is split along its reduction, the
 // slices are summed by a second kernel in a fixed order, so results are
 // deterministic (no atomics); an unsplit product writes its result directly.
+#include <stdlib.h>
+
 #include "common.cuh"
 
 namespace lsq {
@@ -266,7 +268,23 @@ __global__ void to_bf16_rows_kernel(const float* __restrict__ in, int64_t rows, 
 int64_t pad8(int64_t n) { return (n + 7) / 8 * 8; }
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
-int bn_for(int64_t N) { return N <= 64 ? 64 : N <= 128 ? 128 : 192; }
+// Column tile.  Default 64 for every product: 3 CTAs per SM, and a product
+// wider than 64 columns runs several column tiles, which read the same
+// activation rows (the second and third time mostly from L2).  LSQ_LORA_BN=128
+// or 192 selects one tile of up to that many columns instead (fewer activation
+// reads, 2 or 1 CTAs per SM).
+int bn_limit() {
+  static const int v = [] {
+    const char* e = getenv("LSQ_LORA_BN");
+    const int x = e ? atoi(e) : 64;
+    return (x == 128 || x == 192) ? x : 64;
+  }();
+  return v;
+}
+int bn_for(int64_t N) {
+  const int lim = bn_limit();
+  return (N <= 64 || lim == 64) ? 64 : (N <= 128 || lim == 128) ? 128 : 192;
+}
 int ctas_per_sm(int bn) { return bn <= 64 ? 3 : bn <= 128 ? 2 : 1; }
 
 // Splits of the reduction: only where the product's own tiles leave at least
