@@ -166,3 +166,41 @@ def test_layer_shard_plan_reassembles_the_layer(world):
         assert S % 256 == 0 and S * world >= nbytes and (S - 256) * world < nbytes
         assert sum(out[r][1][k][1] for r in range(world)) == nbytes   # every byte read once
         assert all(out[r][1][k][2] for r in range(world))
+
+
+def _absent_peer_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import time
+    from layer_streamed_qlora_nf4_b200 import dp
+    dp.init("gloo", timeout_s=5)
+    if rank == 1:
+        out[rank] = "left"          # this rank leaves between steps, before the id exchange
+        os._exit(0)
+    t0 = time.time()
+    try:
+        dp.broadcast_bytes(lambda: os.urandom(128))
+        out[rank] = ("no error", time.time() - t0)
+    except Exception as e:      # the process group's timeout, or the peer's closed connection
+        out[rank] = (type(e).__name__, time.time() - t0)
+    os._exit(0)
+
+
+def test_id_exchange_fails_instead_of_hanging_when_a_rank_is_gone():
+    """stream_stack_shard's NCCL id reaches the ranks through dp.broadcast_bytes: if a
+    rank has left, the others get an error within the process group's timeout."""
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_absent_peer_worker, args=(r, world, port, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[1] == "left"
+    err, secs = out[0]
+    assert err != "no error" and secs < 60, (err, secs)
