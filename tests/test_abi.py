@@ -146,3 +146,13 @@ def test_shard_bytes(L):
             S = L.lsq_shard_bytes(b, w)
             assert S % 256 == 0 and S * w >= b and (S - 256) * w < b
 
+
+
+def test_big_layer_config_is_above_165mib(L):
+    # the configuration of the large-layer gradient test (hidden 5120, FFN 27648)
+    from layer_streamed_qlora_nf4_b200 import synth
+    big = dict(synth.LLAMA8B, hidden=5120, ffn=27648, n_heads=40, n_kv_heads=8, head_dim=128)
+    lay = L.lsq_layer_layout_get(big)
+    n_w = 5120 * (5120 + 2 * 1024) + 5120 * 5120 + 3 * 27648 * 5120
+    assert lay.bytes == n_w // 2 + 4 * n_w // 64 + 2 * 5120 * 2     # codes + absmax + gains
+    assert lay.bytes > 165 * 2 ** 20
