@@ -316,6 +316,22 @@ typedef struct lsq_step_stats {
 } lsq_step_stats;
 int stream_stack_last_stats(const lsq_stack* stack, lsq_step_stats* out);
 
+/* lsq_stream_plan - the layer-visit schedule every streamed step follows
+ * (host only; exported so that the schedule can be inspected and tested).
+ * A step with micro_batches micro-batches visits layers 0..L-1 (forward), then
+ * L-1..0 (backward, recomputing each layer), per micro-batch.  A visit uses a
+ * buffer that already holds its layer; otherwise its layer is copied into the
+ * buffer the previous visit did not use (the first copy of a step goes to
+ * buffer 0 when neither holds the layer).  held0/held1: the layers the two
+ * buffers hold before the step (-1: none; a stack starts with -1, -1 and keeps
+ * the contents between steps).  Writes, for visit i of 2 * L * micro_batches,
+ * layer[i], buf[i] (0 or 1) and copy[i] (1: copied into buf[i] before use),
+ * and *n_visits.  LSQ_ERR_SHAPE for n_layers or micro_batches < 1 or bad
+ * buffer contents, LSQ_ERR_WORKSPACE if max_visits is too small. */
+int lsq_stream_plan(int32_t n_layers, int32_t micro_batches, int32_t held0, int32_t held1,
+                    int32_t* layer, int32_t* buf, int32_t* copy, int32_t max_visits,
+                    int32_t* n_visits);
+
 /* ------------------------------------------- data-parallel layer sharding */
 /* The pages run layer streaming on one GPU and compare it with multi-GPU
  * sharded training (translated project README, the v3 change list: the

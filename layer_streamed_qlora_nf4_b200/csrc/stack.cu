@@ -387,6 +387,28 @@ extern "C" int stream_stack_last_stats(const lsq_stack* h, lsq_step_stats* out) 
   return LSQ_OK;
 }
 
+extern "C" int lsq_stream_plan(int32_t n_layers, int32_t micro_batches, int32_t held0,
+                               int32_t held1, int32_t* layer, int32_t* buf, int32_t* copy,
+                               int32_t max_visits, int32_t* n_visits) {
+  if (!layer || !buf || !copy || !n_visits)
+    return set_error(LSQ_ERR_INVALID, "lsq_stream_plan: null output");
+  if (n_layers <= 0 || micro_batches <= 0 || held0 < -1 || held0 >= n_layers || held1 < -1 ||
+      held1 >= n_layers || (held0 >= 0 && held0 == held1))
+    return set_error(LSQ_ERR_SHAPE, "lsq_stream_plan: bad layer count or buffer contents");
+  const int64_t n = (int64_t)2 * n_layers * micro_batches;
+  if (n > max_visits)
+    return set_error(LSQ_ERR_WORKSPACE, "lsq_stream_plan: %lld visits, room for %d",
+                     (long long)n, max_visits);
+  const std::vector<Visit> v = plan_visits(n_layers, micro_batches, held0, held1);
+  for (size_t i = 0; i < v.size(); ++i) {
+    layer[i] = v[i].layer;
+    buf[i] = v[i].buf;
+    copy[i] = v[i].copy;
+  }
+  *n_visits = (int32_t)v.size();
+  return LSQ_OK;
+}
+
 extern "C" int64_t lsq_shard_bytes(int64_t layer_bytes, int32_t world) {
   if (layer_bytes <= 0 || world < 1) return 0;
   const int64_t s = (layer_bytes + world - 1) / world;

@@ -26,7 +26,7 @@ EXPORTS = (
     "lora_adamw_step", "lsq_launch_counter", "lsq_profile_enable", "lsq_profile_read",
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
     "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
-    "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard",
+    "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard", "lsq_stream_plan",
 )
 LSQ_NCCL_ID_BYTES = 128
 
@@ -119,6 +119,8 @@ _PROTOS = {
                                              _I64]),
     "lora_adamw_step": (ctypes.c_int, [_P, _P, ctypes.POINTER(lsq_adamw), _I64, _P]),
     "lsq_shard_bytes": (_I64, [_I64, _I32]),
+    "lsq_stream_plan": (ctypes.c_int, [_I32, _I32, _I32, _I32, _P, _P, _P, _I32,
+                                       ctypes.POINTER(ctypes.c_int32)]),
     "lsq_nccl_unique_id": (ctypes.c_int, [_P, _I64]),
     "stream_stack_shard": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64]),
     "lsq_launch_counter": (ctypes.c_int64, []),
@@ -304,6 +306,16 @@ class StreamStack:
             self.close()
         except Exception:
             pass
+
+
+def lsq_stream_plan(n_layers, micro_batches, held0=-1, held1=-1):
+    """-> list of (layer, buf, copy) per visit of one streamed step."""
+    n = max(0, 2 * int(n_layers) * int(micro_batches))
+    arrs = [(ctypes.c_int32 * max(n, 1))() for _ in range(3)]
+    nv = ctypes.c_int32(0)
+    _check(load().lsq_stream_plan(int(n_layers), int(micro_batches), int(held0), int(held1),
+                                  arrs[0], arrs[1], arrs[2], n, ctypes.byref(nv)))
+    return [(arrs[0][i], arrs[1][i], arrs[2][i]) for i in range(nv.value)]
 
 
 def lsq_shard_bytes(layer_bytes, world):
