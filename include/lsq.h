@@ -22,7 +22,8 @@
  *   - Memory: the caller owns every buffer (device tensors, pinned host blobs,
  *     workspaces, streams).  The library never allocates or frees caller memory
  *     and allocates no device memory per call.  Opaque handles (lsq_stack) own
- *     only their CUDA events and copy stream.
+ *     only their CUDA events, copy stream and pinned loss slot, and (once
+ *     stream_stack_shard has run) an NCCL communicator.
  *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Unless stated otherwise a call only enqueues work on it; pointers must stay
  *     valid until that work completes.
@@ -373,7 +374,8 @@ int lsq_nccl_unique_id(void* id_out, int64_t id_bytes);
  * communicator).  If a step times out (LSQ_ERR_TIMEOUT) the communicator is
  * aborted, which ends any all-gather still waiting for a peer, and the stack
  * refuses further steps (LSQ_ERR_INVALID); destroy it.  stream_stack_destroy
- * also destroys the communicator.  Errors: LSQ_ERR_INVALID (null, wrong id
+ * also destroys the communicator.  NCCL allocates the communicator's own
+ * device buffers once, in this call; steps allocate nothing.  Errors: LSQ_ERR_INVALID (null, wrong id
  * size, resident or already sharded stack, bad rank, wrong device),
  * LSQ_ERR_WORKSPACE (buffers too small), LSQ_ERR_CUDA (NCCL). */
 int stream_stack_shard(lsq_stack* stack, const void* nccl_id, int64_t id_bytes, int32_t world,
