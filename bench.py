@@ -502,7 +502,7 @@ def run_layer(args):
     lora = pack.lora_block(cfg, A, B)
     grad = torch.zeros_like(lora)
     T = BATCH * SEQ
-    x = (torch.randn(T, cfg["hidden"], generator=g, device="cuda")).bfloat16()
+    x = (torch.randn(T, cfg["hidden"], generator=g, device="cuda")).bfloat16().float()
     y = torch.empty_like(x)
     dy = torch.randn(T, cfg["hidden"], generator=g, device="cuda")
     dx = torch.empty_like(dy)
@@ -577,8 +577,8 @@ def run_gemm(args):
     wts = [(codes.clone(), absmax.clone()) for _ in range(n_copies)]
     A = torch.randn(r, K, generator=g, device="cuda") / r
     B = torch.randn(N, r, generator=g, device="cuda") * 0.01
-    x = torch.randn(T, K, generator=g, device="cuda").bfloat16()
-    y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    x = torch.randn(T, K, generator=g, device="cuda").bfloat16().half()
+    y = torch.empty(T, N, dtype=torch.float16, device="cuda")
     dy = torch.randn(T, N, generator=g, device="cuda").bfloat16()
     dx = torch.empty(T, K, dtype=torch.bfloat16, device="cuda")
     dA, dB = torch.empty(r, K, device="cuda"), torch.empty(N, r, device="cuda")

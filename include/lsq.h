@@ -27,8 +27,16 @@
  *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Unless stated otherwise a call only enqueues work on it; pointers must stay
  *     valid until that work completes.
- *   - Layouts are row-major and contiguous.  bf16 tensors are passed as uint16_t
- *     bit patterns.  Device pointers must be 16-byte aligned.
+ *   - Layouts are row-major and contiguous.  bf16 and fp16 tensors are passed as
+ *     uint16_t bit patterns.  Device pointers must be 16-byte aligned.
+ *   - Precision.  Forward activations that feed tensor cores are fp16, and the
+ *     forward GEMMs multiply the dequantised weight rounded to fp16 (an 11-bit
+ *     significand: 8x less rounding error than bf16, which keeps a deep stack's
+ *     gradients within tolerance); gradients are bf16 (their range needs bf16's
+ *     8-bit exponent), the residual stream between layers is fp32, and every
+ *     accumulation is fp32.  A forward value beyond the fp16 range (|x| > 65504:
+ *     a weight, an absmax, or an activation) latches LSQ_DEV_ERR_NONFINITE in the
+ *     device status word.
  *   - Kernel-side errors (a bounded wait that gave up) are latched in a device
  *     status word; lsq_device_status() reads it, the synchronous calls check it.
  */
@@ -58,7 +66,11 @@ const char* lsq_last_error(void);
 /* ABI version (major * 100 + minor). */
 int lsq_version(void);
 /* Reads (and, if clear != 0, resets) the device status word of the current
- * device into *flags.  Synchronises the device.  Returns LSQ_OK or LSQ_ERR_CUDA. */
+ * device into *flags.  Synchronises the device.  Returns LSQ_OK or LSQ_ERR_CUDA.
+ * Bits: LSQ_DEV_ERR_WAIT (a bounded in-kernel wait gave up), LSQ_DEV_ERR_NONFINITE
+ * (a non-finite quantiser input, or a forward value beyond the fp16 range). */
+#define LSQ_DEV_ERR_WAIT 1
+#define LSQ_DEV_ERR_NONFINITE 2
 int lsq_device_status(int* flags, int clear);
 
 /* ------------------------------------------------------------------- NF4 */
@@ -77,7 +89,9 @@ int lsq_nf4_codebook(float out_levels[16]);
  *           of w/absmax (fp32 division, exact midpoint -> lower code).
  *   absmax  device fp32 [N*K/64]: max |w| of each block (0 -> all codes 7).
  * Synchronous: waits for the stream, then returns LSQ_ERR_INVALID if W held a
- * NaN or Inf (codes/absmax are then unspecified).  Deterministic. */
+ * NaN, an Inf, or a value beyond 65504 in magnitude (the fp16 range of the
+ * fused GEMM's forward operand); codes/absmax are then unspecified.
+ * Deterministic. */
 int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block, uint8_t* codes,
                  float* absmax, void* stream);
 
@@ -118,25 +132,25 @@ size_t nf4_lora_linear_workspace_bytes(int64_t T, int64_t K, int64_t N, int32_t 
 
 /* nf4_lora_linear_fwd - y = x W~^T + scale * (x A^T) B^T (+ residual).
  * Tutorial part 1 (LoRA A/B trained on top of the frozen NF4 base).
- *   x        device bf16 [T, K];  T >= 1, K % 64 == 0.
+ *   x        device fp16 [T, K];  T >= 1, K % 64 == 0.
  *   codes, absmax  the NF4 weight W [N, K] (layout of nf4_quantize); N % 8 == 0.
  *   A        device fp32 [r, K];  B  device fp32 [N, r];  r % 16 == 0, 16 <= r <= 256.
- *   residual device bf16 [T, N] or NULL.
- *   y        device bf16 [T, N] (output).
+ *   residual device fp32 [T, N] or NULL (needs y_fp32 = 1).
+ *   y        device [T, N] (output): fp16 when y_fp32 == 0, fp32 when y_fp32 == 1.
  *   u_out    device fp32 [T, r] = x A^T, or NULL.
  *   ws       device workspace of nf4_lora_linear_workspace_bytes(T, K, N, r).
- * The dequantised weight is rounded to bf16 for the tensor cores; accumulation
- * is fp32.  Asynchronous, deterministic. */
+ * The dequantised weight, A, B and u are rounded to fp16 for the tensor cores;
+ * accumulation is fp32.  Asynchronous, deterministic. */
 int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int64_t N,
                         const uint8_t* codes, const float* absmax, int32_t block,
                         const float* A, const float* B, int32_t r, float scale,
-                        const uint16_t* residual, uint16_t* y, float* u_out, void* ws,
+                        const float* residual, void* y, int32_t y_fp32, float* u_out, void* ws,
                         size_t ws_bytes, void* stream);
 
 /* nf4_lora_linear_bwd - backward of the linear above (W frozen).
  * Tutorial part 3 and FAQ 4: dX still needs W.
- *   dy [T, N] bf16, x [T, K] bf16 (the forward input).
- *   dx  device bf16 [T, K] = dy W~ + scale (dy B) A.
+ *   dy [T, N] bf16 (the gradient), x [T, K] fp16 (the forward input).
+ *   dx  device bf16 [T, K] = dy W~ + scale (dy B) A (bf16 products, fp32 sums).
  *   dA  device fp32 [r, K] (+)= scale (dy B)^T x;  dB device fp32 [N, r] (+)= scale dy^T (x A^T).
  *   accumulate  0: overwrite dA/dB, 1: add to them.
  * Asynchronous, deterministic (fixed-order reductions, no atomics). */
@@ -216,18 +230,19 @@ size_t decoder_layer_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t 
  *   lora    device fp32, one layer's LoRA block (lsq_lora_layout), or NULL to
  *           run the layer with its adapter off (every LoRA branch removed: the
  *           reference model of the DPO step).
- *   x_in    device bf16 [batch*seq, D]; x_out device bf16 [batch*seq, D].
+ *   x_in    device fp32 [batch*seq, D]; x_out device fp32 [batch*seq, D] (the
+ *           residual stream is fp32; see the precision convention above).
  * Asynchronous, deterministic. */
 int decoder_layer_fwd(const lsq_cfg* cfg, const void* blob, const float* lora,
-                      const uint16_t* x_in, int32_t batch, int32_t seq, uint16_t* x_out,
+                      const float* x_in, int32_t batch, int32_t seq, float* x_out,
                       void* ws, size_t ws_bytes, void* stream);
 
-/* decoder_layer_bwd - recomputes the layer's forward from x_in, then
- * backpropagates dx_out (fp32 [T, D], gradient w.r.t. x_out) into dx_in (fp32
- * [T, D]) and the LoRA gradients (fp32, lsq_lora_layout; accumulate 0/1).
+/* decoder_layer_bwd - recomputes the layer's forward from x_in (fp32 [T, D]),
+ * then backpropagates dx_out (fp32 [T, D], gradient w.r.t. x_out) into dx_in
+ * (fp32 [T, D]) and the LoRA gradients (fp32, lsq_lora_layout; accumulate 0/1).
  * The frozen weights and gains get no gradient.  Asynchronous, deterministic. */
 int decoder_layer_bwd(const lsq_cfg* cfg, const void* blob, const float* lora,
-                      const uint16_t* x_in, const float* dx_out, int32_t batch, int32_t seq,
+                      const float* x_in, const float* dx_out, int32_t batch, int32_t seq,
                       float* dx_in, float* lora_grad, int32_t accumulate, void* ws,
                       size_t ws_bytes, void* stream);
 
@@ -243,7 +258,13 @@ typedef struct lsq_stack lsq_stack;
  *                resident == 1 they are device memory and are used in place
  *                (the two buffers are then ignored and may be NULL).
  *   vram_buf0/1  device buffers of lsq_layer_layout.bytes each.
- * Creates the handle's copy stream and events on the current device. */
+ * Creates the handle's copy stream and events on the current device.
+ * Buffer contract: while the handle lives, vram_buf0 and vram_buf1 belong to
+ * it.  Between steps they keep the layers the last completed step left in them,
+ * and the next step uses those layers in place instead of copying them again;
+ * so the caller must not write either buffer, nor give it to another handle,
+ * until stream_stack_destroy (after a failed step the handle trusts neither
+ * buffer and copies every layer it needs). */
 int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_blobs, int32_t n_layers,
                         void* vram_buf0, void* vram_buf1, int32_t resident, lsq_stack** out);
 int stream_stack_destroy(lsq_stack* stack);
@@ -422,19 +443,24 @@ int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out);
  * synchronisation cudaMalloc/cudaFree may cause).  This entry point is an
  * engineering addition with no counterpart on the pages the method comes from.
  *   Arguments as nf4_lora_linear_fwd, without ws/ws_bytes.
- *   Scratch: a fixed 32 MiB device array built into the library; every GPU that
- *   loads the library holds it until the process exits.  Sizes whose
+ *   Scratch: a fixed 32 MiB device array built into the library.  Sizes whose
  *   nf4_lora_linear_workspace_bytes exceeds 32 MiB are rejected with
- *   LSQ_ERR_WORKSPACE.  No allocation happens in the call.
+ *   LSQ_ERR_WORKSPACE.  Calls after the first on a device allocate nothing.
  *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current).  With CUDA's lazy module loading (the default since
+ *   CUDA 12.2) that lookup is also what loads the array onto the device, i.e.
+ *   it reserves 32 MiB of device memory there and can fail (LSQ_ERR_CUDA) if the
+ *   device is full.  So make the first call on each device early: before the
+ *   caller's own pool takes all device memory, and before any stream capture.
+ *   The array then stays on that device until the process exits.
  *   All calls share the one array: calls that can overlap on the GPU (other
  *   streams, other host threads) race on it and must be serialised by the
  *   caller.  Nothing in the array needs to start at zero. */
 int nf4_lora_linear_fwd_noalloc(const uint16_t* x, int64_t T, int64_t K, int64_t N,
                                 const uint8_t* codes, const float* absmax, int32_t block,
                                 const float* A, const float* B, int32_t r, float scale,
-                                const uint16_t* residual, uint16_t* y, float* u_out, void* stream);
+                                const float* residual, void* y, int32_t y_fp32, float* u_out,
+                                void* stream);
 
 #ifdef __cplusplus
 }

@@ -2,7 +2,9 @@
 //
 // y = x W~^T + s (x A^T) B^T and its backward dX = dY W~ + s (dY B) A,
 // dA = s (dY B)^T x, dB = s dY^T (x A^T) (Soup layer-streaming tutorial,
-// "四段資料路徑" parts 1 and 3, FAQ 4).
+// "四段資料路徑" parts 1 and 3, FAQ 4).  The forward takes fp16 activations (the
+// fused GEMM's forward operand type) and writes fp16, or fp32 with an fp32
+// residual; the backward takes bf16 gradients.
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -38,7 +40,7 @@ struct LinearWs {
 
 GemmDesc fwd_desc(const uint16_t* x, int64_t T, int64_t K, int64_t N, const uint8_t* codes,
                   const float* absmax, const float* B, int r, float scale, const float* u,
-                  const uint16_t* residual, uint16_t* y) {
+                  const float* residual, void* y, int y_f32) {
   GemmDesc d;
   d.wmode = W_NF4_N;
   d.M = N;
@@ -58,6 +60,7 @@ GemmDesc fwd_desc(const uint16_t* x, int64_t T, int64_t K, int64_t N, const uint
   d.lb = u;
   d.lb_ld = r;
   d.out = y;
+  d.out_f32 = y_f32;
   d.ldo = N;
   d.residual = residual;
   d.ldr = N;
@@ -94,7 +97,7 @@ size_t linear_ws_plan(int64_t T, int64_t K, int64_t N, int r, LinearWs* w, void*
   const size_t sb = std::max(lora_scratch_bytes(T, K, r), lora_scratch_bytes(T, N, r));
   const size_t gb = std::max(
       gemm_workspace_bytes(fwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, 0, nullptr,
-                                    nullptr, nullptr)),
+                                    nullptr, nullptr, 0)),
       gemm_workspace_bytes(bwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, 0, nullptr,
                                     nullptr)));
   Arena b;
@@ -136,7 +139,7 @@ int check_linear(const void* x, int64_t T, int64_t K, int64_t N, const void* cod
 using namespace lsq;
 
 extern "C" const char* lsq_last_error(void) { return t_msg; }
-extern "C" int lsq_version(void) { return 100; }
+extern "C" int lsq_version(void) { return 200; }
 
 extern "C" int lsq_device_status(int* flags, int clear) {
   if (!flags) return set_error(LSQ_ERR_INVALID, "lsq_device_status: null output");
@@ -156,10 +159,16 @@ extern "C" size_t nf4_lora_linear_workspace_bytes(int64_t T, int64_t K, int64_t 
 extern "C" int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int64_t N,
                                    const uint8_t* codes, const float* absmax, int32_t block,
                                    const float* A, const float* B, int32_t r, float scale,
-                                   const uint16_t* residual, uint16_t* y, float* u_out, void* ws,
-                                   size_t ws_bytes, void* stream) {
+                                   const float* residual, void* y, int32_t y_fp32, float* u_out,
+                                   void* ws, size_t ws_bytes, void* stream) {
   LSQ_TRY(check_linear(x, T, K, N, codes, absmax, block, A, B, r, "nf4_lora_linear_fwd"));
   if (!y) return set_error(LSQ_ERR_INVALID, "nf4_lora_linear_fwd: null output");
+  if (y_fp32 != 0 && y_fp32 != 1)
+    return set_error(LSQ_ERR_INVALID, "nf4_lora_linear_fwd: y_fp32 must be 0 or 1");
+  if (residual && !y_fp32)
+    return set_error(LSQ_ERR_INVALID, "nf4_lora_linear_fwd: a residual needs an fp32 output");
+  if (!aligned16(y) || (residual && !aligned16(residual)) || (u_out && !aligned16(u_out)))
+    return set_error(LSQ_ERR_ALIGN, "nf4_lora_linear_fwd: pointers must be 16-byte aligned");
   const size_t need = linear_ws_plan(T, K, N, r, nullptr, nullptr);
   if (!ws || ws_bytes < need)
     return set_error(LSQ_ERR_WORKSPACE, "nf4_lora_linear_fwd: workspace %zu < %zu", ws_bytes, need);
@@ -168,7 +177,7 @@ extern "C" int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int6
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* u = u_out ? u_out : w.u;
   LSQ_TRY(launch_lora_down(x, K, A, T, K, r, u, w.scratch, w.scratch_bytes, st));
-  GemmDesc d = fwd_desc(x, T, K, N, codes, absmax, B, r, scale, u, residual, y);
+  GemmDesc d = fwd_desc(x, T, K, N, codes, absmax, B, r, scale, u, residual, y, y_fp32);
   return gemm_run(d, w.gemm, w.gemm_bytes, st);
 }
 

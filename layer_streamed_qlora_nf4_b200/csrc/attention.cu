@@ -3,9 +3,13 @@
 // "維護者的 4GB／8B 成績"): o = softmax(q k^T / sqrt(d), causal) v, with query
 // head h reading kv head h / (H / Hkv), positions restarting at 0 per sequence.
 //
-// Tiles of 64 queries x 64 keys, 4 warps x 16 rows, bf16 tensor-core MMAs
+// Tiles of 64 queries x 64 keys, 4 warps x 16 rows, tensor-core MMAs
 // (m16n8k16) with fp32 accumulation and an online (running max / running sum)
-// softmax in the exp2 domain.  The forward saves the row log-sum-exp.  The
+// softmax in the exp2 domain.  Precision: q, k, v and o are fp16 (the forward
+// activations); the forward and the recomputed scores use fp16 products, with
+// the probabilities rounded to fp16 for P V.  The backward's products with a
+// gradient operand (dO, dS) are bf16: the fp16 q, k, v fragments are rounded to
+// bf16 as they are loaded into registers, and P and dS are rounded to bf16.  The forward saves the row log-sum-exp.  The
 // backward recomputes the probabilities from it and is split into a dK/dV
 // kernel (one CTA per key block and kv head, summing over that head's query
 // heads in a fixed order) and a dQ kernel, so no output is accumulated with
@@ -37,6 +41,20 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// fp16 fragment registers -> bf16 (each fp16 value rounded to bf16)
+template <int N>
+__device__ __forceinline__ void to_bf16(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) r[i] = f16x2_to_bf16x2(r[i]);
 }
 
 // Copy `rows` rows (of `D` bf16 each, global row stride ld) into smem rows of
@@ -147,8 +165,8 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
       for (int j = 0; j < 4; ++j) {
         uint32_t bb[4];
         frag_b_nk<D>(bb, Ks, j * 16, kk * 16);
-        mma16816(s[2 * j], a, bb[0], bb[1]);
-        mma16816(s[2 * j + 1], a, bb[2], bb[3]);
+        mma16816_f16(s[2 * j], a, bb[0], bb[1]);
+        mma16816_f16(s[2 * j + 1], a, bb[2], bb[3]);
       }
     }
     // scale into the log2 domain, mask, row max
@@ -184,8 +202,8 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
       const float p2 = exp2f(s[j][2] - mx[1]), p3 = exp2f(s[j][3] - mx[1]);
       rs[0] += p0 + p1;
       rs[1] += p2 + p3;
-      pa[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);
-      pa[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+      pa[j >> 1][(j & 1) * 2 + 0] = pack_f16x2(p0, p1);
+      pa[j >> 1][(j & 1) * 2 + 1] = pack_f16x2(p2, p3);
     }
 #pragma unroll
     for (int rI = 0; rI < 2; ++rI) {
@@ -208,8 +226,8 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
       for (int j = 0; j < D / 16; ++j) {
         uint32_t bb[4];
         frag_b_kn<D>(bb, Vs, i * 16, j * 16);
-        mma16816(o[2 * j], a, bb[0], bb[1]);
-        mma16816(o[2 * j + 1], a, bb[2], bb[3]);
+        mma16816_f16(o[2 * j], a, bb[0], bb[1]);
+        mma16816_f16(o[2 * j + 1], a, bb[2], bb[3]);
       }
     }
     __syncthreads();  // every warp is done with buffer kb & 1 before it is refilled
@@ -225,14 +243,14 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
     for (int j = 0; j < D / 8; ++j) {
       const int col = 8 * j + 2 * tig;
       *reinterpret_cast<uint32_t*>(orow + col) =
-          pack_bf16x2(o[j][2 * rI] * inv, o[j][2 * rI + 1] * inv);
+          pack_f16x2(o[j][2 * rI] * inv, o[j][2 * rI + 1] * inv);
     }
     if (tig == 0)
       lse_out[(int64_t)h * T + tok0 + qr] = (m_run[rI] + log2f(l_run[rI])) * 0.69314718055994531f;
   }
 }
 
-// delta[h, t] = sum_d dO[t, h, d] * O[t, h, d]
+// delta[h, t] = sum_d dO[t, h, d] * O[t, h, d]  (O fp16, dO bf16)
 template <int D>
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                   int64_t T, int H, float* __restrict__ delta) {
@@ -245,7 +263,7 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
   const uint16_t* c = dout + t * (int64_t)H * D + (int64_t)h * D;
   float acc = 0.f;
   for (int i = lane * 2; i < D; i += 64) {
-    const float2 x = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(a + i));
+    const float2 x = unpack_f16x2(*reinterpret_cast<const uint32_t*>(a + i));
     const float2 y = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(c + i));
     acc += x.x * y.x + x.y * y.y;
   }
@@ -328,8 +346,8 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
         for (int j = 0; j < 4; ++j) {
           uint32_t bb[4];
           frag_b_nk<D>(bb, Qs, j * 16, kk * 16);
-          mma16816(st[2 * j], a, bb[0], bb[1]);
-          mma16816(st[2 * j + 1], a, bb[2], bb[3]);
+          mma16816_f16(st[2 * j], a, bb[0], bb[1]);
+          mma16816_f16(st[2 * j + 1], a, bb[2], bb[3]);
         }
       }
       // P^T
@@ -365,6 +383,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t a[4];
         frag_a<D>(a, Vs, warp * 16, kk * 16);
+        to_bf16(a);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t bb[4];
@@ -391,6 +410,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
         for (int j = 0; j < D / 16; ++j) {
           uint32_t bb[4];
           frag_b_kn<D>(bb, Qs, i * 16, j * 16);
+          to_bf16(bb);
           mma16816(dkacc[2 * j], a, bb[0], bb[1]);
           mma16816(dkacc[2 * j + 1], a, bb[2], bb[3]);
         }
@@ -482,8 +502,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
         uint32_t bb[4], bv[4];
         frag_b_nk<D>(bb, Ks, j * 16, kk * 16);
         frag_b_nk<D>(bv, Vs, j * 16, kk * 16);
-        mma16816(s[2 * j], a, bb[0], bb[1]);
-        mma16816(s[2 * j + 1], a, bb[2], bb[3]);
+        to_bf16(bv);
+        mma16816_f16(s[2 * j], a, bb[0], bb[1]);
+        mma16816_f16(s[2 * j + 1], a, bb[2], bb[3]);
         mma16816(dp[2 * j], ad, bv[0], bv[1]);
         mma16816(dp[2 * j + 1], ad, bv[2], bv[3]);
       }
@@ -509,6 +530,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
       for (int j = 0; j < D / 16; ++j) {
         uint32_t bb[4];
         frag_b_kn<D>(bb, Ks, i * 16, j * 16);
+        to_bf16(bb);
         mma16816(dqacc[2 * j], a, bb[0], bb[1]);
         mma16816(dqacc[2 * j + 1], a, bb[2], bb[3]);
       }

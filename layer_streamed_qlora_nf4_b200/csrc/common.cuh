@@ -1,10 +1,16 @@
-// Shared device helpers for the layer-streamed QLoRA (NF4) library: bf16
-// conversions, bounded mbarrier waits, TMA and tcgen05 (5th-generation tensor
-// core) PTX wrappers for sm_100a.
+// Shared device helpers for the layer-streamed QLoRA (NF4) library: bf16 and
+// fp16 conversions, bounded mbarrier waits, TMA and tcgen05 (5th-generation
+// tensor core) PTX wrappers for sm_100a.
+//
+// Storage precisions on the path: forward activations and the forward GEMMs'
+// tensor-core operands are fp16 (10-bit mantissa); gradients are bf16 (8-bit
+// exponent, for their range); the residual stream, accumulators, norms and
+// softmax are fp32.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -30,6 +36,37 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
   return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
+
+// ------------------------------------------------------------------ fp16 bits
+__device__ __forceinline__ float f16_bits_to_float(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+__device__ __forceinline__ uint16_t float_to_f16_bits(float f) {
+  return __half_as_ushort(__float2half_rn(f));
+}
+// two floats -> packed fp16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2*>(&v));
+}
+// fp16x2 -> bf16x2 (the fp16 value rounded to bf16, nearest even): lets a bf16
+// tensor-core product take an fp16-stored operand
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
+  const float2 f = unpack_f16x2(v);
+  return pack_bf16x2(f.x, f.y);
+}
+// bf16x2 -> fp16x2 (exact for |x| in [2^-14, 65504]; smaller values become fp16
+// subnormals, larger ones infinity)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  const float2 f = unpack_bf16x2(v);
+  return pack_f16x2(f.x, f.y);
+}
+// The largest finite fp16 value: a forward activation or operand beyond it
+// would overflow its fp16 storage.
+constexpr float kF16Max = 65504.f;
 
 // ------------------------------------------------------------------ smem/ptx
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -320,6 +357,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
   return (1u << 4)                       // D format fp32
          | (1u << 7)                     // A format bf16
          | (1u << 10)                    // B format bf16
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+// Instruction descriptor: fp16 x fp16 -> fp32 (A and B formats 0 = fp16).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+  return (1u << 4)                       // D format fp32
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }

@@ -1,7 +1,9 @@
 // Memory-bound kernels of the decoder layer and the stack ends: split-K reduce,
 // RMSNorm fwd/bwd, rotate-half RoPE fwd/bwd, SwiGLU fwd/bwd, embedding gather,
 // cross-entropy, AdamW.  Vectorised 16-byte accesses, warp-shuffle reductions
-// in a fixed order (deterministic), fp32 arithmetic on bf16 storage.
+// in a fixed order (deterministic), fp32 arithmetic.  Storage: the residual
+// stream is fp32, forward activations fp16 (the forward GEMMs' operand type),
+// gradients bf16 or fp32.
 //
 // Definitions (Llama-style decoder named by the Soup layer-streaming tutorial,
 // "維護者的 4GB／8B 成績"; norms kept at higher precision, "四段資料路徑" part 1):
@@ -38,9 +40,11 @@ unsigned grid_for(int64_t n, int threads, int per_thread = 1) {
 }
 
 // ------------------------------------------------------------------ split-K reduce
+// out = sum over splits in order (+ fp32 residual); out_kind OUT_F32, OUT_BF16 or
+// OUT_F16 (an fp16 result beyond the fp16 range latches the non-finite bit)
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t T,
-                                     int64_t M, void* __restrict__ out, int out_f32, int64_t ldo,
-                                     const uint16_t* __restrict__ res, int64_t ldr) {
+                                     int64_t M, void* __restrict__ out, int out_kind, int64_t ldo,
+                                     const float* __restrict__ res, int64_t ldr, int* dev_err) {
   const int64_t n4 = T * M / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -55,15 +59,21 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
       acc.w += v.w;
     }
     if (res) {
-      const uint2 r = *reinterpret_cast<const uint2*>(res + t * ldr + m);
-      const float2 r0 = unpack_bf16x2(r.x), r1 = unpack_bf16x2(r.y);
-      acc.x += r0.x;
-      acc.y += r0.y;
-      acc.z += r1.x;
-      acc.w += r1.y;
+      const float4 r = *reinterpret_cast<const float4*>(res + t * ldr + m);
+      acc.x += r.x;
+      acc.y += r.y;
+      acc.z += r.z;
+      acc.w += r.w;
     }
-    if (out_f32) {
+    if (out_kind == OUT_F32) {
       *reinterpret_cast<float4*>(static_cast<float*>(out) + t * ldo + m) = acc;
+    } else if (out_kind == OUT_F16) {
+      if (!(fmaxf(fmaxf(fabsf(acc.x), fabsf(acc.y)), fmaxf(fabsf(acc.z), fabsf(acc.w))) <= kF16Max))
+        atomicOr(dev_err, DEV_ERR_NONFINITE);
+      uint2 o;
+      o.x = pack_f16x2(acc.x, acc.y);
+      o.y = pack_f16x2(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + t * ldo + m) = o;
     } else {
       uint2 o;
       o.x = pack_bf16x2(acc.x, acc.y);
@@ -74,7 +84,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
 }
 
 // ------------------------------------------------------------------ RMSNorm
-// One CTA per row, 8 elements (16 bytes of bf16) per thread per pass; D % 8 == 0.
+// One CTA per row, 8 elements (two 16-byte loads of fp32) per thread per pass; D % 8 == 0.
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
@@ -86,44 +96,56 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
-__global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ g,
+template <bool F16OUT>
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, const uint16_t* __restrict__ g,
                                    int64_t D, float eps, uint16_t* __restrict__ y,
-                                   float* __restrict__ rstd) {
+                                   float* __restrict__ rstd, int* dev_err) {
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + row * D);
+  const float4* xr = reinterpret_cast<const float4*>(x + row * D);
   const uint4* gr = reinterpret_cast<const uint4*>(g);
   uint4* yr = reinterpret_cast<uint4*>(y + row * D);
   const int nv = (int)(D / 8);
   float ss = 0.f;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-    const uint4 v = xr[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = unpack_bf16x2(w[q]);
-      ss = fmaf(f.x, f.x, ss);
-      ss = fmaf(f.y, f.y, ss);
-    }
+    const float4 a = xr[2 * i], b = xr[2 * i + 1];
+    ss = fmaf(a.x, a.x, ss);
+    ss = fmaf(a.y, a.y, ss);
+    ss = fmaf(a.z, a.z, ss);
+    ss = fmaf(a.w, a.w, ss);
+    ss = fmaf(b.x, b.x, ss);
+    ss = fmaf(b.y, b.y, ss);
+    ss = fmaf(b.z, b.z, ss);
+    ss = fmaf(b.w, b.w, ss);
   }
   ss = block_sum(ss, red);
   const float r = rsqrtf(ss / (float)D + eps);
   if (threadIdx.x == 0 && rstd) rstd[row] = r;
+  bool big = false;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-    const uint4 v = xr[i], gv = gr[i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    const float4 a = xr[2 * i], b = xr[2 * i + 1];
+    const uint4 gv = gr[i];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 f = unpack_bf16x2(w[q]), gg = unpack_bf16x2(gw[q]);
-      o[q] = pack_bf16x2(f.x * r * gg.x, f.y * r * gg.y);
+      const float2 gg = unpack_bf16x2(gw[q]);
+      const float y0 = f[2 * q] * r * gg.x, y1 = f[2 * q + 1] * r * gg.y;
+      if (F16OUT) {
+        big |= !(fmaxf(fabsf(y0), fabsf(y1)) <= kF16Max);
+        o[q] = pack_f16x2(y0, y1);
+      } else {
+        o[q] = pack_bf16x2(y0, y1);
+      }
     }
     yr[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  if (F16OUT && big) atomicOr(dev_err, DEV_ERR_NONFINITE);
 }
 
 // dx = dres + r (g dy) - x r^3 sum(g dy x) / D;  one CTA per row, 4 elements per thread per pass
-__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t* __restrict__ x,
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
                                    const uint16_t* __restrict__ g, const float* __restrict__ rstd,
                                    const float* __restrict__ dres, int64_t D,
                                    float* __restrict__ dx, uint16_t* __restrict__ dxb) {
@@ -131,15 +153,14 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t*
   const int64_t row = blockIdx.x;
   const int nv = (int)(D / 4);
   const float4* dyr = reinterpret_cast<const float4*>(dy + row * D);
-  const uint2* xr = reinterpret_cast<const uint2*>(x + row * D);
+  const float4* xr = reinterpret_cast<const float4*>(x + row * D);
   const uint2* gr = reinterpret_cast<const uint2*>(g);
   float dot = 0.f;
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-    const float4 d = dyr[i];
-    const uint2 xv = xr[i], gv = gr[i];
-    const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
+    const float4 d = dyr[i], xv = xr[i];
+    const uint2 gv = gr[i];
     const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
-    dot += d.x * g0.x * x0.x + d.y * g0.y * x0.y + d.z * g1.x * x1.x + d.w * g1.y * x1.y;
+    dot += d.x * g0.x * xv.x + d.y * g0.y * xv.y + d.z * g1.x * xv.z + d.w * g1.y * xv.w;
   }
   dot = block_sum(dot, red);
   const float r = rstd[row];
@@ -147,15 +168,14 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const uint16_t*
   const float4* rr = dres ? reinterpret_cast<const float4*>(dres + row * D) : nullptr;
   float4* o = reinterpret_cast<float4*>(dx + row * D);
   for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-    const float4 d = dyr[i];
-    const uint2 xv = xr[i], gv = gr[i];
-    const float2 x0 = unpack_bf16x2(xv.x), x1 = unpack_bf16x2(xv.y);
+    const float4 d = dyr[i], xv = xr[i];
+    const uint2 gv = gr[i];
     const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
     float4 v;
-    v.x = r * g0.x * d.x - x0.x * c;
-    v.y = r * g0.y * d.y - x0.y * c;
-    v.z = r * g1.x * d.z - x1.x * c;
-    v.w = r * g1.y * d.w - x1.y * c;
+    v.x = r * g0.x * d.x - xv.x * c;
+    v.y = r * g0.y * d.y - xv.y * c;
+    v.z = r * g1.x * d.z - xv.z * c;
+    v.w = r * g1.y * d.w - xv.w * c;
     if (rr) {
       const float4 a = rr[i];
       v.x += a.x;
@@ -186,7 +206,7 @@ __global__ void rope_table_kernel(int seq, int half, int d, double log_theta, fl
   }
 }
 
-// In-place rotation of the q and k heads of the fused qkv buffer (bf16); a
+// In-place rotation of the q and k heads of the fused qkv buffer (fp16); a
 // thread rotates 8 pairs (i, i + d/2).
 __global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int H, int Hkv, int d,
                             const float2* __restrict__ cs) {
@@ -208,10 +228,10 @@ __global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int 
     uint32_t oa[4], ob[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 x1 = unpack_bf16x2(aw[q]), x2 = unpack_bf16x2(bw[q]);
+      const float2 x1 = unpack_f16x2(aw[q]), x2 = unpack_f16x2(bw[q]);
       const float2 c0 = c[2 * q], c1 = c[2 * q + 1];
-      oa[q] = pack_bf16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
-      ob[q] = pack_bf16x2(x2.x * c0.x + x1.x * c0.y, x2.y * c1.x + x1.y * c1.y);
+      oa[q] = pack_f16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
+      ob[q] = pack_f16x2(x2.x * c0.x + x1.x * c0.y, x2.y * c1.x + x1.y * c1.y);
     }
     *reinterpret_cast<uint4*>(base) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
     *reinterpret_cast<uint4*>(base + half) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
@@ -276,10 +296,12 @@ __global__ void rope_grad_kernel(const float* __restrict__ dq, const float* __re
 // ------------------------------------------------------------------ SwiGLU
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
 
-// 8 elements per thread (F % 8 == 0)
+// 8 elements per thread (F % 8 == 0); fp16 in and out (a product beyond the
+// fp16 range latches the non-finite status bit)
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, int64_t F,
-                                  uint16_t* __restrict__ m) {
+                                  uint16_t* __restrict__ m, int* dev_err) {
   const int64_t nv = T * F / 8;
+  bool big = false;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t e = i * 8;
@@ -290,11 +312,14 @@ __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, in
     uint32_t o[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 g = unpack_bf16x2(gw[q]), u = unpack_bf16x2(uw[q]);
-      o[q] = pack_bf16x2(g.x * sigmoidf_(g.x) * u.x, g.y * sigmoidf_(g.y) * u.y);
+      const float2 g = unpack_f16x2(gw[q]), u = unpack_f16x2(uw[q]);
+      const float m0 = g.x * sigmoidf_(g.x) * u.x, m1 = g.y * sigmoidf_(g.y) * u.y;
+      big |= !(fmaxf(fabsf(m0), fabsf(m1)) <= kF16Max);
+      o[q] = pack_f16x2(m0, m1);
     }
     *reinterpret_cast<uint4*>(m + e) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  if (big) atomicOr(dev_err, DEV_ERR_NONFINITE);
 }
 
 __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* __restrict__ gu,
@@ -313,7 +338,7 @@ __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* 
     uint32_t og[4], ou[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 g = unpack_bf16x2(gw[q]), u = unpack_bf16x2(uw[q]);
+      const float2 g = unpack_f16x2(gw[q]), u = unpack_f16x2(uw[q]);
       const float s0 = sigmoidf_(g.x), s1 = sigmoidf_(g.y);
       const float a = dd[2 * q], b = dd[2 * q + 1];
       og[q] = pack_bf16x2(a * u.x * s0 * (1.f + g.x * (1.f - s0)),
@@ -328,14 +353,19 @@ __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* 
 // ------------------------------------------------------------------ embedding, CE, AdamW
 __global__ void embedding_kernel(const int32_t* __restrict__ tok, int64_t T,
                                  const uint16_t* __restrict__ emb, int64_t D, int64_t V,
-                                 uint16_t* __restrict__ out) {
+                                 float* __restrict__ out) {
   const int64_t nv = D / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T * nv;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = i / nv, c = i % nv;
     int64_t id = tok[t];
     if (id < 0 || id >= V) id = 0;  // ids are validated on the host side where possible
-    reinterpret_cast<uint4*>(out + t * D)[c] = reinterpret_cast<const uint4*>(emb + id * D)[c];
+    const uint4 v = reinterpret_cast<const uint4*>(emb + id * D)[c];
+    const float2 a = unpack_bf16x2(v.x), b = unpack_bf16x2(v.y), e = unpack_bf16x2(v.z),
+                 f = unpack_bf16x2(v.w);
+    float4* o = reinterpret_cast<float4*>(out + t * D + c * 8);
+    o[0] = make_float4(a.x, a.y, b.x, b.y);
+    o[1] = make_float4(e.x, e.y, f.x, f.y);
   }
 }
 
@@ -450,11 +480,13 @@ __global__ void scale_kernel(float* __restrict__ x, int64_t n, float s) {
 }  // namespace
 
 int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
-                         int out_f32, int64_t ldo, const uint16_t* residual, int64_t ldr,
+                         int out_kind, int64_t ldo, const float* residual, int64_t ldr,
                          cudaStream_t st) {
   if (M % 4 != 0) return set_error(LSQ_ERR_SHAPE, "splitk_reduce: M %% 4 != 0");
-  splitk_reduce_kernel<<<grid_for(T * M / 4, 256), 256, 0, st>>>(partial, splits, T, M, out,
-                                                                 out_f32, ldo, residual, ldr);
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  splitk_reduce_kernel<<<grid_for(T * M / 4, 256), 256, 0, st>>>(
+      partial, splits, T, M, out, out_kind, ldo, residual, ldr, dev_err);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -464,14 +496,21 @@ int threads_for_row(int64_t D, int per) {
   return t < 32 ? 32 : t;
 }
 
-int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
-                       uint16_t* y, float* rstd, cudaStream_t st) {
-  rmsnorm_fwd_kernel<<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd);
+int launch_rmsnorm_fwd(const float* x, const uint16_t* g, int64_t T, int64_t D, float eps,
+                       uint16_t* y, int y_kind, float* rstd, cudaStream_t st) {
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  if (y_kind == OUT_F16)
+    rmsnorm_fwd_kernel<true><<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd,
+                                                                           dev_err);
+  else
+    rmsnorm_fwd_kernel<false><<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd,
+                                                                            dev_err);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
-int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
+int launch_rmsnorm_bwd(const float* dy, const float* x, const uint16_t* g, const float* rstd,
                        const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
                        cudaStream_t st) {
   rmsnorm_bwd_kernel<<<(unsigned)T, threads_for_row(D, 4), 0, st>>>(dy, x, g, rstd, dres, D, dx,
@@ -505,7 +544,9 @@ int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t 
 }
 
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st) {
-  swiglu_fwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(gu, T, F, m);
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  swiglu_fwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(gu, T, F, m, dev_err);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -518,7 +559,7 @@ int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F,
 }
 
 int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D, int64_t V,
-                     uint16_t* out, cudaStream_t st) {
+                     float* out, cudaStream_t st) {
   embedding_kernel<<<grid_for(T * D / 8, 256), 256, 0, st>>>(tokens, T, emb, D, V, out);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;

@@ -7,6 +7,10 @@
 // "四段資料路徑" part 1): Wop = deq(W), act = x, la = s*B, lb = u = x A^T.
 // Its input gradient (part 3 and FAQ 4, W is re-read in backward):
 // Wop = deq(W)^T, act = dY, la = s*A^T, lb = v = dY B.
+// Operand precision: the forward multiplies fp16 operands (the dequantised
+// weight rounded once to fp16, fp16 activations, the LoRA slab in fp16); the
+// input gradient multiplies bf16 operands (gradients need bf16's exponent
+// range); both accumulate in fp32 in TMEM.
 //
 // Design for B200 (one CTA per SM, 384 threads, warp-specialised):
 //   warp 0    : TMA producer for the activation tile (128-byte swizzle) [and
@@ -16,8 +20,8 @@
 //               accumulators in TMEM (up to 2 x 256 fp32 columns)
 //   warp 2    : TMA producer for the packed NF4 codes (or the bf16 tile to be
 //               transposed) into a deep staging ring
-//   warps 4-11: operand stage - expand the staged codes to bf16 (level[code] *
-//               absmax in fp32, then round-to-nearest bf16) straight into the
+//   warps 4-11: operand stage - expand the staged codes to fp16 / bf16
+//               (level[code] * absmax in fp32, then round to nearest) straight into the
 //               UMMA canonical K-major 128-byte-swizzle layout, fence the async
 //               proxy, arrive; they also write the LoRA slab.  Two warps per
 //               SM sub-partition, because expanding the codes, not the tensor
@@ -75,7 +79,7 @@ struct KParams {
   void* out;
   int out_f32;
   long long ldo;
-  const uint16_t* residual;
+  const float* residual;
   long long ldr;
   float* partial;
   int* dev_err;
@@ -107,6 +111,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
+  constexpr bool F16 = wmode_f16(WMODE);  // fp16 operands (forward) or bf16 (input gradient)
+  auto pack2 = [](float lo, float hi) -> uint32_t {
+    return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+  };
 
   const int BT = p.nacc * p.bn;
   const uint32_t acc_stride = (p.nacc > 1) ? 256u : 0u;  // TMEM column of accumulator 1
@@ -213,7 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && (!PAIR || leader)) {
     // ---------------------------------------------------------- MMA issuer (lane 0)
-    const uint32_t idesc = umma_idesc_bf16(PAIR ? 2 * kBM : kBM, p.bn);
+    const uint32_t idesc = F16 ? umma_idesc_f16(PAIR ? 2 * kBM : kBM, p.bn)
+                               : umma_idesc_bf16(PAIR ? 2 * kBM : kBM, p.bn);
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -284,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (WMODE == W_NF4_N) tma_load_2d(dst, &tm_w, cb, kt * 32, m0);       // [128 rows][32 B]
           if (WMODE == W_NF4_T) tma_load_2d(dst, &tm_w, cb, m0 / 2, kt * kBK);  // [64 rows][64 B]
           if (WMODE == W_BF16_T) tma_load_2d(dst, &tm_w, cb, m0, kt * kBK);     // [64][128 bf16]
+          if (WMODE == W_BF16C_N) tma_load_2d(dst, &tm_w, cb, kt * kBK, m0);    // [128][64 bf16] SW128
         }
         __syncwarp();
       }
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                   const uint32_t byte = (w >> (8 * b)) & 0xFFu;
-                  o[b] = pack_bf16x2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
+                  o[b] = pack2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
                 }
                 *reinterpret_cast<uint4*>(wst + sw128_offset(r, 4 * h + q)) =
                     make_uint4(o[0], o[1], o[2], o[3]);
@@ -413,11 +423,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                   const uint32_t byte = (words[j] >> (8 * (lane & 3))) & 0xFFu;
-                  regs[j] = pack_bf16x2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
+                  regs[j] = pack2(lv_sh[byte >> 4] * am, lv_sh[byte & 15u] * am);
                 }
                 const int m = mq * 32 + (lane >> 3) * 8 + (lane & 7);
                 stmatrix_x4_trans(smem_u32(wst + sw128_offset(m, nb)), regs);
               }
+            } else if (WMODE == W_BF16C_N) {
+              // bf16 [128 x 64] tile, already in the 128-byte-swizzle layout the MMA
+              // reads: convert each 16-byte chunk to fp16 in place of its position.
+              // A weight beyond the fp16 range latches the non-finite status bit.
+              bool big = false;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int off = (tid + q * kOpThreads) * 16;
+                const uint4 v = *reinterpret_cast<const uint4*>(ring + off);
+                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = unpack_bf16x2(in[e]);
+                  big |= !(fabsf(f.x) <= kF16Max) || !(fabsf(f.y) <= kF16Max);
+                  o[e] = pack_f16x2(f.x, f.y);
+                }
+                *reinterpret_cast<uint4*>(wst + off) = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+              if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
             } else if (tid < 128) {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
               const int bi = tid & 7, bj = tid >> 3;
               uint4 rowv[8];
@@ -470,8 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         : 0.f;
             }
             *reinterpret_cast<uint4*>(wst + sw128_offset(row, q)) =
-                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]),
+                           pack2(v[6], v[7]));
           }
           uint8_t* xst = xs0 + (size_t)s * xs_bytes;
           const int HT = p.nacc * hb;  // token rows of this CTA's activation stage
@@ -483,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 8; ++e)
               v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + j0 + 8 * q + e) : 0.f;
             *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
-                make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]),
+                           pack2(v[6], v[7]));
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -511,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool partial = p.splits > 1;
       const bool f32 = partial || p.out_f32;
       const int es = f32 ? 4 : 2;
-      const bool res = !partial && p.residual != nullptr;
+      const bool res = !partial && p.residual != nullptr;  // fp32, with an fp32 output
+      bool big = false;  // an fp16 output beyond the fp16 range
       const uint32_t sub_bytes = 16u * 32u * (uint32_t)es;   // one [16 x 32] box
       uint8_t* myslots = dsm + (size_t)ow * 8192;            // 2 slots of <= 4 KB
       const int mcol = m0 + qtr * 32;
@@ -548,11 +579,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 16; ++j) {
               float v = __uint_as_float(rg[sb][j]);
               if (f32) {
-                *reinterpret_cast<float*>(base + (j * 32 + lane) * 4) = v;
+                float* d = reinterpret_cast<float*>(base + (j * 32 + lane) * 4);
+                if (res) v += *d;
+                *d = v;
+              } else if (F16) {
+                big |= !(fabsf(v) <= kF16Max);
+                *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_f16_bits(v);
               } else {
-                uint16_t* d = reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2);
-                if (res) v += bf16_bits_to_float(*d);
-                *d = float_to_bf16_bits(v);
+                *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_bf16_bits(v);
               }
             }
           }
@@ -573,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (lane == 0) bulk_wait_all();
+      if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
       __syncwarp();
     }
   }
@@ -682,9 +717,10 @@ Plan make_plan(const GemmDesc& d) {
   pl.kt_per_split = (pl.kt_total + splits - 1) / splits;
   pl.splits = (pl.kt_total + pl.kt_per_split - 1) / pl.kt_per_split;
   pl.partial_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)T * (size_t)d.M * 4 : 0;
-  pl.ring_bytes = (d.wmode == W_BF16_T) ? 64 * 128 * 2 : (d.wmode == W_BF16_N ? 0 : 4096);
+  const bool bf16_tile = d.wmode == W_BF16_T || d.wmode == W_BF16C_N;
+  pl.ring_bytes = bf16_tile ? 64 * 128 * 2 : (d.wmode == W_BF16_N ? 0 : 4096);
   const uint32_t xs = (uint32_t)(pl.pair ? BT / 2 : BT) * 128;
-  int ring = (d.wmode == W_BF16_N) ? 0 : (d.wmode == W_BF16_T ? 2 : kMaxRing);
+  int ring = (d.wmode == W_BF16_N) ? 0 : (bf16_tile ? 2 : kMaxRing);
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
     return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes +
@@ -712,8 +748,11 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
                                   (int)(kSmemBudget - 2048)));
     attr_done[dev] = true;
   }
+  constexpr bool F16 = wmode_f16(WMODE);
+  const CUtensorMapDataType dt16 =
+      F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tm_act, tm_w;
-  LSQ_TRY(make_tmap(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.act, (uint64_t)d.Kc,
+  LSQ_TRY(make_tmap(&tm_act, dt16, 2, d.act, (uint64_t)d.Kc,
                     (uint64_t)d.T, (uint64_t)d.act_ld, kBK, (uint32_t)(PAIR ? pl.bn / 2 : pl.bn),
                     CU_TENSOR_MAP_SWIZZLE_128B));
   if (WMODE == W_NF4_N)
@@ -724,7 +763,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d.w, (uint64_t)d.w_cols / 2,
                       (uint64_t)d.w_rows, (uint64_t)d.w_cols / 2, 64, 64,
                       CU_TENSOR_MAP_SWIZZLE_NONE));
-  if (WMODE == W_BF16_N)
+  if (WMODE == W_BF16_N || WMODE == W_BF16C_N)
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
                       (uint64_t)d.w_rows, (uint64_t)d.w_cols, kBK, kBM,
                       CU_TENSOR_MAP_SWIZZLE_128B));
@@ -749,11 +788,11 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
     LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d.out, (uint64_t)d.M,
                       (uint64_t)d.T, (uint64_t)d.ldo, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
-    LSQ_TRY(make_tmap(&tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.out, (uint64_t)d.M,
-                      (uint64_t)d.T, (uint64_t)d.ldo, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
+    LSQ_TRY(make_tmap(&tm_out, dt16, 2, d.out, (uint64_t)d.M, (uint64_t)d.T, (uint64_t)d.ldo, 32,
+                      16, CU_TENSOR_MAP_SWIZZLE_NONE));
   }
   if (d.residual && !partial)
-    LSQ_TRY(make_tmap(&tm_res, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.residual, (uint64_t)d.M,
+    LSQ_TRY(make_tmap(&tm_res, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d.residual, (uint64_t)d.M,
                       (uint64_t)d.T, (uint64_t)d.ldr, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   else
     tm_res = tm_out;  // unused
@@ -853,7 +892,7 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (d.slab_w % 16 != 0 || d.slab_w < 0)
     return set_error(LSQ_ERR_SHAPE, "gemm: LoRA slab width must be a multiple of 16");
   if (d.slab_w > 0 && (!d.la || !d.lb)) return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
-  if (d.residual && d.out_f32) return set_error(LSQ_ERR_INVALID, "gemm: residual needs a bf16 output");
+  if (d.residual && !d.out_f32) return set_error(LSQ_ERR_INVALID, "gemm: residual needs an fp32 output");
   if (d.ldo % 8 != 0 || (d.residual && d.ldr % 8 != 0))
     return set_error(LSQ_ERR_SHAPE, "gemm: output strides must be multiples of 16 bytes");
   if (d.M > INT32_MAX || d.T > INT32_MAX || d.Kc > INT32_MAX)
@@ -884,11 +923,16 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
       LSQ_TRY((pl.pair ? launch_mode<W_BF16_T, true>(d, pl, partial, st)
                        : launch_mode<W_BF16_T, false>(d, pl, partial, st)));
       break;
+    case W_BF16C_N:
+      LSQ_TRY((pl.pair ? launch_mode<W_BF16C_N, true>(d, pl, partial, st)
+                       : launch_mode<W_BF16C_N, false>(d, pl, partial, st)));
+      break;
     default: return set_error(LSQ_ERR_INVALID, "gemm: bad operand mode");
   }
   if (pl.splits > 1)
-    LSQ_TRY(launch_splitk_reduce(partial, pl.splits, d.T, d.M, d.out, d.out_f32, d.ldo,
-                                 d.residual, d.ldr, st));
+    LSQ_TRY(launch_splitk_reduce(partial, pl.splits, d.T, d.M, d.out,
+                                 d.out_f32 ? OUT_F32 : (wmode_f16(d.wmode) ? OUT_F16 : OUT_BF16),
+                                 d.ldo, d.residual, d.ldr, st));
   if (prof >= 0) {
     // algorithmic work: the contraction plus the LoRA slab; minimum DRAM traffic:
     // the weight once, the activation once, the output (and residual) once
@@ -898,9 +942,9 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
     const double am_bytes = d.absmax_q ? 1.0 / 64.0 + 4.0 / (64.0 * 256.0) : 4.0 / 64.0;
     const double wbytes = nf4 ? M * K * (0.5 + am_bytes) : 2.0 * M * K;
     const double bytes = wbytes + 2.0 * T * K + T * M * (d.out_f32 ? 4.0 : 2.0) +
-                         (d.residual ? 2.0 * T * M : 0.0);
-    static const char* names[4] = {"gemm_nf4_fwd", "gemm_nf4_dx", "gemm_bf16_fwd",
-                                   "gemm_bf16_dx"};
+                         (d.residual ? 4.0 * T * M : 0.0);
+    static const char* names[5] = {"gemm_nf4_fwd", "gemm_nf4_dx", "gemm_bf16_fwd",
+                                   "gemm_bf16_dx", "gemm_bf16_fwd"};
     prof_end(prof, st, d.prof_name ? d.prof_name : names[d.wmode], flops, bytes);
   }
   return LSQ_OK;

@@ -63,7 +63,14 @@ struct Arena {
 //   W_NF4_T : Wop[m, c] = deq(W)[c, m]   (W [w_rows = Kc, w_cols = M] NF4; dX)
 //   W_BF16_N: Wop[m, c] = W[m, c]        (W bf16 [M, Kc])
 //   W_BF16_T: Wop[m, c] = W[c, m]        (W bf16 [Kc, M])
-enum WMode { W_NF4_N = 0, W_NF4_T = 1, W_BF16_N = 2, W_BF16_T = 3 };
+//   W_BF16C_N: Wop[m, c] = W[m, c]       (W bf16 [M, Kc], converted to an fp16 operand)
+// Operand precision: the forward modes of the decoder layer (W_NF4_N, W_BF16C_N)
+// multiply fp16 operands (the weight rounded to fp16, fp16 activations and LoRA
+// slab) and write fp16 (or fp32) outputs; the input-gradient modes (W_NF4_T,
+// W_BF16_T) and the lm_head forward (W_BF16_N) multiply bf16 operands and write
+// bf16 (or fp32).  Accumulation is fp32 in every mode.
+enum WMode { W_NF4_N = 0, W_NF4_T = 1, W_BF16_N = 2, W_BF16_T = 3, W_BF16C_N = 4 };
+__host__ __device__ constexpr bool wmode_f16(int m) { return m == W_NF4_N || m == W_BF16C_N; }
 
 struct GemmDesc {
   int wmode = W_NF4_N;
@@ -90,11 +97,12 @@ struct GemmDesc {
   int part_r = 0;
   int n_parts = 0;
   int64_t part_end[4] = {0, 0, 0, 0};
-  // epilogue
+  // epilogue: out is fp32 when out_f32, else 16-bit in the mode's operand type;
+  // residual (fp32 [T, ldr], added before the store) needs an fp32 output
   void* out = nullptr;
   int out_f32 = 0;
   int64_t ldo = 0;
-  const uint16_t* residual = nullptr;
+  const float* residual = nullptr;
   int64_t ldr = 0;
   int force_splits = 0;             // 0 = heuristic
   const char* prof_name = nullptr;  // profiler class (default: by operand mode)
@@ -104,27 +112,34 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st);
 int gemm_num_sms();
 
 // ---------------------------------------------------------------- small kernels
+// Output kinds of a reduce or normalisation kernel.
+enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
 int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
-                         int out_f32, int64_t ldo, const uint16_t* residual, int64_t ldr,
+                         int out_kind, int64_t ldo, const float* residual, int64_t ldr,
                          cudaStream_t st);
-int launch_rmsnorm_fwd(const uint16_t* x, const uint16_t* g, int64_t T, int64_t D, float eps,
-                       uint16_t* y, float* rstd, cudaStream_t st);
+// y = x (mean(x^2) + eps)^-1/2 g; x fp32 (the residual stream), y fp16 (OUT_F16,
+// a forward GEMM operand) or bf16 (OUT_BF16, the lm_head operand)
+int launch_rmsnorm_fwd(const float* x, const uint16_t* g, int64_t T, int64_t D, float eps,
+                       uint16_t* y, int y_kind, float* rstd, cudaStream_t st);
 // dx = dres + rmsnorm_bwd(dy);  writes fp32 dx and (optionally) its bf16 copy
-int launch_rmsnorm_bwd(const float* dy, const uint16_t* x, const uint16_t* g, const float* rstd,
+int launch_rmsnorm_bwd(const float* dy, const float* x, const uint16_t* g, const float* rstd,
                        const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
                        cudaStream_t st);
 // cos/sin table [seq][d/2] for rotate-half RoPE
 int launch_rope_table(int seq, int d, float theta, float2* cs, cudaStream_t st);
+// in place on the fp16 q and k heads of the fused qkv buffer
 int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, const float2* cs,
                 cudaStream_t st);
 // dk, dv are per query head [T, H d] (summed over each kv group here)
 int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
                      int Hkv, int d, const float2* cs, uint16_t* dqkv, cudaStream_t st);
+// m = silu(gate) * up: gu fp16 [T, 2F] -> m fp16 [T, F]; backward: dgu bf16
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st);
 int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
                       cudaStream_t st);
+// out fp32 [T, D] = emb (bf16) rows of the tokens
 int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D,
-                     int64_t V, uint16_t* out, cudaStream_t st);
+                     int64_t V, float* out, cudaStream_t st);
 // dlogits may be null (row losses only); seq_scale (per sequence) replaces inv_count.
 int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq,
                          int64_t V, float inv_count, uint16_t* dlogits, float* row_loss,
@@ -140,7 +155,8 @@ int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 
 // LoRA rank-r products (tensor cores, bf16 operands, fp32 accumulation, fixed-order
 // reductions)
-// u[t, j] = sum_k x[t, k] * A[j, k]                     x bf16 [T, K], A fp32 [R, K] -> u [T, R]
+// u[t, j] = sum_k x[t, k] * A[j, k]                     x fp16 [T, K], A fp32 [R, K] -> u [T, R]
+// (fp16 products: A rounded once to fp16)
 // scratch: lora_scratch_bytes(T, K, R) bytes for the bf16 copy of the LoRA operand and the
 // fixed-order partials of a product split along its reduction
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
@@ -151,7 +167,8 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r,
                       int n_parts, const int64_t* part_end, float* v, float* scratch,
                       size_t scratch_bytes, cudaStream_t st);
-// dA[j, k] (+)= s * sum_t v[t, j] * x[t, k]              v fp32 [T, R], x bf16 [T, K]
+// dA[j, k] (+)= s * sum_t v[t, j] * x[t, k]              v fp32 [T, R], x fp16 [T, K]
+// (bf16 products: v rounded once to bf16, x from fp16 to bf16 as it is loaded)
 int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
                        int accumulate, float* dA, float* scratch, size_t scratch_bytes,
                        cudaStream_t st);
@@ -160,7 +177,8 @@ int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N,
                        int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
                        float* scratch, size_t scratch_bytes, cudaStream_t st);
 
-// attention (causal GQA), q/k/v read from the fused qkv buffer [T, (H + 2 Hkv) d]
+// attention (causal GQA), q/k/v read from the fused fp16 qkv buffer [T, (H + 2 Hkv) d];
+// o fp16 [T, H d]; dout bf16
 int launch_attention_fwd(const uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d,
                          uint16_t* o, float* lse, cudaStream_t st);
 // dk, dv are written per query head: [T, H d] fp32 (the kv-group sum happens in rope_grad)
@@ -179,10 +197,10 @@ struct LayerShapes {
 int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);
 // dx_out_bf16 may be null (then converted internally).
-int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
-                   int batch, int seq, uint16_t* x_out, void* ws, size_t ws_bytes,
+int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
+                   int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
                    cudaStream_t st);
-int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate,
                    void* ws, size_t ws_bytes, cudaStream_t st);

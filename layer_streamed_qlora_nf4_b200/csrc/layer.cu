@@ -7,6 +7,12 @@
 // Fusions: q|k|v and gate|up are stored back to back in the layer blob, so each
 // group is one NF4 GEMM; the LoRA up-projections ride in those GEMMs as an
 // extra K slab; the o and down GEMMs add the residual in their epilogue.
+//
+// Precision: the residual stream (the layer's input and output, and h) is fp32;
+// the forward activations that feed tensor cores (n1, q|k|v, attention output,
+// n2, gate|up, the SwiGLU product) are fp16, as is the dequantised weight in the
+// forward GEMMs; gradients that feed tensor cores are bf16; every accumulation,
+// norm and softmax is fp32.
 #include "common.cuh"
 
 namespace lsq {
@@ -162,7 +168,9 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
 
 // Workspace carve-up (identical for the forward and the backward).
 struct Buffers {
-  uint16_t *n1, *qkv, *ao, *h, *n2, *gu, *m, *dgu, *dqkv, *da, *dout_b, *dh_b;
+  float* h;                                          // fp32 residual stream after attention
+  uint16_t *n1, *qkv, *ao, *n2, *gu, *m;             // fp16 forward activations
+  uint16_t *dgu, *dqkv, *da, *dout_b, *dh_b;         // bf16 gradients
   float *rstd1, *rstd2, *u_qkv, *u_o, *u_gu, *u_d, *lse, *v_qkv, *v_o, *v_gu, *v_d;
   float *dm, *dn2, *dh, *dn1, *dq, *dk, *dv, *delta;
   float2* rope_cs;
@@ -173,14 +181,15 @@ struct Buffers {
 };
 
 // Forward of a stacked frozen weight W [N, K] (NF4, or bf16 when absmax is
-// empty): out [T, N] = act W^T + s u B^T (+ residual).
+// empty, converted to fp16 in the operand stage): out [T, N] = act W^T + s u B^T,
+// fp16; or, with a residual, out = that + residual in fp32.
 GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
                  const uint16_t* act, int64_t T, const float* B, int r, float s, const float* u,
-                 int64_t u_ld, int n_parts, const int64_t* pe, const uint16_t* res, void* out,
+                 int64_t u_ld, int n_parts, const int64_t* pe, const float* res, void* out,
                  int64_t ldo) {
   GemmDesc d;
   const bool bf16 = absmax.bf16;
-  d.wmode = bf16 ? W_BF16_N : W_NF4_N;
+  d.wmode = bf16 ? W_BF16C_N : W_NF4_N;
   d.M = N;
   d.T = T;
   d.Kc = K;
@@ -204,6 +213,7 @@ GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64
   for (int i = 0; i < n_parts && i < 4; ++i) d.part_end[i] = pe[i];
   d.out = out;
   d.ldo = ldo;
+  d.out_f32 = res != nullptr;
   d.residual = res;
   d.ldr = ldo;
   return d;
@@ -249,7 +259,7 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   x.n1 = a.take<uint16_t>(T * s.D);
   x.qkv = a.take<uint16_t>(T * s.qkv_n);
   x.ao = a.take<uint16_t>(T * s.qd);
-  x.h = a.take<uint16_t>(T * s.D);
+  x.h = a.take<float>(T * s.D);
   x.n2 = a.take<uint16_t>(T * s.D);
   x.gu = a.take<uint16_t>(T * s.gu_n);
   x.m = a.take<uint16_t>(T * s.F);
@@ -322,13 +332,13 @@ int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, co
 
 // Forward through the SwiGLU product (everything the backward needs) and,
 // when x_out is given, the down projection with its residual.
-int forward_core(const LayerShapes& s, const Views& v, const uint16_t* x, int batch, int seq,
-                 float theta, float eps, const Buffers& b, uint16_t* x_out, cudaStream_t st) {
+int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch, int seq,
+                 float theta, float eps, const Buffers& b, float* x_out, cudaStream_t st) {
   const int64_t T = (int64_t)batch * seq;
   const int r = v.lora_on ? s.r : 0;  // r = 0: no LoRA slab in the GEMMs
   const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
   const int64_t pe2[2] = {s.F, s.gu_n};
-  LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, b.rstd1, st));
+  LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, OUT_F16, b.rstd1, st));
   if (v.lora_on) LSQ_TRY(launch_lora_down(b.n1, s.D, v.A_qkv, T, s.D, 3 * r, b.u_qkv, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
                            3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
@@ -340,7 +350,7 @@ int forward_core(const LayerShapes& s, const Views& v, const uint16_t* x, int ba
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
                            pe3, x, b.h, s.D),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, b.rstd2, st));
+  LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, OUT_F16, b.rstd2, st));
   if (v.lora_on) LSQ_TRY(launch_lora_down(b.n2, s.D, v.A_gu, T, s.D, 2 * r, b.u_gu, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
                            2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
@@ -362,8 +372,8 @@ size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
   return plan_buffers(s, T, nullptr, nullptr);
 }
 
-int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
-                   int batch, int seq, uint16_t* x_out, void* ws, size_t ws_bytes,
+int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
+                   int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
                    cudaStream_t st) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd",
@@ -378,7 +388,7 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   return forward_core(s, v, x_in, batch, seq, cfg->rope_theta, cfg->rms_eps, b, x_out, st);
 }
 
-int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const uint16_t* x_in,
+int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate, void* ws,
                    size_t ws_bytes, cudaStream_t st) {
@@ -484,14 +494,14 @@ extern "C" size_t decoder_layer_workspace_bytes(const lsq_cfg* cfg, int32_t batc
 }
 
 extern "C" int decoder_layer_fwd(const lsq_cfg* cfg, const void* blob, const float* lora,
-                                 const uint16_t* x_in, int32_t batch, int32_t seq, uint16_t* x_out,
+                                 const float* x_in, int32_t batch, int32_t seq, float* x_out,
                                  void* ws, size_t ws_bytes, void* stream) {
   return layer_fwd_impl(cfg, blob, lora, x_in, batch, seq, x_out, ws, ws_bytes,
                         static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int decoder_layer_bwd(const lsq_cfg* cfg, const void* blob, const float* lora,
-                                 const uint16_t* x_in, const float* dx_out, int32_t batch,
+                                 const float* x_in, const float* dx_out, int32_t batch,
                                  int32_t seq, float* dx_in, float* lora_grad, int32_t accumulate,
                                  void* ws, size_t ws_bytes, void* stream) {
   return layer_bwd_impl(cfg, blob, lora, x_in, dx_out, nullptr, batch, seq, dx_in, nullptr,

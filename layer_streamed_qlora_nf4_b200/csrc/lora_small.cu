@@ -8,11 +8,14 @@
 // activation and Q an fp32 LoRA tensor.
 //
 // One kernel serves all four.  A CTA owns 128 rows x BN columns of C over one
-// slice of the reduction.  Q is first rounded once to bf16 (nearest even) into
-// scratch, rows padded to a multiple of 8 elements with zeros: bf16 operands
-// with fp32 accumulation, the compute precision of QLoRA's LoRA branch (the
-// tutorial's part 1: the LoRA A/B matrices are computed at a higher precision
-// than the NF4 storage).  Both operands then stream through a ring of 4 to 6
+// slice of the reduction.  Q is first rounded once to a 16-bit type (nearest
+// even) into scratch, rows padded to a multiple of 8 elements with zeros;
+// accumulation is fp32 (the tutorial's part 1: the LoRA A/B matrices are
+// computed at a higher precision than the NF4 storage).  Operand types follow
+// the activations: u = x A^T multiplies fp16 (x is an fp16 forward activation,
+// A is rounded to fp16); v, dA and dB multiply bf16 (each has a gradient
+// operand, which needs bf16's range; dA's fp16 activation is rounded to bf16
+// as it moves from shared memory into registers).  Both operands then stream through a ring of 4 to 6
 // cp.async stages (16-byte chunks along whichever index is contiguous in
 // memory; ldmatrix, transposing where needed, gives the MMA fragments), so
 // that each SM keeps enough bytes in flight to run these HBM-bound products
@@ -66,6 +69,18 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Operand precision of a product: PM_BF16 both operands bf16; PM_F16 both fp16;
+// PM_P16 P stored fp16 and rounded to bf16 in registers, Q bf16.
+enum { PM_BF16 = 0, PM_F16 = 1, PM_P16 = 2 };
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(src_bytes)
@@ -89,7 +104,7 @@ struct Tile {
 
 // P_RED: the reduction index is the contiguous one in P (else the row index m is).
 // Q_RED: the reduction index is the contiguous one in Q (else the column n is).
-template <bool P_RED, bool Q_RED, int BN>
+template <bool P_RED, bool Q_RED, int BN, int PM>
 __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks))
     skinny_kernel(const SkinnyArgs a) {
   using TL = Tile<P_RED, Q_RED, BN>;
@@ -189,6 +204,10 @@ __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks)
           const int i = lane >> 3, j = lane & 7;
           ldsm4_t(af[mi], smem_u32(ps + (k16 + j + 8 * (i >> 1)) * (kBM + 8) + r0 + 8 * (i & 1)));
         }
+        if (PM == PM_P16) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) af[mi][e] = f16x2_to_bf16x2(af[mi][e]);
+        }
       }
 #pragma unroll
       for (int nj = 0; nj < NF; nj += 2) {
@@ -204,8 +223,13 @@ __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks)
         }
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
-          mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
-          mma_bf16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
+          if (PM == PM_F16) {
+            mma_f16(acc[mi][nj], af[mi], bh[0], bh[1]);
+            mma_f16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
+          } else {
+            mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
+            mma_bf16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
+          }
         }
       }
     }
@@ -254,14 +278,17 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
   }
 }
 
-// out[i * ld_out + j] = bf16(in[i * ld_in + j]) for j < cols, 0 for cols <= j < ld_out
-__global__ void to_bf16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
-                                    int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
+// out[i * ld_out + j] = bf16 or fp16 (F16) of in[i * ld_in + j] for j < cols, 0 for
+// cols <= j < ld_out
+template <bool F16>
+__global__ void to_16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
+                                  int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
   const int64_t n_el = rows * ld_out;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / ld_out, j = i % ld_out;
-    out[i] = j < cols ? float_to_bf16_bits(in[r * ld_in + j]) : (uint16_t)0;
+    const float v = j < cols ? in[r * ld_in + j] : 0.f;
+    out[i] = F16 ? float_to_f16_bits(v) : float_to_bf16_bits(v);
   }
 }
 
@@ -302,28 +329,31 @@ int splits_for(int64_t M, int64_t N, int64_t K) {
   return (int)((K + kps - 1) / kps);
 }
 
-template <bool P_RED, bool Q_RED, int BN>
+template <bool P_RED, bool Q_RED, int BN, int PM>
 int launch_bn(const SkinnyArgs& a, dim3 grid, cudaStream_t st) {
   constexpr size_t smem = Tile<P_RED, Q_RED, BN>::kSmem;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    LSQ_CUDA(cudaFuncSetAttribute(skinny_kernel<P_RED, Q_RED, BN>,
+    LSQ_CUDA(cudaFuncSetAttribute(skinny_kernel<P_RED, Q_RED, BN, PM>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     attr_done[dev] = true;
   }
-  skinny_kernel<P_RED, Q_RED, BN><<<grid, kThreads, smem, st>>>(a);
+  skinny_kernel<P_RED, Q_RED, BN, PM><<<grid, kThreads, smem, st>>>(a);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 
 int convert_rows(const float* in, int64_t rows, int64_t cols, int64_t ld_in, uint16_t* out,
-                 int64_t ld_out, cudaStream_t st) {
+                 int64_t ld_out, cudaStream_t st, bool f16 = false) {
   int64_t g = (rows * ld_out + 255) / 256;
   if (g > kSMs * 8) g = kSMs * 8;
   if (g < 1) return LSQ_OK;
-  to_bf16_rows_kernel<<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
+  if (f16)
+    to_16_rows_kernel<true><<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
+  else
+    to_16_rows_kernel<false><<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -331,7 +361,7 @@ int convert_rows(const float* in, int64_t rows, int64_t cols, int64_t ld_in, uin
 // C = P Q over K, then dst[m * c_m + n * c_n] = alpha * C (+ dst if accumulate).
 // scratch holds the bf16 Q (already written at its start) and, after q_bytes,
 // room for the partials when the product is split.
-template <bool P_RED, bool Q_RED>
+template <bool P_RED, bool Q_RED, int PM>
 int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float* dst,
         int64_t c_m, int64_t c_n, float alpha, int accumulate, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return LSQ_OK;
@@ -350,9 +380,9 @@ int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float
   const int bn = bn_for(a.N);
   dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)z);
   switch (bn) {
-    case 64: LSQ_TRY((launch_bn<P_RED, Q_RED, 64>(a, grid, st))); break;
-    case 128: LSQ_TRY((launch_bn<P_RED, Q_RED, 128>(a, grid, st))); break;
-    default: LSQ_TRY((launch_bn<P_RED, Q_RED, 192>(a, grid, st))); break;
+    case 64: LSQ_TRY((launch_bn<P_RED, Q_RED, 64, PM>(a, grid, st))); break;
+    case 128: LSQ_TRY((launch_bn<P_RED, Q_RED, 128, PM>(a, grid, st))); break;
+    default: LSQ_TRY((launch_bn<P_RED, Q_RED, 192, PM>(a, grid, st))); break;
   }
   if (z == 1) return LSQ_OK;
   int64_t g = (a.M * a.N + 255) / 256;
@@ -406,12 +436,12 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
   if (!scratch || scratch_bytes < qb)
     return set_error(LSQ_ERR_WORKSPACE, "lora_down: scratch %zu < %zu", scratch_bytes, qb);
   const int prof = prof_begin(st);
-  LSQ_TRY(convert_rows(A, R, K, K, Ab, K, st));
+  LSQ_TRY(convert_rows(A, R, K, K, Ab, K, st, /*f16=*/true));
   SkinnyArgs a{};
   a.P = x; a.p_m = ldx; a.p_k = 1;
   a.Q = Ab; a.q_k = 1; a.q_n = K;
   a.M = T; a.N = R; a.K = K;
-  LSQ_TRY((run<true, true>(a, sc, qb, scratch_bytes, u, R, 1, 1.f, 0, st)));
+  LSQ_TRY((run<true, true, PM_F16>(a, sc, qb, scratch_bytes, u, R, 1, 1.f, 0, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
   return LSQ_OK;
 }
@@ -437,7 +467,7 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
     a.P = dy + start; a.p_m = N; a.p_k = 1;
     a.Q = Bb; a.q_k = r8; a.q_n = 1;
     a.M = T; a.N = r; a.K = Np;
-    LSQ_TRY((run<true, false>(a, sc, qb, scratch_bytes, v + p * r, R, 1, 1.f, 0, st)));
+    LSQ_TRY((run<true, false, PM_BF16>(a, sc, qb, scratch_bytes, v + p * r, R, 1, 1.f, 0, st)));
     if (prof >= 0)
       prof_end(prof, st, "lora_rank_r_v", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
     start = part_end[p];
@@ -462,7 +492,7 @@ int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, 
   a.P = x; a.p_m = 1; a.p_k = K;
   a.Q = vb; a.q_k = R8; a.q_n = 1;
   a.M = K; a.N = R; a.K = T;
-  LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dA, 1, K, s, accumulate, st)));
+  LSQ_TRY((run<false, false, PM_P16>(a, sc, qb, scratch_bytes, dA, 1, K, s, accumulate, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
   return LSQ_OK;
 }
@@ -487,8 +517,8 @@ int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N,
     a.P = dy + start; a.p_m = 1; a.p_k = N;
     a.Q = ub; a.q_k = r8; a.q_n = 1;
     a.M = Np; a.N = r; a.K = T;
-    LSQ_TRY((run<false, false>(a, sc, qb, scratch_bytes, dB + start * r, r, 1, s, accumulate,
-                               st)));
+    LSQ_TRY((run<false, false, PM_BF16>(a, sc, qb, scratch_bytes, dB + start * r, r, 1, s,
+                                        accumulate, st)));
     if (prof >= 0)
       prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
     start = part_end[p];

@@ -72,7 +72,8 @@ __global__ void nf4_quantize_kernel(const float* __restrict__ W, int64_t n_block
   const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t b = warp_global; b < n_blocks; b += n_warps) {
     const float2 w = reinterpret_cast<const float2*>(W + b * 64)[lane];
-    const bool finite = isfinite(w.x) && isfinite(w.y);
+    // non-finite, or beyond the fp16 range the fused GEMM's forward operand has
+    const bool finite = fabsf(w.x) <= kF16Max && fabsf(w.y) <= kF16Max;
     if (!__all_sync(0xFFFFFFFFu, finite) && lane == 0) atomicOr(dev_err, DEV_ERR_NONFINITE);
     float am = fmaxf(fabsf(w.x), fabsf(w.y));
 #pragma unroll
@@ -210,7 +211,8 @@ extern "C" int nf4_quantize(const float* W, int64_t N, int64_t K, int32_t block,
   if (h_after & DEV_ERR_NONFINITE) {
     int v = h_after & ~DEV_ERR_NONFINITE;
     LSQ_CUDA(cudaMemcpy(err, &v, sizeof(int), cudaMemcpyHostToDevice));
-    return set_error(LSQ_ERR_INVALID, "nf4_quantize: W holds a NaN or Inf");
+    return set_error(LSQ_ERR_INVALID,
+                     "nf4_quantize: W holds a NaN, an Inf or a value beyond 65504 in magnitude");
   }
   return LSQ_OK;
 }

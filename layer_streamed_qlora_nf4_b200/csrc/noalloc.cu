@@ -7,12 +7,16 @@
 // nf4_lora_linear_fwd_noalloc runs exactly the kernels of nf4_lora_linear_fwd
 // but takes its scratch (the x A^T product, the fixed-order split partials of
 // the rank-r product and of the split-K GEMM) from a file-scope device array of
-// kNoAllocScratchBytes that every GPU which loads the library keeps until the
-// process exits.  It calls no allocating routine.
+// kNoAllocScratchBytes.  It calls no allocating routine.
 //
 // Host code must not use the array's name as a device address (on the host it
 // only names a stand-in); the device address is looked up once per device with
 // cudaGetSymbolAddress, with that device current, on the first call made on it.
+// Under CUDA's lazy module loading (the default since CUDA 12.2) this file's
+// module, and with it the 32 MiB array, is loaded onto a device by that first
+// lookup: the first call on a device reserves the array's device memory (and
+// can fail if the device is full); every later call allocates nothing.  The
+// array then stays on the device until the process exits.
 #include <mutex>
 
 #include "common.cuh"
@@ -54,8 +58,8 @@ using namespace lsq;
 extern "C" int nf4_lora_linear_fwd_noalloc(const uint16_t* x, int64_t T, int64_t K, int64_t N,
                                            const uint8_t* codes, const float* absmax,
                                            int32_t block, const float* A, const float* B,
-                                           int32_t r, float scale, const uint16_t* residual,
-                                           uint16_t* y, float* u_out, void* stream) {
+                                           int32_t r, float scale, const float* residual,
+                                           void* y, int32_t y_fp32, float* u_out, void* stream) {
   const size_t need = nf4_lora_linear_workspace_bytes(T, K, N, r);
   if (need == 0)
     return set_error(LSQ_ERR_SHAPE, "nf4_lora_linear_fwd_noalloc: empty or invalid shape");
@@ -68,6 +72,6 @@ extern "C" int nf4_lora_linear_fwd_noalloc(const uint16_t* x, int64_t T, int64_t
   LSQ_TRY(noalloc_scratch(&scratch));
   // Nothing in the scratch needs to start at zero: every byte the kernels read
   // is written earlier in the same call.
-  return nf4_lora_linear_fwd(x, T, K, N, codes, absmax, block, A, B, r, scale, residual, y, u_out,
-                             scratch, kNoAllocScratchBytes, stream);
+  return nf4_lora_linear_fwd(x, T, K, N, codes, absmax, block, A, B, r, scale, residual, y,
+                             y_fp32, u_out, scratch, kNoAllocScratchBytes, stream);
 }

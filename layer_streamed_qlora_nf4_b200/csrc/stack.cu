@@ -68,7 +68,7 @@ namespace lsq {
 namespace {
 
 struct StackWs {
-  uint16_t* xs;      // [L+1][T][D] bf16: layer inputs (saved for backward) and final hidden
+  float* xs;         // [L+1][T][D] fp32: layer inputs (saved for backward) and final hidden
   uint16_t* hf;      // [T][D] final-norm output
   float* rstd_f;     // [T]
   float* logits;     // [T][V]
@@ -83,7 +83,7 @@ struct StackWs {
   void* layer_ws;
   size_t layer_ws_bytes;
   // DPO step only
-  uint16_t* xr[2];   // [T][D] bf16: the reference (adapter-off) hidden state, ping-pong
+  float* xr[2];      // [T][D] fp32: the reference (adapter-off) hidden state, ping-pong
   float* row_ref;    // [T] reference per-row -log p
   float* seq_scale;  // [2 * pairs] dlogits coefficient per sequence
   float* logps;      // [4 * pairs]
@@ -136,7 +136,7 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   a.cap = SIZE_MAX;
   StackWs x{};
   const int64_t V = cfg->vocab, D = s.D;
-  x.xs = a.take<uint16_t>((size_t)(cfg->n_layers + 1) * T * D);
+  x.xs = a.take<float>((size_t)(cfg->n_layers + 1) * T * D);
   x.hf = a.take<uint16_t>(T * D);
   x.rstd_f = a.take<float>(T);
   x.logits = a.take<float>((size_t)T * V);
@@ -155,8 +155,8 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.layer_ws_bytes = layer_ws_bytes(cfg, T);
   x.layer_ws = a.take<uint8_t>(x.layer_ws_bytes);
   if (dpo) {
-    x.xr[0] = a.take<uint16_t>(T * D);
-    x.xr[1] = a.take<uint16_t>(T * D);
+    x.xr[0] = a.take<float>(T * D);
+    x.xr[1] = a.take<float>(T * D);
     x.row_ref = a.take<float>(T);
     x.seq_scale = a.take<float>(2 * kMaxPairs);
     x.logps = a.take<float>(4 * kMaxPairs);
@@ -569,13 +569,14 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
                                w.xr[i & 1], w.layer_ws, w.layer_ws_bytes, cs));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
     }
-    const uint16_t* xL = w.xs + (size_t)L * T * D;
+    const float* xL = w.xs + (size_t)L * T * D;
     if (dpo) {
-      LSQ_TRY(launch_rmsnorm_fwd(w.xr[(L - 1) & 1], final_norm, T, D, cfg->rms_eps, w.hf, w.rstd_f, cs));
+      LSQ_TRY(launch_rmsnorm_fwd(w.xr[(L - 1) & 1], final_norm, T, D, cfg->rms_eps, w.hf, OUT_BF16,
+                                 w.rstd_f, cs));
       LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
       LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_ref, cs));
     }
-    LSQ_TRY(launch_rmsnorm_fwd(xL, final_norm, T, D, cfg->rms_eps, w.hf, w.rstd_f, cs));
+    LSQ_TRY(launch_rmsnorm_fwd(xL, final_norm, T, D, cfg->rms_eps, w.hf, OUT_BF16, w.rstd_f, cs));
     LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
     if (dpo) {
       LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_loss, cs));

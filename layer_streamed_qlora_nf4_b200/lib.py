@@ -91,7 +91,7 @@ _PROTOS = {
     "nf4_dequantize_dq": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I32, _P, _P]),
     "nf4_lora_linear_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I32]),
     "nf4_lora_linear_fwd": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32, _F,
-                                           _P, _P, _P, _P, _SZ, _P]),
+                                           _P, _P, _I32, _P, _P, _SZ, _P]),
     "nf4_lora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
                                            _F, _P, _P, _P, _I32, _P, _SZ, _P]),
     "lsq_layer_layout_get": (ctypes.c_int, [ctypes.POINTER(lsq_cfg),
@@ -125,7 +125,7 @@ _PROTOS = {
     "stream_stack_shard": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64]),
     "lsq_launch_counter": (ctypes.c_int64, []),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
-                                                   _F, _P, _P, _P, _P]),
+                                                   _F, _P, _P, _I32, _P, _P]),
     "lsq_profile_enable": (ctypes.c_int, [ctypes.c_int]),
     "lsq_profile_read": (ctypes.c_int, [ctypes.POINTER(lsq_prof_entry), _I32,
                                         ctypes.POINTER(ctypes.c_int32)]),
@@ -224,19 +224,29 @@ def nf4_lora_linear_workspace_bytes(T, K, N, r):
     return load().nf4_lora_linear_workspace_bytes(T, K, N, r)
 
 
+def _y_fp32(y):
+    """1 for an fp32 output tensor, 0 for an fp16 one (the y_fp32 argument)."""
+    import torch
+    if y.dtype not in (torch.float32, torch.float16):
+        raise TypeError("y must be float16 or float32")
+    return 1 if y.dtype == torch.float32 else 0
+
+
 def nf4_lora_linear_fwd(x, codes, absmax, A, B, scale, y, residual=None, u_out=None, ws=None,
                         block=64, stream=None):
+    """x: fp16 [T, K]; y: fp16 [T, N], or fp32 [T, N] (required with an fp32 residual)."""
     T, K = x.shape
     N = y.shape[1]
     r = A.shape[0]
     _check(load().nf4_lora_linear_fwd(_ptr(x), T, K, N, _ptr(codes), _ptr(absmax), block,
                                       _ptr(A), _ptr(B), r, scale, _ptr(residual), _ptr(y),
-                                      _ptr(u_out), _ptr(ws), 0 if ws is None else ws.numel(),
-                                      _stream(stream)))
+                                      _y_fp32(y), _ptr(u_out), _ptr(ws),
+                                      0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def nf4_lora_linear_bwd(dy, x, codes, absmax, A, B, scale, dx, dA, dB, accumulate=False,
                         ws=None, block=64, stream=None):
+    """dy: bf16 [T, N]; x: fp16 [T, K] (the forward input); dx: bf16 [T, K]."""
     T, K = x.shape
     N = dy.shape[1]
     r = A.shape[0]
@@ -266,6 +276,7 @@ def decoder_layer_workspace_bytes(cfg, batch, seq):
 
 
 def decoder_layer_fwd(cfg, blob, lora, x_in, batch, seq, x_out, ws, stream=None):
+    """x_in, x_out: fp32 [batch * seq, D] (the residual stream)."""
     c = cfg_struct(cfg)
     _check(load().decoder_layer_fwd(ctypes.byref(c), _ptr(blob), _ptr(lora), _ptr(x_in), batch,
                                     seq, _ptr(x_out), _ptr(ws), ws.numel(), _stream(stream)))
@@ -424,4 +435,4 @@ def nf4_lora_linear_fwd_noalloc(x, codes, absmax, A, B, scale, y, residual=None,
     r = A.shape[0]
     _check(load().nf4_lora_linear_fwd_noalloc(_ptr(x), T, K, N, _ptr(codes), _ptr(absmax), block,
                                               _ptr(A), _ptr(B), r, scale, _ptr(residual), _ptr(y),
-                                              _ptr(u_out), _stream(stream)))
+                                              _y_fp32(y), _ptr(u_out), _stream(stream)))

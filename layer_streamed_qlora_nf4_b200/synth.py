@@ -65,6 +65,12 @@ def bf16_bits_to_f32(b):
     return (b.astype(np.uint32) << 16).view(np.float32)
 
 
+def to_f16(a):
+    """fp32 -> fp16 (numpy float16, round to nearest even): the storage of forward
+    activations handed to the library (storage only)."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16)
+
+
 # ------------------------------------------------------------------- generators
 def rng(seed):
     return np.random.default_rng(seed)

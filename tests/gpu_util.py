@@ -16,6 +16,11 @@ def host_bf16_to_f32(t):
     return synth.bf16_bits_to_f32(t.detach().view(torch.int16).cpu().numpy().view(np.uint16))
 
 
+def dev_f16(a16):
+    """numpy float16 -> torch.float16 on cuda (the same values)."""
+    return torch.from_numpy(np.ascontiguousarray(a16, dtype=np.float16)).cuda()
+
+
 def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
@@ -36,19 +41,15 @@ def frobenius_err(got, ref):
     return float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
 
 
-# Stack-level LoRA gradients: every tensor within 2e-2 relative (Frobenius); by the
-# max-element reading every tensor within 2e-2 too, except the q and k projections,
-# whose gradients carry the forward error of all the layers above through the
-# attention backward (measured 0.015-0.022 on the small random-init stacks), bounded
-# at 3e-2.
-STACK_GRAD_TOL, STACK_QK_MAX_TOL = 2e-2, 3e-2
+# Stack-level LoRA gradients: every tensor within 2e-2 by the max-element reading
+# (max |err| / max |ref|) and in the Frobenius norm.
+STACK_GRAD_TOL = 2e-2
 
 
 def check_stack_grad(got, ref, name, where):
     f = frobenius_err(got, ref)
     m = normwise_err(got, ref)
-    lim = STACK_QK_MAX_TOL if name in ("q", "k") else STACK_GRAD_TOL
-    assert f <= STACK_GRAD_TOL and m <= lim, (where, name, f, m)
+    assert f <= STACK_GRAD_TOL and m <= STACK_GRAD_TOL, (where, name, f, m)
 
 
 def elementwise_err(got, ref, floor=1e-3):

@@ -122,9 +122,13 @@ def test_invalid_arguments_are_rejected_without_a_gpu(L):
     assert lib.nf4_quantize(p, 4, 96, 64, p, p, None) == L.LSQ_ERR_SHAPE
     assert lib.nf4_quantize(p, 4, 128, 32, p, p, None) == L.LSQ_ERR_SHAPE
     assert lib.nf4_quantize(None, 4, 128, 64, p, p, None) == L.LSQ_ERR_INVALID
-    assert lib.nf4_lora_linear_fwd(p, 8, 128, 64, p, p, 64, p, p, 8, 2.0, None, p, None, p, 1 << 20,
-                                   None) == L.LSQ_ERR_SHAPE       # r % 16 != 0
+    assert lib.nf4_lora_linear_fwd(p, 8, 128, 64, p, p, 64, p, p, 8, 2.0, None, p, 0, None, p,
+                                   1 << 20, None) == L.LSQ_ERR_SHAPE       # r % 16 != 0
     assert b"r must be" in lib.lsq_last_error()
+    # an fp32 residual needs an fp32 output (y_fp32 = 1)
+    assert lib.nf4_lora_linear_fwd(p, 8, 128, 64, p, p, 64, p, p, 16, 2.0, p, p, 0, None, p,
+                                   1 << 20, None) == L.LSQ_ERR_INVALID
+    assert b"residual" in lib.lsq_last_error()
     bad = dict(synth.SMALL, head_dim=96)
     with pytest.raises(L.LsqError) as e:
         L.lsq_layer_layout_get(bad)

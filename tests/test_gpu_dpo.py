@@ -44,19 +44,19 @@ def _dpo(L, st, h, tokens_np, pairs, seq, opt=None):
 
 def test_layer_forward_with_the_adapter_off(L):
     import torch
-    from gpu_util import dev_bf16, host_bf16_to_f32, normwise_err, workspace
+    from gpu_util import dev, normwise_err, workspace
     from test_gpu_layer import _device_layer, _oracle_params
     cfg, batch, seq = synth.SMALL, 2, 100
     lw = synth.layer_weights(12, cfg)
-    x_bits = synth.activations(13, batch * seq, cfg["hidden"])
+    x = synth.bf16_bits_to_f32(synth.activations(13, batch * seq, cfg["hidden"]))
     blob, _ = _device_layer(L, cfg, lw)
-    y = torch.empty(batch * seq, cfg["hidden"], dtype=torch.bfloat16, device="cuda")
-    L.decoder_layer_fwd(cfg, blob, None, dev_bf16(x_bits), batch, seq, y,
+    y = torch.empty(batch * seq, cfg["hidden"], dtype=torch.float32, device="cuda")
+    L.decoder_layer_fwd(cfg, blob, None, dev(x), batch, seq, y,
                         workspace(L.decoder_layer_workspace_bytes(cfg, batch, seq)))
     torch.cuda.synchronize()
     p = om.adapter_off([_oracle_params(lw, cfg)])[0]
-    ref, _ = om.decoder_layer_fwd(p, synth.bf16_bits_to_f32(x_bits), cfg, seq)
-    assert normwise_err(host_bf16_to_f32(y), ref) <= TOL
+    ref, _ = om.decoder_layer_fwd(p, x, cfg, seq)
+    assert normwise_err(y.cpu().numpy(), ref) <= TOL
 
 
 def test_dpo_step_matches_oracle(L, small):

@@ -1,7 +1,9 @@
 """GPU parity: the fused NF4 + LoRA linear (forward and backward) against the oracle.
 
 Tolerance (stated by the workload): normwise max|gpu - ref| / max|ref| <= 2e-2
-for bf16 activations and gradients against the fp64 oracle.
+for activations and gradients against the fp64 oracle.  The workload's bf16
+activations are handed to the library in fp16 (its forward operand type); both
+the library and the oracle see the same fp16 values.
 """
 import numpy as np
 import pytest
@@ -23,32 +25,33 @@ def L():
 
 def _run(L, N, K, T, r=16, alpha=32.0, seed=0, residual=False, accumulate=False, check_bwd=True):
     import torch
-    from gpu_util import dev, dev_bf16, host_bf16_to_f32, normwise_err, workspace
+    from gpu_util import dev, dev_bf16, dev_f16, host_bf16_to_f32, normwise_err, workspace
     case = synth.linear_case(seed, N, K, T, r)
     s = alpha / r
     codes, absmax = onf4.quantize(case["W"])
     Wt = onf4.dequantize(codes, absmax, N, K)
-    x = synth.bf16_bits_to_f32(case["x"])
+    x16 = synth.to_f16(synth.bf16_bits_to_f32(case["x"]))
+    x = x16.astype(np.float64)
     dy = synth.bf16_bits_to_f32(case["dy"])
-    res_bits = synth.normal_bf16(synth.rng(seed + 1), (T, N)) if residual else None
+    res = synth.bf16_bits_to_f32(synth.normal_bf16(synth.rng(seed + 1), (T, N))) if residual else None
     ref_y = om.lora_linear_fwd(x, Wt, case["A"], case["B"], s)
     if residual:
-        ref_y = ref_y + synth.bf16_bits_to_f32(res_bits)
+        ref_y = ref_y + res
     ws = workspace(L.nf4_lora_linear_workspace_bytes(T, K, N, r))
-    xd, Ad, Bd = dev_bf16(case["x"]), dev(case["A"]), dev(case["B"])
+    xd, Ad, Bd = dev_f16(x16), dev(case["A"]), dev(case["B"])
     cd, ad = dev(codes), dev(absmax)
-    y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+    # fp32 output with a residual (the residual stream), fp16 otherwise
+    y = torch.empty(T, N, dtype=torch.float32 if residual else torch.float16, device="cuda")
     u = torch.empty(T, r, dtype=torch.float32, device="cuda")
-    L.nf4_lora_linear_fwd(xd, cd, ad, Ad, Bd, s, y, residual=dev_bf16(res_bits) if residual else None,
+    L.nf4_lora_linear_fwd(xd, cd, ad, Ad, Bd, s, y, residual=dev(res) if residual else None,
                           u_out=u, ws=ws)
     torch.cuda.synchronize()
-    e_y = normwise_err(host_bf16_to_f32(y), ref_y)
+    e_y = normwise_err(y.float().cpu().numpy(), ref_y)
     e_u = normwise_err(u.cpu().numpy(), x @ case["A"].astype(np.float64).T)
     assert e_y <= TOL, e_y
-    # u = x A^T on tensor cores: x is exact in bf16, A is rounded once to bf16
-    # (an independent error of at most 2^-9 relative per element, standard
-    # deviation 2^-9/sqrt(3)), accumulation in fp32; so du/u is about 1e-3
-    # (measured 1.5e-3) and the check allows 2^-8
+    # u = x A^T on tensor cores: x is exact in fp16, A is rounded once to fp16
+    # (an independent error of at most 2^-11 relative per element), accumulation
+    # in fp32; so du/u is about 3e-4 and the check allows 2^-8
     assert e_u <= 2.0 ** -8, e_u
     if not check_bwd:
         return
@@ -110,8 +113,8 @@ def test_linear_8b_shapes(L, N, K):
 def test_linear_bad_arguments(L):
     import torch
     from gpu_util import workspace
-    x = torch.zeros(16, 100, dtype=torch.bfloat16, device="cuda")   # K % 64 != 0
-    y = torch.zeros(16, 64, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(16, 100, dtype=torch.float16, device="cuda")   # K % 64 != 0
+    y = torch.zeros(16, 64, dtype=torch.float16, device="cuda")
     A = torch.zeros(16, 100, device="cuda")
     B = torch.zeros(64, 16, device="cuda")
     codes = torch.zeros(64 * 100 // 2, dtype=torch.uint8, device="cuda")
@@ -119,8 +122,13 @@ def test_linear_bad_arguments(L):
     with pytest.raises(L.LsqError) as e:
         L.nf4_lora_linear_fwd(x, codes, am, A, B, 2.0, y, ws=workspace(1 << 20))
     assert e.value.code == L.LSQ_ERR_SHAPE
-    x = torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(16, 128, dtype=torch.float16, device="cuda")
     A = torch.zeros(16, 128, device="cuda")
     with pytest.raises(L.LsqError) as e:
         L.nf4_lora_linear_fwd(x, codes, am, A, B, 2.0, y, ws=workspace(16))
     assert e.value.code == L.LSQ_ERR_WORKSPACE
+    # a residual is added in fp32 and needs an fp32 output
+    with pytest.raises(L.LsqError) as e:
+        L.nf4_lora_linear_fwd(x, codes, am, A, B, 2.0, y, residual=torch.zeros(16, 64, device="cuda"),
+                              ws=workspace(1 << 20))
+    assert e.value.code == L.LSQ_ERR_INVALID

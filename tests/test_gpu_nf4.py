@@ -77,6 +77,13 @@ def test_quantize_rejects_nonfinite_and_bad_shapes(L):
     with pytest.raises(L.LsqError) as e:
         _quant_gpu(L, W)
     assert e.value.code == L.LSQ_ERR_INVALID
+    # finite but beyond the fp16 range of the fused GEMM's forward operand
+    W[1, 3] = 65520.0
+    with pytest.raises(L.LsqError) as e:
+        _quant_gpu(L, W)
+    assert e.value.code == L.LSQ_ERR_INVALID
+    W[1, 3] = 65504.0           # the largest finite fp16 value is accepted
+    _quant_gpu(L, W)
     Wd = torch.zeros(4, 96, device="cuda")
     codes = torch.empty(4 * 96 // 2, dtype=torch.uint8, device="cuda")
     absmax = torch.empty(6, dtype=torch.float32, device="cuda")
