@@ -417,11 +417,12 @@ int lora_adamw_step(float* lora, const float* grad, const lsq_adamw* opt, int64_
 /* Number of kernel launches the library has issued in this process. */
 int64_t lsq_launch_counter(void);
 
-/* Per-launch device timing of the library's heavy kernels.  While enabled,
- * every tensor-core GEMM and attention launch is bracketed by CUDA events
- * recorded on the stream it is launched on, together with its algorithmic
- * work (FLOPs, and the minimum DRAM bytes it must move).  Enabling costs two
- * event records per such launch. */
+/* Per-launch device timing of the library's kernels.  While enabled, every
+ * tensor-core GEMM (with its split-K reduce), attention, rank-r LoRA product and
+ * memory-bound kernel (RMSNorm, RoPE, SwiGLU, embedding, cross-entropy, AdamW)
+ * launch is bracketed by CUDA events recorded on the stream it is launched on,
+ * together with its algorithmic work (FLOPs, and the minimum DRAM bytes it must
+ * move).  Enabling costs two event records per such launch. */
 typedef struct lsq_prof_entry {
   char name[32];       /* kernel class, e.g. "gemm_nf4_fwd" */
   int64_t launches;

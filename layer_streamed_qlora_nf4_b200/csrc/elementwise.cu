@@ -496,10 +496,14 @@ int threads_for_row(int64_t D, int per) {
   return t < 32 ? 32 : t;
 }
 
+// The launchers below bracket their kernel with a profiler region (a no-op unless
+// profiling is on) that carries the kernel's algorithmic DRAM bytes: every
+// tensor it must read and write, once.
 int launch_rmsnorm_fwd(const float* x, const uint16_t* g, int64_t T, int64_t D, float eps,
                        uint16_t* y, int y_kind, float* rstd, cudaStream_t st) {
   int* dev_err = device_status_ptr();
   if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  const int prof = prof_begin(st);
   if (y_kind == OUT_F16)
     rmsnorm_fwd_kernel<true><<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd,
                                                                            dev_err);
@@ -507,15 +511,20 @@ int launch_rmsnorm_fwd(const float* x, const uint16_t* g, int64_t T, int64_t D, 
     rmsnorm_fwd_kernel<false><<<(unsigned)T, threads_for_row(D, 8), 0, st>>>(x, g, D, eps, y, rstd,
                                                                             dev_err);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0) prof_end(prof, st, "rmsnorm_fwd", 0.0, 6.0 * T * D + 2.0 * D + 4.0 * T);
   return LSQ_OK;
 }
 
 int launch_rmsnorm_bwd(const float* dy, const float* x, const uint16_t* g, const float* rstd,
                        const float* dres, int64_t T, int64_t D, float* dx, uint16_t* dx_bf16,
                        cudaStream_t st) {
+  const int prof = prof_begin(st);
   rmsnorm_bwd_kernel<<<(unsigned)T, threads_for_row(D, 4), 0, st>>>(dy, x, g, rstd, dres, D, dx,
                                                                    dx_bf16);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0)
+    prof_end(prof, st, "rmsnorm_bwd", 0.0,
+             (12.0 + (dres ? 4.0 : 0.0) + (dx_bf16 ? 2.0 : 0.0)) * T * D + 2.0 * D + 4.0 * T);
   return LSQ_OK;
 }
 
@@ -530,47 +539,64 @@ int launch_rope_table(int seq, int d, float theta, float2* cs, cudaStream_t st) 
 int launch_rope(uint16_t* qkv, int64_t T, int seq, int H, int Hkv, int d, const float2* cs,
                 cudaStream_t st) {
   const int64_t n = T * (H + Hkv) * (d / 16);
+  const int prof = prof_begin(st);
   rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(qkv, T, seq, H, Hkv, d, cs);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // q and k read and written in place (fp16), plus the table rows once
+  if (prof >= 0) prof_end(prof, st, "rope", 0.0, 4.0 * T * (H + Hkv) * d + 4.0 * seq * d);
   return LSQ_OK;
 }
 
 int launch_rope_grad(const float* dq, const float* dk, const float* dv, int64_t T, int seq, int H,
                      int Hkv, int d, const float2* cs, uint16_t* dqkv, cudaStream_t st) {
   const int64_t n = T * (H + 2 * Hkv) * (d / 8);
+  const int prof = prof_begin(st);
   rope_grad_kernel<<<grid_for(n, 256), 256, 0, st>>>(dq, dk, dv, T, seq, H, Hkv, d, cs, dqkv);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // fp32 dq, dk, dv per query head in; bf16 dq|dk|dv out
+  if (prof >= 0)
+    prof_end(prof, st, "rope_grad", 0.0, 12.0 * T * H * d + 2.0 * T * (H + 2 * Hkv) * d);
   return LSQ_OK;
 }
 
 int launch_swiglu_fwd(const uint16_t* gu, int64_t T, int64_t F, uint16_t* m, cudaStream_t st) {
   int* dev_err = device_status_ptr();
   if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  const int prof = prof_begin(st);
   swiglu_fwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(gu, T, F, m, dev_err);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0) prof_end(prof, st, "swiglu_fwd", 0.0, 6.0 * T * F);
   return LSQ_OK;
 }
 
 int launch_swiglu_bwd(const float* dm, const uint16_t* gu, int64_t T, int64_t F, uint16_t* dgu,
                       cudaStream_t st) {
+  const int prof = prof_begin(st);
   swiglu_bwd_kernel<<<grid_for(T * F / 8, 256), 256, 0, st>>>(dm, gu, T, F, dgu);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0) prof_end(prof, st, "swiglu_bwd", 0.0, 12.0 * T * F);
   return LSQ_OK;
 }
 
 int launch_embedding(const int32_t* tokens, int64_t T, const uint16_t* emb, int64_t D, int64_t V,
                      float* out, cudaStream_t st) {
+  const int prof = prof_begin(st);
   embedding_kernel<<<grid_for(T * D / 8, 256), 256, 0, st>>>(tokens, T, emb, D, V, out);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0) prof_end(prof, st, "embedding", 0.0, 6.0 * T * D + 4.0 * T);
   return LSQ_OK;
 }
 
 int launch_cross_entropy(const float* logits, const int32_t* tokens, int64_t T, int seq, int64_t V,
                          float inv_count, uint16_t* dlogits, float* row_loss, cudaStream_t st,
                          const float* seq_scale) {
+  const int prof = prof_begin(st);
   cross_entropy_kernel<<<(unsigned)T, 512, 0, st>>>(logits, tokens, T, seq, V, inv_count, seq_scale,
                                                     dlogits, row_loss);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // fp32 logits read once, bf16 dlogits written once (when asked for)
+  if (prof >= 0)
+    prof_end(prof, st, "cross_entropy", 0.0, (4.0 + (dlogits ? 2.0 : 0.0)) * T * V + 8.0 * T);
   return LSQ_OK;
 }
 
@@ -650,8 +676,11 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
                  float b2, float eps, float wd, int step, cudaStream_t st) {
   const float bc1 = (float)(1.0 - pow((double)b1, (double)step));
   const float bc2 = (float)(1.0 - pow((double)b2, (double)step));
+  const int prof = prof_begin(st);
   adamw_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // p, g, m, v read; p, m, v written (fp32)
+  if (prof >= 0) prof_end(prof, st, "adamw", 0.0, 28.0 * n);
   return LSQ_OK;
 }
 

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "../../include/lsq.h"
 
 namespace lsq {
@@ -21,9 +23,28 @@ int cuda_status(cudaError_t e, const char* what); // LSQ_OK or LSQ_ERR_CUDA with
 
 // Counts a kernel launch (wraps the cudaGetLastError check after every launch).
 cudaError_t launched(cudaError_t e);
+// Launches issued so far, and n more (the kernels of a replayed CUDA graph).
+int64_t launch_count();
+void count_launches(int64_t n);
 // Per-launch event timing of heavy kernels (no-ops unless lsq_profile_enable).
 int prof_begin(cudaStream_t st);
 void prof_end(int token, cudaStream_t st, const char* name, double flops, double bytes);
+bool prof_enabled();
+// A region recorded inside a captured CUDA graph: its events belong to the graph
+// and are re-recorded at every replay.
+struct ProfRec {
+  int cls;
+  cudaEvent_t e0, e1;
+  double flops, bytes;
+};
+// While a sink is set on the calling thread (during a stream capture),
+// prof_begin/prof_end record into fresh events and append the region to *sink.
+void prof_capture_sink(std::vector<ProfRec>* sink);
+// After a replay of a graph has completed: adds its regions' event times to the
+// profile (a no-op unless profiling is enabled).
+int prof_accumulate(const std::vector<ProfRec>& recs);
+// Destroys the regions' events.
+void prof_release(std::vector<ProfRec>& recs);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -197,12 +218,14 @@ struct LayerShapes {
 int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);
 // dx_out_bf16 may be null (then converted internally).
+// rope_cs: the cos/sin table of launch_rope_table for this seq, or null (then the
+// layer builds it in its workspace)
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
-                   cudaStream_t st);
+                   cudaStream_t st, const float2* rope_cs = nullptr);
 int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate,
-                   void* ws, size_t ws_bytes, cudaStream_t st);
+                   void* ws, size_t ws_bytes, cudaStream_t st, const float2* rope_cs = nullptr);
 
 }  // namespace lsq

@@ -333,7 +333,8 @@ int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, co
 // Forward through the SwiGLU product (everything the backward needs) and,
 // when x_out is given, the down projection with its residual.
 int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch, int seq,
-                 float theta, float eps, const Buffers& b, float* x_out, cudaStream_t st) {
+                 const float2* rope_cs, float eps, const Buffers& b, float* x_out,
+                 cudaStream_t st) {
   const int64_t T = (int64_t)batch * seq;
   const int r = v.lora_on ? s.r : 0;  // r = 0: no LoRA slab in the GEMMs
   const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
@@ -343,8 +344,7 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
                            3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_rope_table(seq, s.hd, theta, b.rope_cs, st));
-  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.rope_cs, st));
+  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
   if (v.lora_on) LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
@@ -374,7 +374,7 @@ size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
 
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
-                   cudaStream_t st) {
+                   cudaStream_t st, const float2* rope_cs) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd",
                            true));
@@ -385,13 +385,17 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   Buffers b;
   plan_buffers(s, T, ws, &b);
   const Views v = views(s, blob, lora);
-  return forward_core(s, v, x_in, batch, seq, cfg->rope_theta, cfg->rms_eps, b, x_out, st);
+  if (!rope_cs) {
+    LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, b.rope_cs, st));
+    rope_cs = b.rope_cs;
+  }
+  return forward_core(s, v, x_in, batch, seq, rope_cs, cfg->rms_eps, b, x_out, st);
 }
 
 int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate, void* ws,
-                   size_t ws_bytes, cudaStream_t st) {
+                   size_t ws_bytes, cudaStream_t st, const float2* rope_cs) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, dx_in, &s, "decoder_layer_bwd"));
   if (!dx_out || !lora_grad) return set_error(LSQ_ERR_INVALID, "decoder_layer_bwd: null pointer");
@@ -420,7 +424,11 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   const int64_t pe1[1] = {s.D};
 
   // recompute the forward from the saved input
-  LSQ_TRY(forward_core(s, v, x_in, batch, seq, cfg->rope_theta, cfg->rms_eps, b, nullptr, st));
+  if (!rope_cs) {
+    LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, b.rope_cs, st));
+    rope_cs = b.rope_cs;
+  }
+  LSQ_TRY(forward_core(s, v, x_in, batch, seq, rope_cs, cfg->rms_eps, b, nullptr, st));
 
   const uint16_t* dout_b = dx_out_bf16;
   if (!dout_b) {
@@ -452,7 +460,7 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   // attention, RoPE
   LSQ_TRY(launch_attention_bwd(b.qkv, b.ao, b.da, b.lse, T, seq, s.H, s.Hkv, s.hd, b.delta, b.dq,
                                b.dk, b.dv, st));
-  LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, b.rope_cs, b.dqkv, st));
+  LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, rope_cs, b.dqkv, st));
   // q|k|v projections
   LSQ_TRY(launch_lora_vproj(b.dqkv, T, s.qkv_n, v.B_qkv, r, 3, pe3, b.v_qkv, b.lscratch,
                             b.lscratch_bytes, st));

@@ -1,5 +1,6 @@
 // Measurement hooks: kernel-launch counter, per-launch CUDA-event timing of the
-// heavy kernel classes (recorded on the stream each kernel is launched on),
+// heavy kernel classes (recorded on the stream each kernel is launched on, or,
+// for launches captured into a CUDA graph, by event-record nodes of that graph),
 // and the standalone AdamW entry point.
 #include <atomic>
 #include <mutex>
@@ -17,6 +18,8 @@ cudaError_t launched(cudaError_t e) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return e;
 }
+int64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
+void count_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 namespace {
 
@@ -26,6 +29,11 @@ struct Rec {
   double flops, bytes;
 };
 
+struct Agg {
+  int64_t launches = 0;
+  double ms = 0, flops = 0, bytes = 0;
+};
+
 struct Profiler {
   std::mutex mu;
   bool enabled = false;
@@ -33,6 +41,7 @@ struct Profiler {
   size_t next = 0;
   std::vector<Rec> recs;
   std::vector<std::string> names;
+  std::vector<Agg> graph_acc;  // per class: regions replayed inside CUDA graphs
   int event() {
     if (next == pool.size()) {
       cudaEvent_t e;
@@ -54,12 +63,38 @@ Profiler& prof() {
   return p;
 }
 
+// Capture mode (per thread): the sink of the graph being captured, and the
+// begin events of its open regions (a token is kCapTag | index).
+thread_local std::vector<ProfRec>* t_sink = nullptr;
+thread_local std::vector<cudaEvent_t> t_open;
+constexpr int kCapTag = 1 << 30;
+
 }  // namespace
+
+bool prof_enabled() {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  return p.enabled;
+}
+
+void prof_capture_sink(std::vector<ProfRec>* sink) {
+  t_sink = sink;
+  t_open.clear();
+}
 
 int prof_begin(cudaStream_t st) {
   Profiler& p = prof();
   std::lock_guard<std::mutex> g(p.mu);
   if (!p.enabled) return -1;
+  if (t_sink) {
+    // "external": a real event-record node of the graph (a plain record during
+    // capture would only express an ordering dependency)
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    t_open.push_back(e);
+    return kCapTag | (int)(t_open.size() - 1);
+  }
   const int e = p.event();
   if (e < 0) return -1;
   cudaEventRecord(p.pool[e], st);
@@ -71,10 +106,44 @@ void prof_end(int token, cudaStream_t st, const char* name, double flops, double
   Profiler& p = prof();
   std::lock_guard<std::mutex> g(p.mu);
   if (!p.enabled) return;
+  if (token & kCapTag) {
+    const size_t i = (size_t)(token & ~kCapTag);
+    if (!t_sink || i >= t_open.size()) return;
+    cudaEvent_t e1;
+    if (cudaEventCreate(&e1) != cudaSuccess) return;
+    cudaEventRecordWithFlags(e1, st, cudaEventRecordExternal);
+    t_sink->push_back(ProfRec{p.cls(name), t_open[i], e1, flops, bytes});
+    return;
+  }
   const int e = p.event();
   if (e < 0) return;
   cudaEventRecord(p.pool[e], st);
   p.recs.push_back(Rec{p.cls(name), token, e, flops, bytes});
+}
+
+int prof_accumulate(const std::vector<ProfRec>& recs) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.enabled) return LSQ_OK;
+  if (p.graph_acc.size() < p.names.size()) p.graph_acc.resize(p.names.size());
+  for (const ProfRec& r : recs) {
+    float ms = 0.f;
+    LSQ_CUDA(cudaEventElapsedTime(&ms, r.e0, r.e1));
+    Agg& a = p.graph_acc[r.cls];
+    a.launches += 1;
+    a.ms += ms;
+    a.flops += r.flops;
+    a.bytes += r.bytes;
+  }
+  return LSQ_OK;
+}
+
+void prof_release(std::vector<ProfRec>& recs) {
+  for (ProfRec& r : recs) {
+    cudaEventDestroy(r.e0);
+    cudaEventDestroy(r.e1);
+  }
+  recs.clear();
 }
 
 }  // namespace lsq
@@ -89,6 +158,7 @@ extern "C" int lsq_profile_enable(int enable) {
   if (enable) {
     p.recs.clear();
     p.next = 0;
+    p.graph_acc.clear();
   }
   p.enabled = enable != 0;
   return LSQ_OK;
@@ -112,6 +182,12 @@ extern "C" int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out
     a.total_ms += ms;
     a.flops += r.flops;
     a.bytes += r.bytes;
+  }
+  for (size_t i = 0; i < p.graph_acc.size() && i < agg.size(); ++i) {
+    agg[i].launches += p.graph_acc[i].launches;
+    agg[i].total_ms += p.graph_acc[i].ms;
+    agg[i].flops += p.graph_acc[i].flops;
+    agg[i].bytes += p.graph_acc[i].bytes;
   }
   int n = 0;
   for (size_t i = 0; i < agg.size() && n < max; ++i)

@@ -19,6 +19,14 @@
 // copy ("ready").  Copies run one visit ahead.  Kernels are deterministic, so
 // a streamed step is bit-identical to the same step with the stack resident.
 //
+// Launches: the kernels of each layer visit (a forward, an adapter-off
+// reference forward, or a recomputing backward) are captured once into a CUDA
+// graph and replayed.  Eager launches would each have their command fetched
+// from host memory over the same PCIe link the layer copy saturates, which
+// slowed a layer's kernels by about a quarter on B200; a replayed graph's work
+// is already on the device.  A graph bakes in the step's buffers, so the cache
+// is rebuilt whenever a step passes different ones.
+//
 // Data-parallel layer sharding (stream_stack_shard): with G ranks, one process
 // per GPU, each rank copies only its 1/G slice of a layer from host memory, and
 // an in-place NCCL all-gather on the copy stream (NVLink / NVSwitch, far faster
@@ -33,8 +41,10 @@
 #include <algorithm>
 #include <chrono>
 #include <cmath>
+#include <map>
 #include <mutex>
 #include <thread>
+#include <tuple>
 #include <vector>
 
 #include "common.cuh"
@@ -62,7 +72,29 @@ struct lsq_stack {
   size_t shard = 0;            // bytes of a layer each rank fetches from host
   void* comm = nullptr;        // ncclComm_t
   int aborted = 0;             // the communicator was aborted after a timeout
+  // CUDA graphs of the layer visits, keyed by (kind: 0 forward, 1 adapter-off
+  // reference forward, 2 backward; layer; buffer; accumulate; micro-batch when
+  // profiling), valid while the step's pointers and sizes (graph_sig) are unchanged
+  struct GraphEntry {
+    cudaGraphExec_t exec = nullptr;
+    int64_t launches = 0;               // kernels in the graph
+    std::vector<lsq::ProfRec> recs;     // profiler regions inside it
+  };
+  std::map<std::tuple<int, int, int, int, int>, GraphEntry> graphs;
+  std::vector<uintptr_t> graph_sig;
+  cudaStream_t cap_stream = nullptr;    // capture only (nothing runs on it)
 };
+
+namespace {
+void drop_graphs(lsq_stack* h) {
+  for (auto& kv : h->graphs) {
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    lsq::prof_release(kv.second.recs);
+  }
+  h->graphs.clear();
+  h->graph_sig.clear();
+}
+}  // namespace
 
 namespace lsq {
 namespace {
@@ -76,6 +108,7 @@ struct StackWs {
   float* row_loss;   // [T]
   float* loss_dev;   // [1]
   float* dhf;        // [T][D]
+  float2* rope_cs;   // [seq][d/2] RoPE cos/sin table, built once per step
   float* dh[2];      // [T][D] fp32 residual-stream gradient (ping-pong)
   uint16_t* dhb[2];  // bf16 copies
   void* gemm;
@@ -144,6 +177,7 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.row_loss = a.take<float>(T);
   x.loss_dev = a.take<float>(64);
   x.dhf = a.take<float>(T * D);
+  x.rope_cs = a.take<float2>(T * s.hd / 2);  // >= seq * d/2 entries
   for (int i = 0; i < 2; ++i) {
     x.dh[i] = a.take<float>(T * D);
     x.dhb[i] = a.take<uint16_t>(T * D);
@@ -342,8 +376,9 @@ extern "C" int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_
   h->stats = lsq_step_stats{};
   cudaGetDevice(&h->device);
   int rc = LSQ_OK;
-  if (cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
-    rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create copy stream");
+  if (cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+    rc = set_error(LSQ_ERR_CUDA, "stream_stack_create: cannot create streams");
   for (int i = 0; rc == LSQ_OK && i < 2; ++i)
     if (cudaEventCreateWithFlags(&h->ready[i], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&h->freed[i], cudaEventDisableTiming) != cudaSuccess)
@@ -366,6 +401,8 @@ extern "C" int stream_stack_destroy(lsq_stack* h) {
   if (!h) return LSQ_OK;
   cudaStreamSynchronize(h->copy_stream);
   cudaStreamDestroy(h->copy_stream);
+  drop_graphs(h);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (int i = 0; i < 2; ++i) {
     cudaEventDestroy(h->ready[i]);
     cudaEventDestroy(h->freed[i]);
@@ -536,6 +573,51 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
     ++copies;
     return LSQ_OK;
   };
+  // The layer visits run as replays of cached CUDA graphs.  A graph bakes in
+  // every pointer its kernels get, so the cache is dropped whenever this step's
+  // buffers, sizes or profiling state differ from the ones it was captured with.
+  const bool profiling = prof_enabled();
+  {
+    const std::vector<uintptr_t> sig = {
+        (uintptr_t)lora, (uintptr_t)lora_grad, (uintptr_t)ws, (uintptr_t)ws_bytes,
+        (uintptr_t)batch, (uintptr_t)seq, (uintptr_t)micro_batches, (uintptr_t)profiling,
+        (uintptr_t)(dpo != nullptr)};
+    if (sig != h->graph_sig) {
+      drop_graphs(h);
+      h->graph_sig = sig;
+    }
+  }
+  if (!device_status_ptr()) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  std::vector<const std::vector<ProfRec>*> replayed;  // profiled graphs launched in this step
+  // Replays the graph of key k, capturing it first with enqueue(capture stream).
+  auto visit = [&](std::tuple<int, int, int, int, int> k, auto&& enqueue) -> int {
+    auto it = h->graphs.find(k);
+    if (it == h->graphs.end()) {
+      lsq_stack::GraphEntry e;
+      LSQ_CUDA(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeRelaxed));
+      if (profiling) prof_capture_sink(&e.recs);
+      const int64_t n0 = launch_count();
+      const int rc = enqueue(h->cap_stream);
+      e.launches = launch_count() - n0;
+      prof_capture_sink(nullptr);
+      cudaGraph_t g = nullptr;
+      cudaError_t ce = cudaStreamEndCapture(h->cap_stream, &g);
+      if (rc == LSQ_OK && ce == cudaSuccess) ce = cudaGraphInstantiate(&e.exec, g, 0);
+      if (g) cudaGraphDestroy(g);
+      if (rc != LSQ_OK || ce != cudaSuccess) {
+        prof_release(e.recs);
+        cudaGetLastError();
+        return rc != LSQ_OK ? rc : cuda_status(ce, "layer visit graph");
+      }
+      it = h->graphs.emplace(k, std::move(e)).first;
+    } else {
+      count_launches(it->second.launches);  // the graph's kernels run again
+    }
+    LSQ_CUDA(cudaGraphLaunch(it->second.exec, cs));
+    if (profiling) replayed.push_back(&it->second.recs);
+    return LSQ_OK;
+  };
+
   // Returns the device pointer of visit j's layer, after fencing the compute stream.
   auto acquire = [&](size_t j, const void** blob) -> int {
     if (h->resident) return LSQ_OK;
@@ -549,6 +631,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   };
 
   LSQ_CUDA(cudaEventRecord(h->t_start, cs));
+  LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, w.rope_cs, cs));
   // Sharded: the step's first all-gather waits for everything the caller put on
   // the compute stream before the step (e.g. a gradient all-reduce on another
   // communicator), so that collectives of the two never run interleaved.
@@ -558,15 +641,21 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   for (int mb = 0; mb < micro_batches; ++mb) {
     const int32_t* tok = tokens + (int64_t)mb * T;
     LSQ_TRY(launch_embedding(tok, T, emb, D, V, w.xs, cs));
+    const int mbk = profiling ? mb : 0;  // profiled graphs are replayed once per step
     for (int i = 0; i < L; ++i, ++j) {
       const void* blob = h->blobs[i];
       if (!h->resident) LSQ_TRY(acquire(j, &blob));
-      LSQ_TRY(layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats, w.xs + (size_t)i * T * D,
-                             batch, seq, w.xs + (size_t)(i + 1) * T * D, w.layer_ws,
-                             w.layer_ws_bytes, cs));
+      const int b = h->resident ? -1 : visits[j].buf;
+      LSQ_TRY(visit(std::make_tuple(0, i, b, 0, mbk), [&](cudaStream_t s) {
+        return layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
+                              w.xs + (size_t)i * T * D, batch, seq, w.xs + (size_t)(i + 1) * T * D,
+                              w.layer_ws, w.layer_ws_bytes, s, w.rope_cs);
+      }));
       if (dpo)  // reference model: the same layer with its adapter off
-        LSQ_TRY(layer_fwd_impl(cfg, blob, nullptr, i == 0 ? w.xs : w.xr[(i - 1) & 1], batch, seq,
-                               w.xr[i & 1], w.layer_ws, w.layer_ws_bytes, cs));
+        LSQ_TRY(visit(std::make_tuple(1, i, b, 0, mbk), [&](cudaStream_t s) {
+          return layer_fwd_impl(cfg, blob, nullptr, i == 0 ? w.xs : w.xr[(i - 1) & 1], batch, seq,
+                                w.xr[i & 1], w.layer_ws, w.layer_ws_bytes, s, w.rope_cs);
+        }));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
     }
     const float* xL = w.xs + (size_t)L * T * D;
@@ -594,10 +683,14 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
     for (int i = L - 1; i >= 0; --i, ++j) {
       const void* blob = h->blobs[i];
       if (!h->resident) LSQ_TRY(acquire(j, &blob));
-      LSQ_TRY(layer_bwd_impl(cfg, blob, lora + (int64_t)i * layer_floats, w.xs + (size_t)i * T * D,
-                             w.dh[cur], w.dhb[cur], batch, seq, w.dh[1 - cur], w.dhb[1 - cur],
-                             lora_grad + (int64_t)i * layer_floats, mb > 0 ? 1 : 0, w.layer_ws,
-                             w.layer_ws_bytes, cs));
+      const int b = h->resident ? -1 : visits[j].buf;
+      const int acc = mb > 0 ? 1 : 0;
+      LSQ_TRY(visit(std::make_tuple(2, i, b, acc, mbk), [&](cudaStream_t s) {
+        return layer_bwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
+                              w.xs + (size_t)i * T * D, w.dh[cur], w.dhb[cur], batch, seq,
+                              w.dh[1 - cur], w.dhb[1 - cur], lora_grad + (int64_t)i * layer_floats,
+                              acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs);
+      }));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
       cur = 1 - cur;
     }
@@ -621,6 +714,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
       return rc;
     }
   }
+  for (const std::vector<ProfRec>* r : replayed) LSQ_TRY(prof_accumulate(*r));
   int flags = 0;
   int* st = device_status_ptr();
   if (st) {
