@@ -46,6 +46,25 @@ namespace lsq {
 
 __device__ int g_lsq_dev_status;
 
+#ifdef LSQ_GEMM_STAMPS
+// Diagnostic build only (-DLSQ_GEMM_STAMPS): per-CTA globaltimer stamps of the
+// kernel's phases for the most recent launch, read by lsq_debug_gemm_stamps.
+// Slots: 0 entry, 1 set-up done, 2 first stage ready (MMA issuer), 3 last MMA
+// issued, 4 accumulator ready (epilogue warp 4), 5 epilogue stores done, 6 exit,
+// 7 summed issuer wait on operand-ready barriers (ns).
+constexpr int kStampCtas = 1024;
+__device__ unsigned long long g_gemm_stamps[kStampCtas][8];
+#define LSQ_STAMP(slot, v)                                                         \
+  do {                                                                             \
+    const int _c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (_c < kStampCtas) g_gemm_stamps[_c][slot] = (v);                            \
+  } while (0)
+#else
+#define LSQ_STAMP(slot, v) \
+  do {                     \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 384;   // 4 control warps + 8 operand/epilogue warps
@@ -111,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &abort_sh;
+  if (threadIdx.x == 0) LSQ_STAMP(0, globaltimer_ns());
   constexpr bool F16 = wmode_f16(WMODE);  // fp16 operands (forward) or bf16 (input gradient)
   auto pack2 = [](float lo, float hi) -> uint32_t {
     return F16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
@@ -180,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (PAIR) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  if (threadIdx.x == 0) LSQ_STAMP(1, globaltimer_ns());
 
   if (warp == 0) {
     // ---------------------------------------------------------- activation TMA producer
@@ -223,13 +244,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issuer (lane 0)
     const uint32_t idesc = F16 ? umma_idesc_f16(PAIR ? 2 * kBM : kBM, p.bn)
                                : umma_idesc_bf16(PAIR ? 2 * kBM : kBM, p.bn);
+#ifdef LSQ_GEMM_STAMPS
+    unsigned long long waited = 0;
+#endif
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
+#ifdef LSQ_GEMM_STAMPS
+      const unsigned long long w0 = globaltimer_ns();
+#endif
       bool ok = PAIR ? mbar_wait_bounded_cluster(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
                                                  DEV_ERR_WAIT_GEMM)
                      : mbar_wait_bounded(smem_u32(&bar_full[s]), ph, abort_flag, p.dev_err,
                                          DEV_ERR_WAIT_GEMM);
+#ifdef LSQ_GEMM_STAMPS
+      const unsigned long long w1 = globaltimer_ns();
+      waited += w1 - w0;
+      if (it == 0 && lane == 0) LSQ_STAMP(2, w1);
+#endif
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
       if (lane == 0) {
@@ -261,6 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit_pair(smem_u32(&bar_acc));
       else
         tc_commit(smem_u32(&bar_acc));
+#ifdef LSQ_GEMM_STAMPS
+      LSQ_STAMP(3, globaltimer_ns());
+      LSQ_STAMP(7, waited);
+#endif
     }
     __syncwarp();
   } else if (PAIR && warp == 1) {
@@ -533,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool acc_ok = ok && mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
                                           DEV_ERR_WAIT_GEMM);
     acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
+    if (warp == 4 && lane == 0) LSQ_STAMP(4, globaltimer_ns());
     if (acc_ok) {
       tc_fence_after();
       const int qtr = warp & 3;          // TMEM lane quarter = features 32 qtr .. +31
@@ -607,6 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (lane == 0) bulk_wait_all();
+      if (warp == 4 && lane == 0) LSQ_STAMP(5, globaltimer_ns());
       if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
       __syncwarp();
     }
@@ -626,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     else
       tmem_dealloc(tmem, p.alloc_cols);
   }
+  if (threadIdx.x == 0) LSQ_STAMP(6, globaltimer_ns());
 }
 
 // ------------------------------------------------------------------ host side
@@ -874,6 +913,16 @@ int* device_status_ptr() {
   }
   return ptrs[dev];
 }
+
+#ifdef LSQ_GEMM_STAMPS
+}  // namespace lsq
+// Diagnostic build only: copies the stamps of the last launch (kStampCtas x 8) to host.
+extern "C" int lsq_debug_gemm_stamps(unsigned long long* out) {
+  return cudaMemcpyFromSymbol(out, lsq::g_gemm_stamps, sizeof(lsq::g_gemm_stamps)) == cudaSuccess
+             ? 0 : 3;
+}
+namespace lsq {
+#endif
 
 size_t gemm_workspace_bytes(const GemmDesc& d) {
   if (d.M <= 0 || d.T <= 0 || d.Kc <= 0) return 0;
