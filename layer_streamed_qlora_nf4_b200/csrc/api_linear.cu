@@ -32,6 +32,8 @@ namespace {
 struct LinearWs {
   float* u;
   float* v;
+  uint16_t* u16;  // bf16 copies for the dA / dB products
+  uint16_t* v16;
   float* scratch;
   size_t scratch_bytes;
   void* gemm;
@@ -105,11 +107,15 @@ size_t linear_ws_plan(int64_t T, int64_t K, int64_t N, int r, LinearWs* w, void*
   b.cap = SIZE_MAX;
   float* u = b.take<float>((size_t)T * r);
   float* v = b.take<float>((size_t)T * r);
+  uint16_t* u16 = b.take<uint16_t>((size_t)T * r);
+  uint16_t* v16 = b.take<uint16_t>((size_t)T * r);
   float* s = b.take<float>(sb / sizeof(float) + 1);
   void* g = b.take<uint8_t>(gb + 256);
   if (w) {
     w->u = base ? u : nullptr;
     w->v = base ? v : nullptr;
+    w->u16 = base ? u16 : nullptr;
+    w->v16 = base ? v16 : nullptr;
     w->scratch = base ? s : nullptr;
     w->scratch_bytes = sb;
     w->gemm = base ? g : nullptr;
@@ -176,7 +182,7 @@ extern "C" int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int6
   linear_ws_plan(T, K, N, r, &w, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* u = u_out ? u_out : w.u;
-  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, u, w.scratch, w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, u, nullptr, w.scratch, w.scratch_bytes, st));
   GemmDesc d = fwd_desc(x, T, K, N, codes, absmax, B, r, scale, u, residual, y, y_fp32);
   return gemm_run(d, w.gemm, w.gemm_bytes, st);
 }
@@ -195,12 +201,13 @@ extern "C" int nf4_lora_linear_bwd(const uint16_t* dy, const uint16_t* x, int64_
   linear_ws_plan(T, K, N, r, &w, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t pe[1] = {N};
-  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, w.u, w.scratch, w.scratch_bytes, st));
-  LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, 1, pe, w.v, w.scratch, w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, w.u, w.u16, w.scratch, w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, w.v, w.v16, w.scratch, w.scratch_bytes, st));
   GemmDesc d = bwd_desc(dy, T, K, N, codes, absmax, A, r, scale, w.v, dx);
   LSQ_TRY(gemm_run(d, w.gemm, w.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(w.v, x, T, K, r, scale, accumulate, dA, w.scratch, w.scratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b(dy, w.u, T, N, r, r, 1, pe, scale, accumulate, dB, w.scratch,
-                             w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_a16(w.v16, x, T, K, r, scale, accumulate, dA, w.scratch,
+                               w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b16(dy, w.u16, T, N, r, 1, pe, scale, accumulate, dB, w.scratch,
+                               w.scratch_bytes, st));
   return LSQ_OK;
 }

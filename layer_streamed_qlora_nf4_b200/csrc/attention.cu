@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
                                                        int seq, int H, int Hkv,
                                                        uint16_t* __restrict__ out,
                                                        float* __restrict__ lse_out, float sl2) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Qs = smem_attn;
   uint16_t* Kb = Qs + kTile * (D + 8);      // [2] K tiles
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
 template <int D>
 __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                   int64_t T, int H, float* __restrict__ delta) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= T * H) return;
@@ -279,6 +281,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ dout,
     const float* __restrict__ lse, const float* __restrict__ delta, int64_t T, int seq, int H,
     int Hkv, float sl2, float scale, float* __restrict__ dk, float* __restrict__ dv) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Ks = smem_attn;
   uint16_t* Vs = Ks + kTile * (D + 8);
@@ -440,6 +443,7 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
     const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ dout,
     const float* __restrict__ lse, const float* __restrict__ delta, int64_t T, int seq, int H,
     int Hkv, float sl2, float scale, float* __restrict__ dq) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   extern __shared__ __align__(16) uint16_t smem_attn[];
   uint16_t* Qs = smem_attn;
   uint16_t* dOs = Qs + kTile * (D + 8);

@@ -139,6 +139,19 @@ __device__ __forceinline__ void settle_ns(uint64_t ns) {
   }
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while the
+// kernel before it in the stream still runs; pdl_wait() blocks the calling
+// thread until that kernel has completed and its memory is visible (a no-op
+// for a normally launched kernel).  pdl_trigger() lets the next kernel, if it
+// was launched that way, start once every CTA of this one has triggered or
+// exited (so the next kernel's CTAs only take resources after all of this
+// kernel's CTAs are resident).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // ------------------------------------------------------------------ cp.async
 // 4-byte asynchronous global->shared copy; src_bytes 0 writes zeros instead.
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {

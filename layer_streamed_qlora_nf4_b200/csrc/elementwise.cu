@@ -45,6 +45,7 @@ unsigned grid_for(int64_t n, int threads, int per_thread = 1) {
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t T,
                                      int64_t M, void* __restrict__ out, int out_kind, int64_t ldo,
                                      const float* __restrict__ res, int64_t ldr, int* dev_err) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t n4 = T * M / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -100,6 +101,7 @@ template <bool F16OUT>
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, const uint16_t* __restrict__ g,
                                    int64_t D, float eps, uint16_t* __restrict__ y,
                                    float* __restrict__ rstd, int* dev_err) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const float4* xr = reinterpret_cast<const float4*>(x + row * D);
@@ -149,6 +151,7 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const float* __
                                    const uint16_t* __restrict__ g, const float* __restrict__ rstd,
                                    const float* __restrict__ dres, int64_t D,
                                    float* __restrict__ dx, uint16_t* __restrict__ dxb) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   __shared__ float red[32];
   const int64_t row = blockIdx.x;
   const int nv = (int)(D / 4);
@@ -196,6 +199,7 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const float* __
 // ------------------------------------------------------------------ RoPE
 // cs[pos][i] = (cos, sin)(pos * theta^(-2i/d)), evaluated in double, rounded to fp32.
 __global__ void rope_table_kernel(int seq, int half, int d, double log_theta, float2* __restrict__ cs) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int n = seq * half;
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
     const int pos = k / half, i = k % half;
@@ -210,6 +214,7 @@ __global__ void rope_table_kernel(int seq, int half, int d, double log_theta, fl
 // thread rotates 8 pairs (i, i + d/2).
 __global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int H, int Hkv, int d,
                             const float2* __restrict__ cs) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int half = d / 2, chunks = half / 8;
   const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
   const int64_t n = T * (H + Hkv) * chunks;
@@ -245,6 +250,7 @@ __global__ void rope_grad_kernel(const float* __restrict__ dq, const float* __re
                                  const float* __restrict__ dv, int64_t T, int seq, int H, int Hkv,
                                  int d, const float2* __restrict__ cs,
                                  uint16_t* __restrict__ dqkv) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int half = d / 2, chunks = half / 4, rep = H / Hkv;
   const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
   const int64_t hd = (int64_t)H * d;
@@ -300,6 +306,7 @@ __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-
 // fp16 range latches the non-finite status bit)
 __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, int64_t F,
                                   uint16_t* __restrict__ m, int* dev_err) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t nv = T * F / 8;
   bool big = false;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
@@ -324,6 +331,7 @@ __global__ void swiglu_fwd_kernel(const uint16_t* __restrict__ gu, int64_t T, in
 
 __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* __restrict__ gu,
                                   int64_t T, int64_t F, uint16_t* __restrict__ dgu) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t nv = T * F / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -354,6 +362,7 @@ __global__ void swiglu_bwd_kernel(const float* __restrict__ dm, const uint16_t* 
 __global__ void embedding_kernel(const int32_t* __restrict__ tok, int64_t T,
                                  const uint16_t* __restrict__ emb, int64_t D, int64_t V,
                                  float* __restrict__ out) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t nv = D / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T * nv;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -382,6 +391,7 @@ __global__ void cross_entropy_kernel(const float* __restrict__ logits,
                                      const float* __restrict__ seq_scale,
                                      uint16_t* __restrict__ dlogits,
                                      float* __restrict__ row_loss) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   __shared__ float red[32];
   __shared__ float bcast;
   const int64_t row = blockIdx.x;
@@ -436,6 +446,7 @@ __global__ void cross_entropy_kernel(const float* __restrict__ logits,
 
 __global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float scale,
                                 int accumulate, float* __restrict__ out) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   __shared__ float red[32];
   float s = 0.f;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += v[i];
@@ -452,6 +463,7 @@ __global__ void sum_rows_kernel(const float* __restrict__ v, int64_t n, float sc
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
                              float* __restrict__ m, float* __restrict__ v, int64_t n, float lr,
                              float b1, float b2, float eps, float wd, float bc1, float bc2) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const float gi = g[i];
@@ -466,12 +478,14 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t n,
                                    uint16_t* __restrict__ y) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
     y[i] = float_to_bf16_bits(x[i]);
 }
 
 __global__ void scale_kernel(float* __restrict__ x, int64_t n, float s) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
     x[i] *= s;
@@ -610,6 +624,7 @@ __global__ void dpo_loss_kernel(const float* __restrict__ row_pol,
                                 const float* __restrict__ row_ref, int pairs, int seq, float beta,
                                 float* __restrict__ seq_scale, float* __restrict__ logps,
                                 float* __restrict__ loss_out) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   __shared__ double red[2][32];
   __shared__ double lp[2][64];  // [pol/ref][sequence], pairs <= 32
   const int nseq = 2 * pairs;

@@ -35,6 +35,10 @@
 // results are deterministic and independent of scheduling.
 // Every mbarrier wait is bounded (1 s) and aborts the CTA with a device status
 // bit instead of hanging.
+// Launch: programmatic dependent launch, so that the set-up (barriers, TMEM) and
+// the first weight stages - the frozen weight does not depend on the kernel
+// before - overlap that kernel's last wave; the activation loads, the LoRA slab
+// and the epilogue wait for it (pdl_wait).
 #include <cuda.h>
 
 #include <cstdlib>
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
   __shared__ __align__(8) uint64_t bar_opd[kMaxStages];  // PAIR, odd CTA: its operand warps done
-  __shared__ __align__(8) uint64_t bar_res[kOpWarps];  // per epilogue warp: residual tile landed
+  __shared__ __align__(8) uint64_t bar_res[kThreads / 32];  // per warp: residual tile landed
   __shared__ __align__(8) uint64_t bar_grp;            // the operand warps
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -174,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bar_cempty[c]), kOpWarps);
     }
     mbar_init(smem_u32(&bar_acc), 1);
-    for (int w = 0; w < kOpWarps; ++w) mbar_init(smem_u32(&bar_res[w]), 1);
+    for (int w = 0; w < kThreads / 32; ++w) mbar_init(smem_u32(&bar_res[w]), 1);
     mbar_init(smem_u32(&bar_grp), kOpWarps);
     abort_sh = 0;
     fence_mbar_init();
@@ -205,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------- activation TMA producer
     // The whole warp walks the loop (so it reaches the final barrier converged);
-    // lane 0 issues.
+    // lane 0 issues.  The activations come from the kernel before: wait for it.
+    pdl_wait();
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -510,7 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // LoRA slab: la -> weight stage, lb -> activation stage
+        // LoRA slab: la -> weight stage, lb -> activation stage (lb comes from the
+        // kernel before: wait for it)
+        pdl_wait();
         ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                DEV_ERR_WAIT_GEMM);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -560,20 +567,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(PAIR && !leader ? &bar_opd[s] : &bar_full[s]));
     }
 
-    // ---------------------------------------------------------- epilogue (per warp)
-    // Each warp owns a 32-feature quarter of the tile (its TMEM lanes) and every
-    // other 32-token chunk; it stages a chunk in two private shared-memory slots
-    // and writes it with TMA stores of [16 tokens x 32 features] boxes, so no
-    // warp waits for another.  Residual tiles arrive by TMA into the slot and are
-    // added in place.
-    bool acc_ok = ok && mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
-                                          DEV_ERR_WAIT_GEMM);
+  }
+
+  // ------------------------------------------------------------ epilogue (all 12 warps)
+  // Every warp joins once the accumulator is complete: warp w reads TMEM lane
+  // quarter w % 4 (32 features) and takes every third 32-token chunk of that
+  // quarter (w / 4 selects which); it stages a chunk in two private
+  // shared-memory slots of the drained pipeline and writes it with TMA stores of
+  // [16 tokens x 32 features] boxes, so no warp waits for another.  Residual
+  // tiles arrive by TMA into the slot, the next chunk's while this one stores.
+  {
+    pdl_wait();  // the residual and the output buffers belong to the kernels before
+    bool acc_ok = mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, p.dev_err,
+                                    DEV_ERR_WAIT_GEMM);
     acc_ok = __all_sync(0xFFFFFFFFu, acc_ok && (*abort_flag == 0));
     if (warp == 4 && lane == 0) LSQ_STAMP(4, globaltimer_ns());
     if (acc_ok) {
       tc_fence_after();
       const int qtr = warp & 3;          // TMEM lane quarter = features 32 qtr .. +31
-      const int cgrp = ow >> 2;          // chunks q with q % 2 == cgrp
+      const int part = warp >> 2;        // chunks q with q % 3 == part
       const uint32_t tbase = tmem + ((uint32_t)(qtr * 32) << 16);
       const bool partial = p.splits > 1;
       const bool f32 = partial || p.out_f32;
@@ -581,67 +593,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool res = !partial && p.residual != nullptr;  // fp32, with an fp32 output
       bool big = false;  // an fp16 output beyond the fp16 range
       const uint32_t sub_bytes = 16u * 32u * (uint32_t)es;   // one [16 x 32] box
-      uint8_t* myslots = dsm + (size_t)ow * 8192;            // 2 slots of <= 4 KB
+      uint8_t* myslots = dsm + (size_t)warp * 8192;          // 2 slots of <= 4 KB
+      const uint32_t rbar = smem_u32(&bar_res[warp]);
       const int mcol = m0 + qtr * 32;
-      int q = 0, nq = 0, nres = 0;
-      for (int a = 0; a < p.nacc && acc_ok; ++a) {
-        for (int c0 = 0; c0 < p.bn; c0 += 32, ++q) {
-          const int tb = t0 + a * p.bn + c0;
-          if (tb >= p.T) break;
-          if ((q & 1) != cgrp) continue;
-          const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
-          uint8_t* slot = myslots + (nq & 1) * (2 * sub_bytes);
-          if (nq >= 2 && lane == 0) bulk_wait_read<1>();  // the store that used this slot has read it
-          __syncwarp();
-          if (res) {
-            if (lane == 0) {
-              mbar_arrive_expect_tx(smem_u32(&bar_res[ow]), (uint32_t)nsub * sub_bytes);
-              for (int sb = 0; sb < nsub; ++sb)
-                tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, smem_u32(&bar_res[ow]), mcol,
-                            tb + 16 * sb);
-            }
-            acc_ok = mbar_wait_bounded(smem_u32(&bar_res[ow]), (uint32_t)(nres & 1), abort_flag,
-                                       p.dev_err, DEV_ERR_WAIT_GEMM);
-            acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
-            ++nres;
-            if (!acc_ok) break;
-          }
-          uint32_t rg[2][16];
-          tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, rg[0]);
-          if (nsub == 2) tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0 + 16, rg[1]);
-          tmem_ld_wait();
-          for (int sb = 0; sb < nsub; ++sb) {
-            uint8_t* base = slot + sb * sub_bytes;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              float v = __uint_as_float(rg[sb][j]);
-              if (f32) {
-                float* d = reinterpret_cast<float*>(base + (j * 32 + lane) * 4);
-                if (res) v += *d;
-                *d = v;
-              } else if (F16) {
-                big |= !(fabsf(v) <= kF16Max);
-                *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_f16_bits(v);
-              } else {
-                *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_bf16_bits(v);
-              }
+      // this warp's chunks (at most 6: 2 accumulators x 8 chunks / 3)
+      int ma[8], mc[8], nm = 0;
+      {
+        int q = 0;
+        for (int a = 0; a < p.nacc; ++a)
+          for (int c0 = 0; c0 < p.bn; c0 += 32, ++q) {
+            if (t0 + a * p.bn + c0 >= p.T) break;
+            if (q % 3 == part && nm < 8) {
+              ma[nm] = a;
+              mc[nm] = c0;
+              ++nm;
             }
           }
-          fence_proxy_async_smem();
+      }
+      auto issue_res = [&](int i) {  // lane 0: residual of my chunk i into slot i & 1
+        const int tb = t0 + ma[i] * p.bn + mc[i];
+        const int nsub = (p.bn - mc[i] >= 32) ? 2 : 1;
+        uint8_t* slot = myslots + (i & 1) * (2 * sub_bytes);
+        mbar_arrive_expect_tx(rbar, (uint32_t)nsub * sub_bytes);
+        for (int sb = 0; sb < nsub; ++sb)
+          tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, rbar, mcol, tb + 16 * sb);
+      };
+      if (res && nm > 0 && lane == 0) issue_res(0);
+      for (int i = 0; i < nm && acc_ok; ++i) {
+        const int a = ma[i], c0 = mc[i];
+        const int tb = t0 + a * p.bn + c0;
+        const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
+        uint8_t* slot = myslots + (i & 1) * (2 * sub_bytes);
+        if (res) {
+          acc_ok = mbar_wait_bounded(rbar, (uint32_t)(i & 1), abort_flag, p.dev_err,
+                                     DEV_ERR_WAIT_GEMM);
+          acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
+          if (!acc_ok) break;
+        } else {
+          if (i >= 2 && lane == 0) bulk_wait_read<1>();  // the store that used this slot has read it
           __syncwarp();
-          if (lane == 0) {
-            for (int sb = 0; sb < nsub; ++sb) {
-              if (tb + 16 * sb >= p.T) break;
-              if (partial)
-                tma_store_3d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb, split);
-              else
-                tma_store_2d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb);
-            }
-            bulk_commit();
-          }
-          __syncwarp();
-          ++nq;
         }
+        uint32_t rg[2][16];
+        tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0, rg[0]);
+        if (nsub == 2) tmem_ld16(tbase + (uint32_t)a * acc_stride + (uint32_t)c0 + 16, rg[1]);
+        tmem_ld_wait();
+        for (int sb = 0; sb < nsub; ++sb) {
+          uint8_t* base = slot + sb * sub_bytes;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float v = __uint_as_float(rg[sb][j]);
+            if (f32) {
+              float* d = reinterpret_cast<float*>(base + (j * 32 + lane) * 4);
+              if (res) v += *d;
+              *d = v;
+            } else if (F16) {
+              big |= !(fabsf(v) <= kF16Max);
+              *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_f16_bits(v);
+            } else {
+              *reinterpret_cast<uint16_t*>(base + (j * 32 + lane) * 2) = float_to_bf16_bits(v);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int sb = 0; sb < nsub; ++sb) {
+            if (tb + 16 * sb >= p.T) break;
+            if (partial)
+              tma_store_3d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb, split);
+            else
+              tma_store_2d(&tm_out, smem_u32(slot + sb * sub_bytes), mcol, tb + 16 * sb);
+          }
+          bulk_commit();
+          if (res && i + 1 < nm) {
+            bulk_wait_read<1>();  // chunk i - 1's store has read slot (i + 1) & 1
+            issue_res(i + 1);
+          }
+        }
+        __syncwarp();
       }
       if (lane == 0) bulk_wait_all();
       if (warp == 4 && lane == 0) LSQ_STAMP(5, globaltimer_ns());
@@ -769,7 +798,7 @@ Plan make_plan(const GemmDesc& d) {
   while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;
   pl.stages = stages;
   pl.ring_stages = std::max(ring, 1);
-  pl.smem_bytes = std::max(total(stages, ring), 1024u + 4u * 16384u);  // epilogue chunk slots
+  pl.smem_bytes = std::max(total(stages, ring), 1024u + 12u * 8192u);  // epilogue chunk slots
   uint32_t cols = 32;
   while (cols < (uint32_t)pl.bn) cols <<= 1;
   pl.alloc_cols = (pl.nacc > 1) ? 512u : cols;
@@ -878,13 +907,15 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = pl.smem_bytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = PAIR ? 2 : 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   LSQ_CUDA(::lsq::launched(
       cudaLaunchKernelEx(&cfg, tc_gemm_kernel<WMODE, PAIR>, tm_act, tm_w, tm_out, tm_res, p)));
   return LSQ_OK;

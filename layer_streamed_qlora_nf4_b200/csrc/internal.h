@@ -174,29 +174,59 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st);
 int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 
-// LoRA rank-r products (tensor cores, bf16 operands, fp32 accumulation, fixed-order
-// reductions)
-// u[t, j] = sum_k x[t, k] * A[j, k]                     x fp16 [T, K], A fp32 [R, K] -> u [T, R]
-// (fp16 products: A rounded once to fp16)
-// scratch: lora_scratch_bytes(T, K, R) bytes for the bf16 copy of the LoRA operand and the
-// fixed-order partials of a product split along its reduction
+// LoRA rank-r products (tensor cores, fp32 accumulation, fixed-order reductions).
+// Operands in their product types: u = x A^T multiplies fp16 (x an fp16 forward
+// activation, A rounded to fp16); v, dA, dB multiply bf16 (each has a gradient
+// operand).  Widths R are multiples of 8.  The products that feed another write
+// its operand too (u16, v16: the result rounded to bf16).
+// scratch: lora_scratch_bytes(T, K, R) bytes for the fixed-order partials of a
+// product split along its reduction (and, in the fp32-operand forms, the 16-bit
+// copy of the LoRA operand).
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
-int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K,
-                     int R, float* u, float* scratch, size_t scratch_bytes, cudaStream_t st);
-// v[t, p*r + j] = sum_{n in part p} dy[t, n] * B[n, j] dy bf16 [T, N], B fp32 [N, r]
-// scratch: lora_scratch_bytes(T, max part size, n_parts * r) bytes
-int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r,
-                      int n_parts, const int64_t* part_end, float* v, float* scratch,
-                      size_t scratch_bytes, cudaStream_t st);
-// dA[j, k] (+)= s * sum_t v[t, j] * x[t, k]              v fp32 [T, R], x fp16 [T, K]
-// (bf16 products: v rounded once to bf16, x from fp16 to bf16 as it is loaded)
-int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
-                       int accumulate, float* dA, float* scratch, size_t scratch_bytes,
+// u[t, j] = sum_k x[t, k] A[j, k]        x fp16 [T, ldx], A16 fp16 [R, K] -> u fp32 [T, R]
+int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
+                       int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
                        cudaStream_t st);
-// dB[n, j] (+)= s * sum_t dy[t, n] * u[t, part(n)*r + j]  dy bf16 [T, N], u fp32 [T, R]
-int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
-                       int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
-                       float* scratch, size_t scratch_bytes, cudaStream_t st);
+// v[t, c] = sum_n dy[t, n] Bs[n, c]      dy bf16 [T, N], Bs bf16 [N, R] (block-diagonal:
+// row n of part p holds B_p's row in columns [p r, (p + 1) r), zeros elsewhere)
+int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
+                        float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
+                        cudaStream_t st);
+// dA[j, k] (+)= s sum_t v[t, j] x[t, k]  v16 bf16 [T, R], x fp16 [T, K] (rounded to bf16
+// as it is loaded)
+int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
+                         float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
+                         cudaStream_t st);
+// dB[n, j] (+)= s sum_t dy[t, n] u[t, part(n) r + j]   dy bf16 [T, N], u16 bf16 [T, n_parts r];
+// one product over all parts (parts of rows ending at part_end[])
+int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
+                         int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
+                         float* scratch, size_t scratch_bytes, cudaStream_t st);
+// fp32-operand forms for a single linear (one part): the LoRA operand is rounded
+// once into the scratch first
+int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
+                     float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
+                     cudaStream_t st);
+int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, float* v,
+                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st);
+// One layer's LoRA operands rounded once into their product types: a list of
+// blocks, each an fp16 copy of an A matrix (kind 0: [rows][cols]) or a bf16
+// block-diagonal stack of a B matrix (kind 1: [rows][ld_out], rows split into
+// parts ending at part_end[], part p's rows holding B in columns [p cols,
+// (p + 1) cols)).  Offsets in elements within one layer's LoRA block / output.
+struct LoraPrepSeg {
+  int64_t src_off, dst_off, rows, cols, ld_out;
+  int kind, n_parts;
+  int64_t part_end[4];
+};
+struct LoraPrepSegs {
+  LoraPrepSeg seg[8];
+  int n;
+};
+// Converts n_layers LoRA blocks (stride lora_stride floats) into out (stride
+// out_stride elements per layer).
+int launch_lora_prepare(const float* lora, int64_t lora_stride, int n_layers, uint16_t* out,
+                        int64_t out_stride, const LoraPrepSegs& segs, cudaStream_t st);
 
 // attention (causal GQA), q/k/v read from the fused fp16 qkv buffer [T, (H + 2 Hkv) d];
 // o fp16 [T, H d]; dout bf16
@@ -219,13 +249,22 @@ int layer_shapes(const lsq_cfg* cfg, LayerShapes* out);
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);
 // dx_out_bf16 may be null (then converted internally).
 // rope_cs: the cos/sin table of launch_rope_table for this seq, or null (then the
-// layer builds it in its workspace)
+// layer builds it in its workspace); lora16: this layer's LoRA operands rounded by
+// prepare_lora16, or null (then the layer rounds its masters in its workspace)
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
-                   cudaStream_t st, const float2* rope_cs = nullptr);
+                   cudaStream_t st, const float2* rope_cs = nullptr,
+                   const uint16_t* lora16 = nullptr);
+// The LoRA operands of one layer in their product types (fp16 A, bf16 block-
+// diagonal B stacks): elements per layer, and the rounding of n_layers
+// consecutive LoRA blocks into out (that many elements apart).
+size_t lora16_elems_per_layer(const lsq_cfg* cfg);
+int prepare_lora16(const lsq_cfg* cfg, const float* lora, int n_layers, uint16_t* out,
+                   cudaStream_t st);
 int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate,
-                   void* ws, size_t ws_bytes, cudaStream_t st, const float2* rope_cs = nullptr);
+                   void* ws, size_t ws_bytes, cudaStream_t st, const float2* rope_cs = nullptr,
+                   const uint16_t* lora16 = nullptr);
 
 }  // namespace lsq

@@ -72,6 +72,8 @@ struct Views {  // pointers into one layer blob / one LoRA block
   const uint16_t* g1;
   const uint16_t* g2;
   const float *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_d, *B_d;
+  // the same operands rounded once into their product types (Lora16)
+  const uint16_t *A16_qkv, *A16_o, *A16_gu, *A16_d, *B16_qkv, *B16_o, *B16_gu, *B16_d;
   bool lora_on;  // false: adapter disabled, every LoRA branch removed
 };
 
@@ -132,6 +134,66 @@ void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) 
   R->floats_per_layer = f;
 }
 
+// One layer's LoRA operands in their product types, rounded once from the fp32
+// masters (per optimiser step in the stack): fp16 A_qkv [3r, D], A_o [r, H d],
+// A_gu [2r, D], A_down [r, F] for u = x A^T; bf16 block-diagonal B stacks for
+// v = dY B, one product per projection group: B_qkv -> [qkv rows, 3r],
+// B_o [D, r], B_gu -> [2F, 2r], B_down [D, r].  Offsets in elements, each block
+// 128-element (256-byte) aligned.
+struct Lora16 {
+  int64_t a[4], b[4], elems;
+};
+Lora16 lora16_layout(const LayerShapes& s) {
+  auto al = [](int64_t x) { return (x + 127) & ~int64_t(127); };
+  const int64_t r = s.r;
+  Lora16 o;
+  int64_t f = 0;
+  o.a[0] = f; f = al(f + 3 * r * s.D);
+  o.a[1] = f; f = al(f + r * s.qd);
+  o.a[2] = f; f = al(f + 2 * r * s.D);
+  o.a[3] = f; f = al(f + r * s.F);
+  o.b[0] = f; f = al(f + s.qkv_n * 3 * r);
+  o.b[1] = f; f = al(f + s.D * r);
+  o.b[2] = f; f = al(f + s.gu_n * 2 * r);
+  o.b[3] = f; f = al(f + s.D * r);
+  o.elems = f;
+  return o;
+}
+LoraPrepSegs lora16_segs(const LayerShapes& s, const lsq_lora_layout& R, const Lora16& o) {
+  LoraPrepSegs g{};
+  const int64_t r = s.r;
+  const int64_t arows[4] = {3 * r, r, 2 * r, r}, acols[4] = {s.D, s.qd, s.D, s.F};
+  const int64_t asrc[4] = {R.a_off[0], R.a_off[3], R.a_off[4], R.a_off[6]};
+  for (int i = 0; i < 4; ++i) {
+    LoraPrepSeg& e = g.seg[i];
+    e.kind = 0;
+    e.src_off = asrc[i];
+    e.dst_off = o.a[i];
+    e.rows = arows[i];
+    e.cols = acols[i];
+    e.ld_out = acols[i];
+    e.n_parts = 1;
+  }
+  const int64_t brows[4] = {s.qkv_n, s.D, s.gu_n, s.D};
+  const int64_t bsrc[4] = {R.b_off[0], R.b_off[3], R.b_off[4], R.b_off[6]};
+  const int bparts[4] = {3, 1, 2, 1};
+  const int64_t pe[4][3] = {{s.qd, s.qd + s.kvd, s.qkv_n}, {s.D, 0, 0}, {s.F, s.gu_n, 0},
+                            {s.D, 0, 0}};
+  for (int i = 0; i < 4; ++i) {
+    LoraPrepSeg& e = g.seg[4 + i];
+    e.kind = 1;
+    e.src_off = bsrc[i];
+    e.dst_off = o.b[i];
+    e.rows = brows[i];
+    e.cols = r;
+    e.ld_out = bparts[i] * r;
+    e.n_parts = bparts[i];
+    for (int p = 0; p < bparts[i]; ++p) e.part_end[p] = pe[i][p];
+  }
+  g.n = 8;
+  return g;
+}
+
 Views views(const LayerShapes& s, const void* blob, const float* lora) {
   lsq_layer_layout L;
   lsq_lora_layout R;
@@ -153,6 +215,7 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
   v.g2 = reinterpret_cast<const uint16_t*>(b + L.g2_off);
   v.lora_on = lora != nullptr;
   v.A_qkv = v.B_qkv = v.A_o = v.B_o = v.A_gu = v.B_gu = v.A_d = v.B_d = nullptr;
+  v.A16_qkv = v.A16_o = v.A16_gu = v.A16_d = v.B16_qkv = v.B16_o = v.B16_gu = v.B16_d = nullptr;
   if (v.lora_on) {
     v.A_qkv = lora + R.a_off[0];
     v.B_qkv = lora + R.b_off[0];
@@ -168,6 +231,9 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
 
 // Workspace carve-up (identical for the forward and the backward).
 struct Buffers {
+  uint16_t* lora16;                                  // this layer's Lora16 (when not given)
+  uint16_t *u16_qkv, *u16_o, *u16_gu, *u16_d;        // bf16 copies of u, for dB
+  uint16_t *v16_qkv, *v16_o, *v16_gu, *v16_d;        // bf16 copies of v, for dA
   float* h;                                          // fp32 residual stream after attention
   uint16_t *n1, *qkv, *ao, *n2, *gu, *m;             // fp16 forward activations
   uint16_t *dgu, *dqkv, *da, *dout_b, *dh_b;         // bf16 gradients
@@ -270,6 +336,15 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   x.dh_b = a.take<uint16_t>(T * s.D);
   x.rstd1 = a.take<float>(T);
   x.rstd2 = a.take<float>(T);
+  x.lora16 = a.take<uint16_t>(lora16_layout(s).elems);
+  x.u16_qkv = a.take<uint16_t>(T * 3 * r);
+  x.u16_o = a.take<uint16_t>(T * r);
+  x.u16_gu = a.take<uint16_t>(T * 2 * r);
+  x.u16_d = a.take<uint16_t>(T * r);
+  x.v16_qkv = a.take<uint16_t>(T * 3 * r);
+  x.v16_o = a.take<uint16_t>(T * r);
+  x.v16_gu = a.take<uint16_t>(T * 2 * r);
+  x.v16_d = a.take<uint16_t>(T * r);
   x.u_qkv = a.take<float>(T * 3 * r);
   x.u_o = a.take<float>(T * r);
   x.u_gu = a.take<float>(T * 2 * r);
@@ -318,6 +393,31 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   return a.used;
 }
 
+// Points v at this layer's LoRA operands in product types: the given lora16, or
+// (lora16 null) the masters rounded into the workspace first.
+int attach_lora16(const LayerShapes& s, const float* lora, const uint16_t* lora16,
+                  const Buffers& b, Views* v, cudaStream_t st) {
+  if (!v->lora_on) return LSQ_OK;
+  const Lora16 o = lora16_layout(s);
+  if (!lora16) {
+    lsq_layer_layout L;
+    lsq_lora_layout R;
+    fill_layout(s, &L, &R);
+    LSQ_TRY(launch_lora_prepare(lora, R.floats_per_layer, 1, b.lora16, o.elems,
+                                lora16_segs(s, R, o), st));
+    lora16 = b.lora16;
+  }
+  v->A16_qkv = lora16 + o.a[0];
+  v->A16_o = lora16 + o.a[1];
+  v->A16_gu = lora16 + o.a[2];
+  v->A16_d = lora16 + o.a[3];
+  v->B16_qkv = lora16 + o.b[0];
+  v->B16_o = lora16 + o.b[1];
+  v->B16_gu = lora16 + o.b[2];
+  v->B16_d = lora16 + o.b[3];
+  return LSQ_OK;
+}
+
 int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, const void* x,
                      int batch, int seq, const void* out, LayerShapes* s, const char* who,
                      bool lora_optional = false) {
@@ -340,23 +440,31 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
   const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
   const int64_t pe2[2] = {s.F, s.gu_n};
   LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, OUT_F16, b.rstd1, st));
-  if (v.lora_on) LSQ_TRY(launch_lora_down(b.n1, s.D, v.A_qkv, T, s.D, 3 * r, b.u_qkv, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on)
+    LSQ_TRY(launch_lora_down16(b.n1, s.D, v.A16_qkv, T, s.D, 3 * r, b.u_qkv, b.u16_qkv, b.lscratch,
+                               b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
                            3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
-  if (v.lora_on) LSQ_TRY(launch_lora_down(b.ao, s.qd, v.A_o, T, s.qd, r, b.u_o, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on)
+    LSQ_TRY(launch_lora_down16(b.ao, s.qd, v.A16_o, T, s.qd, r, b.u_o, b.u16_o, b.lscratch,
+                               b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
                            pe3, x, b.h, s.D),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, OUT_F16, b.rstd2, st));
-  if (v.lora_on) LSQ_TRY(launch_lora_down(b.n2, s.D, v.A_gu, T, s.D, 2 * r, b.u_gu, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on)
+    LSQ_TRY(launch_lora_down16(b.n2, s.D, v.A16_gu, T, s.D, 2 * r, b.u_gu, b.u16_gu, b.lscratch,
+                               b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
                            2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_swiglu_fwd(b.gu, T, s.F, b.m, st));
-  if (v.lora_on) LSQ_TRY(launch_lora_down(b.m, s.F, v.A_d, T, s.F, r, b.u_d, b.lscratch, b.lscratch_bytes, st));
+  if (v.lora_on)
+    LSQ_TRY(launch_lora_down16(b.m, s.F, v.A16_d, T, s.F, r, b.u_d, b.u16_d, b.lscratch,
+                               b.lscratch_bytes, st));
   if (x_out)
     LSQ_TRY(gemm_run(nf4_fwd(v.codes[6], v.absmax[6], s.D, s.F, b.m, T, v.B_d, r, s.s, b.u_d, r, 1,
                              pe3, b.h, x_out, s.D),
@@ -366,6 +474,24 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
 
 }  // namespace
 
+size_t lora16_elems_per_layer(const lsq_cfg* cfg) {
+  LayerShapes s;
+  if (layer_shapes(cfg, &s) != LSQ_OK) return 0;
+  return (size_t)lora16_layout(s).elems;
+}
+
+int prepare_lora16(const lsq_cfg* cfg, const float* lora, int n_layers, uint16_t* out,
+                   cudaStream_t st) {
+  LayerShapes s;
+  LSQ_TRY(layer_shapes(cfg, &s));
+  lsq_layer_layout L;
+  lsq_lora_layout R;
+  fill_layout(s, &L, &R);
+  const Lora16 o = lora16_layout(s);
+  return launch_lora_prepare(lora, R.floats_per_layer, n_layers, out, o.elems,
+                             lora16_segs(s, R, o), st);
+}
+
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
   LayerShapes s;
   if (layer_shapes(cfg, &s) != LSQ_OK || T <= 0) return 0;
@@ -374,7 +500,7 @@ size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
 
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
-                   cudaStream_t st, const float2* rope_cs) {
+                   cudaStream_t st, const float2* rope_cs, const uint16_t* lora16) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd",
                            true));
@@ -384,7 +510,8 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     return set_error(LSQ_ERR_WORKSPACE, "decoder_layer_fwd: workspace %zu < %zu", ws_bytes, need);
   Buffers b;
   plan_buffers(s, T, ws, &b);
-  const Views v = views(s, blob, lora);
+  Views v = views(s, blob, lora);
+  LSQ_TRY(attach_lora16(s, lora, lora16, b, &v, st));
   if (!rope_cs) {
     LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, b.rope_cs, st));
     rope_cs = b.rope_cs;
@@ -395,7 +522,8 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
 int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate, void* ws,
-                   size_t ws_bytes, cudaStream_t st, const float2* rope_cs) {
+                   size_t ws_bytes, cudaStream_t st, const float2* rope_cs,
+                   const uint16_t* lora16) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, dx_in, &s, "decoder_layer_bwd"));
   if (!dx_out || !lora_grad) return set_error(LSQ_ERR_INVALID, "decoder_layer_bwd: null pointer");
@@ -405,7 +533,8 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     return set_error(LSQ_ERR_WORKSPACE, "decoder_layer_bwd: workspace %zu < %zu", ws_bytes, need);
   Buffers b;
   plan_buffers(s, T, ws, &b);
-  const Views v = views(s, blob, lora);
+  Views v = views(s, blob, lora);
+  LSQ_TRY(attach_lora16(s, lora, lora16, b, &v, st));
   lsq_layer_layout LL;
   lsq_lora_layout RL;
   fill_layout(s, &LL, &RL);
@@ -436,39 +565,50 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     dout_b = b.dout_b;
   }
   // down projection
-  LSQ_TRY(launch_lora_vproj(dout_b, T, s.D, v.B_d, r, 1, pe1, b.v_d, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj16(dout_b, T, s.D, v.B16_d, r, b.v_d, b.v16_d, b.lscratch,
+                              b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.A_d, r, sc, b.v_d, b.dm, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_d, b.m, T, s.F, r, sc, accumulate, gA_d, b.lscratch, b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b(dout_b, b.u_d, T, s.D, r, r, 1, pe1, sc, accumulate, gB_d, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_a16(b.v16_d, b.m, T, s.F, r, sc, accumulate, gA_d, b.lscratch,
+                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b16(dout_b, b.u16_d, T, s.D, r, 1, pe1, sc, accumulate, gB_d, b.lscratch,
+                               b.lscratch_bytes, st));
   // SwiGLU and gate|up
   LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
-  LSQ_TRY(launch_lora_vproj(b.dgu, T, s.gu_n, v.B_gu, r, 2, pe2, b.v_gu, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj16(b.dgu, T, s.gu_n, v.B16_gu, 2 * r, b.v_gu, b.v16_gu, b.lscratch,
+                              b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc, b.v_gu,
                           b.dn2, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, b.lscratch, b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b(b.dgu, b.u_gu, T, s.gu_n, r, 2 * r, 2, pe2, sc, accumulate, gB_gu, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_a16(b.v16_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, b.lscratch,
+                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b16(b.dgu, b.u16_gu, T, s.gu_n, r, 2, pe2, sc, accumulate, gB_gu,
+                               b.lscratch, b.lscratch_bytes, st));
   // second RMSNorm + residual
   LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
   // o projection
-  LSQ_TRY(launch_lora_vproj(b.dh_b, T, s.D, v.B_o, r, 1, pe1, b.v_o, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj16(b.dh_b, T, s.D, v.B16_o, r, b.v_o, b.v16_o, b.lscratch,
+                              b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.A_o, r, sc, b.v_o, b.da, 0),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, b.lscratch, b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b(b.dh_b, b.u_o, T, s.D, r, r, 1, pe1, sc, accumulate, gB_o, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_a16(b.v16_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, b.lscratch,
+                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b16(b.dh_b, b.u16_o, T, s.D, r, 1, pe1, sc, accumulate, gB_o, b.lscratch,
+                               b.lscratch_bytes, st));
   // attention, RoPE
   LSQ_TRY(launch_attention_bwd(b.qkv, b.ao, b.da, b.lse, T, seq, s.H, s.Hkv, s.hd, b.delta, b.dq,
                                b.dk, b.dv, st));
   LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, rope_cs, b.dqkv, st));
   // q|k|v projections
-  LSQ_TRY(launch_lora_vproj(b.dqkv, T, s.qkv_n, v.B_qkv, r, 3, pe3, b.v_qkv, b.lscratch,
-                            b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj16(b.dqkv, T, s.qkv_n, v.B16_qkv, 3 * r, b.v_qkv, b.v16_qkv,
+                              b.lscratch, b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
                           b.v_qkv, b.dn1, 1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a(b.v_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, b.lscratch, b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b(b.dqkv, b.u_qkv, T, s.qkv_n, r, 3 * r, 3, pe3, sc, accumulate, gB_qkv, b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_a16(b.v16_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, b.lscratch,
+                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_b16(b.dqkv, b.u16_qkv, T, s.qkv_n, r, 3, pe3, sc, accumulate, gB_qkv,
+                               b.lscratch, b.lscratch_bytes, st));
   // first RMSNorm + residual
   LSQ_TRY(launch_rmsnorm_bwd(b.dn1, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16, st));
   return LSQ_OK;

@@ -49,7 +49,30 @@ struct SkinnyArgs {
   float alpha;
   int accumulate;
   int direct;
+  // Output options (applied where the result is written: the direct epilogue or
+  // the slice sum): c16 (nullable) also receives the result rounded to bf16,
+  // c16[m * c16_ld + n], for the product that consumes it; with part_r > 0 the
+  // rows are split into parts ending at part_end[], and row m of part p keeps
+  // only columns [p part_r, (p + 1) part_r), written to column n - p part_r.
+  uint16_t* c16;
+  int64_t c16_ld;
+  int part_r, n_parts;
+  int64_t part_end[4];
 };
+
+// Writes one result element of row m, column n (see SkinnyArgs); false if dropped.
+__device__ __forceinline__ void store_result(const SkinnyArgs& a, int64_t m, int64_t n, float v) {
+  int64_t col = n;
+  if (a.part_r > 0) {
+    int p = 0;
+    while (p + 1 < a.n_parts && m >= a.part_end[p]) ++p;
+    col = n - (int64_t)p * a.part_r;
+    if (col < 0 || col >= a.part_r) return;
+  }
+  float* d = a.dst + m * a.c_m + col * a.c_n;
+  *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
+  if (a.c16) a.c16[m * a.c16_ld + n] = float_to_bf16_bits(v);
+}
 
 __device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -107,6 +130,7 @@ struct Tile {
 template <bool P_RED, bool Q_RED, int BN, int PM>
 __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks))
     skinny_kernel(const SkinnyArgs a) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   using TL = Tile<P_RED, Q_RED, BN>;
   constexpr int S = TL::kStages, PE = TL::kPE, QE = TL::kQE;
   extern __shared__ __align__(16) uint16_t sk_smem[];
@@ -250,8 +274,7 @@ __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks)
           if (n + e >= a.N) continue;
           const float v = acc[mi][nj][2 * h + e];
           if (a.direct) {
-            float* d = a.dst + m * a.c_m + (n + e) * a.c_n;
-            *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
+            store_result(a, m, n + e, v);
           } else {
             a.part[((size_t)blockIdx.z * a.M + m) * a.N + n + e] = v;
           }
@@ -261,10 +284,10 @@ __global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks)
   }
 }
 
-// dst[m * c_m + n * c_n] = alpha * sum_z part[z][m][n] (+ dst if accumulate), z in order
-__global__ void split_sum_kernel(const float* __restrict__ part, int splits, int64_t M, int64_t N,
-                                 float alpha, int accumulate, float* __restrict__ dst, int64_t c_m,
-                                 int64_t c_n) {
+// sum_z part[z][m][n] in z order, written as SkinnyArgs a prescribes (store_result)
+__global__ void split_sum_kernel(const float* __restrict__ part, int splits, const SkinnyArgs a) {
+  const int64_t M = a.M, N = a.N;
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t n_el = M * N;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -272,9 +295,7 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
     // unrolled so that several slices' loads are in flight; the adds stay in z order
 #pragma unroll 8
     for (int z = 0; z < splits; ++z) s += part[(size_t)z * n_el + i];
-    const int64_t m = i / N, n = i % N;
-    float* d = dst + m * c_m + n * c_n;
-    *d = (accumulate ? *d : 0.f) + alpha * s;
+    store_result(a, i / N, i % N, s);
   }
 }
 
@@ -283,6 +304,7 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, int
 template <bool F16>
 __global__ void to_16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
                                   int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t n_el = rows * ld_out;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -358,25 +380,18 @@ int convert_rows(const float* in, int64_t rows, int64_t cols, int64_t ld_in, uin
   return LSQ_OK;
 }
 
-// C = P Q over K, then dst[m * c_m + n * c_n] = alpha * C (+ dst if accumulate).
-// scratch holds the bf16 Q (already written at its start) and, after q_bytes,
-// room for the partials when the product is split.
+// C = P Q over K, written as a prescribes (dst, alpha, accumulate, c16, parts);
+// scratch holds the fixed-order partials when the product is split.
 template <bool P_RED, bool Q_RED, int PM>
-int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float* dst,
-        int64_t c_m, int64_t c_n, float alpha, int accumulate, cudaStream_t st) {
+int run(SkinnyArgs a, float* scratch, size_t scratch_bytes, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return LSQ_OK;
   const int z = splits_for(a.M, a.N, a.K);
-  const size_t need = align256(q_bytes) + (z > 1 ? (size_t)z * a.M * a.N * sizeof(float) : 0);
-  if (scratch_bytes < need)
+  const size_t need = z > 1 ? (size_t)z * a.M * a.N * sizeof(float) : 0;
+  if (need && (!scratch || scratch_bytes < need))
     return set_error(LSQ_ERR_WORKSPACE, "lora product: scratch %zu < %zu", scratch_bytes, need);
   a.k_per_split = a.K > 0 ? ((a.K + z - 1) / z + kBK - 1) / kBK * kBK : kBK;
   a.direct = z == 1;
-  a.part = z > 1 ? reinterpret_cast<float*>(scratch + align256(q_bytes)) : nullptr;
-  a.dst = dst;
-  a.c_m = c_m;
-  a.c_n = c_n;
-  a.alpha = alpha;
-  a.accumulate = accumulate;
+  a.part = z > 1 ? scratch : nullptr;
   const int bn = bn_for(a.N);
   dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)z);
   switch (bn) {
@@ -387,8 +402,7 @@ int run(SkinnyArgs a, char* scratch, size_t q_bytes, size_t scratch_bytes, float
   if (z == 1) return LSQ_OK;
   int64_t g = (a.M * a.N + 255) / 256;
   if (g > kSMs * 8) g = kSMs * 8;
-  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, z, a.M, a.N, alpha, accumulate, dst, c_m,
-                                                c_n);
+  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, z, a);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -397,6 +411,39 @@ int check_ranks(int64_t R) {
   if (R < 1)
     return set_error(LSQ_ERR_SHAPE, "lora: rank-r products need at least one column (got %lld)",
                      (long long)R);
+  if (R % 8 != 0)
+    return set_error(LSQ_ERR_SHAPE, "lora: product widths must be multiples of 8 (got %lld)",
+                     (long long)R);
+  return LSQ_OK;
+}
+
+SkinnyArgs out_args(float* dst, int64_t c_m, int64_t c_n, float alpha, int accumulate,
+                    uint16_t* c16, int64_t c16_ld) {
+  SkinnyArgs a{};
+  a.dst = dst;
+  a.c_m = c_m;
+  a.c_n = c_n;
+  a.alpha = alpha;
+  a.accumulate = accumulate;
+  a.c16 = c16;
+  a.c16_ld = c16_ld;
+  return a;
+}
+
+// 16-bit copies of fp32 LoRA operands, at the start of the scratch; returns the
+// scratch left for the partials.
+struct Split {
+  uint16_t* q;
+  float* rest;
+  size_t rest_bytes;
+};
+int split_scratch(float* scratch, size_t bytes, size_t q_elems, Split* out, const char* who) {
+  const size_t qb = align256(q_elems * 2);
+  if (!scratch || bytes < qb)
+    return set_error(LSQ_ERR_WORKSPACE, "%s: scratch %zu < %zu", who, bytes, qb);
+  out->q = reinterpret_cast<uint16_t*>(scratch);
+  out->rest = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + qb);
+  out->rest_bytes = bytes - qb;
   return LSQ_OK;
 }
 
@@ -404,12 +451,12 @@ int check_ranks(int64_t R) {
 
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
   // An upper bound over every product a caller sizing by (T, K, R) can make:
-  // any rank r' <= R per part, a reduction or a part of up to K elements:
-  //   u = x A^T, v part   M = T, N = r', reduction <= K, Q = A [r'][K] or B [<= K][pad8(r')]
-  //   dA, dB part         M <= K, N = r', reduction T,   Q = v or u [T][pad8(r')]
-  // The first needs z(T, r', K) slices at most (splits grow with the reduction);
+  // any width R' <= R, a reduction or a part of up to K elements:
+  //   u = x A^T, v      M = T, N = R', reduction <= K, Q = A [R'][K] or B [<= K][R']
+  //   dA, dB            M <= K, N = R', reduction T,   Q = v or u [T][R']
+  // The first needs z(T, R', K) slices at most (splits grow with the reduction);
   // the second z * M <= min(64, T / (4 kBK)) K, and z * M <= slots * kBM as well,
-  // since z <= slots / (M / kBM tiles).
+  // since z <= slots / (M / kBM tiles).  The 16-bit copy of an fp32 operand comes first.
   size_t best = 0;
   for (int rr = 1; rr <= R; ++rr) {
     const int64_t q1 = K * pad8(rr);
@@ -425,104 +472,132 @@ size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
   return best;
 }
 
-int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
-                     float* u, float* scratch, size_t scratch_bytes, cudaStream_t st) {
-  LSQ_TRY(check_ranks(R));
-  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
-  // C[t, j] = sum_k x[t, k] A[j, k]
-  char* sc = reinterpret_cast<char*>(scratch);
-  uint16_t* Ab = reinterpret_cast<uint16_t*>(sc);
-  const size_t qb = (size_t)R * K * 2;
-  if (!scratch || scratch_bytes < qb)
-    return set_error(LSQ_ERR_WORKSPACE, "lora_down: scratch %zu < %zu", scratch_bytes, qb);
-  const int prof = prof_begin(st);
-  LSQ_TRY(convert_rows(A, R, K, K, Ab, K, st, /*f16=*/true));
-  SkinnyArgs a{};
-  a.P = x; a.p_m = ldx; a.p_k = 1;
-  a.Q = Ab; a.q_k = 1; a.q_n = K;
-  a.M = T; a.N = R; a.K = K;
-  LSQ_TRY((run<true, true, PM_F16>(a, sc, qb, scratch_bytes, u, R, 1, 1.f, 0, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 4.0 * R * K);
-  return LSQ_OK;
-}
-
-int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, int n_parts,
-                      const int64_t* part_end, float* v, float* scratch, size_t scratch_bytes,
-                      cudaStream_t st) {
-  LSQ_TRY(check_ranks(r));
-  const int R = n_parts * r;
-  const int64_t r8 = pad8(r);
-  char* sc = reinterpret_cast<char*>(scratch);
-  uint16_t* Bb = reinterpret_cast<uint16_t*>(sc);
-  int64_t start = 0;
-  for (int p = 0; p < n_parts; ++p) {
-    const int64_t Np = part_end[p] - start;
-    const size_t qb = (size_t)Np * r8 * 2;
-    if (!scratch || scratch_bytes < qb)
-      return set_error(LSQ_ERR_WORKSPACE, "lora_vproj: scratch %zu < %zu", scratch_bytes, qb);
-    // C[t, j] = sum_n dy[t, start + n] B[start + n, j]
-    const int prof = prof_begin(st);
-    LSQ_TRY(convert_rows(B + start * r, Np, r, r, Bb, r8, st));
-    SkinnyArgs a{};
-    a.P = dy + start; a.p_m = N; a.p_k = 1;
-    a.Q = Bb; a.q_k = r8; a.q_n = 1;
-    a.M = T; a.N = r; a.K = Np;
-    LSQ_TRY((run<true, false, PM_BF16>(a, sc, qb, scratch_bytes, v + p * r, R, 1, 1.f, 0, st)));
-    if (prof >= 0)
-      prof_end(prof, st, "lora_rank_r_v", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * r * Np);
-    start = part_end[p];
-  }
-  return LSQ_OK;
-}
-
-int launch_lora_grad_a(const float* v, const uint16_t* x, int64_t T, int64_t K, int R, float s,
-                       int accumulate, float* dA, float* scratch, size_t scratch_bytes,
+int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
+                       int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
                        cudaStream_t st) {
   LSQ_TRY(check_ranks(R));
-  // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]
-  const int64_t R8 = pad8(R);
-  const size_t qb = (size_t)T * R8 * 2;
-  if (!scratch || scratch_bytes < qb)
-    return set_error(LSQ_ERR_WORKSPACE, "lora_grad_a: scratch %zu < %zu", scratch_bytes, qb);
-  char* sc = reinterpret_cast<char*>(scratch);
-  uint16_t* vb = reinterpret_cast<uint16_t*>(sc);
+  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
+  // C[t, j] = sum_k x[t, k] A[j, k]   (fp16 operands)
   const int prof = prof_begin(st);
-  LSQ_TRY(convert_rows(v, T, R, R, vb, R8, st));
-  SkinnyArgs a{};
-  a.P = x; a.p_m = 1; a.p_k = K;
-  a.Q = vb; a.q_k = R8; a.q_n = 1;
-  a.M = K; a.N = R; a.K = T;
-  LSQ_TRY((run<false, false, PM_P16>(a, sc, qb, scratch_bytes, dA, 1, K, s, accumulate, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 4.0 * T * R);
+  SkinnyArgs a = out_args(u, R, 1, 1.f, 0, u16, R);
+  a.P = x; a.p_m = ldx; a.p_k = 1;
+  a.Q = A16; a.q_k = 1; a.q_n = K;
+  a.M = T; a.N = R; a.K = K;
+  LSQ_TRY((run<true, true, PM_F16>(a, scratch, scratch_bytes, st)));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 2.0 * R * K);
   return LSQ_OK;
 }
 
-int launch_lora_grad_b(const uint16_t* dy, const float* u, int64_t T, int64_t N, int r, int R,
-                       int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
-                       float* scratch, size_t scratch_bytes, cudaStream_t st) {
-  LSQ_TRY(check_ranks(r));
-  const int64_t r8 = pad8(r);
-  const size_t qb = (size_t)T * r8 * 2;
-  if (!scratch || scratch_bytes < qb)
-    return set_error(LSQ_ERR_WORKSPACE, "lora_grad_b: scratch %zu < %zu", scratch_bytes, qb);
-  char* sc = reinterpret_cast<char*>(scratch);
-  uint16_t* ub = reinterpret_cast<uint16_t*>(sc);
-  int64_t start = 0;
-  for (int p = 0; p < n_parts; ++p) {
-    const int64_t Np = part_end[p] - start;
-    // C[n, j] = sum_t dy[t, start + n] u[t, p r + j];  dB[start + n, j] (+)= s C[n, j]
-    const int prof = prof_begin(st);
-    LSQ_TRY(convert_rows(u + p * r, T, r, R, ub, r8, st));
-    SkinnyArgs a{};
-    a.P = dy + start; a.p_m = 1; a.p_k = N;
-    a.Q = ub; a.q_k = r8; a.q_n = 1;
-    a.M = Np; a.N = r; a.K = T;
-    LSQ_TRY((run<false, false, PM_BF16>(a, sc, qb, scratch_bytes, dB + start * r, r, 1, s,
-                                        accumulate, st)));
-    if (prof >= 0)
-      prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * r * Np, 2.0 * T * Np + 4.0 * T * r);
-    start = part_end[p];
+int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
+                        float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
+                        cudaStream_t st) {
+  LSQ_TRY(check_ranks(R));
+  // C[t, c] = sum_n dy[t, n] Bs[n, c]   (bf16 operands; Bs block-diagonal over the parts)
+  const int prof = prof_begin(st);
+  SkinnyArgs a = out_args(v, R, 1, 1.f, 0, v16, R);
+  a.P = dy; a.p_m = N; a.p_k = 1;
+  a.Q = Bs; a.q_k = R; a.q_n = 1;
+  a.M = T; a.N = R; a.K = N;
+  LSQ_TRY((run<true, false, PM_BF16>(a, scratch, scratch_bytes, st)));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_v", 2.0 * T * R * N, 2.0 * T * N + 2.0 * R * N);
+  return LSQ_OK;
+}
+
+int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
+                         float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
+                         cudaStream_t st) {
+  LSQ_TRY(check_ranks(R));
+  // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]   (x rounded from fp16 to bf16)
+  const int prof = prof_begin(st);
+  SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0);
+  a.P = x; a.p_m = 1; a.p_k = K;
+  a.Q = v16; a.q_k = R; a.q_n = 1;
+  a.M = K; a.N = R; a.K = T;
+  LSQ_TRY((run<false, false, PM_P16>(a, scratch, scratch_bytes, st)));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 2.0 * T * R);
+  return LSQ_OK;
+}
+
+int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
+                         int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
+                         float* scratch, size_t scratch_bytes, cudaStream_t st) {
+  const int R = n_parts * r;
+  LSQ_TRY(check_ranks(R));
+  if (n_parts < 1 || n_parts > 4) return set_error(LSQ_ERR_SHAPE, "lora_grad_b: 1..4 parts");
+  // C[n, c] = sum_t dy[t, n] u[t, c];  dB[n, j] (+)= s C[n, part(n) r + j]: one product over
+  // all parts, each row keeping its own part's columns
+  const int prof = prof_begin(st);
+  SkinnyArgs a = out_args(dB, r, 1, s, accumulate, nullptr, 0);
+  a.P = dy; a.p_m = 1; a.p_k = N;
+  a.Q = u16; a.q_k = R; a.q_n = 1;
+  a.M = N; a.N = R; a.K = T;
+  if (n_parts > 1) {
+    a.part_r = r;
+    a.n_parts = n_parts;
+    for (int p = 0; p < n_parts; ++p) a.part_end[p] = part_end[p];
   }
+  LSQ_TRY((run<false, false, PM_BF16>(a, scratch, scratch_bytes, st)));
+  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * R * N, 2.0 * T * N + 2.0 * T * R);
+  return LSQ_OK;
+}
+
+// fp32-operand forms (one part), used by the single-linear entry points: the LoRA
+// operand is rounded once into the start of the scratch, then the product runs.
+int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
+                     float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
+                     cudaStream_t st) {
+  LSQ_TRY(check_ranks(R));
+  Split sp;
+  LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)R * K, &sp, "lora_down"));
+  LSQ_TRY(convert_rows(A, R, K, K, sp.q, K, st, /*f16=*/true));
+  return launch_lora_down16(x, ldx, sp.q, T, K, R, u, u16, sp.rest, sp.rest_bytes, st);
+}
+
+int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, float* v,
+                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st) {
+  LSQ_TRY(check_ranks(r));
+  Split sp;
+  LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)N * r, &sp, "lora_vproj"));
+  LSQ_TRY(convert_rows(B, N, r, r, sp.q, r, st));
+  return launch_lora_vproj16(dy, T, N, sp.q, r, v, v16, sp.rest, sp.rest_bytes, st);
+}
+
+// One layer's LoRA operands in their product types (see internal.h).
+__global__ void lora_prepare_kernel(const float* __restrict__ lora, int64_t lora_stride,
+                                    uint16_t* __restrict__ out, int64_t out_stride,
+                                    const LoraPrepSegs segs) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
+  const int layer = blockIdx.y;
+  const float* src = lora + (int64_t)layer * lora_stride;
+  uint16_t* dst = out + (int64_t)layer * out_stride;
+  for (int b = 0; b < segs.n; ++b) {
+    const LoraPrepSeg& g = segs.seg[b];
+    const int64_t n_el = g.rows * g.ld_out;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
+         i += (int64_t)gridDim.x * blockDim.x) {
+      const int64_t row = i / g.ld_out, col = i % g.ld_out;
+      if (g.kind == 0) {  // A: fp16 copy, [rows][cols]
+        dst[g.dst_off + i] = float_to_f16_bits(src[g.src_off + row * g.cols + col]);
+      } else {            // B: bf16, block-diagonal [rows][n_parts r]
+        int p = 0;
+        while (p + 1 < g.n_parts && row >= g.part_end[p]) ++p;
+        const int64_t j = col - (int64_t)p * g.cols;
+        const float v = (j >= 0 && j < g.cols) ? src[g.src_off + row * g.cols + j] : 0.f;
+        dst[g.dst_off + i] = float_to_bf16_bits(v);
+      }
+    }
+  }
+}
+
+int launch_lora_prepare(const float* lora, int64_t lora_stride, int n_layers, uint16_t* out,
+                        int64_t out_stride, const LoraPrepSegs& segs, cudaStream_t st) {
+  if (n_layers <= 0) return LSQ_OK;
+  int64_t most = 0;
+  for (int b = 0; b < segs.n; ++b) most = std::max(most, segs.seg[b].rows * segs.seg[b].ld_out);
+  unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((most + 255) / 256, 64));
+  lora_prepare_kernel<<<dim3(gx, (unsigned)n_layers), 256, 0, st>>>(lora, lora_stride, out,
+                                                                    out_stride, segs);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
 

@@ -109,6 +109,7 @@ struct StackWs {
   float* loss_dev;   // [1]
   float* dhf;        // [T][D]
   float2* rope_cs;   // [seq][d/2] RoPE cos/sin table, built once per step
+  uint16_t* lora16;  // [L][lora16 elems] LoRA operands in product types, once per step
   float* dh[2];      // [T][D] fp32 residual-stream gradient (ping-pong)
   uint16_t* dhb[2];  // bf16 copies
   void* gemm;
@@ -178,6 +179,7 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.loss_dev = a.take<float>(64);
   x.dhf = a.take<float>(T * D);
   x.rope_cs = a.take<float2>(T * s.hd / 2);  // >= seq * d/2 entries
+  x.lora16 = a.take<uint16_t>((size_t)cfg->n_layers * lora16_elems_per_layer(cfg));
   for (int i = 0; i < 2; ++i) {
     x.dh[i] = a.take<float>(T * D);
     x.dhb[i] = a.take<uint16_t>(T * D);
@@ -632,6 +634,10 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
 
   LSQ_CUDA(cudaEventRecord(h->t_start, cs));
   LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, w.rope_cs, cs));
+  // the LoRA masters in their product types, for every layer (they change only at
+  // the optimiser step, after the last visit)
+  LSQ_TRY(prepare_lora16(cfg, lora, L, w.lora16, cs));
+  const size_t l16 = lora16_elems_per_layer(cfg);
   // Sharded: the step's first all-gather waits for everything the caller put on
   // the compute stream before the step (e.g. a gradient all-reduce on another
   // communicator), so that collectives of the two never run interleaved.
@@ -649,7 +655,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
       LSQ_TRY(visit(std::make_tuple(0, i, b, 0, mbk), [&](cudaStream_t s) {
         return layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
                               w.xs + (size_t)i * T * D, batch, seq, w.xs + (size_t)(i + 1) * T * D,
-                              w.layer_ws, w.layer_ws_bytes, s, w.rope_cs);
+                              w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16);
       }));
       if (dpo)  // reference model: the same layer with its adapter off
         LSQ_TRY(visit(std::make_tuple(1, i, b, 0, mbk), [&](cudaStream_t s) {
@@ -689,7 +695,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
         return layer_bwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
                               w.xs + (size_t)i * T * D, w.dh[cur], w.dhb[cur], batch, seq,
                               w.dh[1 - cur], w.dhb[1 - cur], lora_grad + (int64_t)i * layer_floats,
-                              acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs);
+                              acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16);
       }));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
       cur = 1 - cur;
