@@ -594,7 +594,9 @@ int launch_lora_prepare(const float* lora, int64_t lora_stride, int n_layers, ui
   if (n_layers <= 0) return LSQ_OK;
   int64_t most = 0;
   for (int b = 0; b < segs.n; ++b) most = std::max(most, segs.seg[b].rows * segs.seg[b].ld_out);
-  unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((most + 255) / 256, 64));
+  // about 32 resident CTAs' worth of threads per SM over all layers
+  const int64_t cap = std::max<int64_t>(1, (int64_t)kSMs * 32 / n_layers);
+  unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((most + 255) / 256, cap));
   lora_prepare_kernel<<<dim3(gx, (unsigned)n_layers), 256, 0, st>>>(lora, lora_stride, out,
                                                                     out_stride, segs);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
