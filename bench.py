@@ -332,6 +332,8 @@ def run_ours(args):
     handle = L.StreamStack(cfg, st["host_blobs"], st["bufs"][0], st["bufs"][1], False)
     if args.shard_layers:
         dp.shard_stack(L, handle, buf_bytes)
+    if world > 1:   # the LoRA-gradient average, per layer inside the step (NCCL)
+        dp.reduce_grads_stack(L, handle)
     ws_bytes = (L.stream_stack_dpo_workspace_bytes(cfg, args.pairs, SEQ) if dpo
                 else L.stream_stack_workspace_bytes(cfg, batch, SEQ))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -344,7 +346,7 @@ def run_ours(args):
     cur = dict(h=handle)              # the stack the steps run on
 
     def step(tokens):
-        o = opt if world == 1 else None
+        o = opt
         h = cur["h"]
         if dpo:
             loss, _ = L.stream_stack_dpo_step(h, tokens, args.pairs, SEQ, 0.1, st["emb"],
@@ -352,9 +354,6 @@ def run_ours(args):
         else:
             loss = L.stream_stack_step(h, tokens, mbs, batch, SEQ, st["emb"], st["head"],
                                        st["gf"], lora, grad, o, ws)
-        if world > 1:
-            dp.average_(grad)                       # NCCL all-reduce of the LoRA gradients
-            L.lora_adamw_step(lora, grad, opt)
         opt["step"] += 1
         return loss
 
@@ -416,6 +415,8 @@ def run_ours(args):
                                           profile=True, label="timed_kernels_streamed")
     res_blobs = [hb.cuda() for hb in st["host_blobs"]]
     res_handle = L.StreamStack(cfg, res_blobs, None, None, True)
+    if world > 1:
+        dp.reduce_grads_stack(L, res_handle)
     cur["h"] = res_handle
     step(pool[0])                                  # captures the resident graphs
     torch.cuda.synchronize()

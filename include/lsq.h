@@ -402,6 +402,27 @@ int lsq_nccl_unique_id(void* id_out, int64_t id_bytes);
 int stream_stack_shard(lsq_stack* stack, const void* nccl_id, int64_t id_bytes, int32_t world,
                        int32_t rank, int64_t buf_bytes);
 
+/* stream_stack_reduce_grads - data-parallel gradient averaging inside the step.
+ * With world ranks each streaming the same frozen stack on its own tokens (one
+ * process per GPU), the only exchange the method needs is the mean of the LoRA
+ * gradients before the optimiser.  After this call every later step of the stack
+ * does it itself: as soon as the backward of layer i has finished (in the step's
+ * last micro-batch), that layer's gradient block (lsq_lora_layout
+ * floats_per_layer floats) is all-reduced in place with NCCL's average on the
+ * stack's own reduction stream and communicator, so the exchange overlaps the
+ * backward of layers i-1..0; the step's AdamW (opt) waits for the last one and
+ * then applies the same update on every rank.  loss_out stays this rank's own
+ * loss.  The pages run one GPU; this is the library's data-parallel form.
+ *   nccl_id  LSQ_NCCL_ID_BYTES from lsq_nccl_unique_id, the same on every rank
+ *            (not the id given to stream_stack_shard: this is a second communicator).
+ *   world, rank  this rank among world (world 1 is allowed: the average is a copy).
+ * Collective and blocking like stream_stack_shard; every rank must then run the
+ * same steps.  A step that times out aborts this communicator too.  Errors:
+ * LSQ_ERR_INVALID (null, wrong id size, already set up, bad rank, wrong device),
+ * LSQ_ERR_CUDA (NCCL). */
+int stream_stack_reduce_grads(lsq_stack* stack, const void* nccl_id, int64_t id_bytes,
+                              int32_t world, int32_t rank);
+
 /* ------------------------------------------------------------ optimiser */
 
 /* lora_adamw_step - one AdamW update of n LoRA parameters (fp32, any layout

@@ -72,6 +72,12 @@ struct lsq_stack {
   size_t shard = 0;            // bytes of a layer each rank fetches from host
   void* comm = nullptr;        // ncclComm_t
   int aborted = 0;             // the communicator was aborted after a timeout
+  // data-parallel gradient averaging (stream_stack_reduce_grads): its own
+  // communicator and stream, so the per-layer all-reduces overlap the backward
+  void* grad_comm = nullptr;   // ncclComm_t
+  int grad_world = 1;
+  cudaStream_t red_stream = nullptr;
+  cudaEvent_t red_ev = nullptr, red_done = nullptr;
   // CUDA graphs of the layer visits, keyed by (kind: 0 forward, 1 adapter-off
   // reference forward, 2 backward; layer; buffer; accumulate; micro-batch when
   // profiling), valid while the step's pointers and sizes (graph_sig) are unchanged
@@ -240,6 +246,7 @@ struct NcclFns {
   decltype(&ncclGetUniqueId) get_unique_id = nullptr;
   decltype(&ncclCommInitRank) init_rank = nullptr;
   decltype(&ncclAllGather) all_gather = nullptr;
+  decltype(&ncclAllReduce) all_reduce = nullptr;
   decltype(&ncclCommDestroy) destroy = nullptr;
   decltype(&ncclCommAbort) abort = nullptr;
   decltype(&ncclGetErrorString) error_string = nullptr;
@@ -257,11 +264,12 @@ int nccl_fns(const NcclFns** out) {
       f.get_unique_id = reinterpret_cast<decltype(f.get_unique_id)>(dlsym(lib, "ncclGetUniqueId"));
       f.init_rank = reinterpret_cast<decltype(f.init_rank)>(dlsym(lib, "ncclCommInitRank"));
       f.all_gather = reinterpret_cast<decltype(f.all_gather)>(dlsym(lib, "ncclAllGather"));
+      f.all_reduce = reinterpret_cast<decltype(f.all_reduce)>(dlsym(lib, "ncclAllReduce"));
       f.destroy = reinterpret_cast<decltype(f.destroy)>(dlsym(lib, "ncclCommDestroy"));
       f.abort = reinterpret_cast<decltype(f.abort)>(dlsym(lib, "ncclCommAbort"));
       f.error_string =
           reinterpret_cast<decltype(f.error_string)>(dlsym(lib, "ncclGetErrorString"));
-      if (f.get_unique_id && f.init_rank && f.all_gather && f.destroy && f.abort &&
+      if (f.get_unique_id && f.init_rank && f.all_gather && f.all_reduce && f.destroy && f.abort &&
           f.error_string)
         state = 1;
     }
@@ -296,12 +304,16 @@ int shard_fetch(lsq_stack* h, int b, int layer, size_t bytes) {
   return LSQ_OK;
 }
 
-// After a step timed out: abort the communicator, which ends any all-gather
-// still waiting for a peer, and refuse further steps on this stack.
+// After a step timed out: abort the communicators, which ends any all-gather
+// or all-reduce still waiting for a peer, and refuse further steps on this stack.
 void shard_abort(lsq_stack* h) {
   const NcclFns* f = nullptr;
-  if (h->comm && nccl_fns(&f) == LSQ_OK) f->abort(static_cast<ncclComm_t>(h->comm));
+  if (nccl_fns(&f) == LSQ_OK) {
+    if (h->comm) f->abort(static_cast<ncclComm_t>(h->comm));
+    if (h->grad_comm) f->abort(static_cast<ncclComm_t>(h->grad_comm));
+  }
   h->comm = nullptr;
+  h->grad_comm = nullptr;
   h->aborted = 1;
 }
 
@@ -416,6 +428,13 @@ extern "C" int stream_stack_destroy(lsq_stack* h) {
   cudaFreeHost(h->loss_host);
   const NcclFns* f = nullptr;
   if (h->comm && nccl_fns(&f) == LSQ_OK) f->destroy(static_cast<ncclComm_t>(h->comm));
+  if (h->grad_comm && nccl_fns(&f) == LSQ_OK) f->destroy(static_cast<ncclComm_t>(h->grad_comm));
+  if (h->red_stream) {
+    cudaStreamSynchronize(h->red_stream);
+    cudaStreamDestroy(h->red_stream);
+  }
+  if (h->red_ev) cudaEventDestroy(h->red_ev);
+  if (h->red_done) cudaEventDestroy(h->red_done);
   delete h;
   return LSQ_OK;
 }
@@ -501,6 +520,43 @@ extern "C" int stream_stack_shard(lsq_stack* h, const void* nccl_id, int64_t id_
   h->world = world;
   h->rank = rank;
   h->shard = (size_t)S;
+  return LSQ_OK;
+}
+
+extern "C" int stream_stack_reduce_grads(lsq_stack* h, const void* nccl_id, int64_t id_bytes,
+                                         int32_t world, int32_t rank) {
+  if (!h || !nccl_id) return set_error(LSQ_ERR_INVALID, "stream_stack_reduce_grads: null pointer");
+  if (id_bytes != (int64_t)sizeof(ncclUniqueId))
+    return set_error(LSQ_ERR_INVALID, "stream_stack_reduce_grads: the id has %d bytes",
+                     (int)sizeof(ncclUniqueId));
+  if (h->grad_comm || h->aborted)
+    return set_error(LSQ_ERR_INVALID,
+                     "stream_stack_reduce_grads: gradients are already reduced, or the stack's "
+                     "communicators were aborted");
+  if (world < 1 || rank < 0 || rank >= world)
+    return set_error(LSQ_ERR_INVALID, "stream_stack_reduce_grads: rank %d of world %d", rank,
+                     world);
+  int dev = -1;
+  LSQ_CUDA(cudaGetDevice(&dev));
+  if (dev != h->device)
+    return set_error(LSQ_ERR_INVALID,
+                     "stream_stack_reduce_grads: call on the stack's device (%d, not %d)",
+                     h->device, dev);
+  const NcclFns* f = nullptr;
+  LSQ_TRY(nccl_fns(&f));
+  if (!h->red_stream) {
+    LSQ_CUDA(cudaStreamCreateWithFlags(&h->red_stream, cudaStreamNonBlocking));
+    LSQ_CUDA(cudaEventCreateWithFlags(&h->red_ev, cudaEventDisableTiming));
+    LSQ_CUDA(cudaEventCreateWithFlags(&h->red_done, cudaEventDisableTiming));
+  }
+  ncclUniqueId id;
+  memcpy(&id, nccl_id, sizeof(id));
+  ncclComm_t comm = nullptr;
+  const ncclResult_t r = f->init_rank(&comm, world, id, rank);
+  if (r != ncclSuccess)
+    return set_error(LSQ_ERR_CUDA, "ncclCommInitRank: %s", f->error_string(r));
+  h->grad_comm = comm;
+  h->grad_world = world;
   return LSQ_OK;
 }
 
@@ -698,8 +754,25 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
                               acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16);
       }));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
+      if (h->grad_comm && mb == micro_batches - 1) {
+        // layer i's gradient is final: average it over the ranks on the reduction
+        // stream while the backward of layer i - 1 runs
+        const NcclFns* f = nullptr;
+        LSQ_TRY(nccl_fns(&f));
+        LSQ_CUDA(cudaEventRecord(h->red_ev, cs));
+        LSQ_CUDA(cudaStreamWaitEvent(h->red_stream, h->red_ev, 0));
+        float* g = lora_grad + (int64_t)i * layer_floats;
+        const ncclResult_t r = f->all_reduce(g, g, (size_t)layer_floats, ncclFloat, ncclAvg,
+                                             static_cast<ncclComm_t>(h->grad_comm), h->red_stream);
+        if (r != ncclSuccess)
+          return set_error(LSQ_ERR_CUDA, "ncclAllReduce: %s", f->error_string(r));
+      }
       cur = 1 - cur;
     }
+  }
+  if (h->grad_comm) {  // the optimiser (and the step's end) waits for the last all-reduce
+    LSQ_CUDA(cudaEventRecord(h->red_done, h->red_stream));
+    LSQ_CUDA(cudaStreamWaitEvent(cs, h->red_done, 0));
   }
   if (logits_out)
     LSQ_CUDA(cudaMemcpyAsync(logits_out, w.logits, (size_t)T * V * sizeof(float),
@@ -716,7 +789,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   {
     const int rc = wait_event_timeout(h->done, timeout_ms);
     if (rc != LSQ_OK) {
-      if (rc == LSQ_ERR_TIMEOUT && h->comm) shard_abort(h);
+      if (rc == LSQ_ERR_TIMEOUT && (h->comm || h->grad_comm)) shard_abort(h);
       return rc;
     }
   }

@@ -1,8 +1,10 @@
 """Data-parallel plumbing for running N replicas of the streamed step (one
-process per GPU, torch.distributed).  Each rank streams its own copy of the
-frozen stack on its own micro-batch; the only exchange is the average of the
-LoRA gradients before the (identical) AdamW update on every rank.  Timing is
-the maximum over ranks.  NCCL on GPUs; the same code runs on gloo for tests.
+process per GPU, torch.distributed for the process group and host-side
+exchanges).  Each rank streams its own copy of the frozen stack on its own
+micro-batch; the only exchange is the average of the LoRA gradients before the
+(identical) AdamW update on every rank, which the library performs inside the
+step (stream_stack_reduce_grads; average_ is the same mean written with
+torch.distributed, used by the CPU tests).  Timing is the maximum over ranks.
 """
 import datetime
 import os
@@ -62,6 +64,14 @@ def broadcast_bytes(make, src=0):
     if multi:
         dist.broadcast_object_list(obj, src=src)
     return obj[0]
+
+
+def reduce_grads_stack(L, stack):
+    """stream_stack_reduce_grads over this job's ranks: every later step of the stack
+    averages its LoRA gradients over the ranks itself, layer by layer, overlapping
+    the backward, before its optimiser update."""
+    rank, world = ((dist.get_rank(), dist.get_world_size()) if dist.is_initialized() else (0, 1))
+    stack.reduce_grads(broadcast_bytes(L.lsq_nccl_unique_id), world, rank)
 
 
 def shard_stack(L, stack, buf_bytes):

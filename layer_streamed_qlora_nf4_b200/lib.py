@@ -27,6 +27,7 @@ EXPORTS = (
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
     "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
     "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard", "lsq_stream_plan",
+    "stream_stack_reduce_grads",
 )
 LSQ_NCCL_ID_BYTES = 128
 
@@ -123,6 +124,7 @@ _PROTOS = {
                                        ctypes.POINTER(ctypes.c_int32)]),
     "lsq_nccl_unique_id": (ctypes.c_int, [_P, _I64]),
     "stream_stack_shard": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64]),
+    "stream_stack_reduce_grads": (ctypes.c_int, [_P, _P, _I64, _I32, _I32]),
     "lsq_launch_counter": (ctypes.c_int64, []),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
                                                    _F, _P, _P, _I32, _P, _P]),
@@ -307,6 +309,10 @@ class StreamStack:
         """stream_stack_shard: spread every layer copy over `world` ranks."""
         stream_stack_shard(self, nccl_id, world, rank, buf_bytes)
 
+    def reduce_grads(self, nccl_id, world, rank):
+        """stream_stack_reduce_grads: average the LoRA gradients over `world` ranks in each step."""
+        stream_stack_reduce_grads(self, nccl_id, world, rank)
+
     def close(self):
         if self.handle:
             _check(load().stream_stack_destroy(self.handle))
@@ -347,6 +353,15 @@ def stream_stack_shard(stack, nccl_id, world, rank, buf_bytes):
     buf = ctypes.create_string_buffer(nccl_id, LSQ_NCCL_ID_BYTES)
     _check(load().stream_stack_shard(stack.handle, buf, LSQ_NCCL_ID_BYTES, int(world), int(rank),
                                      int(buf_bytes)))
+
+
+def stream_stack_reduce_grads(stack, nccl_id, world, rank):
+    nccl_id = bytes(nccl_id)
+    if len(nccl_id) != LSQ_NCCL_ID_BYTES:
+        raise ValueError("the NCCL id has %d bytes" % LSQ_NCCL_ID_BYTES)
+    buf = ctypes.create_string_buffer(nccl_id, LSQ_NCCL_ID_BYTES)
+    _check(load().stream_stack_reduce_grads(stack.handle, buf, LSQ_NCCL_ID_BYTES, int(world),
+                                            int(rank)))
 
 
 def stream_stack_workspace_bytes(cfg, batch, seq):

@@ -3,6 +3,10 @@
 A streamed stack sharded over a one-rank NCCL communicator (the layer slice is
 the whole layer, the in-place all-gather a local no-op) must give the same step,
 bit for bit, as the unsharded stack; stream_stack_shard's argument checks hold.
+Likewise a stack whose steps average the LoRA gradients over a one-rank
+communicator (stream_stack_reduce_grads: per-layer all-reduces on their own
+stream, the optimiser waiting for them) must give the same gradients and the
+same AdamW update, bit for bit, as one without.
 """
 import os
 import sys
@@ -59,6 +63,25 @@ def main():
     assert torch.equal(grad1, grad0) and torch.equal(grad2, grad0)
     assert s1["layer_copies"] == s0["layer_copies"]
     assert s1["h2d_bytes"] == s0["h2d_bytes"] == s0["layer_copies"] * st.blob_bytes
+
+    # gradient averaging inside the step, one rank, with the optimiser update
+    def opt_state():
+        return dict(lr=2e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, step=1,
+                    m=torch.zeros_like(st.lora), v=torch.zeros_like(st.lora))
+    tok2 = synth.tokens(34, 2 * batch, seq, st.cfg["vocab"]).reshape(2, batch, seq)
+    h2 = st.handle(L, resident=False)
+    la, lg_a, ga, pa = _step(L, st, h2, tok2, 2, batch, seq, opt=opt_state())
+    h2.close()
+    h3 = st.handle(L, resident=False)
+    gid = L.lsq_nccl_unique_id()
+    _expect(lambda: h3.reduce_grads(gid, 1, 1), L.LSQ_ERR_INVALID)
+    _expect(lambda: h3.reduce_grads(gid, 0, 0), L.LSQ_ERR_INVALID)
+    h3.reduce_grads(gid, 1, 0)
+    _expect(lambda: h3.reduce_grads(gid, 1, 0), L.LSQ_ERR_INVALID)   # already set up
+    lb, lg_b, gb, pb = _step(L, st, h3, tok2, 2, batch, seq, opt=opt_state())
+    h3.close()
+    assert la == lb and torch.equal(lg_a, lg_b)
+    assert torch.equal(ga, gb) and torch.equal(pa, pb)
     assert L.lsq_device_status() == 0
     print("shard ok")
 

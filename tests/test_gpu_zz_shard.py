@@ -1,7 +1,8 @@
-"""Data-parallel layer sharding on the GPU, with the one GPU a test box has: a
-one-rank NCCL communicator drives the sharded copy path (slice copy, in-place
-all-gather on the copy stream, ready event) and the step must equal the
-unsharded one bit for bit.  Several ranks whose all-gathers wait on one another
+"""Data-parallel layer sharding and gradient averaging on the GPU, with the one
+GPU a test box has: one-rank NCCL communicators drive the sharded copy path
+(slice copy, in-place all-gather on the copy stream, ready event) and the
+per-layer gradient all-reduce (reduction stream, the optimiser waiting for it),
+and each step must equal the plain one bit for bit.  Several ranks whose all-gathers wait on one another
 are never run on one GPU; the slice plan for G ranks is checked with gloo ranks
 on the CPU (test_dist_gloo.py).  Runs in a fresh process, bounded by a timeout,
 so that NCCL's set-up stays out of the rest of the suite."""
