@@ -352,6 +352,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Each thread of the warp writes 16 consecutive 32-bit columns of its TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // Shared-memory matrix descriptor for a K-major operand tile stored in the
 // 128-byte-swizzle canonical layout: rows of 64 bf16 (128 B), 8-row groups
@@ -363,6 +375,20 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t saddr) {
   d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset: 8 rows x 128 B
   d |= (uint64_t)1 << 46;                         // descriptor version for sm_100
   d |= (uint64_t)2 << 61;                         // layout: 128-byte swizzle
+  return d;
+}
+// Shared-memory matrix descriptor for an MN-major operand in the 128-byte-swizzle
+// canonical layout: each 128-B row holds 64 consecutive MN elements of one K
+// index, 8-row groups along K are `sbo` bytes apart, and 64-element groups along
+// MN are `lbo` bytes apart; tile base 1024-B aligned.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t lbo,
+                                                       uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
   return d;
 }
 // Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, M x N.
@@ -385,5 +411,11 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
   return row * 128u + (((chunk ^ (row & 7u)) & 7u) << 4);
 }
+
+// 2-D tensor map (defined with the GEMM): `rows` rows of `inner` elements,
+// `row_stride_elems` apart, copied in boxes of box_rows x box_inner.
+int make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
+                 uint64_t inner, uint64_t rows, uint64_t row_stride_elems, uint32_t box_inner,
+                 uint32_t box_rows, CUtensorMapSwizzle sw);
 
 }  // namespace lsq

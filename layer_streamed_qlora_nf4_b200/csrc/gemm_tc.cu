@@ -923,6 +923,12 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
 
 }  // namespace
 
+int make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base,
+                 uint64_t inner, uint64_t rows, uint64_t row_stride_elems, uint32_t box_inner,
+                 uint32_t box_rows, CUtensorMapSwizzle sw) {
+  return make_tmap(m, dt, elem_bytes, base, inner, rows, row_stride_elems, box_inner, box_rows, sw);
+}
+
 int gemm_num_sms() {
   if (g_num_sms == 0) {
     int dev = 0, n = 0;
