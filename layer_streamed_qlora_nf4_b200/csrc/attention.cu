@@ -3,19 +3,19 @@
 // "維護者的 4GB／8B 成績"): o = softmax(q k^T / sqrt(d), causal) v, with query
 // head h reading kv head h / (H / Hkv), positions restarting at 0 per sequence.
 //
-// Forward: 5th-generation tensor cores (tcgen05.mma, accumulators in TMEM, TMA
-// tiles of 128 queries x 128 keys), see attn_fwd_tc_kernel.  Backward: tiles of
-// 64 queries x 64 keys, 4 warps x 16 rows, m16n8k16 tensor-core MMAs with fp32
-// accumulation.  Both use an online (running max / running sum) softmax in the
-// exp2 domain.  Precision: q, k, v and o are fp16 (the forward activations);
-// the forward and the recomputed scores use fp16 products, with the
-// probabilities rounded to fp16 for P V.  The backward's products with a
-// gradient operand (dO, dS) are bf16: the fp16 q, k, v fragments are rounded to
-// bf16 as they are loaded into registers, and P and dS are rounded to bf16.  The
-// forward saves the row log-sum-exp.  The backward recomputes the probabilities
-// from it and is split into a dK/dV kernel (one CTA per key block and kv head,
-// summing over that head's query heads in a fixed order) and a dQ kernel, so no
+// All products run on 5th-generation tensor cores: tcgen05.mma from
+// 128-byte-swizzled shared-memory tiles (loaded by TMA) into TMEM accumulators.
+// The forward (attn_fwd_tc_kernel) keeps an online (running max / running sum)
+// softmax in the exp2 domain and saves the row log-sum-exp.  The backward
+// recomputes the probabilities from it in two kernels: dK/dV (one CTA per key
+// block and query head; the kv-head sums of the query heads' dk, dv are taken
+// later in a fixed order) and dQ (one CTA per query block and head), so no
 // output is accumulated with atomics and every result is deterministic.
+// Precision: q, k, v and o are fp16 (the forward activations); the forward and
+// the recomputed scores use fp16 products, with the probabilities rounded to
+// fp16 for P V.  The backward's products with a gradient operand (dO, dS) are
+// bf16: v and the q (dK) or k (dQ) tiles they meet are converted to bf16 in
+// shared memory, and P and dS are rounded to bf16.
 #include <cuda.h>
 #include <math.h>
 
@@ -24,93 +24,6 @@
 namespace lsq {
 
 namespace {
-
-constexpr int kTile = 64;
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// fp16 fragment registers -> bf16 (each fp16 value rounded to bf16)
-template <int N>
-__device__ __forceinline__ void to_bf16(uint32_t (&r)[N]) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) r[i] = f16x2_to_bf16x2(r[i]);
-}
-
-// Copy `rows` rows (of `D` bf16 each, global row stride ld) into smem rows of
-// stride D+8, zero-filling rows >= valid.
-template <int D>
-__device__ __forceinline__ void load_tile(uint16_t* sm, const uint16_t* g, int64_t ld, int valid) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int i = threadIdx.x; i < kTile * CH; i += blockDim.x) {
-    const int r = i / CH, c = i % CH;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < valid) v = *reinterpret_cast<const uint4*>(g + (int64_t)r * ld + c * 8);
-    *reinterpret_cast<uint4*>(sm + r * (D + 8) + c * 8) = v;
-  }
-}
-
-// The same with cp.async (16-byte chunks, zero-filled rows >= valid): the copy
-// completes at the caller's cp.async wait, so it can overlap the previous tile's math.
-template <int D>
-__device__ __forceinline__ void load_tile_async(uint16_t* sm, const uint16_t* g, int64_t ld,
-                                                int valid) {
-  constexpr int CH = D / 8;
-  for (int i = threadIdx.x; i < kTile * CH; i += blockDim.x) {
-    const int r = i / CH, c = i % CH;
-    const bool in = r < valid;
-    const uint16_t* src = g + (in ? (int64_t)r * ld + c * 8 : 0);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sm + r * (D + 8) + c * 8)),
-                 "l"(src), "r"(in ? 16u : 0u)
-                 : "memory");
-  }
-}
-
-// A-operand fragment (16 rows x 16 cols) of a row-major smem tile: rows r0..r0+15, cols c0..
-template <int D>
-__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const uint16_t* sm, int r0, int c0) {
-  const int lane = threadIdx.x & 31;
-  ldsm_x4(a, smem_u32(sm + (r0 + (lane & 15)) * (D + 8) + c0 + 8 * (lane >> 4)));
-}
-// B fragments of two n8 tiles where the smem tile rows are the N index and the
-// columns the K index (e.g. keys x dims for S = Q K^T): b[0],b[1] -> n rows
-// n0..n0+7, b[2],b[3] -> n0+8..n0+15, k cols k0..k0+15.
-template <int D>
-__device__ __forceinline__ void frag_b_nk(uint32_t (&b)[4], const uint16_t* sm, int n0, int k0) {
-  const int lane = threadIdx.x & 31;
-  ldsm_x4(b, smem_u32(sm + (n0 + (lane & 7) + 8 * (lane >> 4)) * (D + 8) + k0 + 8 * ((lane >> 3) & 1)));
-}
-// B fragments of two n8 tiles where the smem tile rows are the K index and the
-// columns the N index (e.g. keys x dims for O = P V): k rows k0..k0+15,
-// b[0],b[1] -> n cols n0..n0+7, b[2],b[3] -> n0+8..n0+15.
-template <int D>
-__device__ __forceinline__ void frag_b_kn(uint32_t (&b)[4], const uint16_t* sm, int k0, int n0) {
-  const int lane = threadIdx.x & 31;
-  ldsm_x4_t(b, smem_u32(sm + (k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D + 8) + n0 + 8 * (lane >> 4)));
-}
 
 // ------------------------------------------------------------------ forward on tcgen05
 // One CTA per (128 queries of one sequence, query head).  Q and the K/V tiles of
@@ -458,282 +371,537 @@ __global__ void attn_delta_kernel(const uint16_t* __restrict__ o, const uint16_t
 
 // dK, dV contributions of one query head for one key block (written per query
 // head; the sum over a kv head's query heads happens later, in a fixed order).
-template <int D>
-__global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(
-    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ dout,
-    const float* __restrict__ lse, const float* __restrict__ delta, int64_t T, int seq, int H,
-    int Hkv, float sl2, float scale, float* __restrict__ dk, float* __restrict__ dv) {
-  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  extern __shared__ __align__(16) uint16_t smem_attn[];
-  uint16_t* Ks = smem_attn;
-  uint16_t* Vs = Ks + kTile * (D + 8);
-  uint16_t* Qb = Vs + kTile * (D + 8);       // [2] Q tiles
-  uint16_t* dOb = Qb + 2 * kTile * (D + 8);  // [2] dO tiles
-  float* lse_b = reinterpret_cast<float*>(dOb + 2 * kTile * (D + 8));  // [2][kTile]
-  float* del_b = lse_b + 2 * kTile;                                      // [2][kTile]
-  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (H / Hkv);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int64_t ld = (int64_t)(H + 2 * Hkv) * D;
-  const int64_t ldo = (int64_t)H * D;
-  const int64_t tok0 = (int64_t)b * seq;
-  const int k0 = kb * kTile;
-  load_tile<D>(Ks, qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D, ld, min(kTile, seq - k0));
-  load_tile<D>(Vs, qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
-  float dkacc[D / 8][4], dvacc[D / 8][4];
-#pragma unroll
-  for (int j = 0; j < D / 8; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dkacc[j][e] = dvacc[j][e] = 0.f;
-  const int krow[2] = {k0 + warp * 16 + gid, k0 + warp * 16 + gid + 8};
-  const int nqb = (seq + kTile - 1) / kTile;
-  // the Q / dO tiles (and their lse, delta rows) of query block qb go to buffer
-  // (qb - kb) & 1, one block ahead of the math
-  auto load_q = [&](int qb) {
-    const int q0 = qb * kTile, sl = (qb - kb) & 1;
-    load_tile_async<D>(Qb + sl * kTile * (D + 8), qkv + (tok0 + q0) * ld + (int64_t)h * D, ld,
-                       min(kTile, seq - q0));
-    load_tile_async<D>(dOb + sl * kTile * (D + 8), dout + (tok0 + q0) * ldo + (int64_t)h * D, ldo,
-                       min(kTile, seq - q0));
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int i = threadIdx.x; i < kTile; i += blockDim.x) {
-      const bool ok = q0 + i < seq;
-      lse_b[sl * kTile + i] = ok ? lse[(int64_t)h * T + tok0 + q0 + i] * 1.4426950408889634f : 0.f;
-      del_b[sl * kTile + i] = ok ? delta[(int64_t)h * T + tok0 + q0 + i] : 0.f;
-    }
-  };
-  load_q(kb);
-  {
-    for (int qb = kb; qb < nqb; ++qb) {
-      const int q0 = qb * kTile;
-      if (qb + 1 < nqb) {
-        load_q(qb + 1);  // its buffers were last read before the previous iteration's end barrier
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      }
-      __syncthreads();  // block qb (and K, V) visible to every warp
-      const int sl = (qb - kb) & 1;
-      const uint16_t* Qs = Qb + sl * kTile * (D + 8);
-      const uint16_t* dOs = dOb + sl * kTile * (D + 8);
-      const float* lse_s = lse_b + sl * kTile;
-      const float* del_s = del_b + sl * kTile;
-      // S^T = K Q^T  (16 keys of this warp x 64 queries)
-      float st[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) st[j][0] = st[j][1] = st[j][2] = st[j][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4];
-        frag_a<D>(a, Ks, warp * 16, kk * 16);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t bb[4];
-          frag_b_nk<D>(bb, Qs, j * 16, kk * 16);
-          mma16816_f16(st[2 * j], a, bb[0], bb[1]);
-          mma16816_f16(st[2 * j + 1], a, bb[2], bb[3]);
-        }
-      }
-      // P^T
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qi = 8 * j + 2 * tig + (e & 1);
-          const int q = q0 + qi;
-          const int kr = krow[e >> 1];
-          st[j][e] = (q < kr || q >= seq || kr >= seq) ? 0.f : exp2f(st[j][e] * sl2 - lse_s[qi]);
-        }
-      // dV += P^T dO
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t a[4] = {pack_bf16x2(st[2 * i][0], st[2 * i][1]),
-                               pack_bf16x2(st[2 * i][2], st[2 * i][3]),
-                               pack_bf16x2(st[2 * i + 1][0], st[2 * i + 1][1]),
-                               pack_bf16x2(st[2 * i + 1][2], st[2 * i + 1][3])};
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          uint32_t bb[4];
-          frag_b_kn<D>(bb, dOs, i * 16, j * 16);
-          mma16816(dvacc[2 * j], a, bb[0], bb[1]);
-          mma16816(dvacc[2 * j + 1], a, bb[2], bb[3]);
-        }
-      }
-      // dP^T = V dO^T
-      float dp[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dp[j][0] = dp[j][1] = dp[j][2] = dp[j][3] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t a[4];
-        frag_a<D>(a, Vs, warp * 16, kk * 16);
-        to_bf16(a);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t bb[4];
-          frag_b_nk<D>(bb, dOs, j * 16, kk * 16);
-          mma16816(dp[2 * j], a, bb[0], bb[1]);
-          mma16816(dp[2 * j + 1], a, bb[2], bb[3]);
-        }
-      }
-      // dS^T = P^T (dP^T - delta), then dK += dS^T Q
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qi = 8 * j + 2 * tig + (e & 1);
-          st[j][e] = st[j][e] * (dp[j][e] - del_s[qi]);
-        }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t a[4] = {pack_bf16x2(st[2 * i][0], st[2 * i][1]),
-                               pack_bf16x2(st[2 * i][2], st[2 * i][3]),
-                               pack_bf16x2(st[2 * i + 1][0], st[2 * i + 1][1]),
-                               pack_bf16x2(st[2 * i + 1][2], st[2 * i + 1][3])};
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j) {
-          uint32_t bb[4];
-          frag_b_kn<D>(bb, Qs, i * 16, j * 16);
-          to_bf16(bb);
-          mma16816(dkacc[2 * j], a, bb[0], bb[1]);
-          mma16816(dkacc[2 * j + 1], a, bb[2], bb[3]);
-        }
-      }
-      __syncthreads();  // every warp is done with buffer (qb - kb) & 1 before it is refilled
-    }
-  }
-#pragma unroll
-  for (int rI = 0; rI < 2; ++rI) {
-    const int kr = krow[rI];
-    if (kr >= seq) continue;
-    float* dkr = dk + (tok0 + kr) * (int64_t)H * D + (int64_t)h * D;
-    float* dvr = dv + (tok0 + kr) * (int64_t)H * D + (int64_t)h * D;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      const int col = 8 * j + 2 * tig;
-      *reinterpret_cast<float2*>(dkr + col) =
-          make_float2(dkacc[j][2 * rI] * scale, dkacc[j][2 * rI + 1] * scale);
-      *reinterpret_cast<float2*>(dvr + col) = make_float2(dvacc[j][2 * rI], dvacc[j][2 * rI + 1]);
-    }
+// ------------------------------------------------------------------ backward on tcgen05
+// Both kernels recompute the probabilities from the forward's log-sum-exp,
+// p = exp2(s sl2 - lse log2 e), and form ds = p (dp - delta) with
+// delta = rowsum(dO o O).  Products with a gradient operand are bf16: V, and the
+// copies of Q (dK kernel) or K (dQ kernel) that meet dS, are converted from fp16
+// to bf16 in place in shared memory once their fp16 use is over.  P and dS are
+// rounded to bf16.
+//   warps 0-7: the gradient warps (row = TMEM lane, warp / 4 = which half of the
+//              64 columns of a chunk), then the epilogue
+//   warp 8   : TMA producer;  warp 9: TMEM allocation and the MMA issuer
+constexpr int kBC = 64;  // columns of a chunk (queries for dK/dV, keys for dQ)
+
+// fp16 -> bf16 (nearest even) of a tile in place, 16-byte chunks over the 256 gradient threads
+__device__ __forceinline__ void tile_f16_to_bf16(uint8_t* tile, uint32_t bytes, int tid) {
+  for (uint32_t o = (uint32_t)tid * 16u; o < bytes; o += 256u * 16u) {
+    uint4 v = *reinterpret_cast<uint4*>(tile + o);
+    v.x = f16x2_to_bf16x2(v.x);
+    v.y = f16x2_to_bf16x2(v.y);
+    v.z = f16x2_to_bf16x2(v.z);
+    v.w = f16x2_to_bf16x2(v.w);
+    *reinterpret_cast<uint4*>(tile + o) = v;
   }
 }
 
-// dQ for one query block of one query head.
 template <int D>
-__global__ void __launch_bounds__(128) attn_bwd_dq_kernel(
-    const uint16_t* __restrict__ qkv, const uint16_t* __restrict__ dout,
-    const float* __restrict__ lse, const float* __restrict__ delta, int64_t T, int seq, int H,
-    int Hkv, float sl2, float scale, float* __restrict__ dq) {
-  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  extern __shared__ __align__(16) uint16_t smem_attn[];
-  uint16_t* Qs = smem_attn;
-  uint16_t* dOs = Qs + kTile * (D + 8);
-  uint16_t* Kb = dOs + kTile * (D + 8);     // [2] K tiles
-  uint16_t* Vb = Kb + 2 * kTile * (D + 8);  // [2] V tiles
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (H / Hkv);
+struct DkvSmem {
+  static constexpr uint32_t kKV = kAK * D * 2;   // K (fp16) or V (bf16): 128 keys
+  static constexpr uint32_t kQc = kBC * D * 2;   // a chunk of Q or dO: 64 queries
+  static constexpr uint32_t kPc = kAK * kBC * 2; // P^T or dS^T: 128 keys x 64 queries
+  static constexpr uint32_t kBytes = 1024 + 2 * kKV + 4 * kQc + 2 * kPc;
+};
+
+// dK, dV of 128 keys for one query head: loops over the 64-query chunks at and
+// after the key block (causal), accumulating dV += P^T dO and dK += dS^T Q in
+// TMEM; writes dk = scale dK and dv per query head.
+template <int D>
+__global__ void __launch_bounds__(kAThreads, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,   // qkv, boxes of 128 rows
+                            const __grid_constant__ CUtensorMap tm_q,    // qkv, boxes of 64 rows
+                            const __grid_constant__ CUtensorMap tm_do,   // dO, boxes of 64 rows
+                            const float* __restrict__ lse, const float* __restrict__ delta,
+                            int64_t T, int seq, int H, int Hkv, float sl2, float scale,
+                            float* __restrict__ dk, float* __restrict__ dv, int* __restrict__ dev_err) {
+  using SM = DkvSmem<D>;
+  constexpr int DA = D / 64;
+  extern __shared__ uint8_t dkv_raw[];
+  __shared__ __align__(8) uint64_t bar_kv, bar_vconv, bar_q[2], bar_qfree[2], bar_sdp[2],
+      bar_tfree[2], bar_ds, bar_pds;
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  pdl_trigger();
+
+  uint8_t* Ks = align1024_a(dkv_raw);
+  uint8_t* Vs = Ks + SM::kKV;
+  uint8_t* Qb = Vs + SM::kKV;       // [2] Q chunks (fp16, then bf16)
+  uint8_t* dOb = Qb + 2 * SM::kQc;  // [2] dO chunks (bf16)
+  uint8_t* Pt = dOb + 2 * SM::kQc;  // P^T (bf16, K-major over queries)
+  uint8_t* dSt = Pt + SM::kPc;      // dS^T
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int64_t ld = (int64_t)(H + 2 * Hkv) * D;
-  const int64_t ldo = (int64_t)H * D;
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (H / Hkv);
+  const int k0 = kb * kAK;
   const int64_t tok0 = (int64_t)b * seq;
-  const int q0 = qb * kTile;
-  load_tile<D>(Qs, qkv + (tok0 + q0) * ld + (int64_t)h * D, ld, min(kTile, seq - q0));
-  load_tile<D>(dOs, dout + (tok0 + q0) * ldo + (int64_t)h * D, ldo, min(kTile, seq - q0));
-  const int qrow[2] = {q0 + warp * 16 + gid, q0 + warp * 16 + gid + 8};
-  float lse2[2], del[2];
-#pragma unroll
-  for (int rI = 0; rI < 2; ++rI) {
-    const bool ok = qrow[rI] < seq;
-    lse2[rI] = ok ? lse[(int64_t)h * T + tok0 + qrow[rI]] * 1.4426950408889634f : 0.f;
-    del[rI] = ok ? delta[(int64_t)h * T + tok0 + qrow[rI]] : 0.f;
+  const int nc = (seq - k0 + kBC - 1) / kBC;  // query chunks from k0 on
+  constexpr uint32_t kColS = 0, kColP = 2 * kBC, kColV = 4 * kBC, kColK = 4 * kBC + 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar_kv), 1);
+    mbar_init(smem_u32(&bar_vconv), 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_q[i]), 1);
+      mbar_init(smem_u32(&bar_qfree[i]), 1);
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_tfree[i]), 8);
+    }
+    mbar_init(smem_u32(&bar_ds), 8);
+    mbar_init(smem_u32(&bar_pds), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
   }
-  float dqacc[D / 8][4];
-#pragma unroll
-  for (int j = 0; j < D / 8; ++j) dqacc[j][0] = dqacc[j][1] = dqacc[j][2] = dqacc[j][3] = 0.f;
-  // K/V tile kb goes to buffer kb & 1, one tile ahead of the math
-  auto load_kv = [&](int kb) {
-    const int k0 = kb * kTile;
-    load_tile_async<D>(Kb + (kb & 1) * kTile * (D + 8), qkv + (tok0 + k0) * ld + (int64_t)(H + g) * D,
-                       ld, min(kTile, seq - k0));
-    load_tile_async<D>(Vb + (kb & 1) * kTile * (D + 8),
-                       qkv + (tok0 + k0) * ld + (int64_t)(H + Hkv + g) * D, ld, min(kTile, seq - k0));
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  load_kv(0);
-  for (int kb = 0; kb <= qb; ++kb) {
-    const int k0 = kb * kTile;
-    if (kb < qb) {
-      load_kv(kb + 1);  // its buffer was last read before the previous iteration's end barrier
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();  // tile kb (and Q, dO) visible to every warp
-    const uint16_t* Ks = Kb + (kb & 1) * kTile * (D + 8);
-    const uint16_t* Vs = Vb + (kb & 1) * kTile * (D + 8);
-    float s[8][4], dp[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[j][e] = dp[j][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t a[4], ad[4];
-      frag_a<D>(a, Qs, warp * 16, kk * 16);
-      frag_a<D>(ad, dOs, warp * 16, kk * 16);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t bb[4], bv[4];
-        frag_b_nk<D>(bb, Ks, j * 16, kk * 16);
-        frag_b_nk<D>(bv, Vs, j * 16, kk * 16);
-        to_bf16(bv);
-        mma16816_f16(s[2 * j], a, bb[0], bb[1]);
-        mma16816_f16(s[2 * j + 1], a, bb[2], bb[3]);
-        mma16816(dp[2 * j], ad, bv[0], bv[1]);
-        mma16816(dp[2 * j + 1], ad, bv[2], bv[3]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = k0 + 8 * j + 2 * tig + (e & 1);
-        const int qr = qrow[e >> 1];
-        const float p = (key > qr || key >= seq || qr >= seq)
-                            ? 0.f
-                            : exp2f(s[j][e] * sl2 - lse2[e >> 1]);
-        s[j][e] = p * (dp[j][e] - del[e >> 1]);
-      }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t a[4] = {pack_bf16x2(s[2 * i][0], s[2 * i][1]),
-                             pack_bf16x2(s[2 * i][2], s[2 * i][3]),
-                             pack_bf16x2(s[2 * i + 1][0], s[2 * i + 1][1]),
-                             pack_bf16x2(s[2 * i + 1][2], s[2 * i + 1][3])};
-#pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        uint32_t bb[4];
-        frag_b_kn<D>(bb, Ks, i * 16, j * 16);
-        to_bf16(bb);
-        mma16816(dqacc[2 * j], a, bb[0], bb[1]);
-        mma16816(dqacc[2 * j + 1], a, bb[2], bb[3]);
-      }
-    }
-    __syncthreads();  // every warp is done with buffer kb & 1 before it is refilled
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(&tmem_sh), 512);
+    tmem_relinquish();
   }
-#pragma unroll
-  for (int rI = 0; rI < 2; ++rI) {
-    const int qr = qrow[rI];
-    if (qr >= seq) continue;
-    float* dqr = dq + (tok0 + qr) * (int64_t)H * D + (int64_t)h * D;
-#pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      const int col = 8 * j + 2 * tig;
-      *reinterpret_cast<float2*>(dqr + col) =
-          make_float2(dqacc[j][2 * rI] * scale, dqacc[j][2 * rI + 1] * scale);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      pdl_wait();
+      mbar_arrive_expect_tx(smem_u32(&bar_kv), 2 * SM::kKV);
+      for (int a = 0; a < DA; ++a) {
+        tma_load_2d(smem_u32(Ks + a * kAK * 128), &tm_kv, smem_u32(&bar_kv), (H + g) * D + 64 * a,
+                    (int)(tok0 + k0));
+        tma_load_2d(smem_u32(Vs + a * kAK * 128), &tm_kv, smem_u32(&bar_kv),
+                    (H + Hkv + g) * D + 64 * a, (int)(tok0 + k0));
+      }
+      for (int c = 0; c < nc; ++c) {
+        const int qb = c & 1;
+        if (c >= 2 && !mbar_wait_bounded(smem_u32(&bar_qfree[qb]), (uint32_t)(((c - 2) >> 1) & 1),
+                                         abort_flag, dev_err, DEV_ERR_WAIT_GEMM))
+          break;
+        const int row = (int)(tok0 + k0 + c * kBC);
+        const uint32_t fb = smem_u32(&bar_q[qb]);
+        mbar_arrive_expect_tx(fb, 2 * SM::kQc);
+        for (int a = 0; a < DA; ++a) {
+          tma_load_2d(smem_u32(Qb + qb * SM::kQc + a * kBC * 128), &tm_q, fb, h * D + 64 * a, row);
+          tma_load_2d(smem_u32(dOb + qb * SM::kQc + a * kBC * 128), &tm_do, fb, h * D + 64 * a, row);
+        }
+      }
     }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      const uint32_t id_s = umma_idesc_f16(kAK, kBC);            // S^T = K Q^T (fp16)
+      const uint32_t id_dp = umma_idesc_bf16(kAK, kBC);          // dP^T = V dO^T (bf16)
+      const uint32_t id_acc = umma_idesc_bf16(kAK, D) | (1u << 16);  // dV, dK: B MN-major
+      bool ok = mbar_wait_bounded(smem_u32(&bar_kv), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM) &&
+                mbar_wait_bounded(smem_u32(&bar_vconv), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
+      auto issue_sdp = [&](int c) -> bool {
+        const int qb = c & 1;
+        if (!mbar_wait_bounded(smem_u32(&bar_q[qb]), (uint32_t)((c >> 1) & 1), abort_flag, dev_err,
+                               DEV_ERR_WAIT_GEMM))
+          return false;
+        if (c >= 2 && !mbar_wait_bounded(smem_u32(&bar_tfree[qb]), (uint32_t)(((c - 2) >> 1) & 1),
+                                         abort_flag, dev_err, DEV_ERR_WAIT_GEMM))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (uint32_t)((kk >> 2) * kAK * 128 + (kk & 3) * 32);
+          const uint32_t kq = (uint32_t)((kk >> 2) * kBC * 128 + (kk & 3) * 32);
+          tc_mma_bf16(tmem + kColS + (uint32_t)qb * kBC, umma_desc_k_sw128(smem_u32(Ks) + ka),
+                      umma_desc_k_sw128(smem_u32(Qb + qb * SM::kQc) + kq), id_s, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + kColP + (uint32_t)qb * kBC, umma_desc_k_sw128(smem_u32(Vs) + ka),
+                      umma_desc_k_sw128(smem_u32(dOb + qb * SM::kQc) + kq), id_dp, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&bar_sdp[qb]));
+        return true;
+      };
+      ok = ok && issue_sdp(0);
+      for (int c = 0; c < nc && ok; ++c) {
+        const int qb = c & 1;
+        if (c + 1 < nc) ok = issue_sdp(c + 1);
+        if (!ok) break;
+        ok = mbar_wait_bounded(smem_u32(&bar_ds), (uint32_t)(c & 1), abort_flag, dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBC / 16; ++kk) {
+          const uint32_t pa = (uint32_t)(kk * 32);
+          const uint32_t bo = (uint32_t)kk * 16 * 128;
+          const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_bf16(tmem + kColV, umma_desc_k_sw128(smem_u32(Pt) + pa),
+                      umma_desc_mn_sw128(smem_u32(dOb + qb * SM::kQc) + bo, kBC * 128, 1024u), id_acc,
+                      acc);
+          tc_mma_bf16(tmem + kColK, umma_desc_k_sw128(smem_u32(dSt) + pa),
+                      umma_desc_mn_sw128(smem_u32(Qb + qb * SM::kQc) + bo, kBC * 128, 1024u), id_acc,
+                      acc);
+        }
+        tc_commit(smem_u32(&bar_pds));       // P^T, dS^T read; dK, dV updated
+        tc_commit(smem_u32(&bar_qfree[qb]));  // the Q and dO chunk read
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- gradient warps
+    const int tid = threadIdx.x;               // 0..255
+    const int r = (warp & 3) * 32 + lane;      // key row of the block = TMEM lane
+    const int hf = warp >> 2;                  // queries 32 hf .. of each chunk
+    const int kpos = k0 + r;
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    pdl_wait();  // delta comes from the kernel before
+    bool ok = mbar_wait_bounded(smem_u32(&bar_kv), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (ok) {
+      tile_f16_to_bf16(Vs, SM::kKV, tid);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_vconv));
+    }
+    for (int c = 0; c < nc && ok; ++c) {
+      const int qb = c & 1;
+      const int q0 = k0 + c * kBC + 32 * hf;  // this thread's first query
+      float l2[32], dl[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int qq = min(q0 + e, seq - 1);
+        l2[e] = __ldg(lse + (int64_t)h * T + tok0 + qq) * 1.4426950408889634f;
+        dl[e] = __ldg(delta + (int64_t)h * T + tok0 + qq);
+      }
+      ok = mbar_wait_bounded(smem_u32(&bar_sdp[qb]), (uint32_t)((c >> 1) & 1), abort_flag, dev_err,
+                             DEV_ERR_WAIT_GEMM);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[2][16], pv[2][16];
+      tmem_ld16(trow + kColS + (uint32_t)(qb * kBC + 32 * hf), sv[0]);
+      tmem_ld16(trow + kColS + (uint32_t)(qb * kBC + 32 * hf + 16), sv[1]);
+      tmem_ld16(trow + kColP + (uint32_t)(qb * kBC + 32 * hf), pv[0]);
+      tmem_ld16(trow + kColP + (uint32_t)(qb * kBC + 32 * hf + 16), pv[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_tfree[qb]));
+      uint32_t ppk[16], dpk[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        float p[2], d[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int qq = q0 + e + u;
+          const bool live = kpos <= qq && qq < seq && kpos < seq;
+          const float s = __uint_as_float(sv[(e + u) >> 4][(e + u) & 15]);
+          const float dp = __uint_as_float(pv[(e + u) >> 4][(e + u) & 15]);
+          p[u] = live ? exp2f(fmaf(s, sl2, -l2[e + u])) : 0.f;
+          d[u] = p[u] * (dp - dl[e + u]);
+        }
+        ppk[e >> 1] = pack_bf16x2(p[0], p[1]);
+        dpk[e >> 1] = pack_bf16x2(d[0], d[1]);
+      }
+      // the previous chunk's dV, dK products have read P^T and dS^T
+      if (c > 0) {
+        ok = mbar_wait_bounded(smem_u32(&bar_pds), (uint32_t)((c - 1) & 1), abort_flag, dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(hf * 4 + cc));
+        *reinterpret_cast<uint4*>(Pt + off) =
+            make_uint4(ppk[4 * cc], ppk[4 * cc + 1], ppk[4 * cc + 2], ppk[4 * cc + 3]);
+        *reinterpret_cast<uint4*>(dSt + off) =
+            make_uint4(dpk[4 * cc], dpk[4 * cc + 1], dpk[4 * cc + 2], dpk[4 * cc + 3]);
+      }
+      // S^T of this chunk is done with Q: Q becomes dK's bf16 operand
+      tile_f16_to_bf16(Qb + qb * SM::kQc, SM::kQc, tid);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_ds));
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok) ok = mbar_wait_bounded(smem_u32(&bar_pds), (uint32_t)((nc - 1) & 1), abort_flag,
+                                   dev_err, DEV_ERR_WAIT_GEMM);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool live = kpos < seq;
+      const int64_t o = (tok0 + kpos) * (int64_t)H * D + (int64_t)h * D + hf * (D / 2);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t kv[16], vv[16];
+        tmem_ld16(trow + kColK + (uint32_t)(hf * (D / 2) + 16 * c), kv);
+        tmem_ld16(trow + kColV + (uint32_t)(hf * (D / 2) + 16 * c), vv);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            *reinterpret_cast<float4*>(dk + o + 16 * c + e) =
+                make_float4(__uint_as_float(kv[e]) * scale, __uint_as_float(kv[e + 1]) * scale,
+                            __uint_as_float(kv[e + 2]) * scale, __uint_as_float(kv[e + 3]) * scale);
+            *reinterpret_cast<float4*>(dv + o + 16 * c + e) =
+                make_float4(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]),
+                            __uint_as_float(vv[e + 2]), __uint_as_float(vv[e + 3]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_sh) settle_ns(2000000);
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+struct DqSmem {
+  static constexpr uint32_t kQ = kAQ * D * 2;    // Q (fp16) or dO (bf16): 128 queries
+  static constexpr uint32_t kKc = kBC * D * 2;   // a chunk of K or V: 64 keys
+  static constexpr uint32_t kSc = kAQ * kBC * 2; // dS: 128 queries x 64 keys
+  static constexpr uint32_t kBytes = 1024 + 2 * kQ + 4 * kKc + kSc;
+};
+
+// dQ of 128 queries for one query head: loops over the 64-key chunks up to the
+// queries (causal), accumulating dQ += dS K in TMEM; writes dq = scale dQ.
+template <int D>
+__global__ void __launch_bounds__(kAThreads, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q,    // qkv, boxes of 128 rows
+                          const __grid_constant__ CUtensorMap tm_kv,   // qkv, boxes of 64 rows
+                          const __grid_constant__ CUtensorMap tm_do,   // dO, boxes of 128 rows
+                          const float* __restrict__ lse, const float* __restrict__ delta,
+                          int64_t T, int seq, int H, int Hkv, float sl2, float scale,
+                          float* __restrict__ dq, int* __restrict__ dev_err) {
+  using SM = DqSmem<D>;
+  constexpr int DA = D / 64;
+  extern __shared__ uint8_t dq_raw[];
+  __shared__ __align__(8) uint64_t bar_qd, bar_kv[2], bar_vconv[2], bar_kvfree[2], bar_sdp[2],
+      bar_tfree[2], bar_ds, bar_dsfree;
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  pdl_trigger();
+
+  uint8_t* Qs = align1024_a(dq_raw);
+  uint8_t* dOs = Qs + SM::kQ;
+  uint8_t* Kb = dOs + SM::kQ;       // [2] K chunks (fp16, then bf16)
+  uint8_t* Vb = Kb + 2 * SM::kKc;   // [2] V chunks (bf16)
+  uint8_t* dSs = Vb + 2 * SM::kKc;  // dS (bf16, K-major over keys)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qbk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (H / Hkv);
+  const int q0 = qbk * kAQ;
+  const int64_t tok0 = (int64_t)b * seq;
+  const int nc = (min(seq, q0 + kAQ) + kBC - 1) / kBC;  // key chunks up to the block's last query
+  constexpr uint32_t kColS = 0, kColP = 2 * kBC, kColQ = 4 * kBC;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar_qd), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_kv[i]), 1);
+      mbar_init(smem_u32(&bar_vconv[i]), 8);
+      mbar_init(smem_u32(&bar_kvfree[i]), 1);
+      mbar_init(smem_u32(&bar_sdp[i]), 1);
+      mbar_init(smem_u32(&bar_tfree[i]), 8);
+    }
+    mbar_init(smem_u32(&bar_ds), 8);
+    mbar_init(smem_u32(&bar_dsfree), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(&tmem_sh), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+
+  if (warp == kWarpTma) {
+    if (lane == 0) {
+      pdl_wait();
+      mbar_arrive_expect_tx(smem_u32(&bar_qd), 2 * SM::kQ);
+      for (int a = 0; a < DA; ++a) {
+        tma_load_2d(smem_u32(Qs + a * kAQ * 128), &tm_q, smem_u32(&bar_qd), h * D + 64 * a,
+                    (int)(tok0 + q0));
+        tma_load_2d(smem_u32(dOs + a * kAQ * 128), &tm_do, smem_u32(&bar_qd), h * D + 64 * a,
+                    (int)(tok0 + q0));
+      }
+      for (int c = 0; c < nc; ++c) {
+        const int kb = c & 1;
+        if (c >= 2 && !mbar_wait_bounded(smem_u32(&bar_kvfree[kb]), (uint32_t)(((c - 2) >> 1) & 1),
+                                         abort_flag, dev_err, DEV_ERR_WAIT_GEMM))
+          break;
+        const int row = (int)(tok0 + c * kBC);
+        const uint32_t fb = smem_u32(&bar_kv[kb]);
+        mbar_arrive_expect_tx(fb, 2 * SM::kKc);
+        for (int a = 0; a < DA; ++a) {
+          tma_load_2d(smem_u32(Kb + kb * SM::kKc + a * kBC * 128), &tm_kv, fb, (H + g) * D + 64 * a,
+                      row);
+          tma_load_2d(smem_u32(Vb + kb * SM::kKc + a * kBC * 128), &tm_kv, fb,
+                      (H + Hkv + g) * D + 64 * a, row);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    if (lane == 0) {
+      const uint32_t id_s = umma_idesc_f16(kAQ, kBC);            // S = Q K^T (fp16)
+      const uint32_t id_dp = umma_idesc_bf16(kAQ, kBC);          // dP = dO V^T (bf16)
+      const uint32_t id_acc = umma_idesc_bf16(kAQ, D) | (1u << 16);  // dQ += dS K: B MN-major
+      bool ok = mbar_wait_bounded(smem_u32(&bar_qd), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
+      auto issue_sdp = [&](int c) -> bool {
+        const int kb = c & 1;
+        if (!mbar_wait_bounded(smem_u32(&bar_kv[kb]), (uint32_t)((c >> 1) & 1), abort_flag,
+                               dev_err, DEV_ERR_WAIT_GEMM) ||
+            !mbar_wait_bounded(smem_u32(&bar_vconv[kb]), (uint32_t)((c >> 1) & 1), abort_flag,
+                               dev_err, DEV_ERR_WAIT_GEMM))
+          return false;
+        if (c >= 2 && !mbar_wait_bounded(smem_u32(&bar_tfree[kb]), (uint32_t)(((c - 2) >> 1) & 1),
+                                         abort_flag, dev_err, DEV_ERR_WAIT_GEMM))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qa = (uint32_t)((kk >> 2) * kAQ * 128 + (kk & 3) * 32);
+          const uint32_t ka = (uint32_t)((kk >> 2) * kBC * 128 + (kk & 3) * 32);
+          tc_mma_bf16(tmem + kColS + (uint32_t)kb * kBC, umma_desc_k_sw128(smem_u32(Qs) + qa),
+                      umma_desc_k_sw128(smem_u32(Kb + kb * SM::kKc) + ka), id_s, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + kColP + (uint32_t)kb * kBC, umma_desc_k_sw128(smem_u32(dOs) + qa),
+                      umma_desc_k_sw128(smem_u32(Vb + kb * SM::kKc) + ka), id_dp, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&bar_sdp[kb]));
+        return true;
+      };
+      ok = ok && issue_sdp(0);
+      for (int c = 0; c < nc && ok; ++c) {
+        const int kb = c & 1;
+        if (c + 1 < nc) ok = issue_sdp(c + 1);
+        if (!ok) break;
+        ok = mbar_wait_bounded(smem_u32(&bar_ds), (uint32_t)(c & 1), abort_flag, dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBC / 16; ++kk)
+          tc_mma_bf16(tmem + kColQ, umma_desc_k_sw128(smem_u32(dSs) + (uint32_t)(kk * 32)),
+                      umma_desc_mn_sw128(smem_u32(Kb + kb * SM::kKc) + (uint32_t)kk * 16 * 128,
+                                         kBC * 128, 1024u),
+                      id_acc, (c > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bar_dsfree));     // dS read; dQ updated
+        tc_commit(smem_u32(&bar_kvfree[kb]));  // the K and V chunk read
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- gradient warps
+    const int tid = threadIdx.x;
+    const int r = (warp & 3) * 32 + lane;  // query row of the block = TMEM lane
+    const int hf = warp >> 2;              // keys 32 hf .. of each chunk
+    const int q = q0 + r;
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    pdl_wait();  // delta comes from the kernels before
+    const int qq = min(q, seq - 1);
+    const float l2 = __ldg(lse + (int64_t)h * T + tok0 + qq) * 1.4426950408889634f;
+    const float dl = __ldg(delta + (int64_t)h * T + tok0 + qq);
+    bool ok = true;
+    // V of chunk c becomes bf16 (dP's operand) as soon as it lands
+    auto convert_v = [&](int c) -> bool {
+      const int kb = c & 1;
+      bool w = mbar_wait_bounded(smem_u32(&bar_kv[kb]), (uint32_t)((c >> 1) & 1), abort_flag,
+                                 dev_err, DEV_ERR_WAIT_GEMM);
+      w = __all_sync(0xFFFFFFFFu, w);
+      if (!w) return false;
+      tile_f16_to_bf16(Vb + kb * SM::kKc, SM::kKc, tid);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_vconv[kb]));
+      return true;
+    };
+    ok = convert_v(0);
+    for (int c = 0; c < nc && ok; ++c) {
+      const int kb = c & 1;
+      if (c + 1 < nc && !convert_v(c + 1)) { ok = false; break; }
+      ok = mbar_wait_bounded(smem_u32(&bar_sdp[kb]), (uint32_t)((c >> 1) & 1), abort_flag, dev_err,
+                             DEV_ERR_WAIT_GEMM);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[2][16], pv[2][16];
+      tmem_ld16(trow + kColS + (uint32_t)(kb * kBC + 32 * hf), sv[0]);
+      tmem_ld16(trow + kColS + (uint32_t)(kb * kBC + 32 * hf + 16), sv[1]);
+      tmem_ld16(trow + kColP + (uint32_t)(kb * kBC + 32 * hf), pv[0]);
+      tmem_ld16(trow + kColP + (uint32_t)(kb * kBC + 32 * hf + 16), pv[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_tfree[kb]));
+      const int kfirst = c * kBC + 32 * hf;  // this thread's first key
+      uint32_t dpk[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        float d[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int key = kfirst + e + u;
+          const bool live = key <= q && key < seq && q < seq;
+          const float s = __uint_as_float(sv[(e + u) >> 4][(e + u) & 15]);
+          const float dp = __uint_as_float(pv[(e + u) >> 4][(e + u) & 15]);
+          const float p = live ? exp2f(fmaf(s, sl2, -l2)) : 0.f;
+          d[u] = p * (dp - dl);
+        }
+        dpk[e >> 1] = pack_bf16x2(d[0], d[1]);
+      }
+      // the previous chunk's dQ product has read dS
+      if (c > 0) {
+        ok = mbar_wait_bounded(smem_u32(&bar_dsfree), (uint32_t)((c - 1) & 1), abort_flag, dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        *reinterpret_cast<uint4*>(dSs + sw128_offset((uint32_t)r, (uint32_t)(hf * 4 + cc))) =
+            make_uint4(dpk[4 * cc], dpk[4 * cc + 1], dpk[4 * cc + 2], dpk[4 * cc + 3]);
+      // S of this chunk is done with K: K becomes dQ's bf16 operand
+      tile_f16_to_bf16(Kb + kb * SM::kKc, SM::kKc, tid);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_ds));
+    }
+    if (ok) ok = mbar_wait_bounded(smem_u32(&bar_dsfree), (uint32_t)((nc - 1) & 1), abort_flag,
+                                   dev_err, DEV_ERR_WAIT_GEMM);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool live = q < seq;
+      const int64_t o = (tok0 + q) * (int64_t)H * D + (int64_t)h * D + hf * (D / 2);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[16];
+        tmem_ld16(trow + kColQ + (uint32_t)(hf * (D / 2) + 16 * c), v);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(dq + o + 16 * c + e) =
+                make_float4(__uint_as_float(v[e]) * scale, __uint_as_float(v[e + 1]) * scale,
+                            __uint_as_float(v[e + 2]) * scale, __uint_as_float(v[e + 3]) * scale);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_sh) settle_ns(2000000);
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -776,29 +944,55 @@ template <int D>
 int attn_bwd_t(const uint16_t* qkv, const uint16_t* o, const uint16_t* dout, const float* lse,
                int64_t T, int seq, int H, int Hkv, float* delta, float* dq, float* dk, float* dv,
                cudaStream_t st) {
-  const size_t s_kv = 6 * kTile * (D + 8) * sizeof(uint16_t) + 4 * kTile * sizeof(float);
-  const size_t s_q = 6 * kTile * (D + 8) * sizeof(uint16_t);
-  static bool attr = false;
-  if (!attr) {
-    LSQ_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_kv));
-    LSQ_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<D>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_q));
-    attr = true;
+  static bool attr[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr[dev]) {
+    LSQ_CUDA(cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)DkvSmem<D>::kBytes));
+    LSQ_CUDA(cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)DqSmem<D>::kBytes));
+    attr[dev] = true;
   }
+  if (T > INT32_MAX - kAK) return set_error(LSQ_ERR_SHAPE, "attention: too many tokens");
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
   const int batch = (int)(T / seq);
   const float scale = 1.f / sqrtf((float)D);
   const float sl2 = 1.4426950408889634f * scale;
   const int64_t nw = T * H;
   attn_delta_kernel<D><<<(unsigned)((nw * 32 + 255) / 256), 256, 0, st>>>(o, dout, T, H, delta);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  dim3 gkv((seq + kTile - 1) / kTile, H, batch);
-  attn_bwd_dkdv_kernel<D><<<gkv, 128, s_kv, st>>>(qkv, dout, lse, delta, T, seq, H, Hkv, sl2, scale,
-                                                  dk, dv);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  dim3 gq((seq + kTile - 1) / kTile, H, batch);
-  attn_bwd_dq_kernel<D><<<gq, 128, s_q, st>>>(qkv, dout, lse, delta, T, seq, H, Hkv, sl2, scale, dq);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  const int64_t row = (int64_t)(H + 2 * Hkv) * D;  // elements per token of q|k|v
+  CUtensorMap tm_qkv128, tm_qkv64, tm_do128, tm_do64;
+  LSQ_TRY(make_tmap_2d(&tm_qkv128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, qkv, (uint64_t)row,
+                       (uint64_t)T, (uint64_t)row, 64, kAK, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(make_tmap_2d(&tm_qkv64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, qkv, (uint64_t)row,
+                       (uint64_t)T, (uint64_t)row, 64, kBC, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(make_tmap_2d(&tm_do128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)H * D,
+                       (uint64_t)T, (uint64_t)H * D, 64, kAQ, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(make_tmap_2d(&tm_do64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)H * D,
+                       (uint64_t)T, (uint64_t)H * D, 64, kBC, CU_TENSOR_MAP_SWIZZLE_128B));
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((seq + kAK - 1) / kAK), (unsigned)H, (unsigned)batch);
+  cfg.blockDim = dim3(kAThreads);
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cfg.dynamicSmemBytes = DkvSmem<D>::kBytes;
+  LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(&cfg, attn_bwd_dkdv_tc_kernel<D>, tm_qkv128, tm_qkv64,
+                                              tm_do64, lse, (const float*)delta, T, seq, H, Hkv,
+                                              sl2, scale, dk, dv, dev_err)));
+  cfg.gridDim = dim3((unsigned)((seq + kAQ - 1) / kAQ), (unsigned)H, (unsigned)batch);
+  cfg.dynamicSmemBytes = DqSmem<D>::kBytes;
+  LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(&cfg, attn_bwd_dq_tc_kernel<D>, tm_qkv128, tm_qkv64,
+                                              tm_do128, lse, (const float*)delta, T, seq, H, Hkv,
+                                              sl2, scale, dq, dev_err)));
   return LSQ_OK;
 }
 
