@@ -107,8 +107,8 @@ size_t linear_ws_plan(int64_t T, int64_t K, int64_t N, int r, LinearWs* w, void*
   b.cap = SIZE_MAX;
   float* u = b.take<float>((size_t)T * r);
   float* v = b.take<float>((size_t)T * r);
-  uint16_t* u16 = b.take<uint16_t>((size_t)T * r);
-  uint16_t* v16 = b.take<uint16_t>((size_t)T * r);
+  uint16_t* u16 = b.take<uint16_t>((size_t)lora16_ld(T) * r);  // [r][lora16_ld(T)]
+  uint16_t* v16 = b.take<uint16_t>((size_t)lora16_ld(T) * r);
   float* s = b.take<float>(sb / sizeof(float) + 1);
   void* g = b.take<uint8_t>(gb + 256);
   if (w) {

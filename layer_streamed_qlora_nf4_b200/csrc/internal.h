@@ -174,31 +174,34 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st);
 int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 
-// LoRA rank-r products (tensor cores, fp32 accumulation, fixed-order reductions).
-// Operands in their product types: u = x A^T multiplies fp16 (x an fp16 forward
-// activation, A rounded to fp16); v, dA, dB multiply bf16 (each has a gradient
-// operand).  Widths R are multiples of 8.  The products that feed another write
-// its operand too (u16, v16: the result rounded to bf16).
+// LoRA rank-r products (tcgen05 tensor cores, fp32 accumulation, fixed-order
+// reductions).  Operands in their product types: u = x A^T multiplies fp16 (x an
+// fp16 forward activation, A rounded to fp16); v, dA, dB multiply bf16 (each has a
+// gradient operand).  Widths R are multiples of 8.  The products that
+// feed another write its operand too, rounded to bf16 and transposed: u16, v16
+// [R][lora16_ld(T)].
 // scratch: lora_scratch_bytes(T, K, R) bytes for the fixed-order partials of a
 // product split along its reduction (and, in the fp32-operand forms, the 16-bit
 // copy of the LoRA operand).
+int64_t lora16_ld(int64_t T);  // row stride of u16 / v16: T rounded up to 8
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
 // u[t, j] = sum_k x[t, k] A[j, k]        x fp16 [T, ldx], A16 fp16 [R, K] -> u fp32 [T, R]
 int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
                        int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
                        cudaStream_t st);
-// v[t, c] = sum_n dy[t, n] Bs[n, c]      dy bf16 [T, N], Bs bf16 [N, R] (block-diagonal:
-// row n of part p holds B_p's row in columns [p r, (p + 1) r), zeros elsewhere)
+// v[t, c] = sum_n dy[t, n] Bt[c, n]      dy bf16 [T, N], Bt bf16 [R, N]: the block-diagonal
+// stack of the parts' B transposed (column n of part p holds B_p's row n in rows
+// [p r, (p + 1) r), zeros elsewhere)
 int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
                         float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
                         cudaStream_t st);
-// dA[j, k] (+)= s sum_t v[t, j] x[t, k]  v16 bf16 [T, R], x fp16 [T, K] (rounded to bf16
-// as it is loaded)
+// dA[j, k] (+)= s sum_t v[t, j] x[t, k]  v16 bf16 [R, lora16_ld(T)], x fp16 [T, K] (converted
+// to bf16 as it is loaded)
 int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
                          float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
                          cudaStream_t st);
-// dB[n, j] (+)= s sum_t dy[t, n] u[t, part(n) r + j]   dy bf16 [T, N], u16 bf16 [T, n_parts r];
-// one product over all parts (parts of rows ending at part_end[])
+// dB[n, j] (+)= s sum_t dy[t, n] u[t, part(n) r + j]   dy bf16 [T, N], u16 bf16
+// [n_parts r, lora16_ld(T)]; one product over all parts (parts of rows ending at part_end[])
 int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
                          int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
                          float* scratch, size_t scratch_bytes, cudaStream_t st);
@@ -211,9 +214,10 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
                       uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st);
 // One layer's LoRA operands rounded once into their product types: a list of
 // blocks, each an fp16 copy of an A matrix (kind 0: [rows][cols]) or a bf16
-// block-diagonal stack of a B matrix (kind 1: [rows][ld_out], rows split into
-// parts ending at part_end[], part p's rows holding B in columns [p cols,
-// (p + 1) cols)).  Offsets in elements within one layer's LoRA block / output.
+// block-diagonal stack of a B matrix, transposed (kind 1: [ld_out][rows], the
+// rows split into parts ending at part_end[], part p's rows holding B in rows
+// [p cols, (p + 1) cols) of the stack).  Offsets in elements within one layer's
+// LoRA block / output.
 struct LoraPrepSeg {
   int64_t src_off, dst_off, rows, cols, ld_out;
   int kind, n_parts;

@@ -232,8 +232,8 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
 // Workspace carve-up (identical for the forward and the backward).
 struct Buffers {
   uint16_t* lora16;                                  // this layer's Lora16 (when not given)
-  uint16_t *u16_qkv, *u16_o, *u16_gu, *u16_d;        // bf16 copies of u, for dB
-  uint16_t *v16_qkv, *v16_o, *v16_gu, *v16_d;        // bf16 copies of v, for dA
+  uint16_t *u16_qkv, *u16_o, *u16_gu, *u16_d;        // bf16 copies of u, for dB ([R][ld])
+  uint16_t *v16_qkv, *v16_o, *v16_gu, *v16_d;        // bf16 copies of v, for dA ([R][ld])
   float* h;                                          // fp32 residual stream after attention
   uint16_t *n1, *qkv, *ao, *n2, *gu, *m;             // fp16 forward activations
   uint16_t *dgu, *dqkv, *da, *dout_b, *dh_b;         // bf16 gradients
@@ -337,14 +337,15 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   x.rstd1 = a.take<float>(T);
   x.rstd2 = a.take<float>(T);
   x.lora16 = a.take<uint16_t>(lora16_layout(s).elems);
-  x.u16_qkv = a.take<uint16_t>(T * 3 * r);
-  x.u16_o = a.take<uint16_t>(T * r);
-  x.u16_gu = a.take<uint16_t>(T * 2 * r);
-  x.u16_d = a.take<uint16_t>(T * r);
-  x.v16_qkv = a.take<uint16_t>(T * 3 * r);
-  x.v16_o = a.take<uint16_t>(T * r);
-  x.v16_gu = a.take<uint16_t>(T * 2 * r);
-  x.v16_d = a.take<uint16_t>(T * r);
+  const int64_t t16 = lora16_ld(T);  // u16, v16: [R][t16], transposed
+  x.u16_qkv = a.take<uint16_t>(t16 * 3 * r);
+  x.u16_o = a.take<uint16_t>(t16 * r);
+  x.u16_gu = a.take<uint16_t>(t16 * 2 * r);
+  x.u16_d = a.take<uint16_t>(t16 * r);
+  x.v16_qkv = a.take<uint16_t>(t16 * 3 * r);
+  x.v16_o = a.take<uint16_t>(t16 * r);
+  x.v16_gu = a.take<uint16_t>(t16 * 2 * r);
+  x.v16_d = a.take<uint16_t>(t16 * r);
   x.u_qkv = a.take<float>(T * 3 * r);
   x.u_o = a.take<float>(T * r);
   x.u_gu = a.take<float>(T * 2 * r);

@@ -1,27 +1,30 @@
-// LoRA rank-r products around the fused NF4 GEMM (tensor cores, mma.sync).
+// LoRA rank-r products around the fused NF4 GEMM, on 5th-generation tensor cores.
 //
 // For y = x W^T + s (x A^T) B^T (Soup layer-streaming tutorial, "四段資料路徑"
 // part 1) and its backward (part 3): u = x A^T (forward), v = dY B, and the
 // trainable gradients dA = s v^T x, dB = s dY^T u.  All four are "tall x
-// skinny" products: C[m, n] = sum_k P(m, k) Q(k, n) with n spanning r to 3 r
-// columns (one tile of up to 192 columns, more tiles beyond), P a bf16
-// activation and Q an fp32 LoRA tensor.
+// skinny" products C[m, n] = sum_k A(m, k) B(n, k) with n spanning the rank
+// (r to 3 r columns, up to 192) and m and k the long dimensions.
 //
-// One kernel serves all four.  A CTA owns 128 rows x BN columns of C over one
-// slice of the reduction.  Q is first rounded once to a 16-bit type (nearest
-// even) into scratch, rows padded to a multiple of 8 elements with zeros;
-// accumulation is fp32 (the tutorial's part 1: the LoRA A/B matrices are
-// computed at a higher precision than the NF4 storage).  Operand types follow
-// the activations: u = x A^T multiplies fp16 (x is an fp16 forward activation,
-// A is rounded to fp16); v, dA and dB multiply bf16 (each has a gradient
-// operand, which needs bf16's range; dA's fp16 activation is rounded to bf16
-// as it moves from shared memory into registers).  Both operands then stream through a ring of 4 to 6
-// cp.async stages (16-byte chunks along whichever index is contiguous in
-// memory; ldmatrix, transposing where needed, gives the MMA fragments), so
-// that each SM keeps enough bytes in flight to run these HBM-bound products
-// near the memory roofline.  When a product is split along its reduction, the
-// slices are summed by a second kernel in a fixed order, so results are
-// deterministic (no atomics); an unsplit product writes its result directly.
+// One kernel serves all four: a CTA owns 128 rows of C and up to 256 columns
+// (all of them for ranks up to 256), over one slice of the reduction.  A (the activation or gradient, 128 x 64 per
+// stage) and B (the rank-side operand, n_pad x 64) arrive by TMA in the
+// 128-byte-swizzle layout; one thread issues tcgen05.mma (M = 128, N = n_pad,
+// K = 16) into a TMEM accumulator; the four warps read it back in the epilogue.
+// A is K-major for u and v (x, dY read along their rows) and MN-major for dA and
+// dB (x, dY read along their columns, the reduction running over tokens).  B is
+// always K-major: the products that feed dA and dB store their 16-bit result
+// transposed (u16, v16: [R][ld] with ld = T rounded up to 8), and the B operand
+// of v is stored transposed too ([R][N]), so the rank is never the swizzled
+// dimension.  Operand types follow the activations: u = x A^T multiplies fp16;
+// v, dA and dB multiply bf16 (each has a gradient operand, which needs bf16's
+// range); dA's fp16 activation is converted to bf16 in shared memory as each
+// stage lands.  Accumulation is fp32 (the tutorial's part 1: the LoRA A/B
+// matrices are computed at a higher precision than the NF4 storage).  When a
+// product is split along its reduction, the slices are summed by a second
+// kernel in a fixed order, so results are deterministic (no atomics); an
+// unsplit product writes its result directly.
+#include <cuda.h>
 #include <stdlib.h>
 
 #include "common.cuh"
@@ -30,18 +33,16 @@ namespace lsq {
 
 namespace {
 
-constexpr int kBM = 128;  // rows of C per CTA
-constexpr int kBK = 32;   // reduction elements per stage
-constexpr int kThreads = 256;
+constexpr int kSM = 128;       // rows of C per CTA (UMMA M)
+constexpr int kSK = 64;        // reduction per stage: one 128-byte swizzle atom of 16-bit values
+constexpr int kSThreads = 128;
 constexpr int kSMs = 148;
+constexpr int kSMaxN = 256;    // columns per CTA (one MMA's N); wider products tile the columns
+constexpr uint32_t kSAStage = kSM * kSK * 2;  // 16 KB
 
 struct SkinnyArgs {
-  const uint16_t* P;   // bf16: P(m, k) = P[m * p_m + k * p_k]
-  int64_t p_m, p_k;
-  const uint16_t* Q;   // bf16: Q(k, n) = Q[k * q_k + n * q_n]; rows padded to 8 elements
-  int64_t q_k, q_n;
   int64_t M, N, K;     // C is M x N, reduction over K
-  int64_t k_per_split;
+  int kt_per_split;    // reduction stages (of 64) per split
   float* part;         // [splits][M][N] when split
   // unsplit: dst[m * c_m + n * c_n] = alpha * C[m, n] (+ dst if accumulate)
   float* dst;
@@ -51,16 +52,16 @@ struct SkinnyArgs {
   int direct;
   // Output options (applied where the result is written: the direct epilogue or
   // the slice sum): c16 (nullable) also receives the result rounded to bf16,
-  // c16[m * c16_ld + n], for the product that consumes it; with part_r > 0 the
-  // rows are split into parts ending at part_end[], and row m of part p keeps
-  // only columns [p part_r, (p + 1) part_r), written to column n - p part_r.
+  // c16[m * c16_m + n * c16_n], for the product that consumes it; with part_r >
+  // 0 the rows are split into parts ending at part_end[], and row m of part p
+  // keeps only columns [p part_r, (p + 1) part_r), written to column n - p part_r.
   uint16_t* c16;
-  int64_t c16_ld;
+  int64_t c16_m, c16_n;
   int part_r, n_parts;
   int64_t part_end[4];
 };
 
-// Writes one result element of row m, column n (see SkinnyArgs); false if dropped.
+// Writes one result element of row m, column n (see SkinnyArgs).
 __device__ __forceinline__ void store_result(const SkinnyArgs& a, int64_t m, int64_t n, float v) {
   int64_t col = n;
   if (a.part_r > 0) {
@@ -71,216 +72,169 @@ __device__ __forceinline__ void store_result(const SkinnyArgs& a, int64_t m, int
   }
   float* d = a.dst + m * a.c_m + col * a.c_n;
   *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
-  if (a.c16) a.c16[m * a.c16_ld + n] = float_to_bf16_bits(v);
+  if (a.c16) a.c16[m * a.c16_m + n * a.c16_n] = float_to_bf16_bits(v);
 }
 
-__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+__device__ __forceinline__ uint8_t* align1024_s(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Operand precision of a product: PM_BF16 both operands bf16; PM_F16 both fp16;
-// PM_P16 P stored fp16 and rounded to bf16 in registers, Q bf16.
-enum { PM_BF16 = 0, PM_F16 = 1, PM_P16 = 2 };
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-// Shared-memory tiles per stage (bf16, rows padded by 8 elements so that the
-// eight 16-byte rows an ldmatrix reads fall in distinct banks):
-//   P_RED: P as [kBM m][kBK + 8]   else P as [kBK k][kBM + 8]
-//   Q_RED: Q as [BN n][kBK + 8]    else Q as [kBK k][BN + 8]
-// Stages and CTAs per SM: BN 64 -> 4 stages, 3 CTAs (61 KB each); BN 128 -> 4
-// stages, 2 CTAs (82 KB); BN 192 -> 6 stages, 1 CTA (154 KB).
-template <bool P_RED, bool Q_RED, int BN>
-struct Tile {
-  static constexpr int kStages = BN > 128 ? 6 : 4;
-  static constexpr int kMinBlocks = BN <= 64 ? 3 : BN <= 128 ? 2 : 1;
-  static constexpr int kPE = P_RED ? kBM * (kBK + 8) : kBK * (kBM + 8);
-  static constexpr int kQE = Q_RED ? BN * (kBK + 8) : kBK * (BN + 8);
-  static constexpr size_t kSmem = (size_t)kStages * (kPE + kQE) * 2;
-};
-
-// P_RED: the reduction index is the contiguous one in P (else the row index m is).
-// Q_RED: the reduction index is the contiguous one in Q (else the column n is).
-template <bool P_RED, bool Q_RED, int BN, int PM>
-__global__ void __launch_bounds__(kThreads, (Tile<P_RED, Q_RED, BN>::kMinBlocks))
-    skinny_kernel(const SkinnyArgs a) {
+// A_MN: A is MN-major (its m index contiguous in memory); CONV: A is stored fp16
+// and converted to bf16 in shared memory before the MMA reads it.
+//   warp 0: TMA producer (lane 0);  warp 1: TMEM and the MMA issuer (lane 0);
+//   warps 2-3: the conversion (CONV); all four: the epilogue (TMEM lane quarter = warp)
+template <bool A_MN, bool CONV>
+__global__ void __launch_bounds__(kSThreads, 1)
+    tc_skinny_kernel(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ SkinnyArgs a,
+                     uint32_t idesc, int n_pad, int stages, uint32_t tmem_cols, int* dev_err) {
+  extern __shared__ uint8_t sk_raw[];
+  constexpr int kMaxSt = 4;
+  __shared__ __align__(8) uint64_t bar_full[kMaxSt], bar_conv[kMaxSt], bar_empty[kMaxSt], bar_acc;
+  __shared__ uint32_t tmem_sh;
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
   pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  using TL = Tile<P_RED, Q_RED, BN>;
-  constexpr int S = TL::kStages, PE = TL::kPE, QE = TL::kQE;
-  extern __shared__ __align__(16) uint16_t sk_smem[];
-  uint16_t* Ps = sk_smem;        // [S][PE]
-  uint16_t* Qs = Ps + S * PE;    // [S][QE]
-  constexpr int WN = BN / 2;     // columns per warp (warps: 4 along m x 2 along n)
-  constexpr int NF = WN / 8;     // n8 fragments per warp
-  constexpr int QC = BN * kBK / 8 / kThreads;  // 16-byte chunks of Q per thread per stage
-  static_assert(QC >= 1 && (BN * kBK / 8) % kThreads == 0, "Q tile split");
-  static_assert(NF % 2 == 0, "B fragments are loaded in pairs");
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int wm = warp & 3, wn = warp >> 2;
-  const int64_t m0 = (int64_t)blockIdx.x * kBM;
-  const int64_t n0 = (int64_t)blockIdx.y * BN;
-  const int64_t k_begin = (int64_t)blockIdx.z * a.k_per_split;
-  const int64_t k_end = min(a.K, k_begin + a.k_per_split);
-  const int64_t n_it = k_end > k_begin ? (k_end - k_begin + kBK - 1) / kBK : 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t b_bytes = (uint32_t)n_pad * 128u;
+  uint8_t* st0 = align1024_s(sk_raw);
+  const uint32_t st_bytes = kSAStage + ((b_bytes + 1023u) & ~1023u);
+  const int64_t m0 = (int64_t)blockIdx.x * kSM;
+  const int kt_total = (int)((a.K + kSK - 1) / kSK);
+  const int kt_begin = blockIdx.z * a.kt_per_split;
+  const int n_it = max(0, min(kt_total, kt_begin + a.kt_per_split) - kt_begin);
+  const int S = stages;
 
-  float acc[2][NF][4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < NF; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-  // One stage: 512 chunks of P (two per thread) and BN * 4 chunks of Q.  Chunks
-  // outside the product (or this CTA's slice of the reduction) are zero-filled.
-  auto load_stage = [&](int slot, int64_t kb) {
-    uint16_t* pd = Ps + slot * PE;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int c = tid + i * kThreads;
-      if (P_RED) {  // row m, 4 chunks of k per row
-        const int mm = c >> 2, kc = (c & 3) * 8;
-        const int64_t m = m0 + mm, k = kb + kc;
-        const bool in = m < a.M && k < k_end;
-        cp_async16(smem_u32(pd + mm * (kBK + 8) + kc), a.P + (in ? m * a.p_m + k : 0),
-                   in ? 16u : 0u);
-      } else {      // row k, 16 chunks of m per row
-        const int kk = c >> 4, mc = (c & 15) * 8;
-        const int64_t m = m0 + mc, k = kb + kk;
-        const bool in = m < a.M && k < k_end;
-        cp_async16(smem_u32(pd + kk * (kBM + 8) + mc), a.P + (in ? k * a.p_k + m : 0),
-                   in ? 16u : 0u);
-      }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_conv[s]), 2);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
     }
-    uint16_t* qd = Qs + slot * QE;
-#pragma unroll
-    for (int i = 0; i < QC; ++i) {
-      const int c = tid + i * kThreads;
-      if (Q_RED) {  // row n, 4 chunks of k per row
-        const int nn = c >> 2, kc = (c & 3) * 8;
-        const int64_t n = n0 + nn, k = kb + kc;
-        const bool in = n < a.N && k < k_end;
-        cp_async16(smem_u32(qd + nn * (kBK + 8) + kc), a.Q + (in ? n * a.q_n + k : 0),
-                   in ? 16u : 0u);
-      } else {      // row k, BN / 8 chunks of n per row (the padded row ends on a chunk)
-        const int kk = c / (BN / 8), nc = (c % (BN / 8)) * 8;
-        const int64_t n = n0 + nc, k = kb + kk;
-        const bool in = n < a.N && k < k_end;
-        cp_async16(smem_u32(qd + kk * (BN + 8) + nc), a.Q + (in ? k * a.q_k + n : 0),
-                   in ? 16u : 0u);
-      }
-    }
-  };
-
-  // Ring: stage j lives in slot j % S; S - 1 stages are in flight ahead of the math.
-#pragma unroll
-  for (int j = 0; j < S - 1; ++j) {
-    if (j < n_it) load_stage(j, k_begin + (int64_t)j * kBK);
-    cp_async_commit();
+    mbar_init(smem_u32(&bar_acc), 1);
+    abort_sh = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
   }
-  for (int64_t it = 0; it < n_it; ++it) {
-    cp_async_wait<S - 2>();  // stage it has landed (this thread's chunks)
-    __syncthreads();         // ... every thread's, and slot (it - 1) % S is free again
-    {
-      const int64_t nx = it + S - 1;
-      if (nx < n_it) load_stage((int)(nx % S), k_begin + nx * kBK);
-      cp_async_commit();
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_sh), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();  // both operands come from the kernels before
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it % S;
+        if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), (uint32_t)((it / S) & 1) ^ 1u, abort_flag,
+                               dev_err, DEV_ERR_WAIT_GEMM))
+          break;
+        const int k0 = (kt_begin + it) * kSK;
+        uint8_t* sa = st0 + (size_t)s * st_bytes;
+        const uint32_t fb = smem_u32(&bar_full[s]);
+        mbar_arrive_expect_tx(fb, kSAStage + b_bytes);
+        if (A_MN) {  // two [64 k x 64 m] boxes, 64 m apart
+          tma_load_2d(smem_u32(sa), &tm_a, fb, (int)m0, k0);
+          tma_load_2d(smem_u32(sa + kSAStage / 2), &tm_a, fb, (int)m0 + 64, k0);
+        } else {     // one [128 m x 64 k] box
+          tma_load_2d(smem_u32(sa), &tm_a, fb, k0, (int)m0);
+        }
+        tma_load_2d(smem_u32(sa + kSAStage), &tm_b, fb, k0, (int)blockIdx.y * n_pad);
+      }
     }
-    const int slot = (int)(it % S);
-    const uint16_t* ps = Ps + slot * PE;
-    const uint16_t* qs = Qs + slot * QE;
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)((it / S) & 1);
+        if (!mbar_wait_bounded(smem_u32(CONV ? &bar_conv[s] : &bar_full[s]), ph, abort_flag,
+                               dev_err, DEV_ERR_WAIT_GEMM))
+          break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(st0 + (size_t)s * st_bytes);
 #pragma unroll
-    for (int k16 = 0; k16 < kBK; k16 += 16) {
-      uint32_t af[2][4];
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        const int r0 = wm * 32 + mi * 16;
-        if (P_RED) {
-          ldsm4(af[mi], smem_u32(ps + (r0 + (lane & 15)) * (kBK + 8) + k16 + 8 * (lane >> 4)));
-        } else {
-          const int i = lane >> 3, j = lane & 7;
-          ldsm4_t(af[mi], smem_u32(ps + (k16 + j + 8 * (i >> 1)) * (kBM + 8) + r0 + 8 * (i & 1)));
+        for (int kk = 0; kk < kSK / 16; ++kk) {
+          const uint64_t ad = A_MN ? umma_desc_mn_sw128(sa + (uint32_t)kk * 16 * 128, kSAStage / 2, 1024u)
+                                   : umma_desc_k_sw128(sa + (uint32_t)kk * 32);
+          const uint64_t bd = umma_desc_k_sw128(sa + kSAStage + (uint32_t)kk * 32);
+          tc_mma_bf16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        if (PM == PM_P16) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) af[mi][e] = f16x2_to_bf16x2(af[mi][e]);
-        }
+        tc_commit(smem_u32(&bar_empty[s]));
       }
-#pragma unroll
-      for (int nj = 0; nj < NF; nj += 2) {
-        // matrices: (n block nj, k 0-7), (nj, k 8-15), (nj + 1, k 0-7), (nj + 1, k 8-15)
-        const int i = lane >> 3, j = lane & 7;
-        uint32_t bh[4];
-        if (Q_RED) {
-          const int nr = wn * WN + (nj + (i >> 1)) * 8 + j;
-          ldsm4(bh, smem_u32(qs + nr * (kBK + 8) + k16 + 8 * (i & 1)));
-        } else {
-          const int kr = k16 + 8 * (i & 1) + j;
-          ldsm4_t(bh, smem_u32(qs + kr * (BN + 8) + wn * WN + (nj + (i >> 1)) * 8));
-        }
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-          if (PM == PM_F16) {
-            mma_f16(acc[mi][nj], af[mi], bh[0], bh[1]);
-            mma_f16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
-          } else {
-            mma_bf16(acc[mi][nj], af[mi], bh[0], bh[1]);
-            mma_bf16(acc[mi][nj + 1], af[mi], bh[2], bh[3]);
-          }
-        }
+      tc_commit(smem_u32(&bar_acc));
+    }
+    __syncwarp();
+  } else if (CONV) {
+    // warps 2-3: each landed A stage from fp16 to bf16, in place
+    const int tid = threadIdx.x - 64;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % S;
+      bool ok = mbar_wait_bounded(smem_u32(&bar_full[s]), (uint32_t)((it / S) & 1), abort_flag,
+                                  dev_err, DEV_ERR_WAIT_GEMM);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      uint8_t* sa = st0 + (size_t)s * st_bytes;
+      for (uint32_t o = (uint32_t)tid * 16u; o < kSAStage; o += 64u * 16u) {
+        uint4 v = *reinterpret_cast<uint4*>(sa + o);
+        v.x = f16x2_to_bf16x2(v.x);
+        v.y = f16x2_to_bf16x2(v.y);
+        v.z = f16x2_to_bf16x2(v.z);
+        v.w = f16x2_to_bf16x2(v.w);
+        *reinterpret_cast<uint4*>(sa + o) = v;
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_conv[s]));
     }
   }
-  cp_async_wait<0>();  // only empty groups can remain; leave none behind
 
+  // ------------------------------------------------------------------ epilogue
+  {
+    bool ok = true;
+    if (n_it > 0) {
+      ok = mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int64_t m = m0 + warp * 32 + lane;  // this thread's row (its TMEM lane)
+      const int64_t nc = (int64_t)blockIdx.y * n_pad;  // first column of this CTA
+      const bool mok = m < a.M;
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      for (int n0 = 0; n0 < n_pad; n0 += 16) {
+        uint32_t v[16];
+        if (n_it > 0) {
+          tmem_ld16(trow + (uint32_t)n0, v);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi) {
+          for (int j = 0; j < 16; ++j) v[j] = 0u;  // an empty slice contributes zeros
+        }
+        if (!mok) continue;
+        if (a.direct) {
 #pragma unroll
-    for (int nj = 0; nj < NF; ++nj) {
+          for (int j = 0; j < 16; ++j)
+            if (nc + n0 + j < a.N) store_result(a, m, nc + n0 + j, __uint_as_float(v[j]));
+        } else {
+          float* pr = a.part + ((size_t)blockIdx.z * a.M + m) * a.N + nc;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t m = m0 + wm * 32 + mi * 16 + (lane >> 2) + 8 * h;
-        const int64_t n = n0 + wn * WN + nj * 8 + 2 * (lane & 3);
-        if (m >= a.M) continue;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          if (n + e >= a.N) continue;
-          const float v = acc[mi][nj][2 * h + e];
-          if (a.direct) {
-            store_result(a, m, n + e, v);
-          } else {
-            a.part[((size_t)blockIdx.z * a.M + m) * a.N + n + e] = v;
-          }
+          for (int j = 0; j < 16; ++j)
+            if (nc + n0 + j < a.N) pr[n0 + j] = __uint_as_float(v[j]);
         }
       }
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_sh) settle_ns(2000000);  // let issued copies and MMAs land before freeing TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
   }
 }
 
@@ -299,110 +253,129 @@ __global__ void split_sum_kernel(const float* __restrict__ part, int splits, con
   }
 }
 
-// out[i * ld_out + j] = bf16 or fp16 (F16) of in[i * ld_in + j] for j < cols, 0 for
-// cols <= j < ld_out
-template <bool F16>
-__global__ void to_16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
-                                  int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
+// out[i * ld_out + j] = fp16 of in[i * ld_in + j] for j < cols, 0 for cols <= j < ld_out
+__global__ void to_f16_rows_kernel(const float* __restrict__ in, int64_t rows, int64_t cols,
+                                   int64_t ld_in, uint16_t* __restrict__ out, int64_t ld_out) {
   pdl_trigger();  // the next kernel may launch once all CTAs of this one run
   const int64_t n_el = rows * ld_out;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = i / ld_out, j = i % ld_out;
-    const float v = j < cols ? in[r * ld_in + j] : 0.f;
-    out[i] = F16 ? float_to_f16_bits(v) : float_to_bf16_bits(v);
+    out[i] = float_to_f16_bits(j < cols ? in[r * ld_in + j] : 0.f);
   }
 }
 
-int64_t pad8(int64_t n) { return (n + 7) / 8 * 8; }
+// out[j * rows + i] = bf16 of in[i * cols + j]: an [rows x cols] matrix transposed
+__global__ void to_bf16_transposed_kernel(const float* __restrict__ in, int64_t rows,
+                                          int64_t cols, uint16_t* __restrict__ out) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
+  const int64_t n_el = rows * cols;
+  for (int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; o < n_el;
+       o += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = o / rows, i = o % rows;
+    out[o] = float_to_bf16_bits(in[i * cols + j]);
+  }
+}
+
 size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+// columns per CTA: the product's width rounded up to 16, at most 256
+int npad_for(int64_t N) { return (int)std::min<int64_t>(kSMaxN, (N + 15) / 16 * 16); }
 
-// Column tile.  Default 64 for every product: 3 CTAs per SM, and a product
-// wider than 64 columns runs several column tiles, which read the same
-// activation rows (the second and third time mostly from L2).  LSQ_LORA_BN=128
-// or 192 selects one tile of up to that many columns instead (fewer activation
-// reads, 2 or 1 CTAs per SM).
-int bn_limit() {
-  static const int v = [] {
-    const char* e = getenv("LSQ_LORA_BN");
-    const int x = e ? atoi(e) : 64;
-    return (x == 128 || x == 192) ? x : 64;
-  }();
-  return v;
-}
-int bn_for(int64_t N) {
-  const int lim = bn_limit();
-  return (N <= 64 || lim == 64) ? 64 : (N <= 128 || lim == 128) ? 128 : 192;
-}
-int ctas_per_sm(int bn) { return bn <= 64 ? 3 : bn <= 128 ? 2 : 1; }
+// Stages and CTAs per SM: four stages for every width; the widest tiles (n_pad up
+// to 256, up to 48 KB a stage) run one CTA per SM, those up to 64 columns (24 KB a
+// stage) two.  (Up to eight stages were measured: no faster, since the dA product
+// is then paced by its in-place conversion.)
+size_t stage_bytes(int n_pad) { return kSAStage + ((size_t)n_pad * 128 + 1023) / 1024 * 1024; }
+int stages_for(int) { return 4; }
+size_t smem_for(int n_pad) { return 1024 + (size_t)stages_for(n_pad) * stage_bytes(n_pad); }
+int ctas_per_sm(int n_pad) { return smem_for(n_pad) <= 110 * 1024 ? 2 : 1; }
 
-// Splits of the reduction: only where the product's own tiles leave at least
-// half of the resident CTA slots (148 SMs x CTAs per SM) empty, up to filling
-// them, each slice at least four stages long (the partials cost a round trip
-// through HBM, so a grid that already fills the GPU is not split).
+// Splits of the reduction: only where the product's own row tiles leave at least
+// half of the resident CTA slots empty, up to filling them, each slice at least
+// two stages long.
 int splits_for(int64_t M, int64_t N, int64_t K) {
   if (K <= 0 || M <= 0 || N <= 0) return 1;
-  const int bn = bn_for(N);
-  const int64_t xy = ((M + kBM - 1) / kBM) * ((N + bn - 1) / bn);
-  int64_t z = (int64_t)kSMs * ctas_per_sm(bn) / xy;
-  const int64_t zmax = std::max<int64_t>(1, K / (4 * kBK));
-  z = std::max<int64_t>(1, std::min<int64_t>(z, std::min<int64_t>(zmax, 64)));
-  const int64_t kps = ((K + z - 1) / z + kBK - 1) / kBK * kBK;
-  return (int)((K + kps - 1) / kps);
+  const int64_t tiles = (M + kSM - 1) / kSM * ((N + kSMaxN - 1) / kSMaxN);
+  const int64_t slots = (int64_t)kSMs * ctas_per_sm(npad_for(N));
+  if (tiles * 2 > slots) return 1;
+  const int64_t kt = (K + kSK - 1) / kSK;
+  int64_t z = std::max<int64_t>(1, std::min<int64_t>(slots / tiles, std::min<int64_t>(kt / 2, 64)));
+  const int64_t kps = (kt + z - 1) / z;
+  return (int)((kt + kps - 1) / kps);
 }
 
-template <bool P_RED, bool Q_RED, int BN, int PM>
-int launch_bn(const SkinnyArgs& a, dim3 grid, cudaStream_t st) {
-  constexpr size_t smem = Tile<P_RED, Q_RED, BN>::kSmem;
-  static bool attr_done[64] = {false};
+template <bool A_MN, bool CONV>
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const SkinnyArgs& a, uint32_t idesc,
+              int n_pad, dim3 grid, cudaStream_t st) {
+  const size_t smem = smem_for(n_pad);
+  static bool attr[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    LSQ_CUDA(cudaFuncSetAttribute(skinny_kernel<P_RED, Q_RED, BN, PM>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr_done[dev] = true;
+  if (dev < 64 && !attr[dev]) {
+    LSQ_CUDA(cudaFuncSetAttribute(tc_skinny_kernel<A_MN, CONV>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem_for(kSMaxN)));
+    attr[dev] = true;
   }
-  skinny_kernel<P_RED, Q_RED, BN, PM><<<grid, kThreads, smem, st>>>(a);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  uint32_t cols = 32;
+  while (cols < (uint32_t)n_pad) cols <<= 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kSThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(&cfg, tc_skinny_kernel<A_MN, CONV>, ta, tb, a, idesc,
+                                              n_pad, stages_for(n_pad), cols, dev_err)));
   return LSQ_OK;
 }
 
-int convert_rows(const float* in, int64_t rows, int64_t cols, int64_t ld_in, uint16_t* out,
-                 int64_t ld_out, cudaStream_t st, bool f16 = false) {
-  int64_t g = (rows * ld_out + 255) / 256;
-  if (g > kSMs * 8) g = kSMs * 8;
-  if (g < 1) return LSQ_OK;
-  if (f16)
-    to_16_rows_kernel<true><<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
-  else
-    to_16_rows_kernel<false><<<(unsigned)g, 256, 0, st>>>(in, rows, cols, ld_in, out, ld_out);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return LSQ_OK;
-}
+// The operands of one product, as 2-D row-major 16-bit tensors.
+struct Operand {
+  const uint16_t* p;
+  int64_t inner, rows, ld;  // elements per row, rows, row stride (elements)
+  bool f16;
+};
 
-// C = P Q over K, written as a prescribes (dst, alpha, accumulate, c16, parts);
-// scratch holds the fixed-order partials when the product is split.
-template <bool P_RED, bool Q_RED, int PM>
-int run(SkinnyArgs a, float* scratch, size_t scratch_bytes, cudaStream_t st) {
+// C = A B^T over K (A: M x K, K-major unless A_MN; B: N x K, K-major), written as
+// a prescribes (dst, alpha, accumulate, c16, parts); scratch holds the fixed-order
+// partials when the product is split.  CONV: A is fp16 and meets a bf16 B.
+template <bool A_MN, bool CONV>
+int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, float* scratch,
+        size_t scratch_bytes, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return LSQ_OK;
+  if (a.K <= 0) return set_error(LSQ_ERR_SHAPE, "lora product: empty reduction");
+  const int n_pad = npad_for(a.N);
   const int z = splits_for(a.M, a.N, a.K);
   const size_t need = z > 1 ? (size_t)z * a.M * a.N * sizeof(float) : 0;
   if (need && (!scratch || scratch_bytes < need))
     return set_error(LSQ_ERR_WORKSPACE, "lora product: scratch %zu < %zu", scratch_bytes, need);
-  a.k_per_split = a.K > 0 ? ((a.K + z - 1) / z + kBK - 1) / kBK * kBK : kBK;
+  const int kt = (int)((a.K + kSK - 1) / kSK);
+  a.kt_per_split = std::max(1, (kt + z - 1) / z);
   a.direct = z == 1;
   a.part = z > 1 ? scratch : nullptr;
-  const int bn = bn_for(a.N);
-  dim3 grid((unsigned)((a.M + kBM - 1) / kBM), (unsigned)((a.N + bn - 1) / bn), (unsigned)z);
-  switch (bn) {
-    case 64: LSQ_TRY((launch_bn<P_RED, Q_RED, 64, PM>(a, grid, st))); break;
-    case 128: LSQ_TRY((launch_bn<P_RED, Q_RED, 128, PM>(a, grid, st))); break;
-    default: LSQ_TRY((launch_bn<P_RED, Q_RED, 192, PM>(a, grid, st))); break;
-  }
+  CUtensorMap ta, tb;
+  const CUtensorMapDataType dta = A.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dtb = B.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  LSQ_TRY(make_tmap_2d(&ta, dta, 2, A.p, (uint64_t)A.inner, (uint64_t)A.rows, (uint64_t)A.ld, 64,
+                       A_MN ? 64 : kSM, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(make_tmap_2d(&tb, dtb, 2, B.p, (uint64_t)B.inner, (uint64_t)B.rows, (uint64_t)B.ld, 64,
+                       (uint32_t)n_pad, CU_TENSOR_MAP_SWIZZLE_128B));
+  uint32_t idesc = f16 ? umma_idesc_f16(kSM, n_pad) : umma_idesc_bf16(kSM, n_pad);
+  if (A_MN) idesc |= 1u << 15;  // A MN-major
+  const dim3 grid((unsigned)((a.M + kSM - 1) / kSM), (unsigned)((a.N + n_pad - 1) / n_pad),
+                  (unsigned)((kt + a.kt_per_split - 1) / a.kt_per_split));
+  LSQ_TRY((launch_tc<A_MN, CONV>(ta, tb, a, idesc, n_pad, grid, st)));
   if (z == 1) return LSQ_OK;
   int64_t g = (a.M * a.N + 255) / 256;
   if (g > kSMs * 8) g = kSMs * 8;
-  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, z, a);
+  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, (int)grid.z, a);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }
@@ -418,7 +391,7 @@ int check_ranks(int64_t R) {
 }
 
 SkinnyArgs out_args(float* dst, int64_t c_m, int64_t c_n, float alpha, int accumulate,
-                    uint16_t* c16, int64_t c16_ld) {
+                    uint16_t* c16, int64_t c16_m, int64_t c16_n) {
   SkinnyArgs a{};
   a.dst = dst;
   a.c_m = c_m;
@@ -426,7 +399,8 @@ SkinnyArgs out_args(float* dst, int64_t c_m, int64_t c_n, float alpha, int accum
   a.alpha = alpha;
   a.accumulate = accumulate;
   a.c16 = c16;
-  a.c16_ld = c16_ld;
+  a.c16_m = c16_m;
+  a.c16_n = c16_n;
   return a;
 }
 
@@ -447,27 +421,34 @@ int split_scratch(float* scratch, size_t bytes, size_t q_elems, Split* out, cons
   return LSQ_OK;
 }
 
+unsigned grid_for_elems(int64_t n) {
+  int64_t g = (n + 255) / 256;
+  if (g > kSMs * 8) g = kSMs * 8;
+  return (unsigned)std::max<int64_t>(1, g);
+}
+
 }  // namespace
+
+int64_t lora16_ld(int64_t T) { return (T + 7) / 8 * 8; }
 
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
   // An upper bound over every product a caller sizing by (T, K, R) can make:
-  // any width R' <= R, a reduction or a part of up to K elements:
-  //   u = x A^T, v      M = T, N = R', reduction <= K, Q = A [R'][K] or B [<= K][R']
-  //   dA, dB            M <= K, N = R', reduction T,   Q = v or u [T][R']
-  // The first needs z(T, R', K) slices at most (splits grow with the reduction);
-  // the second z * M <= min(64, T / (4 kBK)) K, and z * M <= slots * kBM as well,
-  // since z <= slots / (M / kBM tiles).  The 16-bit copy of an fp32 operand comes first.
+  // any width R' <= R (a multiple of 8), and
+  //   u = x A^T, v      M = T, N = R', reduction <= K
+  //   dA, dB            M <= K, N = R', reduction T
+  // The split count never exceeds the CTA slots over the row tiles, so z M is at
+  // most slots x 128 (or z = 1).  The 16-bit copy of an fp32 LoRA operand
+  // (R x K elements) comes first.
   size_t best = 0;
-  for (int rr = 1; rr <= R; ++rr) {
-    const int64_t q1 = K * pad8(rr);
+  for (int rr = 8; rr <= std::max(8, R); rr += 8) {
+    const int64_t slots = (int64_t)kSMs * ctas_per_sm(npad_for(rr));
     const int z1 = splits_for(T, rr, K);
-    best = std::max(best, align256((size_t)q1 * 2) +
-                              (z1 > 1 ? (size_t)z1 * T * rr * sizeof(float) : 0));
-    const int64_t q2 = T * pad8(rr);
-    const int64_t zcap = std::max<int64_t>(1, std::min<int64_t>(64, T / (4 * kBK)));
-    const int64_t zm = std::min<int64_t>(zcap * K, (int64_t)kSMs * ctas_per_sm(bn_for(rr)) * kBM);
-    best = std::max(best, align256((size_t)q2 * 2) +
-                              (zcap > 1 ? (size_t)zm * rr * sizeof(float) : 0));
+    const size_t p1 = z1 > 1 ? (size_t)z1 * T * rr * sizeof(float) : 0;
+    int64_t zm = 0;  // the largest z M over M <= K for the reduction over T
+    const int64_t kt = (T + kSK - 1) / kSK;
+    if (kt >= 4) zm = std::min<int64_t>(slots * kSM, std::min<int64_t>(64, kt / 2) * K);
+    const size_t p2 = (size_t)zm * rr * sizeof(float);
+    best = std::max(best, align256((size_t)K * rr * 2) + std::max(p1, p2));
   }
   return best;
 }
@@ -476,14 +457,13 @@ int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int6
                        int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
                        cudaStream_t st) {
   LSQ_TRY(check_ranks(R));
-  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
-  // C[t, j] = sum_k x[t, k] A[j, k]   (fp16 operands)
+  if (K % 8 != 0 || ldx % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
+  // C[t, j] = sum_k x[t, k] A[j, k]   (fp16 operands); u16 transposed [R][ld]
   const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(u, R, 1, 1.f, 0, u16, R);
-  a.P = x; a.p_m = ldx; a.p_k = 1;
-  a.Q = A16; a.q_k = 1; a.q_n = K;
+  SkinnyArgs a = out_args(u, R, 1, 1.f, 0, u16, 1, lora16_ld(T));
   a.M = T; a.N = R; a.K = K;
-  LSQ_TRY((run<true, true, PM_F16>(a, scratch, scratch_bytes, st)));
+  const Operand A{x, K, T, ldx, true}, B{A16, K, R, K, true};
+  LSQ_TRY((run<false, false>(a, A, B, true, scratch, scratch_bytes, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 2.0 * R * K);
   return LSQ_OK;
 }
@@ -492,13 +472,13 @@ int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t
                         float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
                         cudaStream_t st) {
   LSQ_TRY(check_ranks(R));
-  // C[t, c] = sum_n dy[t, n] Bs[n, c]   (bf16 operands; Bs block-diagonal over the parts)
+  if (N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_vproj: N %% 8 != 0");
+  // C[t, c] = sum_n dy[t, n] Bs^T[c, n]   (bf16 operands); v16 transposed [R][ld]
   const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(v, R, 1, 1.f, 0, v16, R);
-  a.P = dy; a.p_m = N; a.p_k = 1;
-  a.Q = Bs; a.q_k = R; a.q_n = 1;
+  SkinnyArgs a = out_args(v, R, 1, 1.f, 0, v16, 1, lora16_ld(T));
   a.M = T; a.N = R; a.K = N;
-  LSQ_TRY((run<true, false, PM_BF16>(a, scratch, scratch_bytes, st)));
+  const Operand A{dy, N, T, N, false}, B{Bs, N, R, N, false};
+  LSQ_TRY((run<false, false>(a, A, B, false, scratch, scratch_bytes, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_v", 2.0 * T * R * N, 2.0 * T * N + 2.0 * R * N);
   return LSQ_OK;
 }
@@ -507,13 +487,13 @@ int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int6
                          float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
                          cudaStream_t st) {
   LSQ_TRY(check_ranks(R));
-  // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]   (x rounded from fp16 to bf16)
+  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_a: K %% 8 != 0");
+  // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]   (x converted from fp16 to bf16)
   const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0);
-  a.P = x; a.p_m = 1; a.p_k = K;
-  a.Q = v16; a.q_k = R; a.q_n = 1;
+  SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0, 0);
   a.M = K; a.N = R; a.K = T;
-  LSQ_TRY((run<false, false, PM_P16>(a, scratch, scratch_bytes, st)));
+  const Operand A{x, K, T, K, true}, B{v16, T, R, lora16_ld(T), false};
+  LSQ_TRY((run<true, true>(a, A, B, false, scratch, scratch_bytes, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 2.0 * T * R);
   return LSQ_OK;
 }
@@ -524,19 +504,19 @@ int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int
   const int R = n_parts * r;
   LSQ_TRY(check_ranks(R));
   if (n_parts < 1 || n_parts > 4) return set_error(LSQ_ERR_SHAPE, "lora_grad_b: 1..4 parts");
+  if (N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_b: N %% 8 != 0");
   // C[n, c] = sum_t dy[t, n] u[t, c];  dB[n, j] (+)= s C[n, part(n) r + j]: one product over
   // all parts, each row keeping its own part's columns
   const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(dB, r, 1, s, accumulate, nullptr, 0);
-  a.P = dy; a.p_m = 1; a.p_k = N;
-  a.Q = u16; a.q_k = R; a.q_n = 1;
+  SkinnyArgs a = out_args(dB, r, 1, s, accumulate, nullptr, 0, 0);
   a.M = N; a.N = R; a.K = T;
   if (n_parts > 1) {
     a.part_r = r;
     a.n_parts = n_parts;
     for (int p = 0; p < n_parts; ++p) a.part_end[p] = part_end[p];
   }
-  LSQ_TRY((run<false, false, PM_BF16>(a, scratch, scratch_bytes, st)));
+  const Operand A{dy, N, T, N, false}, B{u16, T, R, lora16_ld(T), false};
+  LSQ_TRY((run<true, false>(a, A, B, false, scratch, scratch_bytes, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * R * N, 2.0 * T * N + 2.0 * T * R);
   return LSQ_OK;
 }
@@ -549,7 +529,8 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
   LSQ_TRY(check_ranks(R));
   Split sp;
   LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)R * K, &sp, "lora_down"));
-  LSQ_TRY(convert_rows(A, R, K, K, sp.q, K, st, /*f16=*/true));
+  to_f16_rows_kernel<<<grid_for_elems((int64_t)R * K), 256, 0, st>>>(A, R, K, K, sp.q, K);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return launch_lora_down16(x, ldx, sp.q, T, K, R, u, u16, sp.rest, sp.rest_bytes, st);
 }
 
@@ -558,7 +539,8 @@ int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, 
   LSQ_TRY(check_ranks(r));
   Split sp;
   LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)N * r, &sp, "lora_vproj"));
-  LSQ_TRY(convert_rows(B, N, r, r, sp.q, r, st));
+  to_bf16_transposed_kernel<<<grid_for_elems((int64_t)N * r), 256, 0, st>>>(B, N, r, sp.q);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return launch_lora_vproj16(dy, T, N, sp.q, r, v, v16, sp.rest, sp.rest_bytes, st);
 }
 
@@ -575,14 +557,15 @@ __global__ void lora_prepare_kernel(const float* __restrict__ lora, int64_t lora
     const int64_t n_el = g.rows * g.ld_out;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
          i += (int64_t)gridDim.x * blockDim.x) {
-      const int64_t row = i / g.ld_out, col = i % g.ld_out;
       if (g.kind == 0) {  // A: fp16 copy, [rows][cols]
+        const int64_t row = i / g.ld_out, col = i % g.ld_out;
         dst[g.dst_off + i] = float_to_f16_bits(src[g.src_off + row * g.cols + col]);
-      } else {            // B: bf16, block-diagonal [rows][n_parts r]
+      } else {            // B: bf16 block-diagonal stack, transposed: [n_parts r][rows]
+        const int64_t j = i / g.rows, row = i % g.rows;
         int p = 0;
         while (p + 1 < g.n_parts && row >= g.part_end[p]) ++p;
-        const int64_t j = col - (int64_t)p * g.cols;
-        const float v = (j >= 0 && j < g.cols) ? src[g.src_off + row * g.cols + j] : 0.f;
+        const int64_t jj = j - (int64_t)p * g.cols;
+        const float v = (jj >= 0 && jj < g.cols) ? src[g.src_off + row * g.cols + jj] : 0.f;
         dst[g.dst_off + i] = float_to_bf16_bits(v);
       }
     }
