@@ -21,9 +21,12 @@
 // range); dA's fp16 activation is converted to bf16 in shared memory as each
 // stage lands.  Accumulation is fp32 (the tutorial's part 1: the LoRA A/B
 // matrices are computed at a higher precision than the NF4 storage).  When a
-// product is split along its reduction, the slices are summed by a second
-// kernel in a fixed order, so results are deterministic (no atomics); an
-// unsplit product writes its result directly.
+// product is split along its reduction (into 2, 4 or 8 slices), the slices of a
+// tile run as one thread-block cluster: each copies its accumulator into its
+// shared memory, and after a cluster barrier each sums its share of the tile's
+// rows over the slices, in slice order, through distributed shared memory.  No
+// partials leave the SMs, no second kernel runs, and the results are
+// deterministic (no atomics).
 #include <cuda.h>
 #include <stdlib.h>
 
@@ -42,16 +45,14 @@ constexpr uint32_t kSAStage = kSM * kSK * 2;  // 16 KB
 
 struct SkinnyArgs {
   int64_t M, N, K;     // C is M x N, reduction over K
-  int kt_per_split;    // reduction stages (of 64) per split
-  float* part;         // [splits][M][N] when split
+  int splits;          // slices of the reduction = CTAs of a cluster (1, 2, 4 or 8); slice
+                       // z takes the stages [z kt / splits, (z + 1) kt / splits) of kt
   // unsplit: dst[m * c_m + n * c_n] = alpha * C[m, n] (+ dst if accumulate)
   float* dst;
   int64_t c_m, c_n;
   float alpha;
   int accumulate;
-  int direct;
-  // Output options (applied where the result is written: the direct epilogue or
-  // the slice sum): c16 (nullable) also receives the result rounded to bf16,
+  // Output options (applied where the result is written): c16 (nullable) also receives the result rounded to bf16,
   // c16[m * c16_m + n * c16_n], for the product that consumes it; with part_r >
   // 0 the rows are split into parts ending at part_end[], and row m of part p
   // keeps only columns [p part_r, (p + 1) part_r), written to column n - p part_r.
@@ -102,8 +103,8 @@ __global__ void __launch_bounds__(kSThreads, 1)
   const uint32_t st_bytes = kSAStage + ((b_bytes + 1023u) & ~1023u);
   const int64_t m0 = (int64_t)blockIdx.x * kSM;
   const int kt_total = (int)((a.K + kSK - 1) / kSK);
-  const int kt_begin = blockIdx.z * a.kt_per_split;
-  const int n_it = max(0, min(kt_total, kt_begin + a.kt_per_split) - kt_begin);
+  const int kt_begin = (int)((int64_t)blockIdx.z * kt_total / a.splits);
+  const int n_it = (int)((int64_t)(blockIdx.z + 1) * kt_total / a.splits) - kt_begin;
   const int S = stages;
 
   if (threadIdx.x == 0) {
@@ -194,40 +195,69 @@ __global__ void __launch_bounds__(kSThreads, 1)
   }
 
   // ------------------------------------------------------------------ epilogue
-  {
-    bool ok = true;
-    if (n_it > 0) {
-      ok = mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-    }
+  const int Z = a.splits;
+  bool ok = mbar_wait_bounded(smem_u32(&bar_acc), 0u, abort_flag, dev_err, DEV_ERR_WAIT_GEMM);
+  ok = __all_sync(0xFFFFFFFFu, ok);
+  tc_fence_after();
+  const int64_t nc = (int64_t)blockIdx.y * n_pad;  // first column of this CTA
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  if (Z == 1) {
     if (ok) {
-      tc_fence_after();
       const int64_t m = m0 + warp * 32 + lane;  // this thread's row (its TMEM lane)
-      const int64_t nc = (int64_t)blockIdx.y * n_pad;  // first column of this CTA
-      const bool mok = m < a.M;
-      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
       for (int n0 = 0; n0 < n_pad; n0 += 16) {
         uint32_t v[16];
-        if (n_it > 0) {
-          tmem_ld16(trow + (uint32_t)n0, v);
-          tmem_ld_wait();
-        } else {
+        tmem_ld16(trow + (uint32_t)n0, v);
+        tmem_ld_wait();
+        if (m >= a.M) continue;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0u;  // an empty slice contributes zeros
-        }
-        if (!mok) continue;
-        if (a.direct) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (nc + n0 + j < a.N) store_result(a, m, nc + n0 + j, __uint_as_float(v[j]));
-        } else {
-          float* pr = a.part + ((size_t)blockIdx.z * a.M + m) * a.N + nc;
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (nc + n0 + j < a.N) pr[n0 + j] = __uint_as_float(v[j]);
-        }
+        for (int j = 0; j < 16; ++j)
+          if (nc + n0 + j < a.N) store_result(a, m, nc + n0 + j, __uint_as_float(v[j]));
       }
     }
+  } else {
+    // The accumulator into this CTA's shared memory (the drained pipeline),
+    // [128 rows][n_pad + 4] fp32 ...
+    float* red = reinterpret_cast<float*>(st0);
+    const int ldr = n_pad + 4;
+    if (ok) {
+      const int row = warp * 32 + lane;
+      for (int n0 = 0; n0 < n_pad; n0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(trow + (uint32_t)n0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          *reinterpret_cast<float4*>(red + row * ldr + n0 + j) =
+              make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                          __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+      }
+    }
+    // ... then every slice of the tile sums its share of the rows over all
+    // slices, in slice order, through distributed shared memory.
+    cluster_sync_all();
+    const int cr = (int)cluster_ctarank();  // = this CTA's slice
+    const int rows = kSM / Z, n4 = n_pad / 4;
+    if (ok && !abort_sh) {
+      for (int e = threadIdx.x; e < rows * n4; e += kSThreads) {
+        const int row = cr * rows + e / n4, c4 = e % n4;
+        const int64_t m = m0 + row;
+        if (m >= a.M) continue;
+        const uint32_t off = smem_u32(red + row * ldr + 4 * c4);
+        float4 acc = ld_shared_cluster_f4(mapa_shared(off, 0));
+        for (int q = 1; q < Z; ++q) {
+          const float4 v = ld_shared_cluster_f4(mapa_shared(off, (uint32_t)q));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const float r4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (nc + 4 * c4 + j < a.N) store_result(a, m, nc + 4 * c4 + j, r4[j]);
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while another reads its shared memory
   }
   tc_fence_before();
   __syncthreads();
@@ -235,21 +265,6 @@ __global__ void __launch_bounds__(kSThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
-  }
-}
-
-// sum_z part[z][m][n] in z order, written as SkinnyArgs a prescribes (store_result)
-__global__ void split_sum_kernel(const float* __restrict__ part, int splits, const SkinnyArgs a) {
-  const int64_t M = a.M, N = a.N;
-  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  const int64_t n_el = M * N;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_el;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    float s = 0.f;
-    // unrolled so that several slices' loads are in flight; the adds stay in z order
-#pragma unroll 8
-    for (int z = 0; z < splits; ++z) s += part[(size_t)z * n_el + i];
-    store_result(a, i / N, i % N, s);
   }
 }
 
@@ -290,18 +305,19 @@ int stages_for(int) { return 4; }
 size_t smem_for(int n_pad) { return 1024 + (size_t)stages_for(n_pad) * stage_bytes(n_pad); }
 int ctas_per_sm(int n_pad) { return smem_for(n_pad) <= 110 * 1024 ? 2 : 1; }
 
-// Splits of the reduction: only where the product's own row tiles leave at least
-// half of the resident CTA slots empty, up to filling them, each slice at least
-// two stages long.
+// Splits of the reduction (a cluster of 2, 4 or 8 CTAs per tile): only where the
+// product's own tiles leave at least half of the resident CTA slots empty, up to
+// filling them, each slice at least two stages long.
 int splits_for(int64_t M, int64_t N, int64_t K) {
   if (K <= 0 || M <= 0 || N <= 0) return 1;
   const int64_t tiles = (M + kSM - 1) / kSM * ((N + kSMaxN - 1) / kSMaxN);
   const int64_t slots = (int64_t)kSMs * ctas_per_sm(npad_for(N));
   if (tiles * 2 > slots) return 1;
   const int64_t kt = (K + kSK - 1) / kSK;
-  int64_t z = std::max<int64_t>(1, std::min<int64_t>(slots / tiles, std::min<int64_t>(kt / 2, 64)));
-  const int64_t kps = (kt + z - 1) / z;
-  return (int)((kt + kps - 1) / kps);
+  const int64_t cap = std::min<int64_t>(8, std::min<int64_t>(slots / tiles, kt / 2));
+  int z = 1;
+  while (z * 2 <= cap) z *= 2;
+  return z;
 }
 
 template <bool A_MN, bool CONV>
@@ -326,11 +342,15 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const SkinnyArgs& a,
   cfg.blockDim = dim3(kSThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;  // the slices of a tile
+  at[1].val.clusterDim.x = 1;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = (unsigned)a.splits;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(&cfg, tc_skinny_kernel<A_MN, CONV>, ta, tb, a, idesc,
                                               n_pad, stages_for(n_pad), cols, dev_err)));
   return LSQ_OK;
@@ -344,22 +364,15 @@ struct Operand {
 };
 
 // C = A B^T over K (A: M x K, K-major unless A_MN; B: N x K, K-major), written as
-// a prescribes (dst, alpha, accumulate, c16, parts); scratch holds the fixed-order
-// partials when the product is split.  CONV: A is fp16 and meets a bf16 B.
+// a prescribes (dst, alpha, accumulate, c16, parts).  CONV: A is fp16 and meets a
+// bf16 B.
 template <bool A_MN, bool CONV>
-int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, float* scratch,
-        size_t scratch_bytes, cudaStream_t st) {
+int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return LSQ_OK;
   if (a.K <= 0) return set_error(LSQ_ERR_SHAPE, "lora product: empty reduction");
   const int n_pad = npad_for(a.N);
-  const int z = splits_for(a.M, a.N, a.K);
-  const size_t need = z > 1 ? (size_t)z * a.M * a.N * sizeof(float) : 0;
-  if (need && (!scratch || scratch_bytes < need))
-    return set_error(LSQ_ERR_WORKSPACE, "lora product: scratch %zu < %zu", scratch_bytes, need);
-  const int kt = (int)((a.K + kSK - 1) / kSK);
-  a.kt_per_split = std::max(1, (kt + z - 1) / z);
-  a.direct = z == 1;
-  a.part = z > 1 ? scratch : nullptr;
+  const int z = splits_for(a.M, a.N, a.K);  // every slice gets at least two stages
+  a.splits = z;
   CUtensorMap ta, tb;
   const CUtensorMapDataType dta = A.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapDataType dtb = B.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -370,14 +383,8 @@ int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, float* scrat
   uint32_t idesc = f16 ? umma_idesc_f16(kSM, n_pad) : umma_idesc_bf16(kSM, n_pad);
   if (A_MN) idesc |= 1u << 15;  // A MN-major
   const dim3 grid((unsigned)((a.M + kSM - 1) / kSM), (unsigned)((a.N + n_pad - 1) / n_pad),
-                  (unsigned)((kt + a.kt_per_split - 1) / a.kt_per_split));
-  LSQ_TRY((launch_tc<A_MN, CONV>(ta, tb, a, idesc, n_pad, grid, st)));
-  if (z == 1) return LSQ_OK;
-  int64_t g = (a.M * a.N + 255) / 256;
-  if (g > kSMs * 8) g = kSMs * 8;
-  split_sum_kernel<<<(unsigned)g, 256, 0, st>>>(a.part, (int)grid.z, a);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return LSQ_OK;
+                  (unsigned)z);
+  return launch_tc<A_MN, CONV>(ta, tb, a, idesc, n_pad, grid, st);
 }
 
 int check_ranks(int64_t R) {
@@ -404,8 +411,7 @@ SkinnyArgs out_args(float* dst, int64_t c_m, int64_t c_n, float alpha, int accum
   return a;
 }
 
-// 16-bit copies of fp32 LoRA operands, at the start of the scratch; returns the
-// scratch left for the partials.
+// 16-bit copies of fp32 LoRA operands, at the start of the scratch.
 struct Split {
   uint16_t* q;
   float* rest;
@@ -432,25 +438,10 @@ unsigned grid_for_elems(int64_t n) {
 int64_t lora16_ld(int64_t T) { return (T + 7) / 8 * 8; }
 
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
-  // An upper bound over every product a caller sizing by (T, K, R) can make:
-  // any width R' <= R (a multiple of 8), and
-  //   u = x A^T, v      M = T, N = R', reduction <= K
-  //   dA, dB            M <= K, N = R', reduction T
-  // The split count never exceeds the CTA slots over the row tiles, so z M is at
-  // most slots x 128 (or z = 1).  The 16-bit copy of an fp32 LoRA operand
-  // (R x K elements) comes first.
-  size_t best = 0;
-  for (int rr = 8; rr <= std::max(8, R); rr += 8) {
-    const int64_t slots = (int64_t)kSMs * ctas_per_sm(npad_for(rr));
-    const int z1 = splits_for(T, rr, K);
-    const size_t p1 = z1 > 1 ? (size_t)z1 * T * rr * sizeof(float) : 0;
-    int64_t zm = 0;  // the largest z M over M <= K for the reduction over T
-    const int64_t kt = (T + kSK - 1) / kSK;
-    if (kt >= 4) zm = std::min<int64_t>(slots * kSM, std::min<int64_t>(64, kt / 2) * K);
-    const size_t p2 = (size_t)zm * rr * sizeof(float);
-    best = std::max(best, align256((size_t)K * rr * 2) + std::max(p1, p2));
-  }
-  return best;
+  // The 16-bit copy of an fp32 LoRA operand (R x K elements, the fp32-operand
+  // forms); the split products need none (their slices meet in shared memory).
+  (void)T;
+  return align256((size_t)std::max(R, 8) * std::max<int64_t>(K, 1) * 2);
 }
 
 int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
@@ -463,7 +454,7 @@ int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int6
   SkinnyArgs a = out_args(u, R, 1, 1.f, 0, u16, 1, lora16_ld(T));
   a.M = T; a.N = R; a.K = K;
   const Operand A{x, K, T, ldx, true}, B{A16, K, R, K, true};
-  LSQ_TRY((run<false, false>(a, A, B, true, scratch, scratch_bytes, st)));
+  LSQ_TRY((run<false, false>(a, A, B, true, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_u", 2.0 * T * R * K, 2.0 * T * K + 2.0 * R * K);
   return LSQ_OK;
 }
@@ -478,7 +469,7 @@ int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t
   SkinnyArgs a = out_args(v, R, 1, 1.f, 0, v16, 1, lora16_ld(T));
   a.M = T; a.N = R; a.K = N;
   const Operand A{dy, N, T, N, false}, B{Bs, N, R, N, false};
-  LSQ_TRY((run<false, false>(a, A, B, false, scratch, scratch_bytes, st)));
+  LSQ_TRY((run<false, false>(a, A, B, false, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_v", 2.0 * T * R * N, 2.0 * T * N + 2.0 * R * N);
   return LSQ_OK;
 }
@@ -493,7 +484,7 @@ int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int6
   SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0, 0);
   a.M = K; a.N = R; a.K = T;
   const Operand A{x, K, T, K, true}, B{v16, T, R, lora16_ld(T), false};
-  LSQ_TRY((run<true, true>(a, A, B, false, scratch, scratch_bytes, st)));
+  LSQ_TRY((run<true, true>(a, A, B, false, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 2.0 * T * R);
   return LSQ_OK;
 }
@@ -516,7 +507,7 @@ int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int
     for (int p = 0; p < n_parts; ++p) a.part_end[p] = part_end[p];
   }
   const Operand A{dy, N, T, N, false}, B{u16, T, R, lora16_ld(T), false};
-  LSQ_TRY((run<true, false>(a, A, B, false, scratch, scratch_bytes, st)));
+  LSQ_TRY((run<true, false>(a, A, B, false, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * R * N, 2.0 * T * N + 2.0 * T * R);
   return LSQ_OK;
 }
