@@ -196,6 +196,139 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const float* __
   }
 }
 
+// RMSNorm of a split product's output: x_out = (sum of the n_parts partials, in
+// slice order) + res, then y = RMSNorm(x_out) - the same sums, in the same order,
+// as launch_splitk_reduce followed by rmsnorm_fwd_kernel (same thread mapping).
+// The summed row is staged in shared memory (D floats) for the second pass.
+template <bool F16OUT>
+__global__ void rmsnorm_fwd_sum_kernel(const float* __restrict__ parts, int n_parts,
+                                       int64_t pstride, const float* __restrict__ res, int64_t D,
+                                       float eps, const uint16_t* __restrict__ g,
+                                       float* __restrict__ xo, uint16_t* __restrict__ y,
+                                       float* __restrict__ rstd, int* dev_err) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
+  extern __shared__ float4 row_sh[];
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const int nv = (int)(D / 8);
+  float ss = 0.f;
+  bool big = false;
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+    const int64_t e = row * D + 8 * (int64_t)i;
+    float4 a = *reinterpret_cast<const float4*>(parts + e);
+    float4 b = *reinterpret_cast<const float4*>(parts + e + 4);
+    for (int s = 1; s < n_parts; ++s) {
+      const float4 pa = *reinterpret_cast<const float4*>(parts + (size_t)s * pstride + e);
+      const float4 pb = *reinterpret_cast<const float4*>(parts + (size_t)s * pstride + e + 4);
+      a.x += pa.x; a.y += pa.y; a.z += pa.z; a.w += pa.w;
+      b.x += pb.x; b.y += pb.y; b.z += pb.z; b.w += pb.w;
+    }
+    if (res) {
+      const float4 ra = *reinterpret_cast<const float4*>(res + e);
+      const float4 rb = *reinterpret_cast<const float4*>(res + e + 4);
+      a.x += ra.x; a.y += ra.y; a.z += ra.z; a.w += ra.w;
+      b.x += rb.x; b.y += rb.y; b.z += rb.z; b.w += rb.w;
+    }
+    *reinterpret_cast<float4*>(xo + e) = a;
+    *reinterpret_cast<float4*>(xo + e + 4) = b;
+    row_sh[2 * i] = a;
+    row_sh[2 * i + 1] = b;
+    ss = fmaf(a.x, a.x, ss);
+    ss = fmaf(a.y, a.y, ss);
+    ss = fmaf(a.z, a.z, ss);
+    ss = fmaf(a.w, a.w, ss);
+    ss = fmaf(b.x, b.x, ss);
+    ss = fmaf(b.y, b.y, ss);
+    ss = fmaf(b.z, b.z, ss);
+    ss = fmaf(b.w, b.w, ss);
+  }
+  ss = block_sum(ss, red);  // (its barriers also publish row_sh)
+  const float r = rsqrtf(ss / (float)D + eps);
+  if (threadIdx.x == 0 && rstd) rstd[row] = r;
+  const uint4* gr = reinterpret_cast<const uint4*>(g);
+  uint4* yr = reinterpret_cast<uint4*>(y + row * D);
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+    const float4 a = row_sh[2 * i], b = row_sh[2 * i + 1];
+    const uint4 gv = gr[i];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 gg = unpack_bf16x2(gw[q]);
+      const float y0 = f[2 * q] * r * gg.x, y1 = f[2 * q + 1] * r * gg.y;
+      if (F16OUT) {
+        big |= !(fmaxf(fabsf(y0), fabsf(y1)) <= kF16Max);
+        o[q] = pack_f16x2(y0, y1);
+      } else {
+        o[q] = pack_bf16x2(y0, y1);
+      }
+    }
+    yr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (F16OUT && big) atomicOr(dev_err, DEV_ERR_NONFINITE);
+}
+
+// rmsnorm_bwd_kernel with dy the sum of a split product's partials (slice order),
+// staged in shared memory (D floats) for the second pass.
+__global__ void rmsnorm_bwd_sum_kernel(const float* __restrict__ parts, int n_parts,
+                                       int64_t pstride, const float* __restrict__ x,
+                                       const uint16_t* __restrict__ g,
+                                       const float* __restrict__ rstd,
+                                       const float* __restrict__ dres, int64_t D,
+                                       float* __restrict__ dx, uint16_t* __restrict__ dxb) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
+  extern __shared__ float4 row_sh[];
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const int nv = (int)(D / 4);
+  const float4* xr = reinterpret_cast<const float4*>(x + row * D);
+  const uint2* gr = reinterpret_cast<const uint2*>(g);
+  float dot = 0.f;
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+    const int64_t e = row * D + 4 * (int64_t)i;
+    float4 d = *reinterpret_cast<const float4*>(parts + e);
+    for (int s = 1; s < n_parts; ++s) {
+      const float4 p = *reinterpret_cast<const float4*>(parts + (size_t)s * pstride + e);
+      d.x += p.x; d.y += p.y; d.z += p.z; d.w += p.w;
+    }
+    row_sh[i] = d;
+    const float4 xv = xr[i];
+    const uint2 gv = gr[i];
+    const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
+    dot += d.x * g0.x * xv.x + d.y * g0.y * xv.y + d.z * g1.x * xv.z + d.w * g1.y * xv.w;
+  }
+  dot = block_sum(dot, red);  // (its barriers also publish row_sh)
+  const float r = rstd[row];
+  const float c = r * r * r * dot / (float)D;
+  const float4* rr = dres ? reinterpret_cast<const float4*>(dres + row * D) : nullptr;
+  float4* o = reinterpret_cast<float4*>(dx + row * D);
+  for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+    const float4 d = row_sh[i], xv = xr[i];
+    const uint2 gv = gr[i];
+    const float2 g0 = unpack_bf16x2(gv.x), g1 = unpack_bf16x2(gv.y);
+    float4 v;
+    v.x = r * g0.x * d.x - xv.x * c;
+    v.y = r * g0.y * d.y - xv.y * c;
+    v.z = r * g1.x * d.z - xv.z * c;
+    v.w = r * g1.y * d.w - xv.w * c;
+    if (rr) {
+      const float4 a = rr[i];
+      v.x += a.x;
+      v.y += a.y;
+      v.z += a.z;
+      v.w += a.w;
+    }
+    o[i] = v;
+    if (dxb) {
+      uint2 b;
+      b.x = pack_bf16x2(v.x, v.y);
+      b.y = pack_bf16x2(v.z, v.w);
+      reinterpret_cast<uint2*>(dxb + row * D)[i] = b;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ RoPE
 // cs[pos][i] = (cos, sin)(pos * theta^(-2i/d)), evaluated in double, rounded to fp32.
 __global__ void rope_table_kernel(int seq, int half, int d, double log_theta, float2* __restrict__ cs) {
@@ -241,6 +374,78 @@ __global__ void rope_kernel(uint16_t* __restrict__ qkv, int64_t T, int seq, int 
     *reinterpret_cast<uint4*>(base) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
     *reinterpret_cast<uint4*>(base + half) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
   }
+}
+
+// The fused q|k|v product's partials summed (slice order) and rounded to fp16 -
+// as launch_splitk_reduce writes them - then the q and k heads rotated as
+// rope_kernel does; the v heads only summed.  Items [0, n_rot): 8 rotation
+// pairs of a q or k head; the rest: 8 consecutive values of a v head.
+__global__ void reduce_rope_kernel(const float* __restrict__ parts, int n_parts, int64_t T,
+                                   int seq, int H, int Hkv, int d,
+                                   const float2* __restrict__ cs, uint16_t* __restrict__ qkv,
+                                   int* dev_err) {
+  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
+  const int half = d / 2, chunks = half / 8;
+  const int64_t ld = (int64_t)(H + 2 * Hkv) * d;
+  const int64_t pstride = T * ld;
+  const int64_t n_rot = T * (H + Hkv) * chunks;
+  const int vq = Hkv * d / 8;  // 8-value groups of the v heads per token
+  const int64_t n = n_rot + T * vq;
+  auto sum8 = [&](int64_t e, float* f) {
+    float4 a = *reinterpret_cast<const float4*>(parts + e);
+    float4 b = *reinterpret_cast<const float4*>(parts + e + 4);
+    for (int s = 1; s < n_parts; ++s) {
+      const float4 pa = *reinterpret_cast<const float4*>(parts + (size_t)s * pstride + e);
+      const float4 pb = *reinterpret_cast<const float4*>(parts + (size_t)s * pstride + e + 4);
+      a.x += pa.x; a.y += pa.y; a.z += pa.z; a.w += pa.w;
+      b.x += pb.x; b.y += pb.y; b.z += pb.z; b.w += pb.w;
+    }
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  };
+  bool big = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < n_rot) {
+      const int ch = (int)(i % chunks);
+      const int64_t th = i / chunks;
+      const int head = (int)(th % (H + Hkv));
+      const int64_t t = th / (H + Hkv);
+      const int pos = (int)(t % seq);
+      const int64_t e = t * ld + (int64_t)head * d + ch * 8;
+      float f1[8], f2[8];
+      sum8(e, f1);
+      sum8(e + half, f2);
+      const float2* c = cs + (int64_t)pos * half + ch * 8;
+      uint32_t oa[4], ob[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        big |= !(fmaxf(fmaxf(fabsf(f1[2 * q]), fabsf(f1[2 * q + 1])),
+                       fmaxf(fabsf(f2[2 * q]), fabsf(f2[2 * q + 1]))) <= kF16Max);
+        const float2 x1 = unpack_f16x2(pack_f16x2(f1[2 * q], f1[2 * q + 1]));
+        const float2 x2 = unpack_f16x2(pack_f16x2(f2[2 * q], f2[2 * q + 1]));
+        const float2 c0 = c[2 * q], c1 = c[2 * q + 1];
+        oa[q] = pack_f16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
+        ob[q] = pack_f16x2(x2.x * c0.x + x1.x * c0.y, x2.y * c1.x + x1.y * c1.y);
+      }
+      *reinterpret_cast<uint4*>(qkv + e) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+      *reinterpret_cast<uint4*>(qkv + e + half) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    } else {
+      const int64_t j = i - n_rot;
+      const int64_t t = j / vq;
+      const int64_t e = t * ld + (int64_t)(H + Hkv) * d + (j % vq) * 8;
+      float f[8];
+      sum8(e, f);
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        big |= !(fmaxf(fabsf(f[2 * q]), fabsf(f[2 * q + 1])) <= kF16Max);
+        o[q] = pack_f16x2(f[2 * q], f[2 * q + 1]);
+      }
+      *reinterpret_cast<uint4*>(qkv + e) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (big) atomicOr(dev_err, DEV_ERR_NONFINITE);
 }
 
 // dqkv (bf16) <- [rope^-1(dq), rope^-1(dk), dv].  dq is fp32 [T, H d]; dk and dv
@@ -539,6 +744,84 @@ int launch_rmsnorm_bwd(const float* dy, const float* x, const uint16_t* g, const
   if (prof >= 0)
     prof_end(prof, st, "rmsnorm_bwd", 0.0,
              (12.0 + (dres ? 4.0 : 0.0) + (dx_bf16 ? 2.0 : 0.0)) * T * D + 2.0 * D + 4.0 * T);
+  return LSQ_OK;
+}
+
+int launch_rmsnorm_fwd_sum(const float* parts, int n_parts, const float* res, int64_t T,
+                           int64_t D, float* x_out, const uint16_t* g, float eps, uint16_t* y,
+                           int y_kind, float* rstd, cudaStream_t st) {
+  if (n_parts < 1 || D % 8 != 0) return set_error(LSQ_ERR_SHAPE, "rmsnorm_fwd_sum: bad shape");
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  const size_t smem = (size_t)D * sizeof(float);
+  if (smem > 48 * 1024) {
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[dev]) {
+      LSQ_CUDA(cudaFuncSetAttribute(rmsnorm_fwd_sum_kernel<true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      LSQ_CUDA(cudaFuncSetAttribute(rmsnorm_fwd_sum_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      attr[dev] = true;
+    }
+    if (smem > 200 * 1024) return set_error(LSQ_ERR_SHAPE, "rmsnorm_fwd_sum: row too long");
+  }
+  const int prof = prof_begin(st);
+  const int64_t ps = T * D;
+  if (y_kind == OUT_F16)
+    rmsnorm_fwd_sum_kernel<true><<<(unsigned)T, threads_for_row(D, 8), smem, st>>>(
+        parts, n_parts, ps, res, D, eps, g, x_out, y, rstd, dev_err);
+  else
+    rmsnorm_fwd_sum_kernel<false><<<(unsigned)T, threads_for_row(D, 8), smem, st>>>(
+        parts, n_parts, ps, res, D, eps, g, x_out, y, rstd, dev_err);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // the product's output read once (as if reduced), the residual, x_out and y written
+  if (prof >= 0)
+    prof_end(prof, st, "rmsnorm_fwd", 0.0,
+             (4.0 + (res ? 4.0 : 0.0) + 4.0 + 2.0) * T * D + 2.0 * D + 4.0 * T);
+  return LSQ_OK;
+}
+
+int launch_rmsnorm_bwd_sum(const float* parts, int n_parts, const float* x, const uint16_t* g,
+                           const float* rstd, const float* dres, int64_t T, int64_t D, float* dx,
+                           uint16_t* dx_bf16, cudaStream_t st) {
+  if (n_parts < 1 || D % 4 != 0) return set_error(LSQ_ERR_SHAPE, "rmsnorm_bwd_sum: bad shape");
+  const size_t smem = (size_t)D * sizeof(float);
+  if (smem > 48 * 1024) {
+    static bool attr[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[dev]) {
+      LSQ_CUDA(cudaFuncSetAttribute(rmsnorm_bwd_sum_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      attr[dev] = true;
+    }
+    if (smem > 200 * 1024) return set_error(LSQ_ERR_SHAPE, "rmsnorm_bwd_sum: row too long");
+  }
+  const int prof = prof_begin(st);
+  rmsnorm_bwd_sum_kernel<<<(unsigned)T, threads_for_row(D, 4), smem, st>>>(
+      parts, n_parts, T * D, x, g, rstd, dres, D, dx, dx_bf16);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  if (prof >= 0)
+    prof_end(prof, st, "rmsnorm_bwd", 0.0,
+             (12.0 + (dres ? 4.0 : 0.0) + (dx_bf16 ? 2.0 : 0.0)) * T * D + 2.0 * D + 4.0 * T);
+  return LSQ_OK;
+}
+
+int launch_reduce_rope(const float* parts, int n_parts, int64_t T, int seq, int H, int Hkv, int d,
+                       const float2* cs, uint16_t* qkv, cudaStream_t st) {
+  if (n_parts < 1 || d % 16 != 0) return set_error(LSQ_ERR_SHAPE, "reduce_rope: bad shape");
+  int* dev_err = device_status_ptr();
+  if (!dev_err) return set_error(LSQ_ERR_CUDA, "device status word unavailable");
+  const int64_t n = T * (H + Hkv) * (d / 16) + T * Hkv * (d / 8);
+  const int prof = prof_begin(st);
+  reduce_rope_kernel<<<grid_for(n, 256), 256, 0, st>>>(parts, n_parts, T, seq, H, Hkv, d, cs, qkv,
+                                                       dev_err);
+  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
+  // the product's output read once (fp32, as if reduced), q|k|v written (fp16), the table
+  if (prof >= 0)
+    prof_end(prof, st, "rope", 0.0, 6.0 * T * (H + 2 * Hkv) * d + 4.0 * seq * d);
   return LSQ_OK;
 }
 

@@ -1015,7 +1015,9 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
       break;
     default: return set_error(LSQ_ERR_INVALID, "gemm: bad operand mode");
   }
-  if (pl.splits > 1)
+  if (d.splits_out) *d.splits_out = pl.splits;
+  if (d.parts_out) *d.parts_out = pl.splits > 1 ? partial : nullptr;
+  if (pl.splits > 1 && !d.parts_out)
     LSQ_TRY(launch_splitk_reduce(partial, pl.splits, d.T, d.M, d.out,
                                  d.out_f32 ? OUT_F32 : (wmode_f16(d.wmode) ? OUT_F16 : OUT_BF16),
                                  d.ldo, d.residual, d.ldr, st));

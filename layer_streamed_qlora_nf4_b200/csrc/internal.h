@@ -127,6 +127,13 @@ struct GemmDesc {
   int64_t ldr = 0;
   int force_splits = 0;             // 0 = heuristic
   const char* prof_name = nullptr;  // profiler class (default: by operand mode)
+  // Partials left to the next kernel: with parts_out set, a product split over K
+  // skips its reduce and reports the fp32 partials ([splits][T][M], in the
+  // workspace, valid until the next GEMM on it) and their count; an unsplit
+  // product writes out as usual and reports 1.  The residual is then the
+  // consumer's to add.
+  const float** parts_out = nullptr;
+  int* splits_out = nullptr;
 };
 size_t gemm_workspace_bytes(const GemmDesc& d);
 int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st);
@@ -135,6 +142,19 @@ int gemm_num_sms();
 // ---------------------------------------------------------------- small kernels
 // Output kinds of a reduce or normalisation kernel.
 enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_F16 = 2 };
+// Kernels that take a split product's partials (n_parts slices T * width apart,
+// summed in slice order, then the residual, as launch_splitk_reduce would):
+//   launch_rmsnorm_fwd_sum: x_out = sum + res (fp32), y = RMSNorm(x_out), rstd;
+//   launch_rmsnorm_bwd_sum: launch_rmsnorm_bwd with dy = the sum;
+//   launch_reduce_rope: qkv (fp16) = the sum rounded to fp16, q and k heads rotated.
+int launch_rmsnorm_fwd_sum(const float* parts, int n_parts, const float* res, int64_t T,
+                           int64_t D, float* x_out, const uint16_t* g, float eps, uint16_t* y,
+                           int y_kind, float* rstd, cudaStream_t st);
+int launch_rmsnorm_bwd_sum(const float* parts, int n_parts, const float* x, const uint16_t* g,
+                           const float* rstd, const float* dres, int64_t T, int64_t D, float* dx,
+                           uint16_t* dx_bf16, cudaStream_t st);
+int launch_reduce_rope(const float* parts, int n_parts, int64_t T, int seq, int H, int Hkv, int d,
+                       const float2* cs, uint16_t* qkv, cudaStream_t st);
 int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
                          int out_kind, int64_t ldo, const float* residual, int64_t ldr,
                          cudaStream_t st);
@@ -255,10 +275,15 @@ size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T);
 // rope_cs: the cos/sin table of launch_rope_table for this seq, or null (then the
 // layer builds it in its workspace); lora16: this layer's LoRA operands rounded by
 // prepare_lora16, or null (then the layer rounds its masters in its workspace)
+// saved_u (layer_saved_u_bytes, 256-byte aligned): where the forward leaves this
+// layer's rank-r products u = x A^T, and from where the backward of the same
+// inputs reads them instead of recomputing them; null in both keeps them in the
+// workspace and recomputes them.
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
                    cudaStream_t st, const float2* rope_cs = nullptr,
-                   const uint16_t* lora16 = nullptr);
+                   const uint16_t* lora16 = nullptr, void* saved_u = nullptr);
+size_t layer_saved_u_bytes(const lsq_cfg* cfg, int64_t T);
 // The LoRA operands of one layer in their product types (fp16 A, bf16 block-
 // diagonal B stacks): elements per layer, and the rounding of n_layers
 // consecutive LoRA blocks into out (that many elements apart).
@@ -269,6 +294,6 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate,
                    void* ws, size_t ws_bytes, cudaStream_t st, const float2* rope_cs = nullptr,
-                   const uint16_t* lora16 = nullptr);
+                   const uint16_t* lora16 = nullptr, const void* saved_u = nullptr);
 
 }  // namespace lsq

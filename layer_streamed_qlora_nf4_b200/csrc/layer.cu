@@ -394,6 +394,36 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   return a.used;
 }
 
+// The rank-r products u = x A^T of one forward (fp32 [T][R] per projection group,
+// read by the GEMMs' LoRA slab, and their bf16 [R][lora16_ld(T)] copies, read by
+// dB), carved from a region the caller keeps from the forward to the backward.
+size_t carve_saved_u(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
+  Arena a;
+  a.base = static_cast<uint8_t*>(base);
+  a.cap = SIZE_MAX;
+  const int r = s.r;
+  const int64_t t16 = lora16_ld(T);
+  float* u_qkv = a.take<float>(T * 3 * r);
+  float* u_o = a.take<float>(T * r);
+  float* u_gu = a.take<float>(T * 2 * r);
+  float* u_d = a.take<float>(T * r);
+  uint16_t* u16_qkv = a.take<uint16_t>(t16 * 3 * r);
+  uint16_t* u16_o = a.take<uint16_t>(t16 * r);
+  uint16_t* u16_gu = a.take<uint16_t>(t16 * 2 * r);
+  uint16_t* u16_d = a.take<uint16_t>(t16 * r);
+  if (b && base) {
+    b->u_qkv = u_qkv;
+    b->u_o = u_o;
+    b->u_gu = u_gu;
+    b->u_d = u_d;
+    b->u16_qkv = u16_qkv;
+    b->u16_o = u16_o;
+    b->u16_gu = u16_gu;
+    b->u16_d = u16_d;
+  }
+  return a.used;
+}
+
 // Points v at this layer's LoRA operands in product types: the given lora16, or
 // (lora16 null) the masters rounded into the workspace first.
 int attach_lora16(const LayerShapes& s, const float* lora, const uint16_t* lora16,
@@ -435,35 +465,51 @@ int check_layer_args(const lsq_cfg* cfg, const void* blob, const float* lora, co
 // when x_out is given, the down projection with its residual.
 int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch, int seq,
                  const float2* rope_cs, float eps, const Buffers& b, float* x_out,
-                 cudaStream_t st) {
+                 cudaStream_t st, bool have_u = false) {
   const int64_t T = (int64_t)batch * seq;
   const int r = v.lora_on ? s.r : 0;  // r = 0: no LoRA slab in the GEMMs
+  const bool down = v.lora_on && !have_u;  // compute u = x A^T here
   const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
   const int64_t pe2[2] = {s.F, s.gu_n};
   LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, OUT_F16, b.rstd1, st));
-  if (v.lora_on)
+  if (down)
     LSQ_TRY(launch_lora_down16(b.n1, s.D, v.A16_qkv, T, s.D, 3 * r, b.u_qkv, b.u16_qkv, b.lscratch,
                                b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s, b.u_qkv,
-                           3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n),
-                   b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, rope_cs, st));
+  // A product split over K leaves its partials to the kernel after it (RoPE here,
+  // the second RMSNorm after the o projection), which sums them in slice order.
+  const float* parts = nullptr;
+  int np = 1;
+  GemmDesc g_qkv = nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s,
+                           b.u_qkv, 3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n);
+  g_qkv.parts_out = &parts;
+  g_qkv.splits_out = &np;
+  LSQ_TRY(gemm_run(g_qkv, b.gemm, b.gemm_bytes, st));
+  if (np > 1)
+    LSQ_TRY(launch_reduce_rope(parts, np, T, seq, s.H, s.Hkv, s.hd, rope_cs, b.qkv, st));
+  else
+    LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
-  if (v.lora_on)
+  if (down)
     LSQ_TRY(launch_lora_down16(b.ao, s.qd, v.A16_o, T, s.qd, r, b.u_o, b.u16_o, b.lscratch,
                                b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
-                           pe3, x, b.h, s.D),
-                   b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, OUT_F16, b.rstd2, st));
-  if (v.lora_on)
+  GemmDesc g_o = nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
+                         pe3, x, b.h, s.D);
+  g_o.parts_out = &parts;
+  g_o.splits_out = &np;
+  LSQ_TRY(gemm_run(g_o, b.gemm, b.gemm_bytes, st));
+  if (np > 1)
+    LSQ_TRY(launch_rmsnorm_fwd_sum(parts, np, x, T, s.D, b.h, v.g2, eps, b.n2, OUT_F16, b.rstd2,
+                                   st));
+  else
+    LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, OUT_F16, b.rstd2, st));
+  if (down)
     LSQ_TRY(launch_lora_down16(b.n2, s.D, v.A16_gu, T, s.D, 2 * r, b.u_gu, b.u16_gu, b.lscratch,
                                b.lscratch_bytes, st));
   LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
                            2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_swiglu_fwd(b.gu, T, s.F, b.m, st));
-  if (v.lora_on)
+  if (down)
     LSQ_TRY(launch_lora_down16(b.m, s.F, v.A16_d, T, s.F, r, b.u_d, b.u16_d, b.lscratch,
                                b.lscratch_bytes, st));
   if (x_out)
@@ -493,6 +539,12 @@ int prepare_lora16(const lsq_cfg* cfg, const float* lora, int n_layers, uint16_t
                              lora16_segs(s, R, o), st);
 }
 
+size_t layer_saved_u_bytes(const lsq_cfg* cfg, int64_t T) {
+  LayerShapes s;
+  if (layer_shapes(cfg, &s) != LSQ_OK || T <= 0) return 0;
+  return carve_saved_u(s, T, nullptr, nullptr);
+}
+
 size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
   LayerShapes s;
   if (layer_shapes(cfg, &s) != LSQ_OK || T <= 0) return 0;
@@ -501,7 +553,8 @@ size_t layer_ws_bytes(const lsq_cfg* cfg, int64_t T) {
 
 int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, const float* x_in,
                    int batch, int seq, float* x_out, void* ws, size_t ws_bytes,
-                   cudaStream_t st, const float2* rope_cs, const uint16_t* lora16) {
+                   cudaStream_t st, const float2* rope_cs, const uint16_t* lora16,
+                   void* saved_u) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, x_out, &s, "decoder_layer_fwd",
                            true));
@@ -511,6 +564,7 @@ int layer_fwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     return set_error(LSQ_ERR_WORKSPACE, "decoder_layer_fwd: workspace %zu < %zu", ws_bytes, need);
   Buffers b;
   plan_buffers(s, T, ws, &b);
+  if (saved_u && lora) carve_saved_u(s, T, saved_u, &b);  // u written where the backward finds it
   Views v = views(s, blob, lora);
   LSQ_TRY(attach_lora16(s, lora, lora16, b, &v, st));
   if (!rope_cs) {
@@ -524,7 +578,7 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
                    const float* dx_out, const uint16_t* dx_out_bf16, int batch, int seq,
                    float* dx_in, uint16_t* dx_in_bf16, float* lora_grad, int accumulate, void* ws,
                    size_t ws_bytes, cudaStream_t st, const float2* rope_cs,
-                   const uint16_t* lora16) {
+                   const uint16_t* lora16, const void* saved_u) {
   LayerShapes s;
   LSQ_TRY(check_layer_args(cfg, blob, lora, x_in, batch, seq, dx_in, &s, "decoder_layer_bwd"));
   if (!dx_out || !lora_grad) return set_error(LSQ_ERR_INVALID, "decoder_layer_bwd: null pointer");
@@ -558,7 +612,11 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     LSQ_TRY(launch_rope_table(seq, s.hd, cfg->rope_theta, b.rope_cs, st));
     rope_cs = b.rope_cs;
   }
-  LSQ_TRY(forward_core(s, v, x_in, batch, seq, rope_cs, cfg->rms_eps, b, nullptr, st));
+  // (the rank-r products u of this layer's forward, when kept, are not recomputed:
+  // the same kernels on the same inputs would reproduce them bit for bit)
+  if (saved_u) carve_saved_u(s, T, const_cast<void*>(saved_u), &b);
+  LSQ_TRY(forward_core(s, v, x_in, batch, seq, rope_cs, cfg->rms_eps, b, nullptr, st,
+                       saved_u != nullptr));
 
   const uint16_t* dout_b = dx_out_bf16;
   if (!dout_b) {
@@ -578,15 +636,25 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
   LSQ_TRY(launch_lora_vproj16(b.dgu, T, s.gu_n, v.B16_gu, 2 * r, b.v_gu, b.v16_gu, b.lscratch,
                               b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc, b.v_gu,
-                          b.dn2, 1),
-                   b.gemm, b.gemm_bytes, st));
+  // (a product split over K leaves its partials to the RMSNorm backward after it;
+  // the rank-r products in between do not use the GEMM workspace)
+  const float* parts = nullptr;
+  int np = 1;
+  GemmDesc g_gu = nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc,
+                         b.v_gu, b.dn2, 1);
+  g_gu.parts_out = &parts;
+  g_gu.splits_out = &np;
+  LSQ_TRY(gemm_run(g_gu, b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_lora_grad_a16(b.v16_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, b.lscratch,
                                b.lscratch_bytes, st));
   LSQ_TRY(launch_lora_grad_b16(b.dgu, b.u16_gu, T, s.gu_n, r, 2, pe2, sc, accumulate, gB_gu,
                                b.lscratch, b.lscratch_bytes, st));
   // second RMSNorm + residual
-  LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
+  if (np > 1)
+    LSQ_TRY(launch_rmsnorm_bwd_sum(parts, np, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b,
+                                   st));
+  else
+    LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
   // o projection
   LSQ_TRY(launch_lora_vproj16(b.dh_b, T, s.D, v.B16_o, r, b.v_o, b.v16_o, b.lscratch,
                               b.lscratch_bytes, st));
@@ -603,15 +671,21 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   // q|k|v projections
   LSQ_TRY(launch_lora_vproj16(b.dqkv, T, s.qkv_n, v.B16_qkv, 3 * r, b.v_qkv, b.v16_qkv,
                               b.lscratch, b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
-                          b.v_qkv, b.dn1, 1),
-                   b.gemm, b.gemm_bytes, st));
+  GemmDesc g_qkv = nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
+                          b.v_qkv, b.dn1, 1);
+  g_qkv.parts_out = &parts;
+  g_qkv.splits_out = &np;
+  LSQ_TRY(gemm_run(g_qkv, b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_lora_grad_a16(b.v16_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, b.lscratch,
                                b.lscratch_bytes, st));
   LSQ_TRY(launch_lora_grad_b16(b.dqkv, b.u16_qkv, T, s.qkv_n, r, 3, pe3, sc, accumulate, gB_qkv,
                                b.lscratch, b.lscratch_bytes, st));
   // first RMSNorm + residual
-  LSQ_TRY(launch_rmsnorm_bwd(b.dn1, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16, st));
+  if (np > 1)
+    LSQ_TRY(launch_rmsnorm_bwd_sum(parts, np, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16,
+                                   st));
+  else
+    LSQ_TRY(launch_rmsnorm_bwd(b.dn1, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16, st));
   return LSQ_OK;
 }
 

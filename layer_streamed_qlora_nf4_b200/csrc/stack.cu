@@ -116,6 +116,8 @@ struct StackWs {
   float* dhf;        // [T][D]
   float2* rope_cs;   // [seq][d/2] RoPE cos/sin table, built once per step
   uint16_t* lora16;  // [L][lora16 elems] LoRA operands in product types, once per step
+  uint8_t* saved_u;  // [L][saved_u_bytes] each layer's rank-r products u, forward -> backward
+  size_t saved_u_bytes;
   float* dh[2];      // [T][D] fp32 residual-stream gradient (ping-pong)
   uint16_t* dhb[2];  // bf16 copies
   void* gemm;
@@ -186,6 +188,8 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.dhf = a.take<float>(T * D);
   x.rope_cs = a.take<float2>(T * s.hd / 2);  // >= seq * d/2 entries
   x.lora16 = a.take<uint16_t>((size_t)cfg->n_layers * lora16_elems_per_layer(cfg));
+  x.saved_u_bytes = layer_saved_u_bytes(cfg, T);
+  x.saved_u = a.take<uint8_t>((size_t)cfg->n_layers * x.saved_u_bytes);
   for (int i = 0; i < 2; ++i) {
     x.dh[i] = a.take<float>(T * D);
     x.dhb[i] = a.take<uint16_t>(T * D);
@@ -711,7 +715,8 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
       LSQ_TRY(visit(std::make_tuple(0, i, b, 0, mbk), [&](cudaStream_t s) {
         return layer_fwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
                               w.xs + (size_t)i * T * D, batch, seq, w.xs + (size_t)(i + 1) * T * D,
-                              w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16);
+                              w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16,
+                              w.saved_u + (size_t)i * w.saved_u_bytes);
       }));
       if (dpo)  // reference model: the same layer with its adapter off
         LSQ_TRY(visit(std::make_tuple(1, i, b, 0, mbk), [&](cudaStream_t s) {
@@ -751,7 +756,8 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
         return layer_bwd_impl(cfg, blob, lora + (int64_t)i * layer_floats,
                               w.xs + (size_t)i * T * D, w.dh[cur], w.dhb[cur], batch, seq,
                               w.dh[1 - cur], w.dhb[1 - cur], lora_grad + (int64_t)i * layer_floats,
-                              acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16);
+                              acc, w.layer_ws, w.layer_ws_bytes, s, w.rope_cs, w.lora16 + i * l16,
+                              w.saved_u + (size_t)i * w.saved_u_bytes);
       }));
       if (!h->resident) LSQ_CUDA(cudaEventRecord(h->freed[visits[j].buf], cs));
       if (h->grad_comm && mb == micro_batches - 1) {
