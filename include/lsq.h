@@ -292,7 +292,11 @@ size_t stream_stack_workspace_bytes(const lsq_cfg* cfg, int32_t batch, int32_t s
  *               (positions 0..seq-2 of each sequence, target = next token).
  *   logits_out  device fp32 [batch*seq, V] of the last micro-batch, or NULL.
  * Each micro-batch streams layers 0..L-1 forward, then the lm_head and loss,
- * then L-1..0 backward with per-layer recomputation.  A layer already in a
+ * then L-1..0 backward with per-layer recomputation (the layer's rank-r LoRA
+ * products x A^T are kept from its forward; everything else is recomputed).
+ * The lm_head, the loss and the head's input gradient run over chunks of whole
+ * sequences whose fp32 logits and bf16 logit gradients fit 4 GiB, so the full
+ * [batch*seq, V] logits are never held in the workspace.  A layer already in a
  * buffer when it is needed again is not copied again.  Synchronous: returns once
  * the loss is on the host, LSQ_ERR_TIMEOUT if that takes longer than
  * timeout_ms (the work is then still in flight on the streams). */

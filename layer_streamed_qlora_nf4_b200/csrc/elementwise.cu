@@ -590,6 +590,21 @@ __global__ void embedding_kernel(const int32_t* __restrict__ tok, int64_t T,
 // scale = inv_count, or seq_scale[row / seq] when seq_scale is given (the DPO
 // step's per-sequence coefficient).  The last position of each sequence has no
 // target: zero loss and zero gradient.
+// Online (max, sum of exp) pair of a set of values, and the union of two such
+// pairs: the sum is kept relative to the running maximum and rescaled when that
+// grows (an empty set is (-inf, 0)).
+__device__ __forceinline__ void lse_merge(float& m, float& s, float mo, float so) {
+  const float mn = fmaxf(m, mo);
+  if (mn == -INFINITY) return;  // both empty
+  s = s * expf(m - mn) + so * expf(mo - mn);
+  m = mn;
+}
+
+// One CTA per row: row_loss = logsumexp(logits) - logits[target] (target = the
+// next token; the last position of a sequence has none and gets 0), and with
+// dlogits the gradient (softmax - onehot) * scale in bf16.  One read of the row
+// for the (max, sum) pair, one more for the gradient; rows are read as float4
+// (V is a multiple of 8).
 __global__ void cross_entropy_kernel(const float* __restrict__ logits,
                                      const int32_t* __restrict__ tok, int64_t T, int seq,
                                      int64_t V, float inv_count,
@@ -597,53 +612,64 @@ __global__ void cross_entropy_kernel(const float* __restrict__ logits,
                                      uint16_t* __restrict__ dlogits,
                                      float* __restrict__ row_loss) {
   pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  __shared__ float red[32];
-  __shared__ float bcast;
+  __shared__ float red_m[32], red_s[32];
+  __shared__ float bcast_m, bcast_s;
   const int64_t row = blockIdx.x;
   const float* lr = logits + row * V;
   uint16_t* dr = dlogits ? dlogits + row * V : nullptr;
   const bool has_target = (row % seq) != (seq - 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int64_t n4 = V / 4;
   if (!has_target) {
     if (dr)
-      for (int64_t i = threadIdx.x; i < V; i += blockDim.x) dr[i] = 0;
+      for (int64_t i = threadIdx.x; i < n4; i += blockDim.x)
+        reinterpret_cast<uint2*>(dr)[i] = make_uint2(0u, 0u);
     if (threadIdx.x == 0) row_loss[row] = 0.f;
     return;
   }
-  float mx = -INFINITY;
-  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) mx = fmaxf(mx, lr[i]);
-  mx = warp_max(mx);
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  if (warp == 0) {
-    float v = lane < nw ? red[lane] : -INFINITY;
-    v = warp_max(v);
-    if (lane == 0) bcast = v;
+  const float4* l4 = reinterpret_cast<const float4*>(lr);
+  float m = -INFINITY, s = 0.f;
+  for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = l4[i];
+    const float mv = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+    if (mv > m) {
+      s *= expf(m - mv);
+      m = mv;
+    }
+    s += expf(v.x - m) + expf(v.y - m) + expf(v.z - m) + expf(v.w - m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float mo = __shfl_xor_sync(0xFFFFFFFFu, m, o);
+    const float so = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    lse_merge(m, s, mo, so);
+  }
+  if (lane == 0) {
+    red_m[warp] = m;
+    red_s[warp] = s;
   }
   __syncthreads();
-  mx = bcast;
-  float sum = 0.f;
-  for (int64_t i = threadIdx.x; i < V; i += blockDim.x) sum += expf(lr[i] - mx);
-  sum = warp_sum(sum);
-  __syncthreads();
-  if (lane == 0) red[warp] = sum;
-  __syncthreads();
-  if (warp == 0) {
-    float v = lane < nw ? red[lane] : 0.f;
-    v = warp_sum(v);
-    if (lane == 0) bcast = v;
+  if (threadIdx.x == 0) {
+    float bm = red_m[0], bs = red_s[0];
+    for (int w = 1; w < nw; ++w) lse_merge(bm, bs, red_m[w], red_s[w]);  // fixed order
+    bcast_m = bm;
+    bcast_s = bs;
   }
   __syncthreads();
-  sum = bcast;
+  const float mx = bcast_m, sum = bcast_s;
   const float lse = mx + logf(sum);
   const int64_t tgt = tok[row + 1];
-  const float inv = 1.f / sum;
   if (dr) {
+    const float inv = 1.f / sum;
     const float scale = seq_scale ? seq_scale[row / seq] : inv_count;
-    for (int64_t i = threadIdx.x; i < V; i += blockDim.x) {
-      float p = expf(lr[i] - mx) * inv;
-      if (i == tgt) p -= 1.f;
-      dr[i] = float_to_bf16_bits(p * scale);
+    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+      const float4 v = l4[i];
+      float p[4] = {expf(v.x - mx) * inv, expf(v.y - mx) * inv, expf(v.z - mx) * inv,
+                    expf(v.w - mx) * inv};
+      const int64_t i0 = 4 * i;
+      if (tgt >= i0 && tgt < i0 + 4) p[tgt - i0] -= 1.f;
+      reinterpret_cast<uint2*>(dr)[i] =
+          make_uint2(pack_bf16x2(p[0] * scale, p[1] * scale), pack_bf16x2(p[2] * scale, p[3] * scale));
     }
   }
   if (threadIdx.x == 0) row_loss[row] = lse - lr[tgt];

@@ -109,8 +109,9 @@ struct StackWs {
   float* xs;         // [L+1][T][D] fp32: layer inputs (saved for backward) and final hidden
   uint16_t* hf;      // [T][D] final-norm output
   float* rstd_f;     // [T]
-  float* logits;     // [T][V]
-  uint16_t* dlogits; // [T][V]
+  int64_t head_T;    // tokens per lm_head / cross-entropy chunk (whole sequences)
+  float* logits;     // [head_T][V]
+  uint16_t* dlogits; // [head_T][V]
   float* row_loss;   // [T]
   float* loss_dev;   // [1]
   float* dhf;        // [T][D]
@@ -171,8 +172,18 @@ GemmDesc head_dx(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* 
   return d;
 }
 
-size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* base, StackWs* w,
-                     bool dpo = false) {
+// Tokens per lm_head chunk: whole sequences, as many as keep the chunk's fp32
+// logits and bf16 logit gradients within 4 GiB (at least one sequence); the DPO
+// step needs every row's loss before any logit gradient, so it takes all T.
+int64_t head_chunk_tokens(const lsq_cfg* cfg, int64_t T, int seq, bool dpo) {
+  if (dpo || seq <= 0) return T;
+  const int64_t per_seq = (int64_t)cfg->vocab * 6 * seq;
+  const int64_t seqs = std::max<int64_t>(1, (int64_t(4) << 30) / std::max<int64_t>(per_seq, 1));
+  return std::min<int64_t>(T, seqs * seq);
+}
+
+size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, int seq, void* base,
+                     StackWs* w, bool dpo = false) {
   Arena a;
   a.base = static_cast<uint8_t*>(base);
   a.cap = SIZE_MAX;
@@ -181,8 +192,9 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
   x.xs = a.take<float>((size_t)(cfg->n_layers + 1) * T * D);
   x.hf = a.take<uint16_t>(T * D);
   x.rstd_f = a.take<float>(T);
-  x.logits = a.take<float>((size_t)T * V);
-  x.dlogits = a.take<uint16_t>((size_t)T * V);
+  x.head_T = head_chunk_tokens(cfg, T, seq, dpo);
+  x.logits = a.take<float>((size_t)x.head_T * V);
+  x.dlogits = a.take<uint16_t>((size_t)x.head_T * V);
   x.row_loss = a.take<float>(T);
   x.loss_dev = a.take<float>(64);
   x.dhf = a.take<float>(T * D);
@@ -194,8 +206,9 @@ size_t plan_stack_ws(const lsq_cfg* cfg, const LayerShapes& s, int64_t T, void* 
     x.dh[i] = a.take<float>(T * D);
     x.dhb[i] = a.take<uint16_t>(T * D);
   }
-  const size_t gb = std::max(gemm_workspace_bytes(head_fwd(nullptr, V, D, nullptr, T, nullptr)),
-                             gemm_workspace_bytes(head_dx(nullptr, V, D, nullptr, T, nullptr)));
+  const size_t gb =
+      std::max(gemm_workspace_bytes(head_fwd(nullptr, V, D, nullptr, x.head_T, nullptr)),
+               gemm_workspace_bytes(head_dx(nullptr, V, D, nullptr, x.head_T, nullptr)));
   x.gemm = a.take<uint8_t>(gb + 256);
   x.gemm_bytes = gb + 256;
   x.layer_ws_bytes = layer_ws_bytes(cfg, T);
@@ -347,7 +360,7 @@ extern "C" size_t stream_stack_workspace_bytes(const lsq_cfg* cfg, int32_t batch
   if (batch <= 0 || seq <= 0 || layer_shapes(cfg, &s) != LSQ_OK || cfg->n_layers <= 0 ||
       cfg->vocab <= 0)
     return 0;
-  return plan_stack_ws(cfg, s, (int64_t)batch * seq, nullptr, nullptr);
+  return plan_stack_ws(cfg, s, (int64_t)batch * seq, seq, nullptr, nullptr);
 }
 
 extern "C" int stream_stack_create(const lsq_cfg* cfg, const void* const* layer_blobs,
@@ -599,11 +612,11 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
   const LayerShapes& s = h->shapes;
   const int L = cfg->n_layers;
   const int64_t T = (int64_t)batch * seq, D = s.D, V = cfg->vocab;
-  const size_t need = plan_stack_ws(cfg, s, T, nullptr, nullptr, dpo != nullptr);
+  const size_t need = plan_stack_ws(cfg, s, T, seq, nullptr, nullptr, dpo != nullptr);
   if (!ws || ws_bytes < need)
     return set_error(LSQ_ERR_WORKSPACE, "stream_stack_step: workspace %zu < %zu", ws_bytes, need);
   StackWs w;
-  plan_stack_ws(cfg, s, T, ws, &w, dpo != nullptr);
+  plan_stack_ws(cfg, s, T, seq, ws, &w, dpo != nullptr);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int64_t layer_floats = h->lora_layout.floats_per_layer;
   const float inv_count = 1.f / (float)((double)micro_batches * batch * (seq - 1));
@@ -733,18 +746,35 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
       LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_ref, cs));
     }
     LSQ_TRY(launch_rmsnorm_fwd(xL, final_norm, T, D, cfg->rms_eps, w.hf, OUT_BF16, w.rstd_f, cs));
-    LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
-    if (dpo) {
+    if (!dpo) {
+      // lm_head, cross-entropy and the head's input gradient, a chunk of whole
+      // sequences at a time, so that the [T, V] logits never exist at once
+      const bool last_mb = mb == micro_batches - 1;
+      for (int64_t c0 = 0; c0 < T; c0 += w.head_T) {
+        const int64_t tc = std::min<int64_t>(w.head_T, T - c0);
+        LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf + c0 * D, tc, w.logits), w.gemm,
+                         w.gemm_bytes, cs));
+        if (logits_out && last_mb)
+          LSQ_CUDA(cudaMemcpyAsync(logits_out + c0 * V, w.logits, (size_t)tc * V * sizeof(float),
+                                   cudaMemcpyDeviceToDevice, cs));
+        LSQ_TRY(launch_cross_entropy(w.logits, tok + c0, tc, seq, V, inv_count, w.dlogits,
+                                     w.row_loss + c0, cs));
+        LSQ_TRY(gemm_run(head_dx(lm_head, V, D, w.dlogits, tc, w.dhf + c0 * D), w.gemm,
+                         w.gemm_bytes, cs));
+      }
+      LSQ_TRY(launch_sum_rows(w.row_loss, T, inv_count, mb > 0 ? 1 : 0, w.loss_dev, cs));
+    } else {
+      LSQ_TRY(gemm_run(head_fwd(lm_head, V, D, w.hf, T, w.logits), w.gemm, w.gemm_bytes, cs));
       LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, nullptr, w.row_loss, cs));
       LSQ_TRY(launch_dpo_loss(w.row_loss, w.row_ref, dpo->pairs, seq, dpo->beta, w.seq_scale,
                               w.logps, w.loss_dev, cs));
       LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, 0.f, w.dlogits, w.row_loss, cs,
                                    w.seq_scale));
-    } else {
-      LSQ_TRY(launch_cross_entropy(w.logits, tok, T, seq, V, inv_count, w.dlogits, w.row_loss, cs));
-      LSQ_TRY(launch_sum_rows(w.row_loss, T, inv_count, mb > 0 ? 1 : 0, w.loss_dev, cs));
+      LSQ_TRY(gemm_run(head_dx(lm_head, V, D, w.dlogits, T, w.dhf), w.gemm, w.gemm_bytes, cs));
+      if (logits_out)
+        LSQ_CUDA(cudaMemcpyAsync(logits_out, w.logits, (size_t)T * V * sizeof(float),
+                                 cudaMemcpyDeviceToDevice, cs));
     }
-    LSQ_TRY(gemm_run(head_dx(lm_head, V, D, w.dlogits, T, w.dhf), w.gemm, w.gemm_bytes, cs));
     LSQ_TRY(launch_rmsnorm_bwd(w.dhf, xL, final_norm, w.rstd_f, nullptr, T, D, w.dh[0], w.dhb[0], cs));
     int cur = 0;
     for (int i = L - 1; i >= 0; --i, ++j) {
@@ -780,9 +810,6 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
     LSQ_CUDA(cudaEventRecord(h->red_done, h->red_stream));
     LSQ_CUDA(cudaStreamWaitEvent(cs, h->red_done, 0));
   }
-  if (logits_out)
-    LSQ_CUDA(cudaMemcpyAsync(logits_out, w.logits, (size_t)T * V * sizeof(float),
-                             cudaMemcpyDeviceToDevice, cs));
   if (opt)
     LSQ_TRY(launch_adamw(lora, lora_grad, opt->m, opt->v, layer_floats * L, opt->lr, opt->beta1,
                          opt->beta2, opt->eps, opt->weight_decay, opt->step, cs));
@@ -854,7 +881,7 @@ extern "C" size_t stream_stack_dpo_workspace_bytes(const lsq_cfg* cfg, int32_t p
   if (pairs <= 0 || pairs > kMaxPairs || seq <= 0 || layer_shapes(cfg, &s) != LSQ_OK ||
       cfg->n_layers <= 0 || cfg->vocab <= 0)
     return 0;
-  return plan_stack_ws(cfg, s, (int64_t)2 * pairs * seq, nullptr, nullptr, true);
+  return plan_stack_ws(cfg, s, (int64_t)2 * pairs * seq, seq, nullptr, nullptr, true);
 }
 
 extern "C" int stream_stack_dpo_step(lsq_stack* h, const int32_t* tokens, int32_t pairs,
