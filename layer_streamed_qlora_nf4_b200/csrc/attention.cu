@@ -557,16 +557,20 @@ __global__ void __launch_bounds__(kAThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_vconv));
     }
+    // lse (log2 units) and delta of the warp's 32 queries of a chunk: lane i holds
+    // query i's, fetched one chunk ahead, and the lanes read them by shuffle
+    auto fetch = [&](int c, float* l2v, float* dlv) {
+      const int qq = min(k0 + c * kBC + 32 * hf + lane, seq - 1);
+      *l2v = __ldg(lse + (int64_t)h * T + tok0 + qq) * 1.4426950408889634f;
+      *dlv = __ldg(delta + (int64_t)h * T + tok0 + qq);
+    };
+    float l2_own = 0.f, dl_own = 0.f;
+    if (nc > 0) fetch(0, &l2_own, &dl_own);
     for (int c = 0; c < nc && ok; ++c) {
       const int qb = c & 1;
       const int q0 = k0 + c * kBC + 32 * hf;  // this thread's first query
-      float l2[32], dl[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int qq = min(q0 + e, seq - 1);
-        l2[e] = __ldg(lse + (int64_t)h * T + tok0 + qq) * 1.4426950408889634f;
-        dl[e] = __ldg(delta + (int64_t)h * T + tok0 + qq);
-      }
+      float l2_next = 0.f, dl_next = 0.f;
+      if (c + 1 < nc) fetch(c + 1, &l2_next, &dl_next);
       ok = mbar_wait_bounded(smem_u32(&bar_sdp[qb]), (uint32_t)((c >> 1) & 1), abort_flag, dev_err,
                              DEV_ERR_WAIT_GEMM);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -591,8 +595,10 @@ __global__ void __launch_bounds__(kAThreads, 1)
           const bool live = kpos <= qq && qq < seq && kpos < seq;
           const float s = __uint_as_float(sv[(e + u) >> 4][(e + u) & 15]);
           const float dp = __uint_as_float(pv[(e + u) >> 4][(e + u) & 15]);
-          p[u] = live ? exp2f(fmaf(s, sl2, -l2[e + u])) : 0.f;
-          d[u] = p[u] * (dp - dl[e + u]);
+          const float l2 = __shfl_sync(0xFFFFFFFFu, l2_own, e + u);
+          const float dl = __shfl_sync(0xFFFFFFFFu, dl_own, e + u);
+          p[u] = live ? exp2f(fmaf(s, sl2, -l2)) : 0.f;
+          d[u] = p[u] * (dp - dl);
         }
         ppk[e >> 1] = pack_bf16x2(p[0], p[1]);
         dpk[e >> 1] = pack_bf16x2(d[0], d[1]);
@@ -618,6 +624,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_ds));
+      l2_own = l2_next;
+      dl_own = dl_next;
     }
     // ---------------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait_bounded(smem_u32(&bar_pds), (uint32_t)((nc - 1) & 1), abort_flag,

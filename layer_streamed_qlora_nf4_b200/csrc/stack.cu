@@ -34,6 +34,7 @@
 // buffer before the "ready" event.  Per-GPU host->device bytes fall by G.  The
 // NCCL library is loaded at run time (the one torch already loaded, else the
 // system's), so the library has no link-time dependency on it.
+#include <cstdlib>
 #include <dlfcn.h>
 #include <nccl.h>
 #include <string.h>
@@ -173,12 +174,17 @@ GemmDesc head_dx(const uint16_t* lm_head, int64_t V, int64_t D, const uint16_t* 
 }
 
 // Tokens per lm_head chunk: whole sequences, as many as keep the chunk's fp32
-// logits and bf16 logit gradients within 4 GiB (at least one sequence); the DPO
+// logits and bf16 logit gradients within 4 GiB (at least one sequence), or
+// LSQ_HEAD_CHUNK_SEQS sequences when that is set in the environment; the DPO
 // step needs every row's loss before any logit gradient, so it takes all T.
 int64_t head_chunk_tokens(const lsq_cfg* cfg, int64_t T, int seq, bool dpo) {
   if (dpo || seq <= 0) return T;
   const int64_t per_seq = (int64_t)cfg->vocab * 6 * seq;
-  const int64_t seqs = std::max<int64_t>(1, (int64_t(4) << 30) / std::max<int64_t>(per_seq, 1));
+  int64_t seqs = std::max<int64_t>(1, (int64_t(4) << 30) / std::max<int64_t>(per_seq, 1));
+  if (const char* e = std::getenv("LSQ_HEAD_CHUNK_SEQS")) {
+    const long v = std::strtol(e, nullptr, 10);
+    if (v > 0) seqs = v;
+  }
   return std::min<int64_t>(T, seqs * seq);
 }
 
@@ -656,7 +662,7 @@ int step_impl(lsq_stack* h, const int32_t* tokens, int32_t micro_batches, int32_
     const std::vector<uintptr_t> sig = {
         (uintptr_t)lora, (uintptr_t)lora_grad, (uintptr_t)ws, (uintptr_t)ws_bytes,
         (uintptr_t)batch, (uintptr_t)seq, (uintptr_t)micro_batches, (uintptr_t)profiling,
-        (uintptr_t)(dpo != nullptr)};
+        (uintptr_t)(dpo != nullptr), (uintptr_t)w.head_T};  // (head_T moves the layer workspace)
     if (sig != h->graph_sig) {
       drop_graphs(h);
       h->graph_sig = sig;

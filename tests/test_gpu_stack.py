@@ -209,6 +209,24 @@ def test_stack_streamed_equals_resident_bitwise(L, small):
     assert st1["h2d_bytes"] == st1["layer_copies"] * small.blob_bytes
 
 
+def test_stack_head_chunks_equal_one_chunk(L, small, monkeypatch):
+    # lm_head, cross-entropy and the head's input gradient over chunks of one
+    # sequence each give the same step as over the whole batch at once (every
+    # row's products and loss are computed the same way in both)
+    import torch
+    cfg = small.cfg
+    batch, seq = 3, 48
+    tokens = synth.tokens(36, batch, seq, cfg["vocab"])
+    h = small.handle(L, resident=True)
+    monkeypatch.setenv("LSQ_HEAD_CHUNK_SEQS", "1")
+    l1, lg1, g1, _ = _step(L, small, h, tokens, 1, batch, seq)
+    monkeypatch.delenv("LSQ_HEAD_CHUNK_SEQS")
+    l0, lg0, g0, _ = _step(L, small, h, tokens, 1, batch, seq)
+    h.close()
+    assert L.stream_stack_workspace_bytes(cfg, batch, seq) > 0
+    assert l1 == l0 and torch.equal(lg1, lg0) and torch.equal(g1, g0)
+
+
 def test_stack_grad_accumulation_and_adamw(L, small):
     import torch
     from gpu_util import check_stack_grad
