@@ -93,6 +93,7 @@ struct KParams {
   const float* am_s;
   int w_rows, w_cols;
   int slab_w, part_r, n_parts;
+  int slab_tma;  // the slab's operands arrive by TMA (tm_la, tm_lb) instead of la / lb
   const float* la;
   long long la_rs, la_cs;
   float la_scale;
@@ -118,7 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                    const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_out,
-                   const __grid_constant__ CUtensorMap tm_res, const __grid_constant__ KParams p) {
+                   const __grid_constant__ CUtensorMap tm_res,
+                   const __grid_constant__ CUtensorMap tm_la,
+                   const __grid_constant__ CUtensorMap tm_lb, const __grid_constant__ KParams p) {
   extern __shared__ uint8_t dsm_raw[];
   __shared__ __align__(8) uint64_t bar_full[kMaxStages];
   __shared__ __align__(8) uint64_t bar_empty[kMaxStages];
@@ -238,6 +241,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                           fb, kt * kBK, t0 + a * p.bn);
             if (WMODE == W_BF16_N)
               tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fb, kt * kBK, m0);
+          }
+        } else if (p.slab_tma) {
+          // LoRA slab: s B (or s A^T) into the weight stage, u (or v) into the
+          // activation stage, 64 slab columns at a time (beyond slab_w: zeros)
+          const int j0 = (it - n_main) * 64;
+          const uint32_t bytes = xs_bytes + (uint32_t)kWStageBytes;
+          if (PAIR) {
+            const uint32_t fl = mapa_shared(fb, 0);
+            if (leader) mbar_arrive_expect_tx(fb, 2 * bytes);
+            for (int a = 0; a < p.nacc; ++a)
+              tma_load_2d_pair(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * hb * 128), &tm_lb,
+                               fl, j0, t0 + a * p.bn + (int)rank * hb);
+            tma_load_2d_pair(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_la, fl, j0, m0);
+          } else {
+            mbar_arrive_expect_tx(fb, bytes);
+            for (int a = 0; a < p.nacc; ++a)
+              tma_load_2d(smem_u32(xs0 + (size_t)s * xs_bytes + (size_t)a * p.bn * 128), &tm_lb,
+                          fb, j0, t0 + a * p.bn);
+            tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_la, fb, j0, m0);
           }
         } else if (!PAIR || leader) {
           mbar_arrive(fb);
@@ -514,6 +536,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(smem_u32(&bar_cempty[c]));
           }
         }
+      } else if (p.slab_tma) {
+        // LoRA slab by TMA: the stage only has to be free before this warp arrives
+        ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
+                               DEV_ERR_WAIT_GEMM);
+        ok = __all_sync(0xFFFFFFFFu, ok);
       } else {
         // LoRA slab: la -> weight stage, lb -> activation stage (lb comes from the
         // kernel before: wait for it)
@@ -864,6 +891,15 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
                       (uint64_t)d.T, (uint64_t)d.ldr, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   else
     tm_res = tm_out;  // unused
+  CUtensorMap tm_la = tm_out, tm_lb = tm_out;  // unused without a TMA-fed slab
+  const bool slab_tma = d.slab_w > 0 && d.la16 != nullptr;
+  if (slab_tma) {
+    LSQ_TRY(make_tmap(&tm_la, dt16, 2, d.la16, (uint64_t)d.slab_w, (uint64_t)d.M,
+                      (uint64_t)d.la16_ld, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B));
+    LSQ_TRY(make_tmap(&tm_lb, dt16, 2, d.lb16, (uint64_t)d.slab_w, (uint64_t)d.T,
+                      (uint64_t)d.lb16_ld, kBK, (uint32_t)(PAIR ? pl.bn / 2 : pl.bn),
+                      CU_TENSOR_MAP_SWIZZLE_128B));
+  }
   KParams p{};
   p.M = (int)d.M;
   p.T = (int)d.T;
@@ -883,6 +919,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   p.w_rows = (int)d.w_rows;
   p.w_cols = (int)d.w_cols;
   p.slab_w = d.slab_w;
+  p.slab_tma = slab_tma ? 1 : 0;
   p.part_r = d.part_r;
   p.n_parts = d.n_parts;
   p.la = d.la;
@@ -917,7 +954,8 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   LSQ_CUDA(::lsq::launched(
-      cudaLaunchKernelEx(&cfg, tc_gemm_kernel<WMODE, PAIR>, tm_act, tm_w, tm_out, tm_res, p)));
+      cudaLaunchKernelEx(&cfg, tc_gemm_kernel<WMODE, PAIR>, tm_act, tm_w, tm_out, tm_res, tm_la,
+                         tm_lb, p)));
   return LSQ_OK;
 }
 
@@ -977,7 +1015,13 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
     return set_error(LSQ_ERR_SHAPE, "gemm: row strides must be multiples of 16 bytes");
   if (d.slab_w % 16 != 0 || d.slab_w < 0)
     return set_error(LSQ_ERR_SHAPE, "gemm: LoRA slab width must be a multiple of 16");
-  if (d.slab_w > 0 && (!d.la || !d.lb)) return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
+  if (d.slab_w > 0 && !d.la16 && (!d.la || !d.lb))
+    return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
+  if (d.slab_w > 0 && d.la16 &&
+      (!d.lb16 || d.la16_ld % 8 != 0 || d.lb16_ld % 8 != 0 || d.la16_ld < d.slab_w ||
+       d.lb16_ld < d.slab_w))
+    return set_error(LSQ_ERR_SHAPE, "gemm: 16-bit LoRA slab operands need row strides >= the "
+                                    "slab width, multiples of 8");
   if (d.residual && !d.out_f32) return set_error(LSQ_ERR_INVALID, "gemm: residual needs an fp32 output");
   if (d.ldo % 8 != 0 || (d.residual && d.ldr % 8 != 0))
     return set_error(LSQ_ERR_SHAPE, "gemm: output strides must be multiples of 16 bytes");

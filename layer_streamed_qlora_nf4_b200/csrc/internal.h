@@ -134,6 +134,13 @@ struct GemmDesc {
   // consumer's to add.
   const float** parts_out = nullptr;
   int* splits_out = nullptr;
+  // The LoRA slab from 16-bit operands by TMA, instead of la / lb above: la16
+  // [M][la16_ld] (the scale applied) and lb16 [T][lb16_ld], slab_w columns of
+  // each, in the mode's operand type (fp16 forward, bf16 input gradient).
+  const uint16_t* la16 = nullptr;
+  int64_t la16_ld = 0;
+  const uint16_t* lb16 = nullptr;
+  int64_t lb16_ld = 0;
 };
 size_t gemm_workspace_bytes(const GemmDesc& d);
 int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st);
@@ -206,15 +213,18 @@ int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 int64_t lora16_ld(int64_t T);  // row stride of u16 / v16: T rounded up to 8
 size_t lora_scratch_bytes(int64_t T, int64_t K, int R);
 // u[t, j] = sum_k x[t, k] A[j, k]        x fp16 [T, ldx], A16 fp16 [R, K] -> u fp32 [T, R]
+// (u may be null), and uh (nullable) the same rounded to fp16, [T, R]: the fused
+// GEMM's LoRA slab operand
 int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
                        int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
-                       cudaStream_t st);
+                       cudaStream_t st, uint16_t* uh = nullptr);
 // v[t, c] = sum_n dy[t, n] Bt[c, n]      dy bf16 [T, N], Bt bf16 [R, N]: the block-diagonal
 // stack of the parts' B transposed (column n of part p holds B_p's row n in rows
 // [p r, (p + 1) r), zeros elsewhere)
+// (v may be null; vh, nullable: the same rounded to bf16, [T, R], the slab operand)
 int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
                         float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
-                        cudaStream_t st);
+                        cudaStream_t st, uint16_t* vh = nullptr);
 // dA[j, k] (+)= s sum_t v[t, j] x[t, k]  v16 bf16 [R, lora16_ld(T)], x fp16 [T, K] (converted
 // to bf16 as it is loaded)
 int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
@@ -233,18 +243,24 @@ int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, 
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, float* v,
                       uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st);
 // One layer's LoRA operands rounded once into their product types: a list of
-// blocks, each an fp16 copy of an A matrix (kind 0: [rows][cols]) or a bf16
-// block-diagonal stack of a B matrix, transposed (kind 1: [ld_out][rows], the
-// rows split into parts ending at part_end[], part p's rows holding B in rows
-// [p cols, (p + 1) cols) of the stack).  Offsets in elements within one layer's
-// LoRA block / output.
+// blocks, each
+//   kind 0: an fp16 copy of an A matrix, [rows][cols];
+//   kind 1: a bf16 block-diagonal stack of a B matrix, transposed ([ld_out][rows],
+//           the rows split into parts ending at part_end[], part p's rows holding
+//           B in rows [p cols, (p + 1) cols) of the stack);
+//   kind 2: scale * the same stack untransposed, fp16 [rows][ld_out] (the forward
+//           GEMM's LoRA slab);
+//   kind 3: scale * A transposed, bf16 [rows][ld_out] from A [ld_out][rows] (the
+//           input-gradient GEMM's LoRA slab).
+// Offsets in elements within one layer's LoRA block / output.
 struct LoraPrepSeg {
   int64_t src_off, dst_off, rows, cols, ld_out;
   int kind, n_parts;
   int64_t part_end[4];
+  float scale;  // kinds 2 and 3
 };
 struct LoraPrepSegs {
-  LoraPrepSeg seg[8];
+  LoraPrepSeg seg[16];
   int n;
 };
 // Converts n_layers LoRA blocks (stride lora_stride floats) into out (stride

@@ -74,6 +74,8 @@ struct Views {  // pointers into one layer blob / one LoRA block
   const float *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_d, *B_d;
   // the same operands rounded once into their product types (Lora16)
   const uint16_t *A16_qkv, *A16_o, *A16_gu, *A16_d, *B16_qkv, *B16_o, *B16_gu, *B16_d;
+  // the fused GEMMs' LoRA slab operands: s B stacks (fp16, forward) and s A^T (bf16, dX)
+  const uint16_t *Bs16_qkv, *Bs16_o, *Bs16_gu, *Bs16_d, *At16_qkv, *At16_o, *At16_gu, *At16_d;
   bool lora_on;  // false: adapter disabled, every LoRA branch removed
 };
 
@@ -138,10 +140,13 @@ void fill_layout(const LayerShapes& s, lsq_layer_layout* L, lsq_lora_layout* R) 
 // masters (per optimiser step in the stack): fp16 A_qkv [3r, D], A_o [r, H d],
 // A_gu [2r, D], A_down [r, F] for u = x A^T; bf16 block-diagonal B stacks for
 // v = dY B, one product per projection group: B_qkv -> [qkv rows, 3r],
-// B_o [D, r], B_gu -> [2F, 2r], B_down [D, r].  Offsets in elements, each block
-// 128-element (256-byte) aligned.
+// B_o [D, r], B_gu -> [2F, 2r], B_down [D, r]; and the fused GEMMs' LoRA slab
+// operands: the scaled B stacks s B in fp16, [qkv rows, 3r] ... (the forward),
+// and the scaled transposed A stacks s A^T in bf16, [D, 3r], [H d, r], [D, 2r],
+// [F, r] (the input gradient).  Offsets in elements, each block 128-element
+// (256-byte) aligned.
 struct Lora16 {
-  int64_t a[4], b[4], elems;
+  int64_t a[4], b[4], bs[4], at[4], elems;
 };
 Lora16 lora16_layout(const LayerShapes& s) {
   auto al = [](int64_t x) { return (x + 127) & ~int64_t(127); };
@@ -156,6 +161,14 @@ Lora16 lora16_layout(const LayerShapes& s) {
   o.b[1] = f; f = al(f + s.D * r);
   o.b[2] = f; f = al(f + s.gu_n * 2 * r);
   o.b[3] = f; f = al(f + s.D * r);
+  o.bs[0] = f; f = al(f + s.qkv_n * 3 * r);
+  o.bs[1] = f; f = al(f + s.D * r);
+  o.bs[2] = f; f = al(f + s.gu_n * 2 * r);
+  o.bs[3] = f; f = al(f + s.D * r);
+  o.at[0] = f; f = al(f + s.D * 3 * r);
+  o.at[1] = f; f = al(f + s.qd * r);
+  o.at[2] = f; f = al(f + s.D * 2 * r);
+  o.at[3] = f; f = al(f + s.F * r);
   o.elems = f;
   return o;
 }
@@ -189,8 +202,24 @@ LoraPrepSegs lora16_segs(const LayerShapes& s, const lsq_lora_layout& R, const L
     e.ld_out = bparts[i] * r;
     e.n_parts = bparts[i];
     for (int p = 0; p < bparts[i]; ++p) e.part_end[p] = pe[i][p];
+    LoraPrepSeg& f = g.seg[8 + i];  // s B, untransposed, fp16
+    f = e;
+    f.kind = 2;
+    f.dst_off = o.bs[i];
+    f.scale = s.s;
   }
-  g.n = 8;
+  for (int i = 0; i < 4; ++i) {  // s A^T, bf16
+    LoraPrepSeg& e = g.seg[12 + i];
+    e.kind = 3;
+    e.src_off = asrc[i];
+    e.dst_off = o.at[i];
+    e.rows = acols[i];
+    e.cols = arows[i];
+    e.ld_out = arows[i];
+    e.n_parts = 1;
+    e.scale = s.s;
+  }
+  g.n = 16;
   return g;
 }
 
@@ -216,6 +245,8 @@ Views views(const LayerShapes& s, const void* blob, const float* lora) {
   v.lora_on = lora != nullptr;
   v.A_qkv = v.B_qkv = v.A_o = v.B_o = v.A_gu = v.B_gu = v.A_d = v.B_d = nullptr;
   v.A16_qkv = v.A16_o = v.A16_gu = v.A16_d = v.B16_qkv = v.B16_o = v.B16_gu = v.B16_d = nullptr;
+  v.Bs16_qkv = v.Bs16_o = v.Bs16_gu = v.Bs16_d = nullptr;
+  v.At16_qkv = v.At16_o = v.At16_gu = v.At16_d = nullptr;
   if (v.lora_on) {
     v.A_qkv = lora + R.a_off[0];
     v.B_qkv = lora + R.b_off[0];
@@ -237,7 +268,9 @@ struct Buffers {
   float* h;                                          // fp32 residual stream after attention
   uint16_t *n1, *qkv, *ao, *n2, *gu, *m;             // fp16 forward activations
   uint16_t *dgu, *dqkv, *da, *dout_b, *dh_b;         // bf16 gradients
-  float *rstd1, *rstd2, *u_qkv, *u_o, *u_gu, *u_d, *lse, *v_qkv, *v_o, *v_gu, *v_d;
+  uint16_t *uh_qkv, *uh_o, *uh_gu, *uh_d;  // u in fp16, [T][R]: the forward GEMMs' LoRA slab
+  uint16_t *vh_qkv, *vh_o, *vh_gu, *vh_d;  // v in bf16, [T][R]: the dX GEMMs' LoRA slab
+  float *rstd1, *rstd2, *lse;
   float *dm, *dn2, *dh, *dn1, *dq, *dk, *dv, *delta;
   float2* rope_cs;
   float* lscratch;
@@ -247,12 +280,13 @@ struct Buffers {
 };
 
 // Forward of a stacked frozen weight W [N, K] (NF4, or bf16 when absmax is
-// empty, converted to fp16 in the operand stage): out [T, N] = act W^T + s u B^T,
-// fp16; or, with a residual, out = that + residual in fp32.
+// empty, converted to fp16 in the operand stage): out [T, N] = act W^T + u Bs^T,
+// fp16; or, with a residual, out = that + residual in fp32.  The LoRA branch is
+// the GEMM's slab of R columns: Bs = s B (fp16 [N][R], each row's part's columns
+// only, zeros elsewhere) and u (fp16 [T][R]); R = 0 without an adapter.
 GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
-                 const uint16_t* act, int64_t T, const float* B, int r, float s, const float* u,
-                 int64_t u_ld, int n_parts, const int64_t* pe, const float* res, void* out,
-                 int64_t ldo) {
+                 const uint16_t* act, int64_t T, const uint16_t* Bs, const uint16_t* u, int R,
+                 const float* res, void* out, int64_t ldo) {
   GemmDesc d;
   const bool bf16 = absmax.bf16;
   d.wmode = bf16 ? W_BF16C_N : W_NF4_N;
@@ -267,16 +301,11 @@ GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64
   d.w_cols = K;
   d.act = act;
   d.act_ld = K;
-  d.slab_w = n_parts > 1 ? n_parts * r : r;
-  d.la = B;
-  d.la_rs = r;
-  d.la_cs = 1;
-  d.la_scale = s;
-  d.lb = u;
-  d.lb_ld = u_ld;
-  d.part_r = n_parts > 1 ? r : 0;
-  d.n_parts = n_parts;
-  for (int i = 0; i < n_parts && i < 4; ++i) d.part_end[i] = pe[i];
+  d.slab_w = R;
+  d.la16 = Bs;
+  d.la16_ld = R;
+  d.lb16 = u;
+  d.lb16_ld = R;
   d.out = out;
   d.ldo = ldo;
   d.out_f32 = res != nullptr;
@@ -285,9 +314,10 @@ GemmDesc nf4_fwd(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64
   return d;
 }
 
-// dX of a stacked NF4 weight W [N, K]: out [T, K] = dy W + s v A_stack, v [T, R], A [R, K]
+// dX of a stacked weight W [N, K]: out [T, K] = dy W + v At^T, with At = s A_stack^T
+// (bf16 [K][R]) and v (bf16 [T][R]) as the GEMM's slab.
 GemmDesc nf4_dx(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_t K,
-                const uint16_t* dy, int64_t T, const float* A, int R, float s, const float* v,
+                const uint16_t* dy, int64_t T, const uint16_t* At, const uint16_t* v, int R,
                 void* out, int out_f32) {
   GemmDesc d;
   const bool bf16 = absmax.bf16;
@@ -304,12 +334,10 @@ GemmDesc nf4_dx(const uint8_t* codes, const AbsmaxRef& absmax, int64_t N, int64_
   d.act = dy;
   d.act_ld = N;
   d.slab_w = R;
-  d.la = A;
-  d.la_rs = 1;
-  d.la_cs = K;
-  d.la_scale = s;
-  d.lb = v;
-  d.lb_ld = R;
+  d.la16 = At;
+  d.la16_ld = R;
+  d.lb16 = v;
+  d.lb16_ld = R;
   d.out = out;
   d.out_f32 = out_f32;
   d.ldo = K;
@@ -346,15 +374,15 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   x.v16_o = a.take<uint16_t>(t16 * r);
   x.v16_gu = a.take<uint16_t>(t16 * 2 * r);
   x.v16_d = a.take<uint16_t>(t16 * r);
-  x.u_qkv = a.take<float>(T * 3 * r);
-  x.u_o = a.take<float>(T * r);
-  x.u_gu = a.take<float>(T * 2 * r);
-  x.u_d = a.take<float>(T * r);
+  x.uh_qkv = a.take<uint16_t>(T * 3 * r);
+  x.uh_o = a.take<uint16_t>(T * r);
+  x.uh_gu = a.take<uint16_t>(T * 2 * r);
+  x.uh_d = a.take<uint16_t>(T * r);
   x.lse = a.take<float>(T * s.H);
-  x.v_qkv = a.take<float>(T * 3 * r);
-  x.v_o = a.take<float>(T * r);
-  x.v_gu = a.take<float>(T * 2 * r);
-  x.v_d = a.take<float>(T * r);
+  x.vh_qkv = a.take<uint16_t>(T * 3 * r);
+  x.vh_o = a.take<uint16_t>(T * r);
+  x.vh_gu = a.take<uint16_t>(T * 2 * r);
+  x.vh_d = a.take<uint16_t>(T * r);
   x.dm = a.take<float>(T * s.F);
   x.dn2 = a.take<float>(T * s.D);
   x.dh = a.take<float>(T * s.D);
@@ -375,18 +403,18 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   const int64_t pe2[2] = {s.F, s.gu_n};
   size_t gb = 0;
   GemmDesc ds[8] = {
-      nf4_fwd(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 3 * r, 3, pe3,
-              nullptr, nullptr, s.qkv_n),
-      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
-              nullptr, s.D),
-      nf4_fwd(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, r, 0, nullptr, 2 * r, 2, pe2,
-              nullptr, nullptr, s.gu_n),
-      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, r, 1, pe3, nullptr,
-              nullptr, s.D),
-      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, r, 0, nullptr, nullptr, 1),
-      nf4_dx(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, 2 * r, 0, nullptr, nullptr, 1),
-      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, r, 0, nullptr, nullptr, 0),
-      nf4_dx(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, 3 * r, 0, nullptr, nullptr, 1)};
+      nf4_fwd(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, nullptr, 3 * r, nullptr,
+              nullptr, s.qkv_n),
+      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, nullptr, r, nullptr, nullptr,
+              s.D),
+      nf4_fwd(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, nullptr, 2 * r, nullptr,
+              nullptr, s.gu_n),
+      nf4_fwd(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, nullptr, r, nullptr, nullptr,
+              s.D),
+      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.F, nullptr, T, nullptr, nullptr, r, nullptr, 1),
+      nf4_dx(nullptr, AbsmaxRef{}, s.gu_n, s.D, nullptr, T, nullptr, nullptr, 2 * r, nullptr, 1),
+      nf4_dx(nullptr, AbsmaxRef{}, s.D, s.qd, nullptr, T, nullptr, nullptr, r, nullptr, 0),
+      nf4_dx(nullptr, AbsmaxRef{}, s.qkv_n, s.D, nullptr, T, nullptr, nullptr, 3 * r, nullptr, 1)};
   for (auto& d : ds) gb = std::max(gb, gemm_workspace_bytes(d));
   x.gemm = a.take<uint8_t>(gb + 256);
   x.gemm_bytes = gb + 256;
@@ -394,7 +422,7 @@ size_t plan_buffers(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   return a.used;
 }
 
-// The rank-r products u = x A^T of one forward (fp32 [T][R] per projection group,
+// The rank-r products u = x A^T of one forward (fp16 [T][R] per projection group,
 // read by the GEMMs' LoRA slab, and their bf16 [R][lora16_ld(T)] copies, read by
 // dB), carved from a region the caller keeps from the forward to the backward.
 size_t carve_saved_u(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
@@ -403,19 +431,19 @@ size_t carve_saved_u(const LayerShapes& s, int64_t T, void* base, Buffers* b) {
   a.cap = SIZE_MAX;
   const int r = s.r;
   const int64_t t16 = lora16_ld(T);
-  float* u_qkv = a.take<float>(T * 3 * r);
-  float* u_o = a.take<float>(T * r);
-  float* u_gu = a.take<float>(T * 2 * r);
-  float* u_d = a.take<float>(T * r);
+  uint16_t* uh_qkv = a.take<uint16_t>(T * 3 * r);
+  uint16_t* uh_o = a.take<uint16_t>(T * r);
+  uint16_t* uh_gu = a.take<uint16_t>(T * 2 * r);
+  uint16_t* uh_d = a.take<uint16_t>(T * r);
   uint16_t* u16_qkv = a.take<uint16_t>(t16 * 3 * r);
   uint16_t* u16_o = a.take<uint16_t>(t16 * r);
   uint16_t* u16_gu = a.take<uint16_t>(t16 * 2 * r);
   uint16_t* u16_d = a.take<uint16_t>(t16 * r);
   if (b && base) {
-    b->u_qkv = u_qkv;
-    b->u_o = u_o;
-    b->u_gu = u_gu;
-    b->u_d = u_d;
+    b->uh_qkv = uh_qkv;
+    b->uh_o = uh_o;
+    b->uh_gu = uh_gu;
+    b->uh_d = uh_d;
     b->u16_qkv = u16_qkv;
     b->u16_o = u16_o;
     b->u16_gu = u16_gu;
@@ -446,6 +474,14 @@ int attach_lora16(const LayerShapes& s, const float* lora, const uint16_t* lora1
   v->B16_o = lora16 + o.b[1];
   v->B16_gu = lora16 + o.b[2];
   v->B16_d = lora16 + o.b[3];
+  v->Bs16_qkv = lora16 + o.bs[0];
+  v->Bs16_o = lora16 + o.bs[1];
+  v->Bs16_gu = lora16 + o.bs[2];
+  v->Bs16_d = lora16 + o.bs[3];
+  v->At16_qkv = lora16 + o.at[0];
+  v->At16_o = lora16 + o.at[1];
+  v->At16_gu = lora16 + o.at[2];
+  v->At16_d = lora16 + o.at[3];
   return LSQ_OK;
 }
 
@@ -469,18 +505,16 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
   const int64_t T = (int64_t)batch * seq;
   const int r = v.lora_on ? s.r : 0;  // r = 0: no LoRA slab in the GEMMs
   const bool down = v.lora_on && !have_u;  // compute u = x A^T here
-  const int64_t pe3[3] = {s.qd, s.qd + s.kvd, s.qkv_n};
-  const int64_t pe2[2] = {s.F, s.gu_n};
   LSQ_TRY(launch_rmsnorm_fwd(x, v.g1, T, s.D, eps, b.n1, OUT_F16, b.rstd1, st));
   if (down)
-    LSQ_TRY(launch_lora_down16(b.n1, s.D, v.A16_qkv, T, s.D, 3 * r, b.u_qkv, b.u16_qkv, b.lscratch,
-                               b.lscratch_bytes, st));
+    LSQ_TRY(launch_lora_down16(b.n1, s.D, v.A16_qkv, T, s.D, 3 * r, nullptr, b.u16_qkv,
+                               b.lscratch, b.lscratch_bytes, st, b.uh_qkv));
   // A product split over K leaves its partials to the kernel after it (RoPE here,
   // the second RMSNorm after the o projection), which sums them in slice order.
   const float* parts = nullptr;
   int np = 1;
-  GemmDesc g_qkv = nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.B_qkv, r, s.s,
-                           b.u_qkv, 3 * r, 3, pe3, nullptr, b.qkv, s.qkv_n);
+  GemmDesc g_qkv = nf4_fwd(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.n1, T, v.Bs16_qkv, b.uh_qkv,
+                           3 * r, nullptr, b.qkv, s.qkv_n);
   g_qkv.parts_out = &parts;
   g_qkv.splits_out = &np;
   LSQ_TRY(gemm_run(g_qkv, b.gemm, b.gemm_bytes, st));
@@ -490,10 +524,10 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
     LSQ_TRY(launch_rope(b.qkv, T, seq, s.H, s.Hkv, s.hd, rope_cs, st));
   LSQ_TRY(launch_attention_fwd(b.qkv, T, seq, s.H, s.Hkv, s.hd, b.ao, b.lse, st));
   if (down)
-    LSQ_TRY(launch_lora_down16(b.ao, s.qd, v.A16_o, T, s.qd, r, b.u_o, b.u16_o, b.lscratch,
-                               b.lscratch_bytes, st));
-  GemmDesc g_o = nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.B_o, r, s.s, b.u_o, r, 1,
-                         pe3, x, b.h, s.D);
+    LSQ_TRY(launch_lora_down16(b.ao, s.qd, v.A16_o, T, s.qd, r, nullptr, b.u16_o, b.lscratch,
+                               b.lscratch_bytes, st, b.uh_o));
+  GemmDesc g_o = nf4_fwd(v.codes[3], v.absmax[3], s.D, s.qd, b.ao, T, v.Bs16_o, b.uh_o, r, x, b.h,
+                         s.D);
   g_o.parts_out = &parts;
   g_o.splits_out = &np;
   LSQ_TRY(gemm_run(g_o, b.gemm, b.gemm_bytes, st));
@@ -503,18 +537,18 @@ int forward_core(const LayerShapes& s, const Views& v, const float* x, int batch
   else
     LSQ_TRY(launch_rmsnorm_fwd(b.h, v.g2, T, s.D, eps, b.n2, OUT_F16, b.rstd2, st));
   if (down)
-    LSQ_TRY(launch_lora_down16(b.n2, s.D, v.A16_gu, T, s.D, 2 * r, b.u_gu, b.u16_gu, b.lscratch,
-                               b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.B_gu, r, s.s, b.u_gu,
-                           2 * r, 2, pe2, nullptr, b.gu, s.gu_n),
+    LSQ_TRY(launch_lora_down16(b.n2, s.D, v.A16_gu, T, s.D, 2 * r, nullptr, b.u16_gu, b.lscratch,
+                               b.lscratch_bytes, st, b.uh_gu));
+  LSQ_TRY(gemm_run(nf4_fwd(v.codes[4], v.absmax[4], s.gu_n, s.D, b.n2, T, v.Bs16_gu, b.uh_gu,
+                           2 * r, nullptr, b.gu, s.gu_n),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_swiglu_fwd(b.gu, T, s.F, b.m, st));
   if (down)
-    LSQ_TRY(launch_lora_down16(b.m, s.F, v.A16_d, T, s.F, r, b.u_d, b.u16_d, b.lscratch,
-                               b.lscratch_bytes, st));
+    LSQ_TRY(launch_lora_down16(b.m, s.F, v.A16_d, T, s.F, r, nullptr, b.u16_d, b.lscratch,
+                               b.lscratch_bytes, st, b.uh_d));
   if (x_out)
-    LSQ_TRY(gemm_run(nf4_fwd(v.codes[6], v.absmax[6], s.D, s.F, b.m, T, v.B_d, r, s.s, b.u_d, r, 1,
-                             pe3, b.h, x_out, s.D),
+    LSQ_TRY(gemm_run(nf4_fwd(v.codes[6], v.absmax[6], s.D, s.F, b.m, T, v.Bs16_d, b.uh_d, r, b.h,
+                             x_out, s.D),
                      b.gemm, b.gemm_bytes, st));
   return LSQ_OK;
 }
@@ -624,9 +658,10 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
     dout_b = b.dout_b;
   }
   // down projection
-  LSQ_TRY(launch_lora_vproj16(dout_b, T, s.D, v.B16_d, r, b.v_d, b.v16_d, b.lscratch,
-                              b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.A_d, r, sc, b.v_d, b.dm, 1),
+  LSQ_TRY(launch_lora_vproj16(dout_b, T, s.D, v.B16_d, r, nullptr, b.v16_d, b.lscratch,
+                              b.lscratch_bytes, st, b.vh_d));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.At16_d, b.vh_d, r, b.dm,
+                          1),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_lora_grad_a16(b.v16_d, b.m, T, s.F, r, sc, accumulate, gA_d, b.lscratch,
                                b.lscratch_bytes, st));
@@ -634,14 +669,14 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
                                b.lscratch_bytes, st));
   // SwiGLU and gate|up
   LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
-  LSQ_TRY(launch_lora_vproj16(b.dgu, T, s.gu_n, v.B16_gu, 2 * r, b.v_gu, b.v16_gu, b.lscratch,
-                              b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj16(b.dgu, T, s.gu_n, v.B16_gu, 2 * r, nullptr, b.v16_gu, b.lscratch,
+                              b.lscratch_bytes, st, b.vh_gu));
   // (a product split over K leaves its partials to the RMSNorm backward after it;
   // the rank-r products in between do not use the GEMM workspace)
   const float* parts = nullptr;
   int np = 1;
-  GemmDesc g_gu = nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.A_gu, 2 * r, sc,
-                         b.v_gu, b.dn2, 1);
+  GemmDesc g_gu = nf4_dx(v.codes[4], v.absmax[4], s.gu_n, s.D, b.dgu, T, v.At16_gu, b.vh_gu,
+                         2 * r, b.dn2, 1);
   g_gu.parts_out = &parts;
   g_gu.splits_out = &np;
   LSQ_TRY(gemm_run(g_gu, b.gemm, b.gemm_bytes, st));
@@ -656,9 +691,10 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   else
     LSQ_TRY(launch_rmsnorm_bwd(b.dn2, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b, st));
   // o projection
-  LSQ_TRY(launch_lora_vproj16(b.dh_b, T, s.D, v.B16_o, r, b.v_o, b.v16_o, b.lscratch,
-                              b.lscratch_bytes, st));
-  LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.A_o, r, sc, b.v_o, b.da, 0),
+  LSQ_TRY(launch_lora_vproj16(b.dh_b, T, s.D, v.B16_o, r, nullptr, b.v16_o, b.lscratch,
+                              b.lscratch_bytes, st, b.vh_o));
+  LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.At16_o, b.vh_o, r, b.da,
+                          0),
                    b.gemm, b.gemm_bytes, st));
   LSQ_TRY(launch_lora_grad_a16(b.v16_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, b.lscratch,
                                b.lscratch_bytes, st));
@@ -669,10 +705,10 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
                                b.dk, b.dv, st));
   LSQ_TRY(launch_rope_grad(b.dq, b.dk, b.dv, T, seq, s.H, s.Hkv, s.hd, rope_cs, b.dqkv, st));
   // q|k|v projections
-  LSQ_TRY(launch_lora_vproj16(b.dqkv, T, s.qkv_n, v.B16_qkv, 3 * r, b.v_qkv, b.v16_qkv,
-                              b.lscratch, b.lscratch_bytes, st));
-  GemmDesc g_qkv = nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.A_qkv, 3 * r, sc,
-                          b.v_qkv, b.dn1, 1);
+  LSQ_TRY(launch_lora_vproj16(b.dqkv, T, s.qkv_n, v.B16_qkv, 3 * r, nullptr, b.v16_qkv,
+                              b.lscratch, b.lscratch_bytes, st, b.vh_qkv));
+  GemmDesc g_qkv = nf4_dx(v.codes[0], v.absmax[0], s.qkv_n, s.D, b.dqkv, T, v.At16_qkv, b.vh_qkv,
+                          3 * r, b.dn1, 1);
   g_qkv.parts_out = &parts;
   g_qkv.splits_out = &np;
   LSQ_TRY(gemm_run(g_qkv, b.gemm, b.gemm_bytes, st));

@@ -58,6 +58,11 @@ struct SkinnyArgs {
   // keeps only columns [p part_r, (p + 1) part_r), written to column n - p part_r.
   uint16_t* c16;
   int64_t c16_m, c16_n;
+  // h16 (nullable): the result rounded to fp16 (h16_f16) or bf16 at
+  // h16[m * h16_m + n * h16_n] - the LoRA slab operand of the fused GEMM
+  uint16_t* h16;
+  int64_t h16_m, h16_n;
+  int h16_f16;
   int part_r, n_parts;
   int64_t part_end[4];
 };
@@ -71,9 +76,13 @@ __device__ __forceinline__ void store_result(const SkinnyArgs& a, int64_t m, int
     col = n - (int64_t)p * a.part_r;
     if (col < 0 || col >= a.part_r) return;
   }
-  float* d = a.dst + m * a.c_m + col * a.c_n;
-  *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
+  if (a.dst) {
+    float* d = a.dst + m * a.c_m + col * a.c_n;
+    *d = (a.accumulate ? *d : 0.f) + a.alpha * v;
+  }
   if (a.c16) a.c16[m * a.c16_m + n * a.c16_n] = float_to_bf16_bits(v);
+  if (a.h16)
+    a.h16[m * a.h16_m + n * a.h16_n] = a.h16_f16 ? float_to_f16_bits(v) : float_to_bf16_bits(v);
 }
 
 __device__ __forceinline__ uint8_t* align1024_s(uint8_t* p) {
@@ -446,12 +455,16 @@ size_t lora_scratch_bytes(int64_t T, int64_t K, int R) {
 
 int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int64_t T, int64_t K,
                        int R, float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
-                       cudaStream_t st) {
+                       cudaStream_t st, uint16_t* uh) {
   LSQ_TRY(check_ranks(R));
   if (K % 8 != 0 || ldx % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_down: K %% 8 != 0");
-  // C[t, j] = sum_k x[t, k] A[j, k]   (fp16 operands); u16 transposed [R][ld]
+  // C[t, j] = sum_k x[t, k] A[j, k]   (fp16 operands); u16 transposed [R][ld]; uh fp16 [T][R]
   const int prof = prof_begin(st);
   SkinnyArgs a = out_args(u, R, 1, 1.f, 0, u16, 1, lora16_ld(T));
+  a.h16 = uh;
+  a.h16_m = R;
+  a.h16_n = 1;
+  a.h16_f16 = 1;
   a.M = T; a.N = R; a.K = K;
   const Operand A{x, K, T, ldx, true}, B{A16, K, R, K, true};
   LSQ_TRY((run<false, false>(a, A, B, true, st)));
@@ -461,12 +474,16 @@ int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int6
 
 int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
                         float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
-                        cudaStream_t st) {
+                        cudaStream_t st, uint16_t* vh) {
   LSQ_TRY(check_ranks(R));
   if (N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_vproj: N %% 8 != 0");
-  // C[t, c] = sum_n dy[t, n] Bs^T[c, n]   (bf16 operands); v16 transposed [R][ld]
+  // C[t, c] = sum_n dy[t, n] Bs^T[c, n]   (bf16 operands); v16 transposed [R][ld]; vh bf16 [T][R]
   const int prof = prof_begin(st);
   SkinnyArgs a = out_args(v, R, 1, 1.f, 0, v16, 1, lora16_ld(T));
+  a.h16 = vh;
+  a.h16_m = R;
+  a.h16_n = 1;
+  a.h16_f16 = 0;
   a.M = T; a.N = R; a.K = N;
   const Operand A{dy, N, T, N, false}, B{Bs, N, R, N, false};
   LSQ_TRY((run<false, false>(a, A, B, false, st)));
@@ -551,13 +568,24 @@ __global__ void lora_prepare_kernel(const float* __restrict__ lora, int64_t lora
       if (g.kind == 0) {  // A: fp16 copy, [rows][cols]
         const int64_t row = i / g.ld_out, col = i % g.ld_out;
         dst[g.dst_off + i] = float_to_f16_bits(src[g.src_off + row * g.cols + col]);
-      } else {            // B: bf16 block-diagonal stack, transposed: [n_parts r][rows]
+      } else if (g.kind == 1) {  // B: bf16 block-diagonal stack, transposed: [n_parts r][rows]
         const int64_t j = i / g.rows, row = i % g.rows;
         int p = 0;
         while (p + 1 < g.n_parts && row >= g.part_end[p]) ++p;
         const int64_t jj = j - (int64_t)p * g.cols;
         const float v = (jj >= 0 && jj < g.cols) ? src[g.src_off + row * g.cols + jj] : 0.f;
         dst[g.dst_off + i] = float_to_bf16_bits(v);
+      } else if (g.kind == 2) {  // scale * B, fp16 block-diagonal stack: [rows][n_parts r]
+        const int64_t row = i / g.ld_out, j = i % g.ld_out;
+        int p = 0;
+        while (p + 1 < g.n_parts && row >= g.part_end[p]) ++p;
+        const int64_t jj = j - (int64_t)p * g.cols;
+        const float v = (jj >= 0 && jj < g.cols) ? g.scale * src[g.src_off + row * g.cols + jj]
+                                                 : 0.f;
+        dst[g.dst_off + i] = float_to_f16_bits(v);
+      } else {  // scale * A^T, bf16: A [ld_out][rows] -> [rows][ld_out]
+        const int64_t row = i / g.ld_out, j = i % g.ld_out;
+        dst[g.dst_off + i] = float_to_bf16_bits(g.scale * src[g.src_off + j * g.rows + row]);
       }
     }
   }
