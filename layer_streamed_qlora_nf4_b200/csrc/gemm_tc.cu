@@ -14,7 +14,8 @@
 //
 // Design for B200 (one CTA per SM, 384 threads, warp-specialised):
 //   warp 0    : TMA producer for the activation tile (128-byte swizzle) [and
-//               the bf16 weight tile in W_BF16_N mode]
+//               the bf16 weight tile in W_BF16_N mode, or in W_BF16_T mode as
+//               two MN-major 64-feature atoms, read by the MMA as an MN-major A]
 //   warp 1    : allocates TMEM, one elected thread issues tcgen05.mma
 //               (M = 128 output features x N = up to 256 tokens x K = 16),
 //               accumulators in TMEM (up to 2 x 256 fp32 columns)
@@ -224,7 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         if (it < n_main) {
           const int kt = kt_begin + it;
-          const uint32_t bytes = xs_bytes + (WMODE == W_BF16_N ? (uint32_t)kWStageBytes : 0u);
+          constexpr bool kWTma = WMODE == W_BF16_N || WMODE == W_BF16_T;  // W by TMA here
+          const uint32_t bytes = xs_bytes + (kWTma ? (uint32_t)kWStageBytes : 0u);
           if (PAIR) {
             // both CTAs' bytes complete on the even CTA's barrier
             const uint32_t fl = mapa_shared(fb, 0);
@@ -234,6 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                fl, kt * kBK, t0 + a * p.bn + (int)rank * hb);
             if (WMODE == W_BF16_N)
               tma_load_2d_pair(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fl, kt * kBK, m0);
+            if (WMODE == W_BF16_T)  // [64 contraction rows x 64 features], twice
+              for (int h2 = 0; h2 < 2; ++h2)
+                tma_load_2d_pair(smem_u32(ws0 + (size_t)s * kWStageBytes + h2 * (kWStageBytes / 2)),
+                                 &tm_w, fl, m0 + 64 * h2, kt * kBK);
           } else {
             mbar_arrive_expect_tx(fb, bytes);
             for (int a = 0; a < p.nacc; ++a)
@@ -241,6 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           fb, kt * kBK, t0 + a * p.bn);
             if (WMODE == W_BF16_N)
               tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, fb, kt * kBK, m0);
+            if (WMODE == W_BF16_T)
+              for (int h2 = 0; h2 < 2; ++h2)
+                tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes + h2 * (kWStageBytes / 2)),
+                            &tm_w, fb, m0 + 64 * h2, kt * kBK);
           }
         } else if (p.slab_tma) {
           // LoRA slab: s B (or s A^T) into the weight stage, u (or v) into the
@@ -271,6 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- MMA issuer (lane 0)
     const uint32_t idesc = F16 ? umma_idesc_f16(PAIR ? 2 * kBM : kBM, p.bn)
                                : umma_idesc_bf16(PAIR ? 2 * kBM : kBM, p.bn);
+    // W_BF16_T: the weight tile is MN-major (two 64-feature atoms of 64 contraction
+    // rows, 8 KB apart); the LoRA slab's A is K-major in every mode
+    constexpr bool kAMn = WMODE == W_BF16_T;
+    const uint32_t idesc_mn = idesc | (1u << 15);
 #ifdef LSQ_GEMM_STAMPS
     unsigned long long waited = 0;
 #endif
@@ -296,15 +310,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it >= n_main) nk = min(4, (p.slab_w - (it - n_main) * 64) / 16);
         const uint32_t wa = smem_u32(ws0 + (size_t)s * kWStageBytes);
         const uint32_t xa = smem_u32(xs0 + (size_t)s * xs_bytes);
+        const bool a_mn = kAMn && it < n_main;
+        const uint32_t id = a_mn ? idesc_mn : idesc;
         for (int kk = 0; kk < nk; ++kk) {
-          const uint64_t ad = umma_desc_k_sw128(wa + kk * 32);
+          const uint64_t ad =
+              a_mn ? umma_desc_mn_sw128(wa + (uint32_t)kk * 16 * 128, (uint32_t)kWStageBytes / 2, 1024u)
+                   : umma_desc_k_sw128(wa + kk * 32);
           for (int a = 0; a < p.nacc; ++a) {
             const uint64_t bd = umma_desc_k_sw128(xa + (uint32_t)(a * hb * 128) + kk * 32);
             if (PAIR)
-              tc_mma_bf16_pair(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
+              tc_mma_bf16_pair(tmem + (uint32_t)a * acc_stride, ad, bd, id,
                                (it > 0 || kk > 0) ? 1u : 0u);
             else
-              tc_mma_bf16(tmem + (uint32_t)a * acc_stride, ad, bd, idesc,
+              tc_mma_bf16(tmem + (uint32_t)a * acc_stride, ad, bd, id,
                           (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
@@ -341,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ---------------------------------------------------------- staging-ring TMA producer
-    if (WMODE != W_BF16_N) {
+    if (WMODE != W_BF16_N && WMODE != W_BF16_T) {
       for (int it = 0; it < n_main; ++it) {
         const int c = it % CS;
         const uint32_t ph = (uint32_t)(it / CS) & 1u;
@@ -425,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       issue_am(it + kAmDepth - 1);
       if (it < n_main) {
-        if (WMODE == W_BF16_N) {
+        if (WMODE == W_BF16_N || WMODE == W_BF16_T) {
           ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                  DEV_ERR_WAIT_GEMM);
           ok = __all_sync(0xFFFFFFFFu, ok);
@@ -511,25 +529,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(wst + off) = make_uint4(o[0], o[1], o[2], o[3]);
               }
               if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
-            } else if (tid < 128) {  // W_BF16_T: transpose a [64 x 128] bf16 tile into K-major
-              const int bi = tid & 7, bj = tid >> 3;
-              uint4 rowv[8];
-#pragma unroll
-              for (int rr = 0; rr < 8; ++rr)
-                rowv[rr] = *reinterpret_cast<const uint4*>(ring + (8 * bi + rr) * 256 + 16 * bj);
-#pragma unroll
-              for (int cc = 0; cc < 8; ++cc) {
-                uint32_t o[4];
-#pragma unroll
-                for (int pr = 0; pr < 4; ++pr) {
-                  const uint4 a = rowv[2 * pr], b = rowv[2 * pr + 1];
-                  const uint32_t wa = (cc >> 1) == 0 ? a.x : (cc >> 1) == 1 ? a.y : (cc >> 1) == 2 ? a.z : a.w;
-                  const uint32_t wb = (cc >> 1) == 0 ? b.x : (cc >> 1) == 1 ? b.y : (cc >> 1) == 2 ? b.z : b.w;
-                  o[pr] = (cc & 1) ? __byte_perm(wa, wb, 0x7632) : __byte_perm(wa, wb, 0x5410);
-                }
-                *reinterpret_cast<uint4*>(wst + sw128_offset(8 * bj + cc, bi)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
-              }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -812,10 +811,11 @@ Plan make_plan(const GemmDesc& d) {
   pl.kt_per_split = (pl.kt_total + splits - 1) / splits;
   pl.splits = (pl.kt_total + pl.kt_per_split - 1) / pl.kt_per_split;
   pl.partial_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)T * (size_t)d.M * 4 : 0;
-  const bool bf16_tile = d.wmode == W_BF16_T || d.wmode == W_BF16C_N;
-  pl.ring_bytes = bf16_tile ? 64 * 128 * 2 : (d.wmode == W_BF16_N ? 0 : 4096);
+  const bool bf16_tile = d.wmode == W_BF16C_N;
+  const bool w_tma = d.wmode == W_BF16_N || d.wmode == W_BF16_T;
+  pl.ring_bytes = bf16_tile ? 64 * 128 * 2 : (w_tma ? 0 : 4096);
   const uint32_t xs = (uint32_t)(pl.pair ? BT / 2 : BT) * 128;
-  int ring = (d.wmode == W_BF16_N) ? 0 : (bf16_tile ? 2 : kMaxRing);
+  int ring = w_tma ? 0 : (bf16_tile ? 2 : kMaxRing);
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
     return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes +
@@ -862,10 +862,10 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
                       (uint64_t)d.w_rows, (uint64_t)d.w_cols, kBK, kBM,
                       CU_TENSOR_MAP_SWIZZLE_128B));
-  if (WMODE == W_BF16_T)
+  if (WMODE == W_BF16_T)  // [64 contraction rows x 64 features] atoms, 128-byte swizzle
     LSQ_TRY(make_tmap(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d.w, (uint64_t)d.w_cols,
-                      (uint64_t)d.w_rows, (uint64_t)d.w_cols, 128, 64,
-                      CU_TENSOR_MAP_SWIZZLE_NONE));
+                      (uint64_t)d.w_rows, (uint64_t)d.w_cols, 64, kBK,
+                      CU_TENSOR_MAP_SWIZZLE_128B));
   CUtensorMap tm_out, tm_res;
   if (partial) {
     PFN_encodeTiled enc = get_encode();
