@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_cempty[kMaxRing];
   __shared__ __align__(8) uint64_t bar_acc;
   __shared__ __align__(8) uint64_t bar_opd[kMaxStages];  // PAIR, odd CTA: its operand warps done
+  __shared__ __align__(8) uint64_t bar_wland[kMaxStages];  // W_BF16C_N: this CTA's bf16 tile landed
   __shared__ __align__(8) uint64_t bar_res[kThreads / 32];  // per warp: residual tile landed
   __shared__ __align__(8) uint64_t bar_grp;            // the operand warps
   __shared__ uint32_t tmem_base_sh;
@@ -175,6 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // producer + this CTA's operand warps (+ one forwarded arrival from the odd CTA)
       mbar_init(smem_u32(&bar_full[s]), 1 + kOpWarps + (PAIR ? 1 : 0));
       mbar_init(smem_u32(&bar_opd[s]), kOpWarps);
+      mbar_init(smem_u32(&bar_wland[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);            // tcgen05.commit
     }
     for (int c = 0; c < CS; ++c) {
@@ -240,6 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int h2 = 0; h2 < 2; ++h2)
                 tma_load_2d_pair(smem_u32(ws0 + (size_t)s * kWStageBytes + h2 * (kWStageBytes / 2)),
                                  &tm_w, fl, m0 + 64 * h2, kt * kBK);
+            if (WMODE == W_BF16C_N) {  // converted in place by this CTA's operand warps
+              const uint32_t wl = smem_u32(&bar_wland[s]);
+              mbar_arrive_expect_tx(wl, (uint32_t)kWStageBytes);
+              tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, wl, kt * kBK, m0);
+            }
           } else {
             mbar_arrive_expect_tx(fb, bytes);
             for (int a = 0; a < p.nacc; ++a)
@@ -251,6 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int h2 = 0; h2 < 2; ++h2)
                 tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes + h2 * (kWStageBytes / 2)),
                             &tm_w, fb, m0 + 64 * h2, kt * kBK);
+            if (WMODE == W_BF16C_N) {
+              const uint32_t wl = smem_u32(&bar_wland[s]);
+              mbar_arrive_expect_tx(wl, (uint32_t)kWStageBytes);
+              tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, wl, kt * kBK, m0);
+            }
           }
         } else if (p.slab_tma) {
           // LoRA slab: s B (or s A^T) into the weight stage, u (or v) into the
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ---------------------------------------------------------- staging-ring TMA producer
-    if (WMODE != W_BF16_N && WMODE != W_BF16_T) {
+    if (WMODE == W_NF4_N || WMODE == W_NF4_T) {
       for (int it = 0; it < n_main; ++it) {
         const int c = it % CS;
         const uint32_t ph = (uint32_t)(it / CS) & 1u;
@@ -447,6 +459,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                  DEV_ERR_WAIT_GEMM);
           ok = __all_sync(0xFFFFFFFFu, ok);
+        } else if (WMODE == W_BF16C_N) {
+          // the bf16 [128 x 64] tile landed in the stage, already in the 128-byte-swizzle
+          // layout the MMA reads (its load was issued once the stage was free): convert
+          // each 16-byte chunk to fp16 in place.  A weight beyond the fp16 range latches
+          // the non-finite status bit.
+          ok = mbar_wait_bounded(smem_u32(&bar_wland[s]), ph, abort_flag, p.dev_err,
+                                 DEV_ERR_WAIT_GEMM);
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          if (ok) {
+            bool big = false;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int off = (tid + q * kOpThreads) * 16;
+              const uint4 v = *reinterpret_cast<const uint4*>(wst + off);
+              const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+              uint32_t o[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = unpack_bf16x2(in[e]);
+                big |= !(fabsf(f.x) <= kF16Max) || !(fabsf(f.y) <= kF16Max);
+                o[e] = pack_f16x2(f.x, f.y);
+              }
+              *reinterpret_cast<uint4*>(wst + off) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
         } else {
           const int c = it % CS;
           const uint32_t cph = (uint32_t)(it / CS) & 1u;
@@ -509,26 +549,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m = mq * 32 + (lane >> 3) * 8 + (lane & 7);
                 stmatrix_x4_trans(smem_u32(wst + sw128_offset(m, nb)), regs);
               }
-            } else if (WMODE == W_BF16C_N) {
-              // bf16 [128 x 64] tile, already in the 128-byte-swizzle layout the MMA
-              // reads: convert each 16-byte chunk to fp16 in place of its position.
-              // A weight beyond the fp16 range latches the non-finite status bit.
-              bool big = false;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int off = (tid + q * kOpThreads) * 16;
-                const uint4 v = *reinterpret_cast<const uint4*>(ring + off);
-                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 f = unpack_bf16x2(in[e]);
-                  big |= !(fabsf(f.x) <= kF16Max) || !(fabsf(f.y) <= kF16Max);
-                  o[e] = pack_f16x2(f.x, f.y);
-                }
-                *reinterpret_cast<uint4*>(wst + off) = make_uint4(o[0], o[1], o[2], o[3]);
-              }
-              if (__any_sync(0xFFFFFFFFu, big) && lane == 0) atomicOr(p.dev_err, DEV_ERR_NONFINITE);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -811,11 +831,10 @@ Plan make_plan(const GemmDesc& d) {
   pl.kt_per_split = (pl.kt_total + splits - 1) / splits;
   pl.splits = (pl.kt_total + pl.kt_per_split - 1) / pl.kt_per_split;
   pl.partial_bytes = pl.splits > 1 ? (size_t)pl.splits * (size_t)T * (size_t)d.M * 4 : 0;
-  const bool bf16_tile = d.wmode == W_BF16C_N;
-  const bool w_tma = d.wmode == W_BF16_N || d.wmode == W_BF16_T;
-  pl.ring_bytes = bf16_tile ? 64 * 128 * 2 : (w_tma ? 0 : 4096);
+  const bool w_tma = d.wmode == W_BF16_N || d.wmode == W_BF16_T || d.wmode == W_BF16C_N;
+  pl.ring_bytes = w_tma ? 0 : 4096;
   const uint32_t xs = (uint32_t)(pl.pair ? BT / 2 : BT) * 128;
-  int ring = w_tma ? 0 : (bf16_tile ? 2 : kMaxRing);
+  int ring = w_tma ? 0 : kMaxRing;
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
     return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes +
