@@ -603,6 +603,9 @@ __global__ void __launch_bounds__(kAThreads, 1)
         ppk[e >> 1] = pack_bf16x2(p[0], p[1]);
         dpk[e >> 1] = pack_bf16x2(d[0], d[1]);
       }
+      // S^T of this chunk is done with Q (its commit covered it): Q becomes dK's bf16
+      // operand, while the previous chunk's dV, dK products may still run
+      tile_f16_to_bf16(Qb + qb * SM::kQc, SM::kQc, tid);
       // the previous chunk's dV, dK products have read P^T and dS^T
       if (c > 0) {
         ok = mbar_wait_bounded(smem_u32(&bar_pds), (uint32_t)((c - 1) & 1), abort_flag, dev_err,
@@ -618,8 +621,6 @@ __global__ void __launch_bounds__(kAThreads, 1)
         *reinterpret_cast<uint4*>(dSt + off) =
             make_uint4(dpk[4 * cc], dpk[4 * cc + 1], dpk[4 * cc + 2], dpk[4 * cc + 3]);
       }
-      // S^T of this chunk is done with Q: Q becomes dK's bf16 operand
-      tile_f16_to_bf16(Qb + qb * SM::kQc, SM::kQc, tid);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -864,6 +865,9 @@ __global__ void __launch_bounds__(kAThreads, 1)
         }
         dpk[e >> 1] = pack_bf16x2(d[0], d[1]);
       }
+      // S of this chunk is done with K (its commit covered it): K becomes dQ's bf16
+      // operand, while the previous chunk's dQ product may still run
+      tile_f16_to_bf16(Kb + kb * SM::kKc, SM::kKc, tid);
       // the previous chunk's dQ product has read dS
       if (c > 0) {
         ok = mbar_wait_bounded(smem_u32(&bar_dsfree), (uint32_t)((c - 1) & 1), abort_flag, dev_err,
@@ -875,8 +879,6 @@ __global__ void __launch_bounds__(kAThreads, 1)
       for (int cc = 0; cc < 4; ++cc)
         *reinterpret_cast<uint4*>(dSs + sw128_offset((uint32_t)r, (uint32_t)(hf * 4 + cc))) =
             make_uint4(dpk[4 * cc], dpk[4 * cc + 1], dpk[4 * cc + 2], dpk[4 * cc + 3]);
-      // S of this chunk is done with K: K becomes dQ's bf16 operand
-      tile_f16_to_bf16(Kb + kb * SM::kKc, SM::kKc, tid);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
