@@ -116,6 +116,22 @@ def test_workspace_queries_are_host_only(L):
     assert L.stream_stack_dpo_workspace_bytes(synth.LLAMA8B, 33, 512) == 0
 
 
+def test_stack_workspace_holds_one_lm_head_chunk(L):
+    # The lm_head / loss run over chunks of whole sequences whose fp32 logits and bf16 logit
+    # gradients fit 4 GiB: below that, every sequence adds its V * seq * 6 bytes of logits to
+    # the step's workspace; above it, a sequence adds only its per-token tensors.
+    cfg = dict(synth.SMALL, vocab=128000)
+    seq = 64
+    per_seq_logits = cfg["vocab"] * seq * 6
+    per_chunk = (4 << 30) // per_seq_logits        # whole sequences per chunk
+    w = lambda b: L.stream_stack_workspace_bytes(cfg, b, seq)
+    below = w(per_chunk - 1) - w(per_chunk - 2)
+    above = w(per_chunk + 11) - w(per_chunk + 10)
+    assert below >= per_seq_logits
+    assert above < per_seq_logits // 4
+    assert w(4 * per_chunk) < w(per_chunk) + 3 * per_chunk * per_seq_logits // 4
+
+
 def test_invalid_arguments_are_rejected_without_a_gpu(L):
     lib = L.load()
     p = ctypes.c_void_p(16)   # never dereferenced: validation fails first
