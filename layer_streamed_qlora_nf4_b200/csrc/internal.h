@@ -235,6 +235,13 @@ int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int6
 int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
                          int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
                          float* scratch, size_t scratch_bytes, cudaStream_t st);
+// Both of a projection group's trainable gradients in one launch: dA as in
+// launch_lora_grad_a16 (v16 [R][lora16_ld(T)], x fp16 [T, K]) and dB as in
+// launch_lora_grad_b16 (dy bf16 [T, N], u16), with R = n_parts r
+int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, float* dA,
+                          const uint16_t* dy, const uint16_t* u16, int64_t N, int r, int n_parts,
+                          const int64_t* part_end, int64_t T, float s, int accumulate, float* dB,
+                          cudaStream_t st);
 // fp32-operand forms for a single linear (one part): the LoRA operand is rounded
 // once into the scratch first
 int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,

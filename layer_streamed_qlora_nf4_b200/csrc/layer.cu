@@ -663,10 +663,8 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   LSQ_TRY(gemm_run(nf4_dx(v.codes[6], v.absmax[6], s.D, s.F, dout_b, T, v.At16_d, b.vh_d, r, b.dm,
                           1),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a16(b.v16_d, b.m, T, s.F, r, sc, accumulate, gA_d, b.lscratch,
-                               b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b16(dout_b, b.u16_d, T, s.D, r, 1, pe1, sc, accumulate, gB_d, b.lscratch,
-                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_ab16(b.v16_d, b.m, s.F, gA_d, dout_b, b.u16_d, s.D, r, 1, pe1, T, sc,
+                                accumulate, gB_d, st));
   // SwiGLU and gate|up
   LSQ_TRY(launch_swiglu_bwd(b.dm, b.gu, T, s.F, b.dgu, st));
   LSQ_TRY(launch_lora_vproj16(b.dgu, T, s.gu_n, v.B16_gu, 2 * r, nullptr, b.v16_gu, b.lscratch,
@@ -680,10 +678,8 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   g_gu.parts_out = &parts;
   g_gu.splits_out = &np;
   LSQ_TRY(gemm_run(g_gu, b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a16(b.v16_gu, b.n2, T, s.D, 2 * r, sc, accumulate, gA_gu, b.lscratch,
-                               b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b16(b.dgu, b.u16_gu, T, s.gu_n, r, 2, pe2, sc, accumulate, gB_gu,
-                               b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_ab16(b.v16_gu, b.n2, s.D, gA_gu, b.dgu, b.u16_gu, s.gu_n, r, 2, pe2, T,
+                                sc, accumulate, gB_gu, st));
   // second RMSNorm + residual
   if (np > 1)
     LSQ_TRY(launch_rmsnorm_bwd_sum(parts, np, b.h, v.g2, b.rstd2, dx_out, T, s.D, b.dh, b.dh_b,
@@ -696,10 +692,8 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   LSQ_TRY(gemm_run(nf4_dx(v.codes[3], v.absmax[3], s.D, s.qd, b.dh_b, T, v.At16_o, b.vh_o, r, b.da,
                           0),
                    b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a16(b.v16_o, b.ao, T, s.qd, r, sc, accumulate, gA_o, b.lscratch,
-                               b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b16(b.dh_b, b.u16_o, T, s.D, r, 1, pe1, sc, accumulate, gB_o, b.lscratch,
-                               b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_ab16(b.v16_o, b.ao, s.qd, gA_o, b.dh_b, b.u16_o, s.D, r, 1, pe1, T, sc,
+                                accumulate, gB_o, st));
   // attention, RoPE
   LSQ_TRY(launch_attention_bwd(b.qkv, b.ao, b.da, b.lse, T, seq, s.H, s.Hkv, s.hd, b.delta, b.dq,
                                b.dk, b.dv, st));
@@ -712,10 +706,8 @@ int layer_bwd_impl(const lsq_cfg* cfg, const void* blob, const float* lora, cons
   g_qkv.parts_out = &parts;
   g_qkv.splits_out = &np;
   LSQ_TRY(gemm_run(g_qkv, b.gemm, b.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a16(b.v16_qkv, b.n1, T, s.D, 3 * r, sc, accumulate, gA_qkv, b.lscratch,
-                               b.lscratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b16(b.dqkv, b.u16_qkv, T, s.qkv_n, r, 3, pe3, sc, accumulate, gB_qkv,
-                               b.lscratch, b.lscratch_bytes, st));
+  LSQ_TRY(launch_lora_grad_ab16(b.v16_qkv, b.n1, s.D, gA_qkv, b.dqkv, b.u16_qkv, s.qkv_n, r, 3,
+                                pe3, T, sc, accumulate, gB_qkv, st));
   // first RMSNorm + residual
   if (np > 1)
     LSQ_TRY(launch_rmsnorm_bwd_sum(parts, np, x_in, v.g1, b.rstd1, b.dh, T, s.D, dx_in, dx_in_bf16,

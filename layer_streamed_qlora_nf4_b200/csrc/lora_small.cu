@@ -89,14 +89,20 @@ __device__ __forceinline__ uint8_t* align1024_s(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// A_MN: A is MN-major (its m index contiguous in memory); CONV: A is stored fp16
-// and converted to bf16 in shared memory before the MMA reads it.
+// A_MN: A is MN-major (its m index contiguous in memory).  One launch may carry two
+// products of the same width and reduction (the dA and dB of a projection group):
+// the first tiles1 row tiles (grid.x) are the first product's (tm_a, tm_b, a0), the
+// rest the second's (tm_a2, tm_b2, a1).  Bit i of conv_mask: product i's A is stored
+// fp16 and converted to bf16 in shared memory before the MMA reads it.
 //   warp 0: TMA producer (lane 0);  warp 1: TMEM and the MMA issuer (lane 0);
-//   warps 2-3: the conversion (CONV); all four: the epilogue (TMEM lane quarter = warp)
-template <bool A_MN, bool CONV>
+//   warps 2-3: the conversion; all four: the epilogue (TMEM lane quarter = warp)
+template <bool A_MN>
 __global__ void __launch_bounds__(kSThreads, 1)
     tc_skinny_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ SkinnyArgs a,
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_a2,
+                     const __grid_constant__ CUtensorMap tm_b2, const __grid_constant__ SkinnyArgs a0,
+                     const __grid_constant__ SkinnyArgs a1, int tiles1, int conv_mask,
                      uint32_t idesc, int n_pad, int stages, uint32_t tmem_cols, int* dev_err) {
   extern __shared__ uint8_t sk_raw[];
   constexpr int kMaxSt = 4;
@@ -110,7 +116,12 @@ __global__ void __launch_bounds__(kSThreads, 1)
   const uint32_t b_bytes = (uint32_t)n_pad * 128u;
   uint8_t* st0 = align1024_s(sk_raw);
   const uint32_t st_bytes = kSAStage + ((b_bytes + 1023u) & ~1023u);
-  const int64_t m0 = (int64_t)blockIdx.x * kSM;
+  const bool second = (int)blockIdx.x >= tiles1;
+  const SkinnyArgs& a = second ? a1 : a0;
+  const CUtensorMap* tma = second ? &tm_a2 : &tm_a;
+  const CUtensorMap* tmb = second ? &tm_b2 : &tm_b;
+  const bool CONV = ((conv_mask >> (second ? 1 : 0)) & 1) != 0;
+  const int64_t m0 = (int64_t)((int)blockIdx.x - (second ? tiles1 : 0)) * kSM;
   const int kt_total = (int)((a.K + kSK - 1) / kSK);
   const int kt_begin = (int)((int64_t)blockIdx.z * kt_total / a.splits);
   const int n_it = (int)((int64_t)(blockIdx.z + 1) * kt_total / a.splits) - kt_begin;
@@ -149,12 +160,12 @@ __global__ void __launch_bounds__(kSThreads, 1)
         const uint32_t fb = smem_u32(&bar_full[s]);
         mbar_arrive_expect_tx(fb, kSAStage + b_bytes);
         if (A_MN) {  // two [64 k x 64 m] boxes, 64 m apart
-          tma_load_2d(smem_u32(sa), &tm_a, fb, (int)m0, k0);
-          tma_load_2d(smem_u32(sa + kSAStage / 2), &tm_a, fb, (int)m0 + 64, k0);
+          tma_load_2d(smem_u32(sa), tma, fb, (int)m0, k0);
+          tma_load_2d(smem_u32(sa + kSAStage / 2), tma, fb, (int)m0 + 64, k0);
         } else {     // one [128 m x 64 k] box
-          tma_load_2d(smem_u32(sa), &tm_a, fb, k0, (int)m0);
+          tma_load_2d(smem_u32(sa), tma, fb, k0, (int)m0);
         }
-        tma_load_2d(smem_u32(sa + kSAStage), &tm_b, fb, k0, (int)blockIdx.y * n_pad);
+        tma_load_2d(smem_u32(sa + kSAStage), tmb, fb, k0, (int)blockIdx.y * n_pad);
       }
     }
     __syncwarp();
@@ -329,15 +340,18 @@ int splits_for(int64_t M, int64_t N, int64_t K) {
   return z;
 }
 
-template <bool A_MN, bool CONV>
-int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const SkinnyArgs& a, uint32_t idesc,
-              int n_pad, dim3 grid, cudaStream_t st) {
+// One launch of one product (second == nullptr) or of two products of the same
+// width and reduction length (dA and dB of a projection group) side by side.
+template <bool A_MN>
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const SkinnyArgs& a, bool conv,
+              const CUtensorMap* ta2, const CUtensorMap* tb2, const SkinnyArgs* a2, bool conv2,
+              int tiles1, uint32_t idesc, int n_pad, dim3 grid, cudaStream_t st) {
   const size_t smem = smem_for(n_pad);
   static bool attr[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr[dev]) {
-    LSQ_CUDA(cudaFuncSetAttribute(tc_skinny_kernel<A_MN, CONV>,
+    LSQ_CUDA(cudaFuncSetAttribute(tc_skinny_kernel<A_MN>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem_for(kSMaxN)));
     attr[dev] = true;
@@ -360,8 +374,10 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const SkinnyArgs& a,
   at[1].val.clusterDim.z = (unsigned)a.splits;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(&cfg, tc_skinny_kernel<A_MN, CONV>, ta, tb, a, idesc,
-                                              n_pad, stages_for(n_pad), cols, dev_err)));
+  const int mask = (conv ? 1 : 0) | ((a2 ? conv2 : conv) ? 2 : 0);
+  LSQ_CUDA(::lsq::launched(cudaLaunchKernelEx(
+      &cfg, tc_skinny_kernel<A_MN>, ta, tb, ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, a, a2 ? *a2 : a,
+      a2 ? tiles1 : (int)grid.x, mask, idesc, n_pad, stages_for(n_pad), cols, dev_err)));
   return LSQ_OK;
 }
 
@@ -371,6 +387,17 @@ struct Operand {
   int64_t inner, rows, ld;  // elements per row, rows, row stride (elements)
   bool f16;
 };
+
+int tmaps_for(bool a_mn, const Operand& A, const Operand& B, int n_pad, CUtensorMap* ta,
+              CUtensorMap* tb) {
+  const CUtensorMapDataType dta = A.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dtb = B.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  LSQ_TRY(make_tmap_2d(ta, dta, 2, A.p, (uint64_t)A.inner, (uint64_t)A.rows, (uint64_t)A.ld, 64,
+                       a_mn ? 64 : kSM, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(make_tmap_2d(tb, dtb, 2, B.p, (uint64_t)B.inner, (uint64_t)B.rows, (uint64_t)B.ld, 64,
+                       (uint32_t)n_pad, CU_TENSOR_MAP_SWIZZLE_128B));
+  return LSQ_OK;
+}
 
 // C = A B^T over K (A: M x K, K-major unless A_MN; B: N x K, K-major), written as
 // a prescribes (dst, alpha, accumulate, c16, parts).  CONV: A is fp16 and meets a
@@ -383,17 +410,33 @@ int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, cudaStream_t
   const int z = splits_for(a.M, a.N, a.K);  // every slice gets at least two stages
   a.splits = z;
   CUtensorMap ta, tb;
-  const CUtensorMapDataType dta = A.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const CUtensorMapDataType dtb = B.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  LSQ_TRY(make_tmap_2d(&ta, dta, 2, A.p, (uint64_t)A.inner, (uint64_t)A.rows, (uint64_t)A.ld, 64,
-                       A_MN ? 64 : kSM, CU_TENSOR_MAP_SWIZZLE_128B));
-  LSQ_TRY(make_tmap_2d(&tb, dtb, 2, B.p, (uint64_t)B.inner, (uint64_t)B.rows, (uint64_t)B.ld, 64,
-                       (uint32_t)n_pad, CU_TENSOR_MAP_SWIZZLE_128B));
+  LSQ_TRY(tmaps_for(A_MN, A, B, n_pad, &ta, &tb));
   uint32_t idesc = f16 ? umma_idesc_f16(kSM, n_pad) : umma_idesc_bf16(kSM, n_pad);
   if (A_MN) idesc |= 1u << 15;  // A MN-major
   const dim3 grid((unsigned)((a.M + kSM - 1) / kSM), (unsigned)((a.N + n_pad - 1) / n_pad),
                   (unsigned)z);
-  return launch_tc<A_MN, CONV>(ta, tb, a, idesc, n_pad, grid, st);
+  return launch_tc<A_MN>(ta, tb, a, CONV, nullptr, nullptr, nullptr, false, 0, idesc, n_pad,
+                         grid, st);
+}
+
+// Two token-reduction products (MN-major A, bf16) of the same width N and
+// reduction K in one launch: the first's row tiles, then the second's.  The
+// reduction is split for their tiles together.
+int run_pair_mn(SkinnyArgs a, const Operand& A, bool conv, SkinnyArgs b, const Operand& Ab,
+                bool conv_b, const Operand& B, const Operand& Bb, cudaStream_t st) {
+  if (a.N <= 0 || a.N != b.N || a.K != b.K) return set_error(LSQ_ERR_SHAPE, "lora pair: widths");
+  if (a.K <= 0) return set_error(LSQ_ERR_SHAPE, "lora product: empty reduction");
+  const int n_pad = npad_for(a.N);
+  const int64_t t1 = (a.M + kSM - 1) / kSM, t2 = (b.M + kSM - 1) / kSM;
+  const int z = splits_for((t1 + t2) * kSM, a.N, a.K);
+  a.splits = b.splits = z;
+  CUtensorMap ta, tb, ta2, tb2;
+  LSQ_TRY(tmaps_for(true, A, B, n_pad, &ta, &tb));
+  LSQ_TRY(tmaps_for(true, Ab, Bb, n_pad, &ta2, &tb2));
+  const uint32_t idesc = umma_idesc_bf16(kSM, n_pad) | (1u << 15);  // A MN-major
+  const dim3 grid((unsigned)(t1 + t2), (unsigned)((a.N + n_pad - 1) / n_pad), (unsigned)z);
+  return launch_tc<true>(ta, tb, a, conv, &ta2, &tb2, &b, conv_b, (int)t1, idesc, n_pad, grid,
+                         st);
 }
 
 int check_ranks(int64_t R) {
@@ -526,6 +569,36 @@ int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int
   const Operand A{dy, N, T, N, false}, B{u16, T, R, lora16_ld(T), false};
   LSQ_TRY((run<true, false>(a, A, B, false, st)));
   if (prof >= 0) prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * R * N, 2.0 * T * N + 2.0 * T * R);
+  return LSQ_OK;
+}
+
+int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, float* dA,
+                          const uint16_t* dy, const uint16_t* u16, int64_t N, int r, int n_parts,
+                          const int64_t* part_end, int64_t T, float s, int accumulate, float* dB,
+                          cudaStream_t st) {
+  const int R = n_parts * r;
+  LSQ_TRY(check_ranks(R));
+  if (n_parts < 1 || n_parts > 4) return set_error(LSQ_ERR_SHAPE, "lora_grad_ab: 1..4 parts");
+  if (K % 8 != 0 || N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_ab: K, N %% 8 != 0");
+  if (T <= 0) return LSQ_OK;
+  // dA as in launch_lora_grad_a16 (x converted to bf16 in shared memory), dB as in
+  // launch_lora_grad_b16, one launch
+  const int prof = prof_begin(st);
+  SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0, 0);
+  a.M = K; a.N = R; a.K = T;
+  SkinnyArgs b = out_args(dB, r, 1, s, accumulate, nullptr, 0, 0);
+  b.M = N; b.N = R; b.K = T;
+  if (n_parts > 1) {
+    b.part_r = r;
+    b.n_parts = n_parts;
+    for (int q = 0; q < n_parts; ++q) b.part_end[q] = part_end[q];
+  }
+  const Operand Aa{x, K, T, K, true}, Ba{v16, T, R, lora16_ld(T), false};
+  const Operand Ab{dy, N, T, N, false}, Bb{u16, T, R, lora16_ld(T), false};
+  LSQ_TRY(run_pair_mn(a, Aa, true, b, Ab, false, Ba, Bb, st));
+  if (prof >= 0)
+    prof_end(prof, st, "lora_rank_r_dAdB", 2.0 * T * R * (K + N),
+             2.0 * T * K + 2.0 * T * N + 4.0 * T * R);
   return LSQ_OK;
 }
 
