@@ -205,9 +205,6 @@ extern "C" int nf4_lora_linear_bwd(const uint16_t* dy, const uint16_t* x, int64_
   LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, w.v, w.v16, w.scratch, w.scratch_bytes, st));
   GemmDesc d = bwd_desc(dy, T, K, N, codes, absmax, A, r, scale, w.v, dx);
   LSQ_TRY(gemm_run(d, w.gemm, w.gemm_bytes, st));
-  LSQ_TRY(launch_lora_grad_a16(w.v16, x, T, K, r, scale, accumulate, dA, w.scratch,
-                               w.scratch_bytes, st));
-  LSQ_TRY(launch_lora_grad_b16(dy, w.u16, T, N, r, 1, pe, scale, accumulate, dB, w.scratch,
-                               w.scratch_bytes, st));
-  return LSQ_OK;
+  return launch_lora_grad_ab16(w.v16, x, K, dA, dy, w.u16, N, r, 1, pe, T, scale, accumulate, dB,
+                               st);
 }

@@ -225,19 +225,12 @@ int launch_lora_down16(const uint16_t* x, int64_t ldx, const uint16_t* A16, int6
 int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t* Bs, int R,
                         float* v, uint16_t* v16, float* scratch, size_t scratch_bytes,
                         cudaStream_t st, uint16_t* vh = nullptr);
-// dA[j, k] (+)= s sum_t v[t, j] x[t, k]  v16 bf16 [R, lora16_ld(T)], x fp16 [T, K] (converted
-// to bf16 as it is loaded)
-int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
-                         float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
-                         cudaStream_t st);
-// dB[n, j] (+)= s sum_t dy[t, n] u[t, part(n) r + j]   dy bf16 [T, N], u16 bf16
-// [n_parts r, lora16_ld(T)]; one product over all parts (parts of rows ending at part_end[])
-int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
-                         int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
-                         float* scratch, size_t scratch_bytes, cudaStream_t st);
-// Both of a projection group's trainable gradients in one launch: dA as in
-// launch_lora_grad_a16 (v16 [R][lora16_ld(T)], x fp16 [T, K]) and dB as in
-// launch_lora_grad_b16 (dy bf16 [T, N], u16), with R = n_parts r
+// Both of a projection group's trainable gradients in one launch, R = n_parts r:
+//   dA[j, k] (+)= s sum_t v[t, j] x[t, k]        v16 bf16 [R, lora16_ld(T)], x fp16 [T, K]
+//                                                (converted to bf16 as it is loaded);
+//   dB[n, j] (+)= s sum_t dy[t, n] u[t, part(n) r + j]   dy bf16 [T, N], u16 bf16
+//                                                [R, lora16_ld(T)], the rows of dB split into
+//                                                parts ending at part_end[].
 int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, float* dA,
                           const uint16_t* dy, const uint16_t* u16, int64_t N, int r, int n_parts,
                           const int64_t* part_end, int64_t T, float s, int accumulate, float* dB,

@@ -534,44 +534,6 @@ int launch_lora_vproj16(const uint16_t* dy, int64_t T, int64_t N, const uint16_t
   return LSQ_OK;
 }
 
-int launch_lora_grad_a16(const uint16_t* v16, const uint16_t* x, int64_t T, int64_t K, int R,
-                         float s, int accumulate, float* dA, float* scratch, size_t scratch_bytes,
-                         cudaStream_t st) {
-  LSQ_TRY(check_ranks(R));
-  if (K % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_a: K %% 8 != 0");
-  // C[k, j] = sum_t x[t, k] v[t, j];  dA[j, k] (+)= s C[k, j]   (x converted from fp16 to bf16)
-  const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0, 0);
-  a.M = K; a.N = R; a.K = T;
-  const Operand A{x, K, T, K, true}, B{v16, T, R, lora16_ld(T), false};
-  LSQ_TRY((run<true, true>(a, A, B, false, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dA", 2.0 * T * R * K, 2.0 * T * K + 2.0 * T * R);
-  return LSQ_OK;
-}
-
-int launch_lora_grad_b16(const uint16_t* dy, const uint16_t* u16, int64_t T, int64_t N, int r,
-                         int n_parts, const int64_t* part_end, float s, int accumulate, float* dB,
-                         float* scratch, size_t scratch_bytes, cudaStream_t st) {
-  const int R = n_parts * r;
-  LSQ_TRY(check_ranks(R));
-  if (n_parts < 1 || n_parts > 4) return set_error(LSQ_ERR_SHAPE, "lora_grad_b: 1..4 parts");
-  if (N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_b: N %% 8 != 0");
-  // C[n, c] = sum_t dy[t, n] u[t, c];  dB[n, j] (+)= s C[n, part(n) r + j]: one product over
-  // all parts, each row keeping its own part's columns
-  const int prof = prof_begin(st);
-  SkinnyArgs a = out_args(dB, r, 1, s, accumulate, nullptr, 0, 0);
-  a.M = N; a.N = R; a.K = T;
-  if (n_parts > 1) {
-    a.part_r = r;
-    a.n_parts = n_parts;
-    for (int p = 0; p < n_parts; ++p) a.part_end[p] = part_end[p];
-  }
-  const Operand A{dy, N, T, N, false}, B{u16, T, R, lora16_ld(T), false};
-  LSQ_TRY((run<true, false>(a, A, B, false, st)));
-  if (prof >= 0) prof_end(prof, st, "lora_rank_r_dB", 2.0 * T * R * N, 2.0 * T * N + 2.0 * T * R);
-  return LSQ_OK;
-}
-
 int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, float* dA,
                           const uint16_t* dy, const uint16_t* u16, int64_t N, int r, int n_parts,
                           const int64_t* part_end, int64_t T, float s, int accumulate, float* dB,
@@ -581,8 +543,9 @@ int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, flo
   if (n_parts < 1 || n_parts > 4) return set_error(LSQ_ERR_SHAPE, "lora_grad_ab: 1..4 parts");
   if (K % 8 != 0 || N % 8 != 0) return set_error(LSQ_ERR_SHAPE, "lora_grad_ab: K, N %% 8 != 0");
   if (T <= 0) return LSQ_OK;
-  // dA as in launch_lora_grad_a16 (x converted to bf16 in shared memory), dB as in
-  // launch_lora_grad_b16, one launch
+  // dA: C[k, j] = sum_t x[t, k] v[t, j], dA[j, k] (+)= s C[k, j] (x converted from fp16 to
+  // bf16 as it lands); dB: C[n, c] = sum_t dy[t, n] u[t, c], dB[n, j] (+)= s C[n, part(n) r +
+  // j], each row keeping its own part's columns; one launch
   const int prof = prof_begin(st);
   SkinnyArgs a = out_args(dA, 1, K, s, accumulate, nullptr, 0, 0);
   a.M = K; a.N = R; a.K = T;
