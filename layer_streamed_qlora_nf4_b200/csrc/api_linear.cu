@@ -30,10 +30,13 @@ int cuda_status(cudaError_t e, const char* what) {
 namespace {
 
 struct LinearWs {
-  float* u;
-  float* v;
-  uint16_t* u16;  // bf16 copies for the dA / dB products
+  float* u;       // u = x A^T, fp32 (the forward's optional output)
+  uint16_t* u16;  // bf16 copies of u, v for the dA / dB products ([r][lora16_ld(T)])
   uint16_t* v16;
+  uint16_t* uh;   // the GEMMs' LoRA slab operands: u in fp16 [T][r], v in bf16 [T][r],
+  uint16_t* vh;   //   s B in fp16 [N][r], s A^T in bf16 [K][r]
+  uint16_t* sb;
+  uint16_t* sat;
   float* scratch;
   size_t scratch_bytes;
   void* gemm;
@@ -41,7 +44,7 @@ struct LinearWs {
 };
 
 GemmDesc fwd_desc(const uint16_t* x, int64_t T, int64_t K, int64_t N, const uint8_t* codes,
-                  const float* absmax, const float* B, int r, float scale, const float* u,
+                  const float* absmax, const uint16_t* sb, int r, const uint16_t* uh,
                   const float* residual, void* y, int y_f32) {
   GemmDesc d;
   d.wmode = W_NF4_N;
@@ -55,12 +58,10 @@ GemmDesc fwd_desc(const uint16_t* x, int64_t T, int64_t K, int64_t N, const uint
   d.act = x;
   d.act_ld = K;
   d.slab_w = r;
-  d.la = B;
-  d.la_rs = r;
-  d.la_cs = 1;
-  d.la_scale = scale;
-  d.lb = u;
-  d.lb_ld = r;
+  d.la16 = sb;
+  d.la16_ld = r;
+  d.lb16 = uh;
+  d.lb16_ld = r;
   d.out = y;
   d.out_f32 = y_f32;
   d.ldo = N;
@@ -70,7 +71,7 @@ GemmDesc fwd_desc(const uint16_t* x, int64_t T, int64_t K, int64_t N, const uint
 }
 
 GemmDesc bwd_desc(const uint16_t* dy, int64_t T, int64_t K, int64_t N, const uint8_t* codes,
-                  const float* absmax, const float* A, int r, float scale, const float* v,
+                  const float* absmax, const uint16_t* sat, int r, const uint16_t* vh,
                   uint16_t* dx) {
   GemmDesc d;
   d.wmode = W_NF4_T;
@@ -84,12 +85,10 @@ GemmDesc bwd_desc(const uint16_t* dy, int64_t T, int64_t K, int64_t N, const uin
   d.act = dy;
   d.act_ld = N;
   d.slab_w = r;
-  d.la = A;
-  d.la_rs = 1;
-  d.la_cs = K;
-  d.la_scale = scale;
-  d.lb = v;
-  d.lb_ld = r;
+  d.la16 = sat;
+  d.la16_ld = r;
+  d.lb16 = vh;
+  d.lb16_ld = r;
   d.out = dx;
   d.ldo = K;
   return d;
@@ -98,30 +97,55 @@ GemmDesc bwd_desc(const uint16_t* dy, int64_t T, int64_t K, int64_t N, const uin
 size_t linear_ws_plan(int64_t T, int64_t K, int64_t N, int r, LinearWs* w, void* base) {
   const size_t sb = std::max(lora_scratch_bytes(T, K, r), lora_scratch_bytes(T, N, r));
   const size_t gb = std::max(
-      gemm_workspace_bytes(fwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, 0, nullptr,
+      gemm_workspace_bytes(fwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, nullptr,
                                     nullptr, nullptr, 0)),
-      gemm_workspace_bytes(bwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, 0, nullptr,
+      gemm_workspace_bytes(bwd_desc(nullptr, T, K, N, nullptr, nullptr, nullptr, r, nullptr,
                                     nullptr)));
   Arena b;
   b.base = static_cast<uint8_t*>(base);
   b.cap = SIZE_MAX;
   float* u = b.take<float>((size_t)T * r);
-  float* v = b.take<float>((size_t)T * r);
   uint16_t* u16 = b.take<uint16_t>((size_t)lora16_ld(T) * r);  // [r][lora16_ld(T)]
   uint16_t* v16 = b.take<uint16_t>((size_t)lora16_ld(T) * r);
+  uint16_t* uh = b.take<uint16_t>((size_t)T * r);
+  uint16_t* vh = b.take<uint16_t>((size_t)T * r);
+  uint16_t* sbm = b.take<uint16_t>((size_t)N * r);
+  uint16_t* sat = b.take<uint16_t>((size_t)K * r);
   float* s = b.take<float>(sb / sizeof(float) + 1);
   void* g = b.take<uint8_t>(gb + 256);
   if (w) {
     w->u = base ? u : nullptr;
-    w->v = base ? v : nullptr;
     w->u16 = base ? u16 : nullptr;
     w->v16 = base ? v16 : nullptr;
+    w->uh = base ? uh : nullptr;
+    w->vh = base ? vh : nullptr;
+    w->sb = base ? sbm : nullptr;
+    w->sat = base ? sat : nullptr;
     w->scratch = base ? s : nullptr;
     w->scratch_bytes = sb;
     w->gemm = base ? g : nullptr;
     w->gemm_bytes = gb + 256;
   }
   return b.used;
+}
+
+// The slab operand s B (fp16 [N][r], kind 2) or s A^T (bf16 [K][r] from A [r][K],
+// kind 3) of one linear, rounded from the caller's fp32 matrix.
+int prepare_slab(const float* src, int kind, int64_t rows, int r, float scale, uint16_t* out,
+                 cudaStream_t st) {
+  LoraPrepSegs g{};
+  LoraPrepSeg& e = g.seg[0];
+  e.kind = kind;
+  e.src_off = 0;
+  e.dst_off = 0;
+  e.rows = rows;
+  e.cols = r;
+  e.ld_out = r;
+  e.n_parts = 1;
+  e.part_end[0] = rows;
+  e.scale = scale;
+  g.n = 1;
+  return launch_lora_prepare(src, 0, 1, out, 0, g, st);
 }
 
 int check_linear(const void* x, int64_t T, int64_t K, int64_t N, const void* codes,
@@ -182,8 +206,9 @@ extern "C" int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int6
   linear_ws_plan(T, K, N, r, &w, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* u = u_out ? u_out : w.u;
-  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, u, nullptr, w.scratch, w.scratch_bytes, st));
-  GemmDesc d = fwd_desc(x, T, K, N, codes, absmax, B, r, scale, u, residual, y, y_fp32);
+  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, u, nullptr, w.scratch, w.scratch_bytes, st, w.uh));
+  LSQ_TRY(prepare_slab(B, 2, N, r, scale, w.sb, st));
+  GemmDesc d = fwd_desc(x, T, K, N, codes, absmax, w.sb, r, w.uh, residual, y, y_fp32);
   return gemm_run(d, w.gemm, w.gemm_bytes, st);
 }
 
@@ -201,9 +226,10 @@ extern "C" int nf4_lora_linear_bwd(const uint16_t* dy, const uint16_t* x, int64_
   linear_ws_plan(T, K, N, r, &w, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t pe[1] = {N};
-  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, w.u, w.u16, w.scratch, w.scratch_bytes, st));
-  LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, w.v, w.v16, w.scratch, w.scratch_bytes, st));
-  GemmDesc d = bwd_desc(dy, T, K, N, codes, absmax, A, r, scale, w.v, dx);
+  LSQ_TRY(launch_lora_down(x, K, A, T, K, r, nullptr, w.u16, w.scratch, w.scratch_bytes, st));
+  LSQ_TRY(launch_lora_vproj(dy, T, N, B, r, nullptr, w.v16, w.scratch, w.scratch_bytes, st, w.vh));
+  LSQ_TRY(prepare_slab(A, 3, K, r, scale, w.sat, st));
+  GemmDesc d = bwd_desc(dy, T, K, N, codes, absmax, w.sat, r, w.vh, dx);
   LSQ_TRY(gemm_run(d, w.gemm, w.gemm_bytes, st));
   return launch_lora_grad_ab16(w.v16, x, K, dA, dy, w.u16, N, r, 1, pe, T, scale, accumulate, dB,
                                st);

@@ -13,33 +13,34 @@
 // range); both accumulate in fp32 in TMEM.
 //
 // Design for B200 (one CTA per SM, 384 threads, warp-specialised):
-//   warp 0    : TMA producer for the activation tile (128-byte swizzle) [and
-//               the bf16 weight tile in W_BF16_N mode, or in W_BF16_T mode as
-//               two MN-major 64-feature atoms, read by the MMA as an MN-major A]
+//   warp 0    : TMA producer for the activation tile (128-byte swizzle), the LoRA
+//               slab's operands (la into the weight stage, lb into the activation
+//               stage) and, in the bf16-weight modes, the weight tile itself:
+//               K-major for W_BF16_N and W_BF16C_N (converted to fp16 in place by
+//               the operand warps), as two MN-major 64-feature atoms for W_BF16_T
+//               (read by the MMA as an MN-major A)
 //   warp 1    : allocates TMEM, one elected thread issues tcgen05.mma
 //               (M = 128 output features x N = up to 256 tokens x K = 16),
 //               accumulators in TMEM (up to 2 x 256 fp32 columns)
-//   warp 2    : TMA producer for the packed NF4 codes (or the bf16 tile to be
-//               transposed) into a deep staging ring
+//   warp 2    : TMA producer for the packed NF4 codes into a deep staging ring
 //   warps 4-11: operand stage - expand the staged codes to fp16 / bf16
 //               (level[code] * absmax in fp32, then round to nearest) straight into the
 //               UMMA canonical K-major 128-byte-swizzle layout, fence the async
-//               proxy, arrive; they also write the LoRA slab.  Two warps per
-//               SM sub-partition, because expanding the codes, not the tensor
-//               core, sets the pace of a k-tile.  Then the epilogue: each warp
-//               reads its TMEM lane quarter (32 features) for every other
+//               proxy, arrive.  Two warps per SM sub-partition.  Then the epilogue:
+//               each warp reads its TMEM lane quarter (32 features) for every third
 //               32-token chunk and writes it with its own TMA stores, with no
 //               barrier between warps.
 // The output tile is 128 features x all tokens of the CTA (up to 512), so each
 // weight element is dequantised once per token tile.  Small problems use a
-// fixed-order split over K with an fp32 partial buffer and a separate reduce:
-// results are deterministic and independent of scheduling.
+// fixed-order split over K with an fp32 partial buffer, summed in slice order by a
+// reduce kernel or by the kernel that consumes the product: results are
+// deterministic and independent of scheduling.
 // Every mbarrier wait is bounded (1 s) and aborts the CTA with a device status
 // bit instead of hanging.
 // Launch: programmatic dependent launch, so that the set-up (barriers, TMEM) and
 // the first weight stages - the frozen weight does not depend on the kernel
-// before - overlap that kernel's last wave; the activation loads, the LoRA slab
-// and the epilogue wait for it (pdl_wait).
+// before - overlap that kernel's last wave; the activation and slab loads and the
+// epilogue wait for it (pdl_wait).
 #include <cuda.h>
 
 #include <cstdlib>
@@ -93,14 +94,7 @@ struct KParams {
   const uint8_t* am_q;  // 8-bit absmax mode when non-null
   const float* am_s;
   int w_rows, w_cols;
-  int slab_w, part_r, n_parts;
-  int slab_tma;  // the slab's operands arrive by TMA (tm_la, tm_lb) instead of la / lb
-  const float* la;
-  long long la_rs, la_cs;
-  float la_scale;
-  const float* lb;
-  long long lb_ld;
-  long long part_end[4];
+  int slab_w;
   void* out;
   int out_f32;
   long long ldo;
@@ -264,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(smem_u32(ws0 + (size_t)s * kWStageBytes), &tm_w, wl, kt * kBK, m0);
             }
           }
-        } else if (p.slab_tma) {
+        } else if (p.slab_w > 0) {
           // LoRA slab: s B (or s A^T) into the weight stage, u (or v) into the
           // activation stage, 64 slab columns at a time (beyond slab_w: zeros)
           const int j0 = (it - n_main) * 64;
@@ -555,59 +549,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(smem_u32(&bar_cempty[c]));
           }
         }
-      } else if (p.slab_tma) {
-        // LoRA slab by TMA: the stage only has to be free before this warp arrives
-        ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
-                               DEV_ERR_WAIT_GEMM);
-        ok = __all_sync(0xFFFFFFFFu, ok);
       } else {
-        // LoRA slab: la -> weight stage, lb -> activation stage (lb comes from the
-        // kernel before: wait for it)
-        pdl_wait();
+        // LoRA slab (by TMA, issued by warp 0): the stage only has to be free before
+        // this warp arrives
         ok = mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                DEV_ERR_WAIT_GEMM);
         ok = __all_sync(0xFFFFFFFFu, ok);
-        if (ok) {
-          const int j0 = (it - n_main) * 64;
-          const int wq = min(64, p.slab_w - j0) / 8;  // chunks of 8 slab columns
-          for (int i = tid; i < 128 * wq; i += kOpThreads) {
-            const int row = i & 127, q = i >> 7;
-            const int m = m0 + row;
-            int jlo = 0;  // this row's slab columns: [jlo, jlo + part_r) of a stacked weight
-            if (p.part_r > 0) {
-              int part = 0;
-              while (part + 1 < p.n_parts && m >= p.part_end[part]) ++part;
-              jlo = part * p.part_r;
-            }
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int j = j0 + 8 * q + e;
-              const int jl = j - jlo;
-              const bool in = m < p.M && (p.part_r == 0 || (jl >= 0 && jl < p.part_r));
-              v[e] = in ? p.la_scale * __ldg(p.la + (long long)m * p.la_rs + (long long)jl * p.la_cs)
-                        : 0.f;
-            }
-            *reinterpret_cast<uint4*>(wst + sw128_offset(row, q)) =
-                make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]),
-                           pack2(v[6], v[7]));
-          }
-          uint8_t* xst = xs0 + (size_t)s * xs_bytes;
-          const int HT = p.nacc * hb;  // token rows of this CTA's activation stage
-          for (int i = tid; i < HT * wq; i += kOpThreads) {
-            const int t = i % HT, q = i / HT;
-            const int tg = t0 + (t / hb) * p.bn + (int)rank * hb + t % hb;
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              v[e] = (tg < p.T) ? __ldg(p.lb + (long long)tg * p.lb_ld + j0 + 8 * q + e) : 0.f;
-            *reinterpret_cast<uint4*>(xst + sw128_offset(t, q)) =
-                make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]),
-                           pack2(v[6], v[7]));
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
       }
       if (ok && lane == 0)
         mbar_arrive(smem_u32(PAIR && !leader ? &bar_opd[s] : &bar_full[s]));
@@ -910,9 +857,8 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
                       (uint64_t)d.T, (uint64_t)d.ldr, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE));
   else
     tm_res = tm_out;  // unused
-  CUtensorMap tm_la = tm_out, tm_lb = tm_out;  // unused without a TMA-fed slab
-  const bool slab_tma = d.slab_w > 0 && d.la16 != nullptr;
-  if (slab_tma) {
+  CUtensorMap tm_la = tm_out, tm_lb = tm_out;  // unused without a slab
+  if (d.slab_w > 0) {
     LSQ_TRY(make_tmap(&tm_la, dt16, 2, d.la16, (uint64_t)d.slab_w, (uint64_t)d.M,
                       (uint64_t)d.la16_ld, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B));
     LSQ_TRY(make_tmap(&tm_lb, dt16, 2, d.lb16, (uint64_t)d.slab_w, (uint64_t)d.T,
@@ -938,16 +884,6 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   p.w_rows = (int)d.w_rows;
   p.w_cols = (int)d.w_cols;
   p.slab_w = d.slab_w;
-  p.slab_tma = slab_tma ? 1 : 0;
-  p.part_r = d.part_r;
-  p.n_parts = d.n_parts;
-  p.la = d.la;
-  p.la_rs = d.la_rs;
-  p.la_cs = d.la_cs;
-  p.la_scale = d.la_scale;
-  p.lb = d.lb;
-  p.lb_ld = d.lb_ld;
-  for (int i = 0; i < 4; ++i) p.part_end[i] = d.part_end[i];
   p.out = d.out;
   p.out_f32 = d.out_f32;
   p.ldo = d.ldo;
@@ -1034,11 +970,10 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
     return set_error(LSQ_ERR_SHAPE, "gemm: row strides must be multiples of 16 bytes");
   if (d.slab_w % 16 != 0 || d.slab_w < 0)
     return set_error(LSQ_ERR_SHAPE, "gemm: LoRA slab width must be a multiple of 16");
-  if (d.slab_w > 0 && !d.la16 && (!d.la || !d.lb))
+  if (d.slab_w > 0 && (!d.la16 || !d.lb16))
     return set_error(LSQ_ERR_INVALID, "gemm: null LoRA slab");
-  if (d.slab_w > 0 && d.la16 &&
-      (!d.lb16 || d.la16_ld % 8 != 0 || d.lb16_ld % 8 != 0 || d.la16_ld < d.slab_w ||
-       d.lb16_ld < d.slab_w))
+  if (d.slab_w > 0 && (d.la16_ld % 8 != 0 || d.lb16_ld % 8 != 0 || d.la16_ld < d.slab_w ||
+                       d.lb16_ld < d.slab_w))
     return set_error(LSQ_ERR_SHAPE, "gemm: 16-bit LoRA slab operands need row strides >= the "
                                     "slab width, multiples of 8");
   if (d.residual && !d.out_f32) return set_error(LSQ_ERR_INVALID, "gemm: residual needs an fp32 output");

@@ -103,21 +103,11 @@ struct GemmDesc {
   int64_t w_rows = 0, w_cols = 0;   // storage shape of W
   const uint16_t* act = nullptr;    // bf16 [T, act_ld], contraction over the first Kc columns
   int64_t act_ld = 0;
-  // LoRA slab (an extra K range appended to split 0): lb[t, j] = lb_ptr[t * lb_ld + j]
-  // and la[m, j] = la_scale * la_ptr[m * la_rs + j * la_cs]; or, for a stacked
-  // weight with part_r > 0 (parts ending at rows part_end[]), slab_w = n_parts *
-  // part_r and la[m, j] = la_scale * la_ptr[m * la_rs + (j - p part_r) * la_cs]
-  // when row m is in part p and j in [p part_r, (p + 1) part_r), else 0: every
-  // row then uses the same lb, as a CTA pair's shared B operand requires.
+  // LoRA slab: an extra K range of slab_w columns appended to split 0, with
+  // operands la16 and lb16 below (for a stacked weight, la16's rows hold only their
+  // own part's columns, zeros elsewhere, so that every row uses the same lb16, as a
+  // CTA pair's shared B operand requires)
   int slab_w = 0;
-  const float* la = nullptr;
-  int64_t la_rs = 0, la_cs = 0;
-  float la_scale = 0.f;
-  const float* lb = nullptr;
-  int64_t lb_ld = 0;
-  int part_r = 0;
-  int n_parts = 0;
-  int64_t part_end[4] = {0, 0, 0, 0};
   // epilogue: out is fp32 when out_f32, else 16-bit in the mode's operand type;
   // residual (fp32 [T, ldr], added before the store) needs an fp32 output
   void* out = nullptr;
@@ -134,9 +124,9 @@ struct GemmDesc {
   // consumer's to add.
   const float** parts_out = nullptr;
   int* splits_out = nullptr;
-  // The LoRA slab from 16-bit operands by TMA, instead of la / lb above: la16
-  // [M][la16_ld] (the scale applied) and lb16 [T][lb16_ld], slab_w columns of
-  // each, in the mode's operand type (fp16 forward, bf16 input gradient).
+  // The LoRA slab's operands, loaded by TMA: la16 [M][la16_ld] (the scale applied)
+  // and lb16 [T][lb16_ld], slab_w columns of each, in the mode's operand type (fp16
+  // forward, bf16 input gradient).
   const uint16_t* la16 = nullptr;
   int64_t la16_ld = 0;
   const uint16_t* lb16 = nullptr;
@@ -239,9 +229,10 @@ int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, flo
 // once into the scratch first
 int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
                      float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
-                     cudaStream_t st);
+                     cudaStream_t st, uint16_t* uh = nullptr);
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, float* v,
-                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st);
+                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st,
+                      uint16_t* vh = nullptr);
 // One layer's LoRA operands rounded once into their product types: a list of
 // blocks, each
 //   kind 0: an fp16 copy of an A matrix, [rows][cols];

@@ -569,23 +569,24 @@ int launch_lora_grad_ab16(const uint16_t* v16, const uint16_t* x, int64_t K, flo
 // operand is rounded once into the start of the scratch, then the product runs.
 int launch_lora_down(const uint16_t* x, int64_t ldx, const float* A, int64_t T, int64_t K, int R,
                      float* u, uint16_t* u16, float* scratch, size_t scratch_bytes,
-                     cudaStream_t st) {
+                     cudaStream_t st, uint16_t* uh) {
   LSQ_TRY(check_ranks(R));
   Split sp;
   LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)R * K, &sp, "lora_down"));
   to_f16_rows_kernel<<<grid_for_elems((int64_t)R * K), 256, 0, st>>>(A, R, K, K, sp.q, K);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return launch_lora_down16(x, ldx, sp.q, T, K, R, u, u16, sp.rest, sp.rest_bytes, st);
+  return launch_lora_down16(x, ldx, sp.q, T, K, R, u, u16, sp.rest, sp.rest_bytes, st, uh);
 }
 
 int launch_lora_vproj(const uint16_t* dy, int64_t T, int64_t N, const float* B, int r, float* v,
-                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st) {
+                      uint16_t* v16, float* scratch, size_t scratch_bytes, cudaStream_t st,
+                      uint16_t* vh) {
   LSQ_TRY(check_ranks(r));
   Split sp;
   LSQ_TRY(split_scratch(scratch, scratch_bytes, (size_t)N * r, &sp, "lora_vproj"));
   to_bf16_transposed_kernel<<<grid_for_elems((int64_t)N * r), 256, 0, st>>>(B, N, r, sp.q);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return launch_lora_vproj16(dy, T, N, sp.q, r, v, v16, sp.rest, sp.rest_bytes, st);
+  return launch_lora_vproj16(dy, T, N, sp.q, r, v, v16, sp.rest, sp.rest_bytes, st, vh);
 }
 
 // One layer's LoRA operands in their product types (see internal.h).
