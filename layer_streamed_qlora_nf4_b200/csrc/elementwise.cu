@@ -715,13 +715,6 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t n,
     y[i] = float_to_bf16_bits(x[i]);
 }
 
-__global__ void scale_kernel(float* __restrict__ x, int64_t n, float s) {
-  pdl_trigger();  // the next kernel may launch once all CTAs of this one run
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    x[i] *= s;
-}
-
 }  // namespace
 
 int launch_splitk_reduce(const float* partial, int splits, int64_t T, int64_t M, void* out,
@@ -1010,12 +1003,6 @@ int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float 
 
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st) {
   f32_to_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, y);
-  LSQ_CUDA(::lsq::launched(cudaGetLastError()));
-  return LSQ_OK;
-}
-
-int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st) {
-  scale_kernel<<<grid_for(n, 256), 256, 0, st>>>(x, n, s);
   LSQ_CUDA(::lsq::launched(cudaGetLastError()));
   return LSQ_OK;
 }

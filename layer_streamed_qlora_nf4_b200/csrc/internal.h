@@ -189,7 +189,6 @@ int launch_sum_rows(const float* row_loss, int64_t T, float scale, int accumulat
 int launch_adamw(float* p, const float* g, float* m, float* v, int64_t n, float lr, float b1,
                  float b2, float eps, float wd, int step, cudaStream_t st);
 int launch_f32_to_bf16(const float* x, int64_t n, uint16_t* y, cudaStream_t st);
-int launch_scale_f32(float* x, int64_t n, float s, cudaStream_t st);
 
 // LoRA rank-r products (tcgen05 tensor cores, fp32 accumulation, fixed-order
 // reductions).  Operands in their product types: u = x A^T multiplies fp16 (x an
