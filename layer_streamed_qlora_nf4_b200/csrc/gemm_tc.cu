@@ -155,8 +155,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* am_ring = reinterpret_cast<float*>(rg0 + (size_t)p.ring_stages * p.ring_bytes);  // [kAmDepth][256]
   float* sc_ring = am_ring + kAmDepth * 256;  // 8-bit mode: the scale of each fetched absmax
 
-  const int m0 = blockIdx.x * kBM;
-  const int t0 = blockIdx.y * BT;
+  // Tile order: CTAs start in launch order (x fastest), and consecutive feature
+  // units (CTA pairs, or CTAs) are given a group of up to 8 token tiles each, so
+  // that the tiles running together share a few weight and activation tiles in L2.
+  int m_tile = blockIdx.x, t_tile = blockIdx.y;
+  if (gridDim.y > 1) {
+    constexpr int kG = 8;
+    const int units = PAIR ? (int)gridDim.x / 2 : (int)gridDim.x;
+    const int lin = (int)blockIdx.y * units + (PAIR ? (int)blockIdx.x / 2 : (int)blockIdx.x);
+    const int full = (int)gridDim.y / kG * kG;  // token tiles in complete groups
+    int unit;
+    if (lin < full * units) {
+      const int g = lin / (kG * units), r = lin % (kG * units);
+      unit = r / kG;
+      t_tile = g * kG + r % kG;
+    } else {
+      const int r = lin - full * units, rest = (int)gridDim.y - full;
+      unit = r / rest;
+      t_tile = full + r % rest;
+    }
+    m_tile = PAIR ? 2 * unit + (int)(blockIdx.x & 1u) : unit;
+  }
+  const int m0 = m_tile * kBM;
+  const int t0 = t_tile * BT;
   const int split = blockIdx.z;
   const int kt_begin = split * p.kt_per_split;
   const int kt_end = min(p.kt_total, kt_begin + p.kt_per_split);
