@@ -139,8 +139,8 @@ size_t nf4_lora_linear_workspace_bytes(int64_t T, int64_t K, int64_t N, int32_t 
  *   y        device [T, N] (output): fp16 when y_fp32 == 0, fp32 when y_fp32 == 1.
  *   u_out    device fp32 [T, r] = x A^T, or NULL.
  *   ws       device workspace of nf4_lora_linear_workspace_bytes(T, K, N, r).
- * The dequantised weight, A, B and u are rounded to fp16 for the tensor cores;
- * accumulation is fp32.  Asynchronous, deterministic. */
+ * The dequantised weight, A, scale * B and u are rounded to fp16 for the tensor
+ * cores; accumulation is fp32.  Asynchronous, deterministic. */
 int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int64_t N,
                         const uint8_t* codes, const float* absmax, int32_t block,
                         const float* A, const float* B, int32_t r, float scale,
@@ -150,7 +150,8 @@ int nf4_lora_linear_fwd(const uint16_t* x, int64_t T, int64_t K, int64_t N,
 /* nf4_lora_linear_bwd - backward of the linear above (W frozen).
  * Tutorial part 3 and FAQ 4: dX still needs W.
  *   dy [T, N] bf16 (the gradient), x [T, K] fp16 (the forward input).
- *   dx  device bf16 [T, K] = dy W~ + scale (dy B) A (bf16 products, fp32 sums).
+ *   dx  device bf16 [T, K] = dy W~ + scale (dy B) A (bf16 products of dy, W~, dy B and
+ *       scale A^T; fp32 sums).
  *   dA  device fp32 [r, K] (+)= scale (dy B)^T x;  dB device fp32 [N, r] (+)= scale dy^T (x A^T).
  *   accumulate  0: overwrite dA/dB, 1: add to them.
  * Asynchronous, deterministic (fixed-order reductions, no atomics). */
