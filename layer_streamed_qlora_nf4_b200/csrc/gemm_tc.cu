@@ -607,7 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool res = !partial && p.residual != nullptr;  // fp32, with an fp32 output
       bool big = false;  // an fp16 output beyond the fp16 range
       const uint32_t sub_bytes = 16u * 32u * (uint32_t)es;   // one [16 x 32] box
-      uint8_t* myslots = dsm + (size_t)warp * 8192;          // 2 slots of <= 4 KB
+      // 4 slots of <= 4 KB: a slot is written again only after the store of the chunk
+      // four back has read it, so stores stay in flight while the next chunks drain
+      uint8_t* myslots = dsm + (size_t)warp * 16384;
       const uint32_t rbar = smem_u32(&bar_res[warp]);
       const int mcol = m0 + qtr * 32;
       // this warp's chunks (at most 6: 2 accumulators x 8 chunks / 3)
@@ -624,10 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
       }
-      auto issue_res = [&](int i) {  // lane 0: residual of my chunk i into slot i & 1
+      auto issue_res = [&](int i) {  // lane 0: residual of my chunk i into slot i & 3
         const int tb = t0 + ma[i] * p.bn + mc[i];
         const int nsub = (p.bn - mc[i] >= 32) ? 2 : 1;
-        uint8_t* slot = myslots + (i & 1) * (2 * sub_bytes);
+        uint8_t* slot = myslots + (i & 3) * (2 * sub_bytes);
         mbar_arrive_expect_tx(rbar, (uint32_t)nsub * sub_bytes);
         for (int sb = 0; sb < nsub; ++sb)
           tma_load_2d(smem_u32(slot + sb * sub_bytes), &tm_res, rbar, mcol, tb + 16 * sb);
@@ -637,14 +639,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int a = ma[i], c0 = mc[i];
         const int tb = t0 + a * p.bn + c0;
         const int nsub = (p.bn - c0 >= 32) ? 2 : 1;   // 16-token sub-chunks
-        uint8_t* slot = myslots + (i & 1) * (2 * sub_bytes);
+        uint8_t* slot = myslots + (i & 3) * (2 * sub_bytes);
         if (res) {
           acc_ok = mbar_wait_bounded(rbar, (uint32_t)(i & 1), abort_flag, p.dev_err,
                                      DEV_ERR_WAIT_GEMM);
           acc_ok = __all_sync(0xFFFFFFFFu, acc_ok);
           if (!acc_ok) break;
         } else {
-          if (i >= 2 && lane == 0) bulk_wait_read<1>();  // the store that used this slot has read it
+          if (i >= 4 && lane == 0) bulk_wait_read<3>();  // the store that used this slot has read it
           __syncwarp();
         }
         uint32_t rg[2][16];
@@ -680,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           bulk_commit();
           if (res && i + 1 < nm) {
-            bulk_wait_read<1>();  // chunk i - 1's store has read slot (i + 1) & 1
+            bulk_wait_read<3>();  // chunk i - 3's store has read slot (i + 1) & 3
             issue_res(i + 1);
           }
         }
@@ -812,7 +814,7 @@ Plan make_plan(const GemmDesc& d) {
   while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;
   pl.stages = stages;
   pl.ring_stages = std::max(ring, 1);
-  pl.smem_bytes = std::max(total(stages, ring), 1024u + 12u * 8192u);  // epilogue chunk slots
+  pl.smem_bytes = std::max(total(stages, ring), 1024u + 12u * 16384u);  // epilogue chunk slots
   uint32_t cols = 32;
   while (cols < (uint32_t)pl.bn) cols <<= 1;
   pl.alloc_cols = (pl.nacc > 1) ? 512u : cols;
