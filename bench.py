@@ -38,7 +38,7 @@ BATCH, SEQ = 1, 512
 # (one ncu capture of every GEMM launch of one layer's forward + recomputing
 # backward; each launch reads its algorithmic bytes once).  The per-step mix of
 # launches is the same as in that layer, so the averages hold for the step.
-DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 36.98e6, "gemm_nf4_dx": 42.12e6}
+DRAM_BYTES_PER_LAUNCH_8B_T512 = {"gemm_nf4_fwd": 37.11e6, "gemm_nf4_dx": 42.15e6}
 # Profiler classes whose one timed region spans several kernels: the rank-r
 # products lora_rank_r_{u,v,dA,dB} (the product and the fixed-order sum of its
 # reduction slices).  The roofline object describes

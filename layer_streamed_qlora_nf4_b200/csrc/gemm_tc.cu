@@ -810,8 +810,11 @@ Plan make_plan(const GemmDesc& d) {
     return 1024u + (uint32_t)st * (xs + kWStageBytes) + (uint32_t)rs * pl.ring_bytes +
            kAmRingBytes;
   };
-  while (stages > 2 && total(stages, ring) > kSmemBudget - 4096) --stages;
+  // Operand stages before codes-ring depth: at 512 tokens per tile, 4 stages with a
+  // 3-deep ring run the transposed (input-gradient) NF4 product 4-7% faster than
+  // 3 stages with an 8-deep ring, and the forward product as fast.
   while (ring > 2 && total(stages, ring) > kSmemBudget - 4096) --ring;
+  while (stages > 2 && total(stages, ring) > kSmemBudget - 4096) --stages;
   pl.stages = stages;
   pl.ring_stages = std::max(ring, 1);
   pl.smem_bytes = std::max(total(stages, ring), 1024u + 12u * 16384u);  // epilogue chunk slots
