@@ -22,7 +22,8 @@
 //   warp 1    : allocates TMEM, one elected thread issues tcgen05.mma
 //               (M = 128 output features x N = up to 256 tokens x K = 16),
 //               accumulators in TMEM (up to 2 x 256 fp32 columns)
-//   warp 2    : TMA producer for the packed NF4 codes into a deep staging ring
+//   warp 2    : TMA producer for the packed NF4 codes into a staging ring (as deep
+//               as the shared memory left after the operand stages allows)
 //   warps 4-11: operand stage - expand the staged codes to fp16 / bf16
 //               (level[code] * absmax in fp32, then round to nearest) straight into the
 //               UMMA canonical K-major 128-byte-swizzle layout, fence the async
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ epilogue (all 12 warps)
   // Every warp joins once the accumulator is complete: warp w reads TMEM lane
   // quarter w % 4 (32 features) and takes every third 32-token chunk of that
-  // quarter (w / 4 selects which); it stages a chunk in two private
+  // quarter (w / 4 selects which); it stages a chunk in one of four private
   // shared-memory slots of the drained pipeline and writes it with TMA stores of
   // [16 tokens x 32 features] boxes, so no warp waits for another.  Residual
   // tiles arrive by TMA into the slot, the next chunk's while this one stores.
