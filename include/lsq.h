@@ -461,6 +461,42 @@ int lsq_profile_enable(int enable);
 /* Synchronises the recorded events and fills up to max entries (one per class). */
 int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out);
 
+/* lsq_gemm_plan_get - the launch plan of the fused tensor-core GEMM behind every
+ * frozen projection (host only; exported so that the planner can be inspected and
+ * tested without a GPU).  The product is out[T, M] = act[T, Kc] . Wop[M, Kc]^T with
+ * the operand mode:
+ *   LSQ_GEMM_NF4_FWD  Wop = deq(W), W NF4 [M, Kc] (forward, fp16 operands);
+ *   LSQ_GEMM_NF4_DX   Wop = deq(W)^T, W NF4 [Kc, M] (input gradient, bf16 operands);
+ *   LSQ_GEMM_BF16_FWD, LSQ_GEMM_BF16_DX  the same with a bf16 W (lm_head);
+ *   LSQ_GEMM_BF16_AS_F16_FWD  a bf16 W [M, Kc] converted to fp16 in the operand stage.
+ * num_sms is the GPU's SM count (148 on B200); allow_pair = 0 asks for one-CTA tiles
+ * (the library uses CTA pairs unless LSQ_GEMM_PAIR=0 is set in the environment).
+ * LSQ_ERR_INVALID for a bad mode or a null out; LSQ_ERR_SHAPE for a non-positive
+ * size or num_sms. */
+#define LSQ_GEMM_NF4_FWD 0
+#define LSQ_GEMM_NF4_DX 1
+#define LSQ_GEMM_BF16_FWD 2
+#define LSQ_GEMM_BF16_DX 3
+#define LSQ_GEMM_BF16_AS_F16_FWD 4
+typedef struct lsq_gemm_plan {
+  int32_t pair;               /* 1: CTA pairs (cta_group::2 MMAs, 256 features per pair) */
+  int32_t bn, nacc;           /* tokens per TMEM accumulator; accumulators per tile (1, 2) */
+  int32_t m_tiles, t_tiles, splits;  /* grid: 128-feature tiles x token tiles x K slices */
+  int32_t kt_total, kt_per_split;    /* 64-wide contraction tiles: all, per slice */
+  int32_t stages, ring_stages;       /* operand stages; NF4 code-ring slots */
+  int32_t x_stage_bytes;      /* activation bytes of one stage, per CTA */
+  int32_t w_stage_bytes;      /* weight-operand bytes of one stage */
+  int32_t ring_bytes;         /* bytes of one code-ring slot (0: no ring) */
+  int32_t absmax_ring_bytes;  /* the absmax prefetch ring */
+  int32_t smem_bytes;         /* dynamic shared memory of the launch */
+  int32_t smem_limit;         /* the most dynamic shared memory the kernel is given */
+  int32_t epilogue_bytes;     /* shared memory the epilogue's staging slots use */
+  int32_t tmem_cols;          /* TMEM columns allocated per CTA */
+  int64_t partial_bytes;      /* split-K workspace (fp32 partials; 0 when unsplit) */
+} lsq_gemm_plan;
+int lsq_gemm_plan_get(int32_t mode, int64_t M, int64_t T, int64_t Kc, int32_t num_sms,
+                      int32_t allow_pair, lsq_gemm_plan* out);
+
 /* --------------------------------------------------- allocation-free variant */
 
 /* nf4_lora_linear_fwd_noalloc - the same computation and kernels as

@@ -85,6 +85,13 @@ constexpr int kMaxRing = 8;
 constexpr uint32_t kSmemBudget = 227 * 1024;
 constexpr int kAmDepth = 8;  // absmax prefetch ring: 8 k-tiles x 256 floats
 constexpr uint32_t kAmRingBytes = kAmDepth * 256 * 4 * 2;  // absmax (or 8-bit words) + scales
+constexpr uint32_t kDynSmemLimit = kSmemBudget - 2048;  // the kernel's dynamic shared memory cap
+// the epilogue's staging: 12 warps x four 4 KB slots, after the 1 KB alignment pad
+constexpr uint32_t kEpilogueBytes = 1024u + 12u * 16384u;
+static_assert(W_NF4_N == LSQ_GEMM_NF4_FWD && W_NF4_T == LSQ_GEMM_NF4_DX &&
+                  W_BF16_N == LSQ_GEMM_BF16_FWD && W_BF16_T == LSQ_GEMM_BF16_DX &&
+                  W_BF16C_N == LSQ_GEMM_BF16_AS_F16_FWD,
+              "operand modes match the public constants");
 
 struct KParams {
   int M, T, Kc;
@@ -771,11 +778,12 @@ bool pair_enabled() {
   return v == 1;
 }
 
-Plan make_plan(const GemmDesc& d) {
+// The launch plan for `sms` SMs; allow_pair = false asks for one-CTA tiles.
+Plan make_plan(const GemmDesc& d, int sms, bool allow_pair) {
   Plan pl{};
   const int64_t T = d.T;
   pl.m_tiles = (int)((d.M + kBM - 1) / kBM);
-  pl.pair = pair_enabled() && pl.m_tiles >= 2;
+  pl.pair = allow_pair && pl.m_tiles >= 2;
   const int64_t gran = pl.pair ? 32 : 16;  // a pair splits each accumulator's tokens in two
   if (T <= 256) {
     pl.nacc = 1;
@@ -789,7 +797,6 @@ Plan make_plan(const GemmDesc& d) {
   const int BT = pl.nacc * pl.bn;
   pl.t_tiles = (int)((T + BT - 1) / BT);
   pl.kt_total = (int)((d.Kc + kBK - 1) / kBK);
-  const int sms = gemm_num_sms();
   const int base = pl.m_tiles * pl.t_tiles;
   int splits = 1;
   if (d.force_splits > 0) {
@@ -818,7 +825,7 @@ Plan make_plan(const GemmDesc& d) {
   while (stages > 2 && total(stages, ring) > kSmemBudget - 4096) --stages;
   pl.stages = stages;
   pl.ring_stages = std::max(ring, 1);
-  pl.smem_bytes = std::max(total(stages, ring), 1024u + 12u * 16384u);  // epilogue chunk slots
+  pl.smem_bytes = std::max(total(stages, ring), kEpilogueBytes);
   uint32_t cols = 32;
   while (cols < (uint32_t)pl.bn) cols <<= 1;
   pl.alloc_cols = (pl.nacc > 1) ? 512u : cols;
@@ -833,7 +840,7 @@ int launch_mode(const GemmDesc& d, const Plan& pl, float* partial, cudaStream_t 
   if (dev < 64 && !attr_done[dev]) {
     LSQ_CUDA(cudaFuncSetAttribute(tc_gemm_kernel<WMODE, PAIR>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)(kSmemBudget - 2048)));
+                                  (int)kDynSmemLimit));
     attr_done[dev] = true;
   }
   constexpr bool F16 = wmode_f16(WMODE);
@@ -983,7 +990,7 @@ namespace lsq {
 
 size_t gemm_workspace_bytes(const GemmDesc& d) {
   if (d.M <= 0 || d.T <= 0 || d.Kc <= 0) return 0;
-  return make_plan(d).partial_bytes;
+  return make_plan(d, gemm_num_sms(), pair_enabled()).partial_bytes;
 }
 
 int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -1008,7 +1015,7 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
     return set_error(LSQ_ERR_SHAPE, "gemm: output strides must be multiples of 16 bytes");
   if (d.M > INT32_MAX || d.T > INT32_MAX || d.Kc > INT32_MAX)
     return set_error(LSQ_ERR_SHAPE, "gemm: dimension too large");
-  Plan pl = make_plan(d);
+  Plan pl = make_plan(d, gemm_num_sms(), pair_enabled());
   float* partial = nullptr;
   if (pl.splits > 1) {
     if (!ws || ws_bytes < pl.partial_bytes)
@@ -1064,3 +1071,42 @@ int gemm_run(const GemmDesc& d, void* ws, size_t ws_bytes, cudaStream_t st) {
 }
 
 }  // namespace lsq
+
+extern "C" int lsq_gemm_plan_get(int32_t mode, int64_t M, int64_t T, int64_t Kc, int32_t num_sms,
+                                 int32_t allow_pair, lsq_gemm_plan* out) {
+  using namespace lsq;
+  if (!out) return set_error(LSQ_ERR_INVALID, "lsq_gemm_plan_get: null output");
+  if (mode < W_NF4_N || mode > W_BF16C_N)
+    return set_error(LSQ_ERR_INVALID, "lsq_gemm_plan_get: bad operand mode %d", (int)mode);
+  if (M <= 0 || T <= 0 || Kc <= 0 || num_sms <= 0 || M > INT32_MAX || T > INT32_MAX ||
+      Kc > INT32_MAX)
+    return set_error(LSQ_ERR_SHAPE, "lsq_gemm_plan_get: bad size");
+  GemmDesc d;
+  d.wmode = mode;
+  d.M = M;
+  d.T = T;
+  d.Kc = Kc;
+  const Plan pl = make_plan(d, num_sms, allow_pair != 0);
+  lsq_gemm_plan o{};
+  o.pair = pl.pair ? 1 : 0;
+  o.bn = pl.bn;
+  o.nacc = pl.nacc;
+  o.m_tiles = pl.m_tiles;
+  o.t_tiles = pl.t_tiles;
+  o.splits = pl.splits;
+  o.kt_total = pl.kt_total;
+  o.kt_per_split = pl.kt_per_split;
+  o.stages = pl.stages;
+  o.ring_stages = pl.ring_stages;
+  o.x_stage_bytes = (pl.pair ? pl.nacc * pl.bn / 2 : pl.nacc * pl.bn) * 128;
+  o.w_stage_bytes = kWStageBytes;
+  o.ring_bytes = (int32_t)pl.ring_bytes;
+  o.absmax_ring_bytes = (int32_t)kAmRingBytes;
+  o.smem_bytes = (int32_t)pl.smem_bytes;
+  o.smem_limit = (int32_t)kDynSmemLimit;
+  o.epilogue_bytes = (int32_t)kEpilogueBytes;
+  o.tmem_cols = (int32_t)pl.alloc_cols;
+  o.partial_bytes = (int64_t)pl.partial_bytes;
+  *out = o;
+  return LSQ_OK;
+}

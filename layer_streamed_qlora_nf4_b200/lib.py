@@ -27,7 +27,7 @@ EXPORTS = (
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
     "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
     "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard", "lsq_stream_plan",
-    "stream_stack_reduce_grads",
+    "stream_stack_reduce_grads", "lsq_gemm_plan_get",
 )
 LSQ_NCCL_ID_BYTES = 128
 
@@ -78,6 +78,19 @@ class lsq_step_stats(ctypes.Structure):
                 ("step_ms", ctypes.c_float), ("copy_wait_ms", ctypes.c_float)]
 
 
+class lsq_gemm_plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "pair", "bn", "nacc", "m_tiles", "t_tiles", "splits", "kt_total", "kt_per_split",
+        "stages", "ring_stages", "x_stage_bytes", "w_stage_bytes", "ring_bytes",
+        "absmax_ring_bytes", "smem_bytes", "smem_limit", "epilogue_bytes", "tmem_cols")] + [
+        ("partial_bytes", ctypes.c_int64)]
+
+
+# operand modes of lsq_gemm_plan_get
+LSQ_GEMM_NF4_FWD, LSQ_GEMM_NF4_DX, LSQ_GEMM_BF16_FWD, LSQ_GEMM_BF16_DX = 0, 1, 2, 3
+LSQ_GEMM_BF16_AS_F16_FWD = 4
+
+
 _P = ctypes.c_void_p
 _I32, _I64, _F, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 _PROTOS = {
@@ -126,6 +139,8 @@ _PROTOS = {
     "stream_stack_shard": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64]),
     "stream_stack_reduce_grads": (ctypes.c_int, [_P, _P, _I64, _I32, _I32]),
     "lsq_launch_counter": (ctypes.c_int64, []),
+    "lsq_gemm_plan_get": (ctypes.c_int, [_I32, _I64, _I64, _I64, _I32, _I32,
+                                         ctypes.POINTER(lsq_gemm_plan)]),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
                                                    _F, _P, _P, _I32, _P, _P]),
     "lsq_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -333,6 +348,14 @@ def lsq_stream_plan(n_layers, micro_batches, held0=-1, held1=-1):
     _check(load().lsq_stream_plan(int(n_layers), int(micro_batches), int(held0), int(held1),
                                   arrs[0], arrs[1], arrs[2], n, ctypes.byref(nv)))
     return [(arrs[0][i], arrs[1][i], arrs[2][i]) for i in range(nv.value)]
+
+
+def lsq_gemm_plan_get(mode, M, T, Kc, num_sms=148, allow_pair=True):
+    """-> dict of the fused GEMM's launch plan for one product (host only)."""
+    out = lsq_gemm_plan()
+    _check(load().lsq_gemm_plan_get(int(mode), int(M), int(T), int(Kc), int(num_sms),
+                                    1 if allow_pair else 0, ctypes.byref(out)))
+    return {n: getattr(out, n) for n, _ in lsq_gemm_plan._fields_}
 
 
 def lsq_shard_bytes(layer_bytes, world):
