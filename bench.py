@@ -176,6 +176,17 @@ def oracle_sample(seed=1):
 
 
 def cpu_threads():
+    """Threads the oracle runs on: the size of numpy's BLAS pool (its only multi-threaded
+    part), else the host's CPU count."""
+    try:
+        import numpy as np
+        from threadpoolctl import threadpool_info
+        np.ones((2, 2)) @ np.ones((2, 2))   # the BLAS library is loaded by its first use
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
     return os.cpu_count()
 
 
