@@ -72,6 +72,27 @@ __device__ unsigned long long g_gemm_stamps[kStampCtas][8];
   } while (0)
 #endif
 
+#ifdef LSQ_GEMM_KTL
+// Diagnostic build only (-DLSQ_GEMM_KTL): a per-k-tile timeline (globaltimer) of
+// every role of the first two CTAs (one pair) of the most recent launch, read by
+// lsq_debug_gemm_ktl.  Rows: 0 warp 0 saw the stage empty, 1 warp 0 issued its
+// loads, 2 warp 2 issued the code load, 3 operand warp 4 may fill the stage (code
+// slot full, stage empty), 4 its expansion is done and fenced, 5 it arrived,
+// 6 the issuer saw the stage full (even CTA) or the forwarder arrived (odd CTA),
+// 7 the issuer committed the stage's MMAs.
+constexpr int kKtlTiles = 256;
+__device__ unsigned long long g_gemm_ktl[2][8][kKtlTiles];
+#define LSQ_KTL(row, it)                                                           \
+  do {                                                                             \
+    const int _c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (_c < 2 && (it) < kKtlTiles) g_gemm_ktl[_c][row][it] = globaltimer_ns();    \
+  } while (0)
+#else
+#define LSQ_KTL(row, it) \
+  do {                   \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 384;   // 4 control warps + 8 operand/epilogue warps
@@ -247,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   DEV_ERR_WAIT_GEMM);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       const uint32_t fb = smem_u32(&bar_full[s]);
+      if (lane == 0) LSQ_KTL(0, it);
       if (lane == 0) {
         if (it < n_main) {
           const int kt = kt_begin + it;
@@ -309,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (!PAIR || leader) {
           mbar_arrive(fb);
         }
+        LSQ_KTL(1, it);
       }
       __syncwarp();
     }
@@ -340,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #endif
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
+      if (lane == 0) LSQ_KTL(6, it);
       if (lane == 0) {
         int nk = 4;
         if (it >= n_main) nk = min(4, (p.slab_w - (it - n_main) * 64) / 16);
@@ -365,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit_pair(smem_u32(&bar_empty[s]));
         else
           tc_commit(smem_u32(&bar_empty[s]));
+        LSQ_KTL(7, it);
       }
       __syncwarp();
     }
@@ -390,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   DEV_ERR_WAIT_GEMM);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bar_full[s]), 0));
+      if (lane == 0) LSQ_KTL(6, it);
       __syncwarp();
     }
   } else if (warp == 2) {
@@ -410,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (WMODE == W_NF4_T) tma_load_2d(dst, &tm_w, cb, m0 / 2, kt * kBK);  // [64 rows][64 B]
           if (WMODE == W_BF16_T) tma_load_2d(dst, &tm_w, cb, m0, kt * kBK);     // [64][128 bf16]
           if (WMODE == W_BF16C_N) tma_load_2d(dst, &tm_w, cb, kt * kBK, m0);    // [128][64 bf16] SW128
+          LSQ_KTL(2, it);
         }
         __syncwarp();
       }
@@ -527,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, abort_flag, p.dev_err,
                                  DEV_ERR_WAIT_GEMM);
           ok = __all_sync(0xFFFFFFFFu, ok);
+          if (ok && warp == 4 && lane == 0) LSQ_KTL(3, it);
           if (ok) {
             if (WMODE == W_NF4_N) {
               // thread: row r, half h of its 64 codes (chunks 4h .. 4h+3)
@@ -575,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
+            if (warp == 4 && lane == 0) LSQ_KTL(4, it);
             if (lane == 0) mbar_arrive(smem_u32(&bar_cempty[c]));
           }
         }
@@ -587,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && lane == 0)
         mbar_arrive(smem_u32(PAIR && !leader ? &bar_opd[s] : &bar_full[s]));
+      if (ok && warp == 4 && lane == 0) LSQ_KTL(5, it);
     }
 
   }
@@ -977,6 +1007,17 @@ int* device_status_ptr() {
   }
   return ptrs[dev];
 }
+
+#ifdef LSQ_GEMM_KTL
+}  // namespace lsq
+// Diagnostic build only: copies the per-k-tile timeline of the last launch
+// (2 CTAs x 8 rows x 256 k-tiles) to host.
+extern "C" int lsq_debug_gemm_ktl(unsigned long long* out) {
+  return cudaMemcpyFromSymbol(out, lsq::g_gemm_ktl, sizeof(lsq::g_gemm_ktl)) == cudaSuccess ? 0
+                                                                                             : 3;
+}
+namespace lsq {
+#endif
 
 #ifdef LSQ_GEMM_STAMPS
 }  // namespace lsq
