@@ -472,7 +472,7 @@ int lsq_profile_read(lsq_prof_entry* out, int32_t max, int32_t* n_out);
  * num_sms is the GPU's SM count (148 on B200); allow_pair = 0 asks for one-CTA tiles
  * (the library uses CTA pairs unless LSQ_GEMM_PAIR=0 is set in the environment).
  * LSQ_ERR_INVALID for a bad mode or a null out; LSQ_ERR_SHAPE for a non-positive
- * size or num_sms. */
+ * size or num_sms, or a size beyond 2^31 - 1.  Added in ABI 2.1. */
 #define LSQ_GEMM_NF4_FWD 0
 #define LSQ_GEMM_NF4_DX 1
 #define LSQ_GEMM_BF16_FWD 2

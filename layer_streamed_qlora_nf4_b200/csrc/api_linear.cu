@@ -169,7 +169,7 @@ int check_linear(const void* x, int64_t T, int64_t K, int64_t N, const void* cod
 using namespace lsq;
 
 extern "C" const char* lsq_last_error(void) { return t_msg; }
-extern "C" int lsq_version(void) { return 200; }
+extern "C" int lsq_version(void) { return 201; }
 
 extern "C" int lsq_device_status(int* flags, int clear) {
   if (!flags) return set_error(LSQ_ERR_INVALID, "lsq_device_status: null output");
