@@ -792,6 +792,7 @@ struct Plan {
   int bn, nacc, t_tiles, m_tiles, kt_total, kt_per_split, splits, stages, ring_stages;
   bool pair;  // CTA pairs with cta_group::2 MMAs (M = 256 per pair)
   uint32_t ring_bytes, smem_bytes, alloc_cols;
+  uint32_t xs_bytes;  // activation bytes of one stage, per CTA
   size_t partial_bytes;
 };
 
@@ -842,6 +843,7 @@ Plan make_plan(const GemmDesc& d, int sms, bool allow_pair) {
   const bool w_tma = d.wmode == W_BF16_N || d.wmode == W_BF16_T || d.wmode == W_BF16C_N;
   pl.ring_bytes = w_tma ? 0 : 4096;
   const uint32_t xs = (uint32_t)(pl.pair ? BT / 2 : BT) * 128;
+  pl.xs_bytes = xs;
   int ring = w_tma ? 0 : kMaxRing;
   int stages = kMaxStages;
   auto total = [&](int st, int rs) {
@@ -1139,7 +1141,7 @@ extern "C" int lsq_gemm_plan_get(int32_t mode, int64_t M, int64_t T, int64_t Kc,
   o.kt_per_split = pl.kt_per_split;
   o.stages = pl.stages;
   o.ring_stages = pl.ring_stages;
-  o.x_stage_bytes = (pl.pair ? pl.nacc * pl.bn / 2 : pl.nacc * pl.bn) * 128;
+  o.x_stage_bytes = (int32_t)pl.xs_bytes;
   o.w_stage_bytes = kWStageBytes;
   o.ring_bytes = (int32_t)pl.ring_bytes;
   o.absmax_ring_bytes = (int32_t)kAmRingBytes;
