@@ -497,6 +497,28 @@ typedef struct lsq_gemm_plan {
 int lsq_gemm_plan_get(int32_t mode, int64_t M, int64_t T, int64_t Kc, int32_t num_sms,
                       int32_t allow_pair, lsq_gemm_plan* out);
 
+/* lsq_lora_plan_get - the launch plan of the tensor-core kernel behind the LoRA
+ * rank-r products (u = x A^T, v = dY B, dA, dB): C [M, N] = A [M, K] . B [N, K]^T
+ * (host only; exported so that the planner can be inspected and tested without a
+ * GPU).  num_sms is the GPU's SM count.  A product whose tiles leave at least half
+ * of the resident CTA slots empty splits its reduction over a thread-block
+ * cluster of `splits` CTAs, whose accumulators are summed in shared memory.
+ * LSQ_ERR_INVALID for a null out; LSQ_ERR_SHAPE for a non-positive size or
+ * num_sms.  Added in ABI 2.1. */
+typedef struct lsq_lora_plan {
+  int32_t n_pad;              /* columns per CTA: N rounded up to 16, at most 256 */
+  int32_t row_tiles, col_tiles, splits;  /* grid: 128-row tiles x column tiles x slices */
+  int32_t kt_total;           /* 64-wide reduction stages */
+  int32_t stages;             /* operand stages in flight */
+  int32_t stage_bytes;        /* bytes of one stage (A tile + B tile) */
+  int32_t smem_bytes;         /* dynamic shared memory of the launch */
+  int32_t smem_limit;         /* the most dynamic shared memory the kernel is given */
+  int32_t ctas_per_sm;        /* resident CTAs per SM the plan assumes */
+  int32_t tmem_cols;          /* TMEM columns allocated per CTA */
+  int32_t reduce_bytes;       /* shared memory of the cluster sum (0 when unsplit) */
+} lsq_lora_plan;
+int lsq_lora_plan_get(int64_t M, int64_t N, int64_t K, int32_t num_sms, lsq_lora_plan* out);
+
 /* --------------------------------------------------- allocation-free variant */
 
 /* nf4_lora_linear_fwd_noalloc - the same computation and kernels as

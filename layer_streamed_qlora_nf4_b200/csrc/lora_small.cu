@@ -325,13 +325,13 @@ int stages_for(int) { return 4; }
 size_t smem_for(int n_pad) { return 1024 + (size_t)stages_for(n_pad) * stage_bytes(n_pad); }
 int ctas_per_sm(int n_pad) { return smem_for(n_pad) <= 110 * 1024 ? 2 : 1; }
 
-// Splits of the reduction (a cluster of 2, 4 or 8 CTAs per tile): only where the
-// product's own tiles leave at least half of the resident CTA slots empty, up to
-// filling them, each slice at least two stages long.
-int splits_for(int64_t M, int64_t N, int64_t K) {
+// Splits of the reduction (a cluster of 2, 4 or 8 CTAs per tile) on `sms` SMs: only
+// where the product's own tiles leave at least half of the resident CTA slots
+// empty, up to filling them, each slice at least two stages long.
+int splits_for(int64_t M, int64_t N, int64_t K, int sms) {
   if (K <= 0 || M <= 0 || N <= 0) return 1;
   const int64_t tiles = (M + kSM - 1) / kSM * ((N + kSMaxN - 1) / kSMaxN);
-  const int64_t slots = (int64_t)kSMs * ctas_per_sm(npad_for(N));
+  const int64_t slots = (int64_t)sms * ctas_per_sm(npad_for(N));
   if (tiles * 2 > slots) return 1;
   const int64_t kt = (K + kSK - 1) / kSK;
   const int64_t cap = std::min<int64_t>(8, std::min<int64_t>(slots / tiles, kt / 2));
@@ -407,7 +407,7 @@ int run(SkinnyArgs a, const Operand& A, const Operand& B, bool f16, cudaStream_t
   if (a.M <= 0 || a.N <= 0) return LSQ_OK;
   if (a.K <= 0) return set_error(LSQ_ERR_SHAPE, "lora product: empty reduction");
   const int n_pad = npad_for(a.N);
-  const int z = splits_for(a.M, a.N, a.K);  // every slice gets at least two stages
+  const int z = splits_for(a.M, a.N, a.K, gemm_num_sms());  // slices of >= two stages
   a.splits = z;
   CUtensorMap ta, tb;
   LSQ_TRY(tmaps_for(A_MN, A, B, n_pad, &ta, &tb));
@@ -428,7 +428,7 @@ int run_pair_mn(SkinnyArgs a, const Operand& A, bool conv, SkinnyArgs b, const O
   if (a.K <= 0) return set_error(LSQ_ERR_SHAPE, "lora product: empty reduction");
   const int n_pad = npad_for(a.N);
   const int64_t t1 = (a.M + kSM - 1) / kSM, t2 = (b.M + kSM - 1) / kSM;
-  const int z = splits_for((t1 + t2) * kSM, a.N, a.K);
+  const int z = splits_for((t1 + t2) * kSM, a.N, a.K, gemm_num_sms());
   a.splits = b.splits = z;
   CUtensorMap ta, tb, ta2, tb2;
   LSQ_TRY(tmaps_for(true, A, B, n_pad, &ta, &tb));
@@ -643,3 +643,30 @@ int launch_lora_prepare(const float* lora, int64_t lora_stride, int n_layers, ui
 }
 
 }  // namespace lsq
+
+extern "C" int lsq_lora_plan_get(int64_t M, int64_t N, int64_t K, int32_t num_sms,
+                                 lsq_lora_plan* out) {
+  using namespace lsq;
+  if (!out) return set_error(LSQ_ERR_INVALID, "lsq_lora_plan_get: null output");
+  if (M <= 0 || N <= 0 || K <= 0 || num_sms <= 0)
+    return set_error(LSQ_ERR_SHAPE, "lsq_lora_plan_get: bad size");
+  const int n_pad = npad_for(N);
+  const int z = splits_for(M, N, K, num_sms);
+  lsq_lora_plan o{};
+  o.n_pad = n_pad;
+  o.row_tiles = (int32_t)((M + kSM - 1) / kSM);
+  o.col_tiles = (int32_t)((N + n_pad - 1) / n_pad);
+  o.splits = z;
+  o.kt_total = (int32_t)((K + kSK - 1) / kSK);
+  o.stages = stages_for(n_pad);
+  o.stage_bytes = (int32_t)stage_bytes(n_pad);
+  o.smem_bytes = (int32_t)smem_for(n_pad);
+  o.smem_limit = (int32_t)smem_for(kSMaxN);
+  o.ctas_per_sm = ctas_per_sm(n_pad);
+  uint32_t cols = 32;
+  while (cols < (uint32_t)n_pad) cols <<= 1;
+  o.tmem_cols = (int32_t)cols;
+  o.reduce_bytes = z > 1 ? kSM * (n_pad + 4) * 4 : 0;
+  *out = o;
+  return LSQ_OK;
+}

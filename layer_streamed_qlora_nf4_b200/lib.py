@@ -27,7 +27,7 @@ EXPORTS = (
     "nf4_lora_linear_fwd_noalloc", "nf4_absmax_quantize8", "nf4_dequantize_dq",
     "stream_stack_dpo_workspace_bytes", "stream_stack_dpo_step", "lsq_bf16_from_f32",
     "lsq_shard_bytes", "lsq_nccl_unique_id", "stream_stack_shard", "lsq_stream_plan",
-    "stream_stack_reduce_grads", "lsq_gemm_plan_get",
+    "stream_stack_reduce_grads", "lsq_gemm_plan_get", "lsq_lora_plan_get",
 )
 LSQ_NCCL_ID_BYTES = 128
 
@@ -86,6 +86,12 @@ class lsq_gemm_plan(ctypes.Structure):
         ("partial_bytes", ctypes.c_int64)]
 
 
+class lsq_lora_plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_pad", "row_tiles", "col_tiles", "splits", "kt_total", "stages", "stage_bytes",
+        "smem_bytes", "smem_limit", "ctas_per_sm", "tmem_cols", "reduce_bytes")]
+
+
 # operand modes of lsq_gemm_plan_get
 LSQ_GEMM_NF4_FWD, LSQ_GEMM_NF4_DX, LSQ_GEMM_BF16_FWD, LSQ_GEMM_BF16_DX = 0, 1, 2, 3
 LSQ_GEMM_BF16_AS_F16_FWD = 4
@@ -141,6 +147,7 @@ _PROTOS = {
     "lsq_launch_counter": (ctypes.c_int64, []),
     "lsq_gemm_plan_get": (ctypes.c_int, [_I32, _I64, _I64, _I64, _I32, _I32,
                                          ctypes.POINTER(lsq_gemm_plan)]),
+    "lsq_lora_plan_get": (ctypes.c_int, [_I64, _I64, _I64, _I32, ctypes.POINTER(lsq_lora_plan)]),
     "nf4_lora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _I32, _P, _P, _I32,
                                                    _F, _P, _P, _I32, _P, _P]),
     "lsq_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -356,6 +363,13 @@ def lsq_gemm_plan_get(mode, M, T, Kc, num_sms=148, allow_pair=True):
     _check(load().lsq_gemm_plan_get(int(mode), int(M), int(T), int(Kc), int(num_sms),
                                     1 if allow_pair else 0, ctypes.byref(out)))
     return {n: getattr(out, n) for n, _ in lsq_gemm_plan._fields_}
+
+
+def lsq_lora_plan_get(M, N, K, num_sms=148):
+    """-> dict of the rank-r product kernel's launch plan (host only)."""
+    out = lsq_lora_plan()
+    _check(load().lsq_lora_plan_get(int(M), int(N), int(K), int(num_sms), ctypes.byref(out)))
+    return {n: getattr(out, n) for n, _ in lsq_lora_plan._fields_}
 
 
 def lsq_shard_bytes(layer_bytes, world):

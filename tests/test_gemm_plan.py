@@ -1,10 +1,12 @@
-"""The fused GEMM's launch planner, checked on the CPU (host only, no GPU).
+"""The launch planners of the two tensor-core kernels, checked on the CPU (host
+only, no GPU): the fused NF4 GEMM and the LoRA rank-r product kernel.
 
-Every plan must fit the kernel's shared-memory cap with room for the epilogue's
-staging slots, cover every token and contraction tile exactly once, and never
-launch an empty K slice; the TMEM allocation must hold the tile's accumulators.
-The shapes span the decoder projections of the 8B- and Qwen2.5-3B-shaped stacks,
-their input gradients, the lm_head, the split-K cases and ragged token counts.
+Every plan must fit the kernel's shared-memory cap (with room for the GEMM
+epilogue's staging slots, or for the rank-r kernel's cluster sum), cover every
+row, column and reduction tile exactly once, and never launch an empty slice; the
+TMEM allocation must hold the tile's accumulators.  The shapes span the decoder
+projections of the 8B- and Qwen2.5-3B-shaped stacks, their input gradients, the
+lm_head, the LoRA products, the split cases and ragged token counts.
 """
 import itertools
 
@@ -103,3 +105,69 @@ def test_bad_queries_are_rejected(L):
         L.lsq_gemm_plan_get(0, 0, 16, 64)
     with pytest.raises(L.LsqError):
         L.lsq_gemm_plan_get(0, 128, 16, 64, num_sms=0)
+
+
+# ---------------------------------------------------------------- rank-r products
+# The LoRA products: C [M, N] = A [M, K] . B [N, K]^T with N the (stacked) rank or,
+# for dA / dB, M the rank side; M, N and K span the 8B and Qwen2.5-3B shapes.
+LM = (16, 48, 128, 512, 2048, 4096, 16384, 28672)
+LN = (8, 16, 48, 64, 96, 128, 192, 256, 384, 4096, 14336)
+LK = (64, 128, 512, 2048, 4096, 16384, 28672)
+
+
+def _check_lora_plan(p, M, N, K, sms):
+    assert p["n_pad"] == min(256, (N + 15) // 16 * 16)
+    assert p["col_tiles"] * p["n_pad"] >= N and (p["col_tiles"] - 1) * p["n_pad"] < N
+    assert p["row_tiles"] * 128 >= M and (p["row_tiles"] - 1) * 128 < M
+    assert p["kt_total"] == (K + 63) // 64
+    # shared memory: a 1 KB alignment pad and the stages, within the kernel's cap
+    assert p["stages"] == 4                       # the kernel keeps 4 stage barriers
+    assert p["stage_bytes"] == 128 * 64 * 2 + (p["n_pad"] * 128 + 1023) // 1024 * 1024
+    assert p["smem_bytes"] == 1024 + p["stages"] * p["stage_bytes"] <= p["smem_limit"]
+    assert p["smem_limit"] <= 227 * 1024
+    # two resident CTAs per SM only where both fit the SM's shared memory and TMEM
+    assert p["ctas_per_sm"] in (1, 2)
+    if p["ctas_per_sm"] == 2:
+        assert 2 * p["smem_bytes"] <= 228 * 1024 and 2 * p["tmem_cols"] <= 512
+    c = p["tmem_cols"]
+    assert 32 <= c <= 512 and c & (c - 1) == 0 and c >= p["n_pad"]
+    # split reduction: a portable cluster whose slices share the 128 rows evenly, each
+    # at least two stages long, only where the tiles alone leave half the slots empty
+    z = p["splits"]
+    slots = sms * p["ctas_per_sm"]
+    tiles = p["row_tiles"] * p["col_tiles"]
+    assert z in (1, 2, 4, 8) and 128 % z == 0
+    if z > 1:
+        assert tiles * 2 <= slots and tiles * z <= slots
+        assert p["kt_total"] // z >= 2
+        # the cluster sum's fp32 [128][n_pad + 4] buffer fits the drained stages
+        assert p["reduce_bytes"] == 128 * (p["n_pad"] + 4) * 4
+        assert p["reduce_bytes"] <= p["stages"] * p["stage_bytes"]
+    else:
+        assert p["reduce_bytes"] == 0
+    assert p["row_tiles"] <= 2 ** 31 - 1 and p["col_tiles"] <= 65535
+
+
+def test_rank_r_plans_fit_and_cover_the_product(L):
+    n = 0
+    for M, N, K in itertools.product(LM, LN, LK):
+        for sms in (148, 132):
+            _check_lora_plan(L.lsq_lora_plan_get(M, N, K, sms), M, N, K, sms)
+            n += 1
+    assert n == len(LM) * len(LN) * len(LK) * 2
+
+
+def test_rank_r_split_choices_at_the_8b_shapes(L):
+    # u = x A^T of the 8B q|k|v group at T = 512 (N = 3 r = 48): 4 row tiles split 8 ways
+    p = L.lsq_lora_plan_get(512, 48, 4096)
+    assert (p["row_tiles"], p["splits"], p["ctas_per_sm"]) == (4, 8, 2)
+    # a product that fills the GPU by its tiles is not split
+    p = L.lsq_lora_plan_get(16384, 256, 4096)
+    assert p["splits"] == 1 and p["reduce_bytes"] == 0
+
+
+def test_bad_rank_r_queries_are_rejected(L):
+    with pytest.raises(L.LsqError):
+        L.lsq_lora_plan_get(0, 16, 64)
+    with pytest.raises(L.LsqError):
+        L.lsq_lora_plan_get(128, 16, 64, num_sms=0)
